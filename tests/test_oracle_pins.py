@@ -1,0 +1,393 @@
+"""Pins for the CPU oracle: what the pages and the mathematics fix.
+
+None of these retypes an oracle formula.  Each checks the oracle against an
+independent fact: a value the pages print, a closed form, a brute-force search,
+a library routine for a special case, or an element-by-element loop.
+"""
+import json
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import scipy.special
+
+from oracle import w1_oracle as O
+from pack_sign_g128_b200 import synth
+
+
+# ---------------------------------------------------------------- fp16 rounding
+
+def _f16bits(v: float) -> int:
+    return int(np.array([v], dtype=np.float64).astype(np.float16).view(np.uint16)[0])
+
+
+def test_fp16_rounding_matches_library_conversion_off_midpoints():
+    g = np.random.default_rng(11)
+    vals = np.concatenate([
+        np.abs(g.standard_normal(2000)) * 10.0 ** g.integers(-9, 5, 2000),
+        np.abs(g.standard_normal(200)) * 1e-7,          # fp16 subnormal range
+        [65503.9, 65519.0, 6.1035e-05, 5.96e-08, 1.0, 0.5],
+    ])
+    for v in vals:
+        assert O.round_to_fp16_bits(Fraction(float(v))) == _f16bits(float(v)), v
+
+
+def test_fp16_ties_go_to_even_and_overflow():
+    one = Fraction(1)
+    u = Fraction(1, 2 ** 10)                 # ulp of binary16 at 1.0
+    assert O.round_to_fp16_bits(one + u / 2) == 0x3C00          # tie -> even (1.0)
+    assert O.round_to_fp16_bits(one + 3 * u / 2) == 0x3C02      # tie -> even (1+2u)
+    assert O.round_to_fp16_bits(one + u / 2 + Fraction(1, 2 ** 60)) == 0x3C01
+    sub = Fraction(1, 2 ** 24)               # subnormal quantum
+    assert O.round_to_fp16_bits(sub / 2) == 0x0000
+    assert O.round_to_fp16_bits(3 * sub / 2) == 0x0002
+    assert O.round_to_fp16_bits(Fraction(65519)) == 0x7BFF       # 65504
+    assert O.round_to_fp16_bits(Fraction(65520)) == 0x7C00       # inf
+    assert O.round_to_fp16_bits(Fraction(0)) == 0
+
+
+# ---------------------------------------------------------------- scale rule
+
+def _sq_err(w, alpha):
+    w = np.asarray(w, dtype=np.float64)
+    sgn = np.where(np.signbit(w), -1.0, 1.0)
+    return float(np.sum((w - alpha * sgn) ** 2))
+
+
+def test_scale_matches_brute_force_search_on_tiny_groups():
+    """mean|w| is the least-squares scale for sign codes (brute-force search)."""
+    g = np.random.default_rng(5)
+    for group in (4, 8):
+        for _ in range(20):
+            w = (g.standard_normal(group) * 0.02).astype(np.float32)
+            grid = np.linspace(0.0, float(np.max(np.abs(w))) * 1.5, 300001)
+            sgn = np.where(np.signbit(w.astype(np.float64)), -1.0, 1.0)
+            errs = ((w.astype(np.float64)[None, :] - grid[:, None] * sgn[None, :]) ** 2).sum(1)
+            best = grid[int(np.argmin(errs))]
+            s = float(np.array([O.group_scale_bits(w)], np.uint16).view(np.float16)[0])
+            step = grid[1] - grid[0]
+            half_ulp = 2.0 ** (math.floor(math.log2(best)) - 11)
+            assert abs(s - best) <= step + half_ulp, (group, s, best)
+
+
+def test_scale_is_the_best_fp16_value_for_each_group():
+    g = synth.rng(7)
+    W = synth.weights(g, 8, 512)
+    _, scales = O.pack_ref(W)
+    for n in range(8):
+        for gi in range(4):
+            w = W[n, gi * 128:(gi + 1) * 128]
+            sb = int(scales[n, gi])
+            s = float(np.array([sb], np.uint16).view(np.float16)[0])
+            lo = float(np.array([sb - 1], np.uint16).view(np.float16)[0])
+            hi = float(np.array([sb + 1], np.uint16).view(np.float16)[0])
+            e = _sq_err(w, s)
+            assert e <= _sq_err(w, lo) and e <= _sq_err(w, hi)
+
+
+def test_flipping_any_sign_increases_error():
+    g = synth.rng(8)
+    W = synth.weights(g, 2, 128)
+    signs, scales = O.pack_ref(W)
+    w_hat = O.dequant_ref(signs, scales, 128)
+    base = np.sum((W.astype(np.float64) - w_hat) ** 2, axis=1)
+    for n in range(2):
+        for k in range(128):
+            alt = w_hat[n].copy()
+            alt[k] = -alt[k]
+            assert np.sum((W[n].astype(np.float64) - alt) ** 2) > base[n]
+
+
+def test_scale_sum_is_exact_tiny_value_breaks_a_tie():
+    """A sum that float64 would round onto an fp16 midpoint must still round
+    from the exact value: 126*M + 2M + 2**-100 with M = 1 + 2**-11."""
+    M = np.float32(1.0 + 2.0 ** -11)
+    vals = np.array([M] * 126 + [np.float32(2.0) * M, np.float32(2.0 ** -100)], dtype=np.float32)
+    assert math.fsum(np.abs(vals.astype(np.float64))) / 128 == float(M)   # fp64 lands on the tie
+    assert O.group_scale_bits(vals) == 0x3C01                               # exact: just above it
+    exact_tie = np.array([M] * 128, dtype=np.float32)
+    assert O.group_scale_bits(exact_tie) == 0x3C00                          # true tie -> even
+
+
+def test_scale_special_groups():
+    assert O.group_scale_bits(np.zeros(128, np.float32)) == 0
+    assert O.group_scale_bits(np.full(128, -0.0, np.float32)) == 0
+    # all |w| = 2**-30: mean 2**-30 is below the fp16 subnormal quantum/2 -> 0
+    assert O.group_scale_bits(np.full(128, 2.0 ** -30, np.float32)) == 0
+    # mean |w| = 3 * 2**-25: subnormal tie between 2**-24 and 2**-23 -> even (2**-23)
+    assert O.group_scale_bits(np.full(128, 3 * 2.0 ** -25, np.float32)) == 0x0002
+    # overflow of the fp16 range
+    assert O.group_scale_bits(np.full(128, 70000.0, np.float32)) == 0x7C00
+    with pytest.raises(ValueError):
+        O.group_scale_bits(np.array([np.nan] + [1.0] * 127, np.float32))
+
+
+# ---------------------------------------------------------------- sign bits
+
+def test_sign_convention_zero_is_plus_one():
+    W = np.zeros((1, 128), np.float32)
+    W[0, 1] = -0.0
+    W[0, 2] = -1.5
+    W[0, 3] = 2.0
+    bits = O.sign_bits_ref(W)[0]
+    assert bits[0] == 0 and bits[1] == 1 and bits[2] == 1 and bits[3] == 0
+    signs, scales = O.pack_ref(W)
+    w_hat = O.dequant_ref(signs, scales, 128)
+    s = float(np.array([scales[0, 0]], np.uint16).view(np.float16)[0])
+    assert w_hat[0, 0] == s and w_hat[0, 2] == -s and w_hat[0, 3] == s
+
+
+def test_bit_order_lsb_first():
+    bits = np.zeros((1, 64), np.uint8)
+    bits[0, 0] = 1
+    bits[0, 33] = 1
+    bits[0, 63] = 1
+    words = O.pack_bits_lsb_first(bits)
+    assert words.tolist() == [[1, (1 << 1) | (1 << 31)]]
+    # little-endian bytes of two LSB-first uint32 words == one LSB-first uint64 block
+    u64 = int.from_bytes(words.astype('<u4').tobytes(), 'little')
+    assert u64 == (1 << 0) | (1 << 33) | (1 << 63)
+
+
+def test_pack_roundtrip():
+    g = synth.rng(9)
+    W = synth.weights(g, 16, 256)
+    signs, _ = O.pack_ref(W)
+    bits = O.unpack_bits_lsb_first(signs, 256)
+    assert np.array_equal(bits.astype(bool), np.signbit(W))
+    assert O.pack_bits_lsb_first(bits).tobytes() == signs.tobytes()
+
+
+# ---------------------------------------------------------------- accounting
+
+def test_bits_per_weight_is_1_125(golden_dir):
+    with open(os.path.join(golden_dir, "format_accounting.json")) as f:
+        gold = json.load(f)
+    for N, K in [(512, 1024), (4096, 4096), (11008, 4096), (14336, 14336)]:
+        assert Fraction(O.sign_group_bits(N, K), N * K) == Fraction(gold["bits_per_weight"])
+    ratio = gold["parent_bits"] / gold["bits_per_weight"]
+    assert round(ratio) == 14
+
+
+def test_dbf_bit_budget_matches_page(golden_dir):
+    with open(os.path.join(golden_dir, "dbf_bit_budget.json")) as f:
+        gold = json.load(f)
+    m, n, r = gold["m"], gold["n"], gold["r"]
+    binary, diag, total = O.dbf_bits(m, n, r)
+    assert binary == gold["binary_factor_bits"]
+    assert diag == gold["fp16_diagonal_bits"]
+    assert total == gold["total_bits"]
+    assert O.dbf_bits_per_element(m, n, r) == Fraction(gold["bits_per_element"])
+    q2k = int(Fraction(gold["q2k_bits_per_element"]) * m * n)
+    assert q2k == gold["q2k_total_bits"]
+    assert (q2k - total) // 8 == gold["dbf_smaller_by_bytes"]
+    cnt = gold["routed_matrices"]
+    bd = gold["routed_matrices_breakdown"]
+    assert bd["layers"] * bd["experts"] * bd["projections"] == cnt
+    gib = 8 * 2 ** 30
+    assert round(total * cnt / gib, 4) == gold["dbf_total_gib"]
+    assert round(q2k * cnt / gib, 4) == gold["q2k_total_gib"]
+    assert round((q2k - total) * cnt / (8 * 2 ** 20)) == gold["margin_mib"]
+
+
+# ---------------------------------------------------------------- products
+
+def _scale_vals(scales):
+    return scales.view(np.float16).astype(np.float64)
+
+
+def test_product_all_positive_signs_is_group_sums():
+    g = synth.rng(10)
+    W = np.abs(synth.weights(g, 4, 384))
+    x = synth.activations_bf16(g, 2, 384)
+    signs, scales = O.pack_ref(W)
+    assert not signs.any()
+    xf = O.bf16_bits_to_f64(x)
+    y, _ = O.matmul_ref(xf, signs, scales, 384)
+    s = _scale_vals(scales)
+    for b in range(2):
+        for n in range(4):
+            exp = sum(s[n, gi] * math.fsum(xf[b, gi * 128:(gi + 1) * 128]) for gi in range(3))
+            assert y[b, n] == pytest.approx(exp, rel=1e-13, abs=1e-15)
+
+
+def test_product_one_hot_reads_back_signed_scale():
+    g = synth.rng(12)
+    W = synth.weights(g, 6, 256)
+    signs, scales = O.pack_ref(W)
+    s = _scale_vals(scales)
+    for k in (0, 1, 31, 32, 127, 128, 255):
+        x = np.zeros((1, 256))
+        x[0, k] = 1.0
+        y, _ = O.matmul_ref(x, signs, scales, 256)
+        for n in range(6):
+            sgn = -1.0 if np.signbit(W[n, k]) else 1.0
+            assert y[0, n] == sgn * s[n, k // 128]
+
+
+def test_product_equals_dense_when_weights_are_already_binary():
+    """W = +-c per group with fp16-exact c: the dequantised matrix is W itself."""
+    g = np.random.default_rng(13)
+    N, K = 5, 256
+    c = np.array([0.015625, 0.0234375, 3.0, 0.5, 1.25, 0.0078125, 2.0, 0.375, 0.75, 1.5],
+                 dtype=np.float32)[:N * 2].reshape(N, 2)
+    sg = np.where(g.random((N, K)) < 0.5, -1.0, 1.0).astype(np.float32)
+    W = sg * np.repeat(c, 128, axis=1)
+    signs, scales = O.pack_ref(W)
+    x = O.bf16_bits_to_f64(synth.activations_bf16(synth.rng(1), 3, K))
+    y, _ = O.matmul_ref(x, signs, scales, K)
+    dense = x @ W.astype(np.float64).T
+    assert np.allclose(y, dense, rtol=1e-14, atol=1e-14)
+
+
+def test_product_integer_inputs_are_exact():
+    g = np.random.default_rng(14)
+    N, K = 7, 384
+    c = (2.0 ** g.integers(-3, 3, size=(N, 3))).astype(np.float32)
+    sg = np.where(g.random((N, K)) < 0.5, -1.0, 1.0).astype(np.float32)
+    W = sg * np.repeat(c, 128, axis=1)
+    signs, scales = O.pack_ref(W)
+    x = g.integers(-2, 3, size=(2, K)).astype(np.float64)
+    y, _ = O.matmul_ref(x, signs, scales, K)
+    for b in range(2):
+        for n in range(N):
+            exact = sum(Fraction(float(W[n, k])) * int(x[b, k]) for k in range(K))
+            assert Fraction(y[b, n]) == exact
+
+
+def test_tolerance_scale_is_abs_product_sum():
+    g = synth.rng(15)
+    W = synth.weights(g, 3, 256)
+    x = O.bf16_bits_to_f64(synth.activations_bf16(g, 2, 256))
+    signs, scales = O.pack_ref(W)
+    _, bound = O.matmul_ref(x, signs, scales, 256)
+    s = _scale_vals(scales)
+    for b in range(2):
+        for n in range(3):
+            exp = math.fsum(abs(s[n, k // 128] * x[b, k]) for k in range(256))
+            assert bound[b, n] == pytest.approx(exp, rel=1e-13)
+
+
+# ---------------------------------------------------------------- DBF chain
+
+def _sylvester(n):
+    H = np.array([[1.0]])
+    while H.shape[0] < n:
+        H = np.block([[H, H], [H, -H]])
+    return H
+
+
+def test_dbf_hadamard_closed_form():
+    n = 256
+    H = _sylvester(n)
+    assert np.array_equal(H @ H, n * np.eye(n))
+    words = O.pack_bits_lsb_first((H < 0).astype(np.uint8))
+    ones = np.full(n, 0x3C00, np.uint16)
+    x = O.bf16_bits_to_f64(synth.activations_bf16(synth.rng(3), 4, n))
+    out = O.dbf_ref(ones, words, ones, words, ones, x, n, n, n)
+    assert np.array_equal(out["y"], n * x)
+
+
+def test_dbf_chain_matches_dense_reconstruction():
+    a, B1, mid, B2, b, x = synth.dbf_case(m=96, r=160, n=128, B=3, seed=21)
+    xf = O.bf16_bits_to_f64(x)
+    out = O.dbf_ref(a, B1, mid, B2, b, xf, 96, 160, 128)
+    dense = O.dbf_dense_ref(a, B1, mid, B2, b, 96, 160, 128)
+    y2 = xf @ dense.T
+    assert np.max(np.abs(out["y"] - y2)) <= 1e-12 * np.max(np.abs(y2))
+
+
+def test_dbf_chain_elementwise_loop():
+    """Explicit triple loop over the chain on a small case (independent of matmul)."""
+    m, r, n = 32, 64, 32
+    a, B1, mid, B2, b, x = synth.dbf_case(m=m, r=r, n=n, B=1, seed=22)
+    xf = O.bf16_bits_to_f64(x)[0]
+    out = O.dbf_ref(a, B1, mid, B2, b, xf[None, :], m, r, n)
+    av, mv, bv = (np.array(v, np.uint16).view(np.float16).astype(float).tolist() for v in (a, mid, b))
+
+    def bit(words, row, col):
+        return (int(words[row, col // 32]) >> (col % 32)) & 1
+
+    for i in range(m):
+        acc = []
+        for j in range(r):
+            hj = math.fsum((1 - 2 * bit(B2, j, k)) * bv[k] * xf[k] for k in range(n))
+            acc.append((1 - 2 * bit(B1, i, j)) * mv[j] * hj)
+        yi = av[i] * math.fsum(acc)
+        assert out["y"][0, i] == pytest.approx(yi, rel=1e-12, abs=1e-14)
+
+
+# ---------------------------------------------------------------- MoE
+
+def test_softmax_matches_library():
+    g = np.random.default_rng(30)
+    logits = g.standard_normal((20, 64)).astype(np.float32)
+    assert np.allclose(O.softmax_ref(logits), scipy.special.softmax(logits.astype(np.float64), axis=1),
+                       rtol=1e-14, atol=1e-16)
+
+
+def test_topk_order_and_ties():
+    p = np.array([[0.1, 0.3, 0.3, 0.05, 0.25]])
+    ids, vals = O.topk_ref(p, 3)
+    assert ids.tolist() == [[1, 2, 4]]
+    assert vals.tolist() == [[0.3, 0.3, 0.25]]
+    ids, w = O.moe_route_ref(np.zeros((2, 8), np.float32), 8)
+    assert ids.tolist() == [list(range(8))] * 2
+    assert np.allclose(w, 1.0 / 8)
+
+
+def _tiny_moe(T=3, H=128, I=128, E=4, seed=31):
+    x, logits, gate, up, down = synth.moe_case(T=T, H=H, I=I, E=E, seed=seed)
+    pk = lambda A: tuple(np.stack(v) for v in zip(*[O.pack_ref(A[e]) for e in range(E)]))
+    return O.bf16_bits_to_f64(x), logits, pk(gate), pk(up), pk(down)
+
+
+def test_moe_elementwise_loop():
+    T, H, I, E, K = 3, 128, 128, 4, 2
+    x, logits, G, U, D = _tiny_moe(T, H, I, E)
+    res = O.moe_ref(x, logits, G, U, D, H, I, E, K)
+    Gd = [O.dequant_ref(G[0][e], G[1][e], H) for e in range(E)]
+    Ud = [O.dequant_ref(U[0][e], U[1][e], H) for e in range(E)]
+    Dd = [O.dequant_ref(D[0][e], D[1][e], I) for e in range(E)]
+    for t in range(T):
+        z = [float(v) for v in logits[t]]
+        mx = max(z)
+        ez = [math.exp(v - mx) for v in z]
+        p = [v / math.fsum(ez) for v in ez]
+        order = sorted(range(E), key=lambda e: (-p[e], e))[:K]
+        for hcol in range(0, H, 37):
+            total = 0.0
+            for e in order:
+                hvec = []
+                for i in range(I):
+                    gv = math.fsum(Gd[e][i, k] * x[t, k] for k in range(H))
+                    uv = math.fsum(Ud[e][i, k] * x[t, k] for k in range(H))
+                    hvec.append(gv / (1 + math.exp(-gv)) * uv)
+                total += p[e] * math.fsum(Dd[e][hcol, i] * hvec[i] for i in range(I))
+            assert res["out"][t, hcol] == pytest.approx(total, rel=1e-10, abs=1e-12)
+
+
+def test_moe_single_expert_reduces_to_swiglu_ffn():
+    T, H, I, E = 4, 256, 128, 1
+    x, logits, G, U, D = _tiny_moe(T, H, I, E, seed=32)
+    res = O.moe_ref(x, logits, G, U, D, H, I, E, 1)
+    assert np.all(res["w"] == 1.0)
+    g = x @ O.dequant_ref(G[0][0], G[1][0], H).T
+    u = x @ O.dequant_ref(U[0][0], U[1][0], H).T
+    h = g * scipy.special.expit(g) * u
+    out = h @ O.dequant_ref(D[0][0], D[1][0], I).T
+    assert np.allclose(res["out"], out, rtol=1e-12, atol=1e-14)
+
+
+def test_moe_token_permutation_invariance():
+    T, H, I, E, K = 6, 128, 128, 8, 3
+    x, logits, G, U, D = _tiny_moe(T, H, I, E, seed=33)
+    res = O.moe_ref(x, logits, G, U, D, H, I, E, K)
+    perm = np.array([3, 0, 5, 1, 4, 2])
+    res_p = O.moe_ref(x[perm], logits[perm], G, U, D, H, I, E, K)
+    assert np.allclose(res_p["out"], res["out"][perm], rtol=1e-13, atol=1e-15)
+    p = scipy.special.softmax(logits.astype(np.float64), axis=1)
+    assert np.allclose(np.take_along_axis(p, res["ids"], 1), res["w"])
+    assert np.all(res["w"].sum(1) <= 1.0 + 1e-12)
