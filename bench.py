@@ -1,0 +1,489 @@
+#!/usr/bin/env python3
+"""Benchmark of the 1-bit group-128 hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Headline workload (one "step"): the decode GEMV sweep -- shapes 4096x4096,
+11008x4096 and 4096x11008 (out x in) at batch 1, 4 and 8, weights N(0, 0.02)
+binarised to 1-bit group-128 with fp16 scales, activations bf16 N(0, 1).  Each
+(shape, batch) pair runs R back-to-back launches (one CUDA graph) over R
+rotating copies of the packed weights whose total exceeds 4x the L2 size, so
+every launch streams its weights from HBM.  value = packed weight bytes moved
+/ device time (GB/s, all ranks, max-over-ranks time).
+
+Also measured and reported under "rows" (outside the timed steps): the
+prefill GEMM (M = 2048) TFLOP/s per shape, with an L2 flush before every
+launch; the MoE layer tokens/s and the DBF chain when those calls exist.
+
+--impl reference times the CPU oracle (fp64 numpy, the repository's test
+oracle) on the host cores over a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "1-bit GEMV HBM GB/s (% of peak); prefill GEMM TFLOP/s; MoE-layer tokens/s"
+GEMV_SHAPES = [(4096, 4096), (11008, 4096), (4096, 11008)]
+GEMV_BATCHES = [1, 4, 8]
+GEMM_SHAPES = [(14336, 4096), (4096, 14336), (14336, 14336)]
+GEMM_M = 2048
+WORKLOAD = ("decode GEMV sweep: (out x in) 4096x4096, 11008x4096, 4096x11008 at B = 1, 4, 8; "
+            "1-bit signs + fp16 scale per 128 weights; x bf16 N(0,1); W N(0,0.02)")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def packed_bytes(N: int, K: int) -> int:
+    return N * K // 8 + N * (K // 128) * 2
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """SM clock / throttle-reason sampling (NVML, every 10 ms) during the timed region."""
+
+    # NVML clocks-event reason bits
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, pci_bus_id: str | None):
+        self.pci = pci_bus_id
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self.ok = False
+
+    def __enter__(self):
+        try:
+            import pynvml as nv
+            nv.nvmlInit()
+            self.nv = nv
+            self.h = nv.nvmlDeviceGetHandleByPciBusId(self.pci) if self.pci else nv.nvmlDeviceGetHandleByIndex(0)
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(self.h, nv.NVML_CLOCK_SM)
+            self.ok = True
+            self.thread = threading.Thread(target=self._poll, daemon=True)
+            self.thread.start()
+        except Exception as e:  # NVML missing: report unsampled
+            self.err = repr(e)
+        return self
+
+    def _poll(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                try:
+                    r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                except AttributeError:
+                    r = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.01)
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self.ok:
+            self.thread.join(timeout=2)
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unsampled"], "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------ distributed
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(world, value: float) -> float:
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(world, value: float) -> float:
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ GPU arm
+
+def build_gemv_sweep(torch, ops, synth, l2_bytes: int):
+    """Packed weight copies + one CUDA graph of back-to-back launches per pair."""
+    dev = torch.device("cuda")
+    stream = torch.cuda.Stream()
+    combos = []
+    for (N, K) in GEMV_SHAPES:
+        W, _ = synth.gemv_case(N, K, 1)
+        Wd = torch.from_numpy(W).to(dev)
+        s0, c0 = ops.w1_pack(Wd)
+        del Wd
+        pb = packed_bytes(N, K)
+        R = max(64, int(math.ceil(4 * l2_bytes / pb)))
+        signs = [s0] + [s0.clone() for _ in range(R - 1)]
+        scales = [c0] + [c0.clone() for _ in range(R - 1)]
+        for B in GEMV_BATCHES:
+            x = torch.from_numpy(synth.activations_bf16(synth.rng(100 + B), B, K).view(np.int16)).to(dev).view(torch.bfloat16)
+            y = torch.empty((B, N), dtype=torch.float32, device=dev)
+            # eager warm-up (plans the launch, sets kernel attributes)
+            with torch.cuda.stream(stream):
+                for r in range(3):
+                    ops.w1_gemv(signs[r], scales[r], x, y)
+            stream.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for r in range(R):
+                    ops.w1_gemv(signs[r], scales[r], x, y)
+            combos.append({"N": N, "K": K, "B": B, "R": R, "graph": g, "x": x, "y": y,
+                           "signs": signs, "scales": scales, "bytes": pb})
+    torch.cuda.synchronize()
+    return combos, stream
+
+
+def time_gemv_steps_detailed(torch, combos, stream, steps: int, warmup: int, world: int):
+    """Timed region: `steps` sweeps; per-pair device time via events on the stream."""
+    for _ in range(warmup):
+        with torch.cuda.stream(stream):
+            for cb in combos:
+                cb["graph"].replay()
+    torch.cuda.synchronize()
+    evs = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in combos] for _ in range(steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        start.record(stream)
+        for s in range(steps):
+            for i, cb in enumerate(combos):
+                evs[s][i][0].record(stream)
+                cb["graph"].replay()
+                evs[s][i][1].record(stream)
+        end.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    total_ms = start.elapsed_time(end)
+    per_pair_ms = [sum(evs[s][i][0].elapsed_time(evs[s][i][1]) for s in range(steps)) for i in range(len(combos))]
+    return total_ms, per_pair_ms
+
+
+def gemv_e2e(torch, ops, combos, steps: int):
+    """Same sweep through the public API with pinned host buffers: every launch
+    copies its x host->device and reads y back device->host."""
+    stream = torch.cuda.Stream()
+    host = []
+    for cb in combos:
+        xh = cb["x"].cpu().pin_memory()
+        yh = torch.empty(cb["y"].shape, dtype=torch.float32).pin_memory()
+        host.append((xh, yh))
+    h2d = d2h = 0
+    launches = 0
+    torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        start.record(stream)
+        for _ in range(steps):
+            for cb, (xh, yh) in zip(combos, host):
+                for r in range(cb["R"]):
+                    cb["x"].copy_(xh, non_blocking=True)
+                    ops.w1_gemv(cb["signs"][r], cb["scales"][r], cb["x"], cb["y"])
+                    yh.copy_(cb["y"], non_blocking=True)
+                    h2d += xh.numel() * 2
+                    d2h += yh.numel() * 4
+                    launches += 1
+        end.record(stream)
+    torch.cuda.synchronize()
+    ms = start.elapsed_time(end)
+    total_bytes = sum(cb["bytes"] * cb["R"] for cb in combos) * steps
+    return {"value": total_bytes / (ms * 1e-3) / 1e9, "unit": "GB/s",
+            "h2d_bytes_per_step": h2d // steps, "d2h_bytes_per_step": d2h // steps,
+            "ms_per_step": ms / steps, "launches": launches}
+
+
+def gemm_rows(torch, ops, synth, peaks, iters: int = 8):
+    dev = torch.device("cuda")
+    flush = torch.empty(int(512 * 2 ** 20), dtype=torch.uint8, device=dev)
+    rows = []
+    for (N, K) in GEMM_SHAPES:
+        W, x = synth.gemm_case(GEMM_M, N, K)
+        Wd = torch.from_numpy(W).to(dev)
+        s, c = ops.w1_pack(Wd)
+        del Wd
+        xd = torch.from_numpy(x.view(np.int16)).to(dev).view(torch.bfloat16)
+        y = torch.empty((GEMM_M, N), dtype=torch.float32, device=dev)
+        for _ in range(3):
+            ops.w1_gemm(s, c, xd, y)
+        torch.cuda.synchronize()
+        times = []
+        for _ in range(iters):
+            flush.zero_()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record()
+            ops.w1_gemm(s, c, xd, y)
+            b.record()
+            torch.cuda.synchronize()
+            times.append(a.elapsed_time(b))
+        ms = statistics.median(times)
+        flops = 2.0 * GEMM_M * N * K
+        tf = flops / (ms * 1e-3) / 1e12
+        rows.append({"M": GEMM_M, "N": N, "K": K, "ms": ms, "TFLOP/s": tf,
+                     "frac_bf16_burst": tf / peaks["bf16_tflops"]})
+        del s, c, xd, y
+    torch.cuda.synchronize()
+    return rows
+
+
+def cpu_oracle_gemv_sample(combos_spec, packed_host, max_seconds: float = 20.0):
+    """Time the fp64 oracle on the sweep (one launch per pair) on the host."""
+    from oracle import w1_oracle as O
+    from pack_sign_g128_b200 import synth
+    t_total = 0.0
+    b_total = 0
+    done = []
+    for (N, K, B) in combos_spec:
+        s, c = packed_host[(N, K)]
+        x = O.bf16_bits_to_f64(synth.activations_bf16(synth.rng(100 + B), B, K))
+        t0 = time.perf_counter()
+        O.matmul_ref(x, s, c, K)
+        t_total += time.perf_counter() - t0
+        b_total += packed_bytes(N, K)
+        done.append(f"{N}x{K}xB{B}")
+        if t_total > max_seconds:
+            break
+    return b_total, t_total, done
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        n = [d.get("num_threads", 1) for d in info if d.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+def _pci_bus_id(torch, dev):
+    """NVML-style PCI bus id string of a torch CUDA device."""
+    try:
+        p = torch.cuda.get_device_properties(dev)
+        return f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
+    except Exception:
+        return None
+
+
+def run_gpu(args):
+    import torch
+    from pack_sign_g128_b200 import ops, synth
+
+    world, rank, local = dist_setup()
+    torch.cuda.set_device(local)
+    peaks, peaks_kind = load_peaks()
+    props = torch.cuda.get_device_properties(local)
+    l2 = int(getattr(props, "L2_cache_size", 126 * 2 ** 20) or 126 * 2 ** 20)
+
+    combos, stream = build_gemv_sweep(torch, ops, synth, l2)
+    launches_per_step = sum(cb["R"] for cb in combos)
+    bytes_per_step = sum(cb["bytes"] * cb["R"] for cb in combos)
+
+    with ClockSampler(_pci_bus_id(torch, local)) as clk:
+        total_ms, per_pair_ms = time_gemv_steps_detailed(torch, combos, stream, args.steps, args.warmup, world)
+    t_max = max_over_ranks(world, total_ms)
+    all_bytes = sum_over_ranks(world, float(bytes_per_step * args.steps))
+    value = all_bytes / (t_max * 1e-3) / 1e9
+
+    gemv_rows = []
+    for cb, ms in zip(combos, per_pair_ms):
+        per_launch_us = ms * 1e3 / (cb["R"] * args.steps)
+        gbs = cb["bytes"] / (per_launch_us * 1e-6) / 1e9
+        gemv_rows.append({"N": cb["N"], "K": cb["K"], "B": cb["B"], "launches": cb["R"],
+                          "us_per_launch": round(per_launch_us, 3), "GB/s": round(gbs, 1),
+                          "frac_hbm": round(gbs / peaks["hbm_gbs"], 4)})
+    pair_sum_ms = sum(per_pair_ms)
+    achieved = bytes_per_step * args.steps / (pair_sum_ms * 1e-3) / 1e9
+
+    e2e = gemv_e2e(torch, ops, combos, max(1, min(args.steps, 3)))
+    rows = {"gemv": gemv_rows}
+    if not args.skip_extra:
+        rows["gemm"] = gemm_rows(torch, ops, synth, peaks)
+    cpu = None
+    if rank == 0 and world == 1 and not args.skip_cpu:
+        packed_host = {}
+        for cb in combos:
+            key = (cb["N"], cb["K"])
+            if key not in packed_host:
+                packed_host[key] = (cb["signs"][0].cpu().numpy().view(np.uint32),
+                                    cb["scales"][0].cpu().view(torch.int16).numpy().view(np.uint16))
+        spec = [(cb["N"], cb["K"], cb["B"]) for cb in combos]
+        nb, secs, done = cpu_oracle_gemv_sample(spec, packed_host)
+        cpu = {"value": nb / secs / 1e9, "unit": "GB/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": f"fp64 numpy oracle (dequantise + BLAS matmul), one product per pair: {', '.join(done)}"}
+
+    out = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(t_max / args.steps, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "s8xs8->s32 tensor MMA + f32 scale fold (x bf16, 1-bit weights, fp16 scales)",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD, "launches_per_step": launches_per_step,
+                   "packed_bytes_per_step": bytes_per_step,
+                   "l2": "inputs larger than L2: each pair cycles R weight copies totalling > 4x L2",
+                   "timing": "CUDA graphs of back-to-back launches, CUDA events on the launch stream",
+                   "parallelism": f"replicas x{world} (independent sweeps, no collective)"},
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+                     "traffic": None, "kernel": "gemv_kernel", "peak_kind": peaks_kind},
+        "cpu_baseline": cpu,
+        "e2e": {k: e2e[k] for k in ("value", "unit", "h2d_bytes_per_step", "d2h_bytes_per_step")},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk.summary(),
+        "rows": rows,
+    }
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def run_reference(args):
+    """The CPU oracle as the reference arm (rank 0 only under torchrun)."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from oracle import w1_oracle as O
+    from pack_sign_g128_b200 import synth
+    # bounded sample: 512 output rows of each shape, every batch
+    rows_per = 512
+    packed = {}
+    for (N, K) in GEMV_SHAPES:
+        W, _ = synth.gemv_case(N, K, 1)
+        packed[(N, K)] = O.pack_ref_fast(W[:rows_per])
+    spec = [(N, K, B) for (N, K) in GEMV_SHAPES for B in GEMV_BATCHES]
+
+    def one_step():
+        t = 0.0
+        nbytes = 0
+        for (N, K, B) in spec:
+            s, c = packed[(N, K)]
+            x = O.bf16_bits_to_f64(synth.activations_bf16(synth.rng(100 + B), B, K))
+            t0 = time.perf_counter()
+            O.matmul_ref(x, s, c, K)
+            t += time.perf_counter() - t0
+            nbytes += packed_bytes(rows_per, K)
+        return nbytes, t
+
+    for _ in range(args.warmup):
+        one_step()
+    nb = 0
+    secs = 0.0
+    for _ in range(args.steps):
+        b, t = one_step()
+        nb += b
+        secs += t
+    value = nb / secs / 1e9
+    sample = f"fp64 numpy oracle, first {rows_per} rows of each sweep shape at B = 1, 4, 8"
+    out = {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": round(value, 4),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(secs * 1e3 / args.steps, 3),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD, "sample": sample},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": blas_threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="w1", choices=["w1", "reference"])
+    ap.add_argument("--skip-extra", action="store_true", help="only the headline sweep")
+    ap.add_argument("--skip-cpu", action="store_true", help="skip the CPU-oracle baseline")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,114 @@
+/*
+ * w1.h -- C ABI of libw1: matrix products against 1-bit weights on B200 (sm_100a).
+ *
+ * Storage format.  A weight matrix W (N rows = outputs, K columns = inputs)
+ * is stored as one sign bit per weight plus one fp16 scale per group of 128
+ * consecutive weights along K: 1 + 16/128 = 1.125 bits per weight
+ * ("Banyan: Converting Pretrained Language Models to 1-Bit Weights ...",
+ * Abstract; "Behaviour-Relearned Quantization", step 02 "Binarize experts").
+ * Bit 0 means +1 and bit 1 means -1, the IEEE sign-bit convention ("LLM
+ * binarization episode 01: DBF", section 1 "The representation").  The
+ * dequantised weight is w_hat[n,k] = s[n, k/128] * (1 - 2*bit[n,k]).
+ *
+ * Layouts (canonical, row-major, no padding):
+ *   signs   uint32 [N][K/32]   bit j of word t is column k = 32*t + j (LSB first);
+ *                              little-endian bytes equal a uint64 LSB-first block
+ *                              of 64 signs (the SIGN1 block, DBF post section 3).
+ *   scales  fp16   [N][K/128]  passed as uint16_t bit patterns.
+ *   x       bf16   [B][K]      activations, uint16_t bit patterns.
+ *   y       fp32   [B][N]      y[b,n] = sum_k w_hat[n,k] * x[b,k].
+ *
+ * Conventions for every call:
+ *   - All array pointers are DEVICE pointers owned by the caller; the library
+ *     allocates no device memory, frees nothing and keeps no state except one
+ *     status word per device.  Inputs and outputs must not alias.
+ *   - Work is enqueued asynchronously on `stream` (NULL = legacy default
+ *     stream) of the CURRENT device; the call returns without synchronising.
+ *   - Argument errors are detected on the host and returned synchronously with
+ *     nothing launched.  A failed launch returns W1_ERR_CUDA.  Conditions found
+ *     on the device (non-finite or out-of-range data, a bounded wait that gave
+ *     up) are recorded in the device status word; read them with
+ *     w1_sync_status().
+ *   - Pointers must be 16-byte aligned; K (and every contracted dimension) must
+ *     be a positive multiple of 128.
+ *   - Kernels use programmatic dependent launch: they may start while the
+ *     previous kernel in the stream finishes, but touch no data before it has
+ *     completed (only L2 prefetches of their own weight bytes are issued early).
+ */
+#ifndef W1_H_
+#define W1_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t / CUstream. */
+typedef struct CUstream_st* w1_stream_t;
+
+typedef enum {
+  W1_OK = 0,
+  W1_ERR_NULL = 1,        /* a required pointer is NULL                         */
+  W1_ERR_SHAPE = 2,       /* dimension <= 0, not a multiple of 128, batch range  */
+  W1_ERR_ALIGN = 3,       /* pointer not 16-byte aligned                         */
+  W1_ERR_NONFINITE = 4,   /* device: NaN/Inf in pack input                       */
+  W1_ERR_RANGE = 5,       /* device: a group scale overflowed fp16 (stored +inf) */
+  W1_ERR_CUDA = 6,        /* CUDA launch / runtime error                         */
+  W1_ERR_TIMEOUT = 7,     /* device: a bounded wait gave up                      */
+  W1_ERR_WORKSPACE = 8,   /* workspace missing or too small                      */
+  W1_ERR_UNSUPPORTED = 9  /* current device is not sm_100 (B200 class)           */
+} w1_status;
+
+/* Static, human-readable name of a status code. */
+const char* w1_status_string(int status);
+
+/* Synchronises `stream`, then returns and clears the current device's status
+ * word (W1_OK if no kernel recorded an error).  Returns W1_ERR_CUDA if the
+ * synchronisation itself failed. */
+int w1_sync_status(w1_stream_t stream);
+
+/*
+ * w1_pack -- binarise W along K ("Behaviour-Relearned Quantization", step 02;
+ * sign convention: DBF post, section 1).
+ *   W       fp32 [N][K], device, read only.
+ *   signs   uint32 [N][K/32] out: bit = IEEE sign bit of W (so -0.0 -> 1).
+ *   scales  fp16 [N][K/128] out: RNE_fp16( sum_{k in group} |W| / 128 ), the sum
+ *           taken exactly (the mean |w| is the least-squares scale for sign
+ *           codes; the pages name "signs plus scales" without a formula).
+ * Device-detected: NaN/Inf in W -> W1_ERR_NONFINITE (that group's scale is
+ * NaN/Inf); a finite group whose scale rounds past fp16 -> W1_ERR_RANGE (+inf).
+ */
+int w1_pack(const float* W, int64_t N, int64_t K, uint32_t* signs, uint16_t* scales,
+            w1_stream_t stream);
+
+/*
+ * w1_gemv -- decode-regime product, one vector per batch row ("LLM binarization
+ * episode 01: DBF", section 4: generation applies each matrix to one vector at
+ * a time; section 5: sign selection and addition).
+ *   y[b][n] = sum_g s[n][g] * sum_{k in g} (1 - 2*bit[n][k]) * x[b][k],  1 <= B <= 8.
+ *   signs [N][K/32], scales [N][K/128], x bf16 [B][K], y fp32 [B][N] (all device).
+ * Accuracy: |y - y_exact| <= 1e-3 * sum_k |s x_k| per element (x is taken as
+ * 24-bit fixed point per 128-group, fp32 accumulation).
+ */
+int w1_gemv(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t K,
+            const uint16_t* x, int64_t B, float* y, w1_stream_t stream);
+
+/*
+ * w1_gemm -- prefill-regime product for many token rows (DBF post, section 4:
+ * prompt processing amortises weight loads across columns).
+ *   y[m][n] = sum_g s[n][g] * sum_{k in g} (1 - 2*bit[n][k]) * x[m][k].
+ *   signs [N][K/32], scales [N][K/128], x bf16 [M][K], y fp32 [M][N] (device).
+ * tcgen05 tensor cores: the sign bits are expanded to +-1 bf16 per 128-wide K
+ * chunk, each chunk is accumulated exactly in TMEM (fp32) and folded into the
+ * running sum with its group scale.  Same accuracy bound as w1_gemv.
+ */
+int w1_gemm(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t K,
+            const uint16_t* x, int64_t M, float* y, w1_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* W1_H_ */

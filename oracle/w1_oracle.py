@@ -368,3 +368,78 @@ def moe_ref(x, logits, gate, up, down, H: int, I: int, E: int, top_k: int,
 def fsum_rows(a: np.ndarray) -> np.ndarray:
     """Correctly rounded row sums (used by tests for tight closed forms)."""
     return np.array([math.fsum(r) for r in np.asarray(a, dtype=np.float64)])
+
+
+# ---------------------------------------------------------------------------
+# Vectorised exact pack (same definition, for full-size test inputs).
+# Pinned against pack_ref / group_scale_bits in the test suite.
+# ---------------------------------------------------------------------------
+
+
+def _bit_length_minus_one(S: np.ndarray) -> np.ndarray:
+    """floor(log2 S) for positive int64 entries (0 where S == 0)."""
+    L = np.zeros(S.shape, dtype=np.int64)
+    s = S.copy()
+    for k in (32, 16, 8, 4, 2, 1):
+        m = (s >> k) > 0
+        L += np.where(m, k, 0)
+        s = np.where(m, s >> k, s)
+    return L
+
+
+def _round_scaled_int_to_fp16_bits(S: np.ndarray, p: np.ndarray) -> np.ndarray:
+    """fp16 bits of RNE(S * 2**p) for int64 S >= 0 (exact integer rounding)."""
+    S = S.astype(np.int64)
+    p = p.astype(np.int64)
+    L = _bit_length_minus_one(S)
+    e = np.maximum(L + p, -14)          # exponent of the result's binade
+    q = e - 10                          # quantum exponent
+    qb = q - p                          # quantum position in units of S
+    n = np.zeros_like(S)
+    pos = qb > 0
+    qbc = np.clip(qb, 1, 62)
+    shifted = S >> qbc
+    rem = S & ((np.int64(1) << qbc) - 1)
+    half = np.int64(1) << (qbc - 1)
+    up = (rem > half) | ((rem == half) & ((shifted & 1) == 1))
+    big = qb >= 63                       # everything below half a quantum
+    n = np.where(pos, np.where(big, 0, shifted + up.astype(np.int64)), S << np.clip(-qb, 0, 62))
+    bits = ((q + 24) << 10) + n
+    bits = np.where(bits >= 0x7C00, 0x7C00, bits)
+    bits = np.where(S == 0, 0, bits)
+    return bits.astype(np.uint16)
+
+
+def pack_ref_fast(W: np.ndarray, group: int = GROUP):
+    """Same result as pack_ref, computed with exact int64 sums per group.
+
+    Each |w| = man * 2**(ex - 150) is aligned to 2**(ex_max - 31 - 150) of its
+    group; a group holding a nonzero value below that alignment falls back to
+    group_scale_bits (exact Python integers).  Rows are processed in blocks.
+    """
+    W = np.asarray(W, dtype=np.float32)
+    if not np.all(np.isfinite(W)):
+        raise ValueError("non-finite weight")
+    N, K = W.shape
+    G = K // group
+    signs = pack_bits_lsb_first(sign_bits_ref(W))
+    scales = np.empty((N, G), dtype=np.uint16)
+    lg = int(np.log2(group))
+    for r0 in range(0, N, 256):
+        Wb = W[r0:r0 + 256]
+        nb = Wb.shape[0]
+        b = (Wb.view(np.uint32) & np.uint32(0x7FFFFFFF)).reshape(nb, G, group)
+        ex = (b >> np.uint32(23)).astype(np.int64)
+        man = (b & np.uint32(0x7FFFFF)).astype(np.int64)
+        man |= np.where(ex > 0, 0x800000, 0)
+        np.maximum(ex, 1, out=ex)
+        base = ex.max(axis=2, keepdims=True) - 31
+        sh = ex - base
+        ok = ((sh >= 0) | (man == 0)).all(axis=2)
+        np.clip(sh, 0, 31, out=sh)
+        S = np.left_shift(man, sh).sum(axis=2)
+        sc = _round_scaled_int_to_fp16_bits(S, base[..., 0] - 150 - lg)
+        for n, g in zip(*np.nonzero(~ok)):
+            sc[n, g] = group_scale_bits(Wb[n, g * group:(g + 1) * group])
+        scales[r0:r0 + nb] = sc
+    return signs, scales

@@ -1,0 +1,6 @@
+// Single translation unit for libw1 (the device status word is shared by all
+// kernels without relocatable device code).
+#include "w1_api.cu"
+#include "pack.cu"
+#include "gemv.cu"
+#include "gemm.cu"

@@ -1,0 +1,129 @@
+// Host side of the libw1 C ABI: argument validation, device capability
+// checks, the device status word and kernel launches.  See include/w1.h.
+#include <cstdint>
+#include <cstdio>
+#include <mutex>
+
+#include "w1_common.cuh"
+
+namespace w1 {
+
+
+
+cudaError_t launch_pack(const float* W, int64_t N, int64_t K, uint32_t* signs, uint16_t* scales,
+                        cudaStream_t stream, int num_sms);
+cudaError_t launch_gemv(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t K,
+                        const uint16_t* x, int B, float* y, cudaStream_t stream, int num_sms,
+                        int smem_cap);
+cudaError_t launch_gemm(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t K,
+                        const uint16_t* x, int64_t M, float* y, cudaStream_t stream, int num_sms);
+
+struct DeviceInfo {
+  bool ok = false;
+  bool valid = false;
+  int sms = 0;
+  int smem_optin = 0;
+};
+
+static constexpr int kMaxDevices = 64;
+static DeviceInfo g_info[kMaxDevices];
+static std::mutex g_info_mu;
+
+// Current device's capabilities; W1_OK only on sm_100 class parts.
+static int device_info(DeviceInfo* out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return W1_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_info_mu);
+  DeviceInfo& d = g_info[dev];
+  if (!d.valid) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
+            cudaSuccess)
+      return W1_ERR_CUDA;
+    d.ok = (major == 10 && minor == 0);
+    d.valid = true;
+  }
+  *out = d;
+  return d.ok ? W1_OK : W1_ERR_UNSUPPORTED;
+}
+
+static inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static inline int launch_result(cudaError_t e) {
+  if (e == cudaSuccess) e = cudaGetLastError();
+  return e == cudaSuccess ? W1_OK : W1_ERR_CUDA;
+}
+
+}  // namespace w1
+
+using namespace w1;
+
+extern "C" {
+
+const char* w1_status_string(int status) {
+  switch (status) {
+    case W1_OK: return "W1_OK";
+    case W1_ERR_NULL: return "W1_ERR_NULL: null pointer";
+    case W1_ERR_SHAPE: return "W1_ERR_SHAPE: invalid dimension";
+    case W1_ERR_ALIGN: return "W1_ERR_ALIGN: pointer not 16-byte aligned";
+    case W1_ERR_NONFINITE: return "W1_ERR_NONFINITE: NaN/Inf in input";
+    case W1_ERR_RANGE: return "W1_ERR_RANGE: scale overflowed fp16";
+    case W1_ERR_CUDA: return "W1_ERR_CUDA: CUDA error";
+    case W1_ERR_TIMEOUT: return "W1_ERR_TIMEOUT: bounded device wait gave up";
+    case W1_ERR_WORKSPACE: return "W1_ERR_WORKSPACE: workspace missing or too small";
+    case W1_ERR_UNSUPPORTED: return "W1_ERR_UNSUPPORTED: device is not sm_100";
+    default: return "unknown w1 status";
+  }
+}
+
+int w1_sync_status(w1_stream_t stream) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return W1_ERR_CUDA;
+  unsigned int v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_status, sizeof(v)) != cudaSuccess) return W1_ERR_CUDA;
+  if (v != 0 && cudaMemcpyToSymbol(g_status, &zero, sizeof(zero)) != cudaSuccess) return W1_ERR_CUDA;
+  return static_cast<int>(v);
+}
+
+int w1_pack(const float* W, int64_t N, int64_t K, uint32_t* signs, uint16_t* scales,
+            w1_stream_t stream) {
+  if (!W || !signs || !scales) return W1_ERR_NULL;
+  if (N <= 0 || K <= 0 || (K % 128) != 0) return W1_ERR_SHAPE;
+  if (!aligned16(W) || !aligned16(signs) || !aligned16(scales)) return W1_ERR_ALIGN;
+  DeviceInfo d;
+  int st = device_info(&d);
+  if (st != W1_OK) return st;
+  return launch_result(launch_pack(W, N, K, signs, scales, reinterpret_cast<cudaStream_t>(stream), d.sms));
+}
+
+int w1_gemv(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t K,
+            const uint16_t* x, int64_t B, float* y, w1_stream_t stream) {
+  if (!signs || !scales || !x || !y) return W1_ERR_NULL;
+  if (N <= 0 || K <= 0 || (K % 128) != 0 || B < 1 || B > 8) return W1_ERR_SHAPE;
+  if (K / 128 > (int64_t)1 << 20 || N > ((int64_t)1 << 40)) return W1_ERR_SHAPE;
+  if (!aligned16(signs) || !aligned16(scales) || !aligned16(x) || !aligned16(y)) return W1_ERR_ALIGN;
+  DeviceInfo d;
+  int st = device_info(&d);
+  if (st != W1_OK) return st;
+  const int cap = d.smem_optin < 110 * 1024 ? d.smem_optin : 110 * 1024;
+  return launch_result(launch_gemv(signs, scales, N, K, x, static_cast<int>(B), y,
+                                   reinterpret_cast<cudaStream_t>(stream), d.sms, cap));
+}
+
+int w1_gemm(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t K,
+            const uint16_t* x, int64_t M, float* y, w1_stream_t stream) {
+  if (!signs || !scales || !x || !y) return W1_ERR_NULL;
+  if (N <= 0 || K <= 0 || M <= 0 || (K % 128) != 0) return W1_ERR_SHAPE;
+  if (M > (int64_t)1 << 31 || N > (int64_t)1 << 31) return W1_ERR_SHAPE;
+  if (!aligned16(signs) || !aligned16(scales) || !aligned16(x) || !aligned16(y)) return W1_ERR_ALIGN;
+  DeviceInfo d;
+  int st = device_info(&d);
+  if (st != W1_OK) return st;
+  return launch_result(
+      launch_gemm(signs, scales, N, K, x, M, y, reinterpret_cast<cudaStream_t>(stream), d.sms));
+}
+
+}  // extern "C"

@@ -1,0 +1,79 @@
+"""Thin torch-facing wrappers over the libw1 C ABI (argument marshalling only).
+
+Tensors are CUDA tensors; 16-bit formats travel as their natural torch dtypes
+(bf16 activations, fp16 scales / diagonals) and sign words as int32 (same bits
+as the ABI's uint32).  Every call runs on the current torch CUDA stream and
+raises W1Error on a non-OK status.  No computation happens here.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import _lib
+
+
+def _ptr(t: torch.Tensor | None) -> int | None:
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("tensor must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream=None) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def sync_status(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device status word."""
+    return _lib.call("w1_sync_status", _stream(stream))
+
+
+def status_string(status: int) -> str:
+    return _lib.call("w1_status_string", int(status)).decode()
+
+
+def w1_pack(W: torch.Tensor, signs: torch.Tensor | None = None, scales: torch.Tensor | None = None,
+            stream=None):
+    """fp32 W [N, K] -> (signs int32 [N, K/32], scales fp16 [N, K/128])."""
+    N, K = W.shape
+    if W.dtype != torch.float32:
+        raise TypeError("W must be float32")
+    if signs is None:
+        signs = torch.empty((N, K // 32), dtype=torch.int32, device=W.device)
+    if scales is None:
+        scales = torch.empty((N, K // 128), dtype=torch.float16, device=W.device)
+    st = _lib.call("w1_pack", _ptr(W), N, K, _ptr(signs), _ptr(scales), _stream(stream))
+    _lib.check(st, "w1_pack")
+    return signs, scales
+
+
+def w1_gemv(signs: torch.Tensor, scales: torch.Tensor, x: torch.Tensor, y: torch.Tensor | None = None,
+            stream=None) -> torch.Tensor:
+    """y [B, N] fp32 = x [B, K] bf16 times the 1-bit matrix (B <= 8)."""
+    N = signs.shape[0]
+    K = signs.shape[1] * 32
+    B = x.shape[0]
+    if x.dtype != torch.bfloat16:
+        raise TypeError("x must be bfloat16")
+    if y is None:
+        y = torch.empty((B, N), dtype=torch.float32, device=x.device)
+    st = _lib.call("w1_gemv", _ptr(signs), _ptr(scales), N, K, _ptr(x), B, _ptr(y), _stream(stream))
+    _lib.check(st, "w1_gemv")
+    return y
+
+
+def w1_gemm(signs: torch.Tensor, scales: torch.Tensor, x: torch.Tensor, y: torch.Tensor | None = None,
+            stream=None) -> torch.Tensor:
+    """y [M, N] fp32 = x [M, K] bf16 times the 1-bit matrix (prefill)."""
+    N = signs.shape[0]
+    K = signs.shape[1] * 32
+    M = x.shape[0]
+    if x.dtype != torch.bfloat16:
+        raise TypeError("x must be bfloat16")
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.float32, device=x.device)
+    st = _lib.call("w1_gemm", _ptr(signs), _ptr(scales), N, K, _ptr(x), M, _ptr(y), _stream(stream))
+    _lib.check(st, "w1_gemm")
+    return y

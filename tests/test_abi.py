@@ -1,0 +1,59 @@
+"""The C-ABI library builds, loads and exports every symbol include/w1.h declares.
+
+Host-side argument checks are exercised without a GPU (no compute call is made:
+every call here is rejected before any CUDA work).
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+from pack_sign_g128_b200 import _lib, build
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "w1.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b((?:w1|dbf)_[a-z0-9_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return _lib.load()
+
+
+def test_header_declares_the_calls():
+    fns = declared_functions()
+    for name in ("w1_pack", "w1_gemv", "w1_gemm", "w1_status_string", "w1_sync_status"):
+        assert name in fns
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+        assert name in _lib.SIGNATURES, f"binding lacks {name}"
+
+
+def test_status_strings(lib):
+    for code, name in _lib.W1_STATUS.items():
+        assert lib.w1_status_string(code).decode().startswith(name)
+
+
+def test_host_side_argument_errors(lib):
+    good = ctypes.c_void_p(1 << 20)     # never dereferenced: calls fail validation first
+    odd = ctypes.c_void_p((1 << 20) + 4)
+    assert lib.w1_pack(None, 4, 128, good, good, None) == _lib.W1_ERR_NULL
+    assert lib.w1_pack(good, 4, 100, good, good, None) == _lib.W1_ERR_SHAPE
+    assert lib.w1_pack(good, 0, 128, good, good, None) == _lib.W1_ERR_SHAPE
+    assert lib.w1_pack(odd, 4, 128, good, good, None) == _lib.W1_ERR_ALIGN
+    assert lib.w1_gemv(good, good, 16, 128, good, 9, good, None) == _lib.W1_ERR_SHAPE
+    assert lib.w1_gemv(good, good, 16, 128, good, 0, good, None) == _lib.W1_ERR_SHAPE
+    assert lib.w1_gemv(good, None, 16, 128, good, 1, good, None) == _lib.W1_ERR_NULL
+    assert lib.w1_gemv(good, good, 16, 130, good, 1, good, None) == _lib.W1_ERR_SHAPE
+    assert lib.w1_gemv(good, good, 16, 128, odd, 1, good, None) == _lib.W1_ERR_ALIGN
+    assert lib.w1_gemm(good, good, 16, 128, good, 0, good, None) == _lib.W1_ERR_SHAPE
+    assert lib.w1_gemm(good, good, 16, 128, good, 4, None, None) == _lib.W1_ERR_NULL

@@ -391,3 +391,26 @@ def test_moe_token_permutation_invariance():
     p = scipy.special.softmax(logits.astype(np.float64), axis=1)
     assert np.allclose(np.take_along_axis(p, res["ids"], 1), res["w"])
     assert np.all(res["w"].sum(1) <= 1.0 + 1e-12)
+
+
+# ---------------------------------------------------------------- fast pack
+
+def test_fast_pack_equals_plain_pack():
+    g = synth.rng(40)
+    W = synth.weights(g, 24, 512)
+    # edge groups: ties, tie broken by a tiny value, subnormal means, zeros,
+    # overflow, a huge exponent spread (forces the exact-integer fallback)
+    M = np.float32(1.0 + 2.0 ** -11)
+    W[0, :128] = M
+    W[1, :128] = np.array([M] * 126 + [np.float32(2.0) * M, np.float32(2.0 ** -100)], np.float32)
+    W[2, :128] = np.float32(3 * 2.0 ** -25)
+    W[3, :128] = 0.0
+    W[4, :128] = -0.0
+    W[5, :128] = np.float32(70000.0)
+    W[6, 5] = np.float32(2.0 ** -140)
+    W[7, :128] = np.float32(2.0 ** -149)
+    W[8, 128:256] = np.float32(65504.0)
+    s1, c1 = O.pack_ref(W)
+    s2, c2 = O.pack_ref_fast(W)
+    assert np.array_equal(s1, s2)
+    assert np.array_equal(c1, c2)
