@@ -107,6 +107,35 @@ int w1_gemv(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t K,
 int w1_gemm(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t K,
             const uint16_t* x, int64_t M, float* y, w1_stream_t stream);
 
+/*
+ * dbf_apply -- Double Binary Factorization chain ("LLM binarization episode 01:
+ * DBF", section 1 "The representation": W ~ D_out U D_mid V D_in; section 4:
+ * evaluated as x_scaled = D_in x, h = V x_scaled, h_scaled = D_mid h,
+ * y_core = U h_scaled, y = D_out y_core -- the chain, not a rebuilt dense W).
+ *   y[b][i] = a[i] * sum_j U[i][j] * mid[j] * sum_k V[j][k] * bdiag[k] * x[b][k]
+ *   a     fp16 [m]          D_out
+ *   B1    uint32 [m][r/32]  U, sign bits (bit 0 -> +1, bit 1 -> -1), LSB first
+ *   mid   fp16 [r]          D_mid
+ *   B2    uint32 [r][n/32]  V
+ *   bdiag fp16 [n]          D_in
+ *   x     bf16 [B][n], y fp32 [B][m]; r and n multiples of 128.  No group scales.
+ * workspace: device buffer of at least dbf_workspace_size(m, r, n, B) bytes,
+ *   16-byte aligned.  Its first 4 bytes are the arrival count of a grid
+ *   barrier: ZERO them before the first call; every call leaves the count at
+ *   zero again (after a W1_ERR_TIMEOUT the caller must re-zero it).  After a call
+ *   it holds h_scaled (fp32 [min(B,8)][r], byte offset 256) of the last group
+ *   of up to 8 batch rows.  Calls sharing a workspace must not overlap.
+ * Both binary products run in one kernel for each group of up to 8 batch rows
+ * (int8 tensor-core products, a grid-wide barrier between them).  Accuracy:
+ * |y - y_exact| <= 1e-3 * |a_i| * sum_j |mid_j h_j| per element.
+ */
+int dbf_apply(const uint16_t* a, const uint32_t* B1, const uint16_t* mid, const uint32_t* B2,
+              const uint16_t* bdiag, int64_t m, int64_t r, int64_t n, const uint16_t* x, int64_t B,
+              float* y, void* workspace, size_t ws_bytes, w1_stream_t stream);
+
+/* Bytes of workspace dbf_apply needs for these sizes (0 for invalid sizes). */
+size_t dbf_workspace_size(int64_t m, int64_t r, int64_t n, int64_t B);
+
 #ifdef __cplusplus
 }
 #endif

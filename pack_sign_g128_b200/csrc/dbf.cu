@@ -1,0 +1,365 @@
+// dbf_apply: the Double Binary Factorization chain
+//
+//   y = a (.) ( B1 . ( mid (.) ( B2 . ( b (.) x ) ) ) )
+//
+// with B2 = V (r x n, input side) and B1 = U (m x r, output side) sign
+// matrices (bit 0 -> +1, bit 1 -> -1) and fp16 diagonals a = D_out [m],
+// mid = D_mid [r], b = D_in [n] ("LLM binarization episode 01: DBF",
+// section 1 "The representation" and section 4: x_scaled = D_in x,
+// h = V x_scaled, h_scaled = D_mid h, y_core = U h_scaled, y = D_out y_core).
+//
+// Small batch (B <= 8): ONE kernel runs both binary products -- the joint
+// V-D_mid-U kernel with a grid-wide synchronisation that the DBF post
+// (section 7, "CUDA/HIP: a starting point") proposes for CUDA.  Each CTA
+//  1. bulk-copies its slices of BOTH sign matrices into shared memory at
+//     once, so U streams in while V . (b x) is computed;
+//  2. phase 1: cluster-split int8-MMA product (as w1_gemv, no group scales)
+//     on b (.) x, cluster reduction, h_scaled = mid (.) h -> workspace (fp32);
+//  3. grid barrier (bounded spin; on timeout W1_ERR_TIMEOUT, no hang);
+//  4. phase 2: the same product of U with h_scaled, y = a (.) (...).
+// The intermediate stays fp32 (exact to 2^-24 relative), so the only
+// quantisation is the 23-bit fixed point of each product's input.
+#include <cstdint>
+#include <cuda_fp16.h>
+#include <mutex>
+
+#include "gemv_core.cuh"
+
+namespace w1 {
+
+struct DbfParams {
+  const uint16_t* a;    // [m] fp16
+  const uint32_t* B1;   // [m][r/32]
+  const uint16_t* mid;  // [r] fp16
+  const uint32_t* B2;   // [r][n/32]
+  const uint16_t* b;    // [n] fp16
+  const uint16_t* x;    // [B][n] bf16
+  float* y;             // [B][m]
+  float* h;             // [B][r] workspace: mid (.) (B2 . (b (.) x))
+  unsigned int* bar;    // workspace: grid barrier {count, generation}
+  int m, r, n;
+  int S;
+  int ns1, ns2;
+  int max_tiles1, max_tiles2, max_ng1, max_ng2;
+};
+
+struct DbfSmem {
+  int st1, st2, xq, xsum, xf, part, bars, total;
+};
+
+template <int NB>
+__host__ __device__ inline DbfSmem dbf_smem_layout(const DbfParams& p) {
+  constexpr int NT = GemvLayout<NB>::NT;
+  const int mng = p.max_ng1 > p.max_ng2 ? p.max_ng1 : p.max_ng2;
+  const int mt = p.max_tiles1 > p.max_tiles2 ? p.max_tiles1 : p.max_tiles2;
+  DbfSmem L;
+  int off = 0;
+  L.st1 = off;
+  off += p.ns1 * 16 * gemv_rowstride(p.max_ng1);
+  off = round_up(off, 128);
+  L.st2 = off;
+  off += p.ns2 * 16 * gemv_rowstride(p.max_ng2);
+  off = round_up(off, 128);
+  L.xq = off;
+  off += mng * 4 * NT * 256;
+  L.xsum = off;
+  off += mng * NB * 4;
+  L.xf = off;
+  off += mng * NB * 4;
+  off = round_up(off, 16);
+  L.part = off;
+  off += NB * mt * 16 * 4;
+  off = round_up(off, 8);
+  L.bars = off;
+  off += 2 * (p.ns1 + p.ns2) * 8;
+  L.total = round_up(off, 128);
+  return L;
+}
+
+// Grid-wide barrier over all CTAs of the launch (all co-resident by
+// construction of the grid).  bar[0] counts arrivals, bar[1] is the
+// generation; the last arrival resets the count, so the state is reusable by
+// the next call.  Returns false (and records W1_ERR_TIMEOUT) if the other
+// CTAs do not arrive within the spin limit.
+__device__ inline bool grid_barrier(unsigned int* bar, unsigned int nblocks) {
+  __syncthreads();
+  int ok = 1;
+  if (threadIdx.x == 0) {
+    __threadfence();
+    unsigned int gen;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(gen) : "l"(bar + 1) : "memory");
+    const unsigned int arrived = atomicAdd(bar, 1u);
+    if (arrived == nblocks - 1) {
+      atomicExch(bar, 0u);
+      __threadfence();
+      atomicAdd(bar + 1, 1u);
+    } else {
+      ok = 0;
+      for (uint32_t i = 0; i < kSpinLimit; ++i) {
+        unsigned int g;
+        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(g) : "l"(bar + 1) : "memory");
+        if (g != gen) {
+          ok = 1;
+          break;
+        }
+        __nanosleep(128);
+      }
+      if (!ok) set_status(W1_ERR_TIMEOUT);
+    }
+    __threadfence();
+  }
+  return __syncthreads_and(ok) != 0;
+}
+
+template <int NB>
+__global__ void __launch_bounds__(kGemvThreads, 1) dbf_small_kernel(const DbfParams p) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  const DbfSmem L = dbf_smem_layout<NB>(p);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
+  GemvSmemView v1{smem + L.st1, p.ns1, bars, bars + p.ns1};
+  GemvSmemView v2{smem + L.st2, p.ns2, bars + 2 * p.ns1, bars + 2 * p.ns1 + p.ns2};
+  GemvXView xv;
+  xv.xq = smem + L.xq;
+  xv.xsum = reinterpret_cast<int*>(smem + L.xsum);
+  xv.xf = reinterpret_cast<float*>(smem + L.xf);
+  xv.sc = nullptr;
+  xv.part = reinterpret_cast<float*>(smem + L.part);
+  xv.part_stride = (p.max_tiles1 > p.max_tiles2 ? p.max_tiles1 : p.max_tiles2) * 16;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int crank = static_cast<int>(cluster_ctarank());
+  const int q = static_cast<int>(cluster_id_x()), Q = static_cast<int>(nclusters_x());
+  const Split sp1 = make_split(p.r, 0, p.n >> 7, p.S, crank, q, Q);  // rows of V, K = n
+  const Split sp2 = make_split(p.m, 0, p.r >> 7, p.S, crank, q, Q);  // rows of U, K = r
+  const int64_t wrow1 = p.n >> 5, wrow2 = p.r >> 5;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < 2 * (p.ns1 + p.ns2); ++s) mbar_init(&bars[s], 1);
+    fence_mbarrier_init();
+  }
+  if (warp == kProducerWarp) {
+    prefetch_weights(sp1, p.B2, wrow1, nullptr, 0, lane);
+    prefetch_weights(sp2, p.B1, wrow2, nullptr, 0, lane);
+  }
+  __syncthreads();
+  pdl_wait();
+  pdl_launch_dependents();
+
+  int first1 = 0, first2 = 0;
+  if (warp == kProducerWarp) {
+    first1 = issue_first_tiles(v1, sp1, p.B2, wrow1, lane);
+    first2 = issue_first_tiles(v2, sp2, p.B1, wrow2, lane);
+  }
+
+  // ---- phase 1: h_scaled = mid (.) (V . (b (.) x))
+  {
+    const uint16_t* xb = p.x;
+    const uint16_t* bd = p.b;
+    const int n = p.n;
+    quantise_input<NB>(xv, sp1,
+                       [&](int bb, int k, float (&vv)[16]) {
+                         load16_bf16(xb + static_cast<int64_t>(bb) * n + k, vv);
+                         const uint4 d0 = *reinterpret_cast<const uint4*>(bd + k);
+                         const uint4 d1 = *reinterpret_cast<const uint4*>(bd + k + 8);
+                         const uint32_t dw[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
+#pragma unroll
+                         for (int i = 0; i < 8; ++i) {
+                           const __half2 hh = *reinterpret_cast<const __half2*>(&dw[i]);
+                           vv[2 * i] *= __low2float(hh);
+                           vv[2 * i + 1] *= __high2float(hh);
+                         }
+                       },
+                       kGemvThreads);
+    __syncthreads();
+    if (warp == kProducerWarp)
+      produce_rest(v1, sp1, p.B2, wrow1, first1, lane);
+    else
+      consume_tiles<NB, false>(v1, xv, sp1, warp, lane);
+    cluster_sync();
+    float* h = p.h;
+    const uint16_t* mid = p.mid;
+    const int r = p.r;
+    cluster_reduce<NB>(xv, sp1, p.S, crank,
+                       [&](int bb, int64_t row, float val) {
+                         h[static_cast<int64_t>(bb) * r + row] = __half2float(__ushort_as_half(mid[row])) * val;
+                       },
+                       kGemvThreads);
+  }
+  // ---- every CTA's h_scaled is in memory
+  if (!grid_barrier(p.bar, gridDim.x)) {
+    cluster_sync();
+    return;
+  }
+  // ---- phase 2: y = a (.) (U . h_scaled)
+  {
+    const float* h = p.h;
+    const int r = p.r;
+    quantise_input<NB>(xv, sp2,
+                       [&](int bb, int k, float (&vv)[16]) {
+                         const float4* hp = reinterpret_cast<const float4*>(h + static_cast<int64_t>(bb) * r + k);
+#pragma unroll
+                         for (int i = 0; i < 4; ++i) {
+                           const float4 f = __ldcg(hp + i);
+                           vv[4 * i] = f.x;
+                           vv[4 * i + 1] = f.y;
+                           vv[4 * i + 2] = f.z;
+                           vv[4 * i + 3] = f.w;
+                         }
+                       },
+                       kGemvThreads);
+    __syncthreads();
+    if (warp == kProducerWarp)
+      produce_rest(v2, sp2, p.B1, wrow2, first2, lane);
+    else
+      consume_tiles<NB, false>(v2, xv, sp2, warp, lane);
+    cluster_sync();
+    float* y = p.y;
+    const uint16_t* a = p.a;
+    const int m = p.m;
+    cluster_reduce<NB>(xv, sp2, p.S, crank,
+                       [&](int bb, int64_t row, float val) {
+                         y[static_cast<int64_t>(bb) * m + row] = __half2float(__ushort_as_half(a[row])) * val;
+                       },
+                       kGemvThreads);
+    cluster_sync();
+  }
+}
+
+// ------------------------------------------------------------------ host side
+
+template <int NB>
+static int dbf_max_clusters(int S, int smem_bytes) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(S * 64));
+  cfg.blockDim = dim3(kGemvThreads);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem_bytes);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(S);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int nclusters = 0;
+  if (cudaFuncSetAttribute(dbf_small_kernel<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes) !=
+          cudaSuccess ||
+      cudaOccupancyMaxActiveClusters(&nclusters, dbf_small_kernel<NB>, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  return nclusters;
+}
+
+// Size the stages of one product: every tile if it fits in `budget` bytes.
+static int stages_for(int max_tiles, int max_ng, int budget) {
+  const int per = 16 * gemv_rowstride(max_ng) + 16;
+  int ns = max_tiles;
+  if (ns * per > budget) ns = budget / per;
+  return ns;
+}
+
+template <int NB>
+static cudaError_t launch_dbf_small_nb(DbfParams p, cudaStream_t stream, int num_sms, int smem_cap) {
+  // K split S and cluster count Q: all CTAs must be co-resident (grid barrier)
+  const int T1 = (p.r + 15) / 16, T2 = (p.m + 15) / 16;
+  const int NG1 = p.n / 128, NG2 = p.r / 128;
+  double best = 1e300;
+  DbfParams bestp = p;
+  int bestQ = 0;
+  for (int S = 1; S <= 8; S *= 2) {
+    if (S > NG1 || S > NG2) break;
+    DbfParams c = p;
+    c.S = S;
+    int Q = num_sms / S;
+    for (int iter = 0; iter < 2; ++iter) {
+      c.max_tiles1 = (T1 + Q - 1) / Q;
+      c.max_tiles2 = (T2 + Q - 1) / Q;
+      c.max_ng1 = (NG1 + S - 1) / S;
+      c.max_ng2 = (NG2 + S - 1) / S;
+      c.ns1 = c.ns2 = 0;
+      const int base = dbf_smem_layout<NB>(c).total + 256;
+      const int budget = smem_cap - base;
+      c.ns1 = stages_for(c.max_tiles1, c.max_ng1, budget / 2);
+      c.ns2 = stages_for(c.max_tiles2, c.max_ng2, budget / 2);
+      if (c.ns1 < 1 || c.ns2 < 1) break;
+      const int occ = dbf_max_clusters<NB>(S, dbf_smem_layout<NB>(c).total);
+      if (occ <= 0) break;
+      if (occ >= Q) {
+        const double work = static_cast<double>(c.max_tiles1) * c.max_ng1 + static_cast<double>(c.max_tiles2) * c.max_ng2;
+        const double cost = work * 2048.0 * (0.55 + 0.05 * NB) + NB * (c.max_ng1 + c.max_ng2) * 128.0 * 9.0 +
+                            (S > 1 ? 3000.0 : 0.0);
+        if (cost < best) {
+          best = cost;
+          bestp = c;
+          bestQ = Q;
+        }
+        break;
+      }
+      Q = occ;
+    }
+  }
+  if (bestQ == 0) return cudaErrorInvalidConfiguration;
+  p = bestp;
+  const int smem = dbf_smem_layout<NB>(p).total;
+  cudaError_t err = cudaFuncSetAttribute(dbf_small_kernel<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (err != cudaSuccess) return err;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(bestQ * p.S));
+  cfg.blockDim = dim3(kGemvThreads);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(p.S);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, dbf_small_kernel<NB>, p);
+}
+
+size_t dbf_workspace_bytes(int64_t m, int64_t r, int64_t n, int64_t B) {
+  (void)m;
+  (void)n;
+  const int64_t rows = B < 8 ? B : 8;
+  return static_cast<size_t>(256 + 4 * rows * r);
+}
+
+cudaError_t launch_dbf(const uint16_t* a, const uint32_t* B1, const uint16_t* mid, const uint32_t* B2,
+                       const uint16_t* b, int64_t m, int64_t r, int64_t n, const uint16_t* x, int64_t B,
+                       float* y, void* workspace, cudaStream_t stream, int num_sms, int smem_cap) {
+  DbfParams p = {};
+  p.a = a;
+  p.B1 = B1;
+  p.mid = mid;
+  p.B2 = B2;
+  p.b = b;
+  p.bar = reinterpret_cast<unsigned int*>(workspace);
+  p.h = reinterpret_cast<float*>(static_cast<unsigned char*>(workspace) + 256);
+  p.m = static_cast<int>(m);
+  p.r = static_cast<int>(r);
+  p.n = static_cast<int>(n);
+  // batches of up to 8 rows through the fused small-batch kernel
+  for (int64_t b0 = 0; b0 < B; b0 += 8) {
+    const int nb = static_cast<int>((B - b0) < 8 ? (B - b0) : 8);
+    p.x = x + b0 * n;
+    p.y = y + b0 * m;
+    cudaError_t err;
+    switch (nb) {
+      case 1: err = launch_dbf_small_nb<1>(p, stream, num_sms, smem_cap); break;
+      case 2: err = launch_dbf_small_nb<2>(p, stream, num_sms, smem_cap); break;
+      case 3: err = launch_dbf_small_nb<3>(p, stream, num_sms, smem_cap); break;
+      case 4: err = launch_dbf_small_nb<4>(p, stream, num_sms, smem_cap); break;
+      case 5: err = launch_dbf_small_nb<5>(p, stream, num_sms, smem_cap); break;
+      case 6: err = launch_dbf_small_nb<6>(p, stream, num_sms, smem_cap); break;
+      case 7: err = launch_dbf_small_nb<7>(p, stream, num_sms, smem_cap); break;
+      default: err = launch_dbf_small_nb<8>(p, stream, num_sms, smem_cap); break;
+    }
+    if (err != cudaSuccess) return err;
+  }
+  return cudaSuccess;
+}
+
+}  // namespace w1

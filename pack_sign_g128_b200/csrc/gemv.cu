@@ -27,9 +27,11 @@
 //    CTA only prefetches its weight bytes into L2.
 #include <cstdint>
 #include <cuda_fp16.h>
+#include <cstdio>
+#include <cstdlib>
 #include <mutex>
 
-#include "w1_common.cuh"
+#include "gemv_core.cuh"
 
 namespace w1 {
 
@@ -48,24 +50,6 @@ struct GemvParams {
   int max_tiles;    // max 16-row tiles per cluster
   int max_ng;       // max groups per CTA
 };
-
-constexpr int kConsumerWarps = 8;
-constexpr int kGemvThreads = (kConsumerWarps + 1) * 32;
-
-template <int NB>
-struct GemvLayout {
-  static constexpr int NT = (NB <= 4) ? 2 : 3;
-};
-
-__host__ __device__ inline int gemv_rowstride(int ng) {
-  // bytes per row slice in a stage; an odd multiple of 16 keeps the 8 rows of
-  // a warp's LDS.32 on distinct banks
-  int rs = ng * 16;
-  if ((ng & 1) == 0) rs += 16;
-  return rs;
-}
-
-__host__ __device__ inline int round_up(int v, int a) { return (v + a - 1) / a * a; }
 
 struct GemvSmem {
   int stages, xq, xsum, xf, sc, part, bars, total;
@@ -98,273 +82,79 @@ __host__ __device__ inline GemvSmem gemv_smem_layout(int ns, int max_tiles, int 
   return L;
 }
 
-// -(bit q + 4i of w) for i = 0..3, as int8 bytes; the shifted copies of w are
-// precomputed (w3 = w >> 3, w16 = w >> 16, w19 = w >> 19).
-__device__ __forceinline__ uint32_t extract_q(int q, uint32_t w, uint32_t w3, uint32_t w16,
-                                              uint32_t w19) {
-  switch (q) {
-    case 0: return prmt(0xFF00FF00u, 0xFF00FF00u, w);
-    case 1: return prmt(0xFFFF0000u, 0xFFFF0000u, w);
-    case 2: return prmt(0x00000000u, 0xFFFFFFFFu, w);
-    case 3: return prmt(0xFF00FF00u, 0xFF00FF00u, w3);
-    case 4: return prmt(0xFF00FF00u, 0xFF00FF00u, w16);
-    case 5: return prmt(0xFFFF0000u, 0xFFFF0000u, w16);
-    case 6: return prmt(0x00000000u, 0xFFFFFFFFu, w16);
-    default: return prmt(0xFF00FF00u, 0xFF00FF00u, w19);
+__device__ __forceinline__ float bf16_bits_to_f32(uint32_t b) { return __uint_as_float(b << 16); }
+
+// 16 consecutive bf16 activations as fp32.
+__device__ __forceinline__ void load16_bf16(const uint16_t* p, float (&v)[16]) {
+  const uint4 u0 = *reinterpret_cast<const uint4*>(p);
+  const uint4 u1 = *reinterpret_cast<const uint4*>(p + 8);
+  const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    v[2 * i] = bf16_bits_to_f32(w[i] & 0xFFFFu);
+    v[2 * i + 1] = bf16_bits_to_f32(w[i] >> 16);
   }
 }
 
-__device__ __forceinline__ float bf16_bits_to_f32(uint32_t b) { return __uint_as_float(b << 16); }
-
 template <int NB>
 __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams p) {
-  constexpr int NT = GemvLayout<NB>::NT;
   extern __shared__ __align__(128) unsigned char smem[];
   const GemvSmem L = gemv_smem_layout<NB>(p.ns, p.max_tiles, p.max_ng);
-  unsigned char* stages = smem + L.stages;
-  unsigned char* xq = smem + L.xq;
-  int* xsum = reinterpret_cast<int*>(smem + L.xsum);
-  float* xf = reinterpret_cast<float*>(smem + L.xf);
-  uint16_t* sc = reinterpret_cast<uint16_t*>(smem + L.sc);
-  float* part = reinterpret_cast<float*>(smem + L.part);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bars);
-  uint64_t* empty = full + p.ns;
+  GemvSmemView v;
+  v.stages = smem + L.stages;
+  v.ns = p.ns;
+  v.full = reinterpret_cast<uint64_t*>(smem + L.bars);
+  v.empty = v.full + p.ns;
+  GemvXView xv;
+  xv.xq = smem + L.xq;
+  xv.xsum = reinterpret_cast<int*>(smem + L.xsum);
+  xv.xf = reinterpret_cast<float*>(smem + L.xf);
+  xv.sc = reinterpret_cast<uint16_t*>(smem + L.sc);
+  xv.part = reinterpret_cast<float*>(smem + L.part);
+  xv.part_stride = p.max_tiles * 16;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int S = p.S;
   const int crank = static_cast<int>(cluster_ctarank());
-  const int q = static_cast<int>(cluster_id_x());
-  const int Q = static_cast<int>(nclusters_x());
-
-  // ---- work split: cluster -> 16-row tiles, CTA -> K groups
-  const int T16 = (p.rows + 15) >> 4;
-  const int tq0 = static_cast<int>((static_cast<int64_t>(q) * T16) / Q);
-  const int tq1 = static_cast<int>((static_cast<int64_t>(q + 1) * T16) / Q);
-  const int ntiles = tq1 - tq0;
-  const int g0 = (crank * p.NG) / S;
-  const int g1 = ((crank + 1) * p.NG) / S;
-  const int ng = g1 - g0;
-  const int rowstride = gemv_rowstride(ng);
-  const int stage_bytes = 16 * rowstride;
-  const int64_t wrow = p.K >> 5;            // words per weight row
-  const int64_t r_first = p.row_base + static_cast<int64_t>(tq0) * 16;
-  const int rows_c = min(ntiles * 16, static_cast<int>(p.row_base + p.rows - r_first));
+  const Split sp = make_split(p.rows, p.row_base, p.NG, p.S, crank, static_cast<int>(cluster_id_x()),
+                              static_cast<int>(nclusters_x()));
+  const int64_t wrow = p.K >> 5;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < p.ns; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
+      mbar_init(&v.full[s], 1);
+      mbar_init(&v.empty[s], 1);
     }
     fence_mbarrier_init();
   }
-  // L2 prefetch of this CTA's weight bytes (safe before the dependency wait:
-  // a prefetch returns no data to the kernel)
-  if (warp == kConsumerWarps) {
-    for (int r = lane; r < rows_c; r += 32) {
-      const int64_t row = r_first + r;
-      bulk_prefetch_l2(p.signs + row * wrow + 4 * g0, static_cast<uint32_t>(ng * 16));
-      prefetch_l2(p.scales + row * p.NG + g0);
-    }
-  }
+  if (warp == kProducerWarp) prefetch_weights(sp, p.signs, wrow, p.scales, p.NG, lane);
   __syncthreads();
   pdl_wait();
-
-  // ---- producer: issue the first stages immediately
-  auto issue_tile = [&](int it) {
-    const int s = it % p.ns;
-    const int64_t row0 = r_first + static_cast<int64_t>(it) * 16;
-    const int64_t nr64 = p.row_base + p.rows - row0;
-    const int nr = nr64 < 16 ? static_cast<int>(nr64) : 16;
-    if (lane == 0) mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(nr * ng * 16));
-    __syncwarp();
-    if (lane < nr) {
-      bulk_g2s(stages + s * stage_bytes + lane * rowstride, p.signs + (row0 + lane) * wrow + 4 * g0,
-               static_cast<uint32_t>(ng * 16), &full[s]);
-    }
-  };
-  const int first = min(ntiles, p.ns);
-  if (warp == kConsumerWarps) {
-    for (int it = 0; it < first; ++it) issue_tile(it);
-  }
-
-  // ---- x preparation (all warps): zero the digit planes, then quantise
-  {
-    uint4* z = reinterpret_cast<uint4*>(xq);
-    const int n16 = ng * 4 * NT * 256 / 16;
-    for (int i = threadIdx.x; i < n16; i += kGemvThreads) z[i] = make_uint4(0, 0, 0, 0);
-  }
-  __syncthreads();
-  {
-    const int sub = lane & 7;       // 8 lanes per (b, group) item
-    const int t = sub >> 1;         // word within group
-    const int hh = sub & 1;         // half word (bits 16*hh .. 16*hh+15)
-    const int items = NB * ng;
-    for (int base = warp * 4; base < items; base += (kConsumerWarps + 1) * 4) {
-      const int item = base + (lane >> 3);
-      const bool valid = item < items;
-      const int b = valid ? item / ng : 0;
-      const int gl = valid ? item - b * ng : 0;
-      float v[16];
-      if (valid) {
-        const uint16_t* xp = p.x + static_cast<int64_t>(b) * p.K + 128 * (g0 + gl) + 32 * t + 16 * hh;
-        const uint4 u0 = *reinterpret_cast<const uint4*>(xp);
-        const uint4 u1 = *reinterpret_cast<const uint4*>(xp + 8);
-        const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          v[2 * i] = bf16_bits_to_f32(w[i] & 0xFFFFu);
-          v[2 * i + 1] = bf16_bits_to_f32(w[i] >> 16);
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) v[i] = 0.f;
-      }
-      float mx = 0.f;
-#pragma unroll
-      for (int i = 0; i < 16; ++i) mx = fmaxf(mx, fabsf(v[i]));
-      mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 1));
-      mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 2));
-      mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 4));
-      int E = 0;
-      if (mx > 0.f) frexpf(mx, &E);  // mx = f * 2^E, f in [0.5, 1)
-      const int sf = 22 - E;
-      const int sf1 = sf / 2, sf2 = sf - sf1;
-      const float m1 = __uint_as_float(static_cast<uint32_t>(sf1 + 127) << 23);
-      const float m2 = __uint_as_float(static_cast<uint32_t>(sf2 + 127) << 23);
-      uint32_t e[16];
-      uint32_t bsum = 0;
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        // x * 2^sf rounded to an integer via the 1.5*2^23 magic constant:
-        // bits = 0x4B400000 + round(x * 2^sf) exactly for |x 2^sf| < 2^22
-        const uint32_t bits = __float_as_uint(fmaf(v[i] * m1, m2, 12582912.0f));
-        bsum += bits;
-        e[i] = (bits - 0x4ABF7F80u) ^ 0x00808080u;  // three signed digit bytes
-      }
-      int xs = static_cast<int>(bsum - 16u * 0x4B400000u);
-      xs += __shfl_xor_sync(0xFFFFFFFFu, xs, 1);
-      xs += __shfl_xor_sync(0xFFFFFFFFu, xs, 2);
-      xs += __shfl_xor_sync(0xFFFFFFFFu, xs, 4);
-      if (valid) {
-        if (sub == 0) {
-          xsum[gl * NB + b] = xs;
-          xf[gl * NB + b] = ldexpf(1.0f, E - 22);
-        }
-        // columns of the three planes of batch row b
-        const int jt_hi = (b < 4) ? 0 : 2;
-        const int c_hi = 2 * (b & 3);
-        const int c_lo = (b < 4) ? 2 * b : 2 * (b - 4) + 1;
-#pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          // elements r, r+4, r+8, r+12 of this lane share q = r + 4*hh
-          const uint32_t e0 = e[r], e1 = e[r + 4], e2 = e[r + 8], e3 = e[r + 12];
-          const uint32_t p01 = prmt(e0, e1, 0x5140u), p23 = prmt(e2, e3, 0x5140u);
-          const uint32_t d0 = prmt(p01, p23, 0x5410u);
-          const uint32_t d1 = prmt(p01, p23, 0x7632u);
-          const uint32_t d2 = prmt(prmt(e0, e1, 0x0062u), prmt(e2, e3, 0x0062u), 0x5410u);
-          const int qq = r + 4 * hh;
-          const int m = qq >> 1, h = qq & 1;
-          unsigned char* slot = xq + ((gl * 4 + m) * NT) * 256 + t * 8 + h * 4;
-          *reinterpret_cast<uint32_t*>(slot + jt_hi * 256 + c_hi * 32) = d2;
-          *reinterpret_cast<uint32_t*>(slot + jt_hi * 256 + (c_hi + 1) * 32) = d1;
-          *reinterpret_cast<uint32_t*>(slot + 1 * 256 + c_lo * 32) = d0;
-        }
-      }
-    }
-  }
-  // ---- scales of this CTA's rows and groups -> shared memory
-  for (int i = threadIdx.x; i < rows_c * ng; i += kGemvThreads) {
-    const int r = i / ng, gl = i - r * ng;
-    sc[r * ng + gl] = p.scales[(r_first + r) * p.NG + g0 + gl];
-  }
-  __syncthreads();
-
-  if (warp == kConsumerWarps) {
-    // ---- producer: remaining tiles as stages free up
-    for (int it = first; it < ntiles; ++it) {
-      const int s = it % p.ns;
-      if (!mbar_wait_warp(&empty[s], ((it / p.ns) - 1) & 1)) break;
-      issue_tile(it);
-    }
-  } else {
-    // ---- consumers
-    const int g = lane >> 2, t = lane & 3;
-    for (int it = warp; it < ntiles; it += kConsumerWarps) {
-      const int s = it % p.ns;
-      if (!mbar_wait_warp(&full[s], (it / p.ns) & 1)) break;
-      const unsigned char* st = stages + s * stage_bytes;
-      const int rl0 = it * 16;  // local row of the tile within this cluster
-      float acc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
-      for (int gl = 0; gl < ng; ++gl) {
-        const uint32_t wA = *reinterpret_cast<const uint32_t*>(st + g * rowstride + (4 * gl + t) * 4);
-        const uint32_t wB =
-            *reinterpret_cast<const uint32_t*>(st + (g + 8) * rowstride + (4 * gl + t) * 4);
-        const uint32_t wA3 = wA >> 3, wA16 = wA >> 16, wA19 = wA >> 19;
-        const uint32_t wB3 = wB >> 3, wB16 = wB >> 16, wB19 = wB >> 19;
-        int C[NT][4];
-#pragma unroll
-        for (int j = 0; j < NT; ++j) C[j][0] = C[j][1] = C[j][2] = C[j][3] = 0;
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {
-          uint32_t a[4];
-          a[0] = extract_q(2 * m, wA, wA3, wA16, wA19);
-          a[1] = extract_q(2 * m, wB, wB3, wB16, wB19);
-          a[2] = extract_q(2 * m + 1, wA, wA3, wA16, wA19);
-          a[3] = extract_q(2 * m + 1, wB, wB3, wB16, wB19);
-#pragma unroll
-          for (int j = 0; j < NT; ++j) {
-            const uint2 bb = *reinterpret_cast<const uint2*>(xq + ((gl * 4 + m) * NT + j) * 256 +
-                                                            g * 32 + t * 8);
-            mma_s8_16832(C[j], a, bb.x, bb.y, C[j]);
-          }
-        }
-        const int rA = rl0 + g, rB = rl0 + g + 8;
-        const float sA = (rA < rows_c) ? __half2float(__ushort_as_half(sc[rA * ng + gl])) : 0.f;
-        const float sB = (rB < rows_c) ? __half2float(__ushort_as_half(sc[rB * ng + gl])) : 0.f;
-#pragma unroll
-        for (int be = 0; be < 2; ++be) {
-          const int b = t + 4 * be;
-          if (b < NB) {
-            const int jh = be ? 2 : 0;
-            const int X = xsum[gl * NB + b];
-            const float f = xf[gl * NB + b];
-            const int VA = X + 131072 * C[jh][0] + 512 * C[jh][1] + 2 * C[1][be ? 1 : 0];
-            const int VB = X + 131072 * C[jh][2] + 512 * C[jh][3] + 2 * C[1][be ? 3 : 2];
-            acc[0][be] = fmaf(sA * f, static_cast<float>(VA), acc[0][be]);
-            acc[1][be] = fmaf(sB * f, static_cast<float>(VB), acc[1][be]);
-          }
-        }
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[s]);
-      const int rA = rl0 + g, rB = rl0 + g + 8;
-#pragma unroll
-      for (int be = 0; be < 2; ++be) {
-        const int b = t + 4 * be;
-        if (b < NB) {
-          if (rA < rows_c) part[b * (p.max_tiles * 16) + rA] = acc[0][be];
-          if (rB < rows_c) part[b * (p.max_tiles * 16) + rB] = acc[1][be];
-        }
-      }
-    }
-  }
+  // the next kernel in the stream may start now: its CTAs only prefetch their
+  // own weights into L2 until this grid has completed
   pdl_launch_dependents();
-  // ---- cluster reduction of the S partial sums, fixed order
+
+  int first = 0;
+  if (warp == kProducerWarp) first = issue_first_tiles(v, sp, p.signs, wrow, lane);
+
+  // activations -> digit planes; scales of this CTA's rows and groups -> smem
+  const uint16_t* xb = p.x;
+  const int64_t K = p.K;
+  quantise_input<NB>(xv, sp,
+                     [&](int b, int k, float (&vv)[16]) { load16_bf16(xb + static_cast<int64_t>(b) * K + k, vv); },
+                     kGemvThreads);
+  stage_scales(xv, sp, p.scales, p.NG, kGemvThreads);
+  __syncthreads();
+
+  if (warp == kProducerWarp)
+    produce_rest(v, sp, p.signs, wrow, first, lane);
+  else
+    consume_tiles<NB, true>(v, xv, sp, warp, lane);
   cluster_sync();
-  {
-    const int r_lo = (crank * rows_c) / S;
-    const int r_hi = ((crank + 1) * rows_c) / S;
-    const int span = r_hi - r_lo;
-    const uint32_t part_base = smem_u32(part);
-    for (int i = threadIdx.x; i < span * NB; i += kGemvThreads) {
-      const int b = i / span, r = r_lo + (i - b * span);
-      const uint32_t off = static_cast<uint32_t>((b * (p.max_tiles * 16) + r) * 4);
-      float sum = 0.f;
-      for (int c = 0; c < S; ++c) sum += ld_dsmem_f32(map_shared_rank(part_base + off, c));
-      p.y[static_cast<int64_t>(b) * p.N + r_first + r] = sum;
-    }
-  }
+  float* y = p.y;
+  const int64_t N = p.N;
+  cluster_reduce<NB>(xv, sp, p.S, crank, [&](int b, int64_t row, float val) { y[b * N + row] = val; },
+                     kGemvThreads);
   cluster_sync();
 }
 
@@ -516,6 +306,15 @@ cudaError_t launch_gemv(const uint32_t* signs, const uint16_t* scales, int64_t N
     }
     gemv_plan_store(rows, NG, B, num_sms, smem_cap, Q, S);
     }
+    if (const char* f = getenv("W1_GEMV_SPLIT")) {  // tuning knob: force the K split
+      const int fs = atoi(f);
+      if (fs == 1 || fs == 2 || fs == 4 || fs == 8) {
+        if (fs != S) Q = (num_sms / fs < (rows + 15) / 16) ? num_sms / fs : static_cast<int>((rows + 15) / 16);
+        S = fs;
+      }
+    }
+    if (getenv("W1_VERBOSE")) fprintf(stderr, "w1_gemv plan: rows=%d K=%lld B=%d -> clusters=%d split=%d\n", rows,
+                                      static_cast<long long>(K), B, Q, S);
     GemvParams p = {};
     p.signs = signs;
     p.scales = scales;

@@ -4,3 +4,4 @@
 #include "pack.cu"
 #include "gemv.cu"
 #include "gemm.cu"
+#include "dbf.cu"

@@ -18,6 +18,11 @@ cudaError_t launch_gemv(const uint32_t* signs, const uint16_t* scales, int64_t N
 cudaError_t launch_gemm(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t K,
                         const uint16_t* x, int64_t M, float* y, cudaStream_t stream, int num_sms);
 
+cudaError_t launch_dbf(const uint16_t* a, const uint32_t* B1, const uint16_t* mid, const uint32_t* B2,
+                       const uint16_t* b, int64_t m, int64_t r, int64_t n, const uint16_t* x, int64_t B,
+                       float* y, void* workspace, cudaStream_t stream, int num_sms, int smem_cap);
+size_t dbf_workspace_bytes(int64_t m, int64_t r, int64_t n, int64_t B);
+
 struct DeviceInfo {
   bool ok = false;
   bool valid = false;
@@ -124,6 +129,30 @@ int w1_gemm(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t K,
   if (st != W1_OK) return st;
   return launch_result(
       launch_gemm(signs, scales, N, K, x, M, y, reinterpret_cast<cudaStream_t>(stream), d.sms));
+}
+
+size_t dbf_workspace_size(int64_t m, int64_t r, int64_t n, int64_t B) {
+  if (m <= 0 || r <= 0 || n <= 0 || B <= 0) return 0;
+  return dbf_workspace_bytes(m, r, n, B);
+}
+
+int dbf_apply(const uint16_t* a, const uint32_t* B1, const uint16_t* mid, const uint32_t* B2,
+              const uint16_t* b, int64_t m, int64_t r, int64_t n, const uint16_t* x, int64_t B, float* y,
+              void* workspace, size_t ws_bytes, w1_stream_t stream) {
+  if (!a || !B1 || !mid || !B2 || !b || !x || !y) return W1_ERR_NULL;
+  if (m <= 0 || r <= 0 || n <= 0 || B <= 0 || (r % 128) != 0 || (n % 128) != 0) return W1_ERR_SHAPE;
+  if (m > (int64_t)1 << 30 || r > (int64_t)1 << 30 || n > (int64_t)1 << 30) return W1_ERR_SHAPE;
+  if (!aligned16(a) || !aligned16(B1) || !aligned16(mid) || !aligned16(B2) || !aligned16(b) || !aligned16(x) ||
+      !aligned16(y))
+    return W1_ERR_ALIGN;
+  if (!workspace || ws_bytes < dbf_workspace_bytes(m, r, n, B)) return W1_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return W1_ERR_ALIGN;
+  DeviceInfo d;
+  int st = device_info(&d);
+  if (st != W1_OK) return st;
+  const int cap = d.smem_optin < 200 * 1024 ? d.smem_optin : 200 * 1024;
+  return launch_result(launch_dbf(a, B1, mid, B2, b, m, r, n, x, B, y, workspace,
+                                  reinterpret_cast<cudaStream_t>(stream), d.sms, cap));
 }
 
 }  // extern "C"

@@ -77,3 +77,31 @@ def w1_gemm(signs: torch.Tensor, scales: torch.Tensor, x: torch.Tensor, y: torch
     st = _lib.call("w1_gemm", _ptr(signs), _ptr(scales), N, K, _ptr(x), M, _ptr(y), _stream(stream))
     _lib.check(st, "w1_gemm")
     return y
+
+
+def dbf_workspace(m: int, r: int, n: int, B: int, device=None) -> torch.Tensor:
+    """A zeroed workspace for dbf_apply (the grid-barrier words start at zero)."""
+    nbytes = _lib.call("dbf_workspace_size", m, r, n, B)
+    if nbytes == 0:
+        raise ValueError("invalid DBF sizes")
+    return torch.zeros(nbytes, dtype=torch.uint8, device=device or "cuda")
+
+
+def dbf_apply(a: torch.Tensor, B1: torch.Tensor, mid: torch.Tensor, B2: torch.Tensor, b: torch.Tensor,
+              x: torch.Tensor, y: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+              stream=None) -> torch.Tensor:
+    """y [B, m] = a * (U @ (mid * (V @ (b * x)))) with U = B1 [m, r/32], V = B2 [r, n/32] sign words."""
+    m = a.shape[0]
+    r = mid.shape[0]
+    n = b.shape[0]
+    B = x.shape[0]
+    if x.dtype != torch.bfloat16:
+        raise TypeError("x must be bfloat16")
+    if workspace is None:
+        workspace = dbf_workspace(m, r, n, B, x.device)
+    if y is None:
+        y = torch.empty((B, m), dtype=torch.float32, device=x.device)
+    st = _lib.call("dbf_apply", _ptr(a), _ptr(B1), _ptr(mid), _ptr(B2), _ptr(b), m, r, n, _ptr(x), B,
+                   _ptr(y), _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
+    _lib.check(st, "dbf_apply")
+    return y

@@ -57,3 +57,17 @@ def test_host_side_argument_errors(lib):
     assert lib.w1_gemv(good, good, 16, 128, odd, 1, good, None) == _lib.W1_ERR_ALIGN
     assert lib.w1_gemm(good, good, 16, 128, good, 0, good, None) == _lib.W1_ERR_SHAPE
     assert lib.w1_gemm(good, good, 16, 128, good, 4, None, None) == _lib.W1_ERR_NULL
+
+
+def test_dbf_host_side_argument_errors(lib):
+    good = ctypes.c_void_p(1 << 20)
+    odd = ctypes.c_void_p((1 << 20) + 8)
+    args = [good] * 5
+    assert lib.dbf_apply(None, *args[1:], 64, 128, 128, good, 1, good, good, 1 << 20, None) == _lib.W1_ERR_NULL
+    assert lib.dbf_apply(*args, 64, 100, 128, good, 1, good, good, 1 << 20, None) == _lib.W1_ERR_SHAPE
+    assert lib.dbf_apply(*args, 64, 128, 128, good, 0, good, good, 1 << 20, None) == _lib.W1_ERR_SHAPE
+    assert lib.dbf_apply(*args, 64, 128, 128, good, 1, good, None, 1 << 20, None) == _lib.W1_ERR_WORKSPACE
+    assert lib.dbf_apply(*args, 64, 128, 128, good, 1, good, good, 16, None) == _lib.W1_ERR_WORKSPACE
+    assert lib.dbf_apply(*args, 64, 128, 128, odd, 1, good, good, 1 << 20, None) == _lib.W1_ERR_ALIGN
+    assert lib.dbf_workspace_size(64, 128, 128, 1) >= 256 + 4 * 128
+    assert lib.dbf_workspace_size(0, 128, 128, 1) == 0

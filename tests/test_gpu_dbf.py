@@ -1,0 +1,99 @@
+"""dbf_apply (fused small-batch kernel) on the GPU vs the fp64 oracle chain."""
+import functools
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import w1_oracle as O
+from pack_sign_g128_b200 import ops, synth, _lib
+from gpu_helpers import assert_within, bf16_dev, fp16_dev, words_dev
+
+pytestmark = pytest.mark.gpu
+
+
+def run_dbf(case, ws=None):
+    a, B1, mid, B2, b, x = case
+    dv = [fp16_dev(a), words_dev(B1), fp16_dev(mid), words_dev(B2), fp16_dev(b), bf16_dev(x)]
+    m, r, n, B = a.shape[0], mid.shape[0], b.shape[0], x.shape[0]
+    if ws is None:
+        ws = ops.dbf_workspace(m, r, n, B)
+    y = ops.dbf_apply(*dv, workspace=ws)
+    st = ops.sync_status()
+    return y.cpu().numpy().astype(np.float64), ws, st
+
+
+def check(case, what, stage1=True):
+    a, B1, mid, B2, b, x = case
+    m, r, n, B = a.shape[0], mid.shape[0], b.shape[0], x.shape[0]
+    y, ws, st = run_dbf(case)
+    assert st == _lib.W1_OK
+    ref = O.dbf_ref(a, B1, mid, B2, b, O.bf16_bits_to_f64(x), m, r, n)
+    assert_within(y, ref["y"], ref["bound"], what=what)
+    if stage1:
+        # workspace holds mid * h of the last group of <= 8 batch rows
+        b0 = ((B - 1) // 8) * 8
+        nb = B - b0
+        hw = ws[256:256 + 4 * nb * r].view(torch.float32).cpu().numpy().reshape(nb, r).astype(np.float64)
+        midv = O.fp16_bits_to_f64(mid)
+        assert_within(hw, ref["h_scaled"][b0:], np.abs(midv)[None, :] * ref["h_bound"][b0:], what=what + " stage 1")
+    return y
+
+
+@pytest.mark.parametrize("B", [1, 8])
+def test_dbf_config(B):
+    check(synth.dbf_case(B=B), f"4096^3 B={B}")
+
+
+def test_dbf_config_batch512():
+    check(synth.dbf_case(B=512), "4096^3 B=512")
+
+
+@pytest.mark.parametrize("m,r,n,B", [(200, 384, 256, 3), (1, 128, 128, 1), (1000, 640, 1152, 5),
+                                     (4096, 1024, 2048, 2), (33, 256, 128, 7)])
+def test_dbf_ragged(m, r, n, B):
+    check(synth.dbf_case(m=m, r=r, n=n, B=B, seed=m + r + n + B), f"{m}x{r}x{n} B={B}")
+
+
+def _sylvester_words(n):
+    H = np.array([[1.0]])
+    while H.shape[0] < n:
+        H = np.block([[H, H], [H, -H]])
+    return O.pack_bits_lsb_first((H < 0).astype(np.uint8))
+
+
+def test_dbf_hadamard_closed_form():
+    n = 1024
+    Hw = _sylvester_words(n)
+    ones = np.full(n, 0x3C00, np.uint16)
+    x = synth.activations_bf16(synth.rng(5), 4, n)
+    y, _, st = run_dbf((ones, Hw, ones, Hw, ones, x))
+    assert st == _lib.W1_OK
+    exact = n * O.bf16_bits_to_f64(x)
+    assert np.max(np.abs(y - exact)) <= 1e-5 * np.max(np.abs(exact))
+
+
+def test_dbf_workspace_reuse_and_determinism():
+    case = synth.dbf_case(m=512, r=1024, n=768, B=4, seed=9)
+    y1, ws, st = run_dbf(case)
+    assert st == _lib.W1_OK
+    assert int(ws[:4].view(torch.int32).item()) == 0        # barrier count back at zero
+    y2, _, st = run_dbf(case, ws)
+    assert st == _lib.W1_OK
+    assert np.array_equal(y1, y2)
+
+
+def test_dbf_barrier_timeout_reports_status():
+    """A barrier count that no arrival can complete: every CTA's bounded wait
+    runs out, the call reports W1_ERR_TIMEOUT and the context stays usable."""
+    case = synth.dbf_case(m=256, r=256, n=256, B=1, seed=10)
+    a, B1, mid, B2, b, x = case
+    ws = ops.dbf_workspace(256, 256, 256, 1)
+    ws[:4].view(torch.int32).fill_(-(2 ** 31))
+    _, _, st = run_dbf(case, ws)
+    assert st == _lib.W1_ERR_TIMEOUT
+    ws.zero_()
+    y, _, st = run_dbf(case, ws)
+    assert st == _lib.W1_OK
+    ref = O.dbf_ref(a, B1, mid, B2, b, O.bf16_bits_to_f64(x), 256, 256, 256)
+    assert_within(y, ref["y"], ref["bound"], what="after timeout")
