@@ -108,6 +108,40 @@ int w1_gemm(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t K,
             const uint16_t* x, int64_t M, float* y, w1_stream_t stream);
 
 /*
+ * w1_moe_grouped -- routed SwiGLU expert layer with 1-bit group-128 experts
+ * ("LLM binarization episode 01: DBF", section 4: every (token, slot) route
+ * carries an expert id and a route weight; gate/up consume the token's shared
+ * hidden state, down consumes the route's own intermediate).
+ *   p[t] = softmax(router_logits[t]) over the E experts (fp32); the top_k
+ *   experts by probability (ties to the lower index) are the routes, each with
+ *   weight p (no renormalisation).  For route (t, e):
+ *     g = G_e x_t, u = U_e x_t, h = bf16( silu(g) * u ), out[t] += p * D_e h,
+ *   the slot terms summed in slot order.  silu(z) = z / (1 + exp(-z)).
+ *   x              bf16 [T][H]
+ *   router_logits  fp32 [T][E]
+ *   gate_*, up_*   experts stacked: signs uint32 [E][I][H/32], scales fp16 [E][I][H/128]
+ *   down_*         signs uint32 [E][H][I/32], scales fp16 [E][H][I/128]
+ *   out            fp32 [T][H]
+ *   H, I multiples of 128; 1 <= top_k <= min(E, 32); E <= 256.
+ * workspace: >= w1_moe_workspace_size(...) bytes, 1024-byte aligned; holds the
+ *   routing (expert ids, weights, the expert-sorted route order), the tile
+ *   lists, h (bf16, expert-sorted) and the weighted route outputs.  No state is
+ *   carried between calls.  Calls sharing a workspace must not overlap.
+ * Five kernels on `stream`: router, counting sort, grouped gate/up GEMM (tokens
+ * gathered from x by TMA, fused SwiGLU), grouped down GEMM (route weight
+ * applied), slot-ordered combine.  Deterministic.  Accuracy per stage as
+ * w1_gemm: 1e-3 * sum|s x| for g, u and D_e h.
+ */
+int w1_moe_grouped(const uint16_t* x, const float* router_logits, int64_t T, int64_t H, int64_t I, int64_t E,
+                   int64_t top_k, const uint32_t* gate_signs, const uint16_t* gate_scales,
+                   const uint32_t* up_signs, const uint16_t* up_scales, const uint32_t* down_signs,
+                   const uint16_t* down_scales, float* out, void* workspace, size_t ws_bytes,
+                   w1_stream_t stream);
+
+/* Bytes of workspace w1_moe_grouped needs (0 for invalid sizes). */
+size_t w1_moe_workspace_size(int64_t T, int64_t H, int64_t I, int64_t E, int64_t top_k);
+
+/*
  * dbf_apply -- Double Binary Factorization chain ("LLM binarization episode 01:
  * DBF", section 1 "The representation": W ~ D_out U D_mid V D_in; section 4:
  * evaluated as x_scaled = D_in x, h = V x_scaled, h_scaled = D_mid h,

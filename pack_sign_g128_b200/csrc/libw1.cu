@@ -5,3 +5,4 @@
 #include "gemv.cu"
 #include "gemm.cu"
 #include "dbf.cu"
+#include "moe.cu"

@@ -79,6 +79,54 @@ def w1_gemm(signs: torch.Tensor, scales: torch.Tensor, x: torch.Tensor, y: torch
     return y
 
 
+def moe_workspace(T: int, H: int, I: int, E: int, top_k: int, device=None) -> torch.Tensor:
+    nbytes = _lib.call("w1_moe_workspace_size", T, H, I, E, top_k)
+    if nbytes == 0:
+        raise ValueError("invalid MoE sizes")
+    return torch.empty(nbytes, dtype=torch.uint8, device=device or "cuda")
+
+
+def w1_moe_grouped(x: torch.Tensor, logits: torch.Tensor, gate, up, down, top_k: int,
+                   out: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+                   stream=None) -> torch.Tensor:
+    """Routed SwiGLU layer.  gate/up/down = (signs int32 [E, rows, K/32], scales fp16 [E, rows, K/128])."""
+    T, H = x.shape
+    E = logits.shape[1]
+    I = gate[0].shape[1]
+    if x.dtype != torch.bfloat16 or logits.dtype != torch.float32:
+        raise TypeError("x must be bfloat16 and logits float32")
+    if workspace is None:
+        workspace = moe_workspace(T, H, I, E, top_k, x.device)
+    if out is None:
+        out = torch.empty((T, H), dtype=torch.float32, device=x.device)
+    st = _lib.call("w1_moe_grouped", _ptr(x), _ptr(logits), T, H, I, E, top_k, _ptr(gate[0]), _ptr(gate[1]),
+                   _ptr(up[0]), _ptr(up[1]), _ptr(down[0]), _ptr(down[1]), _ptr(out), _ptr(workspace),
+                   workspace.numel() * workspace.element_size(), _stream(stream))
+    _lib.check(st, "w1_moe_grouped")
+    return out
+
+
+def moe_workspace_views(workspace: torch.Tensor, T: int, H: int, I: int, E: int, top_k: int) -> dict:
+    """Typed views of the MoE workspace (routing, sorted order, h) for inspection."""
+    R = T * top_k
+
+    def up(v, a):
+        return (v + a - 1) // a * a
+    off = 256
+    views = {}
+    for name in ("ids", "wts", "pos", "sroute", "stok"):
+        views[name] = workspace[off:off + 4 * R].view(torch.float32 if name == "wts" else torch.int32)
+        off = up(off + 4 * R, 256)
+    views["offsets"] = workspace[off:off + 4 * (E + 1)].view(torch.int32)
+    off = up(off + 4 * (E + 1), 256)
+    mtg = ((R + 63) // 64 + E) * (I // 128)
+    mtd = ((R + 127) // 128 + E) * (H // 128)
+    off = up(off + 16 * mtg, 256)
+    off = up(off + 16 * mtd, 256)
+    views["h"] = workspace[off:off + 2 * R * I].view(torch.bfloat16).view(R, I)
+    return views
+
+
 def dbf_workspace(m: int, r: int, n: int, B: int, device=None) -> torch.Tensor:
     """A zeroed workspace for dbf_apply (the grid-barrier words start at zero)."""
     nbytes = _lib.call("dbf_workspace_size", m, r, n, B)
@@ -105,3 +153,4 @@ def dbf_apply(a: torch.Tensor, B1: torch.Tensor, mid: torch.Tensor, B2: torch.Te
                    _ptr(y), _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
     _lib.check(st, "dbf_apply")
     return y
+

@@ -71,3 +71,21 @@ def test_dbf_host_side_argument_errors(lib):
     assert lib.dbf_apply(*args, 64, 128, 128, odd, 1, good, good, 1 << 20, None) == _lib.W1_ERR_ALIGN
     assert lib.dbf_workspace_size(64, 128, 128, 1) >= 256 + 4 * 128
     assert lib.dbf_workspace_size(0, 128, 128, 1) == 0
+
+
+def test_moe_host_side_argument_errors(lib):
+    good = ctypes.c_void_p(1 << 20)
+    ws = ctypes.c_void_p(1 << 30)
+    base = [good, good, 16, 256, 128, 8, 2] + [good] * 7
+    n = lib.w1_moe_workspace_size(16, 256, 128, 8, 2)
+    assert n > 0
+    assert lib.w1_moe_workspace_size(16, 256, 128, 8, 9) == 0          # top_k > E
+    assert lib.w1_moe_workspace_size(16, 256, 128, 300, 2) == 0        # E > 256
+    assert lib.w1_moe_grouped(*base, ws, n - 1, None) == _lib.W1_ERR_WORKSPACE
+    bad = list(base)
+    bad[3] = 200                                                       # H not a multiple of 128
+    assert lib.w1_moe_grouped(*bad, ws, n, None) == _lib.W1_ERR_SHAPE
+    bad = list(base)
+    bad[0] = None
+    assert lib.w1_moe_grouped(*bad, ws, n, None) == _lib.W1_ERR_NULL
+    assert lib.w1_moe_grouped(*base, ctypes.c_void_p((1 << 30) + 256), n, None) == _lib.W1_ERR_ALIGN
