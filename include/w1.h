@@ -58,7 +58,8 @@ typedef enum {
   W1_ERR_CUDA = 6,        /* CUDA launch / runtime error                         */
   W1_ERR_TIMEOUT = 7,     /* device: a bounded wait gave up                      */
   W1_ERR_WORKSPACE = 8,   /* workspace missing or too small                      */
-  W1_ERR_UNSUPPORTED = 9  /* current device is not sm_100 (B200 class)           */
+  W1_ERR_UNSUPPORTED = 9, /* current device is not sm_100 (B200 class)           */
+  W1_ERR_TOO_LARGE = 10   /* sizes exceed dbf_apply_noalloc's static scratch     */
 } w1_status;
 
 /* Static, human-readable name of a status code. */
@@ -169,6 +170,27 @@ int dbf_apply(const uint16_t* a, const uint32_t* B1, const uint16_t* mid, const 
 
 /* Bytes of workspace dbf_apply needs for these sizes (0 for invalid sizes). */
 size_t dbf_workspace_size(int64_t m, int64_t r, int64_t n, int64_t B);
+
+/*
+ * dbf_apply_noalloc -- dbf_apply for callers that cannot allocate device memory
+ * (the pages have no counterpart: this is a deployment variant).  Some callers
+ * cannot call cudaMalloc or take memory from an allocator: code embedded in a
+ * host framework whose device memory is owned by that framework's pool, or a
+ * latency-critical decode loop where an allocation would synchronise the
+ * device or fail.  This entry point takes the same inputs and output as
+ * dbf_apply but no workspace: its scratch is a fixed array inside the library
+ * (256 bytes + 4*8*16384 bytes, held on every GPU that loads the library until
+ * the process exits).  It allocates nothing and calls no allocating routine.
+ *   Limit: r <= 16384, else W1_ERR_TOO_LARGE (other limits as dbf_apply).
+ *   The first call on a device looks up the array's device address (with that
+ *   device current); make that first call before any stream capture.
+ *   Every call shares the one array and clears its barrier count first; calls
+ *   that overlap on the GPU (for instance on two streams) race on it.  After a
+ *   call the array still holds that call's fp32 intermediate.
+ */
+int dbf_apply_noalloc(const uint16_t* a, const uint32_t* B1, const uint16_t* mid, const uint32_t* B2,
+                      const uint16_t* bdiag, int64_t m, int64_t r, int64_t n, const uint16_t* x, int64_t B,
+                      float* y, w1_stream_t stream);
 
 #ifdef __cplusplus
 }

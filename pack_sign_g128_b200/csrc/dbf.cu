@@ -362,4 +362,68 @@ cudaError_t launch_dbf(const uint16_t* a, const uint32_t* B1, const uint16_t* mi
   return cudaSuccess;
 }
 
+// ------------------------------------------------------------------ static scratch
+// Scratch for callers that cannot allocate device memory: a fixed array in the
+// library's own device image (every GPU that loads the library holds it until
+// the process exits).  Holds the barrier count (first 256 bytes) and the fp32
+// intermediate for up to 8 batch rows of r <= kDbfStaticMaxR.
+constexpr int64_t kDbfStaticMaxR = 16384;
+constexpr size_t kDbfStaticScratchBytes = 256 + 4 * 8 * kDbfStaticMaxR;
+static __device__ __align__(256) unsigned char g_dbf_static_scratch[kDbfStaticScratchBytes];
+
+// Device address of the scratch array for the current device.  In host code
+// the symbol is only a stand-in, so the address is looked up once per device
+// (with that device current) and cached.
+static void* dbf_static_scratch_ptr(int* status) {
+  static void* ptrs[64] = {};
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    *status = W1_ERR_CUDA;
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  if (!ptrs[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_dbf_static_scratch) != cudaSuccess || p == nullptr) {
+      cudaGetLastError();
+      *status = W1_ERR_CUDA;
+      return nullptr;
+    }
+    ptrs[dev] = p;
+  }
+  *status = W1_OK;
+  return ptrs[dev];
+}
+
 }  // namespace w1
+
+// ------------------------------------------------------------------ C entry point
+using w1::aligned16;
+extern "C" {
+
+// dbf_apply without a workspace argument (see include/w1.h): same kernel, the
+// scratch being the static array above.  Allocates nothing.
+int dbf_apply_noalloc(const uint16_t* a, const uint32_t* B1, const uint16_t* mid, const uint32_t* B2,
+                      const uint16_t* b, int64_t m, int64_t r, int64_t n, const uint16_t* x, int64_t B, float* y,
+                      w1_stream_t stream) {
+  if (!a || !B1 || !mid || !B2 || !b || !x || !y) return W1_ERR_NULL;
+  if (m <= 0 || r <= 0 || n <= 0 || B <= 0 || (r % 128) != 0 || (n % 128) != 0) return W1_ERR_SHAPE;
+  if (m > (int64_t)1 << 30 || n > (int64_t)1 << 30) return W1_ERR_SHAPE;
+  if (r > w1::kDbfStaticMaxR) return W1_ERR_TOO_LARGE;
+  if (!aligned16(a) || !aligned16(B1) || !aligned16(mid) || !aligned16(B2) || !aligned16(b) || !aligned16(x) ||
+      !aligned16(y))
+    return W1_ERR_ALIGN;
+  w1::DeviceInfo d;
+  int st = w1::device_info(&d);
+  if (st != W1_OK) return st;
+  void* scratch = w1::dbf_static_scratch_ptr(&st);
+  if (st != W1_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // the barrier count must start at zero (a previous call may have timed out)
+  if (cudaMemsetAsync(scratch, 0, 8, s) != cudaSuccess) return W1_ERR_CUDA;
+  const int cap = d.smem_optin < 200 * 1024 ? d.smem_optin : 200 * 1024;
+  return w1::launch_result(w1::launch_dbf(a, B1, mid, B2, b, m, r, n, x, B, y, scratch, s, d.sms, cap));
+}
+
+}  // extern "C"

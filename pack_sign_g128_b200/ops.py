@@ -154,3 +154,12 @@ def dbf_apply(a: torch.Tensor, B1: torch.Tensor, mid: torch.Tensor, B2: torch.Te
     _lib.check(st, "dbf_apply")
     return y
 
+
+def dbf_apply_noalloc(a: torch.Tensor, B1: torch.Tensor, mid: torch.Tensor, B2: torch.Tensor, b: torch.Tensor,
+                      x: torch.Tensor, y: torch.Tensor, stream=None) -> torch.Tensor:
+    """dbf_apply without a workspace (the library's static scratch); y must be given."""
+    m, r, n, B = a.shape[0], mid.shape[0], b.shape[0], x.shape[0]
+    st = _lib.call("dbf_apply_noalloc", _ptr(a), _ptr(B1), _ptr(mid), _ptr(B2), _ptr(b), m, r, n, _ptr(x), B,
+                   _ptr(y), _stream(stream))
+    _lib.check(st, "dbf_apply_noalloc")
+    return y
