@@ -286,6 +286,116 @@ def gemm_rows(torch, ops, synth, peaks, iters: int = 8):
     return rows
 
 
+MOE = dict(T=512, H=2048, I=1024, E=64, top_k=8)
+DBF_BATCHES = [1, 8, 512]
+
+
+def moe_rows(torch, ops, synth, peaks, iters: int = 8):
+    """Routed MoE layer (OLMoE-like): tokens/s and TFLOP/s, L2 flushed per call."""
+    dev = torch.device("cuda")
+    T, H, I, E, K = MOE["T"], MOE["H"], MOE["I"], MOE["E"], MOE["top_k"]
+    x, logits, gate, up, down = synth.moe_case(T=T, H=H, I=I, E=E)
+
+    def pack(Wt):
+        s, c = ops.w1_pack(torch.from_numpy(Wt.reshape(-1, Wt.shape[-1])).to(dev))
+        return s.view(E, Wt.shape[1], -1), c.view(E, Wt.shape[1], -1)
+    G, U, D = pack(gate), pack(up), pack(down)
+    del gate, up, down
+    xd = torch.from_numpy(x.view(np.int16)).to(dev).view(torch.bfloat16)
+    ld = torch.from_numpy(logits).to(dev)
+    ws = ops.moe_workspace(T, H, I, E, K)
+    out = torch.empty((T, H), dtype=torch.float32, device=dev)
+    flush = torch.empty(int(512 * 2 ** 20), dtype=torch.uint8, device=dev)
+    for _ in range(3):
+        ops.w1_moe_grouped(xd, ld, G, U, D, K, out=out, workspace=ws)
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(iters):
+        flush.zero_()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        ops.w1_moe_grouped(xd, ld, G, U, D, K, out=out, workspace=ws)
+        b.record()
+        torch.cuda.synchronize()
+        times.append(a.elapsed_time(b))
+    ms = statistics.median(times)
+    flops = 2.0 * T * K * 3 * H * I
+    tf = flops / (ms * 1e-3) / 1e12
+    return {"T": T, "H": H, "I": I, "E": E, "top_k": K, "ms": ms, "tokens/s": T / (ms * 1e-3),
+            "TFLOP/s": tf, "frac_bf16_burst": tf / peaks["bf16_tflops"], "launches_per_call": 5}
+
+
+def dbf_rows(torch, ops, synth, peaks, l2_bytes: int, iters: int = 5):
+    """DBF chain 4096^3: B = 1, 8 as GB/s of sign bytes (rotating copies > 4x L2,
+    CUDA graph of back-to-back calls); B = 512 as TFLOP/s (L2 flushed)."""
+    dev = torch.device("cuda")
+    m = r = n = 4096
+    rows = []
+    for B in DBF_BATCHES:
+        a, B1, mid, B2, b, x = synth.dbf_case(m=m, r=r, n=n, B=B)
+        to16 = lambda v: torch.from_numpy(v.view(np.int16)).to(dev).view(torch.float16)
+        tow = lambda v: torch.from_numpy(v.view(np.int32)).to(dev)
+        ad, md, bd = to16(a), to16(mid), to16(b)
+        xd = torch.from_numpy(x.view(np.int16)).to(dev).view(torch.bfloat16)
+        y = torch.empty((B, m), dtype=torch.float32, device=dev)
+        ws = ops.dbf_workspace(m, r, n, B)
+        sign_bytes = (m * r + r * n) // 8
+        alg_bytes = sign_bytes + 2 * (m + r + n)
+        flops = 2.0 * B * (r * n + m * r)
+        if B <= 8:
+            R = max(16, int(math.ceil(4 * l2_bytes / sign_bytes)))
+            B1s = [tow(B1)] + [None] * (R - 1)
+            B2s = [tow(B2)] + [None] * (R - 1)
+            for i in range(1, R):
+                B1s[i] = B1s[0].clone()
+                B2s[i] = B2s[0].clone()
+            st = torch.cuda.Stream()
+            with torch.cuda.stream(st):
+                for i in range(3):
+                    ops.dbf_apply(ad, B1s[i], md, B2s[i], bd, xd, y=y, workspace=ws)
+            st.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=st):
+                for i in range(R):
+                    ops.dbf_apply(ad, B1s[i], md, B2s[i], bd, xd, y=y, workspace=ws)
+            g.replay()
+            torch.cuda.synchronize()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(iters):
+                g.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            us = e0.elapsed_time(e1) * 1e3 / (iters * R)
+            gbs = alg_bytes / (us * 1e-6) / 1e9
+            rows.append({"B": B, "us_per_call": round(us, 3), "GB/s": round(gbs, 1),
+                         "frac_hbm": round(gbs / peaks["hbm_gbs"], 4), "calls": R})
+            del B1s, B2s, g
+        else:
+            B1d, B2d = tow(B1), tow(B2)
+            flush = torch.empty(int(512 * 2 ** 20), dtype=torch.uint8, device=dev)
+            for _ in range(2):
+                ops.dbf_apply(ad, B1d, md, B2d, bd, xd, y=y, workspace=ws)
+            torch.cuda.synchronize()
+            times = []
+            for _ in range(iters):
+                flush.zero_()
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record()
+                ops.dbf_apply(ad, B1d, md, B2d, bd, xd, y=y, workspace=ws)
+                e1.record()
+                torch.cuda.synchronize()
+                times.append(e0.elapsed_time(e1))
+            ms = statistics.median(times)
+            tf = flops / (ms * 1e-3) / 1e12
+            rows.append({"B": B, "ms": ms, "TFLOP/s": tf, "frac_bf16_burst": tf / peaks["bf16_tflops"]})
+    torch.cuda.synchronize()
+    return rows
+
+
 def cpu_oracle_gemv_sample(combos_spec, packed_host, max_seconds: float = 20.0):
     """Time the fp64 oracle on the sweep (one launch per pair) on the host."""
     from oracle import w1_oracle as O
@@ -337,6 +447,17 @@ def run_gpu(args):
     props = torch.cuda.get_device_properties(local)
     l2 = int(getattr(props, "L2_cache_size", 126 * 2 ** 20) or 126 * 2 ** 20)
 
+    if args.section != "all":
+        rows = {}
+        if args.section == "gemm":
+            rows["gemm"] = gemm_rows(torch, ops, synth, peaks)
+        elif args.section == "moe":
+            rows["moe"] = moe_rows(torch, ops, synth, peaks)
+        elif args.section == "dbf":
+            rows["dbf"] = dbf_rows(torch, ops, synth, peaks, l2)
+        if rank == 0:
+            print(json.dumps({"section": args.section, "rows": rows}), flush=True)
+        return
     combos, stream = build_gemv_sweep(torch, ops, synth, l2)
     launches_per_step = sum(cb["R"] for cb in combos)
     bytes_per_step = sum(cb["bytes"] * cb["R"] for cb in combos)
@@ -361,6 +482,8 @@ def run_gpu(args):
     rows = {"gemv": gemv_rows}
     if not args.skip_extra:
         rows["gemm"] = gemm_rows(torch, ops, synth, peaks)
+        rows["moe"] = moe_rows(torch, ops, synth, peaks)
+        rows["dbf"] = dbf_rows(torch, ops, synth, peaks, l2)
     cpu = None
     if rank == 0 and world == 1 and not args.skip_cpu:
         packed_host = {}
@@ -476,6 +599,8 @@ def main():
     ap.add_argument("--impl", default="w1", choices=["w1", "reference"])
     ap.add_argument("--skip-extra", action="store_true", help="only the headline sweep")
     ap.add_argument("--skip-cpu", action="store_true", help="skip the CPU-oracle baseline")
+    ap.add_argument("--section", default="all", choices=["all", "gemm", "moe", "dbf"],
+                    help="run one row only (for profiling); prints a rows-only JSON line")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

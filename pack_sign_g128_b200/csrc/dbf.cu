@@ -21,6 +21,8 @@
 // quantisation is the 23-bit fixed point of each product's input.
 #include <cstdint>
 #include <cuda_fp16.h>
+#include <cstdio>
+#include <cstdlib>
 #include <mutex>
 
 #include "gemv_core.cuh"
@@ -29,51 +31,55 @@ namespace w1 {
 
 struct DbfParams {
   const uint16_t* a;    // [m] fp16
-  const uint32_t* B1;   // [m][r/32]
   const uint16_t* mid;  // [r] fp16
-  const uint32_t* B2;   // [r][n/32]
   const uint16_t* b;    // [n] fp16
   const uint16_t* x;    // [B][n] bf16
   float* y;             // [B][m]
   float* h;             // [B][r] workspace: mid (.) (B2 . (b (.) x))
   unsigned int* bar;    // workspace: grid barrier {count, generation}
   int m, r, n;
-  int S;
+  int S, bw1, bw2;
   int ns1, ns2;
   int max_tiles1, max_tiles2, max_ng1, max_ng2;
 };
 
 struct DbfSmem {
-  int st1, st2, xq, xsum, xf, part, bars, total;
+  int st1, sb1, st2, sb2, xq, zero, xsum, xf, part, bars, total;
 };
 
 template <int NB>
 __host__ __device__ inline DbfSmem dbf_smem_layout(const DbfParams& p) {
-  constexpr int NT = GemvLayout<NB>::NT;
+  using L = GemvLayout<NB>;
   const int mng = p.max_ng1 > p.max_ng2 ? p.max_ng1 : p.max_ng2;
   const int mt = p.max_tiles1 > p.max_tiles2 ? p.max_tiles1 : p.max_tiles2;
-  DbfSmem L;
+  const int wp = gemv_wpt(p.max_tiles1) > gemv_wpt(p.max_tiles2) ? gemv_wpt(p.max_tiles1) : gemv_wpt(p.max_tiles2);
+  DbfSmem M;
   int off = 0;
-  L.st1 = off;
-  off += p.ns1 * 16 * gemv_rowstride(p.max_ng1);
+  M.st1 = off;
+  M.sb1 = ((p.max_ng1 + p.bw1 - 1) / p.bw1) * 16 * 16 * p.bw1;
+  off += p.ns1 * M.sb1;
+  off = round_up(off, 1024);
+  M.st2 = off;
+  M.sb2 = ((p.max_ng2 + p.bw2 - 1) / p.bw2) * 16 * 16 * p.bw2;
+  off += p.ns2 * M.sb2;
   off = round_up(off, 128);
-  L.st2 = off;
-  off += p.ns2 * 16 * gemv_rowstride(p.max_ng2);
-  off = round_up(off, 128);
-  L.xq = off;
-  off += mng * 4 * NT * 256;
-  L.xsum = off;
+  M.xq = off;
+  off += mng * 4 * L::BLOCK;
+  off = round_up(off, 16);
+  M.zero = off;
+  off += 16;
+  M.xsum = off;
   off += mng * NB * 4;
-  L.xf = off;
+  M.xf = off;
   off += mng * NB * 4;
   off = round_up(off, 16);
-  L.part = off;
-  off += NB * mt * 16 * 4;
+  M.part = off;
+  off += wp * NB * mt * 16 * 4;
   off = round_up(off, 8);
-  L.bars = off;
+  M.bars = off;
   off += 2 * (p.ns1 + p.ns2) * 8;
-  L.total = round_up(off, 128);
-  return L;
+  M.total = round_up(off, 128) + 1024;
+  return M;
 }
 
 // Grid-wide barrier over all CTAs of the launch (all co-resident by
@@ -112,44 +118,56 @@ __device__ inline bool grid_barrier(unsigned int* bar, unsigned int nblocks) {
 }
 
 template <int NB>
-__global__ void __launch_bounds__(kGemvThreads, 1) dbf_small_kernel(const DbfParams p) {
-  extern __shared__ __align__(128) unsigned char smem[];
-  const DbfSmem L = dbf_smem_layout<NB>(p);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
-  GemvSmemView v1{smem + L.st1, p.ns1, bars, bars + p.ns1};
-  GemvSmemView v2{smem + L.st2, p.ns2, bars + 2 * p.ns1, bars + 2 * p.ns1 + p.ns2};
+__global__ void __launch_bounds__(kGemvThreads, 1)
+    dbf_small_kernel(const __grid_constant__ CUtensorMap tm2, const __grid_constant__ CUtensorMap tm1,
+                     const DbfParams p) {
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem =
+      reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const DbfSmem M = dbf_smem_layout<NB>(p);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + M.bars);
+  GemvSmemView v1{smem + M.st1, p.ns1, M.sb1, bars, bars + p.ns1};
+  GemvSmemView v2{smem + M.st2, p.ns2, M.sb2, bars + 2 * p.ns1, bars + 2 * p.ns1 + p.ns2};
   GemvXView xv;
-  xv.xq = smem + L.xq;
-  xv.xsum = reinterpret_cast<int*>(smem + L.xsum);
-  xv.xf = reinterpret_cast<float*>(smem + L.xf);
+  xv.xq = smem + M.xq;
+  xv.xsum = reinterpret_cast<int*>(smem + M.xsum);
+  xv.xf = reinterpret_cast<float*>(smem + M.xf);
   xv.sc = nullptr;
-  xv.part = reinterpret_cast<float*>(smem + L.part);
+  xv.part = reinterpret_cast<float*>(smem + M.part);
   xv.part_stride = (p.max_tiles1 > p.max_tiles2 ? p.max_tiles1 : p.max_tiles2) * 16;
+  unsigned char* zero16 = smem + M.zero;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int crank = static_cast<int>(cluster_ctarank());
   const int q = static_cast<int>(cluster_id_x()), Q = static_cast<int>(nclusters_x());
-  const Split sp1 = make_split(p.r, 0, p.n >> 7, p.S, crank, q, Q);  // rows of V, K = n
-  const Split sp2 = make_split(p.m, 0, p.r >> 7, p.S, crank, q, Q);  // rows of U, K = r
-  const int64_t wrow1 = p.n >> 5, wrow2 = p.r >> 5;
+  // rows of V with K = n, then rows of U with K = r
+  const Split sp1 = make_split(p.r, 0, p.n >> 7, p.S, crank, q, Q, p.bw1, p.bw1, p.max_tiles1);
+  const Split sp2 = make_split(p.m, 0, p.r >> 7, p.S, crank, q, Q, p.bw2, p.bw2, p.max_tiles2);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < 2 * (p.ns1 + p.ns2); ++s) mbar_init(&bars[s], 1);
+    for (int s = 0; s < p.ns1; ++s) {
+      mbar_init(&v1.full[s], 1);
+      mbar_init(&v1.empty[s], static_cast<uint32_t>(sp1.wpt));
+    }
+    for (int s = 0; s < p.ns2; ++s) {
+      mbar_init(&v2.full[s], 1);
+      mbar_init(&v2.empty[s], static_cast<uint32_t>(sp2.wpt));
+    }
     fence_mbarrier_init();
+    asm volatile("prefetch.tensormap [%0];" ::"l"(&tm2) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(&tm1) : "memory");
   }
-  if (warp == kProducerWarp) {
-    prefetch_weights(sp1, p.B2, wrow1, nullptr, 0, lane);
-    prefetch_weights(sp2, p.B1, wrow2, nullptr, 0, lane);
-  }
+  if (threadIdx.x < 4) reinterpret_cast<uint32_t*>(zero16)[threadIdx.x] = 0u;
   __syncthreads();
   pdl_wait();
   pdl_launch_dependents();
 
   int first1 = 0, first2 = 0;
-  if (warp == kProducerWarp) {
-    first1 = issue_first_tiles(v1, sp1, p.B2, wrow1, lane);
-    first2 = issue_first_tiles(v2, sp2, p.B1, wrow2, lane);
+  if (warp == kProducerWarp && lane == 0) {
+    first1 = issue_first_tiles(v1, sp1, &tm2, p.bw1);
+    first2 = issue_first_tiles(v2, sp2, &tm1, p.bw2);
   }
+  __syncwarp();
 
   // ---- phase 1: h_scaled = mid (.) (V . (b (.) x))
   {
@@ -171,11 +189,13 @@ __global__ void __launch_bounds__(kGemvThreads, 1) dbf_small_kernel(const DbfPar
                        },
                        kGemvThreads);
     __syncthreads();
-    if (warp == kProducerWarp)
-      produce_rest(v1, sp1, p.B2, wrow1, first1, lane);
-    else
-      consume_tiles<NB, false>(v1, xv, sp1, warp, lane);
-    cluster_sync();
+    if (warp == kProducerWarp) {
+      if (lane == 0) produce_rest(v1, sp1, &tm2, p.bw1, first1);
+      __syncwarp();  // converge before the (cluster) barrier, which is .aligned
+    } else {
+      consume_tiles<NB, false>(v1, xv, sp1, p.bw1, zero16, warp, lane);
+    }
+    if (p.S > 1) cluster_sync(); else __syncthreads();
     float* h = p.h;
     const uint16_t* mid = p.mid;
     const int r = p.r;
@@ -185,9 +205,9 @@ __global__ void __launch_bounds__(kGemvThreads, 1) dbf_small_kernel(const DbfPar
                        },
                        kGemvThreads);
   }
-  // ---- every CTA's h_scaled is in memory
+  // ---- every CTA's h_scaled is in memory (and every peer is done with part)
   if (!grid_barrier(p.bar, gridDim.x)) {
-    cluster_sync();
+    if (p.S > 1) cluster_sync();
     return;
   }
   // ---- phase 2: y = a (.) (U . h_scaled)
@@ -208,11 +228,13 @@ __global__ void __launch_bounds__(kGemvThreads, 1) dbf_small_kernel(const DbfPar
                        },
                        kGemvThreads);
     __syncthreads();
-    if (warp == kProducerWarp)
-      produce_rest(v2, sp2, p.B1, wrow2, first2, lane);
-    else
-      consume_tiles<NB, false>(v2, xv, sp2, warp, lane);
-    cluster_sync();
+    if (warp == kProducerWarp) {
+      if (lane == 0) produce_rest(v2, sp2, &tm1, p.bw2, first2);
+      __syncwarp();
+    } else {
+      consume_tiles<NB, false>(v2, xv, sp2, p.bw2, zero16, warp, lane);
+    }
+    if (p.S > 1) cluster_sync(); else __syncthreads();
     float* y = p.y;
     const uint16_t* a = p.a;
     const int m = p.m;
@@ -221,7 +243,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) dbf_small_kernel(const DbfPar
                          y[static_cast<int64_t>(bb) * m + row] = __half2float(__ushort_as_half(a[row])) * val;
                        },
                        kGemvThreads);
-    cluster_sync();
+    if (p.S > 1) cluster_sync();
   }
 }
 
@@ -250,91 +272,105 @@ static int dbf_max_clusters(int S, int smem_bytes) {
   return nclusters;
 }
 
-// Size the stages of one product: every tile if it fits in `budget` bytes.
-static int stages_for(int max_tiles, int max_ng, int budget) {
-  const int per = 16 * gemv_rowstride(max_ng) + 16;
-  int ns = max_tiles;
-  if (ns * per > budget) ns = budget / per;
-  return ns;
-}
+static int dbf_bw(int NG, int S) { return (S == 1 || NG % (8 * S) == 0) ? 8 : 4; }
 
 template <int NB>
-static cudaError_t launch_dbf_small_nb(DbfParams p, cudaStream_t stream, int num_sms, int smem_cap) {
-  // K split S and cluster count Q: all CTAs must be co-resident (grid barrier)
+static cudaError_t launch_dbf_small_nb(DbfParams p, const uint32_t* B1, const uint32_t* B2, cudaStream_t stream,
+                                       int num_sms, int smem_cap) {
+  using L = GemvLayout<NB>;
+  // K split S (x digits within budget) and cluster count Q: all CTAs must be
+  // co-resident (grid barrier), so Q never exceeds the occupancy limit
   const int T1 = (p.r + 15) / 16, T2 = (p.m + 15) / 16;
   const int NG1 = p.n / 128, NG2 = p.r / 128;
-  double best = 1e300;
-  DbfParams bestp = p;
-  int bestQ = 0;
   for (int S = 1; S <= 8; S *= 2) {
-    if (S > NG1 || S > NG2) break;
+    if (S > 1 && (S > NG1 || S > NG2)) break;
     DbfParams c = p;
     c.S = S;
+    c.bw1 = dbf_bw(NG1, S);
+    c.bw2 = dbf_bw(NG2, S);
+    c.max_ng1 = ((NG1 + c.bw1 - 1) / c.bw1 + S - 1) / S * c.bw1;
+    c.max_ng2 = ((NG2 + c.bw2 - 1) / c.bw2 + S - 1) / S * c.bw2;
+    const int mng = c.max_ng1 > c.max_ng2 ? c.max_ng1 : c.max_ng2;
+    if (mng * 4 * L::BLOCK > 72 * 1024 && S < 8) continue;
     int Q = num_sms / S;
-    for (int iter = 0; iter < 2; ++iter) {
+    for (int iter = 0; iter < 3; ++iter) {
       c.max_tiles1 = (T1 + Q - 1) / Q;
       c.max_tiles2 = (T2 + Q - 1) / Q;
-      c.max_ng1 = (NG1 + S - 1) / S;
-      c.max_ng2 = (NG2 + S - 1) / S;
       c.ns1 = c.ns2 = 0;
-      const int base = dbf_smem_layout<NB>(c).total + 256;
+      const int base = dbf_smem_layout<NB>(c).total;
       const int budget = smem_cap - base;
-      c.ns1 = stages_for(c.max_tiles1, c.max_ng1, budget / 2);
-      c.ns2 = stages_for(c.max_tiles2, c.max_ng2, budget / 2);
-      if (c.ns1 < 1 || c.ns2 < 1) break;
-      const int occ = dbf_max_clusters<NB>(S, dbf_smem_layout<NB>(c).total);
-      if (occ <= 0) break;
-      if (occ >= Q) {
-        const double work = static_cast<double>(c.max_tiles1) * c.max_ng1 + static_cast<double>(c.max_tiles2) * c.max_ng2;
-        const double cost = work * 2048.0 * (0.55 + 0.05 * NB) + NB * (c.max_ng1 + c.max_ng2) * 128.0 * 9.0 +
-                            (S > 1 ? 3000.0 : 0.0);
-        if (cost < best) {
-          best = cost;
-          bestp = c;
-          bestQ = Q;
-        }
-        break;
+      const int per1 = ((c.max_ng1 + c.bw1 - 1) / c.bw1) * 256 * c.bw1 + 16;
+      const int per2 = ((c.max_ng2 + c.bw2 - 1) / c.bw2) * 256 * c.bw2 + 16;
+      c.ns1 = c.max_tiles1;
+      c.ns2 = c.max_tiles2;
+      if (c.ns1 * per1 + c.ns2 * per2 > budget) {
+        c.ns1 = (budget / 2) / per1;
+        c.ns2 = (budget / 2) / per2;
       }
-      Q = occ;
+      if (c.ns1 < 1 || c.ns2 < 1) break;
+      const int smem = dbf_smem_layout<NB>(c).total;
+      const int occ = dbf_max_clusters<NB>(S, smem);
+      if (occ <= 0) break;
+      if (occ < Q) {
+        Q = occ;
+        continue;
+      }
+      CUtensorMap tm2, tm1;
+      if (!make_tmap_u32_rows(&tm2, B2, c.r, c.n / 32, 4 * c.bw1) ||
+          !make_tmap_u32_rows(&tm1, B1, c.m, c.r / 32, 4 * c.bw2))
+        return cudaErrorInvalidValue;
+      cudaError_t err = cudaFuncSetAttribute(dbf_small_kernel<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      if (err != cudaSuccess) return err;
+      if (getenv("W1_VERBOSE"))
+        fprintf(stderr, "dbf plan: B=%d -> clusters=%d split=%d stages=%d/%d smem=%d\n", NB, Q, S, c.ns1, c.ns2, smem);
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(static_cast<unsigned>(Q * S));
+      cfg.blockDim = dim3(kGemvThreads);
+      cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+      cfg.stream = stream;
+      cudaLaunchAttribute attr[2];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = static_cast<unsigned>(S);
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+      attr[1].val.programmaticStreamSerializationAllowed = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 2;
+      return cudaLaunchKernelEx(&cfg, dbf_small_kernel<NB>, tm2, tm1, c);
     }
   }
-  if (bestQ == 0) return cudaErrorInvalidConfiguration;
-  p = bestp;
-  const int smem = dbf_smem_layout<NB>(p).total;
-  cudaError_t err = cudaFuncSetAttribute(dbf_small_kernel<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (err != cudaSuccess) return err;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(bestQ * p.S));
-  cfg.blockDim = dim3(kGemvThreads);
-  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[2];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = static_cast<unsigned>(p.S);
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[1].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, dbf_small_kernel<NB>, p);
+  return cudaErrorInvalidConfiguration;
 }
+
+size_t dbf_tc_workspace_bytes(int64_t r, int64_t n, int64_t B);
+cudaError_t launch_dbf_tc(const uint16_t* a, const uint32_t* B1, const uint16_t* mid, const uint32_t* B2,
+                          const uint16_t* b, int64_t m, int64_t r, int64_t n, const uint16_t* x, int64_t B, float* y,
+                          void* workspace, cudaStream_t stream, int num_sms);
+
+// Batches of at least this many rows run on the tensor-core path.
+constexpr int64_t kDbfTensorMinBatch = 64;
 
 size_t dbf_workspace_bytes(int64_t m, int64_t r, int64_t n, int64_t B) {
   (void)m;
-  (void)n;
   const int64_t rows = B < 8 ? B : 8;
-  return static_cast<size_t>(256 + 4 * rows * r);
+  size_t bytes = static_cast<size_t>(256 + 4 * rows * r);
+  if (B >= kDbfTensorMinBatch) {
+    const size_t tc = dbf_tc_workspace_bytes(r, n, B);
+    if (tc > bytes) bytes = tc;
+  }
+  return bytes;
 }
 
 cudaError_t launch_dbf(const uint16_t* a, const uint32_t* B1, const uint16_t* mid, const uint32_t* B2,
                        const uint16_t* b, int64_t m, int64_t r, int64_t n, const uint16_t* x, int64_t B,
-                       float* y, void* workspace, cudaStream_t stream, int num_sms, int smem_cap) {
+                       float* y, void* workspace, cudaStream_t stream, int num_sms, int smem_cap,
+                       bool allow_tensor_path = true) {
+  if (allow_tensor_path && B >= kDbfTensorMinBatch)
+    return launch_dbf_tc(a, B1, mid, B2, b, m, r, n, x, B, y, workspace, stream, num_sms);
   DbfParams p = {};
   p.a = a;
-  p.B1 = B1;
   p.mid = mid;
-  p.B2 = B2;
   p.b = b;
   p.bar = reinterpret_cast<unsigned int*>(workspace);
   p.h = reinterpret_cast<float*>(static_cast<unsigned char*>(workspace) + 256);
@@ -348,14 +384,14 @@ cudaError_t launch_dbf(const uint16_t* a, const uint32_t* B1, const uint16_t* mi
     p.y = y + b0 * m;
     cudaError_t err;
     switch (nb) {
-      case 1: err = launch_dbf_small_nb<1>(p, stream, num_sms, smem_cap); break;
-      case 2: err = launch_dbf_small_nb<2>(p, stream, num_sms, smem_cap); break;
-      case 3: err = launch_dbf_small_nb<3>(p, stream, num_sms, smem_cap); break;
-      case 4: err = launch_dbf_small_nb<4>(p, stream, num_sms, smem_cap); break;
-      case 5: err = launch_dbf_small_nb<5>(p, stream, num_sms, smem_cap); break;
-      case 6: err = launch_dbf_small_nb<6>(p, stream, num_sms, smem_cap); break;
-      case 7: err = launch_dbf_small_nb<7>(p, stream, num_sms, smem_cap); break;
-      default: err = launch_dbf_small_nb<8>(p, stream, num_sms, smem_cap); break;
+      case 1: err = launch_dbf_small_nb<1>(p, B1, B2, stream, num_sms, smem_cap); break;
+      case 2: err = launch_dbf_small_nb<2>(p, B1, B2, stream, num_sms, smem_cap); break;
+      case 3: err = launch_dbf_small_nb<3>(p, B1, B2, stream, num_sms, smem_cap); break;
+      case 4: err = launch_dbf_small_nb<4>(p, B1, B2, stream, num_sms, smem_cap); break;
+      case 5: err = launch_dbf_small_nb<5>(p, B1, B2, stream, num_sms, smem_cap); break;
+      case 6: err = launch_dbf_small_nb<6>(p, B1, B2, stream, num_sms, smem_cap); break;
+      case 7: err = launch_dbf_small_nb<7>(p, B1, B2, stream, num_sms, smem_cap); break;
+      default: err = launch_dbf_small_nb<8>(p, B1, B2, stream, num_sms, smem_cap); break;
     }
     if (err != cudaSuccess) return err;
   }
@@ -423,7 +459,7 @@ int dbf_apply_noalloc(const uint16_t* a, const uint32_t* B1, const uint16_t* mid
   // the barrier count must start at zero (a previous call may have timed out)
   if (cudaMemsetAsync(scratch, 0, 8, s) != cudaSuccess) return W1_ERR_CUDA;
   const int cap = d.smem_optin < 200 * 1024 ? d.smem_optin : 200 * 1024;
-  return w1::launch_result(w1::launch_dbf(a, B1, mid, B2, b, m, r, n, x, B, y, scratch, s, d.sms, cap));
+  return w1::launch_result(w1::launch_dbf(a, B1, mid, B2, b, m, r, n, x, B, y, scratch, s, d.sms, cap, false));
 }
 
 }  // extern "C"

@@ -265,6 +265,26 @@ bool make_tmap_bf16_sw128(CUtensorMap* map, const void* base, int64_t rows, int6
   return r == CUDA_SUCCESS;
 }
 
+// 2-D uint32 tensor map over row-major sign words [rows][words], box
+// {box_words, 16 rows}, swizzle equal to the box row bytes (16 B: none, 32, 64
+// or 128 B), zero fill out of bounds.
+bool make_tmap_u32_rows(CUtensorMap* map, const void* base, int64_t rows, int64_t words, int box_words) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(words), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(words) * 4};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(box_words), 16};
+  cuuint32_t estr[2] = {1, 1};
+  CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_NONE;
+  if (box_words * 4 == 32) sw = CU_TENSOR_MAP_SWIZZLE_32B;
+  if (box_words * 4 == 64) sw = CU_TENSOR_MAP_SWIZZLE_64B;
+  if (box_words * 4 == 128) sw = CU_TENSOR_MAP_SWIZZLE_128B;
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 cudaError_t launch_gemm(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t K,
                         const uint16_t* x, int64_t M, float* y, cudaStream_t stream, int num_sms) {
   using namespace gemm;

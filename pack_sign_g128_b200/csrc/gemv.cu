@@ -19,12 +19,15 @@
 //    exactly the order the bit extraction produces, so the canonical weight
 //    layout is read unchanged (the DBF post, section 5 items 7-8: repack the
 //    activation locally, keep the weight file canonical).
-//  * Memory: a cluster of S CTAs splits K; each CTA streams its rows' K-slice
-//    of sign words with 1-D bulk copies (all stages issued up front when they
-//    fit), and the S partial results are reduced through distributed shared
-//    memory in a fixed order (deterministic, no atomics, no workspace).
-//  * Programmatic dependent launch: before waiting on the previous kernel the
-//    CTA only prefetches its weight bytes into L2.
+//  * Memory: each 16-row tile of sign words arrives by swizzled 2-D TMA boxes
+//    (16 rows x 4 or 8 groups, one instruction each; all stages issued up
+//    front when they fit).  Up to 16 consumer warps share a tile, each taking
+//    a K sub-range, so every warp's dependency chain is short.  When B x K is
+//    too large for one CTA's shared memory a cluster of S CTAs splits K; the
+//    sub-range and cluster partial sums are reduced in a fixed order through
+//    (distributed) shared memory: deterministic, no atomics, no workspace.
+//  * Programmatic dependent launch: the kernel waits for the previous kernel
+//    before touching memory and lets the next one launch right away.
 #include <cstdint>
 #include <cuda_fp16.h>
 #include <cstdio>
@@ -36,7 +39,6 @@
 namespace w1 {
 
 struct GemvParams {
-  const uint32_t* signs;
   const uint16_t* scales;
   const uint16_t* x;
   float* y;
@@ -46,40 +48,45 @@ struct GemvParams {
   int rows;         // rows handled by this launch
   int NG;           // K / 128
   int S;            // cluster size (K split)
+  int bw;           // groups per TMA box (4 or 8)
   int ns;           // pipeline stages
   int max_tiles;    // max 16-row tiles per cluster
   int max_ng;       // max groups per CTA
 };
 
 struct GemvSmem {
-  int stages, xq, xsum, xf, sc, part, bars, total;
+  int stages, stage_bytes, xq, zero, xsum, xf, sc, part, bars, total;
 };
 
 template <int NB>
-__host__ __device__ inline GemvSmem gemv_smem_layout(int ns, int max_tiles, int max_ng) {
-  constexpr int NT = GemvLayout<NB>::NT;
-  GemvSmem L;
+__host__ __device__ inline GemvSmem gemv_smem_layout(int ns, int max_tiles, int max_ng, int bw) {
+  using L = GemvLayout<NB>;
+  GemvSmem M;
   int off = 0;
-  L.stages = off;
-  off += ns * 16 * gemv_rowstride(max_ng);
+  M.stages = off;
+  M.stage_bytes = ((max_ng + bw - 1) / bw) * 16 * 16 * bw;
+  off += ns * M.stage_bytes;
   off = round_up(off, 128);
-  L.xq = off;
-  off += max_ng * 4 * NT * 256;
-  L.xsum = off;
+  M.xq = off;
+  off += max_ng * 4 * L::BLOCK;
+  off = round_up(off, 16);
+  M.zero = off;
+  off += 16;
+  M.xsum = off;
   off += max_ng * NB * 4;
-  L.xf = off;
+  M.xf = off;
   off += max_ng * NB * 4;
   off = round_up(off, 16);
-  L.sc = off;
+  M.sc = off;
   off += max_tiles * 16 * max_ng * 2;
   off = round_up(off, 16);
-  L.part = off;
-  off += NB * max_tiles * 16 * 4;
+  M.part = off;
+  off += gemv_wpt(max_tiles) * NB * max_tiles * 16 * 4;
   off = round_up(off, 8);
-  L.bars = off;
+  M.bars = off;
   off += 2 * ns * 8;
-  L.total = round_up(off, 128);
-  return L;
+  M.total = round_up(off, 128) + 1024;  // + alignment slack for the 1024-aligned stages
+  return M;
 }
 
 __device__ __forceinline__ float bf16_bits_to_f32(uint32_t b) { return __uint_as_float(b << 16); }
@@ -97,45 +104,51 @@ __device__ __forceinline__ void load16_bf16(const uint16_t* p, float (&v)[16]) {
 }
 
 template <int NB>
-__global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams p) {
-  extern __shared__ __align__(128) unsigned char smem[];
-  const GemvSmem L = gemv_smem_layout<NB>(p.ns, p.max_tiles, p.max_ng);
+__global__ void __launch_bounds__(kGemvThreads, 1)
+    gemv_kernel(const __grid_constant__ CUtensorMap tmap, const GemvParams p) {
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem =
+      reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const GemvSmem M = gemv_smem_layout<NB>(p.ns, p.max_tiles, p.max_ng, p.bw);
   GemvSmemView v;
-  v.stages = smem + L.stages;
+  v.stages = smem + M.stages;
   v.ns = p.ns;
-  v.full = reinterpret_cast<uint64_t*>(smem + L.bars);
+  v.stage_bytes = M.stage_bytes;
+  v.full = reinterpret_cast<uint64_t*>(smem + M.bars);
   v.empty = v.full + p.ns;
   GemvXView xv;
-  xv.xq = smem + L.xq;
-  xv.xsum = reinterpret_cast<int*>(smem + L.xsum);
-  xv.xf = reinterpret_cast<float*>(smem + L.xf);
-  xv.sc = reinterpret_cast<uint16_t*>(smem + L.sc);
-  xv.part = reinterpret_cast<float*>(smem + L.part);
+  xv.xq = smem + M.xq;
+  xv.xsum = reinterpret_cast<int*>(smem + M.xsum);
+  xv.xf = reinterpret_cast<float*>(smem + M.xf);
+  xv.sc = reinterpret_cast<uint16_t*>(smem + M.sc);
+  xv.part = reinterpret_cast<float*>(smem + M.part);
   xv.part_stride = p.max_tiles * 16;
+  unsigned char* zero16 = smem + M.zero;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int crank = static_cast<int>(cluster_ctarank());
   const Split sp = make_split(p.rows, p.row_base, p.NG, p.S, crank, static_cast<int>(cluster_id_x()),
-                              static_cast<int>(nclusters_x()));
-  const int64_t wrow = p.K >> 5;
+                              static_cast<int>(nclusters_x()), p.bw, p.bw, p.max_tiles);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < p.ns; ++s) {
       mbar_init(&v.full[s], 1);
-      mbar_init(&v.empty[s], 1);
+      mbar_init(&v.empty[s], static_cast<uint32_t>(sp.wpt));
     }
     fence_mbarrier_init();
+    asm volatile("prefetch.tensormap [%0];" ::"l"(&tmap) : "memory");
   }
-  if (warp == kProducerWarp) prefetch_weights(sp, p.signs, wrow, p.scales, p.NG, lane);
+  if (threadIdx.x < 4) reinterpret_cast<uint32_t*>(zero16)[threadIdx.x] = 0u;
   __syncthreads();
   pdl_wait();
-  // the next kernel in the stream may start now: its CTAs only prefetch their
-  // own weights into L2 until this grid has completed
+  // the next kernel in the stream may launch now; it touches no memory before
+  // its own dependency wait, i.e. before this grid has completed
   pdl_launch_dependents();
 
   int first = 0;
-  if (warp == kProducerWarp) first = issue_first_tiles(v, sp, p.signs, wrow, lane);
+  if (warp == kProducerWarp && lane == 0) first = issue_first_tiles(v, sp, &tmap, p.bw);
+  __syncwarp();
 
   // activations -> digit planes; scales of this CTA's rows and groups -> smem
   const uint16_t* xb = p.x;
@@ -146,62 +159,24 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(const GemvParams 
   stage_scales(xv, sp, p.scales, p.NG, kGemvThreads);
   __syncthreads();
 
-  if (warp == kProducerWarp)
-    produce_rest(v, sp, p.signs, wrow, first, lane);
-  else
-    consume_tiles<NB, true>(v, xv, sp, warp, lane);
-  cluster_sync();
+  if (warp == kProducerWarp) {
+    if (lane == 0) produce_rest(v, sp, &tmap, p.bw, first);
+    __syncwarp();  // converge before the (cluster) barrier, which is .aligned
+  } else {
+    consume_tiles<NB, true>(v, xv, sp, p.bw, zero16, warp, lane);
+  }
+  if (p.S > 1) cluster_sync(); else __syncthreads();
   float* y = p.y;
   const int64_t N = p.N;
   cluster_reduce<NB>(xv, sp, p.S, crank, [&](int b, int64_t row, float val) { y[b * N + row] = val; },
                      kGemvThreads);
-  cluster_sync();
+  if (p.S > 1) cluster_sync();
 }
 
 // ------------------------------------------------------------------ host side
 
-template <int NB>
-static cudaError_t launch_gemv_nb(const GemvParams& base, int Q, int S, cudaStream_t stream,
-                                  int smem_cap) {
-  GemvParams p = base;
-  p.S = S;
-  const int T16 = (p.rows + 15) / 16;
-  p.max_tiles = (T16 + Q - 1) / Q;
-  p.max_ng = (p.NG + S - 1) / S;
-  const int stage_bytes = 16 * gemv_rowstride(p.max_ng);
-  // stage count: every tile if it fits, else what the budget allows
-  const GemvSmem L0 = gemv_smem_layout<NB>(0, p.max_tiles, p.max_ng);
-  int ns = p.max_tiles;
-  const int budget = smem_cap - L0.total - 256;
-  if (ns * (stage_bytes + 16) > budget) ns = budget / (stage_bytes + 16);
-  if (ns < 1) return cudaErrorInvalidConfiguration;
-  p.ns = ns;
-  const GemvSmem L = gemv_smem_layout<NB>(ns, p.max_tiles, p.max_ng);
-  cudaError_t err = cudaFuncSetAttribute(gemv_kernel<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         L.total);
-  if (err != cudaSuccess) return err;
-  if (S > 8) {
-    err = cudaFuncSetAttribute(gemv_kernel<NB>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-    if (err != cudaSuccess) return err;
-  }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(Q * S));
-  cfg.blockDim = dim3(kGemvThreads);
-  cfg.dynamicSmemBytes = static_cast<size_t>(L.total);
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[2];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = static_cast<unsigned>(S);
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[1].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, gemv_kernel<NB>, p);
-}
+bool make_tmap_u32_rows(CUtensorMap* map, const void* base, int64_t rows, int64_t words, int box_words);
 
-// Largest number of co-resident clusters of size S for this kernel/smem.
 template <int NB>
 static int gemv_max_clusters(int S, int smem_bytes) {
   cudaLaunchConfig_t cfg = {};
@@ -225,63 +200,112 @@ static int gemv_max_clusters(int S, int smem_bytes) {
   return n;
 }
 
-// Choose the K split S (cluster size) and the number of clusters Q so that
-// every cluster is co-resident (one wave) and the per-CTA work is smallest.
+struct GemvPlan {
+  int Q, S, bw, ns, max_tiles, max_ng, smem;
+};
+
+// K split S: the smallest that keeps this CTA's activation digits within
+// budget (K split only pays off when x is large); clusters Q: one resident
+// wave; stages: every tile when it fits.
 template <int NB>
-static void gemv_plan(int64_t rows, int NG, int num_sms, int smem_cap, int* Q_out, int* S_out) {
-  const int T16 = static_cast<int>((rows + 15) / 16);
-  double best = 1e300;
-  int bq = 1, bs = 1;
+static bool gemv_make_plan(int rows, int NG, int num_sms, int smem_cap, int force_s, GemvPlan* out) {
+  using L = GemvLayout<NB>;
+  const int T16 = (rows + 15) / 16;
   for (int S = 1; S <= 8; S *= 2) {
-    if (S > NG) break;
+    if (force_s && S != force_s) continue;
+    if (S > NG && S > 1) break;
+    const int bw = (NG % (8 * S) == 0 || S == 1) ? 8 : 4;
+    const int units = (NG + bw - 1) / bw;
+    const int max_ng = ((units + S - 1) / S) * bw;
+    if (!force_s && max_ng * 4 * L::BLOCK > 80 * 1024 && S < 8) continue;
     int Q = num_sms / S;
-    const int occ = gemv_max_clusters<NB>(S, smem_cap);
-    if (occ > 0 && occ < Q) Q = occ;
     if (Q > T16) Q = T16;
     if (Q < 1) Q = 1;
-    const double tiles = static_cast<double>((T16 + Q - 1) / Q);
-    const double groups = static_cast<double>((NG + S - 1) / S);
-    // weights: ~0.6 issue slots per weight; x prep: ~9 per element per cluster
-    const double cost = tiles * groups * 2048.0 * (0.55 + 0.05 * NB) + NB * groups * 128.0 * 9.0 +
-                        (S > 1 ? 1500.0 : 0.0);
-    if (cost < best * 0.98) {
-      best = cost;
-      bq = Q;
-      bs = S;
-    }
-  }
-  *Q_out = bq;
-  *S_out = bs;
-}
-
-struct GemvPlanEntry {
-  int64_t rows;
-  int NG, NB, sms, cap, dev, Q, S;
-};
-static GemvPlanEntry g_plan_cache[64];
-static int g_plan_count = 0;
-static std::mutex g_plan_mu;
-
-static bool gemv_plan_cached(int64_t rows, int NG, int NB, int sms, int cap, int* Q, int* S) {
-  int dev = 0;
-  cudaGetDevice(&dev);
-  std::lock_guard<std::mutex> lock(g_plan_mu);
-  for (int i = 0; i < g_plan_count; ++i) {
-    const GemvPlanEntry& e = g_plan_cache[i];
-    if (e.rows == rows && e.NG == NG && e.NB == NB && e.sms == sms && e.cap == cap && e.dev == dev) {
-      *Q = e.Q;
-      *S = e.S;
+    for (int iter = 0; iter < 3; ++iter) {
+      const int max_tiles = (T16 + Q - 1) / Q;
+      const GemvSmem M0 = gemv_smem_layout<NB>(0, max_tiles, max_ng, bw);
+      const int stage_bytes = ((max_ng + bw - 1) / bw) * 16 * 16 * bw;
+      int ns = max_tiles;
+      const int budget = smem_cap - M0.total;
+      if (ns * (stage_bytes + 16) > budget) ns = budget / (stage_bytes + 16);
+      if (ns < 1) return false;
+      const int smem = gemv_smem_layout<NB>(ns, max_tiles, max_ng, bw).total;
+      const int occ = gemv_max_clusters<NB>(S, smem);
+      if (occ > 0 && occ < Q) {
+        Q = occ;
+        continue;
+      }
+      *out = GemvPlan{Q, S, bw, ns, max_tiles, max_ng, smem};
       return true;
     }
   }
   return false;
 }
-static void gemv_plan_store(int64_t rows, int NG, int NB, int sms, int cap, int Q, int S) {
+
+struct GemvPlanEntry {
+  int rows, NG, NB, sms, cap, dev, force;
+  GemvPlan plan;
+};
+static GemvPlanEntry g_plan_cache[64];
+static int g_plan_count = 0;
+static std::mutex g_plan_mu;
+
+template <int NB>
+static cudaError_t launch_gemv_nb(const uint32_t* signs, const GemvParams& base, cudaStream_t stream, int num_sms,
+                                  int smem_cap) {
+  int force = 0;
+  if (const char* f = getenv("W1_GEMV_SPLIT")) force = atoi(f);  // tuning knob: force the K split
+  if (force != 1 && force != 2 && force != 4 && force != 8) force = 0;
   int dev = 0;
   cudaGetDevice(&dev);
-  std::lock_guard<std::mutex> lock(g_plan_mu);
-  const int i = g_plan_count < 64 ? g_plan_count++ : static_cast<int>((rows + NG) & 63);
-  g_plan_cache[i] = GemvPlanEntry{rows, NG, NB, sms, cap, dev, Q, S};
+  GemvPlan plan;
+  bool found = false;
+  {
+    std::lock_guard<std::mutex> lock(g_plan_mu);
+    for (int i = 0; i < g_plan_count; ++i) {
+      const GemvPlanEntry& e = g_plan_cache[i];
+      if (e.rows == base.rows && e.NG == base.NG && e.NB == NB && e.sms == num_sms && e.cap == smem_cap &&
+          e.dev == dev && e.force == force) {
+        plan = e.plan;
+        found = true;
+        break;
+      }
+    }
+  }
+  if (!found) {
+    if (!gemv_make_plan<NB>(base.rows, base.NG, num_sms, smem_cap, force, &plan)) return cudaErrorInvalidConfiguration;
+    std::lock_guard<std::mutex> lock(g_plan_mu);
+    const int i = g_plan_count < 64 ? g_plan_count++ : (base.rows + base.NG + NB) & 63;
+    g_plan_cache[i] = GemvPlanEntry{base.rows, base.NG, NB, num_sms, smem_cap, dev, force, plan};
+  }
+  if (getenv("W1_VERBOSE"))
+    fprintf(stderr, "w1_gemv plan: rows=%d NG=%d B=%d -> clusters=%d split=%d box=%d stages=%d tiles=%d smem=%d\n",
+            base.rows, base.NG, NB, plan.Q, plan.S, plan.bw, plan.ns, plan.max_tiles, plan.smem);
+  GemvParams p = base;
+  p.S = plan.S;
+  p.bw = plan.bw;
+  p.ns = plan.ns;
+  p.max_tiles = plan.max_tiles;
+  p.max_ng = plan.max_ng;
+  CUtensorMap tmap;
+  if (!make_tmap_u32_rows(&tmap, signs, base.N, base.K / 32, 4 * plan.bw)) return cudaErrorInvalidValue;
+  cudaError_t err = cudaFuncSetAttribute(gemv_kernel<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize, plan.smem);
+  if (err != cudaSuccess) return err;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(plan.Q * plan.S));
+  cfg.blockDim = dim3(kGemvThreads);
+  cfg.dynamicSmemBytes = static_cast<size_t>(plan.smem);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(plan.S);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, gemv_kernel<NB>, tmap, p);
 }
 
 cudaError_t launch_gemv(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t K,
@@ -292,31 +316,7 @@ cudaError_t launch_gemv(const uint32_t* signs, const uint16_t* scales, int64_t N
   const int64_t max_rows = 32768;
   for (int64_t r0 = 0; r0 < N; r0 += max_rows) {
     const int rows = static_cast<int>((N - r0) < max_rows ? (N - r0) : max_rows);
-    int Q = 1, S = 1;
-    if (!gemv_plan_cached(rows, NG, B, num_sms, smem_cap, &Q, &S)) {
-    switch (B) {
-      case 1: gemv_plan<1>(rows, NG, num_sms, smem_cap, &Q, &S); break;
-      case 2: gemv_plan<2>(rows, NG, num_sms, smem_cap, &Q, &S); break;
-      case 3: gemv_plan<3>(rows, NG, num_sms, smem_cap, &Q, &S); break;
-      case 4: gemv_plan<4>(rows, NG, num_sms, smem_cap, &Q, &S); break;
-      case 5: gemv_plan<5>(rows, NG, num_sms, smem_cap, &Q, &S); break;
-      case 6: gemv_plan<6>(rows, NG, num_sms, smem_cap, &Q, &S); break;
-      case 7: gemv_plan<7>(rows, NG, num_sms, smem_cap, &Q, &S); break;
-      default: gemv_plan<8>(rows, NG, num_sms, smem_cap, &Q, &S); break;
-    }
-    gemv_plan_store(rows, NG, B, num_sms, smem_cap, Q, S);
-    }
-    if (const char* f = getenv("W1_GEMV_SPLIT")) {  // tuning knob: force the K split
-      const int fs = atoi(f);
-      if (fs == 1 || fs == 2 || fs == 4 || fs == 8) {
-        if (fs != S) Q = (num_sms / fs < (rows + 15) / 16) ? num_sms / fs : static_cast<int>((rows + 15) / 16);
-        S = fs;
-      }
-    }
-    if (getenv("W1_VERBOSE")) fprintf(stderr, "w1_gemv plan: rows=%d K=%lld B=%d -> clusters=%d split=%d\n", rows,
-                                      static_cast<long long>(K), B, Q, S);
     GemvParams p = {};
-    p.signs = signs;
     p.scales = scales;
     p.x = x;
     p.y = y;
@@ -327,14 +327,14 @@ cudaError_t launch_gemv(const uint32_t* signs, const uint16_t* scales, int64_t N
     p.NG = NG;
     cudaError_t err;
     switch (B) {
-      case 1: err = launch_gemv_nb<1>(p, Q, S, stream, smem_cap); break;
-      case 2: err = launch_gemv_nb<2>(p, Q, S, stream, smem_cap); break;
-      case 3: err = launch_gemv_nb<3>(p, Q, S, stream, smem_cap); break;
-      case 4: err = launch_gemv_nb<4>(p, Q, S, stream, smem_cap); break;
-      case 5: err = launch_gemv_nb<5>(p, Q, S, stream, smem_cap); break;
-      case 6: err = launch_gemv_nb<6>(p, Q, S, stream, smem_cap); break;
-      case 7: err = launch_gemv_nb<7>(p, Q, S, stream, smem_cap); break;
-      default: err = launch_gemv_nb<8>(p, Q, S, stream, smem_cap); break;
+      case 1: err = launch_gemv_nb<1>(signs, p, stream, num_sms, smem_cap); break;
+      case 2: err = launch_gemv_nb<2>(signs, p, stream, num_sms, smem_cap); break;
+      case 3: err = launch_gemv_nb<3>(signs, p, stream, num_sms, smem_cap); break;
+      case 4: err = launch_gemv_nb<4>(signs, p, stream, num_sms, smem_cap); break;
+      case 5: err = launch_gemv_nb<5>(signs, p, stream, num_sms, smem_cap); break;
+      case 6: err = launch_gemv_nb<6>(signs, p, stream, num_sms, smem_cap); break;
+      case 7: err = launch_gemv_nb<7>(signs, p, stream, num_sms, smem_cap); break;
+      default: err = launch_gemv_nb<8>(signs, p, stream, num_sms, smem_cap); break;
     }
     if (err != cudaSuccess) return err;
   }

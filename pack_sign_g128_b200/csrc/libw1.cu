@@ -4,5 +4,6 @@
 #include "pack.cu"
 #include "gemv.cu"
 #include "gemm.cu"
+#include "dbf_tc.cu"
 #include "dbf.cu"
 #include "moe.cu"

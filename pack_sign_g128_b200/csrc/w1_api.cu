@@ -20,7 +20,8 @@ cudaError_t launch_gemm(const uint32_t* signs, const uint16_t* scales, int64_t N
 
 cudaError_t launch_dbf(const uint16_t* a, const uint32_t* B1, const uint16_t* mid, const uint32_t* B2,
                        const uint16_t* b, int64_t m, int64_t r, int64_t n, const uint16_t* x, int64_t B,
-                       float* y, void* workspace, cudaStream_t stream, int num_sms, int smem_cap);
+                       float* y, void* workspace, cudaStream_t stream, int num_sms, int smem_cap,
+                       bool allow_tensor_path);
 size_t dbf_workspace_bytes(int64_t m, int64_t r, int64_t n, int64_t B);
 
 struct DeviceInfo {
@@ -153,7 +154,7 @@ int dbf_apply(const uint16_t* a, const uint32_t* B1, const uint16_t* mid, const 
   if (st != W1_OK) return st;
   const int cap = d.smem_optin < 200 * 1024 ? d.smem_optin : 200 * 1024;
   return launch_result(launch_dbf(a, B1, mid, B2, b, m, r, n, x, B, y, workspace,
-                                  reinterpret_cast<cudaStream_t>(stream), d.sms, cap));
+                                  reinterpret_cast<cudaStream_t>(stream), d.sms, cap, true));
 }
 
 }  // extern "C"
