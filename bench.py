@@ -184,7 +184,15 @@ def build_gemv_sweep(torch, ops, synth, l2_bytes: int):
             with torch.cuda.graph(g, stream=stream):
                 for r in range(R):
                     ops.w1_gemv(signs[r], scales[r], x, y)
-            combos.append({"N": N, "K": K, "B": B, "R": R, "graph": g, "x": x, "y": y,
+            # the same chain with W1_GEMV_STATIC_WEIGHTS (weights written long before)
+            with torch.cuda.stream(stream):
+                ops.w1_gemv(signs[0], scales[0], x, y, static_weights=True)
+            stream.synchronize()
+            gs = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gs, stream=stream):
+                for r in range(R):
+                    ops.w1_gemv(signs[r], scales[r], x, y, static_weights=True)
+            combos.append({"N": N, "K": K, "B": B, "R": R, "graph": g, "graph_static": gs, "x": x, "y": y,
                            "signs": signs, "scales": scales, "bytes": pb})
     torch.cuda.synchronize()
     return combos, stream
@@ -216,6 +224,25 @@ def time_gemv_steps_detailed(torch, combos, stream, steps: int, warmup: int, wor
     total_ms = start.elapsed_time(end)
     per_pair_ms = [sum(evs[s][i][0].elapsed_time(evs[s][i][1]) for s in range(steps)) for i in range(len(combos))]
     return total_ms, per_pair_ms
+
+
+def time_gemv_static(torch, combos, stream, reps: int = 3):
+    """Per-pair device time of the W1_GEMV_STATIC_WEIGHTS chains (outside the timed steps)."""
+    out = []
+    for cb in combos:
+        with torch.cuda.stream(stream):
+            cb["graph_static"].replay()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(reps):
+                cb["graph_static"].replay()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        out.append(e0.elapsed_time(e1) * 1e3 / (reps * cb["R"]))
+    return out
 
 
 def gemv_e2e(torch, ops, combos, steps: int):
@@ -468,13 +495,17 @@ def run_gpu(args):
     all_bytes = sum_over_ranks(world, float(bytes_per_step * args.steps))
     value = all_bytes / (t_max * 1e-3) / 1e9
 
+    static_us = time_gemv_static(torch, combos, stream)
     gemv_rows = []
-    for cb, ms in zip(combos, per_pair_ms):
+    for cb, ms, st_us in zip(combos, per_pair_ms, static_us):
         per_launch_us = ms * 1e3 / (cb["R"] * args.steps)
         gbs = cb["bytes"] / (per_launch_us * 1e-6) / 1e9
         gemv_rows.append({"N": cb["N"], "K": cb["K"], "B": cb["B"], "launches": cb["R"],
+                          "kernel": "gemv_direct_kernel" if cb["B"] <= 4 else "gemv_tc_kernel",
                           "us_per_launch": round(per_launch_us, 3), "GB/s": round(gbs, 1),
-                          "frac_hbm": round(gbs / peaks["hbm_gbs"], 4)})
+                          "frac_hbm": round(gbs / peaks["hbm_gbs"], 4),
+                          "static_weights_us_per_launch": round(st_us, 3),
+                          "static_weights_GB/s": round(cb["bytes"] / (st_us * 1e-6) / 1e9, 1)})
     pair_sum_ms = sum(per_pair_ms)
     achieved = bytes_per_step * args.steps / (pair_sum_ms * 1e-3) / 1e9
 
@@ -508,7 +539,7 @@ def run_gpu(args):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "s8xs8->s32 tensor MMA + f32 scale fold (x bf16, 1-bit weights, fp16 scales)",
+        "dtype": "s8 x s8 -> s32 MMA (mma.sync at B<=4, tcgen05 kind::i8 at B>4) + f32 scale fold; x bf16, 1-bit weights, fp16 scales",
         "data": "synthetic",
         "config": {"workload": WORKLOAD, "launches_per_step": launches_per_step,
                    "packed_bytes_per_step": bytes_per_step,
@@ -517,7 +548,8 @@ def run_gpu(args):
                    "parallelism": f"replicas x{world} (independent sweeps, no collective)"},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                      "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
-                     "traffic": None, "kernel": "gemv_kernel", "peak_kind": peaks_kind},
+                     "traffic": None, "kernel": "gemv_direct_kernel (B<=4), gemv_tc_kernel (B=8)",
+                     "peak_kind": peaks_kind},
         "cpu_baseline": cpu,
         "e2e": {k: e2e[k] for k in ("value", "unit", "h2d_bytes_per_step", "d2h_bytes_per_step")},
         "gpu_launches": launches_per_step * args.steps,

@@ -96,6 +96,25 @@ int w1_pack(const float* W, int64_t N, int64_t K, uint32_t* signs, uint16_t* sca
 int w1_gemv(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t K,
             const uint16_t* x, int64_t B, float* y, w1_stream_t stream);
 
+/* Flags for w1_gemv_ex. */
+enum { W1_GEMV_STATIC_WEIGHTS = 1 };
+
+/*
+ * w1_gemv_ex -- w1_gemv with flags (0 gives w1_gemv exactly).  The pages have
+ * no counterpart: this is a scheduling contract, not new arithmetic.
+ * W1_GEMV_STATIC_WEIGHTS: the caller promises that `signs` and `scales` were
+ * written before the kernel that precedes this call on `stream` began (weights
+ * loaded once, used by many decode steps).  The kernel may then start reading
+ * them while that kernel is still running (programmatic dependent launch),
+ * which hides most of its load latency in a chain of back-to-back products.
+ * Without the promise (or with weights written by the preceding kernel, e.g.
+ * w1_pack immediately before) the flag can return stale weights: leave it 0.
+ * x and y are always ordered after the preceding kernel.  Other flag bits:
+ * W1_ERR_SHAPE.
+ */
+int w1_gemv_ex(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t K,
+               const uint16_t* x, int64_t B, float* y, uint32_t flags, w1_stream_t stream);
+
 /*
  * w1_gemm -- prefill-regime product for many token rows (DBF post, section 4:
  * prompt processing amortises weight loads across columns).

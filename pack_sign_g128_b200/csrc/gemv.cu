@@ -308,9 +308,32 @@ static cudaError_t launch_gemv_nb(const uint32_t* signs, const GemvParams& base,
   return cudaLaunchKernelEx(&cfg, gemv_kernel<NB>, tmap, p);
 }
 
+cudaError_t launch_gemv_tc(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t K, const uint16_t* x,
+                           int B, float* y, cudaStream_t stream, int num_sms);
+cudaError_t launch_gemv_direct(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t K,
+                               const uint16_t* x, int B, float* y, bool static_weights, cudaStream_t stream,
+                               int num_sms, int smem_cap);
+
+// Kernel choice, from measurements on the decode shapes: the direct kernel
+// (gemv_direct.cu) for B <= 4, the tcgen05 kernel (gemv_tc.cu) for larger
+// batches, each only where its plan fits the shape, else the mma.sync ring
+// kernel below.  W1_GEMV_PATH=direct|tc|mma forces one kernel (tuning and
+// testing knob; a forced kernel whose plan does not fit the shape fails with
+// W1_ERR_UNSUPPORTED).
 cudaError_t launch_gemv(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t K,
                         const uint16_t* x, int B, float* y, cudaStream_t stream, int num_sms,
-                        int smem_cap) {
+                        int smem_cap, bool static_weights) {
+  const char* path = getenv("W1_GEMV_PATH");
+  const char which = path ? path[0] : 'a';
+  if (which == 'd' || (which == 'a' && B <= 4)) {
+    const cudaError_t e =
+        launch_gemv_direct(signs, scales, N, K, x, B, y, static_weights, stream, num_sms, smem_cap);
+    if (e != cudaErrorNotSupported || which == 'd') return e;
+  }
+  if (which == 't' || (which == 'a' && B > 4)) {
+    const cudaError_t e = launch_gemv_tc(signs, scales, N, K, x, B, y, stream, num_sms);
+    if (e != cudaErrorNotSupported || which == 't') return e;
+  }
   const int NG = static_cast<int>(K / 128);
   // rows per launch bounded so that per-CTA scale / partial buffers fit
   const int64_t max_rows = 32768;

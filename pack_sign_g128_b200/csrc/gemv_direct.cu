@@ -1,0 +1,741 @@
+// w1_gemv: the decode kernel (1 <= B <= 8).
+//
+//   y[b,n] = sum_g s[n,g] * sum_{k in g} (1 - 2 bit[n,k]) x[b,k]
+//
+// Storage format: "1-bit group-128 sign packing" (one sign bit per weight,
+// LSB-first in uint32 words along K, one fp16 mean|w| scale per 128 weights).
+//
+// Built for latency: a decode GEMV moves a few MB, so the time of one launch is
+// set by its serial chain, not by bandwidth.  The kernel therefore
+//  * issues every weight byte it will need at its first instruction: each warp
+//    copies its rows x K-range of sign words into shared memory with 16-byte
+//    asynchronous copies (cp.async, every lane, all in flight at once) and,
+//    with the W1_GEMV_STATIC_WEIGHTS flag, does so before waiting on the
+//    previous kernel in the stream (programmatic dependent launch);
+//  * quantises the activations of its K range once per CTA while those copies
+//    are in flight, then lets every warp run alone until the final reduction;
+//  * reduces a K split over a thread-block cluster with one barrier: partial
+//    sums are stored straight into the owning CTA's shared memory (DSMEM), and
+//    only the owner reads them.
+//
+// Arithmetic (exact up to the fp32 fold):
+//  * Activations -> fixed point.  Per (batch row, group) x is scaled by
+//    2^(22-E) (E from the group max), rounded to a 23-bit integer and split
+//    into three signed int8 digits hi/mid/lo.  Error <= 2^(E-23) per element.
+//  * Signs -> int8 {0, -1} with one PRMT per 4 weights (a byte table keyed on
+//    bit 0, 1 or 2 of each selector nibble; bit 3 via w >> 3; upper half via
+//    w >> 16), so  sum (1-2b) n = X + 2 * sum (-b) n  with X = sum n.
+//  * int8 mma.sync m16n8k32, A = activation digits (rows), B = sign bytes
+//    (8 weight rows), s32 accumulators; one fold per group:
+//    acc += s * (f*W_p * D_p + [p = hi] f*X),  W = {2^17, 2^9, 2}, f = 2^(E-22).
+//  * At B = 1 and 2 the 16-row MMA would hold only 3 or 6 digit rows, so 4 or
+//    2 groups share one MMA: lane quad c of an MMA contributes the sign bytes
+//    of group (c * G / 4), and the digit rows of group j carry zeros in the
+//    slots of the other groups (block-diagonal A).  The MMA count per weight
+//    stays the same, the folds drop by the same factor G.
+// K order inside one MMA is free as long as A and B agree: k-slot 4c+i+16h of
+// MMA (w, q) holds bit q + 4i + 16h of word (c*G + w) of the set, which is the
+// order the PRMT extraction produces.
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstdio>
+#include <cstdlib>
+#include <cuda_fp16.h>
+#include <mutex>
+#include <type_traits>
+
+#include "w1_common.cuh"
+
+namespace w1 {
+
+namespace gd {
+constexpr int kWarps = 8;
+constexpr int kThreads = kWarps * 32;
+constexpr int kMaxTw = 4;        // 8-row n-tiles per warp
+constexpr int kDigitStride = 34;  // words per digit row of the activation scratch (bank spread)
+constexpr int kMaxSets = 64;      // sets (of G groups) per CTA
+
+template <int NB>
+struct Cfg {
+  static constexpr int G = NB == 1 ? 4 : (NB == 2 ? 2 : 1);  // groups per MMA set
+  static constexpr int ROWS = 3 * NB * G;                     // digit rows in use
+  static constexpr int MT = (ROWS + 15) / 16;                 // m16 tiles
+  static constexpr int ITEMS = G * NB * 8;                    // 16-element activation items per set
+  static constexpr int IPL = (ITEMS + 31) / 32;               // items per lane
+  static constexpr int SCR = ROWS * kDigitStride + 2 * ROWS;  // scratch words: digits, f*W_p, f*X
+};
+}  // namespace gd
+
+struct GdParams {
+  const uint32_t* signs;
+  const uint16_t* scales;
+  const uint16_t* x;
+  float* y;
+  int N, K, NG;
+  int S;      // CTAs per cluster (K split)
+  int Q;      // clusters
+  int NT;     // 8-row n-tiles in total
+  int Wn, Wg;  // warps along n-tiles x along sets (Wn * Wg = 8)
+  int Tw;     // n-tiles per warp (max)
+  int NSw;    // sets per warp (max)
+  int P;      // bytes per staged weight row
+  int chunk;  // rows owned per CTA in the cluster reduction
+  int NSc;    // sets per CTA (max)
+  int lgS, lgWg;  // log2 of S and Wg
+  int lgGw;   // log2 of the power-of-two stride >= NSw * G (staging loops)
+  int tq, tr;  // NT = Q * tq + tr
+  int early;  // read weights before the grid dependency wait
+};
+
+struct GdSmem {
+  int warp_bytes, wts, scl, xs, red, part, total;
+};
+
+// Per warp: staged sign words (8*Tw rows of P bytes), scales (float,
+// [group][row]).  Per CTA: activation scratch (nsc sets of SCR words), the
+// reduction buffer and (cluster) the owner partials.
+template <int NB>
+__host__ __device__ inline GdSmem gd_layout(int Tw, int NSw, int P, int S, int chunk, int nsc) {
+  using C = gd::Cfg<NB>;
+  GdSmem L;
+  L.wts = 0;
+  L.scl = L.wts + 8 * Tw * P;
+  L.warp_bytes = (L.scl + NSw * C::G * 8 * Tw * 4 + 15) / 16 * 16;
+  L.xs = gd::kWarps * L.warp_bytes;
+  L.red = L.xs + (nsc * C::SCR * 4 + 15) / 16 * 16;
+  L.part = L.red + gd::kWarps * Tw * 16 * C::MT * 8 * 4;
+  L.total = L.part + (S > 1 ? S * NB * chunk * 4 : 0);
+  return L;
+}
+
+// -(bit q + 4i of w), i = 0..3, as int8 bytes; q in 0..7 (4..7: upper half).
+template <int Q>
+__device__ __forceinline__ uint32_t sign_bytes(uint32_t w) {
+  if constexpr (Q == 0) return prmt(0xFF00FF00u, 0xFF00FF00u, w);
+  else if constexpr (Q == 1) return prmt(0xFFFF0000u, 0xFFFF0000u, w);
+  else if constexpr (Q == 2) return prmt(0x00000000u, 0xFFFFFFFFu, w);
+  else if constexpr (Q == 3) return prmt(0xFF00FF00u, 0xFF00FF00u, w >> 3);
+  else if constexpr (Q == 4) return prmt(0xFF00FF00u, 0xFF00FF00u, w >> 16);
+  else if constexpr (Q == 5) return prmt(0xFFFF0000u, 0xFFFF0000u, w >> 16);
+  else if constexpr (Q == 6) return prmt(0x00000000u, 0xFFFFFFFFu, w >> 16);
+  else return prmt(0xFF00FF00u, 0xFF00FF00u, w >> 19);
+}
+
+__device__ __forceinline__ void mma_s8(int (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+  asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gsrc) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void st_dsmem_f32(uint32_t addr, float v) {
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
+
+// Quantise one 16-element activation item and store its digit words and
+// (lane 0 of the item) the fold factors.  `v` holds x[k0 .. k0+15].
+template <int NB>
+__device__ __forceinline__ void quantise_item(const float (&v)[16], bool valid, int it, uint32_t* scr) {
+  using C = gd::Cfg<NB>;
+  float mx = 0.f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) mx = fmaxf(mx, fabsf(v[i]));
+  mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 1));
+  mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 2));
+  mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 4));
+  int E = 0;
+  if (mx > 0.f) frexpf(mx, &E);  // mx = f 2^E, f in [0.5, 1): |x 2^(22-E)| < 2^22
+  const int sf = 22 - E, sf1 = sf / 2, sf2 = sf - sf1;
+  const float m1 = __uint_as_float(static_cast<uint32_t>(sf1 + 127) << 23);
+  const float m2 = __uint_as_float(static_cast<uint32_t>(sf2 + 127) << 23);
+  uint32_t e[16];
+  uint32_t bsum = 0;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    // 0x4B400000 + round(x 2^sf): exact rounding to an integer for |x 2^sf| < 2^22
+    const uint32_t bits = __float_as_uint(fmaf(v[i] * m1, m2, 12582912.0f));
+    bsum += bits;
+    e[i] = (bits - 0x4ABF7F80u) ^ 0x00808080u;  // bytes: signed digits lo, mid, hi
+  }
+  int xs = static_cast<int>(bsum - 16u * 0x4B400000u);
+  xs += __shfl_xor_sync(0xFFFFFFFFu, xs, 1);
+  xs += __shfl_xor_sync(0xFFFFFFFFu, xs, 2);
+  xs += __shfl_xor_sync(0xFFFFFFFFu, xs, 4);
+  if (!valid) return;
+  const int sub = it & 7, wi = sub >> 1, hh = sub & 1, gb = it >> 3;
+  const int r0 = 3 * gb;  // digit rows r0 (hi), r0+1 (mid), r0+2 (lo)
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    // elements q, q+4, q+8, q+12 are bits q + 4i + 16 hh of word wi
+    const uint32_t e0 = e[q], e1 = e[q + 4], e2 = e[q + 8], e3 = e[q + 12];
+    const uint32_t p01 = prmt(e0, e1, 0x5140u), p23 = prmt(e2, e3, 0x5140u);
+    const uint32_t dlo = prmt(p01, p23, 0x5410u);
+    const uint32_t dmid = prmt(p01, p23, 0x7632u);
+    const uint32_t dhi = prmt(prmt(e0, e1, 0x0062u), prmt(e2, e3, 0x0062u), 0x5410u);
+    const int off = wi * 8 + q * 2 + hh;
+    scr[(r0 + 0) * gd::kDigitStride + off] = dhi;
+    scr[(r0 + 1) * gd::kDigitStride + off] = dmid;
+    scr[(r0 + 2) * gd::kDigitStride + off] = dlo;
+  }
+  if (sub == 0) {
+    const float f = ldexpf(1.0f, E - 22);
+    float* fw = reinterpret_cast<float*>(scr + C::ROWS * gd::kDigitStride);
+    float* cx = fw + C::ROWS;
+    fw[r0 + 0] = f * 131072.0f;
+    fw[r0 + 1] = f * 512.0f;
+    fw[r0 + 2] = f * 2.0f;
+    cx[r0 + 0] = f * static_cast<float>(xs);
+    cx[r0 + 1] = 0.f;
+    cx[r0 + 2] = 0.f;
+  }
+}
+
+// One warp's products over its n-tiles (TW of them, a compile-time count so that
+// no MMA sits under a per-tile branch) and its sets; returns the fp32 partial
+// sums in acc[t][mt][e] (C-fragment order: rows 16mt + 8(e>>1) + lane/4, weight
+// rows 2(lane&3) + (e&1) of n-tile t).
+template <int NB, int TW>
+__device__ __forceinline__ void gd_compute(const unsigned char* wts, int P, const float* scl, int sstride,
+                                           const uint32_t* xs, int nsw, int lane,
+                                           float (&acc)[gd::kMaxTw][gd::Cfg<NB>::MT][4]) {
+  using C = gd::Cfg<NB>;
+  constexpr int G = C::G, MT = C::MT;
+  const int r1 = lane >> 2, cq = lane & 3;
+  // per-lane constants: A-fragment sources and fold rows
+  int abase[MT][2], sbase[MT][2];
+  bool aact[MT][2], rval[MT][2];
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {
+      const int r = 16 * mt + 8 * hf + r1;
+      const int rg = r / (3 * NB);
+      rval[mt][hf] = r < C::ROWS;
+      aact[mt][hf] = rval[mt][hf] && rg == (cq * G) / 4;
+      abase[mt][hf] = r * gd::kDigitStride + ((cq * G) & 3) * 8;
+      sbase[mt][hf] = (rval[mt][hf] ? rg : 0) * sstride + 2 * cq;
+    }
+  const unsigned char* wrow = wts + r1 * P + cq * 4 * G;
+  for (int si = 0; si < nsw; ++si) {
+    const uint32_t* scr = xs + si * C::SCR;
+    const float* fwv = reinterpret_cast<const float*>(scr + C::ROWS * gd::kDigitStride);
+    float fw[MT][2], cx[MT][2];
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        const int r = 16 * mt + 8 * hf + r1;
+        fw[mt][hf] = rval[mt][hf] ? fwv[r] : 0.f;
+        cx[mt][hf] = rval[mt][hf] ? fwv[C::ROWS + r] : 0.f;
+      }
+    // sign words: lane (r1, cq) takes G words of row r1 of each n-tile
+    uint32_t W[TW][G];
+#pragma unroll
+    for (int t = 0; t < TW; ++t) {
+      const unsigned char* src = wrow + t * 8 * P + si * 16 * G;
+      if constexpr (G == 4) {
+        const uint4 u = *reinterpret_cast<const uint4*>(src);
+        W[t][0] = u.x; W[t][G > 1 ? 1 : 0] = u.y; W[t][G > 2 ? 2 : 0] = u.z; W[t][G > 3 ? 3 : 0] = u.w;
+      } else if constexpr (G == 2) {
+        const uint2 u = *reinterpret_cast<const uint2*>(src);
+        W[t][0] = u.x; W[t][G > 1 ? 1 : 0] = u.y;
+      } else {
+        W[t][0] = *reinterpret_cast<const uint32_t*>(src);
+      }
+    }
+    int Cacc[TW][MT][4];
+#pragma unroll
+    for (int t = 0; t < TW; ++t)
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) Cacc[t][mt][e] = 0;
+#pragma unroll
+    for (int w = 0; w < G; ++w) {
+      auto step = [&](auto qc) {
+        constexpr int qq = decltype(qc)::value;
+        uint32_t A[MT][4];
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf) {
+            uint2 u = make_uint2(0, 0);
+            if (aact[mt][hf]) u = *reinterpret_cast<const uint2*>(scr + abase[mt][hf] + w * 8 + qq * 2);
+            A[mt][hf] = u.x;
+            A[mt][2 + hf] = u.y;
+          }
+#pragma unroll
+        for (int t = 0; t < TW; ++t) {
+          const uint32_t b0 = sign_bytes<qq>(W[t][w]);
+          const uint32_t b1 = sign_bytes<qq + 4>(W[t][w]);
+#pragma unroll
+          for (int mt = 0; mt < MT; ++mt) mma_s8(Cacc[t][mt], A[mt], b0, b1);
+        }
+      };
+      step(std::integral_constant<int, 0>{});
+      step(std::integral_constant<int, 1>{});
+      step(std::integral_constant<int, 2>{});
+      step(std::integral_constant<int, 3>{});
+    }
+    // fold: acc += s[n, group of row] * (f W_p D + [hi] f X)
+    const float* sset = scl + si * G * sstride;
+#pragma unroll
+    for (int t = 0; t < TW; ++t)
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          if (rval[mt][hf]) {
+            const float2 sv = *reinterpret_cast<const float2*>(sset + sbase[mt][hf] + t * 8);
+            acc[t][mt][2 * hf + 0] =
+                fmaf(sv.x, fmaf(fw[mt][hf], static_cast<float>(Cacc[t][mt][2 * hf + 0]), cx[mt][hf]),
+                     acc[t][mt][2 * hf + 0]);
+            acc[t][mt][2 * hf + 1] =
+                fmaf(sv.y, fmaf(fw[mt][hf], static_cast<float>(Cacc[t][mt][2 * hf + 1]), cx[mt][hf]),
+                     acc[t][mt][2 * hf + 1]);
+          }
+        }
+  }
+}
+
+template <int NB>
+__global__ void __launch_bounds__(gd::kThreads, 1) gemv_direct_kernel(const GdParams p) {
+  using C = gd::Cfg<NB>;
+  constexpr int G = C::G, MT = C::MT;
+  extern __shared__ __align__(16) unsigned char smem[];
+  const int NS = (p.NG + G - 1) / G;
+  const int crank = p.S > 1 ? static_cast<int>(cluster_ctarank()) : 0;
+  const int cs0 = (crank * NS) >> p.lgS, nsc = (((crank + 1) * NS) >> p.lgS) - cs0;
+  const GdSmem L = gd_layout<NB>(p.Tw, p.NSw, p.P, p.S, p.chunk, p.NSc);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  unsigned char* wreg = smem + warp * L.warp_bytes;
+  unsigned char* wts = wreg + L.wts;
+  float* scl = reinterpret_cast<float*>(wreg + L.scl);
+  uint32_t* xs = reinterpret_cast<uint32_t*>(smem + L.xs);
+
+  if (p.S > 1) cluster_arrive_relaxed();  // matched by the wait before the first remote store
+
+  // ---- this CTA: cluster q's n-tiles, K sets [cs0, cs0 + nsc); this warp: a block of both
+  const int q = p.S > 1 ? static_cast<int>(cluster_id_x()) : static_cast<int>(blockIdx.x);
+  const int t0c = q * p.tq + min(q, p.tr);              // NT = Q * tq + tr tiles, the first tr clusters one more
+  const int Tq = p.tq + (q < p.tr ? 1 : 0);
+  const int wn = warp >> p.lgWg, wg = warp & (p.Wg - 1);
+  const int tw = max(0, min(p.Tw, Tq - wn * p.Tw));        // n-tiles of this warp
+  const int ws0 = cs0 + ((wg * nsc) >> p.lgWg);             // first set of this warp
+  const int nsw = cs0 + (((wg + 1) * nsc) >> p.lgWg) - ws0;  // sets of this warp
+  const int row0 = (t0c + wn * p.Tw) * 8;                   // first weight row of this warp
+  const int nrows = max(0, min(8 * tw, p.N - row0));
+  const bool busy = tw > 0 && nsw > 0;
+  const int g0 = ws0 * G;                                    // first group of this warp
+  const int ngw = busy ? min(nsw * G, p.NG - g0) : 0;       // real groups of this warp
+  const int KW = p.K >> 5;                                   // words per weight row
+  const int lgw = p.lgGw, gmask = (1 << lgw) - 1;           // power-of-two stride over a row's groups
+
+  // ---- weight staging: 16-byte asynchronous copies, every lane, all up front
+  auto stage_weights = [&]() {
+    const int n = nrows << lgw;
+    for (int i = lane; i < n; i += 32) {
+      const int r = i >> lgw, g = i & gmask;
+      if (g < ngw)
+        cp_async16(wts + r * p.P + g * 16, p.signs + static_cast<int64_t>(row0 + r) * KW + 4 * (g0 + g));
+    }
+    cp_async_commit();
+  };
+  // ---- scales: plain loads now, converted and stored once the activations are in flight
+  constexpr int kSpl = 8;
+  const int sstride = 8 * p.Tw;                  // scl[group][row]
+  const int nscl = busy ? (8 * tw) << lgw : 0;   // rows x (power-of-two) groups
+  uint16_t sreg[kSpl];
+  auto load_scales = [&](int base) {
+#pragma unroll
+    for (int j = 0; j < kSpl; ++j) {
+      const int i = base + lane + 32 * j;
+      const int rl = i >> lgw, gl = i & gmask;
+      sreg[j] = 0;
+      if (i < nscl && gl < nsw * G && row0 + rl < p.N && g0 + gl < p.NG)
+        sreg[j] = __ldg(p.scales + static_cast<int64_t>(row0 + rl) * p.NG + g0 + gl);
+    }
+  };
+  auto store_scales = [&](int base) {
+#pragma unroll
+    for (int j = 0; j < kSpl; ++j) {
+      const int i = base + lane + 32 * j;
+      const int rl = i >> lgw, gl = i & gmask;
+      if (i < nscl && gl < nsw * G) scl[gl * sstride + rl] = __half2float(__ushort_as_half(sreg[j]));
+    }
+  };
+
+  if (p.early) {
+    stage_weights();
+    load_scales(0);
+  }
+  pdl_wait();
+  pdl_launch_dependents();
+  if (!p.early) {
+    stage_weights();
+    load_scales(0);
+  }
+
+  // ---- activations of the CTA's sets -> digit scratch.  Unit = (set, group j,
+  // batch b): 8 lanes x 16 elements; 32 units per pass of the CTA.
+  {
+    const int units = nsc * G * NB;
+    const int sub = lane & 7;
+    auto load_unit = [&](int u, uint4 (&r)[2]) {  // unit u of this CTA -> 16 bf16 of this lane
+      r[0] = make_uint4(0, 0, 0, 0);
+      r[1] = make_uint4(0, 0, 0, 0);
+      if (u < units) {
+        const int sl = u / (G * NB), gb = u - sl * (G * NB);
+        const int gj = gb / NB, b = gb - gj * NB;
+        const int g = (cs0 + sl) * G + gj;
+        if (g < p.NG) {
+          const uint4* src =
+              reinterpret_cast<const uint4*>(p.x + static_cast<int64_t>(b) * p.K + g * 128 + sub * 16);
+          r[0] = __ldg(src);
+          r[1] = __ldg(src + 1);
+        }
+      }
+    };
+    auto process = [&](const uint4 (&r)[2], int u) {
+      const uint32_t w[8] = {r[0].x, r[0].y, r[0].z, r[0].w, r[1].x, r[1].y, r[1].z, r[1].w};
+      float v[16];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        v[2 * i] = __uint_as_float(w[i] << 16);
+        v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+      }
+      const int sl = u / (G * NB);
+      const int it = (u - sl * (G * NB)) * 8 + sub;  // item index within the set
+      quantise_item<NB>(v, u < units, it, xs + sl * C::SCR);
+    };
+    // two passes per iteration: the loads of one pass overlap the other's math
+    const int u0 = warp * 4 + (lane >> 3);
+    uint4 xa[2], xb[2];
+    load_unit(u0, xa);
+    for (int u = u0; u - u0 < units; u += 64) {  // trip count uniform over the CTA
+      load_unit(u + 32, xb);
+      process(xa, u);
+      if (u - u0 + 32 >= units) break;
+      load_unit(u + 64, xa);
+      process(xb, u + 32);
+    }
+  }
+  if (busy) {
+    store_scales(0);
+    for (int base = 32 * kSpl; base < nscl; base += 32 * kSpl) {  // long K ranges
+      load_scales(base);
+      store_scales(base);
+    }
+  }
+  cp_async_wait_all();
+  __syncthreads();
+
+  float acc[gd::kMaxTw][MT][4];
+#pragma unroll
+  for (int t = 0; t < gd::kMaxTw; ++t)
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[t][mt][e] = 0.f;
+  if (busy) {
+    const uint32_t* xw = xs + (ws0 - cs0) * C::SCR;
+    switch (tw) {  // warp-uniform
+      case 1: gd_compute<NB, 1>(wts, p.P, scl, sstride, xw, nsw, lane, acc); break;
+      case 2: gd_compute<NB, 2>(wts, p.P, scl, sstride, xw, nsw, lane, acc); break;
+      case 3: gd_compute<NB, 3>(wts, p.P, scl, sstride, xw, nsw, lane, acc); break;
+      default: gd_compute<NB, 4>(wts, p.P, scl, sstride, xw, nsw, lane, acc); break;
+    }
+  }
+
+  // ---- CTA reduction: red[wg][tile][row r][n], tile = wn * Tw + t (CTA-local)
+  const int r1 = lane >> 2, cq = lane & 3;
+  float* red = reinterpret_cast<float*>(smem + L.red);
+  const int TT = p.Wn * p.Tw;  // tiles per CTA (max)
+#pragma unroll
+  for (int t = 0; t < gd::kMaxTw; ++t) {
+    if (t < tw) {
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          const int r = 16 * mt + 8 * hf + r1;
+          *reinterpret_cast<float2*>(red + ((wg * TT + wn * p.Tw + t) * 16 * MT + r) * 8 + 2 * cq) =
+              make_float2(acc[t][mt][2 * hf], acc[t][mt][2 * hf + 1]);
+        }
+    }
+  }
+  __syncthreads();
+  // per (b, row of this cluster): sum over the warps of the same tile (set
+  // blocks, fixed order) and over the digit rows of batch b; then to the owning
+  // CTA (or straight to y when S = 1).  Warps with no sets wrote nothing: skip.
+  const int R8 = 8 * Tq;
+  float* part = reinterpret_cast<float*>(smem + L.part);
+  if (p.S > 1) cluster_wait();  // every CTA of the cluster has started
+  for (int b = 0; b < NB; ++b) {
+    for (int rl = threadIdx.x; rl < R8; rl += gd::kThreads) {
+      const int tile = rl >> 3, n = rl & 7;
+      float sum = 0.f;
+      for (int g2 = 0; g2 < p.Wg; ++g2) {
+        const int s0 = cs0 + ((g2 * nsc) >> p.lgWg), s1 = cs0 + (((g2 + 1) * nsc) >> p.lgWg);
+        if (s1 <= s0) continue;
+        const float* rp = red + ((g2 * TT + tile) * 16 * MT) * 8 + n;
+#pragma unroll
+        for (int gj = 0; gj < G; ++gj)
+#pragma unroll
+          for (int pp = 0; pp < 3; ++pp) sum += rp[((gj * NB + b) * 3 + pp) * 8];
+      }
+      const int row = t0c * 8 + rl;
+      if (p.S == 1) {
+        if (row < p.N) p.y[static_cast<int64_t>(b) * p.N + row] = sum;
+      } else {
+        int owner = 0;
+        while (owner + 1 < p.S && rl >= (owner + 1) * p.chunk) ++owner;
+        const uint32_t local = smem_u32(part + (crank * NB + b) * p.chunk + (rl - owner * p.chunk));
+        st_dsmem_f32(map_shared_rank(local, static_cast<uint32_t>(owner)), sum);
+      }
+    }
+  }
+  if (p.S > 1) {
+    cluster_sync();
+    const int lo = crank * p.chunk, hi = min(R8, lo + p.chunk);
+    for (int b = 0; b < NB; ++b) {
+      for (int ro = threadIdx.x; ro < hi - lo; ro += gd::kThreads) {
+        float sum = 0.f;
+        for (int c = 0; c < p.S; ++c) sum += part[(c * NB + b) * p.chunk + ro];
+        const int row = t0c * 8 + lo + ro;
+        if (row < p.N) p.y[static_cast<int64_t>(b) * p.N + row] = sum;
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------------ host side
+
+template <int NB>
+static int gd_max_clusters(int S, int smem_bytes) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(S * 64));
+  cfg.blockDim = dim3(gd::kThreads);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem_bytes);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(S);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = S > 1 ? 1 : 0;
+  int n = 0;
+  if (cudaFuncSetAttribute(gemv_direct_kernel<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  if (S > 1) {
+    if (cudaOccupancyMaxActiveClusters(&n, gemv_direct_kernel<NB>, &cfg) != cudaSuccess) {
+      cudaGetLastError();
+      return 0;
+    }
+    return n;
+  }
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, gemv_direct_kernel<NB>, gd::kThreads, smem_bytes) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  return n;  // per SM
+}
+
+struct GdPlan {
+  int S, Q, Wn, Wg, Tw, NSw, NSc, P, chunk, smem;
+  double cost;
+};
+
+// Instruction-count model per SM (lane instructions / 128 per clock):
+// activation quantisation ~24 per element of the CTA's K range (its chain is
+// latency-bound; fitted to measured K splits), weights ~c_w
+// per weight, CTAs per SM rounded up, plus a fixed charge for a cluster
+// barrier.
+template <int NB>
+static bool gd_plan_for(int N, int NG, int S, int num_sms, int smem_cap, GdPlan* out) {
+  using C = gd::Cfg<NB>;
+  const int NT = (N + 7) / 8;
+  const int NS = (NG + C::G - 1) / C::G;
+  if (S > 1 && S > NS) return false;
+  const int nsc = (NS + S - 1) / S;
+  if (nsc > gd::kMaxSets) return false;
+  int Q = std::max(1, std::min(NT, num_sms / S));
+  for (int iter = 0; iter < 8; ++iter) {
+    const int Tmax = (NT + Q - 1) / Q;
+    int Wn = 0;
+    for (int w = 1; w <= 8; w *= 2)
+      if ((Tmax + w - 1) / w <= gd::kMaxTw) {
+        Wn = w;
+        break;
+      }
+    if (Wn == 0) {  // more rows per cluster than 8 warps x 4 n-tiles: more clusters
+      Q = (NT + 8 * gd::kMaxTw - 1) / (8 * gd::kMaxTw);
+      continue;
+    }
+    const int Wg = 8 / Wn;
+    const int Tw = (Tmax + Wn - 1) / Wn;
+    const int NSw = (nsc + Wg - 1) / Wg;
+    const int span = NSw * 16 * C::G;
+    const int P = ((span / (16 * C::G)) & 1) ? span : span + 16 * C::G;  // odd multiple: bank spread
+    const int chunk = (8 * Tmax + S - 1) / S;
+    const GdSmem L = gd_layout<NB>(Tw, NSw, P, S, chunk, nsc);
+    if (L.total > smem_cap) {
+      if (Q >= NT) return false;
+      Q = std::min(NT, Q * 2);  // fewer rows per CTA
+      continue;
+    }
+    const int occ = gd_max_clusters<NB>(S, L.total);
+    if (occ <= 0) return false;
+    const double cw = NB <= 2 ? 0.6 : (NB <= 5 ? 1.0 : 1.5);
+    const double xprep = 24.0 * NB * 128.0 * C::G * nsc;          // per CTA
+    const double wts = 8.0 * Tmax * 128.0 * C::G * nsc * cw;      // per CTA
+    const double ctas_per_sm = std::ceil(static_cast<double>(Q) * S / num_sms);
+    const double cost = (xprep + wts) / 128.0 * ctas_per_sm + (S > 1 ? 800.0 : 0.0);
+    *out = GdPlan{S, Q, Wn, Wg, Tw, NSw, nsc, P, chunk, L.total, cost};
+    return true;
+  }
+  return false;
+}
+
+struct GdPlanEntry {
+  int N, NG, NB, sms, dev, force;
+  bool ok;
+  GdPlan plan;
+};
+static GdPlanEntry g_gd_cache[64];
+static int g_gd_count = 0;
+static std::mutex g_gd_mu;
+
+template <int NB>
+static bool gd_cached_plan(int N, int NG, int num_sms, int smem_cap, GdPlan* out) {
+  int force = 0;
+  if (const char* f = getenv("W1_GEMV_SPLIT")) force = atoi(f);  // tuning knob: force the K split
+  if (force != 1 && force != 2 && force != 4 && force != 8) force = 0;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  {
+    std::lock_guard<std::mutex> lock(g_gd_mu);
+    for (int i = 0; i < g_gd_count; ++i) {
+      const GdPlanEntry& e = g_gd_cache[i];
+      if (e.N == N && e.NG == NG && e.NB == NB && e.sms == num_sms && e.dev == dev && e.force == force) {
+        *out = e.plan;
+        return e.ok;
+      }
+    }
+  }
+  GdPlan best = {};
+  bool ok = false;
+  for (int S = 1; S <= 8; S *= 2) {
+    if (force && S != force) continue;
+    GdPlan pl;
+    if (gd_plan_for<NB>(N, NG, S, num_sms, smem_cap, &pl) && (!ok || pl.cost < best.cost)) {
+      best = pl;
+      ok = true;
+    }
+  }
+  std::lock_guard<std::mutex> lock(g_gd_mu);
+  const int i = g_gd_count < 64 ? g_gd_count++ : (N + NG + NB) & 63;
+  g_gd_cache[i] = GdPlanEntry{N, NG, NB, num_sms, dev, force, ok, best};
+  *out = best;
+  return ok;
+}
+
+template <int NB>
+static cudaError_t launch_gemv_direct_nb(const GdParams& base, cudaStream_t stream, int num_sms, int smem_cap) {
+  GdPlan plan;
+  if (!gd_cached_plan<NB>(base.N, base.NG, num_sms, smem_cap, &plan)) return cudaErrorNotSupported;
+  if (getenv("W1_VERBOSE"))
+    fprintf(stderr,
+            "w1_gemv(direct) plan: N=%d NG=%d B=%d -> clusters=%d split=%d warps=%dx%d tiles/warp=%d "
+            "sets/warp=%d smem=%d\n",
+            base.N, base.NG, NB, plan.Q, plan.S, plan.Wn, plan.Wg, plan.Tw, plan.NSw, plan.smem);
+
+  GdParams p = base;
+  p.S = plan.S;
+  p.Q = plan.Q;
+  p.NT = (base.N + 7) / 8;
+  p.Wn = plan.Wn;
+  p.Wg = plan.Wg;
+  p.Tw = plan.Tw;
+  p.NSw = plan.NSw;
+  p.P = plan.P;
+  p.chunk = plan.chunk;
+  p.NSc = plan.NSc;
+  auto lg2 = [](int v) {
+    int l = 0;
+    while ((1 << l) < v) ++l;
+    return l;
+  };
+  p.lgS = lg2(plan.S);
+  p.lgWg = lg2(plan.Wg);
+  p.lgGw = lg2(plan.NSw * gd::Cfg<NB>::G);
+  p.tq = p.NT / plan.Q;
+  p.tr = p.NT - p.tq * plan.Q;
+  cudaError_t err =
+      cudaFuncSetAttribute(gemv_direct_kernel<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize, plan.smem);
+  if (err != cudaSuccess) return err;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(plan.Q * plan.S));
+  cfg.blockDim = dim3(gd::kThreads);
+  cfg.dynamicSmemBytes = static_cast<size_t>(plan.smem);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[na].val.programmaticStreamSerializationAllowed = 1;
+  ++na;
+  if (plan.S > 1) {
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = static_cast<unsigned>(plan.S);
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = na;
+  return cudaLaunchKernelEx(&cfg, gemv_direct_kernel<NB>, p);
+}
+
+// Returns cudaErrorNotSupported when the shape is outside this kernel's plan.
+cudaError_t launch_gemv_direct(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t K,
+                               const uint16_t* x, int B, float* y, bool static_weights, cudaStream_t stream,
+                               int num_sms, int smem_cap) {
+  if (N > (int64_t)1 << 30 || K > (int64_t)1 << 30) return cudaErrorNotSupported;
+  GdParams p = {};
+  p.signs = signs;
+  p.scales = scales;
+  p.x = x;
+  p.y = y;
+  p.N = static_cast<int>(N);
+  p.K = static_cast<int>(K);
+  p.NG = static_cast<int>(K / 128);
+  p.early = static_weights ? 1 : 0;
+  switch (B) {
+    case 1: return launch_gemv_direct_nb<1>(p, stream, num_sms, smem_cap);
+    case 2: return launch_gemv_direct_nb<2>(p, stream, num_sms, smem_cap);
+    case 3: return launch_gemv_direct_nb<3>(p, stream, num_sms, smem_cap);
+    case 4: return launch_gemv_direct_nb<4>(p, stream, num_sms, smem_cap);
+    case 5: return launch_gemv_direct_nb<5>(p, stream, num_sms, smem_cap);
+    case 6: return launch_gemv_direct_nb<6>(p, stream, num_sms, smem_cap);
+    case 7: return launch_gemv_direct_nb<7>(p, stream, num_sms, smem_cap);
+    default: return launch_gemv_direct_nb<8>(p, stream, num_sms, smem_cap);
+  }
+}
+
+}  // namespace w1

@@ -3,6 +3,8 @@
 #include "w1_api.cu"
 #include "pack.cu"
 #include "gemv.cu"
+#include "gemv_tc.cu"
+#include "gemv_direct.cu"
 #include "gemm.cu"
 #include "dbf_tc.cu"
 #include "dbf.cu"

@@ -14,7 +14,7 @@ cudaError_t launch_pack(const float* W, int64_t N, int64_t K, uint32_t* signs, u
                         cudaStream_t stream, int num_sms);
 cudaError_t launch_gemv(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t K,
                         const uint16_t* x, int B, float* y, cudaStream_t stream, int num_sms,
-                        int smem_cap);
+                        int smem_cap, bool static_weights);
 cudaError_t launch_gemm(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t K,
                         const uint16_t* x, int64_t M, float* y, cudaStream_t stream, int num_sms);
 
@@ -59,6 +59,10 @@ static int device_info(DeviceInfo* out) {
 static inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 static inline int launch_result(cudaError_t e) {
+  if (e == cudaErrorNotSupported) {
+    cudaGetLastError();
+    return W1_ERR_UNSUPPORTED;
+  }
   if (e == cudaSuccess) e = cudaGetLastError();
   return e == cudaSuccess ? W1_OK : W1_ERR_CUDA;
 }
@@ -106,18 +110,25 @@ int w1_pack(const float* W, int64_t N, int64_t K, uint32_t* signs, uint16_t* sca
   return launch_result(launch_pack(W, N, K, signs, scales, reinterpret_cast<cudaStream_t>(stream), d.sms));
 }
 
-int w1_gemv(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t K,
-            const uint16_t* x, int64_t B, float* y, w1_stream_t stream) {
+int w1_gemv_ex(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t K,
+               const uint16_t* x, int64_t B, float* y, uint32_t flags, w1_stream_t stream) {
   if (!signs || !scales || !x || !y) return W1_ERR_NULL;
   if (N <= 0 || K <= 0 || (K % 128) != 0 || B < 1 || B > 8) return W1_ERR_SHAPE;
   if (K / 128 > (int64_t)1 << 20 || N > ((int64_t)1 << 40)) return W1_ERR_SHAPE;
+  if ((flags & ~static_cast<uint32_t>(W1_GEMV_STATIC_WEIGHTS)) != 0) return W1_ERR_SHAPE;
   if (!aligned16(signs) || !aligned16(scales) || !aligned16(x) || !aligned16(y)) return W1_ERR_ALIGN;
   DeviceInfo d;
   int st = device_info(&d);
   if (st != W1_OK) return st;
   const int cap = d.smem_optin < 110 * 1024 ? d.smem_optin : 110 * 1024;
   return launch_result(launch_gemv(signs, scales, N, K, x, static_cast<int>(B), y,
-                                   reinterpret_cast<cudaStream_t>(stream), d.sms, cap));
+                                   reinterpret_cast<cudaStream_t>(stream), d.sms, cap,
+                                   (flags & W1_GEMV_STATIC_WEIGHTS) != 0));
+}
+
+int w1_gemv(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t K,
+            const uint16_t* x, int64_t B, float* y, w1_stream_t stream) {
+  return w1_gemv_ex(signs, scales, N, K, x, B, y, 0u, stream);
 }
 
 int w1_gemm(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t K,

@@ -49,9 +49,16 @@ def w1_pack(W: torch.Tensor, signs: torch.Tensor | None = None, scales: torch.Te
     return signs, scales
 
 
+W1_GEMV_STATIC_WEIGHTS = 1
+
+
 def w1_gemv(signs: torch.Tensor, scales: torch.Tensor, x: torch.Tensor, y: torch.Tensor | None = None,
-            stream=None) -> torch.Tensor:
-    """y [B, N] fp32 = x [B, K] bf16 times the 1-bit matrix (B <= 8)."""
+            stream=None, static_weights: bool = False) -> torch.Tensor:
+    """y [B, N] fp32 = x [B, K] bf16 times the 1-bit matrix (B <= 8).
+
+    static_weights=True calls w1_gemv_ex with W1_GEMV_STATIC_WEIGHTS: the
+    weights must not have been written by the kernel just before on the stream.
+    """
     N = signs.shape[0]
     K = signs.shape[1] * 32
     B = x.shape[0]
@@ -59,7 +66,11 @@ def w1_gemv(signs: torch.Tensor, scales: torch.Tensor, x: torch.Tensor, y: torch
         raise TypeError("x must be bfloat16")
     if y is None:
         y = torch.empty((B, N), dtype=torch.float32, device=x.device)
-    st = _lib.call("w1_gemv", _ptr(signs), _ptr(scales), N, K, _ptr(x), B, _ptr(y), _stream(stream))
+    if static_weights:
+        st = _lib.call("w1_gemv_ex", _ptr(signs), _ptr(scales), N, K, _ptr(x), B, _ptr(y),
+                       W1_GEMV_STATIC_WEIGHTS, _stream(stream))
+    else:
+        st = _lib.call("w1_gemv", _ptr(signs), _ptr(scales), N, K, _ptr(x), B, _ptr(y), _stream(stream))
     _lib.check(st, "w1_gemv")
     return y
 

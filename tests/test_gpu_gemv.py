@@ -1,4 +1,8 @@
-"""w1_gemv on the GPU vs the fp64 oracle (element-wise, 1e-3 * sum|s x| bound)."""
+"""w1_gemv on the GPU vs the fp64 oracle (element-wise, 1e-3 * sum|s x| bound).
+
+Every test runs on each of the three kernels: the direct kernel
+(W1_GEMV_PATH=direct, the default wherever its plan fits), the tcgen05 kernel
+(=tc) and the mma.sync ring kernel (=mma, the fallback for other shapes)."""
 import functools
 
 import numpy as np
@@ -10,6 +14,12 @@ from pack_sign_g128_b200 import ops, synth, _lib
 from gpu_helpers import assert_within, bf16_dev, fp16_dev, words_dev
 
 pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True, params=["direct", "tc", "mma"])
+def gemv_path(request, monkeypatch):
+    monkeypatch.setenv("W1_GEMV_PATH", request.param)
+    return request.param
 
 
 @functools.lru_cache(maxsize=None)
@@ -96,3 +106,33 @@ def test_gemv_is_deterministic():
     a = run_gemv(s, c, x)
     b = run_gemv(s, c, x)
     assert np.array_equal(a, b)
+
+
+@pytest.mark.parametrize("split", ["1", "2", "4", "8"])
+@pytest.mark.parametrize("N,K,B", [(4096, 4096, 1), (1000, 1152, 5), (4097, 2176, 8), (300, 1024, 2)])
+def test_gemv_direct_every_split(N, K, B, split, gemv_path, monkeypatch):
+    """The direct kernel's cluster K split (1..8 CTAs) on the same inputs."""
+    if gemv_path != "direct":
+        pytest.skip("split sweep is for the direct kernel")
+    monkeypatch.setenv("W1_GEMV_SPLIT", split)
+    W, x = synth.gemv_case(N, K, B, seed=N + B)
+    s, c = O.pack_ref_fast(W)
+    try:
+        check(s, c, x, K, f"{N}x{K} B={B} split={split}")
+    except _lib.W1Error as e:
+        if e.status != _lib.W1_ERR_UNSUPPORTED:
+            raise
+        pytest.skip(f"split {split} does not fit {N}x{K}")
+
+
+def test_gemv_static_weights_flag_same_result(gemv_path):
+    """W1_GEMV_STATIC_WEIGHTS changes only when the weights are read: the
+    weights here were written long before, so results are identical."""
+    s, c = packed_case(4096, 4096, synth.SEEDS["gemv"])
+    x = bf16_dev(synth.activations_bf16(synth.rng(65), 4, 4096))
+    sd, cd = words_dev(s), fp16_dev(c)
+    torch.cuda.synchronize()
+    a = ops.w1_gemv(sd, cd, x)
+    b = ops.w1_gemv(sd, cd, x, static_weights=True)
+    assert ops.sync_status() == _lib.W1_OK
+    assert torch.equal(a, b)
