@@ -158,8 +158,19 @@ def sum_over_ranks(world, value: float) -> float:
 
 # ------------------------------------------------------------------ GPU arm
 
-def build_gemv_sweep(torch, ops, synth, l2_bytes: int):
-    """Packed weight copies + one CUDA graph of back-to-back launches per pair."""
+class EagerChain:
+    """Stands in for a captured graph: replay() issues the launches directly."""
+
+    def __init__(self, fn):
+        self.fn = fn
+
+    def replay(self):
+        self.fn()
+
+
+def build_gemv_sweep(torch, ops, synth, l2_bytes: int, eager: bool = False):
+    """Packed weight copies + one CUDA graph of back-to-back launches per pair
+    (eager=True: the same launches issued one by one, for ncu launch lists)."""
     dev = torch.device("cuda")
     stream = torch.cuda.Stream()
     combos = []
@@ -180,18 +191,23 @@ def build_gemv_sweep(torch, ops, synth, l2_bytes: int):
                 for r in range(3):
                     ops.w1_gemv(signs[r], scales[r], x, y)
             stream.synchronize()
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=stream):
+            def chain(static, signs=signs, scales=scales, x=x, y=y, R=R):
                 for r in range(R):
-                    ops.w1_gemv(signs[r], scales[r], x, y)
-            # the same chain with W1_GEMV_STATIC_WEIGHTS (weights written long before)
+                    ops.w1_gemv(signs[r], scales[r], x, y, static_weights=static)
             with torch.cuda.stream(stream):
                 ops.w1_gemv(signs[0], scales[0], x, y, static_weights=True)
             stream.synchronize()
-            gs = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(gs, stream=stream):
-                for r in range(R):
-                    ops.w1_gemv(signs[r], scales[r], x, y, static_weights=True)
+            if eager:
+                g = EagerChain(lambda c=chain: c(False))
+                gs = EagerChain(lambda c=chain: c(True))
+            else:
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=stream):
+                    chain(False)
+                # the same chain with W1_GEMV_STATIC_WEIGHTS (weights written long before)
+                gs = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(gs, stream=stream):
+                    chain(True)
             combos.append({"N": N, "K": K, "B": B, "R": R, "graph": g, "graph_static": gs, "x": x, "y": y,
                            "signs": signs, "scales": scales, "bytes": pb})
     torch.cuda.synchronize()
@@ -279,6 +295,19 @@ def gemv_e2e(torch, ops, combos, steps: int):
             "ms_per_step": ms / steps, "launches": launches}
 
 
+def gemv_one(torch, ops, synth, shape: str, launches: int = 4):
+    """A few eager launches of one GEMV (N, K, B): the small case for ncu."""
+    N, K, B = (int(v) for v in shape.split(","))
+    W, _ = synth.gemv_case(N, K, 1)
+    s, c = ops.w1_pack(torch.from_numpy(W).cuda())
+    x = torch.from_numpy(synth.activations_bf16(synth.rng(100 + B), B, K).view(np.int16)).cuda().view(torch.bfloat16)
+    y = torch.empty((B, N), dtype=torch.float32, device="cuda")
+    for _ in range(launches):
+        ops.w1_gemv(s, c, x, y)
+    torch.cuda.synchronize()
+    return {"N": N, "K": K, "B": B, "launches": launches}
+
+
 def gemm_rows(torch, ops, synth, peaks, iters: int = 8):
     dev = torch.device("cuda")
     flush = torch.empty(int(512 * 2 ** 20), dtype=torch.uint8, device=dev)
@@ -290,8 +319,9 @@ def gemm_rows(torch, ops, synth, peaks, iters: int = 8):
         del Wd
         xd = torch.from_numpy(x.view(np.int16)).to(dev).view(torch.bfloat16)
         y = torch.empty((GEMM_M, N), dtype=torch.float32, device=dev)
+        ws = ops.gemm_workspace(GEMM_M, K, device=dev)
         for _ in range(3):
-            ops.w1_gemm(s, c, xd, y)
+            ops.w1_gemm(s, c, xd, y, workspace=ws)
         torch.cuda.synchronize()
         times = []
         for _ in range(iters):
@@ -299,7 +329,7 @@ def gemm_rows(torch, ops, synth, peaks, iters: int = 8):
             a = torch.cuda.Event(enable_timing=True)
             b = torch.cuda.Event(enable_timing=True)
             a.record()
-            ops.w1_gemm(s, c, xd, y)
+            ops.w1_gemm(s, c, xd, y, workspace=ws)
             b.record()
             torch.cuda.synchronize()
             times.append(a.elapsed_time(b))
@@ -308,7 +338,7 @@ def gemm_rows(torch, ops, synth, peaks, iters: int = 8):
         tf = flops / (ms * 1e-3) / 1e12
         rows.append({"M": GEMM_M, "N": N, "K": K, "ms": ms, "TFLOP/s": tf,
                      "frac_bf16_burst": tf / peaks["bf16_tflops"]})
-        del s, c, xd, y
+        del s, c, xd, y, ws
     torch.cuda.synchronize()
     return rows
 
@@ -482,10 +512,12 @@ def run_gpu(args):
             rows["moe"] = moe_rows(torch, ops, synth, peaks)
         elif args.section == "dbf":
             rows["dbf"] = dbf_rows(torch, ops, synth, peaks, l2)
+        elif args.section == "gemv1":
+            rows["gemv1"] = gemv_one(torch, ops, synth, args.shape)
         if rank == 0:
             print(json.dumps({"section": args.section, "rows": rows}), flush=True)
         return
-    combos, stream = build_gemv_sweep(torch, ops, synth, l2)
+    combos, stream = build_gemv_sweep(torch, ops, synth, l2, eager=args.eager)
     launches_per_step = sum(cb["R"] for cb in combos)
     bytes_per_step = sum(cb["bytes"] * cb["R"] for cb in combos)
 
@@ -544,7 +576,8 @@ def run_gpu(args):
         "config": {"workload": WORKLOAD, "launches_per_step": launches_per_step,
                    "packed_bytes_per_step": bytes_per_step,
                    "l2": "inputs larger than L2: each pair cycles R weight copies totalling > 4x L2",
-                   "timing": "CUDA graphs of back-to-back launches, CUDA events on the launch stream",
+                   "timing": ("eager launches (profiling form)" if args.eager else
+                              "CUDA graphs of back-to-back launches") + ", CUDA events on the launch stream",
                    "parallelism": f"replicas x{world} (independent sweeps, no collective)"},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                      "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
@@ -631,7 +664,11 @@ def main():
     ap.add_argument("--impl", default="w1", choices=["w1", "reference"])
     ap.add_argument("--skip-extra", action="store_true", help="only the headline sweep")
     ap.add_argument("--skip-cpu", action="store_true", help="skip the CPU-oracle baseline")
-    ap.add_argument("--section", default="all", choices=["all", "gemm", "moe", "dbf"],
+    ap.add_argument("--eager", action="store_true",
+                    help="issue the sweep's launches one by one instead of CUDA graphs (for ncu launch lists)")
+    ap.add_argument("--shape", default="4096,4096,1",
+                    help="N,K,B of the single GEMV that --section gemv1 launches (for ncu captures)")
+    ap.add_argument("--section", default="all", choices=["all", "gemm", "moe", "dbf", "gemv1"],
                     help="run one row only (for profiling); prints a rows-only JSON line")
     args = ap.parse_args()
     if args.warmup < 3:

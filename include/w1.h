@@ -120,12 +120,23 @@ int w1_gemv_ex(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t
  * prompt processing amortises weight loads across columns).
  *   y[m][n] = sum_g s[n][g] * sum_{k in g} (1 - 2*bit[n][k]) * x[m][k].
  *   signs [N][K/32], scales [N][K/128], x bf16 [M][K], y fp32 [M][N] (device).
- * tcgen05 tensor cores: the sign bits are expanded to +-1 bf16 per 128-wide K
- * chunk, each chunk is accumulated exactly in TMEM (fp32) and folded into the
- * running sum with its group scale.  Same accuracy bound as w1_gemv.
+ * tcgen05 tensor cores.  x is first rewritten to fp16 with an exact
+ * power-of-two per token row (max |x| in [2^14, 2^15)); the weight operand is
+ * the group scale with the weight's sign bit (+-s, exact in fp16), so the
+ * blockwise scale is applied inside the MMA and all of K accumulates in one
+ * fp32 TMEM tile.  Same accuracy bound as w1_gemv.
+ * workspace: >= w1_gemm_workspace_size(M, K) bytes of device memory, 256-byte
+ *   aligned (the fp16 copy of x and the token scales); contents on entry are
+ *   ignored, nothing is carried between calls; calls sharing a workspace must
+ *   not overlap.  Too small / null: W1_ERR_WORKSPACE; misaligned: W1_ERR_ALIGN.
+ * Two kernels on `stream` (prep, GEMM).
  */
 int w1_gemm(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t K,
-            const uint16_t* x, int64_t M, float* y, w1_stream_t stream);
+            const uint16_t* x, int64_t M, float* y, void* workspace, size_t ws_bytes,
+            w1_stream_t stream);
+
+/* Bytes of workspace w1_gemm needs (0 for invalid sizes). */
+size_t w1_gemm_workspace_size(int64_t M, int64_t K);
 
 /*
  * w1_moe_grouped -- routed SwiGLU expert layer with 1-bit group-128 experts

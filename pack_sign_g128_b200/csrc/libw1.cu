@@ -5,6 +5,7 @@
 #include "gemv.cu"
 #include "gemv_tc.cu"
 #include "gemv_direct.cu"
+#include "sign_gemm.cu"
 #include "gemm.cu"
 #include "dbf_tc.cu"
 #include "dbf.cu"

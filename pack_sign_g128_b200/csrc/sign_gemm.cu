@@ -1,0 +1,378 @@
+// Tensor-core product of 1-bit weight rows with many token rows (tcgen05),
+// shared by w1_gemm (group-128 scales) and the DBF chain (+-1 factors with
+// diagonals):
+//
+//   D[n][m] = sum_k (1 - 2 bit[n][k]) * s[n][k/128] * xs[m][k]
+//
+// ("1-bit group-128 sign packing": y = sum_g s_g sum_{k in g} sign * x; the
+// group scale is folded into the weight operand, which is exact because s is
+// an fp16 value and a sign flip only sets its top bit.)
+//  * sg_prep_kernel: xs = fp16(x * 2^c_t) per token row (exact scaling).
+//  * sg_gemm_kernel: one CTA per SM, persistent over 128 x 256 output tiles
+//    (128 weight rows x 256 tokens), swap-AB: D^T (TMEM, fp32, 256 columns,
+//    two accumulators) = A (shared memory, +-s fp16) x xs^T (shared memory,
+//    fp16, by TMA), 128 x 256 x 16 MMAs (N = 256 keeps the tensor pipe busy
+//    per instruction).  Pipeline stages are 64 wide in K (one 128-byte swizzle
+//    row of fp16), four deep:
+//    warp 0 TMA producer (xs: one 256 x 64 box per stage); warp 1 MMA issuer
+//    (4 MMAs per stage, all of K into one accumulator per tile); warps 2-5
+//    expanders (thread = weight row: 2 sign words + the group scale -> 32
+//    fp16 pairs, written in the 128B-swizzled K-major layout the MMA reads);
+//    warps 6-9 epilogue (thread = TMEM lane: row diagonal and token scale,
+//    store), draining one accumulator while the MMA fills the other.
+// Products of +-s and fp16 are exact in the tensor core; accumulation is fp32.
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_fp16.h>
+
+#include "w1_common.cuh"
+
+namespace w1 {
+
+bool make_tmap_bf16_sw128(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int box_rows);
+
+namespace sg {
+constexpr int BN = 128;   // weight rows per tile (MMA M, TMEM lanes)
+constexpr int BM = 256;   // tokens per tile (MMA N)
+constexpr int BK = 128;   // K per scale group
+constexpr int BKS = 64;   // K per pipeline stage
+constexpr int NS = 4;     // stages
+constexpr int kThreads = 320;  // 10 warps
+constexpr int kXStage = BM * BKS * 2;  // 32 KB
+constexpr int kAStage = BN * BKS * 2;  // 16 KB
+constexpr uint32_t kIdesc = idesc_f16(BN, BM, 0, 0);  // fp16 x fp16 -> fp32
+constexpr uint32_t kTmemCols = 512;                   // two accumulators of BM columns
+
+struct Smem {
+  alignas(1024) unsigned char x[NS][kXStage];
+  alignas(1024) unsigned char a[NS][kAStage];
+  uint64_t full_x[NS], full_a[NS], empty[NS];
+  uint64_t full_c[2], empty_c[2];
+  uint32_t tmem_base;
+};
+}  // namespace sg
+
+// Activation prep, one CTA per token row t:
+//   xs[t] = fp16( b (.) x[t] * 2^c_t ), 2^c_t putting max |b x| in [2^14, 2^15)
+// (exact power-of-two scaling; fp16 keeps all 8 significant bits of a bf16
+// product with a unit diagonal, and 11 of b x), cscale[t] = 2^-c_t.  With a
+// middle diagonal `mid`, also d_t with max|mid| * ||b x||_1 * 2^d_t <= 2^15
+// (dscale = 2^d, dinv = 2^-d) so that an fp16 intermediate cannot overflow.
+// bdiag == nullptr means b = 1; mid == nullptr skips d.
+__global__ void __launch_bounds__(256) sg_prep_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ bdiag,
+                                                       const uint16_t* __restrict__ mid, int n, int r,
+                                                       __half* __restrict__ xs, float* __restrict__ cscale,
+                                                       float* __restrict__ dscale, float* __restrict__ dinv) {
+  pdl_wait();
+  __shared__ float red[2][8];
+  const int t = blockIdx.x;
+  const uint16_t* xr = x + static_cast<int64_t>(t) * n;
+  float mx = 0.f, l1 = 0.f;
+  for (int k = threadIdx.x; k < n; k += blockDim.x) {
+    const float v = __uint_as_float(static_cast<uint32_t>(xr[k]) << 16) *
+                    (bdiag ? __half2float(__ushort_as_half(bdiag[k])) : 1.0f);
+    mx = fmaxf(mx, fabsf(v));
+    l1 += fabsf(v);
+  }
+  float mm = 0.f;
+  if (mid)
+    for (int j = threadIdx.x; j < r; j += blockDim.x) mm = fmaxf(mm, fabsf(__half2float(__ushort_as_half(mid[j]))));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+    l1 += __shfl_xor_sync(0xFFFFFFFFu, l1, o);
+    mm = fmaxf(mm, __shfl_xor_sync(0xFFFFFFFFu, mm, o));
+  }
+  __shared__ float red_mm[8];
+  if ((threadIdx.x & 31) == 0) {
+    red[0][threadIdx.x >> 5] = mx;
+    red[1][threadIdx.x >> 5] = l1;
+    red_mm[threadIdx.x >> 5] = mm;
+  }
+  __syncthreads();
+  mx = 0.f;
+  l1 = 0.f;
+  mm = 0.f;
+  for (int i = 0; i < static_cast<int>(blockDim.x >> 5); ++i) {
+    mx = fmaxf(mx, red[0][i]);
+    l1 += red[1][i];
+    mm = fmaxf(mm, red_mm[i]);
+  }
+  // c: max |b x| 2^c in [2^14, 2^15);  d: mm * l1 * 2^d <= 2^15 (l1 rounded up)
+  int c = 0, d = 0;
+  if (mx > 0.f) {
+    int E;
+    frexpf(mx, &E);  // mx < 2^E
+    c = 15 - E;
+  }
+  if (mm > 0.f && l1 > 0.f) {
+    int E;
+    frexpf(mm * l1 * 1.0001f, &E);  // < 2^E
+    d = 15 - E;
+  }
+  const float cs = ldexpf(1.f, c);
+  for (int k = threadIdx.x; k < n; k += blockDim.x) {
+    const float v = __uint_as_float(static_cast<uint32_t>(xr[k]) << 16) *
+                    (bdiag ? __half2float(__ushort_as_half(bdiag[k])) : 1.0f);
+    xs[static_cast<int64_t>(t) * n + k] = __float2half_rn(v * cs);
+  }
+  if (threadIdx.x == 0) {
+    cscale[t] = ldexpf(1.f, -c);
+    if (dscale) dscale[t] = ldexpf(1.f, d);
+    if (dinv) dinv[t] = ldexpf(1.f, -d);
+  }
+  pdl_launch_dependents();
+}
+
+// D[n][m] = sum_k A[n][k] xs[m][k],  A[n][k] = (1 - 2 bit[n][k]) * s[n][k/128]
+// (s = 1 without group scales): an exact fp16 value, so every product is exact
+// and all of K accumulates in one fp32 TMEM tile.
+struct SgParams {
+  const uint32_t* signs;   // [rows][K/32]
+  const uint16_t* gscales; // [rows][K/128] fp16 group scales, or nullptr (+-1)
+  const uint16_t* rdiag;   // [rows] fp16 row diagonal (mid, a), or nullptr (1)
+  const float* s1;         // per token: 2^-c (phase 1) or 2^-d (phase 2)
+  const float* s2;         // per token: 2^d (phase 1) or unused
+  __half* out_h;           // phase 1 output [M][rows]
+  float* out_f;            // phase 2 output [M][rows]
+  int M, rows, K, MT, NT, NK;
+};
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
+template <bool PHASE1>
+__global__ void __launch_bounds__(sg::kThreads, 1)
+    sg_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const SgParams p) {
+  using namespace sg;
+  extern __shared__ unsigned char smem_raw[];
+  Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < NS; ++i) {
+      mbar_init(&sm.full_x[i], 1);
+      mbar_init(&sm.full_a[i], 128);
+      mbar_init(&sm.empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sm.full_c[i], 1);
+      mbar_init(&sm.empty_c[i], 128);
+    }
+    fence_mbarrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&sm.tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) asm volatile("prefetch.tensormap [%0];" ::"l"(&tmap_b) : "memory");
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  pdl_wait();
+  const int ntiles = p.MT * p.NT;
+  const int NKS = p.NK * (BK / BKS);  // stages per tile
+  const int my_tiles = (ntiles - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) /
+                       static_cast<int>(gridDim.x);
+
+  if (warp == 0) {
+    if (lane == 0) {
+      uint32_t c = 0;
+      for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+        const int mt = tile % p.MT;
+        for (int ks = 0; ks < NKS; ++ks, ++c) {
+          const int s = c % NS;
+          if (!mbar_wait(&sm.empty[s], ((c / NS) & 1) ^ 1)) goto done_prod;
+          mbar_arrive_expect_tx(&sm.full_x[s], kXStage);
+          tma_load_2d(sm.x[s], &tmap_b, ks * BKS, mt * BM, &sm.full_x[s]);
+        }
+      }
+    done_prod:;
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      uint32_t c = 0, tl = 0;
+      for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++tl) {
+        const int cb = tl & 1;
+        if (!mbar_wait(&sm.empty_c[cb], ((tl >> 1) & 1) ^ 1)) goto done_mma;
+        tc_fence_after();
+        const uint32_t d = tmem + cb * BM;
+        for (int ks = 0; ks < NKS; ++ks, ++c) {
+          const int s = c % NS;
+          if (!mbar_wait(&sm.full_x[s], (c / NS) & 1)) goto done_mma;
+          if (!mbar_wait(&sm.full_a[s], (c / NS) & 1)) goto done_mma;
+          tc_fence_after();
+          const uint32_t xbase = smem_u32(sm.x[s]);
+          const uint32_t abase = smem_u32(sm.a[s]);
+#pragma unroll
+          for (int kk = 0; kk < BKS / 16; ++kk)
+            tc_mma_ss(d, smem_desc_sw128(abase + kk * 32), smem_desc_sw128(xbase + kk * 32), kIdesc,
+                      (ks > 0 || kk > 0) ? 1u : 0u);
+          tc_commit(&sm.empty[s]);
+        }
+        tc_commit(&sm.full_c[cb]);
+      }
+    done_mma:;
+    }
+  } else if (warp < 6) {
+    // expanders: thread = weight row.  Per stage: 2 sign words (64 k) + the
+    // group scale -> 32 fp16 pairs +-s (s = the group scale, or 0x3C00 = 1.0;
+    // the sign bit comes straight from the word), stored as eight 16-byte
+    // chunks of the row in the 128B-swizzled K-major layout.  Words and scales
+    // stream through a kPf-deep register ring over this CTA's (tile, stage)
+    // sequence so L2 latency hides behind kPf stages.
+    constexpr int kPf = 8;
+    const int rl = (warp - 2) * 32 + lane;
+    const int64_t wrow = p.K >> 5;
+    int ld_tile = blockIdx.x, ld_ks = 0;
+    auto fetch = [&](uint2& w, uint32_t& sc) {
+      w = make_uint2(0, 0);
+      sc = 0x3C00u;
+      if (ld_tile < ntiles) {
+        const int n = (ld_tile / p.MT) * BN + rl;
+        if (n < p.rows) {
+          w = __ldg(reinterpret_cast<const uint2*>(p.signs + static_cast<int64_t>(n) * wrow) + ld_ks);
+          if (p.gscales) sc = __ldg(p.gscales + static_cast<int64_t>(n) * p.NK + (ld_ks >> 1));
+        }
+        if (++ld_ks == NKS) {
+          ld_ks = 0;
+          ld_tile += gridDim.x;
+        }
+      }
+    };
+    uint2 wr[kPf];
+    uint32_t sr[kPf];
+#pragma unroll
+    for (int j = 0; j < kPf; ++j) fetch(wr[j], sr[j]);
+    const int my_stages = my_tiles * NKS;
+    const uint32_t row_off = static_cast<uint32_t>(rl) * 128u;
+    const uint32_t sw = static_cast<uint32_t>(rl & 7);
+    uint32_t c = 0;
+    for (int c0 = 0; c0 < my_stages; c0 += kPf) {
+#pragma unroll
+      for (int j = 0; j < kPf; ++j) {
+        if (c0 + j >= my_stages) break;
+        const uint2 cur = wr[j];
+        const uint32_t ss = sr[j] * 0x00010001u;  // the scale in both fp16 halves
+        fetch(wr[j], sr[j]);
+        const int s = c % NS;
+        if (!mbar_wait_warp(&sm.empty[s], ((c / NS) & 1) ^ 1)) goto done_exp;
+        const uint32_t abase = smem_u32(sm.a[s]) + row_off;
+        const uint32_t words[2] = {cur.x, cur.y};
+#pragma unroll
+        for (int wi = 0; wi < 2; ++wi) {
+          const uint32_t w = words[wi];
+          uint32_t rr[16];
+#pragma unroll
+          for (int pp = 0; pp < 16; ++pp) {
+            const uint32_t src = (pp < 8) ? w : (w >> 16);
+            const int b = 2 * (pp & 7);
+            const uint32_t m = src & (3u << b);
+            const uint32_t tt = m * (0x40008000u >> b);
+            rr[pp] = (tt & 0x80008000u) | ss;
+          }
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const uint32_t chunk = static_cast<uint32_t>(wi * 4 + q);
+            st_shared_v4(abase + ((chunk ^ sw) << 4), rr[4 * q], rr[4 * q + 1], rr[4 * q + 2], rr[4 * q + 3]);
+          }
+        }
+        fence_async_shared();
+        mbar_arrive(&sm.full_a[s]);
+        ++c;
+      }
+    }
+  done_exp:;
+  } else {
+    // epilogue: one accumulator per tile, scaled by the row diagonal and the token scales
+    const int quarter = warp & 3;
+    const int rl = quarter * 32 + lane;
+    const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
+    uint32_t tl = 0;
+    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++tl) {
+      const int mt = tile % p.MT, nt = tile / p.MT;
+      const int n = nt * BN + rl;
+      const bool valid = n < p.rows;
+      const float rd = valid ? (p.rdiag ? __half2float(__ushort_as_half(p.rdiag[n])) : 1.0f) : 0.f;
+      const int cb = tl & 1;
+      if (!mbar_wait_warp(&sm.full_c[cb], (tl >> 1) & 1)) goto done_epi;
+      tc_fence_after();
+      const int mrem = min(BM, p.M - mt * BM);
+#pragma unroll 1
+      for (int q4 = 0; q4 < BM / 32; ++q4) {
+        if (q4 * 32 >= mrem) break;
+        uint32_t rr[32];
+        tmem_ld32(tmem + lane_addr + cb * BM + q4 * 32, rr);
+        tc_wait_ld();
+        if (valid) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int m = q4 * 32 + j;
+            if (m < mrem) {
+              const int64_t tok = static_cast<int64_t>(mt) * BM + m;
+              if (PHASE1) {
+                const float v = rd * __uint_as_float(rr[j]) * (__ldg(p.s1 + tok) * __ldg(p.s2 + tok));
+                p.out_h[tok * p.rows + n] = __float2half_rn(v);
+              } else {
+                p.out_f[tok * p.rows + n] = rd * __uint_as_float(rr[j]) * __ldg(p.s1 + tok);
+              }
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&sm.empty_c[cb]);
+    }
+  done_epi:;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+  pdl_launch_dependents();
+}
+
+// ------------------------------------------------------------------ host side
+
+template <bool PHASE1>
+cudaError_t launch_sg_gemm(const SgParams& p, const void* bmat, int64_t bcols, cudaStream_t stream,
+                                   int num_sms) {
+  using namespace sg;
+  CUtensorMap tm;
+  // fp16 and bf16 share the 2-byte element layout the tensor map describes
+  if (!make_tmap_bf16_sw128(&tm, bmat, p.M, bcols, BM)) return cudaErrorInvalidValue;  // box {64, BM}
+  const size_t smem = sizeof(Smem) + 1024;
+  cudaError_t err =
+      cudaFuncSetAttribute(sg_gemm_kernel<PHASE1>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (err != cudaSuccess) return err;
+  const int ntiles = p.MT * p.NT;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(ntiles < num_sms ? ntiles : num_sms));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, sg_gemm_kernel<PHASE1>, tm, p);
+}
+
+cudaError_t launch_sg_prep(const uint16_t* x, const uint16_t* bdiag, const uint16_t* mid, int64_t n, int64_t r,
+                          int64_t B, __half* xs, float* cscale, float* dscale, float* dinv, cudaStream_t stream) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(B));
+  cfg.blockDim = dim3(256);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, sg_prep_kernel, x, bdiag, mid, static_cast<int>(n), static_cast<int>(r), xs, cscale,
+                            dscale, dinv);
+}
+
+}  // namespace w1

@@ -16,7 +16,9 @@ cudaError_t launch_gemv(const uint32_t* signs, const uint16_t* scales, int64_t N
                         const uint16_t* x, int B, float* y, cudaStream_t stream, int num_sms,
                         int smem_cap, bool static_weights);
 cudaError_t launch_gemm(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t K,
-                        const uint16_t* x, int64_t M, float* y, cudaStream_t stream, int num_sms);
+                        const uint16_t* x, int64_t M, float* y, void* workspace, cudaStream_t stream,
+                        int num_sms);
+size_t gemm_workspace_bytes(int64_t M, int64_t K);
 
 cudaError_t launch_dbf(const uint16_t* a, const uint32_t* B1, const uint16_t* mid, const uint32_t* B2,
                        const uint16_t* b, int64_t m, int64_t r, int64_t n, const uint16_t* x, int64_t B,
@@ -132,16 +134,24 @@ int w1_gemv(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t K,
 }
 
 int w1_gemm(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t K,
-            const uint16_t* x, int64_t M, float* y, w1_stream_t stream) {
+            const uint16_t* x, int64_t M, float* y, void* workspace, size_t ws_bytes,
+            w1_stream_t stream) {
   if (!signs || !scales || !x || !y) return W1_ERR_NULL;
   if (N <= 0 || K <= 0 || M <= 0 || (K % 128) != 0) return W1_ERR_SHAPE;
   if (M > (int64_t)1 << 31 || N > (int64_t)1 << 31) return W1_ERR_SHAPE;
   if (!aligned16(signs) || !aligned16(scales) || !aligned16(x) || !aligned16(y)) return W1_ERR_ALIGN;
+  if (!workspace || ws_bytes < gemm_workspace_bytes(M, K)) return W1_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return W1_ERR_ALIGN;
   DeviceInfo d;
   int st = device_info(&d);
   if (st != W1_OK) return st;
-  return launch_result(
-      launch_gemm(signs, scales, N, K, x, M, y, reinterpret_cast<cudaStream_t>(stream), d.sms));
+  return launch_result(launch_gemm(signs, scales, N, K, x, M, y, workspace,
+                                   reinterpret_cast<cudaStream_t>(stream), d.sms));
+}
+
+size_t w1_gemm_workspace_size(int64_t M, int64_t K) {
+  if (M <= 0 || K <= 0 || (K % 128) != 0 || M > (int64_t)1 << 31) return 0;
+  return gemm_workspace_bytes(M, K);
 }
 
 size_t dbf_workspace_size(int64_t m, int64_t r, int64_t n, int64_t B) {

@@ -7,6 +7,8 @@ raises W1Error on a non-OK status.  No computation happens here.
 """
 from __future__ import annotations
 
+import ctypes
+
 import torch
 
 from . import _lib
@@ -75,9 +77,25 @@ def w1_gemv(signs: torch.Tensor, scales: torch.Tensor, x: torch.Tensor, y: torch
     return y
 
 
+def gemm_workspace(M: int, K: int, device=None) -> torch.Tensor:
+    """Workspace bytes for w1_gemm (fp16 copy of x, token scales)."""
+    n = _lib.call("w1_gemm_workspace_size", M, K)
+    if n == 0:
+        raise ValueError("invalid w1_gemm sizes")
+    return torch.empty(n + 256, dtype=torch.uint8, device=device)
+
+
+def _aligned256(ws: torch.Tensor) -> int:
+    p = ws.data_ptr()
+    return (p + 255) // 256 * 256
+
+
 def w1_gemm(signs: torch.Tensor, scales: torch.Tensor, x: torch.Tensor, y: torch.Tensor | None = None,
-            stream=None) -> torch.Tensor:
-    """y [M, N] fp32 = x [M, K] bf16 times the 1-bit matrix (prefill)."""
+            stream=None, workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """y [M, N] fp32 = x [M, K] bf16 times the 1-bit matrix (prefill).
+
+    workspace: a gemm_workspace(M, K) buffer; allocated here when omitted.
+    """
     N = signs.shape[0]
     K = signs.shape[1] * 32
     M = x.shape[0]
@@ -85,7 +103,12 @@ def w1_gemm(signs: torch.Tensor, scales: torch.Tensor, x: torch.Tensor, y: torch
         raise TypeError("x must be bfloat16")
     if y is None:
         y = torch.empty((M, N), dtype=torch.float32, device=x.device)
-    st = _lib.call("w1_gemm", _ptr(signs), _ptr(scales), N, K, _ptr(x), M, _ptr(y), _stream(stream))
+    if workspace is None:
+        workspace = gemm_workspace(M, K, device=x.device)
+    base = _aligned256(workspace)
+    avail = workspace.numel() - (base - workspace.data_ptr())
+    st = _lib.call("w1_gemm", _ptr(signs), _ptr(scales), N, K, _ptr(x), M, _ptr(y),
+                   ctypes.c_void_p(base), avail, _stream(stream))
     _lib.check(st, "w1_gemm")
     return y
 

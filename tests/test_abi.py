@@ -55,8 +55,14 @@ def test_host_side_argument_errors(lib):
     assert lib.w1_gemv(good, None, 16, 128, good, 1, good, None) == _lib.W1_ERR_NULL
     assert lib.w1_gemv(good, good, 16, 130, good, 1, good, None) == _lib.W1_ERR_SHAPE
     assert lib.w1_gemv(good, good, 16, 128, odd, 1, good, None) == _lib.W1_ERR_ALIGN
-    assert lib.w1_gemm(good, good, 16, 128, good, 0, good, None) == _lib.W1_ERR_SHAPE
-    assert lib.w1_gemm(good, good, 16, 128, good, 4, None, None) == _lib.W1_ERR_NULL
+    assert lib.w1_gemm(good, good, 16, 128, good, 0, good, good, 1 << 30, None) == _lib.W1_ERR_SHAPE
+    assert lib.w1_gemm(good, good, 16, 128, good, 4, None, good, 1 << 30, None) == _lib.W1_ERR_NULL
+    need = lib.w1_gemm_workspace_size(4, 128)
+    assert need >= 4 * 128 * 2 + 4
+    assert lib.w1_gemm(good, good, 16, 128, good, 4, good, good, need - 1, None) == _lib.W1_ERR_WORKSPACE
+    assert lib.w1_gemm(good, good, 16, 128, good, 4, good, None, need, None) == _lib.W1_ERR_WORKSPACE
+    assert lib.w1_gemm(good, good, 16, 128, good, 4, good, odd, need, None) == _lib.W1_ERR_ALIGN
+    assert lib.w1_gemm_workspace_size(4, 100) == 0
 
 
 def test_dbf_host_side_argument_errors(lib):
