@@ -42,6 +42,12 @@ GEMM_SHAPES = [(14336, 4096), (4096, 14336), (14336, 14336)]
 GEMM_M = 2048
 WORKLOAD = ("decode GEMV sweep: (out x in) 4096x4096, 11008x4096, 4096x11008 at B = 1, 4, 8; "
             "1-bit signs + fp16 scale per 128 weights; x bf16 N(0,1); W N(0,0.02)")
+# DRAM bytes per launch from ncu captures (dram__bytes_read.sum + write), with the
+# shape captured; see profiles/.  Used to report the dominant kernel's traffic.
+CAPTURED_TRAFFIC = {
+    "gemv_tc_kernel": {"shape": (4096, 11008, 8), "bytes": 6585344},
+    "gemv_direct_kernel": {"shape": (4096, 4096, 1), "bytes": 2433280},
+}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -538,8 +544,23 @@ def run_gpu(args):
                           "frac_hbm": round(gbs / peaks["hbm_gbs"], 4),
                           "static_weights_us_per_launch": round(st_us, 3),
                           "static_weights_GB/s": round(cb["bytes"] / (st_us * 1e-6) / 1e9, 1)})
-    pair_sum_ms = sum(per_pair_ms)
-    achieved = bytes_per_step * args.steps / (pair_sum_ms * 1e-3) / 1e9
+    # roofline of the dominant kernel (largest share of the step's device time)
+    per_kernel = {}
+    for cb, ms, row in zip(combos, per_pair_ms, gemv_rows):
+        k = per_kernel.setdefault(row["kernel"], {"ms": 0.0, "bytes": 0.0, "launches": 0})
+        k["ms"] += ms
+        k["bytes"] += cb["bytes"] * cb["R"] * args.steps
+        k["launches"] += cb["R"] * args.steps
+    dom = max(per_kernel, key=lambda k: per_kernel[k]["ms"])
+    dk = per_kernel[dom]
+    achieved = dk["bytes"] / (dk["ms"] * 1e-3) / 1e9
+    traffic = None
+    cap = CAPTURED_TRAFFIC.get(dom)
+    if cap is not None:
+        n_, k_, _b = cap["shape"]
+        # scale the captured DRAM bytes to this kernel's mean launch by algorithmic bytes
+        traffic = round(cap["bytes"] / packed_bytes(n_, k_) * dk["bytes"] / dk["launches"])
+    dom_share = dk["ms"] / sum(per_pair_ms)
 
     e2e = gemv_e2e(torch, ops, combos, max(1, min(args.steps, 3)))
     rows = {"gemv": gemv_rows}
@@ -581,7 +602,9 @@ def run_gpu(args):
                    "parallelism": f"replicas x{world} (independent sweeps, no collective)"},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                      "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
-                     "traffic": None, "kernel": "gemv_direct_kernel (B<=4), gemv_tc_kernel (B=8)",
+                     "traffic": traffic, "kernel": dom, "time_share": round(dom_share, 4),
+                     "algorithmic_bytes_per_launch": round(dk["bytes"] / dk["launches"]),
+                     "traffic_note": "ncu DRAM bytes of one captured launch, scaled by algorithmic bytes",
                      "peak_kind": peaks_kind},
         "cpu_baseline": cpu,
         "e2e": {k: e2e[k] for k in ("value", "unit", "h2d_bytes_per_step", "d2h_bytes_per_step")},

@@ -62,9 +62,6 @@ cudaError_t launch_dbf_tc(const uint16_t* a, const uint32_t* B1, const uint16_t*
                           const uint16_t* b, int64_t m, int64_t r, int64_t n, const uint16_t* x, int64_t B, float* y,
                           void* workspace, cudaStream_t stream, int num_sms) {
   using namespace dbftc;
-  using sg::BN;
-  using sg::BM;
-  using sg::BK;
   const Ws L = ws_layout(B, r, n);
   unsigned char* ws = static_cast<unsigned char*>(workspace);
   float* cs = reinterpret_cast<float*>(ws + L.cscale);
@@ -83,9 +80,6 @@ cudaError_t launch_dbf_tc(const uint16_t* a, const uint32_t* B1, const uint16_t*
   p1.M = static_cast<int>(B);
   p1.rows = static_cast<int>(r);
   p1.K = static_cast<int>(n);
-  p1.MT = static_cast<int>((B + BM - 1) / BM);
-  p1.NT = static_cast<int>((r + BN - 1) / BN);
-  p1.NK = static_cast<int>(n / BK);
   err = launch_sg_gemm<true>(p1, xs, n, stream, num_sms);
   if (err != cudaSuccess) return err;
   // phase 2 undoes the intermediate's scale: s1 = 2^-d
@@ -97,9 +91,6 @@ cudaError_t launch_dbf_tc(const uint16_t* a, const uint32_t* B1, const uint16_t*
   p2.M = static_cast<int>(B);
   p2.rows = static_cast<int>(m);
   p2.K = static_cast<int>(r);
-  p2.MT = p1.MT;
-  p2.NT = static_cast<int>((m + BN - 1) / BN);
-  p2.NK = static_cast<int>(r / BK);
   return launch_sg_gemm<false>(p2, hs, r, stream, num_sms);
 }
 

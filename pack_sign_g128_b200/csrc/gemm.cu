@@ -89,9 +89,6 @@ size_t gemm_workspace_bytes(int64_t M, int64_t K) {
 cudaError_t launch_gemm(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t K,
                         const uint16_t* x, int64_t M, float* y, void* workspace, cudaStream_t stream,
                         int num_sms) {
-  using sg::BK;
-  using sg::BM;
-  using sg::BN;
   const size_t xs_bytes = (static_cast<size_t>(M) * K * 2 + 1023) / 1024 * 1024;
   __half* xs = static_cast<__half*>(workspace);
   float* cscale = reinterpret_cast<float*>(static_cast<unsigned char*>(workspace) + xs_bytes);
@@ -105,9 +102,6 @@ cudaError_t launch_gemm(const uint32_t* signs, const uint16_t* scales, int64_t N
   p.M = static_cast<int>(M);
   p.rows = static_cast<int>(N);
   p.K = static_cast<int>(K);
-  p.MT = static_cast<int>((M + BM - 1) / BM);
-  p.NT = static_cast<int>((N + BN - 1) / BN);
-  p.NK = static_cast<int>(K / BK);
   return launch_sg_gemm<false>(p, xs, K, stream, num_sms);
 }
 

@@ -9,7 +9,7 @@
 // an fp16 value and a sign flip only sets its top bit.)
 //  * sg_prep_kernel: xs = fp16(x * 2^c_t) per token row (exact scaling).
 //  * sg_gemm_kernel: one CTA per SM, persistent over 128 x 256 output tiles
-//    (128 weight rows x 256 tokens), swap-AB: D^T (TMEM, fp32, 256 columns,
+//    (128 weight rows x 256 tokens; 128 tokens when that fills more SMs), swap-AB: D^T (TMEM, fp32, 256 columns,
 //    two accumulators) = A (shared memory, +-s fp16) x xs^T (shared memory,
 //    fp16, by TMA), 128 x 256 x 16 MMAs (N = 256 keeps the tensor pipe busy
 //    per instruction).  Pipeline stages are 64 wide in K (one 128-byte swizzle
@@ -33,17 +33,17 @@ bool make_tmap_bf16_sw128(CUtensorMap* map, const void* base, int64_t rows, int6
 
 namespace sg {
 constexpr int BN = 128;   // weight rows per tile (MMA M, TMEM lanes)
-constexpr int BM = 256;   // tokens per tile (MMA N)
 constexpr int BK = 128;   // K per scale group
 constexpr int BKS = 64;   // K per pipeline stage
 constexpr int NS = 4;     // stages
 constexpr int kThreads = 320;  // 10 warps
-constexpr int kXStage = BM * BKS * 2;  // 32 KB
 constexpr int kAStage = BN * BKS * 2;  // 16 KB
-constexpr uint32_t kIdesc = idesc_f16(BN, BM, 0, 0);  // fp16 x fp16 -> fp32
-constexpr uint32_t kTmemCols = 512;                   // two accumulators of BM columns
 
+// BMT tokens per tile (MMA N): 256 when there are enough tiles to fill the
+// GPU, 128 for few token rows (more tiles, each MMA half as long).
+template <int BMT>
 struct Smem {
+  static constexpr int kXStage = BMT * BKS * 2;
   alignas(1024) unsigned char x[NS][kXStage];
   alignas(1024) unsigned char a[NS][kAStage];
   uint64_t full_x[NS], full_a[NS], empty[NS];
@@ -142,12 +142,15 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
 
-template <bool PHASE1>
+template <bool PHASE1, int BM>
 __global__ void __launch_bounds__(sg::kThreads, 1)
     sg_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const SgParams p) {
   using namespace sg;
+  constexpr int kXStage = Smem<BM>::kXStage;
+  constexpr uint32_t kIdesc = idesc_f16(BN, BM, 0, 0);  // fp16 x fp16 -> fp32
+  constexpr uint32_t kTmemCols = 2 * BM;                // two accumulators of BM columns
   extern __shared__ unsigned char smem_raw[];
-  Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Smem<BM>& sm = *reinterpret_cast<Smem<BM>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int i = 0; i < NS; ++i) {
@@ -335,16 +338,18 @@ __global__ void __launch_bounds__(sg::kThreads, 1)
 
 // ------------------------------------------------------------------ host side
 
-template <bool PHASE1>
-cudaError_t launch_sg_gemm(const SgParams& p, const void* bmat, int64_t bcols, cudaStream_t stream,
-                                   int num_sms) {
+template <bool PHASE1, int BM>
+static cudaError_t launch_sg_gemm_bm(SgParams p, const void* bmat, int64_t bcols, cudaStream_t stream, int num_sms) {
   using namespace sg;
+  p.MT = (p.M + BM - 1) / BM;
+  p.NT = (p.rows + BN - 1) / BN;
+  p.NK = p.K / BK;
   CUtensorMap tm;
-  // fp16 and bf16 share the 2-byte element layout the tensor map describes
-  if (!make_tmap_bf16_sw128(&tm, bmat, p.M, bcols, BM)) return cudaErrorInvalidValue;  // box {64, BM}
-  const size_t smem = sizeof(Smem) + 1024;
-  cudaError_t err =
-      cudaFuncSetAttribute(sg_gemm_kernel<PHASE1>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  // fp16 and bf16 share the 2-byte element layout the tensor map describes; box {64, BM}
+  if (!make_tmap_bf16_sw128(&tm, bmat, p.M, bcols, BM)) return cudaErrorInvalidValue;
+  const size_t smem = sizeof(Smem<BM>) + 1024;
+  cudaError_t err = cudaFuncSetAttribute(sg_gemm_kernel<PHASE1, BM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
   if (err != cudaSuccess) return err;
   const int ntiles = p.MT * p.NT;
   cudaLaunchConfig_t cfg = {};
@@ -357,7 +362,16 @@ cudaError_t launch_sg_gemm(const SgParams& p, const void* bmat, int64_t bcols, c
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, sg_gemm_kernel<PHASE1>, tm, p);
+  return cudaLaunchKernelEx(&cfg, sg_gemm_kernel<PHASE1, BM>, tm, p);
+}
+
+// p: signs, gscales, rdiag, s1, s2, outputs, M, rows, K (tiles are derived here).
+template <bool PHASE1>
+cudaError_t launch_sg_gemm(const SgParams& p, const void* bmat, int64_t bcols, cudaStream_t stream, int num_sms) {
+  const int nt = (p.rows + sg::BN - 1) / sg::BN;
+  const int tiles256 = ((p.M + 255) / 256) * nt;
+  if (tiles256 >= num_sms) return launch_sg_gemm_bm<PHASE1, 256>(p, bmat, bcols, stream, num_sms);
+  return launch_sg_gemm_bm<PHASE1, 128>(p, bmat, bcols, stream, num_sms);
 }
 
 cudaError_t launch_sg_prep(const uint16_t* x, const uint16_t* bdiag, const uint16_t* mid, int64_t n, int64_t r,
