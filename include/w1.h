@@ -156,12 +156,16 @@ size_t w1_gemm_workspace_size(int64_t M, int64_t K);
  *   H, I multiples of 128; 1 <= top_k <= min(E, 32); E <= 256.
  * workspace: >= w1_moe_workspace_size(...) bytes, 1024-byte aligned; holds the
  *   routing (expert ids, weights, the expert-sorted route order), the tile
- *   lists, h (bf16, expert-sorted) and the weighted route outputs.  No state is
- *   carried between calls.  Calls sharing a workspace must not overlap.
- * Five kernels on `stream`: router, counting sort, grouped gate/up GEMM (tokens
- * gathered from x by TMA, fused SwiGLU), grouped down GEMM (route weight
- * applied), slot-ordered combine.  Deterministic.  Accuracy per stage as
- * w1_gemm: 1e-3 * sum|s x| for g, u and D_e h.
+ *   lists, h (bf16, expert-sorted), the weighted route outputs, and the fp16
+ *   copies of x rows and h rows in sorted route order with one power-of-two
+ *   scale per route.  No state is carried between calls.  Calls sharing a
+ *   workspace must not overlap.
+ * Seven kernels on `stream`: router, counting sort, gather of x rows into
+ * sorted order (fp16, exact per-route power of two), grouped gate/up GEMM
+ * (tcgen05, +-s fp16 weight operand, fused SwiGLU), h to fp16 per route,
+ * grouped down GEMM (route weight applied), slot-ordered combine.
+ * Deterministic.  Accuracy per stage as w1_gemm: 1e-3 * sum|s x| for g, u and
+ * D_e h.
  */
 int w1_moe_grouped(const uint16_t* x, const float* router_logits, int64_t T, int64_t H, int64_t I, int64_t E,
                    int64_t top_k, const uint32_t* gate_signs, const uint16_t* gate_scales,

@@ -10,22 +10,28 @@
 // expert-major compaction of route-specific inputs, shared gate/up inputs
 // kept un-duplicated, fused SwiGLU, skipped empty tiles.
 //
-// Five launches on one stream (programmatic dependent launch between them):
+// Seven launches on one stream (programmatic dependent launch between them):
 //  1. route_kernel     warp per token: fp32 softmax, top-k by logit, weights.
 //  2. sort_kernel      one CTA: stable counting sort of the routes by expert
 //                      (deterministic), route -> sorted position map, and the
 //                      tile lists of the two grouped GEMMs (no empty tiles).
-//  3. moe_gemm<GATEUP> tcgen05 grouped GEMM, swap-AB as in w1_gemm: the gate
-//                      and up rows of expert e (TMEM, +-1 bf16) times token
-//                      rows gathered from x by TMA tile::gather4 (x is never
-//                      duplicated per route); the epilogue applies the group
-//                      scales, SiLU(g) * u and stores h (bf16) in sorted order.
-//  4. moe_gemm<DOWN>   the down rows of expert e times h rows (contiguous per
-//                      expert); epilogue multiplies by the route weight and
+//  3. gather_kernel    x rows in expert-sorted route order as fp16 with an
+//                      exact power of two per route (max |x| in [2^14, 2^15)).
+//  4. moe_gemm<GATEUP> tcgen05 grouped GEMM, swap-AB as in w1_gemm: the gate
+//                      and up rows of expert e as +-s fp16 (the group scale
+//                      with the weight's sign, exact) times the expert's
+//                      contiguous route rows; each accumulates all of K in
+//                      TMEM; the epilogue applies the route scale, SiLU(g) * u
+//                      and stores h (bf16) in sorted order.
+//  5. sg_prep_kernel   h -> fp16 with a power of two per route (sign_gemm.cu).
+//  6. moe_gemm<DOWN>   the down rows of expert e times those rows; epilogue
+//                      multiplies by the route scale and the route weight and
 //                      stores the route output (fp32, sorted order).
-//  5. combine_kernel   out[t] = sum over slots, in slot order.
-// MMA N (tokens per tile) is set per tile from the expert's route count
+//  7. combine_kernel   out[t] = sum over slots, in slot order.
+// MMA N (routes per tile) is set per tile from the expert's route count
 // (rounded up to 16), so partially filled tiles cost only what they hold.
+// On B200 x is duplicated once per route (top_k copies, fp16): one plain TMA
+// box per pipeline stage replaces 32 row gathers, for a few MB of traffic.
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_fp16.h>
@@ -36,9 +42,11 @@
 namespace w1 {
 
 bool make_tmap_bf16_sw128(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int box_rows);
+cudaError_t launch_sg_prep(const uint16_t* x, const uint16_t* bdiag, const uint16_t* mid, int64_t n, int64_t r,
+                          int64_t B, __half* xs, float* cscale, float* dscale, float* dinv, cudaStream_t stream);
 
 namespace moe {
-constexpr int TN_GU = 64;    // routes per gate/up tile
+constexpr int TN_GU = 128;   // routes per gate/up tile
 constexpr int TN_D = 128;    // routes per down tile
 constexpr int kMaxE = 256;
 constexpr int kMaxTopK = 32;
@@ -49,7 +57,7 @@ struct Tile {
 };
 
 struct Workspace {
-  size_t hdr, ids, wts, pos, sroute, stok, offsets, tiles_gu, tiles_d, h, rout, total;
+  size_t hdr, ids, wts, pos, sroute, stok, offsets, tiles_gu, tiles_d, h, rout, xs, xscale, hs, hscale, total;
   int max_tiles_gu, max_tiles_d;
 };
 
@@ -82,7 +90,15 @@ __host__ __device__ inline Workspace workspace_layout(int64_t T, int64_t H, int6
   w.h = off;
   off = align_up(off + 2 * static_cast<size_t>(R) * I, 1024);
   w.rout = off;
-  off = align_up(off + 4 * static_cast<size_t>(R) * H, 256);
+  off = align_up(off + 4 * static_cast<size_t>(R) * H, 1024);
+  w.xs = off;
+  off = align_up(off + 2 * static_cast<size_t>(R) * H, 1024);
+  w.xscale = off;
+  off = align_up(off + 4 * static_cast<size_t>(R), 1024);
+  w.hs = off;
+  off = align_up(off + 2 * static_cast<size_t>(R) * I, 1024);
+  w.hscale = off;
+  off = align_up(off + 4 * static_cast<size_t>(R), 256);
   w.total = off;
   return w;
 }
@@ -283,6 +299,7 @@ struct MoeGemmParams {
   const int* stok;           // sorted position -> token (gather rows)
   const int* sroute;         // sorted position -> route
   const float* wts;          // route weights
+  const float* rscale;       // per sorted route: 2^-c of the fp16 B rows
   __nv_bfloat16* h;          // gate/up output [R][I]
   float* rout;               // down output [R][H]
   int rows;                  // rows of each expert matrix (I for gate/up, H for down)
@@ -292,43 +309,34 @@ struct MoeGemmParams {
 
 template <bool GATEUP>
 struct MoeCfg {
-  static constexpr int TN = GATEUP ? moe::TN_GU : moe::TN_D;
-  static constexpr int NMAT = GATEUP ? 2 : 1;                 // A matrices per tile
-  static constexpr int NSX = 4;                               // X stages
-  static constexpr int NSA = GATEUP ? 2 : 4;                  // A stages (64 cols per matrix)
-  static constexpr int XSTAGE = TN * 128 * 2;                 // bytes of one X stage
-  static constexpr uint32_t ACOL0 = 2 * NMAT * TN;            // chunk buffers first
-  static constexpr uint32_t ASTRIDE = NMAT * 64;              // TMEM cols per A stage
+  static constexpr int TN = GATEUP ? moe::TN_GU : moe::TN_D;  // routes per tile (max MMA N)
+  static constexpr int NMAT = GATEUP ? 2 : 1;                 // weight matrices per tile
+  static constexpr int BKS = 64;                              // K per pipeline stage
+  static constexpr int NS = 4;                                // stages
+  static constexpr int XSTAGE = TN * BKS * 2;                 // bytes of one B stage (fp16)
+  static constexpr int ASTAGE = 128 * BKS * 2;                // bytes of one weight matrix stage
+  static constexpr uint32_t kTmemCols = GATEUP ? 512 : 256;   // two accumulator sets
 };
 
 template <bool GATEUP>
 struct MoeSmem {
-  alignas(1024) unsigned char x[MoeCfg<GATEUP>::NSX][MoeCfg<GATEUP>::XSTAGE];
-  uint64_t full_x[MoeCfg<GATEUP>::NSX], empty_x[MoeCfg<GATEUP>::NSX];
-  uint64_t full_a[MoeCfg<GATEUP>::NSA], empty_a[MoeCfg<GATEUP>::NSA];
+  alignas(1024) unsigned char x[MoeCfg<GATEUP>::NS][MoeCfg<GATEUP>::XSTAGE];
+  alignas(1024) unsigned char a[MoeCfg<GATEUP>::NS][MoeCfg<GATEUP>::NMAT][MoeCfg<GATEUP>::ASTAGE];
+  uint64_t full_x[MoeCfg<GATEUP>::NS], full_a[MoeCfg<GATEUP>::NS], empty[MoeCfg<GATEUP>::NS];
   uint64_t full_c[2], empty_c[2];
-  int rows_idx[MoeCfg<GATEUP>::TN];
   uint32_t tmem_base;
 };
 
-__device__ __forceinline__ void tma_gather4(void* smem_dst, const void* tmap, int32_t col, int32_t r0, int32_t r1,
-                                            int32_t r2, int32_t r3, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes [%0], [%1, {%2, "
-      "%3, %4, %5, %6}], [%7];" ::"r"(smem_u32(smem_dst)),
-      "l"(tmap), "r"(col), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(smem_u32(bar))
-      : "memory");
+__device__ __forceinline__ void moe_st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
 
-__device__ __forceinline__ uint32_t expand_pair(uint32_t w, int pp) {
-  // bf16 pair for columns (2pp, 2pp+1) of a 32-bit sign word: sign bits to 15 / 31
-  const uint32_t src = (pp < 8) ? w : (w >> 16);
-  const int b = 2 * (pp & 7);
-  const uint32_t m = src & (3u << b);
-  const uint32_t t = m * (0x40008000u >> b);
-  return (t & 0x80008000u) | 0x3F803F80u;
-}
-
+// Warp roles: 0 TMA producer (route rows of B), 1 MMA issuer, 2-5 expanders
+// (thread = weight row: 2 sign words + the group scale per matrix -> 32 fp16
+// pairs +-s in the 128B-swizzled K-major layout), 6-9 epilogue (thread =
+// TMEM lane).  One 64-wide K stage: NMAT x 4 MMAs (M = 128, N = the tile's
+// route count rounded up to 16, K = 16), all of K into one accumulator per
+// matrix per tile; two accumulator sets alternate between tiles.
 template <bool GATEUP>
 __global__ void __launch_bounds__(moe::kThreads, 1)
     moe_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const MoeGemmParams p) {
@@ -338,13 +346,10 @@ __global__ void __launch_bounds__(moe::kThreads, 1)
       *reinterpret_cast<MoeSmem<GATEUP>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    for (int i = 0; i < C::NSX; ++i) {
+    for (int i = 0; i < C::NS; ++i) {
       mbar_init(&sm.full_x[i], 1);
-      mbar_init(&sm.empty_x[i], 1);
-    }
-    for (int i = 0; i < C::NSA; ++i) {
       mbar_init(&sm.full_a[i], 128);
-      mbar_init(&sm.empty_a[i], 1);
+      mbar_init(&sm.empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sm.full_c[i], 1);
@@ -353,7 +358,7 @@ __global__ void __launch_bounds__(moe::kThreads, 1)
     fence_mbarrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(&sm.tmem_base, 512);
+    tmem_alloc(&sm.tmem_base, C::kTmemCols);
     tmem_relinquish();
   }
   if (warp == 0 && lane == 0) asm volatile("prefetch.tensormap [%0];" ::"l"(&tmap_b) : "memory");
@@ -363,195 +368,281 @@ __global__ void __launch_bounds__(moe::kThreads, 1)
   const uint32_t tmem = sm.tmem_base;
   pdl_wait();
   const int ntiles = p.hdr[GATEUP ? 0 : 1];
-  const int NK = p.K >> 7;
+  const int NG = p.K >> 7;          // scale groups per row
+  const int NKS = p.K / C::BKS;     // stages per tile
 
   if (warp == 0) {
-    // ---------------------------------------- producer: token rows of X
-    uint32_t c = 0;
-    for (int ti = blockIdx.x; ti < ntiles; ti += gridDim.x) {
-      const moe::Tile tl = p.tiles[ti];
-      if (GATEUP) {
-        // gather indices of this tile (rows past the count repeat the first)
-        __syncwarp();
-        for (int j = lane; j < C::TN; j += 32) sm.rows_idx[j] = p.stok[tl.start + (j < tl.count ? j : 0)];
-        __syncwarp();
-      }
-      for (int kc = 0; kc < NK; ++kc, ++c) {
-        const int s = c % C::NSX;
-        if (!mbar_wait_warp(&sm.empty_x[s], ((c / C::NSX) & 1) ^ 1)) goto done_prod;
-        if (lane == 0) {
-          mbar_arrive_expect_tx(&sm.full_x[s], C::XSTAGE);
-          if (GATEUP) {
-#pragma unroll 1
-            for (int half = 0; half < 2; ++half)
-#pragma unroll 1
-              for (int q = 0; q < C::TN / 4; ++q)
-                tma_gather4(sm.x[s] + half * (C::XSTAGE / 2) + q * 512, &tmap_b, kc * 128 + half * 64,
-                            sm.rows_idx[4 * q], sm.rows_idx[4 * q + 1], sm.rows_idx[4 * q + 2],
-                            sm.rows_idx[4 * q + 3], &sm.full_x[s]);
-          } else {
-            tma_load_2d(sm.x[s], &tmap_b, kc * 128, tl.start, &sm.full_x[s]);
-            tma_load_2d(sm.x[s] + C::XSTAGE / 2, &tmap_b, kc * 128 + 64, tl.start, &sm.full_x[s]);
-          }
-        }
-        __syncwarp();
-      }
-    }
-  done_prod:;
-  } else if (warp == 1) {
-    // ---------------------------------------- MMA issuer
     if (lane == 0) {
       uint32_t c = 0;
       for (int ti = blockIdx.x; ti < ntiles; ti += gridDim.x) {
         const moe::Tile tl = p.tiles[ti];
+        for (int ks = 0; ks < NKS; ++ks, ++c) {
+          const int s = c % C::NS;
+          if (!mbar_wait(&sm.empty[s], ((c / C::NS) & 1) ^ 1)) goto done_prod;
+          mbar_arrive_expect_tx(&sm.full_x[s], C::XSTAGE);
+          tma_load_2d(sm.x[s], &tmap_b, ks * C::BKS, tl.start, &sm.full_x[s]);
+        }
+      }
+    done_prod:;
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      uint32_t c = 0, tli = 0;
+      for (int ti = blockIdx.x; ti < ntiles; ti += gridDim.x, ++tli) {
+        const moe::Tile tl = p.tiles[ti];
         const int n_mma = ((tl.count + 15) >> 4) << 4;
-        const uint32_t idesc = idesc_f16(128, n_mma, 1, 1);
-        for (int kc = 0; kc < NK; ++kc, ++c) {
-          const int sx = c % C::NSX, sa = c % C::NSA, cb = c & 1;
-          if (!mbar_wait(&sm.full_x[sx], (c / C::NSX) & 1)) goto done_mma;
-          if (!mbar_wait(&sm.full_a[sa], (c / C::NSA) & 1)) goto done_mma;
-          if (!mbar_wait(&sm.empty_c[cb], ((c >> 1) & 1) ^ 1)) goto done_mma;
+        const uint32_t idesc = idesc_f16(128, n_mma, 0, 0);  // fp16 x fp16 -> fp32
+        const int cb = tli & 1;
+        if (!mbar_wait(&sm.empty_c[cb], ((tli >> 1) & 1) ^ 1)) goto done_mma;
+        tc_fence_after();
+        for (int ks = 0; ks < NKS; ++ks, ++c) {
+          const int s = c % C::NS;
+          if (!mbar_wait(&sm.full_x[s], (c / C::NS) & 1)) goto done_mma;
+          if (!mbar_wait(&sm.full_a[s], (c / C::NS) & 1)) goto done_mma;
           tc_fence_after();
-          const uint32_t xbase = smem_u32(sm.x[sx]);
+          const uint32_t xbase = smem_u32(sm.x[s]);
 #pragma unroll
           for (int mat = 0; mat < C::NMAT; ++mat) {
-            const uint32_t d = tmem + cb * (C::NMAT * C::TN) + mat * C::TN;
-            const uint32_t a = tmem + C::ACOL0 + sa * C::ASTRIDE + mat * 64;
+            const uint32_t d = tmem + (cb * C::NMAT + mat) * C::TN;
+            const uint32_t abase = smem_u32(sm.a[s][mat]);
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-              const uint32_t baddr = xbase + (kk >> 2) * (C::XSTAGE / 2) + (kk & 3) * 32;
-              tc_mma_ts(d, a + kk * 8, smem_desc_sw128(baddr), idesc, kk > 0 ? 1u : 0u);
-            }
+            for (int kk = 0; kk < C::BKS / 16; ++kk)
+              tc_mma_ss(d, smem_desc_sw128(abase + kk * 32), smem_desc_sw128(xbase + kk * 32), idesc,
+                        (ks > 0 || kk > 0) ? 1u : 0u);
           }
-          tc_commit(&sm.empty_x[sx]);
-          tc_commit(&sm.empty_a[sa]);
-          tc_commit(&sm.full_c[cb]);
+          tc_commit(&sm.empty[s]);
         }
+        tc_commit(&sm.full_c[cb]);
       }
     done_mma:;
     }
   } else if (warp < 6) {
-    // ---------------------------------------- expanders: thread = weight row
-    const int quarter = warp & 3;
-    const int rl = quarter * 32 + lane;
-    const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
+    // expanders: thread = weight row of the tile's 128-row block
+    constexpr int kPf = 4;
+    const int rl = (warp - 2) * 32 + lane;
     const int64_t wrow = p.K >> 5;
-    uint32_t c = 0;
-    for (int ti = blockIdx.x; ti < ntiles; ti += gridDim.x) {
-      const moe::Tile tl = p.tiles[ti];
-      const int row = tl.rt * 128 + rl;
-      const bool valid = row < p.rows;
-      const int64_t ridx = static_cast<int64_t>(tl.e) * p.rows + (valid ? row : 0);
-      const uint4* wa = reinterpret_cast<const uint4*>(p.a_signs + ridx * wrow);
-      const uint4* wu = GATEUP ? reinterpret_cast<const uint4*>(p.u_signs + ridx * wrow) : wa;
-      uint4 na = valid ? __ldg(wa) : make_uint4(0, 0, 0, 0);
-      uint4 nu = (GATEUP && valid) ? __ldg(wu) : make_uint4(0, 0, 0, 0);
-      for (int kc = 0; kc < NK; ++kc, ++c) {
-        const uint4 ca = na, cu = nu;
-        if (kc + 1 < NK && valid) {
-          na = __ldg(wa + kc + 1);
-          if (GATEUP) nu = __ldg(wu + kc + 1);
-        }
-        const int sa = c % C::NSA;
-        if (!mbar_wait_warp(&sm.empty_a[sa], ((c / C::NSA) & 1) ^ 1)) goto done_exp;
-        tc_fence_after();
+    // the stream's current tile: row pointers cached in registers, the tile
+    // descriptor read once per tile (not once per stage)
+    int ld_ti = blockIdx.x, ld_ks = 0;
+    const uint2* wp[C::NMAT];
+    const uint16_t* sp[C::NMAT];
+    bool ld_valid = false;
+    auto load_tile = [&]() {
+      ld_valid = false;
+      if (ld_ti < ntiles) {
+        const moe::Tile tl = p.tiles[ld_ti];
+        const int row = tl.rt * 128 + rl;
+        ld_valid = row < p.rows;
+        const int64_t ridx = static_cast<int64_t>(tl.e) * p.rows + (ld_valid ? row : 0);
 #pragma unroll
         for (int mat = 0; mat < C::NMAT; ++mat) {
-          const uint4 cw = mat ? cu : ca;
-          const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
+          wp[mat] = reinterpret_cast<const uint2*>((mat ? p.u_signs : p.a_signs) + ridx * wrow);
+          sp[mat] = (mat ? p.u_scales : p.a_scales) + ridx * NG;
+        }
+      }
+    };
+    load_tile();
+    auto fetch = [&](uint2 (&w)[C::NMAT], uint32_t (&sc)[C::NMAT]) {
 #pragma unroll
-          for (int half = 0; half < 2; ++half) {
-            uint32_t r[32];
+      for (int mat = 0; mat < C::NMAT; ++mat) {
+        w[mat] = make_uint2(0, 0);
+        sc[mat] = 0x3C00u;
+      }
+      if (ld_ti < ntiles) {
+        if (ld_valid) {
 #pragma unroll
-            for (int wi = 0; wi < 2; ++wi)
-#pragma unroll
-              for (int pp = 0; pp < 16; ++pp) r[wi * 16 + pp] = expand_pair(words[half * 2 + wi], pp);
-            tmem_st32(tmem + lane_addr + C::ACOL0 + sa * C::ASTRIDE + mat * 64 + half * 32, r);
+          for (int mat = 0; mat < C::NMAT; ++mat) {
+            w[mat] = __ldg(wp[mat] + ld_ks);
+            sc[mat] = __ldg(sp[mat] + (ld_ks >> 1));
           }
         }
-        tc_wait_st();
-        tc_fence_before();
-        mbar_arrive(&sm.full_a[sa]);
+        if (++ld_ks == NKS) {
+          ld_ks = 0;
+          ld_ti += gridDim.x;
+          load_tile();
+        }
+      }
+    };
+    uint2 wr[kPf][C::NMAT];
+    uint32_t sr[kPf][C::NMAT];
+#pragma unroll
+    for (int j = 0; j < kPf; ++j) fetch(wr[j], sr[j]);
+    const int my_tiles = (ntiles - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) /
+                         static_cast<int>(gridDim.x);
+    const int my_stages = (my_tiles > 0 ? my_tiles : 0) * NKS;
+    const uint32_t row_off = static_cast<uint32_t>(rl) * 128u;
+    const uint32_t swz = static_cast<uint32_t>(rl & 7);
+    uint32_t c = 0;
+    for (int c0 = 0; c0 < my_stages; c0 += kPf) {
+#pragma unroll
+      for (int j = 0; j < kPf; ++j) {
+        if (c0 + j >= my_stages) break;
+        uint2 cur[C::NMAT];
+        uint32_t ss[C::NMAT];
+#pragma unroll
+        for (int mat = 0; mat < C::NMAT; ++mat) {
+          cur[mat] = wr[j][mat];
+          ss[mat] = sr[j][mat] * 0x00010001u;  // the scale in both fp16 halves
+        }
+        fetch(wr[j], sr[j]);
+        const int s = c % C::NS;
+        if (!mbar_wait_warp(&sm.empty[s], ((c / C::NS) & 1) ^ 1)) goto done_exp;
+#pragma unroll
+        for (int mat = 0; mat < C::NMAT; ++mat) {
+          const uint32_t abase = smem_u32(sm.a[s][mat]) + row_off;
+          const uint32_t words[2] = {cur[mat].x, cur[mat].y};
+#pragma unroll
+          for (int wi = 0; wi < 2; ++wi) {
+            const uint32_t w = words[wi];
+            uint32_t rr[16];
+#pragma unroll
+            for (int pp = 0; pp < 16; ++pp) {
+              const uint32_t src = (pp < 8) ? w : (w >> 16);
+              const int b = 2 * (pp & 7);
+              const uint32_t m = src & (3u << b);
+              const uint32_t tt = m * (0x40008000u >> b);
+              rr[pp] = (tt & 0x80008000u) | ss[mat];
+            }
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const uint32_t chunk = static_cast<uint32_t>(wi * 4 + q);
+              moe_st_shared_v4(abase + ((chunk ^ swz) << 4), rr[4 * q], rr[4 * q + 1], rr[4 * q + 2], rr[4 * q + 3]);
+            }
+          }
+        }
+        fence_async_shared();
+        mbar_arrive(&sm.full_a[s]);
+        ++c;
       }
     }
   done_exp:;
   } else {
-    // ---------------------------------------- promoters + epilogue: thread = weight row
+    // epilogue: thread = weight row (TMEM lane)
     const int quarter = warp & 3;
     const int rl = quarter * 32 + lane;
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
-    const int NG = p.K >> 7;
-    uint32_t c = 0;
-    for (int ti = blockIdx.x; ti < ntiles; ti += gridDim.x) {
+    uint32_t tli = 0;
+    for (int ti = blockIdx.x; ti < ntiles; ti += gridDim.x, ++tli) {
       const moe::Tile tl = p.tiles[ti];
       const int row = tl.rt * 128 + rl;
       const bool valid = row < p.rows;
-      const int64_t ridx = static_cast<int64_t>(tl.e) * p.rows + (valid ? row : 0);
-      const uint16_t* sa_p = p.a_scales + ridx * NG;
-      const uint16_t* su_p = GATEUP ? p.u_scales + ridx * NG : sa_p;
-      float acc[C::NMAT][C::TN];
-#pragma unroll
-      for (int mat = 0; mat < C::NMAT; ++mat)
-#pragma unroll
-        for (int j = 0; j < C::TN; ++j) acc[mat][j] = 0.f;
-      const int nq = (tl.count + 31) >> 5;  // 32-column pieces holding routes
-      uint16_t sa_next = valid ? __ldg(sa_p) : 0, su_next = (GATEUP && valid) ? __ldg(su_p) : 0;
-      for (int kc = 0; kc < NK; ++kc, ++c) {
-        const float s_a = __half2float(__ushort_as_half(sa_next));
-        const float s_u = __half2float(__ushort_as_half(su_next));
-        if (kc + 1 < NK && valid) {
-          sa_next = __ldg(sa_p + kc + 1);
-          if (GATEUP) su_next = __ldg(su_p + kc + 1);
-        }
-        const int cb = c & 1;
-        if (!mbar_wait_warp(&sm.full_c[cb], (c >> 1) & 1)) goto done_prom;
-        tc_fence_after();
-#pragma unroll
-        for (int mat = 0; mat < C::NMAT; ++mat) {
-          const float s = mat ? s_u : s_a;
-#pragma unroll
-          for (int q4 = 0; q4 < C::TN / 32; ++q4) {
-            if (q4 < nq) {
-              uint32_t r[32];
-              tmem_ld32(tmem + lane_addr + cb * (C::NMAT * C::TN) + mat * C::TN + q4 * 32, r);
-              tc_wait_ld();
-#pragma unroll
-              for (int j = 0; j < 32; ++j) acc[mat][q4 * 32 + j] = fmaf(s, __uint_as_float(r[j]), acc[mat][q4 * 32 + j]);
-            }
-          }
-        }
-        tc_fence_before();
-        mbar_arrive(&sm.empty_c[cb]);
-      }
-      if (valid) {
+      const int cb = tli & 1;
+      if (!mbar_wait_warp(&sm.full_c[cb], (tli >> 1) & 1)) goto done_epi;
+      tc_fence_after();
+#pragma unroll 1
+      for (int q4 = 0; q4 < C::TN / 32; ++q4) {
+        if (q4 * 32 >= tl.count) break;
+        uint32_t rg[32];
+        tmem_ld32(tmem + lane_addr + (cb * C::NMAT) * C::TN + q4 * 32, rg);
         if (GATEUP) {
-          __nv_bfloat16* hp = p.h + static_cast<int64_t>(tl.start) * p.out_ld + row;
+          uint32_t ru[32];
+          tmem_ld32(tmem + lane_addr + (cb * C::NMAT + C::NMAT - 1) * C::TN + q4 * 32, ru);
+          tc_wait_ld();
+          if (valid) {
+            __nv_bfloat16* hp = p.h + static_cast<int64_t>(tl.start) * p.out_ld + row;
 #pragma unroll
-          for (int j = 0; j < C::TN; ++j) {
-            if (j < tl.count) {
-              const float g = acc[0][j];
-              const float hv = g / (1.0f + expf(-g)) * acc[C::NMAT - 1][j];
-              hp[static_cast<int64_t>(j) * p.out_ld] = __float2bfloat16_rn(hv);
+            for (int j = 0; j < 32; ++j) {
+              const int jj = q4 * 32 + j;
+              if (jj < tl.count) {
+                const float rs = __ldg(p.rscale + tl.start + jj);
+                const float g = __uint_as_float(rg[j]) * rs;
+                const float u = __uint_as_float(ru[j]) * rs;
+                const float hv = g / (1.0f + expf(-g)) * u;
+                hp[static_cast<int64_t>(jj) * p.out_ld] = __float2bfloat16_rn(hv);
+              }
             }
           }
         } else {
-          float* op = p.rout + static_cast<int64_t>(tl.start) * p.out_ld + row;
+          tc_wait_ld();
+          if (valid) {
+            float* op = p.rout + static_cast<int64_t>(tl.start) * p.out_ld + row;
 #pragma unroll
-          for (int j = 0; j < C::TN; ++j) {
-            if (j < tl.count) {
-              const float wgt = __ldg(p.wts + __ldg(p.sroute + tl.start + j));
-              __stcs(op + static_cast<int64_t>(j) * p.out_ld, wgt * acc[0][j]);
+            for (int j = 0; j < 32; ++j) {
+              const int jj = q4 * 32 + j;
+              if (jj < tl.count) {
+                const float wgt = __ldg(p.wts + __ldg(p.sroute + tl.start + jj)) * __ldg(p.rscale + tl.start + jj);
+                __stcs(op + static_cast<int64_t>(jj) * p.out_ld, wgt * __uint_as_float(rg[j]));
+              }
             }
           }
         }
       }
+      tc_fence_before();
+      mbar_arrive(&sm.empty_c[cb]);
     }
-  done_prom:;
+  done_epi:;
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem, 512);
+  if (warp == 1) tmem_dealloc(tmem, C::kTmemCols);
+  pdl_launch_dependents();
+}
+
+// ------------------------------------------------------------------ gather x rows (sorted, fp16)
+
+// One CTA per sorted route p: xs[p] = fp16(x[stok[p]] * 2^c), xscale[p] = 2^-c
+// with max |x| * 2^c in [2^14, 2^15) (exact scaling of every bf16 value in range).
+// 16-byte loads and stores; the row stays in registers between the max and the
+// conversion (H <= 8 * 256 * kMaxV), longer rows are read twice.
+__global__ void __launch_bounds__(256) moe_gather_kernel(const uint16_t* __restrict__ x, const int* __restrict__ stok,
+                                                         int H, __half* __restrict__ xs, float* __restrict__ xscale) {
+  constexpr int kMaxV = 4;
+  pdl_wait();
+  __shared__ float red[8];
+  const int pr = blockIdx.x;
+  const uint4* xr = reinterpret_cast<const uint4*>(x + static_cast<int64_t>(__ldg(stok + pr)) * H);
+  const int nv = H >> 3;  // 16-byte vectors per row
+  uint4 v[kMaxV];
+  float mx = 0.f;
+#pragma unroll
+  for (int j = 0; j < kMaxV; ++j) {
+    const int i = threadIdx.x + 256 * j;
+    v[j] = i < nv ? __ldg(xr + i) : make_uint4(0, 0, 0, 0);
+    const uint32_t w[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      mx = fmaxf(mx, fmaxf(fabsf(__uint_as_float(w[q] << 16)), fabsf(__uint_as_float(w[q] & 0xFFFF0000u))));
+  }
+  for (int i = threadIdx.x + 256 * kMaxV; i < nv; i += 256) {
+    const uint4 u = __ldg(xr + i);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      mx = fmaxf(mx, fmaxf(fabsf(__uint_as_float(w[q] << 16)), fabsf(__uint_as_float(w[q] & 0xFFFF0000u))));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
+  __syncthreads();
+  mx = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) mx = fmaxf(mx, red[i]);
+  int c = 0;
+  if (mx > 0.f) {
+    int E;
+    frexpf(mx, &E);  // mx < 2^E
+    c = 15 - E;
+  }
+  const float cs = ldexpf(1.f, c);
+  uint4* dst = reinterpret_cast<uint4*>(xs + static_cast<int64_t>(pr) * H);
+  auto convert = [&](const uint4& u) {
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const __half2 h2 = __floats2half2_rn(__uint_as_float(w[q] << 16) * cs, __uint_as_float(w[q] & 0xFFFF0000u) * cs);
+      o[q] = *reinterpret_cast<const uint32_t*>(&h2);
+    }
+    return make_uint4(o[0], o[1], o[2], o[3]);
+  };
+#pragma unroll
+  for (int j = 0; j < kMaxV; ++j) {
+    const int i = threadIdx.x + 256 * j;
+    if (i < nv) dst[i] = convert(v[j]);
+  }
+  for (int i = threadIdx.x + 256 * kMaxV; i < nv; i += 256) dst[i] = convert(__ldg(xr + i));
+  if (threadIdx.x == 0) xscale[pr] = ldexpf(1.f, -c);
   pdl_launch_dependents();
 }
 
@@ -629,10 +720,18 @@ cudaError_t launch_moe(const uint16_t* x, const float* logits, int64_t T, int64_
               tiles_gu, tiles_d, hdr};
   err = launch_pdl(moe_sort_kernel, dim3(1), dim3(1024), 0, stream, sa);
   if (err != cudaSuccess) return err;
-  // 3. gate/up with fused SwiGLU
+  __half* xs = reinterpret_cast<__half*>(ws + L.xs);
+  float* xscale = reinterpret_cast<float*>(ws + L.xscale);
+  __half* hs = reinterpret_cast<__half*>(ws + L.hs);
+  float* hscale = reinterpret_cast<float*>(ws + L.hscale);
+  // 3. x rows in sorted route order, fp16 with a power of two per route
+  err = launch_pdl(moe_gather_kernel, dim3(static_cast<unsigned>(R)), dim3(256), 0, stream, x, stok,
+                   static_cast<int>(H), xs, xscale);
+  if (err != cudaSuccess) return err;
+  // 4. gate/up with fused SwiGLU
   {
     CUtensorMap tm;
-    if (!make_tmap_bf16_sw128(&tm, x, T, H, 1)) return cudaErrorInvalidValue;
+    if (!make_tmap_bf16_sw128(&tm, xs, R, H, moe::TN_GU)) return cudaErrorInvalidValue;
     MoeGemmParams p = {};
     p.a_signs = gs;
     p.a_scales = gc;
@@ -643,6 +742,7 @@ cudaError_t launch_moe(const uint16_t* x, const float* logits, int64_t T, int64_
     p.stok = stok;
     p.sroute = sroute;
     p.wts = wts;
+    p.rscale = xscale;
     p.h = h;
     p.rows = static_cast<int>(I);
     p.K = static_cast<int>(H);
@@ -654,10 +754,14 @@ cudaError_t launch_moe(const uint16_t* x, const float* logits, int64_t T, int64_
     err = launch_pdl(moe_gemm_kernel<true>, dim3(grid), dim3(moe::kThreads), smem, stream, tm, p);
     if (err != cudaSuccess) return err;
   }
-  // 4. down with route weights
+  // 5. h -> fp16 with a power of two per route
+  err = launch_sg_prep(reinterpret_cast<const uint16_t*>(h), nullptr, nullptr, I, 0, R, hs, hscale, nullptr, nullptr,
+                       stream);
+  if (err != cudaSuccess) return err;
+  // 6. down with route weights
   {
     CUtensorMap tm;
-    if (!make_tmap_bf16_sw128(&tm, h, R, I, moe::TN_D)) return cudaErrorInvalidValue;
+    if (!make_tmap_bf16_sw128(&tm, hs, R, I, moe::TN_D)) return cudaErrorInvalidValue;
     MoeGemmParams p = {};
     p.a_signs = ds;
     p.a_scales = dc;
@@ -666,6 +770,7 @@ cudaError_t launch_moe(const uint16_t* x, const float* logits, int64_t T, int64_
     p.stok = stok;
     p.sroute = sroute;
     p.wts = wts;
+    p.rscale = hscale;
     p.rout = rout;
     p.rows = static_cast<int>(H);
     p.K = static_cast<int>(I);

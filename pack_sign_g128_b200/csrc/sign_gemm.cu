@@ -60,19 +60,60 @@ struct Smem {
 // (dscale = 2^d, dinv = 2^-d) so that an fp16 intermediate cannot overflow.
 // bdiag == nullptr means b = 1; mid == nullptr skips d.
 __global__ void __launch_bounds__(256) sg_prep_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ bdiag,
-                                                       const uint16_t* __restrict__ mid, int n, int r,
-                                                       __half* __restrict__ xs, float* __restrict__ cscale,
-                                                       float* __restrict__ dscale, float* __restrict__ dinv) {
+                                                      const uint16_t* __restrict__ mid, int n, int r,
+                                                      __half* __restrict__ xs, float* __restrict__ cscale,
+                                                      float* __restrict__ dscale, float* __restrict__ dinv) {
+  // 16-byte vectors (8 values); the row stays in registers between the
+  // reductions and the conversion when n <= 8 * 256 * kMaxV, else it is re-read.
+  constexpr int kMaxV = 4;
   pdl_wait();
-  __shared__ float red[2][8];
+  __shared__ float red[3][8];
   const int t = blockIdx.x;
-  const uint16_t* xr = x + static_cast<int64_t>(t) * n;
+  const uint4* xr = reinterpret_cast<const uint4*>(x + static_cast<int64_t>(t) * n);
+  const uint4* br = reinterpret_cast<const uint4*>(bdiag);
+  const int nv = n >> 3;
+  auto values = [&](int i, const uint4& u, float (&v)[8]) {
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      v[2 * q] = __uint_as_float(w[q] << 16);
+      v[2 * q + 1] = __uint_as_float(w[q] & 0xFFFF0000u);
+    }
+    if (bdiag) {
+      const uint4 bb = __ldg(br + i);
+      const uint32_t bw[4] = {bb.x, bb.y, bb.z, bb.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&bw[q]));
+        v[2 * q] *= f.x;
+        v[2 * q + 1] *= f.y;
+      }
+    }
+  };
+  uint4 keep[kMaxV];
   float mx = 0.f, l1 = 0.f;
-  for (int k = threadIdx.x; k < n; k += blockDim.x) {
-    const float v = __uint_as_float(static_cast<uint32_t>(xr[k]) << 16) *
-                    (bdiag ? __half2float(__ushort_as_half(bdiag[k])) : 1.0f);
-    mx = fmaxf(mx, fabsf(v));
-    l1 += fabsf(v);
+#pragma unroll
+  for (int j = 0; j < kMaxV; ++j) {
+    const int i = threadIdx.x + 256 * j;
+    keep[j] = i < nv ? __ldg(xr + i) : make_uint4(0, 0, 0, 0);
+    if (i < nv) {
+      float v[8];
+      values(i, keep[j], v);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        mx = fmaxf(mx, fabsf(v[q]));
+        l1 += fabsf(v[q]);
+      }
+    }
+  }
+  for (int i = threadIdx.x + 256 * kMaxV; i < nv; i += 256) {
+    float v[8];
+    values(i, __ldg(xr + i), v);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      mx = fmaxf(mx, fabsf(v[q]));
+      l1 += fabsf(v[q]);
+    }
   }
   float mm = 0.f;
   if (mid)
@@ -83,20 +124,20 @@ __global__ void __launch_bounds__(256) sg_prep_kernel(const uint16_t* __restrict
     l1 += __shfl_xor_sync(0xFFFFFFFFu, l1, o);
     mm = fmaxf(mm, __shfl_xor_sync(0xFFFFFFFFu, mm, o));
   }
-  __shared__ float red_mm[8];
   if ((threadIdx.x & 31) == 0) {
     red[0][threadIdx.x >> 5] = mx;
     red[1][threadIdx.x >> 5] = l1;
-    red_mm[threadIdx.x >> 5] = mm;
+    red[2][threadIdx.x >> 5] = mm;
   }
   __syncthreads();
   mx = 0.f;
   l1 = 0.f;
   mm = 0.f;
-  for (int i = 0; i < static_cast<int>(blockDim.x >> 5); ++i) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
     mx = fmaxf(mx, red[0][i]);
     l1 += red[1][i];
-    mm = fmaxf(mm, red_mm[i]);
+    mm = fmaxf(mm, red[2][i]);
   }
   // c: max |b x| 2^c in [2^14, 2^15);  d: mm * l1 * 2^d <= 2^15 (l1 rounded up)
   int c = 0, d = 0;
@@ -111,11 +152,24 @@ __global__ void __launch_bounds__(256) sg_prep_kernel(const uint16_t* __restrict
     d = 15 - E;
   }
   const float cs = ldexpf(1.f, c);
-  for (int k = threadIdx.x; k < n; k += blockDim.x) {
-    const float v = __uint_as_float(static_cast<uint32_t>(xr[k]) << 16) *
-                    (bdiag ? __half2float(__ushort_as_half(bdiag[k])) : 1.0f);
-    xs[static_cast<int64_t>(t) * n + k] = __float2half_rn(v * cs);
+  uint4* dst = reinterpret_cast<uint4*>(xs + static_cast<int64_t>(t) * n);
+  auto convert = [&](int i, const uint4& u) {
+    float v[8];
+    values(i, u, v);
+    uint32_t o[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const __half2 h2 = __floats2half2_rn(v[2 * q] * cs, v[2 * q + 1] * cs);
+      o[q] = *reinterpret_cast<const uint32_t*>(&h2);
+    }
+    dst[i] = make_uint4(o[0], o[1], o[2], o[3]);
+  };
+#pragma unroll
+  for (int j = 0; j < kMaxV; ++j) {
+    const int i = threadIdx.x + 256 * j;
+    if (i < nv) convert(i, keep[j]);
   }
+  for (int i = threadIdx.x + 256 * kMaxV; i < nv; i += 256) convert(i, __ldg(xr + i));
   if (threadIdx.x == 0) {
     cscale[t] = ldexpf(1.f, -c);
     if (dscale) dscale[t] = ldexpf(1.f, d);

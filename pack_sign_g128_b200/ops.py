@@ -153,7 +153,7 @@ def moe_workspace_views(workspace: torch.Tensor, T: int, H: int, I: int, E: int,
         off = up(off + 4 * R, 256)
     views["offsets"] = workspace[off:off + 4 * (E + 1)].view(torch.int32)
     off = up(off + 4 * (E + 1), 256)
-    mtg = ((R + 63) // 64 + E) * (I // 128)
+    mtg = ((R + 127) // 128 + E) * (I // 128)
     mtd = ((R + 127) // 128 + E) * (H // 128)
     off = up(off + 16 * mtg, 256)
     off = up(off + 16 * mtd, 256)
