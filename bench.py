@@ -42,6 +42,7 @@ GEMM_SHAPES = [(14336, 4096), (4096, 14336), (14336, 14336)]
 GEMM_M = 2048
 WORKLOAD = ("decode GEMV sweep: (out x in) 4096x4096, 11008x4096, 4096x11008 at B = 1, 4, 8; "
             "1-bit signs + fp16 scale per 128 weights; x bf16 N(0,1); W N(0,0.02)")
+KERNEL_OF_CHOICE = {"direct": "gemv_direct_kernel", "tc": "gemv_tc_kernel", "ring": "gemv_kernel"}
 # DRAM bytes per launch from ncu captures (dram__bytes_read.sum + write), with the
 # shape captured; see profiles/.  Used to report the dominant kernel's traffic.
 CAPTURED_TRAFFIC = {
@@ -539,7 +540,8 @@ def run_gpu(args):
         per_launch_us = ms * 1e3 / (cb["R"] * args.steps)
         gbs = cb["bytes"] / (per_launch_us * 1e-6) / 1e9
         gemv_rows.append({"N": cb["N"], "K": cb["K"], "B": cb["B"], "launches": cb["R"],
-                          "kernel": "gemv_direct_kernel" if cb["B"] <= 4 else "gemv_tc_kernel",
+                          "choice": ops.gemv_choice(cb["N"], cb["K"], cb["B"]),
+                          "kernel": KERNEL_OF_CHOICE.get(ops.gemv_choice(cb["N"], cb["K"], cb["B"]).split("/")[0], "?"),
                           "us_per_launch": round(per_launch_us, 3), "GB/s": round(gbs, 1),
                           "frac_hbm": round(gbs / peaks["hbm_gbs"], 4),
                           "static_weights_us_per_launch": round(st_us, 3),
@@ -592,7 +594,7 @@ def run_gpu(args):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "s8 x s8 -> s32 MMA (mma.sync at B<=4, tcgen05 kind::i8 at B>4) + f32 scale fold; x bf16, 1-bit weights, fp16 scales",
+        "dtype": "s8 x s8 -> s32 MMA (mma.sync or tcgen05 kind::i8, chosen per shape by timing) + f32 scale fold; x bf16, 1-bit weights, fp16 scales",
         "data": "synthetic",
         "config": {"workload": WORKLOAD, "launches_per_step": launches_per_step,
                    "packed_bytes_per_step": bytes_per_step,

@@ -92,6 +92,13 @@ int w1_pack(const float* W, int64_t N, int64_t K, uint32_t* signs, uint16_t* sca
  *   signs [N][K/32], scales [N][K/128], x bf16 [B][K], y fp32 [B][N] (all device).
  * Accuracy: |y - y_exact| <= 1e-3 * sum_k |s x_k| per element (x is taken as
  * 24-bit fixed point per 128-group, fp32 accumulation).
+ * Kernel choice: the first call for a new (N, K, B) on a device, when `stream`
+ * is not being captured, times the candidate kernels and K splits on `stream`
+ * with the caller's buffers and keeps the fastest; that call blocks the host
+ * until the timing finishes (about a millisecond).  Later calls, and calls
+ * during stream capture, launch without synchronising.  Results of different
+ * candidates differ only in fp32 summation order; a shape's choice is fixed
+ * once made, so repeated calls are bitwise reproducible.
  */
 int w1_gemv(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t K,
             const uint16_t* x, int64_t B, float* y, w1_stream_t stream);
@@ -114,6 +121,14 @@ enum { W1_GEMV_STATIC_WEIGHTS = 1 };
  */
 int w1_gemv_ex(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t K,
                const uint16_t* x, int64_t B, float* y, uint32_t flags, w1_stream_t stream);
+
+/*
+ * w1_gemv_choice -- inspection: writes the kernel and K split that w1_gemv /
+ * w1_gemv_ex has chosen for (N, K, B, flags) on the current device, as
+ * "direct/<split>", "tc/<split>" or "ring/<split>" (split 0: the kernel's own
+ * planner), or "" when no call has chosen yet.  Host only, no GPU work.
+ */
+int w1_gemv_choice(int64_t N, int64_t K, int64_t B, uint32_t flags, char* out, size_t out_len);
 
 /*
  * w1_gemm -- prefill-regime product for many token rows (DBF post, section 4:

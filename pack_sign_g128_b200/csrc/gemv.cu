@@ -309,31 +309,16 @@ static cudaError_t launch_gemv_nb(const uint32_t* signs, const GemvParams& base,
 }
 
 cudaError_t launch_gemv_tc(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t K, const uint16_t* x,
-                           int B, float* y, cudaStream_t stream, int num_sms);
+                           int B, float* y, cudaStream_t stream, int num_sms, int force_s);
 cudaError_t launch_gemv_direct(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t K,
                                const uint16_t* x, int B, float* y, bool static_weights, cudaStream_t stream,
-                               int num_sms, int smem_cap);
+                               int num_sms, int smem_cap, int force_s);
 
-// Kernel choice, from measurements on the decode shapes: the direct kernel
-// (gemv_direct.cu) for B <= 4, the tcgen05 kernel (gemv_tc.cu) for larger
-// batches, each only where its plan fits the shape, else the mma.sync ring
-// kernel below.  W1_GEMV_PATH=direct|tc|mma forces one kernel (tuning and
-// testing knob; a forced kernel whose plan does not fit the shape fails with
-// W1_ERR_UNSUPPORTED).
-cudaError_t launch_gemv(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t K,
-                        const uint16_t* x, int B, float* y, cudaStream_t stream, int num_sms,
-                        int smem_cap, bool static_weights) {
-  const char* path = getenv("W1_GEMV_PATH");
-  const char which = path ? path[0] : 'a';
-  if (which == 'd' || (which == 'a' && B <= 4)) {
-    const cudaError_t e =
-        launch_gemv_direct(signs, scales, N, K, x, B, y, static_weights, stream, num_sms, smem_cap);
-    if (e != cudaErrorNotSupported || which == 'd') return e;
-  }
-  if (which == 't' || (which == 'a' && B > 4)) {
-    const cudaError_t e = launch_gemv_tc(signs, scales, N, K, x, B, y, stream, num_sms);
-    if (e != cudaErrorNotSupported || which == 't') return e;
-  }
+// The mma.sync ring kernel over row chunks (the fallback for shapes outside
+// the other two kernels' plans).
+static cudaError_t launch_gemv_ring(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t K,
+                                   const uint16_t* x, int B, float* y, cudaStream_t stream, int num_sms,
+                                   int smem_cap) {
   const int NG = static_cast<int>(K / 128);
   // rows per launch bounded so that per-CTA scale / partial buffers fit
   const int64_t max_rows = 32768;
@@ -364,4 +349,160 @@ cudaError_t launch_gemv(const uint32_t* signs, const uint16_t* scales, int64_t N
   return cudaSuccess;
 }
 
+// ------------------------------------------------------------------ dispatch
+
+// Kernel and K split per (device, N, K, B, static weights), chosen by timing.
+// The first call for a shape (outside stream capture) runs each candidate --
+// the direct kernel with K split 1, 2, 4, 8, the tcgen05 kernel, the ring
+// kernel -- twice untimed and five times between CUDA events on the caller's
+// stream with the caller's buffers, keeps the fastest, and blocks the host
+// until that finishes (about a millisecond).  Calls made while the stream is
+// being captured, or with W1_GEMV_AUTOTUNE=0, use the static rule instead:
+// direct for B <= 4, tcgen05 above, each only where its plan fits, else the
+// ring kernel.  W1_GEMV_PATH=direct|tc|mma forces one kernel (testing knob;
+// a forced kernel whose plan does not fit fails with W1_ERR_UNSUPPORTED).
+namespace {
+struct GemvChoice {
+  char kind;  // 'd' direct, 't' tcgen05, 'm' ring
+  int s;      // forced K split, 0 = the kernel's planner
+};
+struct GemvChoiceEntry {
+  int dev;
+  int64_t N, K;
+  int B;
+  bool st;
+  GemvChoice c;
+};
+GemvChoiceEntry g_choice[256];
+int g_nchoice = 0;
+std::mutex g_choice_mu;
+}  // namespace
+
+static cudaError_t run_gemv_choice(const GemvChoice& c, const uint32_t* signs, const uint16_t* scales, int64_t N,
+                                   int64_t K, const uint16_t* x, int B, float* y, cudaStream_t stream, int num_sms,
+                                   int smem_cap, bool static_weights) {
+  switch (c.kind) {
+    case 'd':
+      return launch_gemv_direct(signs, scales, N, K, x, B, y, static_weights, stream, num_sms, smem_cap, c.s);
+    case 't':
+      return launch_gemv_tc(signs, scales, N, K, x, B, y, stream, num_sms, c.s);
+    default:
+      return launch_gemv_ring(signs, scales, N, K, x, B, y, stream, num_sms, smem_cap);
+  }
+}
+
+// The static rule with fallbacks (direct or tcgen05 first by batch, then ring).
+static cudaError_t run_gemv_rule(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t K,
+                                 const uint16_t* x, int B, float* y, cudaStream_t stream, int num_sms, int smem_cap,
+                                 bool static_weights) {
+  const GemvChoice first = B <= 4 ? GemvChoice{'d', 0} : GemvChoice{'t', 0};
+  const GemvChoice second = B <= 4 ? GemvChoice{'t', 0} : GemvChoice{'d', 0};
+  cudaError_t e = run_gemv_choice(first, signs, scales, N, K, x, B, y, stream, num_sms, smem_cap, static_weights);
+  if (e != cudaErrorNotSupported) return e;
+  e = run_gemv_choice(second, signs, scales, N, K, x, B, y, stream, num_sms, smem_cap, static_weights);
+  if (e != cudaErrorNotSupported) return e;
+  return launch_gemv_ring(signs, scales, N, K, x, B, y, stream, num_sms, smem_cap);
+}
+
+cudaError_t launch_gemv(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t K,
+                        const uint16_t* x, int B, float* y, cudaStream_t stream, int num_sms,
+                        int smem_cap, bool static_weights) {
+  if (const char* path = getenv("W1_GEMV_PATH")) {
+    const GemvChoice c{path[0] == 'd' ? 'd' : (path[0] == 't' ? 't' : 'm'), 0};
+    return run_gemv_choice(c, signs, scales, N, K, x, B, y, stream, num_sms, smem_cap, static_weights);
+  }
+  int dev = 0;
+  cudaGetDevice(&dev);
+  {
+    std::lock_guard<std::mutex> lock(g_choice_mu);
+    for (int i = 0; i < g_nchoice; ++i) {
+      const GemvChoiceEntry& e = g_choice[i];
+      if (e.dev == dev && e.N == N && e.K == K && e.B == B && e.st == static_weights)
+        return run_gemv_choice(e.c, signs, scales, N, K, x, B, y, stream, num_sms, smem_cap, static_weights);
+    }
+  }
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(stream, &cap) != cudaSuccess) {
+    cudaGetLastError();
+    cap = cudaStreamCaptureStatusActive;
+  }
+  const char* at = getenv("W1_GEMV_AUTOTUNE");
+  if (cap != cudaStreamCaptureStatusNone || (at && at[0] == '0'))
+    return run_gemv_rule(signs, scales, N, K, x, B, y, stream, num_sms, smem_cap, static_weights);
+
+  const GemvChoice cands[] = {{'d', 1}, {'d', 2}, {'d', 4}, {'d', 8}, {'t', 0}, {'m', 0}};
+  cudaEvent_t e0, e1;
+  if (cudaEventCreate(&e0) != cudaSuccess) return cudaGetLastError();
+  if (cudaEventCreate(&e1) != cudaSuccess) {
+    cudaEventDestroy(e0);
+    return cudaGetLastError();
+  }
+  GemvChoice best{0, 0};
+  float best_ms = 0.f;
+  cudaError_t fatal = cudaSuccess;
+  for (const GemvChoice& c : cands) {
+    bool ok = true;
+    for (int i = 0; i < 2 && ok; ++i) {
+      const cudaError_t e =
+          run_gemv_choice(c, signs, scales, N, K, x, B, y, stream, num_sms, smem_cap, static_weights);
+      if (e != cudaSuccess) {
+        cudaGetLastError();
+        ok = false;
+      }
+    }
+    if (!ok) continue;
+    cudaEventRecord(e0, stream);
+    for (int i = 0; i < 5; ++i)
+      run_gemv_choice(c, signs, scales, N, K, x, B, y, stream, num_sms, smem_cap, static_weights);
+    cudaEventRecord(e1, stream);
+    fatal = cudaEventSynchronize(e1);
+    if (fatal != cudaSuccess) break;  // a device error: report it, choose nothing
+    float ms = 0.f;
+    cudaEventElapsedTime(&ms, e0, e1);
+    if (best.kind == 0 || ms < best_ms) {
+      best = c;
+      best_ms = ms;
+    }
+  }
+  cudaEventDestroy(e0);
+  cudaEventDestroy(e1);
+  if (fatal != cudaSuccess) return fatal;
+  if (best.kind == 0) return run_gemv_rule(signs, scales, N, K, x, B, y, stream, num_sms, smem_cap, static_weights);
+  if (getenv("W1_VERBOSE"))
+    fprintf(stderr, "w1_gemv tuned: N=%lld K=%lld B=%d static=%d -> %c split=%d (%.2f us)\n",
+            static_cast<long long>(N), static_cast<long long>(K), B, static_weights ? 1 : 0, best.kind, best.s,
+            best_ms * 1e3f / 5.f);
+  {
+    std::lock_guard<std::mutex> lock(g_choice_mu);
+    const int i = g_nchoice < 256 ? g_nchoice++ : static_cast<int>((N + K + B) & 255);
+    g_choice[i] = GemvChoiceEntry{dev, N, K, B, static_weights, best};
+  }
+  return run_gemv_choice(best, signs, scales, N, K, x, B, y, stream, num_sms, smem_cap, static_weights);
+}
+
+// Name of the cached choice for a shape ("direct/2", "tc/0", "ring/0"), or ""
+// when none has been made on the current device.
+static int gemv_choice_name(int64_t N, int64_t K, int B, bool st, char* out, size_t out_len) {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  GemvChoice c{0, 0};
+  {
+    std::lock_guard<std::mutex> lock(g_choice_mu);
+    for (int i = 0; i < g_nchoice; ++i) {
+      const GemvChoiceEntry& e = g_choice[i];
+      if (e.dev == dev && e.N == N && e.K == K && e.B == B && e.st == st) c = e.c;
+    }
+  }
+  const char* kind = c.kind == 'd' ? "direct" : (c.kind == 't' ? "tc" : (c.kind == 'm' ? "ring" : ""));
+  if (c.kind == 0) return snprintf(out, out_len, "%s", "");
+  return snprintf(out, out_len, "%s/%d", kind, c.s);
+}
+
 }  // namespace w1
+
+extern "C" int w1_gemv_choice(int64_t N, int64_t K, int64_t B, uint32_t flags, char* out, size_t out_len) {
+  if (!out || out_len == 0) return W1_ERR_NULL;
+  if (N <= 0 || K <= 0 || (K % 128) != 0 || B < 1 || B > 8) return W1_ERR_SHAPE;
+  w1::gemv_choice_name(N, K, static_cast<int>(B), (flags & W1_GEMV_STATIC_WEIGHTS) != 0, out, out_len);
+  return W1_OK;
+}

@@ -623,9 +623,10 @@ static int g_gd_count = 0;
 static std::mutex g_gd_mu;
 
 template <int NB>
-static bool gd_cached_plan(int N, int NG, int num_sms, int smem_cap, GdPlan* out) {
-  int force = 0;
-  if (const char* f = getenv("W1_GEMV_SPLIT")) force = atoi(f);  // tuning knob: force the K split
+static bool gd_cached_plan(int N, int NG, int num_sms, int smem_cap, int force_s, GdPlan* out) {
+  int force = force_s;
+  if (!force)
+    if (const char* f = getenv("W1_GEMV_SPLIT")) force = atoi(f);  // tuning knob: force the K split
   if (force != 1 && force != 2 && force != 4 && force != 8) force = 0;
   int dev = 0;
   cudaGetDevice(&dev);
@@ -657,9 +658,10 @@ static bool gd_cached_plan(int N, int NG, int num_sms, int smem_cap, GdPlan* out
 }
 
 template <int NB>
-static cudaError_t launch_gemv_direct_nb(const GdParams& base, cudaStream_t stream, int num_sms, int smem_cap) {
+static cudaError_t launch_gemv_direct_nb(const GdParams& base, cudaStream_t stream, int num_sms, int smem_cap,
+                                         int force_s) {
   GdPlan plan;
-  if (!gd_cached_plan<NB>(base.N, base.NG, num_sms, smem_cap, &plan)) return cudaErrorNotSupported;
+  if (!gd_cached_plan<NB>(base.N, base.NG, num_sms, smem_cap, force_s, &plan)) return cudaErrorNotSupported;
   if (getenv("W1_VERBOSE"))
     fprintf(stderr,
             "w1_gemv(direct) plan: N=%d NG=%d B=%d -> clusters=%d split=%d warps=%dx%d tiles/warp=%d "
@@ -712,10 +714,11 @@ static cudaError_t launch_gemv_direct_nb(const GdParams& base, cudaStream_t stre
   return cudaLaunchKernelEx(&cfg, gemv_direct_kernel<NB>, p);
 }
 
-// Returns cudaErrorNotSupported when the shape is outside this kernel's plan.
+// Returns cudaErrorNotSupported when the shape is outside this kernel's plan
+// (or outside the plan with the forced K split force_s; 0 = planner's choice).
 cudaError_t launch_gemv_direct(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t K,
                                const uint16_t* x, int B, float* y, bool static_weights, cudaStream_t stream,
-                               int num_sms, int smem_cap) {
+                               int num_sms, int smem_cap, int force_s) {
   if (N > (int64_t)1 << 30 || K > (int64_t)1 << 30) return cudaErrorNotSupported;
   GdParams p = {};
   p.signs = signs;
@@ -727,14 +730,14 @@ cudaError_t launch_gemv_direct(const uint32_t* signs, const uint16_t* scales, in
   p.NG = static_cast<int>(K / 128);
   p.early = static_weights ? 1 : 0;
   switch (B) {
-    case 1: return launch_gemv_direct_nb<1>(p, stream, num_sms, smem_cap);
-    case 2: return launch_gemv_direct_nb<2>(p, stream, num_sms, smem_cap);
-    case 3: return launch_gemv_direct_nb<3>(p, stream, num_sms, smem_cap);
-    case 4: return launch_gemv_direct_nb<4>(p, stream, num_sms, smem_cap);
-    case 5: return launch_gemv_direct_nb<5>(p, stream, num_sms, smem_cap);
-    case 6: return launch_gemv_direct_nb<6>(p, stream, num_sms, smem_cap);
-    case 7: return launch_gemv_direct_nb<7>(p, stream, num_sms, smem_cap);
-    default: return launch_gemv_direct_nb<8>(p, stream, num_sms, smem_cap);
+    case 1: return launch_gemv_direct_nb<1>(p, stream, num_sms, smem_cap, force_s);
+    case 2: return launch_gemv_direct_nb<2>(p, stream, num_sms, smem_cap, force_s);
+    case 3: return launch_gemv_direct_nb<3>(p, stream, num_sms, smem_cap, force_s);
+    case 4: return launch_gemv_direct_nb<4>(p, stream, num_sms, smem_cap, force_s);
+    case 5: return launch_gemv_direct_nb<5>(p, stream, num_sms, smem_cap, force_s);
+    case 6: return launch_gemv_direct_nb<6>(p, stream, num_sms, smem_cap, force_s);
+    case 7: return launch_gemv_direct_nb<7>(p, stream, num_sms, smem_cap, force_s);
+    default: return launch_gemv_direct_nb<8>(p, stream, num_sms, smem_cap, force_s);
   }
 }
 

@@ -447,9 +447,10 @@ static std::mutex g_tc_plan_mu;
 
 // Cached plan lookup; false when the shape is outside this kernel's limits.
 template <int NB>
-static bool gemv_tc_cached_plan(int N, int NG, int num_sms, GemvTcPlan* out) {
-  int force = 0;
-  if (const char* f = getenv("W1_GEMV_SPLIT")) force = atoi(f);  // tuning knob: force the K split
+static bool gemv_tc_cached_plan(int N, int NG, int num_sms, int force_s, GemvTcPlan* out) {
+  int force = force_s;
+  if (!force)
+    if (const char* f = getenv("W1_GEMV_SPLIT")) force = atoi(f);  // tuning knob: force the K split
   if (force != 1 && force != 2 && force != 4 && force != 8) force = 0;
   int dev = 0;
   cudaGetDevice(&dev);
@@ -473,9 +474,9 @@ static bool gemv_tc_cached_plan(int N, int NG, int num_sms, GemvTcPlan* out) {
 }
 
 template <int NB>
-static cudaError_t launch_gemv_tc_nb(const GemvTcParams& base, cudaStream_t stream, int num_sms) {
+static cudaError_t launch_gemv_tc_nb(const GemvTcParams& base, cudaStream_t stream, int num_sms, int force_s) {
   GemvTcPlan plan;
-  if (!gemv_tc_cached_plan<NB>(base.N, base.NG, num_sms, &plan)) return cudaErrorNotSupported;
+  if (!gemv_tc_cached_plan<NB>(base.N, base.NG, num_sms, force_s, &plan)) return cudaErrorNotSupported;
   if (getenv("W1_VERBOSE"))
     fprintf(stderr, "w1_gemv(tc) plan: N=%d NG=%d B=%d -> clusters=%d split=%d groups=%d smem=%d\n", base.N,
             base.NG, NB, plan.Q, plan.S, plan.max_ng, plan.smem);
@@ -504,7 +505,7 @@ static cudaError_t launch_gemv_tc_nb(const GemvTcParams& base, cudaStream_t stre
 // Returns cudaErrorNotSupported when the shape is outside this kernel's plan
 // (the caller then uses the mma.sync kernel).
 cudaError_t launch_gemv_tc(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t K, const uint16_t* x,
-                           int B, float* y, cudaStream_t stream, int num_sms) {
+                           int B, float* y, cudaStream_t stream, int num_sms, int force_s) {
   if (N > (int64_t)1 << 30) return cudaErrorNotSupported;
   GemvTcParams p = {};
   p.signs = signs;
@@ -515,14 +516,14 @@ cudaError_t launch_gemv_tc(const uint32_t* signs, const uint16_t* scales, int64_
   p.K = static_cast<int>(K);
   p.NG = static_cast<int>(K / 128);
   switch (B) {
-    case 1: return launch_gemv_tc_nb<1>(p, stream, num_sms);
-    case 2: return launch_gemv_tc_nb<2>(p, stream, num_sms);
-    case 3: return launch_gemv_tc_nb<3>(p, stream, num_sms);
-    case 4: return launch_gemv_tc_nb<4>(p, stream, num_sms);
-    case 5: return launch_gemv_tc_nb<5>(p, stream, num_sms);
-    case 6: return launch_gemv_tc_nb<6>(p, stream, num_sms);
-    case 7: return launch_gemv_tc_nb<7>(p, stream, num_sms);
-    default: return launch_gemv_tc_nb<8>(p, stream, num_sms);
+    case 1: return launch_gemv_tc_nb<1>(p, stream, num_sms, force_s);
+    case 2: return launch_gemv_tc_nb<2>(p, stream, num_sms, force_s);
+    case 3: return launch_gemv_tc_nb<3>(p, stream, num_sms, force_s);
+    case 4: return launch_gemv_tc_nb<4>(p, stream, num_sms, force_s);
+    case 5: return launch_gemv_tc_nb<5>(p, stream, num_sms, force_s);
+    case 6: return launch_gemv_tc_nb<6>(p, stream, num_sms, force_s);
+    case 7: return launch_gemv_tc_nb<7>(p, stream, num_sms, force_s);
+    default: return launch_gemv_tc_nb<8>(p, stream, num_sms, force_s);
   }
 }
 

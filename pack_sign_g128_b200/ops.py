@@ -90,6 +90,14 @@ def _aligned256(ws: torch.Tensor) -> int:
     return (p + 255) // 256 * 256
 
 
+def gemv_choice(N: int, K: int, B: int, static_weights: bool = False) -> str:
+    """The kernel/K split w1_gemv chose for this shape ("" before the first call)."""
+    buf = ctypes.create_string_buffer(64)
+    st = _lib.call("w1_gemv_choice", N, K, B, W1_GEMV_STATIC_WEIGHTS if static_weights else 0, buf, 64)
+    _lib.check(st, "w1_gemv_choice")
+    return buf.value.decode()
+
+
 def w1_gemm(signs: torch.Tensor, scales: torch.Tensor, x: torch.Tensor, y: torch.Tensor | None = None,
             stream=None, workspace: torch.Tensor | None = None) -> torch.Tensor:
     """y [M, N] fp32 = x [M, K] bf16 times the 1-bit matrix (prefill).

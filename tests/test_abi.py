@@ -55,6 +55,10 @@ def test_host_side_argument_errors(lib):
     assert lib.w1_gemv(good, None, 16, 128, good, 1, good, None) == _lib.W1_ERR_NULL
     assert lib.w1_gemv(good, good, 16, 130, good, 1, good, None) == _lib.W1_ERR_SHAPE
     assert lib.w1_gemv(good, good, 16, 128, odd, 1, good, None) == _lib.W1_ERR_ALIGN
+    buf = ctypes.create_string_buffer(32)
+    assert lib.w1_gemv_choice(16, 128, 1, 0, None, 32) == _lib.W1_ERR_NULL
+    assert lib.w1_gemv_choice(16, 100, 1, 0, buf, 32) == _lib.W1_ERR_SHAPE
+    assert lib.w1_gemv_choice(16, 128, 9, 0, buf, 32) == _lib.W1_ERR_SHAPE
     assert lib.w1_gemm(good, good, 16, 128, good, 0, good, good, 1 << 30, None) == _lib.W1_ERR_SHAPE
     assert lib.w1_gemm(good, good, 16, 128, good, 4, None, good, 1 << 30, None) == _lib.W1_ERR_NULL
     need = lib.w1_gemm_workspace_size(4, 128)
