@@ -309,7 +309,7 @@ static cudaError_t launch_gemv_nb(const uint32_t* signs, const GemvParams& base,
 }
 
 cudaError_t launch_gemv_tc(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t K, const uint16_t* x,
-                           int B, float* y, cudaStream_t stream, int num_sms, int force_s);
+                           int B, float* y, bool static_weights, cudaStream_t stream, int num_sms, int force_s);
 cudaError_t launch_gemv_direct(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t K,
                                const uint16_t* x, int B, float* y, bool static_weights, cudaStream_t stream,
                                int num_sms, int smem_cap, int force_s);
@@ -385,7 +385,7 @@ static cudaError_t run_gemv_choice(const GemvChoice& c, const uint32_t* signs, c
     case 'd':
       return launch_gemv_direct(signs, scales, N, K, x, B, y, static_weights, stream, num_sms, smem_cap, c.s);
     case 't':
-      return launch_gemv_tc(signs, scales, N, K, x, B, y, stream, num_sms, c.s);
+      return launch_gemv_tc(signs, scales, N, K, x, B, y, static_weights, stream, num_sms, c.s);
     default:
       return launch_gemv_ring(signs, scales, N, K, x, B, y, stream, num_sms, smem_cap);
   }

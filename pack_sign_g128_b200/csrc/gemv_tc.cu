@@ -63,11 +63,12 @@ struct GemvTcParams {
   int N, K, NG;
   int S;       // cluster size (K split)
   int max_ng;  // max groups per CTA
+  int early;   // read weights before the grid dependency wait
 };
 
 template <int NB>
 struct GemvTcSmem {
-  int xb, xsum, xf, part, bars, total;
+  int xb, xsum, xf, part, inbox, bars, total;
 };
 
 template <int NB>
@@ -84,6 +85,8 @@ __host__ __device__ inline GemvTcSmem<NB> gemv_tc_layout(int max_ng) {
   off = (off + 15) / 16 * 16;
   L.part = off;
   off += 4 * NB * 128 * 4;
+  L.inbox = off;  // cluster reduction: [S][NB][ceil(rows / S)] floats, S x ceil(128 / S) <= 136
+  off += NB * 136 * 4;
   off = (off + 7) / 8 * 8;
   L.bars = off;
   off += 4 * 8 + 16;
@@ -124,6 +127,7 @@ __global__ void __launch_bounds__(gtc::kThreads, 1) gemv_tc_kernel(const GemvTcP
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(a_ready + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (p.S > 1) cluster_arrive_relaxed();  // matched by the wait before the first remote store
   const int crank = static_cast<int>(cluster_ctarank());
   const int q = static_cast<int>(cluster_id_x()), Q = static_cast<int>(nclusters_x());
   // rows of this cluster, groups of this CTA
@@ -149,8 +153,10 @@ __global__ void __launch_bounds__(gtc::kThreads, 1) gemv_tc_kernel(const GemvTcP
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  pdl_wait();
-  pdl_launch_dependents();
+  if (!p.early) {
+    pdl_wait();
+    pdl_launch_dependents();
+  }
 
   // ---- worker identity: TMEM lane quarter lq, K part kp; row rr = 32 lq + lane
   const int lq = warp & 3, kp = warp >> 2;
@@ -174,6 +180,10 @@ __global__ void __launch_bounds__(gtc::kThreads, 1) gemv_tc_kernel(const GemvTcP
     load_words(r, wv[r]);
     load_scale(r, sv[r]);
   }
+  if (p.early) {  // weights were written before the previous kernel began (W1_GEMV_STATIC_WEIGHTS)
+    pdl_wait();
+    pdl_launch_dependents();
+  }
 
   // ---- activations -> int8 digit tiles (B operand) in shared memory
   {
@@ -187,25 +197,28 @@ __global__ void __launch_bounds__(gtc::kThreads, 1) gemv_tc_kernel(const GemvTcP
     }
     const int sub = lane & 7, t = sub >> 1, hh = sub & 1;
     const int items = NB * ng;
-    for (int base = warp * 4; base < items; base += (gtc::kThreads / 32) * 4) {
-      const int item = base + (lane >> 3);
+    // item = (batch row b, group gl): 8 lanes x 16 elements.  Two items per
+    // lane in flight: the next item's loads are issued before this one's math.
+    auto load_item = [&](int item, uint4 (&u)[2]) {
+      u[0] = make_uint4(0, 0, 0, 0);
+      u[1] = make_uint4(0, 0, 0, 0);
+      if (item < items) {
+        const int b = item / ng, gl = item - b * ng;
+        const uint16_t* xp = p.x + static_cast<int64_t>(b) * p.K + 128 * (g0 + gl) + 32 * t + 16 * hh;
+        u[0] = *reinterpret_cast<const uint4*>(xp);
+        u[1] = *reinterpret_cast<const uint4*>(xp + 8);
+      }
+    };
+    auto process = [&](const uint4 (&u)[2], int item) {
       const bool valid = item < items;
       const int b = valid ? item / ng : 0;
       const int gl = valid ? item - b * ng : 0;
       float v[16];
-      if (valid) {
-        const uint16_t* xp = p.x + static_cast<int64_t>(b) * p.K + 128 * (g0 + gl) + 32 * t + 16 * hh;
-        const uint4 u0 = *reinterpret_cast<const uint4*>(xp);
-        const uint4 u1 = *reinterpret_cast<const uint4*>(xp + 8);
-        const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+      const uint32_t w[8] = {u[0].x, u[0].y, u[0].z, u[0].w, u[1].x, u[1].y, u[1].z, u[1].w};
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          v[2 * i] = __uint_as_float(w[i] << 16);
-          v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) v[i] = 0.f;
+      for (int i = 0; i < 8; ++i) {
+        v[2 * i] = __uint_as_float(w[i] << 16);
+        v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
       }
       float mx = 0.f;
 #pragma unroll
@@ -257,6 +270,17 @@ __global__ void __launch_bounds__(gtc::kThreads, 1) gemv_tc_kernel(const GemvTcP
           }
         }
       }
+    };
+    constexpr int kStep = (gtc::kThreads / 32) * 4;  // items per pass of the CTA
+    const int i0 = warp * 4 + (lane >> 3);
+    uint4 xa[2], xb[2];
+    load_item(i0, xa);
+    for (int j = 0; warp * 4 + j * kStep < items; j += 2) {  // trip count uniform per warp
+      load_item(i0 + (j + 1) * kStep, xb);
+      process(xa, i0 + j * kStep);
+      if (warp * 4 + (j + 1) * kStep >= items) break;
+      load_item(i0 + (j + 2) * kStep, xa);
+      process(xb, i0 + (j + 1) * kStep);
     }
   }
   fence_async_shared();
@@ -345,33 +369,42 @@ __global__ void __launch_bounds__(gtc::kThreads, 1) gemv_tc_kernel(const GemvTcP
     for (int b = 0; b < NB; ++b) part[(kp * NB + b) * 128 + rr] = acc[b];
   }
   tc_fence_before();
-  if (p.S > 1) cluster_sync(); else __syncthreads();
+  __syncthreads();  // every partial written; every MMA complete (the workers waited for them)
   tc_fence_after();
   if (warp == gtc::kCtl) tmem_dealloc(tmem, C::COLS);
-  // ---- reduce: 4 K parts x S CTAs, fixed order; CTA c stores its share of rows
-  {
-    const int lo = (crank * R) / p.S, hi = ((crank + 1) * R) / p.S, span = hi - lo;
-    const uint32_t pbase = smem_u32(part);
-    for (int i = threadIdx.x; i < span * NB; i += gtc::kThreads) {
-      const int b = i / span, r = lo + (i - b * span);
+  // ---- reduce: the 4 K parts here (fixed order), then the S CTAs of the
+  // cluster: each CTA stores its per-row sums straight into the owning CTA's
+  // inbox (DSMEM) and one cluster barrier later the owner adds them in order.
+  if (p.S == 1) {
+    for (int i = threadIdx.x; i < R * NB; i += gtc::kThreads) {
+      const int b = i / R, r = i - b * R;
       float sum = 0.f;
-      if (p.S == 1) {
 #pragma unroll
-        for (int k4 = 0; k4 < 4; ++k4) sum += part[(k4 * NB + b) * 128 + r];
-      } else {
-        for (int c = 0; c < p.S; ++c) {
-          float vals[4];
-#pragma unroll
-          for (int k4 = 0; k4 < 4; ++k4)
-            vals[k4] = ld_dsmem_f32(map_shared_rank(pbase + static_cast<uint32_t>(((k4 * NB + b) * 128 + r) * 4), c));
-#pragma unroll
-          for (int k4 = 0; k4 < 4; ++k4) sum += vals[k4];
-        }
-      }
+      for (int k4 = 0; k4 < 4; ++k4) sum += part[(k4 * NB + b) * 128 + r];
       p.y[static_cast<int64_t>(b) * p.N + r0 + r] = sum;
     }
+  } else {
+    float* inbox = reinterpret_cast<float*>(smem + L.inbox);
+    const int chunk = (R + p.S - 1) / p.S;
+    cluster_wait();  // every CTA of the cluster has started (arrived at kernel entry)
+    for (int i = threadIdx.x; i < R * NB; i += gtc::kThreads) {
+      const int b = i / R, r = i - b * R;
+      float sum = 0.f;
+#pragma unroll
+      for (int k4 = 0; k4 < 4; ++k4) sum += part[(k4 * NB + b) * 128 + r];
+      const int owner = r / chunk, ro = r - owner * chunk;
+      const uint32_t local = smem_u32(inbox + (crank * NB + b) * chunk + ro);
+      st_dsmem_f32(map_shared_rank(local, static_cast<uint32_t>(owner)), sum);
+    }
+    cluster_sync();
+    const int lo = crank * chunk, hi = min(R, lo + chunk), span = hi - lo;
+    for (int i = threadIdx.x; i < span * NB; i += gtc::kThreads) {
+      const int b = i / span, ro = i - b * span;
+      float sum = 0.f;
+      for (int c = 0; c < p.S; ++c) sum += inbox[(c * NB + b) * chunk + ro];
+      p.y[static_cast<int64_t>(b) * p.N + r0 + lo + ro] = sum;
+    }
   }
-  if (p.S > 1) cluster_sync();
 }
 
 // ------------------------------------------------------------------ host side
@@ -505,7 +538,7 @@ static cudaError_t launch_gemv_tc_nb(const GemvTcParams& base, cudaStream_t stre
 // Returns cudaErrorNotSupported when the shape is outside this kernel's plan
 // (the caller then uses the mma.sync kernel).
 cudaError_t launch_gemv_tc(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t K, const uint16_t* x,
-                           int B, float* y, cudaStream_t stream, int num_sms, int force_s) {
+                           int B, float* y, bool static_weights, cudaStream_t stream, int num_sms, int force_s) {
   if (N > (int64_t)1 << 30) return cudaErrorNotSupported;
   GemvTcParams p = {};
   p.signs = signs;
@@ -515,6 +548,7 @@ cudaError_t launch_gemv_tc(const uint32_t* signs, const uint16_t* scales, int64_
   p.N = static_cast<int>(N);
   p.K = static_cast<int>(K);
   p.NG = static_cast<int>(K / 128);
+  p.early = static_weights ? 1 : 0;
   switch (B) {
     case 1: return launch_gemv_tc_nb<1>(p, stream, num_sms, force_s);
     case 2: return launch_gemv_tc_nb<2>(p, stream, num_sms, force_s);
