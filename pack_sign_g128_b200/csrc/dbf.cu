@@ -8,15 +8,18 @@
 // section 1 "The representation" and section 4: x_scaled = D_in x,
 // h = V x_scaled, h_scaled = D_mid h, y_core = U h_scaled, y = D_out y_core).
 //
-// Small batch (B <= 8): ONE kernel runs both binary products -- the joint
-// V-D_mid-U kernel with a grid-wide synchronisation that the DBF post
-// (section 7, "CUDA/HIP: a starting point") proposes for CUDA.  Each CTA
-//  1. bulk-copies its slices of BOTH sign matrices into shared memory at
-//     once, so U streams in while V . (b x) is computed;
-//  2. phase 1: cluster-split int8-MMA product (as w1_gemv, no group scales)
-//     on b (.) x, cluster reduction, h_scaled = mid (.) h -> workspace (fp32);
+// Small batch (B < 64, groups of up to 8 rows): ONE kernel runs both binary
+// products -- the joint V-D_mid-U kernel with a grid-wide synchronisation that
+// the DBF post (section 7, "CUDA/HIP: a starting point") proposes for CUDA --
+// built from the steps of the direct GEMV kernel (gemv_direct.cu).  Each CTA
+//  1. issues the asynchronous copies of its slices of BOTH sign matrices at
+//     once (two commit groups), so U streams in while V . (b x) is computed;
+//  2. phase 1: int8-MMA product of V with b (.) x (the column diagonal applied
+//     while quantising, exact in fp32), cluster reduction, h_scaled =
+//     mid (.) h -> workspace (fp32);
 //  3. grid barrier (bounded spin; on timeout W1_ERR_TIMEOUT, no hang);
-//  4. phase 2: the same product of U with h_scaled, y = a (.) (...).
+//  4. phase 2: the same product of U with h_scaled (read through L2), y =
+//     a (.) (...).
 // The intermediate stays fp32 (exact to 2^-24 relative), so the only
 // quantisation is the 23-bit fixed point of each product's input.
 #include <cstdint>
@@ -25,235 +28,143 @@
 #include <cstdlib>
 #include <mutex>
 
-#include "gemv_core.cuh"
+#include "w1_common.cuh"
 
 namespace w1 {
 
-struct DbfParams {
-  const uint16_t* a;    // [m] fp16
-  const uint16_t* mid;  // [r] fp16
-  const uint16_t* b;    // [n] fp16
-  const uint16_t* x;    // [B][n] bf16
-  float* y;             // [B][m]
-  float* h;             // [B][r] workspace: mid (.) (B2 . (b (.) x))
-  unsigned int* bar;    // workspace: grid barrier {count, generation}
-  int m, r, n;
-  int S, bw1, bw2;
-  int ns1, ns2;
-  int max_tiles1, max_tiles2, max_ng1, max_ng2;
-};
-
-struct DbfSmem {
-  int st1, sb1, st2, sb2, xq, zero, xsum, xf, part, bars, total;
+// Shared memory of the chain kernel: both products' per-warp regions (sign
+// words, scales), then the activation scratch, reduction buffer and cluster
+// inbox sized for the larger of the two.
+struct DbfdSmem {
+  int wb1, wb2, w1, w2, xs, red, part, total;
 };
 
 template <int NB>
-__host__ __device__ inline DbfSmem dbf_smem_layout(const DbfParams& p) {
-  using L = GemvLayout<NB>;
-  const int mng = p.max_ng1 > p.max_ng2 ? p.max_ng1 : p.max_ng2;
-  const int mt = p.max_tiles1 > p.max_tiles2 ? p.max_tiles1 : p.max_tiles2;
-  const int wp = gemv_wpt(p.max_tiles1) > gemv_wpt(p.max_tiles2) ? gemv_wpt(p.max_tiles1) : gemv_wpt(p.max_tiles2);
-  DbfSmem M;
-  int off = 0;
-  M.st1 = off;
-  M.sb1 = ((p.max_ng1 + p.bw1 - 1) / p.bw1) * 16 * 16 * p.bw1;
-  off += p.ns1 * M.sb1;
-  off = round_up(off, 1024);
-  M.st2 = off;
-  M.sb2 = ((p.max_ng2 + p.bw2 - 1) / p.bw2) * 16 * 16 * p.bw2;
-  off += p.ns2 * M.sb2;
-  off = round_up(off, 128);
-  M.xq = off;
-  off += mng * 4 * L::BLOCK;
-  off = round_up(off, 16);
-  M.zero = off;
-  off += 16;
-  M.xsum = off;
-  off += mng * NB * 4;
-  M.xf = off;
-  off += mng * NB * 4;
-  off = round_up(off, 16);
-  M.part = off;
-  off += wp * NB * mt * 16 * 4;
-  off = round_up(off, 8);
-  M.bars = off;
-  off += 2 * (p.ns1 + p.ns2) * 8;
-  M.total = round_up(off, 128) + 1024;
+__host__ __device__ inline DbfdSmem dbfd_layout(const GdParams& p1, const GdParams& p2) {
+  using C = gd::Cfg<NB>;
+  const GdSmem L1 = gd_layout<NB>(p1.Tw, p1.NSw, p1.P, p1.S, p1.chunk, p1.NSc);
+  const GdSmem L2 = gd_layout<NB>(p2.Tw, p2.NSw, p2.P, p2.S, p2.chunk, p2.NSc);
+  DbfdSmem M;
+  M.wb1 = L1.warp_bytes;
+  M.wb2 = L2.warp_bytes;
+  M.w1 = 0;
+  M.w2 = gd::kWarps * M.wb1;
+  M.xs = M.w2 + gd::kWarps * M.wb2;
+  const int nsc = p1.NSc > p2.NSc ? p1.NSc : p2.NSc;
+  M.red = M.xs + (nsc * C::SCR * 4 + 15) / 16 * 16;
+  const int tw = p1.Tw > p2.Tw ? p1.Tw : p2.Tw;
+  M.part = M.red + gd::kWarps * tw * 16 * C::MT * 8 * 4;
+  const int chunk = p1.chunk > p2.chunk ? p1.chunk : p2.chunk;
+  M.total = M.part + (p1.S > 1 ? p1.S * NB * chunk * 4 : 0);
   return M;
 }
 
-// Grid-wide barrier over all CTAs of the launch (all co-resident by
-// construction of the grid).  bar[0] counts arrivals, bar[1] is the
-// generation; the last arrival resets the count, so the state is reusable by
-// the next call.  Returns false (and records W1_ERR_TIMEOUT) if the other
-// CTAs do not arrive within the spin limit.
-__device__ inline bool grid_barrier(unsigned int* bar, unsigned int nblocks) {
-  __syncthreads();
-  int ok = 1;
-  if (threadIdx.x == 0) {
-    __threadfence();
-    unsigned int gen;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(gen) : "l"(bar + 1) : "memory");
-    const unsigned int arrived = atomicAdd(bar, 1u);
-    if (arrived == nblocks - 1) {
-      atomicExch(bar, 0u);
-      __threadfence();
-      atomicAdd(bar + 1, 1u);
-    } else {
-      ok = 0;
-      for (uint32_t i = 0; i < kSpinLimit; ++i) {
-        unsigned int g;
-        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(g) : "l"(bar + 1) : "memory");
-        if (g != gen) {
-          ok = 1;
-          break;
-        }
-        __nanosleep(128);
-      }
-      if (!ok) set_status(W1_ERR_TIMEOUT);
-    }
-    __threadfence();
-  }
-  return __syncthreads_and(ok) != 0;
-}
-
 template <int NB>
-__global__ void __launch_bounds__(kGemvThreads, 1)
-    dbf_small_kernel(const __grid_constant__ CUtensorMap tm2, const __grid_constant__ CUtensorMap tm1,
-                     const DbfParams p) {
-  extern __shared__ unsigned char smem_raw[];
-  unsigned char* smem =
-      reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const DbfSmem M = dbf_smem_layout<NB>(p);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + M.bars);
-  GemvSmemView v1{smem + M.st1, p.ns1, M.sb1, bars, bars + p.ns1};
-  GemvSmemView v2{smem + M.st2, p.ns2, M.sb2, bars + 2 * p.ns1, bars + 2 * p.ns1 + p.ns2};
-  GemvXView xv;
-  xv.xq = smem + M.xq;
-  xv.xsum = reinterpret_cast<int*>(smem + M.xsum);
-  xv.xf = reinterpret_cast<float*>(smem + M.xf);
-  xv.sc = nullptr;
-  xv.part = reinterpret_cast<float*>(smem + M.part);
-  xv.part_stride = (p.max_tiles1 > p.max_tiles2 ? p.max_tiles1 : p.max_tiles2) * 16;
-  unsigned char* zero16 = smem + M.zero;
-
+__global__ void __launch_bounds__(gd::kThreads, 1) dbf_direct_kernel(const GdParams p1, const GdParams p2,
+                                                                     unsigned int* bar) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  const DbfdSmem M = dbfd_layout<NB>(p1, p2);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int crank = static_cast<int>(cluster_ctarank());
-  const int q = static_cast<int>(cluster_id_x()), Q = static_cast<int>(nclusters_x());
-  // rows of V with K = n, then rows of U with K = r
-  const Split sp1 = make_split(p.r, 0, p.n >> 7, p.S, crank, q, Q, p.bw1, p.bw1, p.max_tiles1);
-  const Split sp2 = make_split(p.m, 0, p.r >> 7, p.S, crank, q, Q, p.bw2, p.bw2, p.max_tiles2);
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < p.ns1; ++s) {
-      mbar_init(&v1.full[s], 1);
-      mbar_init(&v1.empty[s], static_cast<uint32_t>(sp1.wpt));
-    }
-    for (int s = 0; s < p.ns2; ++s) {
-      mbar_init(&v2.full[s], 1);
-      mbar_init(&v2.empty[s], static_cast<uint32_t>(sp2.wpt));
-    }
-    fence_mbarrier_init();
-    asm volatile("prefetch.tensormap [%0];" ::"l"(&tm2) : "memory");
-    asm volatile("prefetch.tensormap [%0];" ::"l"(&tm1) : "memory");
-  }
-  if (threadIdx.x < 4) reinterpret_cast<uint32_t*>(zero16)[threadIdx.x] = 0u;
-  __syncthreads();
+  unsigned char* wr1 = smem + M.w1 + warp * M.wb1;
+  unsigned char* wr2 = smem + M.w2 + warp * M.wb2;
+  const GdSmem L1 = gd_layout<NB>(p1.Tw, p1.NSw, p1.P, p1.S, p1.chunk, p1.NSc);
+  const GdSmem L2 = gd_layout<NB>(p2.Tw, p2.NSw, p2.P, p2.S, p2.chunk, p2.NSc);
+  unsigned char* wts1 = wr1 + L1.wts;
+  float* scl1 = reinterpret_cast<float*>(wr1 + L1.scl);
+  unsigned char* wts2 = wr2 + L2.wts;
+  float* scl2 = reinterpret_cast<float*>(wr2 + L2.scl);
+  uint32_t* xs = reinterpret_cast<uint32_t*>(smem + M.xs);
+  float* red = reinterpret_cast<float*>(smem + M.red);
+  float* part = reinterpret_cast<float*>(smem + M.part);
+  if (p1.S > 1) cluster_arrive_relaxed();  // matched by the wait before phase 1's first remote store
+  const GdGeom g1 = gd_geom<NB>(p1, warp);
+  const GdGeom g2 = gd_geom<NB>(p2, warp);
   pdl_wait();
   pdl_launch_dependents();
-
-  int first1 = 0, first2 = 0;
-  if (warp == kProducerWarp && lane == 0) {
-    first1 = issue_first_tiles(v1, sp1, &tm2, p.bw1);
-    first2 = issue_first_tiles(v2, sp2, &tm1, p.bw2);
-  }
-  __syncwarp();
-
-  // ---- phase 1: h_scaled = mid (.) (V . (b (.) x))
+  // both sign matrices in flight at once: commit group 1 = V, group 2 = U
+  if (g1.busy) gd_stage<NB>(p1, g1, wts1, lane);
+  else cp_async_commit();
+  if (g2.busy) gd_stage<NB>(p2, g2, wts2, lane);
+  else cp_async_commit();
   {
-    const uint16_t* xb = p.x;
-    const uint16_t* bd = p.b;
-    const int n = p.n;
-    quantise_input<NB>(xv, sp1,
-                       [&](int bb, int k, float (&vv)[16]) {
-                         load16_bf16(xb + static_cast<int64_t>(bb) * n + k, vv);
-                         const uint4 d0 = *reinterpret_cast<const uint4*>(bd + k);
-                         const uint4 d1 = *reinterpret_cast<const uint4*>(bd + k + 8);
-                         const uint32_t dw[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
-#pragma unroll
-                         for (int i = 0; i < 8; ++i) {
-                           const __half2 hh = *reinterpret_cast<const __half2*>(&dw[i]);
-                           vv[2 * i] *= __low2float(hh);
-                           vv[2 * i + 1] *= __high2float(hh);
-                         }
-                       },
-                       kGemvThreads);
-    __syncthreads();
-    if (warp == kProducerWarp) {
-      if (lane == 0) produce_rest(v1, sp1, &tm2, p.bw1, first1);
-      __syncwarp();  // converge before the (cluster) barrier, which is .aligned
-    } else {
-      consume_tiles<NB, false>(v1, xv, sp1, p.bw1, zero16, warp, lane);
-    }
-    if (p.S > 1) cluster_sync(); else __syncthreads();
-    float* h = p.h;
-    const uint16_t* mid = p.mid;
-    const int r = p.r;
-    cluster_reduce<NB>(xv, sp1, p.S, crank,
-                       [&](int bb, int64_t row, float val) {
-                         h[static_cast<int64_t>(bb) * r + row] = __half2float(__ushort_as_half(mid[row])) * val;
-                       },
-                       kGemvThreads);
+    uint16_t sreg[kGdSpl];  // no group scales: every s = 1
+    gd_load_scales<NB>(p1, g1, 0, lane, sreg);
+    gd_finish_scales<NB>(p1, g1, lane, sreg, scl1);
+    gd_load_scales<NB>(p2, g2, 0, lane, sreg);
+    gd_finish_scales<NB>(p2, g2, lane, sreg, scl2);
   }
-  // ---- every CTA's h_scaled is in memory (and every peer is done with part)
-  if (!grid_barrier(p.bar, gridDim.x)) {
-    if (p.S > 1) cluster_sync();
+  // ---- phase 1: h_scaled = mid (.) (V . (b (.) x))
+  gd_prep_x<NB, false>(p1, g1, xs, warp, lane);
+  asm volatile("cp.async.wait_group 1;" ::: "memory");  // V landed (U may still be in flight)
+  __syncthreads();
+  gd_finish<NB>(p1, g1, wts1, scl1, xs, red, part, warp, lane, true);
+  // ---- every CTA's h_scaled is in memory, and every reader of this CTA's
+  // scratch and inbox is done with phase 1
+  if (!grid_barrier(bar, gridDim.x)) {
+    cp_async_wait_all();
+    if (p2.S > 1) cluster_sync();  // the one cluster barrier phase 2 would have taken
     return;
   }
   // ---- phase 2: y = a (.) (U . h_scaled)
-  {
-    const float* h = p.h;
-    const int r = p.r;
-    quantise_input<NB>(xv, sp2,
-                       [&](int bb, int k, float (&vv)[16]) {
-                         const float4* hp = reinterpret_cast<const float4*>(h + static_cast<int64_t>(bb) * r + k);
-#pragma unroll
-                         for (int i = 0; i < 4; ++i) {
-                           const float4 f = __ldcg(hp + i);
-                           vv[4 * i] = f.x;
-                           vv[4 * i + 1] = f.y;
-                           vv[4 * i + 2] = f.z;
-                           vv[4 * i + 3] = f.w;
-                         }
-                       },
-                       kGemvThreads);
-    __syncthreads();
-    if (warp == kProducerWarp) {
-      if (lane == 0) produce_rest(v2, sp2, &tm1, p.bw2, first2);
-      __syncwarp();
-    } else {
-      consume_tiles<NB, false>(v2, xv, sp2, p.bw2, zero16, warp, lane);
-    }
-    if (p.S > 1) cluster_sync(); else __syncthreads();
-    float* y = p.y;
-    const uint16_t* a = p.a;
-    const int m = p.m;
-    cluster_reduce<NB>(xv, sp2, p.S, crank,
-                       [&](int bb, int64_t row, float val) {
-                         y[static_cast<int64_t>(bb) * m + row] = __half2float(__ushort_as_half(a[row])) * val;
-                       },
-                       kGemvThreads);
-    if (p.S > 1) cluster_sync();
-  }
+  gd_prep_x<NB, true>(p2, g2, xs, warp, lane);
+  cp_async_wait_all();
+  __syncthreads();
+  gd_finish<NB>(p2, g2, wts2, scl2, xs, red, part, warp, lane, false);
 }
 
 // ------------------------------------------------------------------ host side
 
+// Plan of one product for a fixed cluster size S and cluster count Q (the chain
+// kernel needs both products on the same grid).  False if a cluster's rows do
+// not fit the warps.
 template <int NB>
-static int dbf_max_clusters(int S, int smem_bytes) {
+static bool dbfd_plan(int N, int NG, int S, int Q, GdParams* p) {
+  using C = gd::Cfg<NB>;
+  const int NT = (N + 7) / 8;
+  const int NS = (NG + C::G - 1) / C::G;
+  if (S > 1 && S > NS) return false;
+  const int nsc = (NS + S - 1) / S;
+  if (nsc > gd::kMaxSets) return false;
+  const int Tmax = (NT + Q - 1) / Q;
+  int Wn = 0;
+  for (int w = 1; w <= gd::kWarps; w *= 2)
+    if ((Tmax + w - 1) / w <= gd::kMaxTw) {
+      Wn = w;
+      break;
+    }
+  if (Wn == 0) return false;
+  auto lg2 = [](int v) {
+    int l = 0;
+    while ((1 << l) < v) ++l;
+    return l;
+  };
+  p->N = N;
+  p->NG = NG;
+  p->K = NG * 128;
+  p->S = S;
+  p->Q = Q;
+  p->NT = NT;
+  p->Wn = Wn;
+  p->Wg = gd::kWarps / Wn;
+  p->Tw = (Tmax + Wn - 1) / Wn;
+  p->NSw = (nsc + p->Wg - 1) / p->Wg;
+  const int span = p->NSw * 16 * C::G;
+  p->P = ((span / (16 * C::G)) & 1) ? span : span + 16 * C::G;  // odd multiple: bank spread
+  p->chunk = (8 * Tmax + S - 1) / S;
+  p->NSc = nsc;
+  p->lgS = lg2(S);
+  p->lgWg = lg2(p->Wg);
+  p->lgGw = lg2(p->NSw * C::G);
+  p->tq = NT / Q;
+  p->tr = NT - p->tq * Q;
+  return true;
+}
+
+template <int NB>
+static int dbfd_max_clusters(int S, int smem_bytes) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(S * 64));
-  cfg.blockDim = dim3(kGemvThreads);
+  cfg.blockDim = dim3(gd::kThreads);
   cfg.dynamicSmemBytes = static_cast<size_t>(smem_bytes);
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -262,85 +173,101 @@ static int dbf_max_clusters(int S, int smem_bytes) {
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  int nclusters = 0;
-  if (cudaFuncSetAttribute(dbf_small_kernel<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes) !=
+  int n = 0;
+  if (cudaFuncSetAttribute(dbf_direct_kernel<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes) !=
           cudaSuccess ||
-      cudaOccupancyMaxActiveClusters(&nclusters, dbf_small_kernel<NB>, &cfg) != cudaSuccess) {
+      cudaOccupancyMaxActiveClusters(&n, dbf_direct_kernel<NB>, &cfg) != cudaSuccess) {
     cudaGetLastError();
     return 0;
   }
-  return nclusters;
+  return n;
 }
 
-static int dbf_bw(int NG, int S) { return (S == 1 || NG % (8 * S) == 0) ? 8 : 4; }
+// One group of up to 8 batch rows: the chain kernel on one grid whose CTAs are
+// all co-resident (the grid barrier); among the K splits whose shared memory
+// fits, the one with the least modelled per-CTA work (activation
+// quantisation ~24 instructions per element of a CTA's K range, ~0.6-1.5 per
+// weight, a fixed charge per cluster barrier; the GEMV planner's model).
+template <int NB>
+static double dbfd_cost(const GdParams& p) {
+  using C = gd::Cfg<NB>;
+  const double cw = NB <= 2 ? 0.6 : (NB <= 5 ? 1.0 : 1.5);
+  const int Tmax = (p.NT + p.Q - 1) / p.Q;
+  const double xprep = 24.0 * NB * 128.0 * C::G * p.NSc;
+  const double wts = 8.0 * Tmax * 128.0 * C::G * p.NSc * cw;
+  return (xprep + wts) / 128.0 + (p.S > 1 ? 800.0 : 0.0);
+}
 
 template <int NB>
-static cudaError_t launch_dbf_small_nb(DbfParams p, const uint32_t* B1, const uint32_t* B2, cudaStream_t stream,
-                                       int num_sms, int smem_cap) {
-  using L = GemvLayout<NB>;
-  // K split S (x digits within budget) and cluster count Q: all CTAs must be
-  // co-resident (grid barrier), so Q never exceeds the occupancy limit
-  const int T1 = (p.r + 15) / 16, T2 = (p.m + 15) / 16;
-  const int NG1 = p.n / 128, NG2 = p.r / 128;
+static cudaError_t launch_dbf_small_nb(const uint16_t* a, const uint32_t* B1, const uint16_t* mid,
+                                       const uint32_t* B2, const uint16_t* bd, int m, int r, int n,
+                                       const uint16_t* x, float* y, float* h, unsigned int* bar,
+                                       cudaStream_t stream, int num_sms, int smem_cap) {
+  GdParams best1 = {}, best2 = {};
+  int best_smem = 0;
+  double best_cost = 0.0;
   for (int S = 1; S <= 8; S *= 2) {
-    if (S > 1 && (S > NG1 || S > NG2)) break;
-    DbfParams c = p;
-    c.S = S;
-    c.bw1 = dbf_bw(NG1, S);
-    c.bw2 = dbf_bw(NG2, S);
-    c.max_ng1 = ((NG1 + c.bw1 - 1) / c.bw1 + S - 1) / S * c.bw1;
-    c.max_ng2 = ((NG2 + c.bw2 - 1) / c.bw2 + S - 1) / S * c.bw2;
-    const int mng = c.max_ng1 > c.max_ng2 ? c.max_ng1 : c.max_ng2;
-    if (mng * 4 * L::BLOCK > 72 * 1024 && S < 8) continue;
     int Q = num_sms / S;
-    for (int iter = 0; iter < 3; ++iter) {
-      c.max_tiles1 = (T1 + Q - 1) / Q;
-      c.max_tiles2 = (T2 + Q - 1) / Q;
-      c.ns1 = c.ns2 = 0;
-      const int base = dbf_smem_layout<NB>(c).total;
-      const int budget = smem_cap - base;
-      const int per1 = ((c.max_ng1 + c.bw1 - 1) / c.bw1) * 256 * c.bw1 + 16;
-      const int per2 = ((c.max_ng2 + c.bw2 - 1) / c.bw2) * 256 * c.bw2 + 16;
-      c.ns1 = c.max_tiles1;
-      c.ns2 = c.max_tiles2;
-      if (c.ns1 * per1 + c.ns2 * per2 > budget) {
-        c.ns1 = (budget / 2) / per1;
-        c.ns2 = (budget / 2) / per2;
-      }
-      if (c.ns1 < 1 || c.ns2 < 1) break;
-      const int smem = dbf_smem_layout<NB>(c).total;
-      const int occ = dbf_max_clusters<NB>(S, smem);
+    for (int iter = 0; iter < 4; ++iter) {
+      GdParams p1 = {}, p2 = {};
+      if (!dbfd_plan<NB>(r, n / 128, S, Q, &p1) || !dbfd_plan<NB>(m, r / 128, S, Q, &p2)) break;
+      const int smem = dbfd_layout<NB>(p1, p2).total;
+      if (smem > smem_cap) break;
+      const int occ = dbfd_max_clusters<NB>(S, smem);
       if (occ <= 0) break;
-      if (occ < Q) {
+      if (occ < Q) {  // every CTA must be resident for the grid barrier
         Q = occ;
         continue;
       }
-      CUtensorMap tm2, tm1;
-      if (!make_tmap_u32_rows(&tm2, B2, c.r, c.n / 32, 4 * c.bw1) ||
-          !make_tmap_u32_rows(&tm1, B1, c.m, c.r / 32, 4 * c.bw2))
-        return cudaErrorInvalidValue;
-      cudaError_t err = cudaFuncSetAttribute(dbf_small_kernel<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-      if (err != cudaSuccess) return err;
-      if (getenv("W1_VERBOSE"))
-        fprintf(stderr, "dbf plan: B=%d -> clusters=%d split=%d stages=%d/%d smem=%d\n", NB, Q, S, c.ns1, c.ns2, smem);
-      cudaLaunchConfig_t cfg = {};
-      cfg.gridDim = dim3(static_cast<unsigned>(Q * S));
-      cfg.blockDim = dim3(kGemvThreads);
-      cfg.dynamicSmemBytes = static_cast<size_t>(smem);
-      cfg.stream = stream;
-      cudaLaunchAttribute attr[2];
-      attr[0].id = cudaLaunchAttributeClusterDimension;
-      attr[0].val.clusterDim.x = static_cast<unsigned>(S);
-      attr[0].val.clusterDim.y = 1;
-      attr[0].val.clusterDim.z = 1;
-      attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-      attr[1].val.programmaticStreamSerializationAllowed = 1;
-      cfg.attrs = attr;
-      cfg.numAttrs = 2;
-      return cudaLaunchKernelEx(&cfg, dbf_small_kernel<NB>, tm2, tm1, c);
+      const double cost = dbfd_cost<NB>(p1) + dbfd_cost<NB>(p2);
+      if (best_smem == 0 || cost < best_cost) {
+        best1 = p1;
+        best2 = p2;
+        best_smem = smem;
+        best_cost = cost;
+      }
+      break;
     }
   }
-  return cudaErrorInvalidConfiguration;
+  if (best_smem == 0) return cudaErrorInvalidConfiguration;
+  GdParams p1 = best1, p2 = best2;
+  const int smem = best_smem, S = p1.S, Q = p1.Q;
+  p1.signs = B2;
+  p1.x = x;
+  p1.cdiag = bd;
+  p1.rdiag = mid;
+  p1.y = h;
+  p2.signs = B1;
+  p2.x = h;
+  p2.x_f32 = 1;
+  p2.rdiag = a;
+  p2.y = y;
+  cudaError_t err =
+      cudaFuncSetAttribute(dbf_direct_kernel<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (err != cudaSuccess) return err;
+  if (getenv("W1_VERBOSE"))
+    fprintf(stderr, "dbf plan: B=%d -> clusters=%d split=%d warps=%dx%d / %dx%d smem=%d\n", NB, Q, S, p1.Wn,
+            p1.Wg, p2.Wn, p2.Wg, smem);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(Q * S));
+  cfg.blockDim = dim3(gd::kThreads);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[na].val.programmaticStreamSerializationAllowed = 1;
+  ++na;
+  if (S > 1) {
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = static_cast<unsigned>(S);
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = na;
+  return cudaLaunchKernelEx(&cfg, dbf_direct_kernel<NB>, p1, p2, bar);
 }
 
 size_t dbf_tc_workspace_bytes(int64_t r, int64_t n, int64_t B);
@@ -368,36 +295,64 @@ cudaError_t launch_dbf(const uint16_t* a, const uint32_t* B1, const uint16_t* mi
                        bool allow_tensor_path = true) {
   if (allow_tensor_path && B >= kDbfTensorMinBatch)
     return launch_dbf_tc(a, B1, mid, B2, b, m, r, n, x, B, y, workspace, stream, num_sms);
-  DbfParams p = {};
-  p.a = a;
-  p.mid = mid;
-  p.b = b;
-  p.bar = reinterpret_cast<unsigned int*>(workspace);
-  p.h = reinterpret_cast<float*>(static_cast<unsigned char*>(workspace) + 256);
-  p.m = static_cast<int>(m);
-  p.r = static_cast<int>(r);
-  p.n = static_cast<int>(n);
-  // batches of up to 8 rows through the fused small-batch kernel
+  unsigned int* bar = reinterpret_cast<unsigned int*>(workspace);
+  float* h = reinterpret_cast<float*>(static_cast<unsigned char*>(workspace) + 256);
+  // batches of up to 8 rows through a fused chain kernel: the direct core for
+  // groups of up to 4 rows, the ring core (dbf_ring.cu) above, as measured;
+  // W1_DBF_PATH=direct|ring forces one (testing knob)
+  const char* path = getenv("W1_DBF_PATH");
+  DbfParams rp = {};
+  rp.a = a;
+  rp.mid = mid;
+  rp.b = b;
+  rp.bar = bar;
+  rp.h = h;
+  rp.m = static_cast<int>(m);
+  rp.r = static_cast<int>(r);
+  rp.n = static_cast<int>(n);
   for (int64_t b0 = 0; b0 < B; b0 += 8) {
     const int nb = static_cast<int>((B - b0) < 8 ? (B - b0) : 8);
-    p.x = x + b0 * n;
-    p.y = y + b0 * m;
+    const uint16_t* xg = x + b0 * n;
+    float* yg = y + b0 * m;
+    const int im = static_cast<int>(m), ir = static_cast<int>(r), in = static_cast<int>(n);
+    const bool direct = path ? path[0] == 'd' : nb <= 4;
     cudaError_t err;
-    switch (nb) {
-      case 1: err = launch_dbf_small_nb<1>(p, B1, B2, stream, num_sms, smem_cap); break;
-      case 2: err = launch_dbf_small_nb<2>(p, B1, B2, stream, num_sms, smem_cap); break;
-      case 3: err = launch_dbf_small_nb<3>(p, B1, B2, stream, num_sms, smem_cap); break;
-      case 4: err = launch_dbf_small_nb<4>(p, B1, B2, stream, num_sms, smem_cap); break;
-      case 5: err = launch_dbf_small_nb<5>(p, B1, B2, stream, num_sms, smem_cap); break;
-      case 6: err = launch_dbf_small_nb<6>(p, B1, B2, stream, num_sms, smem_cap); break;
-      case 7: err = launch_dbf_small_nb<7>(p, B1, B2, stream, num_sms, smem_cap); break;
-      default: err = launch_dbf_small_nb<8>(p, B1, B2, stream, num_sms, smem_cap); break;
+    if (direct) {
+      switch (nb) {
+#define W1_DBF_CASE(NBV)                                                                                        \
+  case NBV:                                                                                                     \
+    err = launch_dbf_small_nb<NBV>(a, B1, mid, B2, b, im, ir, in, xg, yg, h, bar, stream, num_sms, smem_cap); \
+    break;
+        W1_DBF_CASE(1)
+        W1_DBF_CASE(2)
+        W1_DBF_CASE(3)
+        W1_DBF_CASE(4)
+        W1_DBF_CASE(5)
+        W1_DBF_CASE(6)
+        W1_DBF_CASE(7)
+        default:
+          err = launch_dbf_small_nb<8>(a, B1, mid, B2, b, im, ir, in, xg, yg, h, bar, stream, num_sms, smem_cap);
+          break;
+#undef W1_DBF_CASE
+      }
+    } else {
+      rp.x = xg;
+      rp.y = yg;
+      switch (nb) {
+        case 1: err = launch_dbf_ring_nb<1>(rp, B1, B2, stream, num_sms, smem_cap); break;
+        case 2: err = launch_dbf_ring_nb<2>(rp, B1, B2, stream, num_sms, smem_cap); break;
+        case 3: err = launch_dbf_ring_nb<3>(rp, B1, B2, stream, num_sms, smem_cap); break;
+        case 4: err = launch_dbf_ring_nb<4>(rp, B1, B2, stream, num_sms, smem_cap); break;
+        case 5: err = launch_dbf_ring_nb<5>(rp, B1, B2, stream, num_sms, smem_cap); break;
+        case 6: err = launch_dbf_ring_nb<6>(rp, B1, B2, stream, num_sms, smem_cap); break;
+        case 7: err = launch_dbf_ring_nb<7>(rp, B1, B2, stream, num_sms, smem_cap); break;
+        default: err = launch_dbf_ring_nb<8>(rp, B1, B2, stream, num_sms, smem_cap); break;
+      }
     }
     if (err != cudaSuccess) return err;
   }
   return cudaSuccess;
 }
-
 // ------------------------------------------------------------------ static scratch
 // Scratch for callers that cannot allocate device memory: a fixed array in the
 // library's own device image (every GPU that loads the library holds it until

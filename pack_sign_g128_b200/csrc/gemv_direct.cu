@@ -69,9 +69,12 @@ struct Cfg {
 
 struct GdParams {
   const uint32_t* signs;
-  const uint16_t* scales;
-  const uint16_t* x;
-  float* y;
+  const uint16_t* scales;  // fp16 group scales, or nullptr (every s = 1)
+  const void* x;           // [B][K] bf16, or fp32 with x_f32
+  const uint16_t* cdiag;   // fp16 [K] multiplied into x (bf16 x only), or nullptr
+  const uint16_t* rdiag;   // fp16 [N] multiplied into y, or nullptr
+  float* y;                // [B][N]
+  int x_f32;
   int N, K, NG;
   int S;      // CTAs per cluster (K split)
   int Q;      // clusters
@@ -301,138 +304,195 @@ __device__ __forceinline__ void gd_compute(const unsigned char* wts, int P, cons
   }
 }
 
+// ---- one product, split into device steps (the GEMV kernel runs one, the
+// DBF chain kernel two, with a grid barrier between them)
+
+// This CTA's share (cluster q's n-tiles, K sets [cs0, cs0 + nsc)) and this
+// warp's block of both.
+struct GdGeom {
+  int crank, cs0, nsc, t0c, Tq, wn, wg, tw, ws0, nsw, row0, nrows, g0, ngw;
+  bool busy;
+};
+
 template <int NB>
-__global__ void __launch_bounds__(gd::kThreads, 1) gemv_direct_kernel(const GdParams p) {
-  using C = gd::Cfg<NB>;
-  constexpr int G = C::G, MT = C::MT;
-  extern __shared__ __align__(16) unsigned char smem[];
+__device__ __forceinline__ GdGeom gd_geom(const GdParams& p, int warp) {
+  constexpr int G = gd::Cfg<NB>::G;
+  GdGeom g;
   const int NS = (p.NG + G - 1) / G;
-  const int crank = p.S > 1 ? static_cast<int>(cluster_ctarank()) : 0;
-  const int cs0 = (crank * NS) >> p.lgS, nsc = (((crank + 1) * NS) >> p.lgS) - cs0;
-  const GdSmem L = gd_layout<NB>(p.Tw, p.NSw, p.P, p.S, p.chunk, p.NSc);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  unsigned char* wreg = smem + warp * L.warp_bytes;
-  unsigned char* wts = wreg + L.wts;
-  float* scl = reinterpret_cast<float*>(wreg + L.scl);
-  uint32_t* xs = reinterpret_cast<uint32_t*>(smem + L.xs);
-
-  if (p.S > 1) cluster_arrive_relaxed();  // matched by the wait before the first remote store
-
-  // ---- this CTA: cluster q's n-tiles, K sets [cs0, cs0 + nsc); this warp: a block of both
+  g.crank = p.S > 1 ? static_cast<int>(cluster_ctarank()) : 0;
   const int q = p.S > 1 ? static_cast<int>(cluster_id_x()) : static_cast<int>(blockIdx.x);
-  const int t0c = q * p.tq + min(q, p.tr);              // NT = Q * tq + tr tiles, the first tr clusters one more
-  const int Tq = p.tq + (q < p.tr ? 1 : 0);
-  const int wn = warp >> p.lgWg, wg = warp & (p.Wg - 1);
-  const int tw = max(0, min(p.Tw, Tq - wn * p.Tw));        // n-tiles of this warp
-  const int ws0 = cs0 + ((wg * nsc) >> p.lgWg);             // first set of this warp
-  const int nsw = cs0 + (((wg + 1) * nsc) >> p.lgWg) - ws0;  // sets of this warp
-  const int row0 = (t0c + wn * p.Tw) * 8;                   // first weight row of this warp
-  const int nrows = max(0, min(8 * tw, p.N - row0));
-  const bool busy = tw > 0 && nsw > 0;
-  const int g0 = ws0 * G;                                    // first group of this warp
-  const int ngw = busy ? min(nsw * G, p.NG - g0) : 0;       // real groups of this warp
-  const int KW = p.K >> 5;                                   // words per weight row
-  const int lgw = p.lgGw, gmask = (1 << lgw) - 1;           // power-of-two stride over a row's groups
+  g.cs0 = (g.crank * NS) >> p.lgS;
+  g.nsc = (((g.crank + 1) * NS) >> p.lgS) - g.cs0;
+  g.t0c = q * p.tq + min(q, p.tr);  // NT = Q * tq + tr tiles, the first tr clusters one more
+  g.Tq = q < p.Q ? p.tq + (q < p.tr ? 1 : 0) : 0;
+  g.wn = warp >> p.lgWg;
+  g.wg = warp & (p.Wg - 1);
+  g.tw = max(0, min(p.Tw, g.Tq - g.wn * p.Tw));              // n-tiles of this warp
+  g.ws0 = g.cs0 + ((g.wg * g.nsc) >> p.lgWg);                 // first set of this warp
+  g.nsw = g.cs0 + (((g.wg + 1) * g.nsc) >> p.lgWg) - g.ws0;   // sets of this warp
+  g.row0 = (g.t0c + g.wn * p.Tw) * 8;                         // first weight row of this warp
+  g.nrows = max(0, min(8 * g.tw, p.N - g.row0));
+  g.busy = g.tw > 0 && g.nsw > 0;
+  g.g0 = g.ws0 * G;                                           // first group of this warp
+  g.ngw = g.busy ? min(g.nsw * G, p.NG - g.g0) : 0;           // real groups of this warp
+  return g;
+}
 
-  // ---- weight staging: 16-byte asynchronous copies, every lane, all up front
-  auto stage_weights = [&]() {
-    const int n = nrows << lgw;
-    for (int i = lane; i < n; i += 32) {
-      const int r = i >> lgw, g = i & gmask;
-      if (g < ngw)
-        cp_async16(wts + r * p.P + g * 16, p.signs + static_cast<int64_t>(row0 + r) * KW + 4 * (g0 + g));
-    }
-    cp_async_commit();
-  };
-  // ---- scales: plain loads now, converted and stored once the activations are in flight
-  constexpr int kSpl = 8;
-  const int sstride = 8 * p.Tw;                  // scl[group][row]
-  const int nscl = busy ? (8 * tw) << lgw : 0;   // rows x (power-of-two) groups
-  uint16_t sreg[kSpl];
-  auto load_scales = [&](int base) {
-#pragma unroll
-    for (int j = 0; j < kSpl; ++j) {
-      const int i = base + lane + 32 * j;
-      const int rl = i >> lgw, gl = i & gmask;
-      sreg[j] = 0;
-      if (i < nscl && gl < nsw * G && row0 + rl < p.N && g0 + gl < p.NG)
-        sreg[j] = __ldg(p.scales + static_cast<int64_t>(row0 + rl) * p.NG + g0 + gl);
-    }
-  };
-  auto store_scales = [&](int base) {
-#pragma unroll
-    for (int j = 0; j < kSpl; ++j) {
-      const int i = base + lane + 32 * j;
-      const int rl = i >> lgw, gl = i & gmask;
-      if (i < nscl && gl < nsw * G) scl[gl * sstride + rl] = __half2float(__ushort_as_half(sreg[j]));
-    }
-  };
-
-  if (p.early) {
-    stage_weights();
-    load_scales(0);
+// This warp's sign words -> shared memory: 16-byte asynchronous copies, every
+// lane, one commit group.
+template <int NB>
+__device__ __forceinline__ void gd_stage(const GdParams& p, const GdGeom& g, unsigned char* wts, int lane) {
+  const int lgw = p.lgGw, gmask = (1 << lgw) - 1;  // power-of-two stride over a row's groups
+  const int KW = p.K >> 5;
+  const int n = g.nrows << lgw;
+  for (int i = lane; i < n; i += 32) {
+    const int r = i >> lgw, gg = i & gmask;
+    if (gg < g.ngw)
+      cp_async16(wts + r * p.P + gg * 16, p.signs + static_cast<int64_t>(g.row0 + r) * KW + 4 * (g.g0 + gg));
   }
-  pdl_wait();
-  pdl_launch_dependents();
-  if (!p.early) {
-    stage_weights();
-    load_scales(0);
-  }
+  cp_async_commit();
+}
 
-  // ---- activations of the CTA's sets -> digit scratch.  Unit = (set, group j,
-  // batch b): 8 lanes x 16 elements; 32 units per pass of the CTA.
-  {
-    const int units = nsc * G * NB;
-    const int sub = lane & 7;
-    auto load_unit = [&](int u, uint4 (&r)[2]) {  // unit u of this CTA -> 16 bf16 of this lane
-      r[0] = make_uint4(0, 0, 0, 0);
-      r[1] = make_uint4(0, 0, 0, 0);
-      if (u < units) {
-        const int sl = u / (G * NB), gb = u - sl * (G * NB);
-        const int gj = gb / NB, b = gb - gj * NB;
-        const int g = (cs0 + sl) * G + gj;
-        if (g < p.NG) {
-          const uint4* src =
-              reinterpret_cast<const uint4*>(p.x + static_cast<int64_t>(b) * p.K + g * 128 + sub * 16);
+// Scales: plain loads into registers (issued early), converted and stored to
+// scl[group][row] later.  Without scales every value is 1.
+constexpr int kGdSpl = 8;
+template <int NB>
+__device__ __forceinline__ void gd_load_scales(const GdParams& p, const GdGeom& g, int base, int lane,
+                                               uint16_t (&sreg)[kGdSpl]) {
+  constexpr int G = gd::Cfg<NB>::G;
+  const int lgw = p.lgGw, gmask = (1 << lgw) - 1;
+  const int nscl = g.busy ? (8 * g.tw) << lgw : 0;
+#pragma unroll
+  for (int j = 0; j < kGdSpl; ++j) {
+    const int i = base + lane + 32 * j;
+    const int rl = i >> lgw, gl = i & gmask;
+    sreg[j] = 0;
+    if (i < nscl && gl < g.nsw * G && g.row0 + rl < p.N && g.g0 + gl < p.NG)
+      sreg[j] = p.scales ? __ldg(p.scales + static_cast<int64_t>(g.row0 + rl) * p.NG + g.g0 + gl)
+                         : static_cast<uint16_t>(0x3C00u);
+  }
+}
+template <int NB>
+__device__ __forceinline__ void gd_store_scales(const GdParams& p, const GdGeom& g, int base, int lane,
+                                                const uint16_t (&sreg)[kGdSpl], float* scl) {
+  constexpr int G = gd::Cfg<NB>::G;
+  const int lgw = p.lgGw, gmask = (1 << lgw) - 1;
+  const int nscl = g.busy ? (8 * g.tw) << lgw : 0;
+  const int sstride = 8 * p.Tw;
+#pragma unroll
+  for (int j = 0; j < kGdSpl; ++j) {
+    const int i = base + lane + 32 * j;
+    const int rl = i >> lgw, gl = i & gmask;
+    if (i < nscl && gl < g.nsw * G) scl[gl * sstride + rl] = __half2float(__ushort_as_half(sreg[j]));
+  }
+}
+// The first register batch is stored; longer K ranges load and store the rest.
+template <int NB>
+__device__ __forceinline__ void gd_finish_scales(const GdParams& p, const GdGeom& g, int lane,
+                                                 const uint16_t (&sreg)[kGdSpl], float* scl) {
+  if (!g.busy) return;
+  gd_store_scales<NB>(p, g, 0, lane, sreg, scl);
+  const int nscl = (8 * g.tw) << p.lgGw;
+  for (int base = 32 * kGdSpl; base < nscl; base += 32 * kGdSpl) {
+    uint16_t r2[kGdSpl];
+    gd_load_scales<NB>(p, g, base, lane, r2);
+    gd_store_scales<NB>(p, g, base, lane, r2, scl);
+  }
+}
+
+// The CTA's activations -> digit scratch.  Unit = (set, group j, batch b):
+// 8 lanes x 16 elements; 4 units per warp per pass, two passes in flight.
+// bf16 x (optionally times the fp16 column diagonal, exact in fp32) or fp32 x
+// (read through L2: it may have been written by other CTAs of this grid).
+template <int NB, bool XF32>
+__device__ __forceinline__ void gd_prep_x(const GdParams& p, const GdGeom& g, uint32_t* xs, int warp, int lane) {
+  using C = gd::Cfg<NB>;
+  constexpr int G = C::G;
+  const int units = g.nsc * G * NB;
+  const int sub = lane & 7;
+  auto load_unit = [&](int u, uint4 (&r)[4]) {  // unit u of this CTA -> this lane's 16 values (+ diagonal)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) r[i] = make_uint4(0, 0, 0, 0);
+    if (u < units) {
+      const int sl = u / (G * NB), gb = u - sl * (G * NB);
+      const int gj = gb / NB, b = gb - gj * NB;
+      const int gi = (g.cs0 + sl) * G + gj;
+      if (gi < p.NG) {
+        const int64_t k0 = static_cast<int64_t>(gi) * 128 + sub * 16;
+        if (XF32) {
+          const uint4* src = reinterpret_cast<const uint4*>(static_cast<const float*>(p.x) +
+                                                            static_cast<int64_t>(b) * p.K + k0);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) r[i] = __ldcg(src + i);
+        } else {
+          const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.x) +
+                                                            static_cast<int64_t>(b) * p.K + k0);
           r[0] = __ldg(src);
           r[1] = __ldg(src + 1);
+          if (p.cdiag) {
+            const uint4* dg = reinterpret_cast<const uint4*>(p.cdiag + k0);
+            r[2] = __ldg(dg);
+            r[3] = __ldg(dg + 1);
+          }
         }
       }
-    };
-    auto process = [&](const uint4 (&r)[2], int u) {
+    }
+  };
+  auto process = [&](const uint4 (&r)[4], int u) {
+    float v[16];
+    if (XF32) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        v[4 * i] = __uint_as_float(r[i].x);
+        v[4 * i + 1] = __uint_as_float(r[i].y);
+        v[4 * i + 2] = __uint_as_float(r[i].z);
+        v[4 * i + 3] = __uint_as_float(r[i].w);
+      }
+    } else {
       const uint32_t w[8] = {r[0].x, r[0].y, r[0].z, r[0].w, r[1].x, r[1].y, r[1].z, r[1].w};
-      float v[16];
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         v[2 * i] = __uint_as_float(w[i] << 16);
         v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
       }
-      const int sl = u / (G * NB);
-      const int it = (u - sl * (G * NB)) * 8 + sub;  // item index within the set
-      quantise_item<NB>(v, u < units, it, xs + sl * C::SCR);
-    };
-    // two passes per iteration: the loads of one pass overlap the other's math
-    const int u0 = warp * 4 + (lane >> 3);
-    uint4 xa[2], xb[2];
-    load_unit(u0, xa);
-    for (int u = u0; u - u0 < units; u += 64) {  // trip count uniform over the CTA
-      load_unit(u + 32, xb);
-      process(xa, u);
-      if (u - u0 + 32 >= units) break;
-      load_unit(u + 64, xa);
-      process(xb, u + 32);
+      if (p.cdiag) {
+        const uint32_t d[8] = {r[2].x, r[2].y, r[2].z, r[2].w, r[3].x, r[3].y, r[3].z, r[3].w};
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&d[i]));
+          v[2 * i] *= f.x;  // bf16 x fp16: exact in fp32
+          v[2 * i + 1] *= f.y;
+        }
+      }
     }
+    const int sl = u / (G * NB);
+    const int it = (u - sl * (G * NB)) * 8 + sub;  // item index within the set
+    quantise_item<NB>(v, u < units, it, xs + sl * C::SCR);
+  };
+  constexpr int kPass = 4 * gd::kWarps;  // units per pass of the CTA
+  const int u0 = warp * 4 + (lane >> 3);
+  uint4 xa[4], xb[4];
+  load_unit(u0, xa);
+  for (int u = u0; u - u0 < units; u += 2 * kPass) {  // trip count uniform over the CTA
+    load_unit(u + kPass, xb);
+    process(xa, u);
+    if (u - u0 + kPass >= units) break;
+    load_unit(u + 2 * kPass, xa);
+    process(xb, u + kPass);
   }
-  if (busy) {
-    store_scales(0);
-    for (int base = 32 * kSpl; base < nscl; base += 32 * kSpl) {  // long K ranges
-      load_scales(base);
-      store_scales(base);
-    }
-  }
-  cp_async_wait_all();
-  __syncthreads();
+}
 
+// Products, CTA reduction, cluster reduction and output:
+// y[b][row] = rdiag[row] * sum.  Call after the weights, scales and digits are
+// in shared memory (and a __syncthreads).  `wait_cluster`: wait on the
+// cluster barrier arrived at kernel entry before the first remote store.
+template <int NB>
+__device__ __forceinline__ void gd_finish(const GdParams& p, const GdGeom& g, const unsigned char* wts,
+                                          const float* scl, const uint32_t* xs, float* red, float* part, int warp,
+                                          int lane, bool wait_cluster) {
+  using C = gd::Cfg<NB>;
+  constexpr int G = C::G, MT = C::MT;
+  const int sstride = 8 * p.Tw;
   float acc[gd::kMaxTw][MT][4];
 #pragma unroll
   for (int t = 0; t < gd::kMaxTw; ++t)
@@ -440,29 +500,27 @@ __global__ void __launch_bounds__(gd::kThreads, 1) gemv_direct_kernel(const GdPa
     for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) acc[t][mt][e] = 0.f;
-  if (busy) {
-    const uint32_t* xw = xs + (ws0 - cs0) * C::SCR;
-    switch (tw) {  // warp-uniform
-      case 1: gd_compute<NB, 1>(wts, p.P, scl, sstride, xw, nsw, lane, acc); break;
-      case 2: gd_compute<NB, 2>(wts, p.P, scl, sstride, xw, nsw, lane, acc); break;
-      case 3: gd_compute<NB, 3>(wts, p.P, scl, sstride, xw, nsw, lane, acc); break;
-      default: gd_compute<NB, 4>(wts, p.P, scl, sstride, xw, nsw, lane, acc); break;
+  if (g.busy) {
+    const uint32_t* xw = xs + (g.ws0 - g.cs0) * C::SCR;
+    switch (g.tw) {  // warp-uniform
+      case 1: gd_compute<NB, 1>(wts, p.P, scl, sstride, xw, g.nsw, lane, acc); break;
+      case 2: gd_compute<NB, 2>(wts, p.P, scl, sstride, xw, g.nsw, lane, acc); break;
+      case 3: gd_compute<NB, 3>(wts, p.P, scl, sstride, xw, g.nsw, lane, acc); break;
+      default: gd_compute<NB, 4>(wts, p.P, scl, sstride, xw, g.nsw, lane, acc); break;
     }
   }
-
   // ---- CTA reduction: red[wg][tile][row r][n], tile = wn * Tw + t (CTA-local)
   const int r1 = lane >> 2, cq = lane & 3;
-  float* red = reinterpret_cast<float*>(smem + L.red);
   const int TT = p.Wn * p.Tw;  // tiles per CTA (max)
 #pragma unroll
   for (int t = 0; t < gd::kMaxTw; ++t) {
-    if (t < tw) {
+    if (t < g.tw) {
 #pragma unroll
       for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf) {
           const int r = 16 * mt + 8 * hf + r1;
-          *reinterpret_cast<float2*>(red + ((wg * TT + wn * p.Tw + t) * 16 * MT + r) * 8 + 2 * cq) =
+          *reinterpret_cast<float2*>(red + ((g.wg * TT + g.wn * p.Tw + t) * 16 * MT + r) * 8 + 2 * cq) =
               make_float2(acc[t][mt][2 * hf], acc[t][mt][2 * hf + 1]);
         }
     }
@@ -470,16 +528,15 @@ __global__ void __launch_bounds__(gd::kThreads, 1) gemv_direct_kernel(const GdPa
   __syncthreads();
   // per (b, row of this cluster): sum over the warps of the same tile (set
   // blocks, fixed order) and over the digit rows of batch b; then to the owning
-  // CTA (or straight to y when S = 1).  Warps with no sets wrote nothing: skip.
-  const int R8 = 8 * Tq;
-  float* part = reinterpret_cast<float*>(smem + L.part);
-  if (p.S > 1) cluster_wait();  // every CTA of the cluster has started
+  // CTA (or straight to y when S = 1).  Set blocks without sets are skipped.
+  const int R8 = 8 * g.Tq;
+  if (p.S > 1 && wait_cluster) cluster_wait();  // every CTA of the cluster has started
   for (int b = 0; b < NB; ++b) {
     for (int rl = threadIdx.x; rl < R8; rl += gd::kThreads) {
       const int tile = rl >> 3, n = rl & 7;
       float sum = 0.f;
       for (int g2 = 0; g2 < p.Wg; ++g2) {
-        const int s0 = cs0 + ((g2 * nsc) >> p.lgWg), s1 = cs0 + (((g2 + 1) * nsc) >> p.lgWg);
+        const int s0 = g.cs0 + ((g2 * g.nsc) >> p.lgWg), s1 = g.cs0 + (((g2 + 1) * g.nsc) >> p.lgWg);
         if (s1 <= s0) continue;
         const float* rp = red + ((g2 * TT + tile) * 16 * MT) * 8 + n;
 #pragma unroll
@@ -487,29 +544,62 @@ __global__ void __launch_bounds__(gd::kThreads, 1) gemv_direct_kernel(const GdPa
 #pragma unroll
           for (int pp = 0; pp < 3; ++pp) sum += rp[((gj * NB + b) * 3 + pp) * 8];
       }
-      const int row = t0c * 8 + rl;
+      const int row = g.t0c * 8 + rl;
       if (p.S == 1) {
-        if (row < p.N) p.y[static_cast<int64_t>(b) * p.N + row] = sum;
+        if (row < p.N)
+          p.y[static_cast<int64_t>(b) * p.N + row] = p.rdiag ? __half2float(__ushort_as_half(p.rdiag[row])) * sum : sum;
       } else {
         int owner = 0;
         while (owner + 1 < p.S && rl >= (owner + 1) * p.chunk) ++owner;
-        const uint32_t local = smem_u32(part + (crank * NB + b) * p.chunk + (rl - owner * p.chunk));
+        const uint32_t local = smem_u32(part + (g.crank * NB + b) * p.chunk + (rl - owner * p.chunk));
         st_dsmem_f32(map_shared_rank(local, static_cast<uint32_t>(owner)), sum);
       }
     }
   }
   if (p.S > 1) {
     cluster_sync();
-    const int lo = crank * p.chunk, hi = min(R8, lo + p.chunk);
+    const int lo = g.crank * p.chunk, hi = min(R8, lo + p.chunk);
     for (int b = 0; b < NB; ++b) {
       for (int ro = threadIdx.x; ro < hi - lo; ro += gd::kThreads) {
         float sum = 0.f;
         for (int c = 0; c < p.S; ++c) sum += part[(c * NB + b) * p.chunk + ro];
-        const int row = t0c * 8 + lo + ro;
-        if (row < p.N) p.y[static_cast<int64_t>(b) * p.N + row] = sum;
+        const int row = g.t0c * 8 + lo + ro;
+        if (row < p.N)
+          p.y[static_cast<int64_t>(b) * p.N + row] = p.rdiag ? __half2float(__ushort_as_half(p.rdiag[row])) * sum : sum;
       }
     }
   }
+}
+
+template <int NB>
+__global__ void __launch_bounds__(gd::kThreads, 1) gemv_direct_kernel(const GdParams p) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  const GdSmem L = gd_layout<NB>(p.Tw, p.NSw, p.P, p.S, p.chunk, p.NSc);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  unsigned char* wreg = smem + warp * L.warp_bytes;
+  unsigned char* wts = wreg + L.wts;
+  float* scl = reinterpret_cast<float*>(wreg + L.scl);
+  uint32_t* xs = reinterpret_cast<uint32_t*>(smem + L.xs);
+  if (p.S > 1) cluster_arrive_relaxed();  // matched by the wait before the first remote store
+  const GdGeom g = gd_geom<NB>(p, warp);
+  uint16_t sreg[kGdSpl];
+  if (p.early) {
+    if (g.busy) gd_stage<NB>(p, g, wts, lane);
+    gd_load_scales<NB>(p, g, 0, lane, sreg);
+  }
+  pdl_wait();
+  pdl_launch_dependents();
+  if (!p.early) {
+    if (g.busy) gd_stage<NB>(p, g, wts, lane);
+    gd_load_scales<NB>(p, g, 0, lane, sreg);
+  }
+  if (p.x_f32) gd_prep_x<NB, true>(p, g, xs, warp, lane);
+  else gd_prep_x<NB, false>(p, g, xs, warp, lane);
+  gd_finish_scales<NB>(p, g, lane, sreg, scl);
+  cp_async_wait_all();
+  __syncthreads();
+  gd_finish<NB>(p, g, wts, scl, xs, reinterpret_cast<float*>(smem + L.red), reinterpret_cast<float*>(smem + L.part),
+                warp, lane, true);
 }
 
 // ------------------------------------------------------------------ host side
@@ -716,6 +806,7 @@ cudaError_t launch_gemv_direct(const uint32_t* signs, const uint16_t* scales, in
   p.scales = scales;
   p.x = x;
   p.y = y;
+  p.x_f32 = 0;
   p.N = static_cast<int>(N);
   p.K = static_cast<int>(K);
   p.NG = static_cast<int>(K / 128);

@@ -169,6 +169,42 @@ __device__ __forceinline__ float ld_dsmem_f32(uint32_t addr) {
   return v;
 }
 
+// ---------------------------------------------------------------- grid barrier
+// Grid-wide barrier over all CTAs of the launch (all co-resident by
+// construction of the grid).  bar[0] counts arrivals, bar[1] is the
+// generation; the last arrival resets the count, so the state is reusable by
+// the next call.  Returns false (and records W1_ERR_TIMEOUT) if the other
+// CTAs do not arrive within the spin limit.
+__device__ inline bool grid_barrier(unsigned int* bar, unsigned int nblocks) {
+  __syncthreads();
+  int ok = 1;
+  if (threadIdx.x == 0) {
+    __threadfence();
+    unsigned int gen;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(gen) : "l"(bar + 1) : "memory");
+    const unsigned int arrived = atomicAdd(bar, 1u);
+    if (arrived == nblocks - 1) {
+      atomicExch(bar, 0u);
+      __threadfence();
+      atomicAdd(bar + 1, 1u);
+    } else {
+      ok = 0;
+      for (uint32_t i = 0; i < kSpinLimit; ++i) {
+        unsigned int g;
+        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(g) : "l"(bar + 1) : "memory");
+        if (g != gen) {
+          ok = 1;
+          break;
+        }
+        __nanosleep(128);
+      }
+      if (!ok) set_status(W1_ERR_TIMEOUT);
+    }
+    __threadfence();
+  }
+  return __syncthreads_and(ok) != 0;
+}
+
 // ---------------------------------------------------------------- warp MMA (int8)
 // D = A(16x32, s8, row) * B(32x8, s8, col) + C, s32 accumulate.
 __device__ __forceinline__ void mma_s8_16832(int (&d)[4], const uint32_t (&a)[4], uint32_t b0,

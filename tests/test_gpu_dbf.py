@@ -1,4 +1,9 @@
-"""dbf_apply (fused small-batch kernel) on the GPU vs the fp64 oracle chain."""
+"""dbf_apply on the GPU vs the fp64 oracle chain.
+
+Every test runs with each of the two fused small-batch chain kernels forced
+(W1_DBF_PATH=direct: the direct GEMV core, the default for groups of up to 4
+rows; =ring: the ring core, the default above); batches of 64 and more take
+the tensor-core path either way."""
 import functools
 
 import numpy as np
@@ -10,6 +15,12 @@ from pack_sign_g128_b200 import ops, synth, _lib
 from gpu_helpers import assert_within, bf16_dev, fp16_dev, words_dev
 
 pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True, params=["direct", "ring"])
+def dbf_path(request, monkeypatch):
+    monkeypatch.setenv("W1_DBF_PATH", request.param)
+    return request.param
 
 
 def run_dbf(case, ws=None):
