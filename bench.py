@@ -126,6 +126,15 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ distributed
 
+def _backend() -> str:
+    """nccl on GPUs; W1_BENCH_BACKEND=gloo runs the rank logic on CPU (tests)."""
+    return os.environ.get("W1_BENCH_BACKEND", "nccl")
+
+
+def _reduce_device() -> str:
+    return "cpu" if _backend() == "gloo" else "cuda"
+
+
 def dist_setup():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -133,7 +142,7 @@ def dist_setup():
     if world > 1:
         import torch.distributed as dist
         import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        dist.init_process_group(_backend(), timeout=datetime.timedelta(seconds=120))
     return world, rank, local
 
 
@@ -148,7 +157,7 @@ def max_over_ranks(world, value: float) -> float:
         return value
     import torch
     import torch.distributed as dist
-    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    t = torch.tensor([value], dtype=torch.float64, device=_reduce_device())
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
@@ -158,7 +167,7 @@ def sum_over_ranks(world, value: float) -> float:
         return value
     import torch
     import torch.distributed as dist
-    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    t = torch.tensor([value], dtype=torch.float64, device=_reduce_device())
     dist.all_reduce(t, op=dist.ReduceOp.SUM)
     return float(t.item())
 
