@@ -280,8 +280,9 @@ def time_gemv_static(torch, combos, stream, reps: int = 3):
 
 
 def gemv_e2e(torch, ops, combos, steps: int):
-    """Same sweep through the public API with pinned host buffers: every launch
-    copies its x host->device and reads y back device->host."""
+    """The same sweep through the public API (eager w1_gemv calls, no graphs).
+    Every step copies its inputs host->device from pinned memory (each pair's
+    x) and reads its results back device->host (each pair's y)."""
     stream = torch.cuda.Stream()
     host = []
     for cb in combos:
@@ -297,13 +298,13 @@ def gemv_e2e(torch, ops, combos, steps: int):
         start.record(stream)
         for _ in range(steps):
             for cb, (xh, yh) in zip(combos, host):
+                cb["x"].copy_(xh, non_blocking=True)
+                h2d += xh.numel() * 2
                 for r in range(cb["R"]):
-                    cb["x"].copy_(xh, non_blocking=True)
                     ops.w1_gemv(cb["signs"][r], cb["scales"][r], cb["x"], cb["y"])
-                    yh.copy_(cb["y"], non_blocking=True)
-                    h2d += xh.numel() * 2
-                    d2h += yh.numel() * 4
                     launches += 1
+                yh.copy_(cb["y"], non_blocking=True)
+                d2h += yh.numel() * 4
         end.record(stream)
     torch.cuda.synchronize()
     ms = start.elapsed_time(end)

@@ -174,7 +174,7 @@ static int dbfd_max_clusters(int S, int smem_bytes) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaFuncSetAttribute(dbf_direct_kernel<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes) !=
+  if (ensure_dyn_smem(reinterpret_cast<const void*>(dbf_direct_kernel<NB>), smem_bytes) !=
           cudaSuccess ||
       cudaOccupancyMaxActiveClusters(&n, dbf_direct_kernel<NB>, &cfg) != cudaSuccess) {
     cudaGetLastError();
@@ -242,8 +242,7 @@ static cudaError_t launch_dbf_small_nb(const uint16_t* a, const uint32_t* B1, co
   p2.x_f32 = 1;
   p2.rdiag = a;
   p2.y = y;
-  cudaError_t err =
-      cudaFuncSetAttribute(dbf_direct_kernel<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  cudaError_t err = ensure_dyn_smem(reinterpret_cast<const void*>(dbf_direct_kernel<NB>), smem);
   if (err != cudaSuccess) return err;
   if (getenv("W1_VERBOSE"))
     fprintf(stderr, "dbf plan: B=%d -> clusters=%d split=%d warps=%dx%d / %dx%d smem=%d\n", NB, Q, S, p1.Wn,

@@ -213,7 +213,7 @@ static int dbf_ring_max_clusters(int S, int smem_bytes) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int nclusters = 0;
-  if (cudaFuncSetAttribute(dbf_ring_kernel<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes) !=
+  if (ensure_dyn_smem(reinterpret_cast<const void*>(dbf_ring_kernel<NB>), smem_bytes) !=
           cudaSuccess ||
       cudaOccupancyMaxActiveClusters(&nclusters, dbf_ring_kernel<NB>, &cfg) != cudaSuccess) {
     cudaGetLastError();
@@ -269,7 +269,7 @@ static cudaError_t launch_dbf_ring_nb(DbfParams p, const uint32_t* B1, const uin
       if (!make_tmap_u32_rows(&tm2, B2, c.r, c.n / 32, 4 * c.bw1) ||
           !make_tmap_u32_rows(&tm1, B1, c.m, c.r / 32, 4 * c.bw2))
         return cudaErrorInvalidValue;
-      cudaError_t err = cudaFuncSetAttribute(dbf_ring_kernel<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      cudaError_t err = ensure_dyn_smem(reinterpret_cast<const void*>(dbf_ring_kernel<NB>), smem);
       if (err != cudaSuccess) return err;
       if (getenv("W1_VERBOSE"))
         fprintf(stderr, "dbf plan: B=%d -> clusters=%d split=%d stages=%d/%d smem=%d\n", NB, Q, S, c.ns1, c.ns2, smem);

@@ -191,7 +191,7 @@ static int gemv_max_clusters(int S, int smem_bytes) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaFuncSetAttribute(gemv_kernel<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes) !=
+  if (ensure_dyn_smem(reinterpret_cast<const void*>(gemv_kernel<NB>), smem_bytes) !=
           cudaSuccess ||
       cudaOccupancyMaxActiveClusters(&n, gemv_kernel<NB>, &cfg) != cudaSuccess) {
     cudaGetLastError();
@@ -289,7 +289,7 @@ static cudaError_t launch_gemv_nb(const uint32_t* signs, const GemvParams& base,
   p.max_ng = plan.max_ng;
   CUtensorMap tmap;
   if (!make_tmap_u32_rows(&tmap, signs, base.N, base.K / 32, 4 * plan.bw)) return cudaErrorInvalidValue;
-  cudaError_t err = cudaFuncSetAttribute(gemv_kernel<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize, plan.smem);
+  cudaError_t err = ensure_dyn_smem(reinterpret_cast<const void*>(gemv_kernel<NB>), plan.smem);
   if (err != cudaSuccess) return err;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(plan.Q * plan.S));

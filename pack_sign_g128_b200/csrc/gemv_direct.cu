@@ -618,7 +618,7 @@ static int gd_max_clusters(int S, int smem_bytes) {
   cfg.attrs = attr;
   cfg.numAttrs = S > 1 ? 1 : 0;
   int n = 0;
-  if (cudaFuncSetAttribute(gemv_direct_kernel<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes) !=
+  if (ensure_dyn_smem(reinterpret_cast<const void*>(gemv_direct_kernel<NB>), smem_bytes) !=
       cudaSuccess) {
     cudaGetLastError();
     return 0;
@@ -770,8 +770,7 @@ static cudaError_t launch_gemv_direct_nb(const GdParams& base, cudaStream_t stre
   p.lgGw = lg2(plan.NSw * gd::Cfg<NB>::G);
   p.tq = p.NT / plan.Q;
   p.tr = p.NT - p.tq * plan.Q;
-  cudaError_t err =
-      cudaFuncSetAttribute(gemv_direct_kernel<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize, plan.smem);
+  cudaError_t err = ensure_dyn_smem(reinterpret_cast<const void*>(gemv_direct_kernel<NB>), plan.smem);
   if (err != cudaSuccess) return err;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(plan.Q * plan.S));

@@ -423,7 +423,7 @@ static int gemv_tc_max_clusters(int S, int smem_bytes) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaFuncSetAttribute(gemv_tc_kernel<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes) !=
+  if (ensure_dyn_smem(reinterpret_cast<const void*>(gemv_tc_kernel<NB>), smem_bytes) !=
           cudaSuccess ||
       cudaOccupancyMaxActiveClusters(&n, gemv_tc_kernel<NB>, &cfg) != cudaSuccess) {
     cudaGetLastError();
@@ -516,7 +516,7 @@ static cudaError_t launch_gemv_tc_nb(const GemvTcParams& base, cudaStream_t stre
   GemvTcParams p = base;
   p.S = plan.S;
   p.max_ng = plan.max_ng;
-  cudaError_t err = cudaFuncSetAttribute(gemv_tc_kernel<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize, plan.smem);
+  cudaError_t err = ensure_dyn_smem(reinterpret_cast<const void*>(gemv_tc_kernel<NB>), plan.smem);
   if (err != cudaSuccess) return err;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(plan.Q * plan.S));

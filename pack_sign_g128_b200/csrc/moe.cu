@@ -748,7 +748,7 @@ cudaError_t launch_moe(const uint16_t* x, const float* logits, int64_t T, int64_
     p.K = static_cast<int>(H);
     p.out_ld = static_cast<int>(I);
     const size_t smem = sizeof(MoeSmem<true>) + 1024;
-    err = cudaFuncSetAttribute(moe_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    err = ensure_dyn_smem(reinterpret_cast<const void*>(moe_gemm_kernel<true>), static_cast<int>(smem));
     if (err != cudaSuccess) return err;
     const int grid = L.max_tiles_gu < num_sms ? L.max_tiles_gu : num_sms;
     err = launch_pdl(moe_gemm_kernel<true>, dim3(grid), dim3(moe::kThreads), smem, stream, tm, p);
@@ -776,7 +776,7 @@ cudaError_t launch_moe(const uint16_t* x, const float* logits, int64_t T, int64_
     p.K = static_cast<int>(I);
     p.out_ld = static_cast<int>(H);
     const size_t smem = sizeof(MoeSmem<false>) + 1024;
-    err = cudaFuncSetAttribute(moe_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    err = ensure_dyn_smem(reinterpret_cast<const void*>(moe_gemm_kernel<false>), static_cast<int>(smem));
     if (err != cudaSuccess) return err;
     const int grid = L.max_tiles_d < num_sms ? L.max_tiles_d : num_sms;
     err = launch_pdl(moe_gemm_kernel<false>, dim3(grid), dim3(moe::kThreads), smem, stream, tm, p);

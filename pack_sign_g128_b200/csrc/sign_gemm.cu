@@ -402,8 +402,7 @@ static cudaError_t launch_sg_gemm_bm(SgParams p, const void* bmat, int64_t bcols
   // fp16 and bf16 share the 2-byte element layout the tensor map describes; box {64, BM}
   if (!make_tmap_bf16_sw128(&tm, bmat, p.M, bcols, BM)) return cudaErrorInvalidValue;
   const size_t smem = sizeof(Smem<BM>) + 1024;
-  cudaError_t err = cudaFuncSetAttribute(sg_gemm_kernel<PHASE1, BM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
+  cudaError_t err = ensure_dyn_smem(reinterpret_cast<const void*>(sg_gemm_kernel<PHASE1, BM>), static_cast<int>(smem));
   if (err != cudaSuccess) return err;
   const int ntiles = p.MT * p.NT;
   cudaLaunchConfig_t cfg = {};

@@ -358,3 +358,38 @@ __host__ __device__ constexpr uint32_t idesc_i8(int M, int N) {
 __device__ __forceinline__ void fence_async_shared() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 }  // namespace w1
+
+// Host: raise a kernel's dynamic shared memory limit to at least `bytes` on
+// the current device, calling the driver only when the cached value is lower
+// (the attribute is set on every launch path, so this keeps it off the hot
+// path).
+#include <mutex>
+namespace w1 {
+inline cudaError_t ensure_dyn_smem(const void* kernel, int bytes) {
+  struct Entry {
+    const void* k;
+    int dev;
+    int bytes;
+  };
+  static Entry tab[256];
+  static int n = 0;
+  static std::mutex mu;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < n; ++i)
+      if (tab[i].k == kernel && tab[i].dev == dev && tab[i].bytes >= bytes) return cudaSuccess;
+  }
+  const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < n; ++i)
+    if (tab[i].k == kernel && tab[i].dev == dev) {
+      if (tab[i].bytes < bytes) tab[i].bytes = bytes;
+      return cudaSuccess;
+    }
+  if (n < 256) tab[n++] = Entry{kernel, dev, bytes};
+  return cudaSuccess;
+}
+}  // namespace w1
