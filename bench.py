@@ -42,7 +42,8 @@ GEMM_SHAPES = [(14336, 4096), (4096, 14336), (14336, 14336)]
 GEMM_M = 2048
 WORKLOAD = ("decode GEMV sweep: (out x in) 4096x4096, 11008x4096, 4096x11008 at B = 1, 4, 8; "
             "1-bit signs + fp16 scale per 128 weights; x bf16 N(0,1); W N(0,0.02)")
-KERNEL_OF_CHOICE = {"direct": "gemv_direct_kernel", "tc": "gemv_tc_kernel", "ring": "gemv_kernel"}
+KERNEL_OF_CHOICE = {"direct": "gemv_direct_kernel", "direct16": "gemv_direct_kernel", "tc": "gemv_tc_kernel",
+                    "ring": "gemv_kernel"}
 # DRAM bytes per launch from ncu captures (dram__bytes_read.sum + write), with the
 # shape captured; see profiles/.  Used to report the dominant kernel's traffic.
 CAPTURED_TRAFFIC = {

@@ -53,7 +53,7 @@ __host__ __device__ inline DbfdSmem dbfd_layout(const GdParams& p1, const GdPara
   const int nsc = p1.NSc > p2.NSc ? p1.NSc : p2.NSc;
   M.red = M.xs + (nsc * C::SCR * 4 + 15) / 16 * 16;
   const int tw = p1.Tw > p2.Tw ? p1.Tw : p2.Tw;
-  M.part = M.red + gd::kWarps * tw * 16 * C::MT * 8 * 4;
+  M.part = M.red + gd::gd_red_bytes<NB>(tw);
   const int chunk = p1.chunk > p2.chunk ? p1.chunk : p2.chunk;
   M.total = M.part + (p1.S > 1 ? p1.S * NB * chunk * 4 : 0);
   return M;
@@ -86,6 +86,8 @@ __global__ void __launch_bounds__(gd::kThreads, 1) dbf_direct_kernel(const GdPar
   else cp_async_commit();
   if (g2.busy) gd_stage<NB>(p2, g2, wts2, lane);
   else cp_async_commit();
+  uint4 xa[4];
+  gd_x_first<NB, false>(p1, g1, warp, lane, xa);
   {
     uint16_t sreg[kGdSpl];  // no group scales: every s = 1
     gd_load_scales<NB>(p1, g1, 0, lane, sreg);
@@ -94,7 +96,7 @@ __global__ void __launch_bounds__(gd::kThreads, 1) dbf_direct_kernel(const GdPar
     gd_finish_scales<NB>(p2, g2, lane, sreg, scl2);
   }
   // ---- phase 1: h_scaled = mid (.) (V . (b (.) x))
-  gd_prep_x<NB, false>(p1, g1, xs, warp, lane);
+  gd_prep_x<NB, false>(p1, g1, xs, warp, lane, xa);
   asm volatile("cp.async.wait_group 1;" ::: "memory");  // V landed (U may still be in flight)
   __syncthreads();
   gd_finish<NB>(p1, g1, wts1, scl1, xs, red, part, warp, lane, true);
@@ -106,7 +108,8 @@ __global__ void __launch_bounds__(gd::kThreads, 1) dbf_direct_kernel(const GdPar
     return;
   }
   // ---- phase 2: y = a (.) (U . h_scaled)
-  gd_prep_x<NB, true>(p2, g2, xs, warp, lane);
+  gd_x_first<NB, true>(p2, g2, warp, lane, xa);
+  gd_prep_x<NB, true>(p2, g2, xs, warp, lane, xa);
   cp_async_wait_all();
   __syncthreads();
   gd_finish<NB>(p2, g2, wts2, scl2, xs, red, part, warp, lane, false);
@@ -191,7 +194,7 @@ static int dbfd_max_clusters(int S, int smem_bytes) {
 template <int NB>
 static double dbfd_cost(const GdParams& p) {
   using C = gd::Cfg<NB>;
-  const double cw = NB <= 2 ? 0.6 : (NB <= 5 ? 1.0 : 1.5);
+  const double cw = NB <= 2 ? 0.35 : (NB <= 5 ? 1.0 : 1.2);
   const int Tmax = (p.NT + p.Q - 1) / p.Q;
   const double xprep = 24.0 * NB * 128.0 * C::G * p.NSc;
   const double wts = 8.0 * Tmax * 128.0 * C::G * p.NSc * cw;

@@ -31,6 +31,7 @@
 #include <cstdint>
 #include <cuda_fp16.h>
 #include <cstdio>
+#include <cstring>
 #include <cstdlib>
 #include <mutex>
 
@@ -312,7 +313,7 @@ cudaError_t launch_gemv_tc(const uint32_t* signs, const uint16_t* scales, int64_
                            int B, float* y, bool static_weights, cudaStream_t stream, int num_sms, int force_s);
 cudaError_t launch_gemv_direct(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t K,
                                const uint16_t* x, int B, float* y, bool static_weights, cudaStream_t stream,
-                               int num_sms, int smem_cap, int force_s);
+                               int num_sms, int smem_cap, int force_s, int warps);
 
 // The mma.sync ring kernel over row chunks (the fallback for shapes outside
 // the other two kernels' plans).
@@ -353,18 +354,20 @@ static cudaError_t launch_gemv_ring(const uint32_t* signs, const uint16_t* scale
 
 // Kernel and K split per (device, N, K, B, static weights), chosen by timing.
 // The first call for a shape (outside stream capture) runs each candidate --
-// the direct kernel with K split 1, 2, 4, 8, the tcgen05 kernel, the ring
-// kernel -- three times untimed and twelve times between CUDA events on the
-// caller's stream with the caller's buffers, keeps the fastest, and blocks the
-// host until that finishes (one to two milliseconds).  Calls made while the stream is
-// being captured, or with W1_GEMV_AUTOTUNE=0, use the static rule instead:
-// direct for B <= 4, tcgen05 above, each only where its plan fits, else the
-// ring kernel.  W1_GEMV_PATH=direct|tc|mma forces one kernel (testing knob;
-// a forced kernel whose plan does not fit fails with W1_ERR_UNSUPPORTED).
+// the direct kernel with K split 1, 2, 4, 8 at 8 and at 16 warps per CTA, the
+// tcgen05 kernel, the ring kernel -- three times plainly and twelve times back
+// to back as one captured CUDA graph (timed between CUDA events), on a private
+// stream ordered after the caller's work, with the caller's buffers; keeps the
+// fastest, and blocks the host until that finishes (a few milliseconds).
+// Calls made while the stream is being captured, or with W1_GEMV_AUTOTUNE=0,
+// use the static rule instead: direct for B <= 4, tcgen05 above, each only
+// where its plan fits, else the ring kernel.  W1_GEMV_PATH=direct|direct16|tc|mma forces one kernel (testing
+// knob; a forced kernel whose plan does not fit fails with W1_ERR_UNSUPPORTED).
 namespace {
 struct GemvChoice {
   char kind;  // 'd' direct, 't' tcgen05, 'm' ring
   int s;      // forced K split, 0 = the kernel's planner
+  int w;      // direct kernel: warps per CTA (8 or 16)
 };
 struct GemvChoiceEntry {
   int dev;
@@ -383,7 +386,7 @@ static cudaError_t run_gemv_choice(const GemvChoice& c, const uint32_t* signs, c
                                    int smem_cap, bool static_weights) {
   switch (c.kind) {
     case 'd':
-      return launch_gemv_direct(signs, scales, N, K, x, B, y, static_weights, stream, num_sms, smem_cap, c.s);
+      return launch_gemv_direct(signs, scales, N, K, x, B, y, static_weights, stream, num_sms, smem_cap, c.s, c.w);
     case 't':
       return launch_gemv_tc(signs, scales, N, K, x, B, y, static_weights, stream, num_sms, c.s);
     default:
@@ -395,8 +398,8 @@ static cudaError_t run_gemv_choice(const GemvChoice& c, const uint32_t* signs, c
 static cudaError_t run_gemv_rule(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t K,
                                  const uint16_t* x, int B, float* y, cudaStream_t stream, int num_sms, int smem_cap,
                                  bool static_weights) {
-  const GemvChoice first = B <= 4 ? GemvChoice{'d', 0} : GemvChoice{'t', 0};
-  const GemvChoice second = B <= 4 ? GemvChoice{'t', 0} : GemvChoice{'d', 0};
+  const GemvChoice first = B <= 4 ? GemvChoice{'d', 0, 8} : GemvChoice{'t', 0, 0};
+  const GemvChoice second = B <= 4 ? GemvChoice{'t', 0, 0} : GemvChoice{'d', 0, 8};
   cudaError_t e = run_gemv_choice(first, signs, scales, N, K, x, B, y, stream, num_sms, smem_cap, static_weights);
   if (e != cudaErrorNotSupported) return e;
   e = run_gemv_choice(second, signs, scales, N, K, x, B, y, stream, num_sms, smem_cap, static_weights);
@@ -404,11 +407,54 @@ static cudaError_t run_gemv_rule(const uint32_t* signs, const uint16_t* scales, 
   return launch_gemv_ring(signs, scales, N, K, x, B, y, stream, num_sms, smem_cap);
 }
 
+// One autotune measurement: `reps` back-to-back launches of candidate c
+// captured as one CUDA graph on the private stream ts (the way a decode loop
+// replays them), after three plain launches that also check that c fits.
+// Returns 1 with *ms set, 0 when c does not fit or cannot be captured, -1 on
+// a device error (in *err).
+static int time_gemv_choice(const GemvChoice& c, const uint32_t* signs, const uint16_t* scales, int64_t N,
+                            int64_t K, const uint16_t* x, int B, float* y, cudaStream_t ts, int num_sms,
+                            int smem_cap, bool static_weights, int reps, cudaEvent_t e0, cudaEvent_t e1, float* ms,
+                            cudaError_t* err) {
+  for (int i = 0; i < 3; ++i) {
+    if (run_gemv_choice(c, signs, scales, N, K, x, B, y, ts, num_sms, smem_cap, static_weights) != cudaSuccess) {
+      cudaGetLastError();
+      return 0;
+    }
+  }
+  cudaGraph_t g = nullptr;
+  if (cudaStreamBeginCapture(ts, cudaStreamCaptureModeThreadLocal) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  cudaError_t le = cudaSuccess;
+  for (int i = 0; i < reps && le == cudaSuccess; ++i)
+    le = run_gemv_choice(c, signs, scales, N, K, x, B, y, ts, num_sms, smem_cap, static_weights);
+  const cudaError_t ce = cudaStreamEndCapture(ts, &g);
+  cudaGraphExec_t ge = nullptr;
+  const bool built = le == cudaSuccess && ce == cudaSuccess && g && cudaGraphInstantiate(&ge, g, 0) == cudaSuccess;
+  if (g) cudaGraphDestroy(g);
+  if (!built) {
+    cudaGetLastError();
+    return 0;
+  }
+  cudaGraphLaunch(ge, ts);  // warm
+  cudaEventRecord(e0, ts);
+  cudaGraphLaunch(ge, ts);
+  cudaEventRecord(e1, ts);
+  *err = cudaEventSynchronize(e1);
+  cudaGraphExecDestroy(ge);
+  if (*err != cudaSuccess) return -1;
+  cudaEventElapsedTime(ms, e0, e1);
+  return 1;
+}
+
 cudaError_t launch_gemv(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t K,
                         const uint16_t* x, int B, float* y, cudaStream_t stream, int num_sms,
                         int smem_cap, bool static_weights) {
   if (const char* path = getenv("W1_GEMV_PATH")) {
-    const GemvChoice c{path[0] == 'd' ? 'd' : (path[0] == 't' ? 't' : 'm'), 0};
+    const GemvChoice c{path[0] == 'd' ? 'd' : (path[0] == 't' ? 't' : 'm'), 0,
+                       strcmp(path, "direct16") == 0 ? 16 : 8};
     return run_gemv_choice(c, signs, scales, N, K, x, B, y, stream, num_sms, smem_cap, static_weights);
   }
   int dev = 0;
@@ -430,40 +476,49 @@ cudaError_t launch_gemv(const uint32_t* signs, const uint16_t* scales, int64_t N
   if (cap != cudaStreamCaptureStatusNone || (at && at[0] == '0'))
     return run_gemv_rule(signs, scales, N, K, x, B, y, stream, num_sms, smem_cap, static_weights);
 
-  const GemvChoice cands[] = {{'d', 1}, {'d', 2}, {'d', 4}, {'d', 8}, {'t', 0}, {'m', 0}};
+  const GemvChoice cands[] = {{'d', 1, 8},  {'d', 2, 8},  {'d', 4, 8},  {'d', 8, 8}, {'d', 1, 16},
+                              {'d', 2, 16}, {'d', 4, 16}, {'d', 8, 16}, {'t', 0, 0}, {'m', 0, 0}};
   constexpr int kTimed = 12;
-  cudaEvent_t e0, e1;
-  if (cudaEventCreate(&e0) != cudaSuccess) return cudaGetLastError();
-  if (cudaEventCreate(&e1) != cudaSuccess) {
-    cudaEventDestroy(e0);
-    return cudaGetLastError();
+  // A private stream, ordered after the caller's work so far, takes the
+  // captures (the caller's stream is not captured or reordered).
+  cudaStream_t ts = nullptr;
+  cudaEvent_t e0 = nullptr, e1 = nullptr, ready = nullptr;
+  cudaError_t setup = cudaStreamCreateWithFlags(&ts, cudaStreamNonBlocking);
+  if (setup == cudaSuccess) setup = cudaEventCreate(&e0);
+  if (setup == cudaSuccess) setup = cudaEventCreate(&e1);
+  if (setup == cudaSuccess) setup = cudaEventCreateWithFlags(&ready, cudaEventDisableTiming);
+  if (setup == cudaSuccess) setup = cudaEventRecord(ready, stream);
+  if (setup == cudaSuccess) setup = cudaStreamWaitEvent(ts, ready, 0);
+  auto release = [&]() {
+    if (ts) {
+      cudaStreamSynchronize(ts);
+      cudaStreamDestroy(ts);
+    }
+    if (e0) cudaEventDestroy(e0);
+    if (e1) cudaEventDestroy(e1);
+    if (ready) cudaEventDestroy(ready);
+  };
+  if (setup != cudaSuccess) {
+    release();
+    cudaGetLastError();
+    return run_gemv_rule(signs, scales, N, K, x, B, y, stream, num_sms, smem_cap, static_weights);
   }
   // The candidates run on one weight matrix that stays in L2, which flatters
   // the kernels least sensitive to memory latency; the static rule's kernel
   // is kept unless another is more than 5% faster.
   const char rule_kind = B <= 4 ? 'd' : 't';
-  GemvChoice best{0, 0}, best_rule{0, 0};
+  GemvChoice best{0, 0, 0}, best_rule{0, 0, 0};
   float best_ms = 0.f, best_rule_ms = 0.f;
   cudaError_t fatal = cudaSuccess;
   for (const GemvChoice& c : cands) {
-    bool ok = true;
-    for (int i = 0; i < 3 && ok; ++i) {
-      const cudaError_t e =
-          run_gemv_choice(c, signs, scales, N, K, x, B, y, stream, num_sms, smem_cap, static_weights);
-      if (e != cudaSuccess) {
-        cudaGetLastError();
-        ok = false;
-      }
-    }
-    if (!ok) continue;
-    cudaEventRecord(e0, stream);
-    for (int i = 0; i < kTimed; ++i)
-      run_gemv_choice(c, signs, scales, N, K, x, B, y, stream, num_sms, smem_cap, static_weights);
-    cudaEventRecord(e1, stream);
-    fatal = cudaEventSynchronize(e1);
-    if (fatal != cudaSuccess) break;  // a device error: report it, choose nothing
     float ms = 0.f;
-    cudaEventElapsedTime(&ms, e0, e1);
+    const int r = time_gemv_choice(c, signs, scales, N, K, x, B, y, ts, num_sms, smem_cap, static_weights, kTimed,
+                                   e0, e1, &ms, &fatal);
+    if (r < 0) break;  // a device error: report it, choose nothing
+    if (r == 0) continue;
+    if (getenv("W1_VERBOSE"))
+      fprintf(stderr, "w1_gemv candidate: N=%lld K=%lld B=%d %c split=%d warps=%d %.2f us\n",
+              static_cast<long long>(N), static_cast<long long>(K), B, c.kind, c.s, c.w, ms * 1e3f / kTimed);
     if (best.kind == 0 || ms < best_ms) {
       best = c;
       best_ms = ms;
@@ -477,14 +532,13 @@ cudaError_t launch_gemv(const uint32_t* signs, const uint16_t* scales, int64_t N
     best = best_rule;
     best_ms = best_rule_ms;
   }
-  cudaEventDestroy(e0);
-  cudaEventDestroy(e1);
+  release();
   if (fatal != cudaSuccess) return fatal;
   if (best.kind == 0) return run_gemv_rule(signs, scales, N, K, x, B, y, stream, num_sms, smem_cap, static_weights);
   if (getenv("W1_VERBOSE"))
-    fprintf(stderr, "w1_gemv tuned: N=%lld K=%lld B=%d static=%d -> %c split=%d (%.2f us)\n",
+    fprintf(stderr, "w1_gemv tuned: N=%lld K=%lld B=%d static=%d -> %c split=%d warps=%d (%.2f us)\n",
             static_cast<long long>(N), static_cast<long long>(K), B, static_weights ? 1 : 0, best.kind, best.s,
-            best_ms * 1e3f / kTimed);
+            best.w, best_ms * 1e3f / kTimed);
   {
     std::lock_guard<std::mutex> lock(g_choice_mu);
     const int i = g_nchoice < 256 ? g_nchoice++ : static_cast<int>((N + K + B) & 255);
@@ -493,12 +547,13 @@ cudaError_t launch_gemv(const uint32_t* signs, const uint16_t* scales, int64_t N
   return run_gemv_choice(best, signs, scales, N, K, x, B, y, stream, num_sms, smem_cap, static_weights);
 }
 
-// Name of the cached choice for a shape ("direct/2", "tc/0", "ring/0"), or ""
+// Name of the cached choice for a shape ("direct/2", "direct16/1", "tc/0",
+// "ring/0"), or ""
 // when none has been made on the current device.
 static int gemv_choice_name(int64_t N, int64_t K, int B, bool st, char* out, size_t out_len) {
   int dev = 0;
   cudaGetDevice(&dev);
-  GemvChoice c{0, 0};
+  GemvChoice c{0, 0, 0};
   {
     std::lock_guard<std::mutex> lock(g_choice_mu);
     for (int i = 0; i < g_nchoice; ++i) {
@@ -506,7 +561,8 @@ static int gemv_choice_name(int64_t N, int64_t K, int B, bool st, char* out, siz
       if (e.dev == dev && e.N == N && e.K == K && e.B == B && e.st == st) c = e.c;
     }
   }
-  const char* kind = c.kind == 'd' ? "direct" : (c.kind == 't' ? "tc" : (c.kind == 'm' ? "ring" : ""));
+  const char* kind = c.kind == 'd' ? (c.w == 16 ? "direct16" : "direct")
+                                    : (c.kind == 't' ? "tc" : (c.kind == 'm' ? "ring" : ""));
   if (c.kind == 0) return snprintf(out, out_len, "%s", "");
   return snprintf(out, out_len, "%s/%d", kind, c.s);
 }

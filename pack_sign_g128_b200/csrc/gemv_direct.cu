@@ -25,16 +25,13 @@
 //  * Signs -> int8 {0, -1} with one PRMT per 4 weights (a byte table keyed on
 //    bit 0, 1 or 2 of each selector nibble; bit 3 via w >> 3; upper half via
 //    w >> 16), so  sum (1-2b) n = X + 2 * sum (-b) n  with X = sum n.
-//  * int8 mma.sync m16n8k32, A = activation digits (rows), B = sign bytes
-//    (8 weight rows), s32 accumulators; one fold per group:
+//  * int8 mma.sync m16n8k32, A = sign bytes (16 weight rows: two 8-row
+//    n-tiles), B = activation digits (column 3b + p for batch row b and digit
+//    p; columns past 3B are zero), s32 accumulators.  Four MMAs cover one
+//    group of 16 rows (2048 weights), and each group is folded once:
 //    acc += s * (f*W_p * D_p + [p = hi] f*X),  W = {2^17, 2^9, 2}, f = 2^(E-22).
-//  * At B = 1 and 2 the 16-row MMA would hold only 3 or 6 digit rows, so 4 or
-//    2 groups share one MMA: lane quad c of an MMA contributes the sign bytes
-//    of group (c * G / 4), and the digit rows of group j carry zeros in the
-//    slots of the other groups (block-diagonal A).  The MMA count per weight
-//    stays the same, the folds drop by the same factor G.
 // K order inside one MMA is free as long as A and B agree: k-slot 4c+i+16h of
-// MMA (w, q) holds bit q + 4i + 16h of word (c*G + w) of the set, which is the
+// MMA q of a group holds bit q + 4i + 16h of the group's word c, which is the
 // order the PRMT extraction produces.
 #include <algorithm>
 #include <cmath>
@@ -50,21 +47,29 @@
 namespace w1 {
 
 namespace gd {
-constexpr int kWarps = 8;
+constexpr int kWarps = 8;           // warps per CTA (the GEMV kernel also runs with 16)
 constexpr int kThreads = kWarps * 32;
 constexpr int kMaxTw = 4;        // 8-row n-tiles per warp
+constexpr int kMaxTp = (kMaxTw + 1) / 2;  // 16-row MMA tiles per warp
 constexpr int kDigitStride = 34;  // words per digit row of the activation scratch (bank spread)
 constexpr int kMaxSets = 64;      // sets (of G groups) per CTA
 
 template <int NB>
 struct Cfg {
-  static constexpr int G = NB == 1 ? 4 : (NB == 2 ? 2 : 1);  // groups per MMA set
-  static constexpr int ROWS = 3 * NB * G;                     // digit rows in use
-  static constexpr int MT = (ROWS + 15) / 16;                 // m16 tiles
-  static constexpr int ITEMS = G * NB * 8;                    // 16-element activation items per set
-  static constexpr int IPL = (ITEMS + 31) / 32;               // items per lane
+  static constexpr int G = 1;                      // groups per set
+  static constexpr int NCOL = 3 * NB;              // digit columns: 3 per batch row
+  static constexpr int NN = (NCOL + 7) / 8;        // 8-column MMA n-tiles
+  static constexpr int ROWS = NCOL;                // digit rows of the activation scratch
   static constexpr int SCR = ROWS * kDigitStride + 2 * ROWS;  // scratch words: digits, f*W_p, f*X
+  static constexpr int RED = 8 * NCOL;             // reduction floats per warp and n-tile
 };
+
+// Reduction buffer: per (warp block along sets, CTA n-tile) 8 rows x NCOL
+// columns, plus one float of padding per warp block (bank spread).
+template <int NB, int NW = kWarps>
+__host__ __device__ inline int gd_red_bytes(int Tw) {
+  return ((NW * Tw * Cfg<NB>::RED + NW) * 4 + 15) / 16 * 16;
+}
 }  // namespace gd
 
 struct GdParams {
@@ -79,7 +84,7 @@ struct GdParams {
   int S;      // CTAs per cluster (K split)
   int Q;      // clusters
   int NT;     // 8-row n-tiles in total
-  int Wn, Wg;  // warps along n-tiles x along sets (Wn * Wg = 8)
+  int Wn, Wg;  // warps along n-tiles x along sets (Wn * Wg = warps per CTA)
   int Tw;     // n-tiles per warp (max)
   int NSw;    // sets per warp (max)
   int P;      // bytes per staged weight row
@@ -98,16 +103,16 @@ struct GdSmem {
 // Per warp: staged sign words (8*Tw rows of P bytes), scales (float,
 // [group][row]).  Per CTA: activation scratch (nsc sets of SCR words), the
 // reduction buffer and (cluster) the owner partials.
-template <int NB>
+template <int NB, int NW = gd::kWarps>
 __host__ __device__ inline GdSmem gd_layout(int Tw, int NSw, int P, int S, int chunk, int nsc) {
   using C = gd::Cfg<NB>;
   GdSmem L;
   L.wts = 0;
   L.scl = L.wts + 8 * Tw * P;
   L.warp_bytes = (L.scl + NSw * C::G * 8 * Tw * 4 + 15) / 16 * 16;
-  L.xs = gd::kWarps * L.warp_bytes;
+  L.xs = NW * L.warp_bytes;
   L.red = L.xs + (nsc * C::SCR * 4 + 15) / 16 * 16;
-  L.part = L.red + gd::kWarps * Tw * 16 * C::MT * 8 * 4;
+  L.part = L.red + gd::gd_red_bytes<NB, NW>(Tw);
   L.total = L.part + (S > 1 ? S * NB * chunk * 4 : 0);
   return L;
 }
@@ -143,9 +148,14 @@ __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wai
 template <int NB>
 __device__ __forceinline__ void quantise_item(const float (&v)[16], bool valid, int it, uint32_t* scr) {
   using C = gd::Cfg<NB>;
-  float mx = 0.f;
+  float m8[8];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) mx = fmaxf(mx, fabsf(v[i]));
+  for (int i = 0; i < 8; ++i) m8[i] = fmaxf(fabsf(v[2 * i]), fabsf(v[2 * i + 1]));
+#pragma unroll
+  for (int w = 4; w >= 1; w >>= 1)
+#pragma unroll
+    for (int i = 0; i < w; ++i) m8[i] = fmaxf(m8[i], m8[i + w]);
+  float mx = m8[0];
   mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 1));
   mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 2));
   mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 4));
@@ -154,16 +164,20 @@ __device__ __forceinline__ void quantise_item(const float (&v)[16], bool valid, 
   const int sf = 22 - E, sf1 = sf / 2, sf2 = sf - sf1;
   const float m1 = __uint_as_float(static_cast<uint32_t>(sf1 + 127) << 23);
   const float m2 = __uint_as_float(static_cast<uint32_t>(sf2 + 127) << 23);
-  uint32_t e[16];
-  uint32_t bsum = 0;
+  uint32_t e[16], bs[8];
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
     // 0x4B400000 + round(x 2^sf): exact rounding to an integer for |x 2^sf| < 2^22
     const uint32_t bits = __float_as_uint(fmaf(v[i] * m1, m2, 12582912.0f));
-    bsum += bits;
+    if (i & 1) bs[i >> 1] += bits;
+    else bs[i >> 1] = bits;
     e[i] = (bits - 0x4ABF7F80u) ^ 0x00808080u;  // bytes: signed digits lo, mid, hi
   }
-  int xs = static_cast<int>(bsum - 16u * 0x4B400000u);
+#pragma unroll
+  for (int w = 4; w >= 1; w >>= 1)
+#pragma unroll
+    for (int i = 0; i < w; ++i) bs[i] += bs[i + w];
+  int xs = static_cast<int>(bs[0] - 16u * 0x4B400000u);
   xs += __shfl_xor_sync(0xFFFFFFFFu, xs, 1);
   xs += __shfl_xor_sync(0xFFFFFFFFu, xs, 2);
   xs += __shfl_xor_sync(0xFFFFFFFFu, xs, 4);
@@ -197,110 +211,90 @@ __device__ __forceinline__ void quantise_item(const float (&v)[16], bool valid, 
 }
 
 // One warp's products over its n-tiles (TW of them, a compile-time count so that
-// no MMA sits under a per-tile branch) and its sets; returns the fp32 partial
-// sums in acc[t][mt][e] (C-fragment order: rows 16mt + 8(e>>1) + lane/4, weight
-// rows 2(lane&3) + (e&1) of n-tile t).
+// no MMA sits under a per-tile branch) and its sets (one group each).  An MMA
+// takes n-tiles 2tp and 2tp+1 as its A rows 0-7 and 8-15.  Returns the fp32
+// partial sums in acc[tp][nn][e] (C-fragment order: weight row lane/4 of n-tile
+// 2tp + (e>>1), digit column 8nn + 2(lane&3) + (e&1)).
 template <int NB, int TW>
 __device__ __forceinline__ void gd_compute(const unsigned char* wts, int P, const float* scl, int sstride,
                                            const uint32_t* xs, int nsw, int lane,
-                                           float (&acc)[gd::kMaxTw][gd::Cfg<NB>::MT][4]) {
+                                           float (&acc)[gd::kMaxTp][gd::Cfg<NB>::NN][4]) {
   using C = gd::Cfg<NB>;
-  constexpr int G = C::G, MT = C::MT;
+  constexpr int NN = C::NN, NCOL = C::NCOL, TP = (TW + 1) / 2;
   const int r1 = lane >> 2, cq = lane & 3;
-  // per-lane constants: A-fragment sources and fold rows
-  int abase[MT][2], sbase[MT][2];
-  bool aact[MT][2], rval[MT][2];
+  // B-fragment source of this lane: digit column 8nn + lane/4, word lane&3
+  int bofs[NN];
+  bool bact[NN];
 #pragma unroll
-  for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-    for (int hf = 0; hf < 2; ++hf) {
-      const int r = 16 * mt + 8 * hf + r1;
-      const int rg = r / (3 * NB);
-      rval[mt][hf] = r < C::ROWS;
-      aact[mt][hf] = rval[mt][hf] && rg == (cq * G) / 4;
-      abase[mt][hf] = r * gd::kDigitStride + ((cq * G) & 3) * 8;
-      sbase[mt][hf] = (rval[mt][hf] ? rg : 0) * sstride + 2 * cq;
-    }
-  const unsigned char* wrow = wts + r1 * P + cq * 4 * G;
+  for (int nn = 0; nn < NN; ++nn) {
+    const int n = 8 * nn + r1;
+    bact[nn] = n < NCOL;
+    bofs[nn] = n * gd::kDigitStride + cq * 8;
+  }
+  // A-fragment source: word lane&3 of the group in weight rows lane/4 (+8)
+  const unsigned char* wrow = wts + r1 * P + cq * 4;
   for (int si = 0; si < nsw; ++si) {
     const uint32_t* scr = xs + si * C::SCR;
+    uint32_t W0[TP], W1[TP];
+#pragma unroll
+    for (int tp = 0; tp < TP; ++tp) {
+      W0[tp] = *reinterpret_cast<const uint32_t*>(wrow + 16 * tp * P + si * 16);
+      W1[tp] = (2 * tp + 1 < TW) ? *reinterpret_cast<const uint32_t*>(wrow + (16 * tp + 8) * P + si * 16) : 0u;
+    }
+    int Cacc[TP][NN][4];
+#pragma unroll
+    for (int tp = 0; tp < TP; ++tp)
+#pragma unroll
+      for (int nn = 0; nn < NN; ++nn)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) Cacc[tp][nn][e] = 0;
+    auto step = [&](auto qc) {
+      constexpr int qq = decltype(qc)::value;
+      uint32_t B0[NN], B1[NN];
+#pragma unroll
+      for (int nn = 0; nn < NN; ++nn) {
+        uint2 u = make_uint2(0, 0);
+        if (bact[nn]) u = *reinterpret_cast<const uint2*>(scr + bofs[nn] + qq * 2);
+        B0[nn] = u.x;
+        B1[nn] = u.y;
+      }
+#pragma unroll
+      for (int tp = 0; tp < TP; ++tp) {
+        const uint32_t A[4] = {sign_bytes<qq>(W0[tp]), sign_bytes<qq>(W1[tp]), sign_bytes<qq + 4>(W0[tp]),
+                               sign_bytes<qq + 4>(W1[tp])};
+#pragma unroll
+        for (int nn = 0; nn < NN; ++nn) mma_s8(Cacc[tp][nn], A, B0[nn], B1[nn]);
+      }
+    };
+    step(std::integral_constant<int, 0>{});
+    step(std::integral_constant<int, 1>{});
+    step(std::integral_constant<int, 2>{});
+    step(std::integral_constant<int, 3>{});
+    // fold: acc += s[row, group] * (f W_p D + [hi] f X)
     const float* fwv = reinterpret_cast<const float*>(scr + C::ROWS * gd::kDigitStride);
-    float fw[MT][2], cx[MT][2];
+    float fw[NN][2], cx[NN][2];
 #pragma unroll
-    for (int mt = 0; mt < MT; ++mt)
+    for (int nn = 0; nn < NN; ++nn)
 #pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        const int r = 16 * mt + 8 * hf + r1;
-        fw[mt][hf] = rval[mt][hf] ? fwv[r] : 0.f;
-        cx[mt][hf] = rval[mt][hf] ? fwv[C::ROWS + r] : 0.f;
+      for (int c = 0; c < 2; ++c) {
+        const int n = 8 * nn + 2 * cq + c;
+        fw[nn][c] = n < NCOL ? fwv[n] : 0.f;
+        cx[nn][c] = n < NCOL ? fwv[C::ROWS + n] : 0.f;
       }
-    // sign words: lane (r1, cq) takes G words of row r1 of each n-tile
-    uint32_t W[TW][G];
+    const float* sset = scl + si * sstride + r1;
 #pragma unroll
-    for (int t = 0; t < TW; ++t) {
-      const unsigned char* src = wrow + t * 8 * P + si * 16 * G;
-      if constexpr (G == 4) {
-        const uint4 u = *reinterpret_cast<const uint4*>(src);
-        W[t][0] = u.x; W[t][G > 1 ? 1 : 0] = u.y; W[t][G > 2 ? 2 : 0] = u.z; W[t][G > 3 ? 3 : 0] = u.w;
-      } else if constexpr (G == 2) {
-        const uint2 u = *reinterpret_cast<const uint2*>(src);
-        W[t][0] = u.x; W[t][G > 1 ? 1 : 0] = u.y;
-      } else {
-        W[t][0] = *reinterpret_cast<const uint32_t*>(src);
-      }
-    }
-    int Cacc[TW][MT][4];
+    for (int tp = 0; tp < TP; ++tp) {
+      const float s0 = sset[16 * tp];
+      const float s1 = (2 * tp + 1 < TW) ? sset[16 * tp + 8] : 0.f;
 #pragma unroll
-    for (int t = 0; t < TW; ++t)
+      for (int nn = 0; nn < NN; ++nn)
 #pragma unroll
-      for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) Cacc[t][mt][e] = 0;
-#pragma unroll
-    for (int w = 0; w < G; ++w) {
-      auto step = [&](auto qc) {
-        constexpr int qq = decltype(qc)::value;
-        uint32_t A[MT][4];
-#pragma unroll
-        for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-          for (int hf = 0; hf < 2; ++hf) {
-            uint2 u = make_uint2(0, 0);
-            if (aact[mt][hf]) u = *reinterpret_cast<const uint2*>(scr + abase[mt][hf] + w * 8 + qq * 2);
-            A[mt][hf] = u.x;
-            A[mt][2 + hf] = u.y;
-          }
-#pragma unroll
-        for (int t = 0; t < TW; ++t) {
-          const uint32_t b0 = sign_bytes<qq>(W[t][w]);
-          const uint32_t b1 = sign_bytes<qq + 4>(W[t][w]);
-#pragma unroll
-          for (int mt = 0; mt < MT; ++mt) mma_s8(Cacc[t][mt], A[mt], b0, b1);
+        for (int c = 0; c < 2; ++c) {
+          acc[tp][nn][c] = fmaf(s0, fmaf(fw[nn][c], static_cast<float>(Cacc[tp][nn][c]), cx[nn][c]), acc[tp][nn][c]);
+          acc[tp][nn][2 + c] =
+              fmaf(s1, fmaf(fw[nn][c], static_cast<float>(Cacc[tp][nn][2 + c]), cx[nn][c]), acc[tp][nn][2 + c]);
         }
-      };
-      step(std::integral_constant<int, 0>{});
-      step(std::integral_constant<int, 1>{});
-      step(std::integral_constant<int, 2>{});
-      step(std::integral_constant<int, 3>{});
     }
-    // fold: acc += s[n, group of row] * (f W_p D + [hi] f X)
-    const float* sset = scl + si * G * sstride;
-#pragma unroll
-    for (int t = 0; t < TW; ++t)
-#pragma unroll
-      for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          if (rval[mt][hf]) {
-            const float2 sv = *reinterpret_cast<const float2*>(sset + sbase[mt][hf] + t * 8);
-            acc[t][mt][2 * hf + 0] =
-                fmaf(sv.x, fmaf(fw[mt][hf], static_cast<float>(Cacc[t][mt][2 * hf + 0]), cx[mt][hf]),
-                     acc[t][mt][2 * hf + 0]);
-            acc[t][mt][2 * hf + 1] =
-                fmaf(sv.y, fmaf(fw[mt][hf], static_cast<float>(Cacc[t][mt][2 * hf + 1]), cx[mt][hf]),
-                     acc[t][mt][2 * hf + 1]);
-          }
-        }
   }
 }
 
@@ -404,40 +398,55 @@ __device__ __forceinline__ void gd_finish_scales(const GdParams& p, const GdGeom
 // 8 lanes x 16 elements; 4 units per warp per pass, two passes in flight.
 // bf16 x (optionally times the fp16 column diagonal, exact in fp32) or fp32 x
 // (read through L2: it may have been written by other CTAs of this grid).
+// Unit u of this CTA -> this lane's 16 values (+ diagonal); zeros past the end.
 template <int NB, bool XF32>
-__device__ __forceinline__ void gd_prep_x(const GdParams& p, const GdGeom& g, uint32_t* xs, int warp, int lane) {
+__device__ __forceinline__ void gd_load_unit(const GdParams& p, const GdGeom& g, int u, int sub, uint4 (&r)[4]) {
+  constexpr int G = gd::Cfg<NB>::G;
+  const int units = g.nsc * G * NB;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) r[i] = make_uint4(0, 0, 0, 0);
+  if (u < units) {
+    const int sl = u / (G * NB), gb = u - sl * (G * NB);
+    const int gj = gb / NB, b = gb - gj * NB;
+    const int gi = (g.cs0 + sl) * G + gj;
+    if (gi < p.NG) {
+      const int64_t k0 = static_cast<int64_t>(gi) * 128 + sub * 16;
+      if (XF32) {
+        const uint4* src =
+            reinterpret_cast<const uint4*>(static_cast<const float*>(p.x) + static_cast<int64_t>(b) * p.K + k0);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) r[i] = __ldcg(src + i);
+      } else {
+        const uint4* src =
+            reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.x) + static_cast<int64_t>(b) * p.K + k0);
+        r[0] = __ldg(src);
+        r[1] = __ldg(src + 1);
+        if (p.cdiag) {
+          const uint4* dg = reinterpret_cast<const uint4*>(p.cdiag + k0);
+          r[2] = __ldg(dg);
+          r[3] = __ldg(dg + 1);
+        }
+      }
+    }
+  }
+}
+
+// The loads of this warp's first unit (split from the loop so that a caller
+// can place them among its other copies).
+template <int NB, bool XF32>
+__device__ __forceinline__ void gd_x_first(const GdParams& p, const GdGeom& g, int warp, int lane, uint4 (&xa)[4]) {
+  gd_load_unit<NB, XF32>(p, g, warp * 4 + (lane >> 3), lane & 7, xa);
+}
+
+// xa: this lane's first unit, from gd_x_first.
+template <int NB, bool XF32, int NW = gd::kWarps>
+__device__ __forceinline__ void gd_prep_x(const GdParams& p, const GdGeom& g, uint32_t* xs, int warp, int lane,
+                                          uint4 (&xa)[4]) {
   using C = gd::Cfg<NB>;
   constexpr int G = C::G;
   const int units = g.nsc * G * NB;
   const int sub = lane & 7;
-  auto load_unit = [&](int u, uint4 (&r)[4]) {  // unit u of this CTA -> this lane's 16 values (+ diagonal)
-#pragma unroll
-    for (int i = 0; i < 4; ++i) r[i] = make_uint4(0, 0, 0, 0);
-    if (u < units) {
-      const int sl = u / (G * NB), gb = u - sl * (G * NB);
-      const int gj = gb / NB, b = gb - gj * NB;
-      const int gi = (g.cs0 + sl) * G + gj;
-      if (gi < p.NG) {
-        const int64_t k0 = static_cast<int64_t>(gi) * 128 + sub * 16;
-        if (XF32) {
-          const uint4* src = reinterpret_cast<const uint4*>(static_cast<const float*>(p.x) +
-                                                            static_cast<int64_t>(b) * p.K + k0);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) r[i] = __ldcg(src + i);
-        } else {
-          const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.x) +
-                                                            static_cast<int64_t>(b) * p.K + k0);
-          r[0] = __ldg(src);
-          r[1] = __ldg(src + 1);
-          if (p.cdiag) {
-            const uint4* dg = reinterpret_cast<const uint4*>(p.cdiag + k0);
-            r[2] = __ldg(dg);
-            r[3] = __ldg(dg + 1);
-          }
-        }
-      }
-    }
-  };
+  auto load_unit = [&](int u, uint4 (&r)[4]) { gd_load_unit<NB, XF32>(p, g, u, sub, r); };
   auto process = [&](const uint4 (&r)[4], int u) {
     float v[16];
     if (XF32) {
@@ -469,10 +478,9 @@ __device__ __forceinline__ void gd_prep_x(const GdParams& p, const GdGeom& g, ui
     const int it = (u - sl * (G * NB)) * 8 + sub;  // item index within the set
     quantise_item<NB>(v, u < units, it, xs + sl * C::SCR);
   };
-  constexpr int kPass = 4 * gd::kWarps;  // units per pass of the CTA
+  constexpr int kPass = 4 * NW;  // units per pass of the CTA
   const int u0 = warp * 4 + (lane >> 3);
-  uint4 xa[4], xb[4];
-  load_unit(u0, xa);
+  uint4 xb[4];
   for (int u = u0; u - u0 < units; u += 2 * kPass) {  // trip count uniform over the CTA
     load_unit(u + kPass, xb);
     process(xa, u);
@@ -486,20 +494,20 @@ __device__ __forceinline__ void gd_prep_x(const GdParams& p, const GdGeom& g, ui
 // y[b][row] = rdiag[row] * sum.  Call after the weights, scales and digits are
 // in shared memory (and a __syncthreads).  `wait_cluster`: wait on the
 // cluster barrier arrived at kernel entry before the first remote store.
-template <int NB>
+template <int NB, int NW = gd::kWarps>
 __device__ __forceinline__ void gd_finish(const GdParams& p, const GdGeom& g, const unsigned char* wts,
                                           const float* scl, const uint32_t* xs, float* red, float* part, int warp,
                                           int lane, bool wait_cluster) {
   using C = gd::Cfg<NB>;
-  constexpr int G = C::G, MT = C::MT;
+  constexpr int NN = C::NN, NCOL = C::NCOL;
   const int sstride = 8 * p.Tw;
-  float acc[gd::kMaxTw][MT][4];
+  float acc[gd::kMaxTp][NN][4];
 #pragma unroll
-  for (int t = 0; t < gd::kMaxTw; ++t)
+  for (int tp = 0; tp < gd::kMaxTp; ++tp)
 #pragma unroll
-    for (int mt = 0; mt < MT; ++mt)
+    for (int nn = 0; nn < NN; ++nn)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) acc[t][mt][e] = 0.f;
+      for (int e = 0; e < 4; ++e) acc[tp][nn][e] = 0.f;
   if (g.busy) {
     const uint32_t* xw = xs + (g.ws0 - g.cs0) * C::SCR;
     switch (g.tw) {  // warp-uniform
@@ -509,41 +517,51 @@ __device__ __forceinline__ void gd_finish(const GdParams& p, const GdGeom& g, co
       default: gd_compute<NB, 4>(wts, p.P, scl, sstride, xw, g.nsw, lane, acc); break;
     }
   }
-  // ---- CTA reduction: red[wg][tile][row r][n], tile = wn * Tw + t (CTA-local)
+  // ---- CTA reduction buffer: red[wg * GS + (tile * 8 + row) * NCOL + column],
+  // tile = wn * Tw + t (CTA-local); GS is odd so that the warp blocks spread
+  // over the banks.
   const int r1 = lane >> 2, cq = lane & 3;
-  const int TT = p.Wn * p.Tw;  // tiles per CTA (max)
+  const int GS = p.Wn * p.Tw * C::RED + 1;
+  {
+    float* wr = red + g.wg * GS + (g.wn * p.Tw * 8 + r1) * NCOL;
 #pragma unroll
-  for (int t = 0; t < gd::kMaxTw; ++t) {
-    if (t < g.tw) {
+    for (int tp = 0; tp < gd::kMaxTp; ++tp)
 #pragma unroll
-      for (int mt = 0; mt < MT; ++mt)
+      for (int e = 0; e < 4; ++e) {
+        const int t = 2 * tp + (e >> 1);
+        if (t < g.tw) {
 #pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          const int r = 16 * mt + 8 * hf + r1;
-          *reinterpret_cast<float2*>(red + ((g.wg * TT + g.wn * p.Tw + t) * 16 * MT + r) * 8 + 2 * cq) =
-              make_float2(acc[t][mt][2 * hf], acc[t][mt][2 * hf + 1]);
+          for (int nn = 0; nn < NN; ++nn) {
+            const int n = 8 * nn + 2 * cq + (e & 1);
+            if (n < NCOL) wr[t * 8 * NCOL + n] = acc[tp][nn][e];
+          }
         }
-    }
+      }
   }
   __syncthreads();
-  // per (b, row of this cluster): sum over the warps of the same tile (set
-  // blocks, fixed order) and over the digit rows of batch b; then to the owning
-  // CTA (or straight to y when S = 1).  Set blocks without sets are skipped.
-  const int R8 = 8 * g.Tq;
+  // Output o = (row rl of this cluster, batch b), o = rl * NB + b: T threads
+  // each sum the three digit columns of b over every T-th warp block (fixed
+  // order; blocks without sets wrote nothing and are skipped), then a T-lane
+  // butterfly.  The sum goes to the owning CTA (or straight to y when S = 1).
+  const int R8 = 8 * g.Tq, O = NB * R8;
+  int lgT = 0;
+  while (lgT < p.lgWg && (O << (lgT + 1)) <= NW * 32) ++lgT;
+  const int T = 1 << lgT, j = threadIdx.x & (T - 1);
   if (p.S > 1 && wait_cluster) cluster_wait();  // every CTA of the cluster has started
-  for (int b = 0; b < NB; ++b) {
-    for (int rl = threadIdx.x; rl < R8; rl += gd::kThreads) {
-      const int tile = rl >> 3, n = rl & 7;
-      float sum = 0.f;
-      for (int g2 = 0; g2 < p.Wg; ++g2) {
-        const int s0 = g.cs0 + ((g2 * g.nsc) >> p.lgWg), s1 = g.cs0 + (((g2 + 1) * g.nsc) >> p.lgWg);
-        if (s1 <= s0) continue;
-        const float* rp = red + ((g2 * TT + tile) * 16 * MT) * 8 + n;
-#pragma unroll
-        for (int gj = 0; gj < G; ++gj)
-#pragma unroll
-          for (int pp = 0; pp < 3; ++pp) sum += rp[((gj * NB + b) * 3 + pp) * 8];
+  for (int o0 = 0; o0 < O; o0 += NW * 32 >> lgT) {  // trip count uniform over the CTA
+    const int o = o0 + (threadIdx.x >> lgT);
+    const int rl = o / NB, b = o - rl * NB;
+    float sum = 0.f;
+    if (o < O) {
+      const float* rp = red + rl * NCOL + 3 * b;
+      for (int g2 = j; g2 < p.Wg; g2 += T) {
+        if ((((g2 + 1) * g.nsc) >> p.lgWg) <= ((g2 * g.nsc) >> p.lgWg)) continue;
+        const float* q = rp + g2 * GS;
+        sum += (q[0] + q[1]) + q[2];
       }
+    }
+    for (int m = 1; m < T; m <<= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, m);
+    if (o < O && j == 0) {
       const int row = g.t0c * 8 + rl;
       if (p.S == 1) {
         if (row < p.N)
@@ -558,23 +576,22 @@ __device__ __forceinline__ void gd_finish(const GdParams& p, const GdGeom& g, co
   }
   if (p.S > 1) {
     cluster_sync();
-    const int lo = g.crank * p.chunk, hi = min(R8, lo + p.chunk);
-    for (int b = 0; b < NB; ++b) {
-      for (int ro = threadIdx.x; ro < hi - lo; ro += gd::kThreads) {
-        float sum = 0.f;
-        for (int c = 0; c < p.S; ++c) sum += part[(c * NB + b) * p.chunk + ro];
-        const int row = g.t0c * 8 + lo + ro;
-        if (row < p.N)
-          p.y[static_cast<int64_t>(b) * p.N + row] = p.rdiag ? __half2float(__ushort_as_half(p.rdiag[row])) * sum : sum;
-      }
+    const int lo = g.crank * p.chunk, cnt = max(0, min(R8, lo + p.chunk) - lo);
+    for (int i = threadIdx.x; i < NB * cnt; i += NW * 32) {
+      const int ro = i / NB, b = i - ro * NB;
+      float sum = 0.f;
+      for (int c = 0; c < p.S; ++c) sum += part[(c * NB + b) * p.chunk + ro];
+      const int row = g.t0c * 8 + lo + ro;
+      if (row < p.N)
+        p.y[static_cast<int64_t>(b) * p.N + row] = p.rdiag ? __half2float(__ushort_as_half(p.rdiag[row])) * sum : sum;
     }
   }
 }
 
-template <int NB>
-__global__ void __launch_bounds__(gd::kThreads, 1) gemv_direct_kernel(const GdParams p) {
+template <int NB, int NW>
+__global__ void __launch_bounds__(NW * 32, 1) gemv_direct_kernel(const GdParams p) {
   extern __shared__ __align__(16) unsigned char smem[];
-  const GdSmem L = gd_layout<NB>(p.Tw, p.NSw, p.P, p.S, p.chunk, p.NSc);
+  const GdSmem L = gd_layout<NB, NW>(p.Tw, p.NSw, p.P, p.S, p.chunk, p.NSc);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   unsigned char* wreg = smem + warp * L.warp_bytes;
   unsigned char* wts = wreg + L.wts;
@@ -593,22 +610,25 @@ __global__ void __launch_bounds__(gd::kThreads, 1) gemv_direct_kernel(const GdPa
     if (g.busy) gd_stage<NB>(p, g, wts, lane);
     gd_load_scales<NB>(p, g, 0, lane, sreg);
   }
-  if (p.x_f32) gd_prep_x<NB, true>(p, g, xs, warp, lane);
-  else gd_prep_x<NB, false>(p, g, xs, warp, lane);
+  uint4 xa[4];  // after the weight copies: the weights are the longer path
+  if (p.x_f32) gd_x_first<NB, true>(p, g, warp, lane, xa);
+  else gd_x_first<NB, false>(p, g, warp, lane, xa);
+  if (p.x_f32) gd_prep_x<NB, true, NW>(p, g, xs, warp, lane, xa);
+  else gd_prep_x<NB, false, NW>(p, g, xs, warp, lane, xa);
   gd_finish_scales<NB>(p, g, lane, sreg, scl);
   cp_async_wait_all();
   __syncthreads();
-  gd_finish<NB>(p, g, wts, scl, xs, reinterpret_cast<float*>(smem + L.red), reinterpret_cast<float*>(smem + L.part),
-                warp, lane, true);
+  gd_finish<NB, NW>(p, g, wts, scl, xs, reinterpret_cast<float*>(smem + L.red),
+                    reinterpret_cast<float*>(smem + L.part), warp, lane, true);
 }
 
 // ------------------------------------------------------------------ host side
 
-template <int NB>
+template <int NB, int NW>
 static int gd_max_clusters(int S, int smem_bytes) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(S * 64));
-  cfg.blockDim = dim3(gd::kThreads);
+  cfg.blockDim = dim3(NW * 32);
   cfg.dynamicSmemBytes = static_cast<size_t>(smem_bytes);
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -618,19 +638,19 @@ static int gd_max_clusters(int S, int smem_bytes) {
   cfg.attrs = attr;
   cfg.numAttrs = S > 1 ? 1 : 0;
   int n = 0;
-  if (ensure_dyn_smem(reinterpret_cast<const void*>(gemv_direct_kernel<NB>), smem_bytes) !=
+  if (ensure_dyn_smem(reinterpret_cast<const void*>(gemv_direct_kernel<NB, NW>), smem_bytes) !=
       cudaSuccess) {
     cudaGetLastError();
     return 0;
   }
   if (S > 1) {
-    if (cudaOccupancyMaxActiveClusters(&n, gemv_direct_kernel<NB>, &cfg) != cudaSuccess) {
+    if (cudaOccupancyMaxActiveClusters(&n, gemv_direct_kernel<NB, NW>, &cfg) != cudaSuccess) {
       cudaGetLastError();
       return 0;
     }
     return n;
   }
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, gemv_direct_kernel<NB>, gd::kThreads, smem_bytes) !=
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, gemv_direct_kernel<NB, NW>, NW * 32, smem_bytes) !=
       cudaSuccess) {
     cudaGetLastError();
     return 0;
@@ -648,7 +668,7 @@ struct GdPlan {
 // latency-bound; fitted to measured K splits), weights ~c_w
 // per weight, CTAs per SM rounded up, plus a fixed charge for a cluster
 // barrier.
-template <int NB>
+template <int NB, int NW>
 static bool gd_plan_for(int N, int NG, int S, int num_sms, int smem_cap, GdPlan* out) {
   using C = gd::Cfg<NB>;
   const int NT = (N + 7) / 8;
@@ -660,30 +680,30 @@ static bool gd_plan_for(int N, int NG, int S, int num_sms, int smem_cap, GdPlan*
   for (int iter = 0; iter < 8; ++iter) {
     const int Tmax = (NT + Q - 1) / Q;
     int Wn = 0;
-    for (int w = 1; w <= 8; w *= 2)
+    for (int w = 1; w <= NW; w *= 2)
       if ((Tmax + w - 1) / w <= gd::kMaxTw) {
         Wn = w;
         break;
       }
-    if (Wn == 0) {  // more rows per cluster than 8 warps x 4 n-tiles: more clusters
-      Q = (NT + 8 * gd::kMaxTw - 1) / (8 * gd::kMaxTw);
+    if (Wn == 0) {  // more rows per cluster than the warps' n-tiles: more clusters
+      Q = (NT + NW * gd::kMaxTw - 1) / (NW * gd::kMaxTw);
       continue;
     }
-    const int Wg = 8 / Wn;
+    const int Wg = NW / Wn;
     const int Tw = (Tmax + Wn - 1) / Wn;
     const int NSw = (nsc + Wg - 1) / Wg;
     const int span = NSw * 16 * C::G;
     const int P = ((span / (16 * C::G)) & 1) ? span : span + 16 * C::G;  // odd multiple: bank spread
     const int chunk = (8 * Tmax + S - 1) / S;
-    const GdSmem L = gd_layout<NB>(Tw, NSw, P, S, chunk, nsc);
+    const GdSmem L = gd_layout<NB, NW>(Tw, NSw, P, S, chunk, nsc);
     if (L.total > smem_cap) {
       if (Q >= NT) return false;
       Q = std::min(NT, Q * 2);  // fewer rows per CTA
       continue;
     }
-    const int occ = gd_max_clusters<NB>(S, L.total);
+    const int occ = gd_max_clusters<NB, NW>(S, L.total);
     if (occ <= 0) return false;
-    const double cw = NB <= 2 ? 0.6 : (NB <= 5 ? 1.0 : 1.5);
+    const double cw = NB <= 2 ? 0.35 : (NB <= 5 ? 1.0 : 1.2);
     const double xprep = 24.0 * NB * 128.0 * C::G * nsc;          // per CTA
     const double wts = 8.0 * Tmax * 128.0 * C::G * nsc * cw;      // per CTA
     const double ctas_per_sm = std::ceil(static_cast<double>(Q) * S / num_sms);
@@ -695,7 +715,7 @@ static bool gd_plan_for(int N, int NG, int S, int num_sms, int smem_cap, GdPlan*
 }
 
 struct GdPlanEntry {
-  int N, NG, NB, sms, dev, force;
+  int N, NG, NB, NW, sms, dev, force;
   bool ok;
   GdPlan plan;
 };
@@ -703,7 +723,7 @@ static GdPlanEntry g_gd_cache[64];
 static int g_gd_count = 0;
 static std::mutex g_gd_mu;
 
-template <int NB>
+template <int NB, int NW>
 static bool gd_cached_plan(int N, int NG, int num_sms, int smem_cap, int force_s, GdPlan* out) {
   int force = force_s;
   if (!force)
@@ -715,7 +735,8 @@ static bool gd_cached_plan(int N, int NG, int num_sms, int smem_cap, int force_s
     std::lock_guard<std::mutex> lock(g_gd_mu);
     for (int i = 0; i < g_gd_count; ++i) {
       const GdPlanEntry& e = g_gd_cache[i];
-      if (e.N == N && e.NG == NG && e.NB == NB && e.sms == num_sms && e.dev == dev && e.force == force) {
+      if (e.N == N && e.NG == NG && e.NB == NB && e.NW == NW && e.sms == num_sms && e.dev == dev &&
+          e.force == force) {
         *out = e.plan;
         return e.ok;
       }
@@ -726,28 +747,28 @@ static bool gd_cached_plan(int N, int NG, int num_sms, int smem_cap, int force_s
   for (int S = 1; S <= 8; S *= 2) {
     if (force && S != force) continue;
     GdPlan pl;
-    if (gd_plan_for<NB>(N, NG, S, num_sms, smem_cap, &pl) && (!ok || pl.cost < best.cost)) {
+    if (gd_plan_for<NB, NW>(N, NG, S, num_sms, smem_cap, &pl) && (!ok || pl.cost < best.cost)) {
       best = pl;
       ok = true;
     }
   }
   std::lock_guard<std::mutex> lock(g_gd_mu);
   const int i = g_gd_count < 64 ? g_gd_count++ : (N + NG + NB) & 63;
-  g_gd_cache[i] = GdPlanEntry{N, NG, NB, num_sms, dev, force, ok, best};
+  g_gd_cache[i] = GdPlanEntry{N, NG, NB, NW, num_sms, dev, force, ok, best};
   *out = best;
   return ok;
 }
 
-template <int NB>
+template <int NB, int NW>
 static cudaError_t launch_gemv_direct_nb(const GdParams& base, cudaStream_t stream, int num_sms, int smem_cap,
                                          int force_s) {
   GdPlan plan;
-  if (!gd_cached_plan<NB>(base.N, base.NG, num_sms, smem_cap, force_s, &plan)) return cudaErrorNotSupported;
+  if (!gd_cached_plan<NB, NW>(base.N, base.NG, num_sms, smem_cap, force_s, &plan)) return cudaErrorNotSupported;
   if (getenv("W1_VERBOSE"))
     fprintf(stderr,
-            "w1_gemv(direct) plan: N=%d NG=%d B=%d -> clusters=%d split=%d warps=%dx%d tiles/warp=%d "
+            "w1_gemv(direct) plan: N=%d NG=%d B=%d warps=%d -> clusters=%d split=%d warps=%dx%d tiles/warp=%d "
             "sets/warp=%d smem=%d\n",
-            base.N, base.NG, NB, plan.Q, plan.S, plan.Wn, plan.Wg, plan.Tw, plan.NSw, plan.smem);
+            base.N, base.NG, NB, NW, plan.Q, plan.S, plan.Wn, plan.Wg, plan.Tw, plan.NSw, plan.smem);
 
   GdParams p = base;
   p.S = plan.S;
@@ -770,11 +791,11 @@ static cudaError_t launch_gemv_direct_nb(const GdParams& base, cudaStream_t stre
   p.lgGw = lg2(plan.NSw * gd::Cfg<NB>::G);
   p.tq = p.NT / plan.Q;
   p.tr = p.NT - p.tq * plan.Q;
-  cudaError_t err = ensure_dyn_smem(reinterpret_cast<const void*>(gemv_direct_kernel<NB>), plan.smem);
+  cudaError_t err = ensure_dyn_smem(reinterpret_cast<const void*>(gemv_direct_kernel<NB, NW>), plan.smem);
   if (err != cudaSuccess) return err;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(plan.Q * plan.S));
-  cfg.blockDim = dim3(gd::kThreads);
+  cfg.blockDim = dim3(NW * 32);
   cfg.dynamicSmemBytes = static_cast<size_t>(plan.smem);
   cfg.stream = stream;
   cudaLaunchAttribute attr[2];
@@ -791,14 +812,30 @@ static cudaError_t launch_gemv_direct_nb(const GdParams& base, cudaStream_t stre
   }
   cfg.attrs = attr;
   cfg.numAttrs = na;
-  return cudaLaunchKernelEx(&cfg, gemv_direct_kernel<NB>, p);
+  return cudaLaunchKernelEx(&cfg, gemv_direct_kernel<NB, NW>, p);
 }
 
 // Returns cudaErrorNotSupported when the shape is outside this kernel's plan
 // (or outside the plan with the forced K split force_s; 0 = planner's choice).
+// warps: 8 or 16 per CTA.
+template <int NW>
+static cudaError_t launch_gemv_direct_nw(const GdParams& p, int B, cudaStream_t stream, int num_sms, int smem_cap,
+                                         int force_s) {
+  switch (B) {
+    case 1: return launch_gemv_direct_nb<1, NW>(p, stream, num_sms, smem_cap, force_s);
+    case 2: return launch_gemv_direct_nb<2, NW>(p, stream, num_sms, smem_cap, force_s);
+    case 3: return launch_gemv_direct_nb<3, NW>(p, stream, num_sms, smem_cap, force_s);
+    case 4: return launch_gemv_direct_nb<4, NW>(p, stream, num_sms, smem_cap, force_s);
+    case 5: return launch_gemv_direct_nb<5, NW>(p, stream, num_sms, smem_cap, force_s);
+    case 6: return launch_gemv_direct_nb<6, NW>(p, stream, num_sms, smem_cap, force_s);
+    case 7: return launch_gemv_direct_nb<7, NW>(p, stream, num_sms, smem_cap, force_s);
+    default: return launch_gemv_direct_nb<8, NW>(p, stream, num_sms, smem_cap, force_s);
+  }
+}
+
 cudaError_t launch_gemv_direct(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t K,
                                const uint16_t* x, int B, float* y, bool static_weights, cudaStream_t stream,
-                               int num_sms, int smem_cap, int force_s) {
+                               int num_sms, int smem_cap, int force_s, int warps) {
   if (N > (int64_t)1 << 30 || K > (int64_t)1 << 30) return cudaErrorNotSupported;
   GdParams p = {};
   p.signs = signs;
@@ -810,16 +847,8 @@ cudaError_t launch_gemv_direct(const uint32_t* signs, const uint16_t* scales, in
   p.K = static_cast<int>(K);
   p.NG = static_cast<int>(K / 128);
   p.early = static_weights ? 1 : 0;
-  switch (B) {
-    case 1: return launch_gemv_direct_nb<1>(p, stream, num_sms, smem_cap, force_s);
-    case 2: return launch_gemv_direct_nb<2>(p, stream, num_sms, smem_cap, force_s);
-    case 3: return launch_gemv_direct_nb<3>(p, stream, num_sms, smem_cap, force_s);
-    case 4: return launch_gemv_direct_nb<4>(p, stream, num_sms, smem_cap, force_s);
-    case 5: return launch_gemv_direct_nb<5>(p, stream, num_sms, smem_cap, force_s);
-    case 6: return launch_gemv_direct_nb<6>(p, stream, num_sms, smem_cap, force_s);
-    case 7: return launch_gemv_direct_nb<7>(p, stream, num_sms, smem_cap, force_s);
-    default: return launch_gemv_direct_nb<8>(p, stream, num_sms, smem_cap, force_s);
-  }
+  if (warps == 16) return launch_gemv_direct_nw<16>(p, B, stream, num_sms, smem_cap, force_s);
+  return launch_gemv_direct_nw<8>(p, B, stream, num_sms, smem_cap, force_s);
 }
 
 }  // namespace w1
