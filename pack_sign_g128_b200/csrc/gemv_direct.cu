@@ -847,7 +847,10 @@ cudaError_t launch_gemv_direct(const uint32_t* signs, const uint16_t* scales, in
   p.K = static_cast<int>(K);
   p.NG = static_cast<int>(K / 128);
   p.early = static_weights ? 1 : 0;
-  if (warps == 16) return launch_gemv_direct_nw<16>(p, B, stream, num_sms, smem_cap, force_s);
+  // A 16-warp CTA never shares an SM with the next launch's CTA (registers),
+  // so its plans may use up to twice the shared memory cap of 8-warp plans.
+  if (warps == 16)
+    return launch_gemv_direct_nw<16>(p, B, stream, num_sms, std::min(2 * smem_cap, 200 * 1024), force_s);
   return launch_gemv_direct_nw<8>(p, B, stream, num_sms, smem_cap, force_s);
 }
 
