@@ -48,7 +48,7 @@ KERNEL_OF_CHOICE = {"direct": "gemv_direct_kernel", "direct16": "gemv_direct_ker
 # shape captured; see profiles/.  Used to report the dominant kernel's traffic.
 CAPTURED_TRAFFIC = {
     "gemv_tc_kernel": {"shape": (4096, 11008, 8), "bytes": 6585344},
-    "gemv_direct_kernel": {"shape": (4096, 4096, 1), "bytes": 2433280},
+    "gemv_direct_kernel": {"shape": (4096, 4096, 1), "bytes": 2426880},
 }
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -518,6 +518,17 @@ def _pci_bus_id(torch, dev):
         return None
 
 
+def pin_gemv_choices(ops, path: str):
+    """Pin each sweep pair's kernel to the choice a previous bench line recorded
+    (its rows.gemv[*].choice), so that a profiled run launches the same kernels
+    as the plain run whose numbers it explains."""
+    with open(path) as f:
+        line = [ln for ln in f.read().splitlines() if ln.strip().startswith("{")][-1]
+    for r in json.loads(line)["rows"]["gemv"]:
+        if r.get("choice"):
+            ops.gemv_set_choice(r["N"], r["K"], r["B"], r["choice"])
+
+
 def run_gpu(args):
     import torch
     from pack_sign_g128_b200 import ops, synth
@@ -528,6 +539,8 @@ def run_gpu(args):
     props = torch.cuda.get_device_properties(local)
     l2 = int(getattr(props, "L2_cache_size", 126 * 2 ** 20) or 126 * 2 ** 20)
 
+    if args.choices:
+        pin_gemv_choices(ops, args.choices)
     if args.section != "all":
         rows = {}
         if args.section == "gemm":
@@ -710,6 +723,8 @@ def main():
                     help="issue the sweep's launches one by one instead of CUDA graphs (for ncu launch lists)")
     ap.add_argument("--shape", default="4096,4096,1",
                     help="N,K,B of the single GEMV that --section gemv1 launches (for ncu captures)")
+    ap.add_argument("--choices", default=None,
+                    help="JSON line of an earlier run: pin each GEMV pair to the kernel it chose (profiling)")
     ap.add_argument("--section", default="all", choices=["all", "gemm", "moe", "dbf", "gemv1"],
                     help="run one row only (for profiling); prints a rows-only JSON line")
     args = ap.parse_args()

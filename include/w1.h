@@ -125,10 +125,23 @@ int w1_gemv_ex(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t
 /*
  * w1_gemv_choice -- inspection: writes the kernel and K split that w1_gemv /
  * w1_gemv_ex has chosen for (N, K, B, flags) on the current device, as
- * "direct/<split>", "tc/<split>" or "ring/<split>" (split 0: the kernel's own
- * planner), or "" when no call has chosen yet.  Host only, no GPU work.
+ * "direct/<split>" (8 warps per CTA), "direct16/<split>" (16 warps),
+ * "tc/<split>" or "ring/<split>" (split 0: the kernel's own planner), or ""
+ * when no call has chosen yet.  Host only, no GPU work.
  */
 int w1_gemv_choice(int64_t N, int64_t K, int64_t B, uint32_t flags, char* out, size_t out_len);
+
+/*
+ * w1_gemv_set_choice -- pins the kernel for (N, K, B, flags) on the current
+ * device, in the same notation as w1_gemv_choice ("direct/1", "direct16/2",
+ * "tc/0", "ring/0"; direct splits 1, 2, 4, 8), replacing any earlier choice:
+ * later calls for that shape skip the first-call timing and use it.  For
+ * persisting a tuning across processes, or for profiling runs whose timing
+ * would choose differently.  A pinned kernel whose plan does not fit the
+ * shape fails its calls with W1_ERR_UNSUPPORTED.  Unknown name or invalid
+ * sizes: W1_ERR_SHAPE; null name: W1_ERR_NULL.  Host only, no GPU work.
+ */
+int w1_gemv_set_choice(int64_t N, int64_t K, int64_t B, uint32_t flags, const char* name);
 
 /*
  * w1_gemm -- prefill-regime product for many token rows (DBF post, section 4:

@@ -33,6 +33,7 @@ SIGNATURES = {
     "w1_gemv": (_int, [_p, _p, _i64, _i64, _p, _i64, _p, _p]),
     "w1_gemv_ex": (_int, [_p, _p, _i64, _i64, _p, _i64, _p, ctypes.c_uint32, _p]),
     "w1_gemv_choice": (_int, [_i64, _i64, _i64, ctypes.c_uint32, ctypes.c_char_p, _sz]),
+    "w1_gemv_set_choice": (_int, [_i64, _i64, _i64, ctypes.c_uint32, ctypes.c_char_p]),
     "w1_gemm": (_int, [_p, _p, _i64, _i64, _p, _i64, _p, _p, _sz, _p]),
     "w1_gemm_workspace_size": (_sz, [_i64, _i64]),
     "w1_moe_grouped": (_int, [_p, _p, _i64, _i64, _i64, _i64, _i64, _p, _p, _p, _p, _p, _p, _p, _p, _sz, _p]),

@@ -567,7 +567,58 @@ static int gemv_choice_name(int64_t N, int64_t K, int B, bool st, char* out, siz
   return snprintf(out, out_len, "%s/%d", kind, c.s);
 }
 
+// Parses "direct/<s>", "direct16/<s>", "tc/<s>", "ring/<s>" (w1_gemv_choice's
+// notation); false for anything else.
+static bool parse_gemv_choice(const char* name, GemvChoice* c) {
+  const char* slash = strchr(name, '/');
+  if (!slash) return false;
+  const size_t len = static_cast<size_t>(slash - name);
+  char* end = nullptr;
+  const long sp = strtol(slash + 1, &end, 10);
+  if (end == slash + 1 || *end != '\0' || sp < 0 || sp > 8) return false;
+  auto is = [&](const char* k) { return strlen(k) == len && strncmp(name, k, len) == 0; };
+  if (is("direct") || is("direct16")) {
+    if (sp != 1 && sp != 2 && sp != 4 && sp != 8) return false;
+    *c = GemvChoice{'d', static_cast<int>(sp), is("direct16") ? 16 : 8};
+  } else if (is("tc")) {
+    *c = GemvChoice{'t', static_cast<int>(sp), 0};
+  } else if (is("ring")) {
+    *c = GemvChoice{'m', 0, 0};
+  } else {
+    return false;
+  }
+  return true;
+}
+
+static int gemv_set_choice(int64_t N, int64_t K, int B, bool st, const GemvChoice& c) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return W1_ERR_CUDA;
+  }
+  std::lock_guard<std::mutex> lock(g_choice_mu);
+  for (int i = 0; i < g_nchoice; ++i) {
+    GemvChoiceEntry& e = g_choice[i];
+    if (e.dev == dev && e.N == N && e.K == K && e.B == B && e.st == st) {
+      e.c = c;
+      return W1_OK;
+    }
+  }
+  const int i = g_nchoice < 256 ? g_nchoice++ : static_cast<int>((N + K + B) & 255);
+  g_choice[i] = GemvChoiceEntry{dev, N, K, B, st, c};
+  return W1_OK;
+}
+
 }  // namespace w1
+
+extern "C" int w1_gemv_set_choice(int64_t N, int64_t K, int64_t B, uint32_t flags, const char* name) {
+  if (!name) return W1_ERR_NULL;
+  if (N <= 0 || K <= 0 || (K % 128) != 0 || B < 1 || B > 8) return W1_ERR_SHAPE;
+  if ((flags & ~static_cast<uint32_t>(W1_GEMV_STATIC_WEIGHTS)) != 0) return W1_ERR_SHAPE;
+  w1::GemvChoice c{0, 0, 0};
+  if (!w1::parse_gemv_choice(name, &c)) return W1_ERR_SHAPE;
+  return w1::gemv_set_choice(N, K, static_cast<int>(B), (flags & W1_GEMV_STATIC_WEIGHTS) != 0, c);
+}
 
 extern "C" int w1_gemv_choice(int64_t N, int64_t K, int64_t B, uint32_t flags, char* out, size_t out_len) {
   if (!out || out_len == 0) return W1_ERR_NULL;

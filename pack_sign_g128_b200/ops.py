@@ -91,11 +91,18 @@ def _aligned256(ws: torch.Tensor) -> int:
 
 
 def gemv_choice(N: int, K: int, B: int, static_weights: bool = False) -> str:
-    """The kernel/K split w1_gemv chose for this shape ("" before the first call)."""
+    """The kernel/K split w1_gemv chose for this shape ("" before the first call):
+    "direct/<split>" (8 warps per CTA), "direct16/<split>", "tc/<split>", "ring/<split>"."""
     buf = ctypes.create_string_buffer(64)
     st = _lib.call("w1_gemv_choice", N, K, B, W1_GEMV_STATIC_WEIGHTS if static_weights else 0, buf, 64)
     _lib.check(st, "w1_gemv_choice")
     return buf.value.decode()
+
+
+def gemv_set_choice(N: int, K: int, B: int, name: str, static_weights: bool = False) -> None:
+    """Pin w1_gemv's kernel for this shape ("direct/1", "direct16/2", "tc/0", "ring/0")."""
+    st = _lib.call("w1_gemv_set_choice", N, K, B, W1_GEMV_STATIC_WEIGHTS if static_weights else 0, name.encode())
+    _lib.check(st, "w1_gemv_set_choice")
 
 
 def w1_gemm(signs: torch.Tensor, scales: torch.Tensor, x: torch.Tensor, y: torch.Tensor | None = None,

@@ -59,6 +59,12 @@ def test_host_side_argument_errors(lib):
     assert lib.w1_gemv_choice(16, 128, 1, 0, None, 32) == _lib.W1_ERR_NULL
     assert lib.w1_gemv_choice(16, 100, 1, 0, buf, 32) == _lib.W1_ERR_SHAPE
     assert lib.w1_gemv_choice(16, 128, 9, 0, buf, 32) == _lib.W1_ERR_SHAPE
+    assert lib.w1_gemv_set_choice(16, 128, 1, 0, None) == _lib.W1_ERR_NULL
+    for bad in (b"direct", b"direct/3", b"direct/0", b"direct32/1", b"tc/x", b"gemv/1", b"direct/1 ", b""):
+        assert lib.w1_gemv_set_choice(16, 128, 1, 0, bad) == _lib.W1_ERR_SHAPE, bad
+    assert lib.w1_gemv_set_choice(16, 100, 1, 0, b"direct/1") == _lib.W1_ERR_SHAPE
+    assert lib.w1_gemv_set_choice(16, 128, 9, 0, b"direct/1") == _lib.W1_ERR_SHAPE
+    assert lib.w1_gemv_set_choice(16, 128, 1, 2, b"direct/1") == _lib.W1_ERR_SHAPE
     assert lib.w1_gemm(good, good, 16, 128, good, 0, good, good, 1 << 30, None) == _lib.W1_ERR_SHAPE
     assert lib.w1_gemm(good, good, 16, 128, good, 4, None, good, 1 << 30, None) == _lib.W1_ERR_NULL
     need = lib.w1_gemm_workspace_size(4, 128)

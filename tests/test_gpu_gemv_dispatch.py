@@ -42,3 +42,19 @@ def test_autotune_off_uses_the_rule(monkeypatch):
     assert ops.sync_status() == _lib.W1_OK
     y_ref, bound = O.matmul_ref(O.bf16_bits_to_f64(x), s, c, K)
     assert_within(y.cpu().numpy().astype(np.float64), y_ref, bound, what="rule dispatch")
+
+
+@pytest.mark.parametrize("name", ["direct/1", "direct/2", "direct16/1", "direct16/4", "tc/0", "ring/0"])
+def test_pinned_choice_is_used_and_reported(name):
+    """w1_gemv_set_choice replaces the timed choice: later calls report and run it."""
+    N, K, B = 2056, 2048, 4
+    W, x = synth.gemv_case(N, K, B, seed=19)
+    s, c = O.pack_ref_fast(W)
+    sd, cd, xd = words_dev(s), fp16_dev(c), bf16_dev(x)
+    ops.gemv_set_choice(N, K, B, name)
+    y = ops.w1_gemv(sd, cd, xd)
+    assert ops.sync_status() == _lib.W1_OK
+    assert ops.gemv_choice(N, K, B) == name
+    y_ref, bound = O.matmul_ref(O.bf16_bits_to_f64(x), s, c, K)
+    assert_within(y.cpu().numpy().astype(np.float64), y_ref, bound, what=f"pinned {name}")
+    assert ops.gemv_choice(N, K, B, static_weights=True) in ("", name)  # the flag keys its own entry
