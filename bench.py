@@ -404,7 +404,7 @@ def moe_rows(torch, ops, synth, peaks, iters: int = 8):
     flops = 2.0 * T * K * 3 * H * I
     tf = flops / (ms * 1e-3) / 1e12
     return {"T": T, "H": H, "I": I, "E": E, "top_k": K, "ms": ms, "tokens/s": T / (ms * 1e-3),
-            "TFLOP/s": tf, "frac_bf16_burst": tf / peaks["bf16_tflops"], "launches_per_call": 5}
+            "TFLOP/s": tf, "frac_bf16_burst": tf / peaks["bf16_tflops"], "launches_per_call": 7}
 
 
 def dbf_rows(torch, ops, synth, peaks, l2_bytes: int, iters: int = 5):

@@ -11,19 +11,20 @@
 // kept un-duplicated, fused SwiGLU, skipped empty tiles.
 //
 // Seven launches on one stream (programmatic dependent launch between them):
-//  1. route_kernel     warp per token: fp32 softmax, top-k by logit, weights.
+//  1. route_kernel     warp per token: fp32 softmax, top-k by logit, weights,
+//                      and the token's fp16 multiplier (a power of two).
 //  2. sort_kernel      one CTA: stable counting sort of the routes by expert
 //                      (deterministic), route -> sorted position map, and the
 //                      tile lists of the two grouped GEMMs (no empty tiles).
-//  3. gather_kernel    x rows in expert-sorted route order as fp16 with an
-//                      exact power of two per route (max |x| in [2^14, 2^15)).
+//  3. gather_kernel    x rows in expert-sorted route order as fp16, scaled by
+//                      the token's power of two (max |x| in [2^14, 2^15)).
 //  4. moe_gemm<GATEUP> tcgen05 grouped GEMM, swap-AB as in w1_gemm: the gate
 //                      and up rows of expert e as +-s fp16 (the group scale
 //                      with the weight's sign, exact) times the expert's
 //                      contiguous route rows; each accumulates all of K in
 //                      TMEM; the epilogue applies the route scale, SiLU(g) * u
 //                      and stores h (bf16) in sorted order.
-//  5. sg_prep_kernel   h -> fp16 with a power of two per route (sign_gemm.cu).
+//  5. hprep_kernel     h -> fp16 with a power of two per route.
 //  6. moe_gemm<DOWN>   the down rows of expert e times those rows; epilogue
 //                      multiplies by the route scale and the route weight and
 //                      stores the route output (fp32, sorted order).
@@ -42,8 +43,6 @@
 namespace w1 {
 
 bool make_tmap_bf16_sw128(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int box_rows);
-cudaError_t launch_sg_prep(const uint16_t* x, const uint16_t* bdiag, const uint16_t* mid, int64_t n, int64_t r,
-                          int64_t B, __half* xs, float* cscale, float* dscale, float* dinv, cudaStream_t stream);
 
 namespace moe {
 constexpr int TN_GU = 128;   // routes per gate/up tile
@@ -57,7 +56,7 @@ struct Tile {
 };
 
 struct Workspace {
-  size_t hdr, ids, wts, pos, sroute, stok, offsets, tiles_gu, tiles_d, h, rout, xs, xscale, hs, hscale, total;
+  size_t hdr, ids, wts, pos, sroute, stok, offsets, tiles_gu, tiles_d, h, rout, xs, xscale, hs, hscale, xcs, total;
   int max_tiles_gu, max_tiles_d;
 };
 
@@ -99,17 +98,63 @@ __host__ __device__ inline Workspace workspace_layout(int64_t T, int64_t H, int6
   off = align_up(off + 2 * static_cast<size_t>(R) * I, 1024);
   w.hscale = off;
   off = align_up(off + 4 * static_cast<size_t>(R), 256);
+  w.xcs = off;
+  off = align_up(off + 4 * static_cast<size_t>(T), 256);
   w.total = off;
   return w;
 }
 }  // namespace moe
 
+// ------------------------------------------------------------------ fp16 operand rows
+
+// Exponent c with max * 2^c in [2^14, 2^15) (0 for an all-zero row), at most
+// 126 so that 2^c and 2^-c stay normal floats.  Scaling a bf16 row by 2^c
+// keeps every value exact in fp16 (8 significant bits, no overflow).
+__device__ __forceinline__ int moe_pow2_exp(float mx) {
+  int c = 0;
+  if (mx > 0.f) {
+    int E;
+    frexpf(mx, &E);  // mx < 2^E
+    c = 15 - E;
+  }
+  return c < 126 ? c : 126;
+}
+
+__device__ __forceinline__ float bf16x8_absmax(const uint4& u, float mx) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    mx = fmaxf(mx, fmaxf(fabsf(__uint_as_float(w[q] << 16)), fabsf(__uint_as_float(w[q] & 0xFFFF0000u))));
+  return mx;
+}
+
+__device__ __forceinline__ uint4 bf16x8_to_f16(const uint4& u, float cs) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+  uint32_t o[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const __half2 h2 = __floats2half2_rn(__uint_as_float(w[q] << 16) * cs, __uint_as_float(w[q] & 0xFFFF0000u) * cs);
+    o[q] = *reinterpret_cast<const uint32_t*>(&h2);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+  return v;
+}
+
 // ------------------------------------------------------------------ 1. router
 
 // One warp per token.  Selection is by logit (the softmax is monotone, so this
-// is selection by probability without rounding ties); weights are fp32.
+// is selection by probability without rounding ties); weights are fp32.  The
+// warp also finds the token's fp16 multiplier 2^c for the gate/up operand
+// (xcs[t]), once per token instead of once per route.
 __global__ void __launch_bounds__(256) moe_route_kernel(const float* __restrict__ logits, int T, int E, int top_k,
-                                                        int* __restrict__ ids, float* __restrict__ wts) {
+                                                        int* __restrict__ ids, float* __restrict__ wts,
+                                                        const uint16_t* __restrict__ x, int H,
+                                                        float* __restrict__ xcs) {
   pdl_wait();
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
@@ -159,39 +204,17 @@ __global__ void __launch_bounds__(256) moe_route_kernel(const float* __restrict_
       }
       if ((be & 31) == lane) z[be >> 5] = -INFINITY;  // taken
     }
+    const uint4* xr = reinterpret_cast<const uint4*>(x + static_cast<int64_t>(warp) * H);
+    float m = 0.f;
+#pragma unroll 4
+    for (int i = lane; i < (H >> 3); i += 32) m = bf16x8_absmax(__ldg(xr + i), m);
+    m = warp_max(m);
+    if (lane == 0) xcs[warp] = ldexpf(1.f, moe_pow2_exp(m));
   }
   pdl_launch_dependents();
 }
 
 // ------------------------------------------------------------------ 2. sort + tiles
-
-// Block-wide exclusive scan of v over threads [0, n) (n <= blockDim.x <= 1024).
-__device__ inline int block_exclusive_scan(int v, int* tmp) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int incl = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int t = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-    if (lane >= o) incl += t;
-  }
-  if (lane == 31) tmp[warp] = incl;
-  __syncthreads();
-  if (warp == 0) {
-    const int nw = blockDim.x >> 5;
-    int w = (lane < nw) ? tmp[lane] : 0;
-    int wi = w;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int t = __shfl_up_sync(0xFFFFFFFFu, wi, o);
-      if (lane >= o) wi += t;
-    }
-    if (lane < nw) tmp[32 + lane] = wi - w;
-  }
-  __syncthreads();
-  const int r = incl - v + tmp[32 + warp];
-  __syncthreads();
-  return r;
-}
 
 struct SortArgs {
   const int* ids;
@@ -203,84 +226,177 @@ struct SortArgs {
   moe::Tile* tiles_gu;
   moe::Tile* tiles_d;
   int* hdr;
+  int stage;  // sorted routes staged in dynamic shared memory (R ints), written out coalesced
 };
+
+// Lanes of this warp holding the same expert id as this lane (ids in
+// [0, kMaxE), -1 for none): one ballot per id bit and one for validity.
+// Deterministic, and far cheaper than __match_any_sync on this part.
+__device__ __forceinline__ unsigned same_id_lanes(int e) {
+  static_assert(moe::kMaxE <= 256, "8 id bits");
+  const bool valid = e >= 0;
+  const unsigned vb = __ballot_sync(0xFFFFFFFFu, valid);
+  unsigned m = valid ? vb : ~vb;
+#pragma unroll
+  for (int b = 0; b < 8; ++b) {
+    const bool bit = (e >> b) & 1;
+    const unsigned bb = __ballot_sync(0xFFFFFFFFu, bit);
+    m &= bit ? bb : ~bb;
+  }
+  return m;
+}
 
 // One CTA of 1024 threads.  Warp w owns the contiguous route segment
 // [w L, (w+1) L); positions inside an expert follow route order (stable).
 __global__ void __launch_bounds__(1024) moe_sort_kernel(const SortArgs a) {
+  extern __shared__ int sorted[];  // a.stage: sorted position -> route
   __shared__ int cnt[moe::kMaxE];
-  __shared__ int tbl[32][moe::kMaxE];
-  __shared__ int tmp[64];
+  __shared__ int tbl[32][moe::kMaxE];  // per (segment, expert): count, then exclusive prefix
   __shared__ int offs[moe::kMaxE + 1];
+  __shared__ int pgu[moe::kMaxE + 1], pd[moe::kMaxE + 1];  // tile-list prefixes per expert
   pdl_wait();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   for (int i = threadIdx.x; i < 32 * moe::kMaxE; i += blockDim.x) (&tbl[0][0])[i] = 0;
-  __syncthreads();
   const int L = (a.R + 31) / 32;
   const int s0 = warp * L, s1 = min(a.R, s0 + L);
-  // per-(warp, expert) counts
-  for (int base = s0; base < s1; base += 32) {
-    const int r = base + lane;
-    const int e = (r < s1) ? a.ids[r] : -1;
-    const unsigned peers = __match_any_sync(0xFFFFFFFFu, e);
-    if (e >= 0 && (__ffs(peers) - 1) == lane) tbl[warp][e] += __popc(peers);
-    __syncwarp();
+  // this warp's expert ids: the first kPre rounds loaded at once (independent
+  // loads), later rounds (R > 32 * 32 * kPre) read in the loops
+  constexpr int kPre = 8;
+  int pre[kPre];
+#pragma unroll
+  for (int it = 0; it < kPre; ++it) {
+    const int r = s0 + 32 * it + lane;
+    pre[it] = (r < s1) ? a.ids[r] : -1;
+  }
+  auto id_of = [&](int it) {
+    int e = -1;
+#pragma unroll
+    for (int j = 0; j < kPre; ++j)
+      if (it == j) e = pre[j];
+    if (it >= kPre) {
+      const int r = s0 + 32 * it + lane;
+      e = (r < s1) ? a.ids[r] : -1;
+    }
+    return e;
+  };
+  const int rounds = (s1 - s0 + 31) / 32;  // uniform over the warp
+  __syncthreads();
+  // per-(segment, expert) counts (order-free: shared-memory atomics)
+  for (int it = 0; it < rounds; ++it) {
+    const int e = id_of(it);
+    if (e >= 0) atomicAdd(&tbl[warp][e], 1);
   }
   __syncthreads();
-  // expert totals and offsets
-  int c = 0;
-  if (threadIdx.x < a.E)
-    for (int w = 0; w < 32; ++w) c += tbl[w][threadIdx.x];
-  const int off = block_exclusive_scan(threadIdx.x < a.E ? c : 0, tmp);
-  if (threadIdx.x < a.E) {
-    cnt[threadIdx.x] = c;
-    offs[threadIdx.x] = off;
-    a.offsets[threadIdx.x] = off;
-    int run = off;
-    for (int w = 0; w < 32; ++w) {
-      const int t = tbl[w][threadIdx.x];
-      tbl[w][threadIdx.x] = run;
-      run += t;
+  // per expert: exclusive prefix over the segments (warp j takes experts j,
+  // j + 32, ...; lane = segment) and the expert's total
+  for (int e = warp; e < a.E; e += 32) {
+    const int v = tbl[lane][e];
+    int incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+      if (lane >= o) incl += t;
     }
-    if (threadIdx.x == a.E - 1) {
-      offs[a.E] = run;
-      a.offsets[a.E] = run;
+    tbl[lane][e] = incl - v;
+    if (lane == 31) cnt[e] = incl;
+  }
+  __syncthreads();
+  // expert offsets and tile-list prefixes: one warp, lane l takes experts
+  // [l EPL, (l+1) EPL) in order, then a warp scan of the lane totals
+  if (warp == 0) {
+    const int EPL = (a.E + 31) / 32;
+    int c0 = 0, g0 = 0, d0 = 0;
+    for (int k = 0; k < EPL; ++k) {
+      const int e = lane * EPL + k;
+      if (e < a.E) {
+        const int c = cnt[e];
+        c0 += c;
+        g0 += (c + moe::TN_GU - 1) / moe::TN_GU * a.rt_gu;
+        d0 += (c + moe::TN_D - 1) / moe::TN_D * a.rt_d;
+      }
+    }
+    int ci = c0, gi = g0, di = d0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int tc = __shfl_up_sync(0xFFFFFFFFu, ci, o);
+      const int tg = __shfl_up_sync(0xFFFFFFFFu, gi, o);
+      const int td = __shfl_up_sync(0xFFFFFFFFu, di, o);
+      if (lane >= o) {
+        ci += tc;
+        gi += tg;
+        di += td;
+      }
+    }
+    int cb = ci - c0, gb = gi - g0, db = di - d0;
+    for (int k = 0; k < EPL; ++k) {
+      const int e = lane * EPL + k;
+      if (e < a.E) {
+        const int c = cnt[e];
+        offs[e] = cb;
+        pgu[e] = gb;
+        pd[e] = db;
+        cb += c;
+        gb += (c + moe::TN_GU - 1) / moe::TN_GU * a.rt_gu;
+        db += (c + moe::TN_D - 1) / moe::TN_D * a.rt_d;
+      }
+    }
+    if (lane == 31) {
+      offs[a.E] = ci;
+      pgu[a.E] = gi;
+      pd[a.E] = di;
     }
   }
   __syncthreads();
+  if (threadIdx.x <= a.E) a.offsets[threadIdx.x] = offs[threadIdx.x];
   // stable scatter
-  for (int base = s0; base < s1; base += 32) {
-    const int r = base + lane;
-    const int e = (r < s1) ? a.ids[r] : -1;
-    const unsigned peers = __match_any_sync(0xFFFFFFFFu, e);
+  for (int it = 0; it < rounds; ++it) {
+    const int r = s0 + 32 * it + lane;
+    const int e = id_of(it);
+    const unsigned peers = same_id_lanes(e);
     if (e >= 0) {
-      const int p = tbl[warp][e] + __popc(peers & ((1u << lane) - 1u));
-      a.sroute[p] = r;
-      a.stok[p] = r / a.top_k;
+      const int p = offs[e] + tbl[warp][e] + __popc(peers & ((1u << lane) - 1u));
+      if (a.stage) {
+        sorted[p] = r;
+      } else {
+        a.sroute[p] = r;
+        a.stok[p] = r / a.top_k;
+      }
       a.pos[r] = p;
     }
     __syncwarp();
     if (e >= 0 && (__ffs(peers) - 1) == lane) tbl[warp][e] += __popc(peers);
     __syncwarp();
   }
-  // tile lists: expert-major, every tile holds >= 1 route
-  const int e = threadIdx.x;
-  const int ce = (e < a.E) ? cnt[e] : 0;
-  const int ngu = (ce + moe::TN_GU - 1) / moe::TN_GU, nd = (ce + moe::TN_D - 1) / moe::TN_D;
-  const int bgu = block_exclusive_scan(e < a.E ? ngu * a.rt_gu : 0, tmp);
-  const int bd = block_exclusive_scan(e < a.E ? nd * a.rt_d : 0, tmp);
-  if (e < a.E) {
-    int k = bgu;
-    for (int j = 0; j < ngu; ++j)
-      for (int rt = 0; rt < a.rt_gu; ++rt)
-        a.tiles_gu[k++] = moe::Tile{e, rt, offs[e] + j * moe::TN_GU, min(moe::TN_GU, ce - j * moe::TN_GU)};
-    k = bd;
-    for (int j = 0; j < nd; ++j)
-      for (int rt = 0; rt < a.rt_d; ++rt)
-        a.tiles_d[k++] = moe::Tile{e, rt, offs[e] + j * moe::TN_D, min(moe::TN_D, ce - j * moe::TN_D)};
-    if (e == a.E - 1) {  // totals = last exclusive prefix + last expert's tiles
-      a.hdr[0] = bgu + ngu * a.rt_gu;
-      a.hdr[1] = bd + nd * a.rt_d;
+  // tile lists, expert-major (route tile, then row tile), one tile per thread
+  auto expert_of = [&](const int* pre_e, int i) {  // largest e with pre_e[e] <= i
+    int lo = 0, hi = a.E - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (pre_e[mid] <= i) lo = mid;
+      else hi = mid - 1;
+    }
+    return lo;
+  };
+  for (int i = threadIdx.x; i < pgu[a.E]; i += blockDim.x) {
+    const int e = expert_of(pgu, i), loc = i - pgu[e];
+    const int j = loc / a.rt_gu, rt = loc - j * a.rt_gu;
+    a.tiles_gu[i] = moe::Tile{e, rt, offs[e] + j * moe::TN_GU, min(moe::TN_GU, cnt[e] - j * moe::TN_GU)};
+  }
+  for (int i = threadIdx.x; i < pd[a.E]; i += blockDim.x) {
+    const int e = expert_of(pd, i), loc = i - pd[e];
+    const int j = loc / a.rt_d, rt = loc - j * a.rt_d;
+    a.tiles_d[i] = moe::Tile{e, rt, offs[e] + j * moe::TN_D, min(moe::TN_D, cnt[e] - j * moe::TN_D)};
+  }
+  if (threadIdx.x == 0) {
+    a.hdr[0] = pgu[a.E];
+    a.hdr[1] = pd[a.E];
+  }
+  if (a.stage) {  // sorted route order out, coalesced
+    __syncthreads();
+    for (int i = threadIdx.x; i < a.R; i += blockDim.x) {
+      const int r = sorted[i];
+      a.sroute[i] = r;
+      a.stok[i] = r / a.top_k;
     }
   }
   pdl_launch_dependents();
@@ -581,68 +697,62 @@ __global__ void __launch_bounds__(moe::kThreads, 1)
 
 // ------------------------------------------------------------------ gather x rows (sorted, fp16)
 
-// One CTA per sorted route p: xs[p] = fp16(x[stok[p]] * 2^c), xscale[p] = 2^-c
-// with max |x| * 2^c in [2^14, 2^15) (exact scaling of every bf16 value in range).
-// 16-byte loads and stores; the row stays in registers between the max and the
-// conversion (H <= 8 * 256 * kMaxV), longer rows are read twice.
+// One warp per sorted route p: xs[p] = fp16(x[t] * 2^c_t) for t = stok[p], with
+// the token's multiplier from the router (max |x_t| * 2^c_t in [2^14, 2^15):
+// exact for every bf16 value), xscale[p] = 2^-c_t.  A plain streaming copy:
+// 16-byte loads and stores, no reduction.
 __global__ void __launch_bounds__(256) moe_gather_kernel(const uint16_t* __restrict__ x, const int* __restrict__ stok,
-                                                         int H, __half* __restrict__ xs, float* __restrict__ xscale) {
-  constexpr int kMaxV = 4;
+                                                         const float* __restrict__ xcs, int R, int H,
+                                                         __half* __restrict__ xs, float* __restrict__ xscale) {
   pdl_wait();
-  __shared__ float red[8];
-  const int pr = blockIdx.x;
-  const uint4* xr = reinterpret_cast<const uint4*>(x + static_cast<int64_t>(__ldg(stok + pr)) * H);
-  const int nv = H >> 3;  // 16-byte vectors per row
-  uint4 v[kMaxV];
-  float mx = 0.f;
-#pragma unroll
-  for (int j = 0; j < kMaxV; ++j) {
-    const int i = threadIdx.x + 256 * j;
-    v[j] = i < nv ? __ldg(xr + i) : make_uint4(0, 0, 0, 0);
-    const uint32_t w[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
-#pragma unroll
-    for (int q = 0; q < 4; ++q)
-      mx = fmaxf(mx, fmaxf(fabsf(__uint_as_float(w[q] << 16)), fabsf(__uint_as_float(w[q] & 0xFFFF0000u))));
+  const int p = static_cast<int>((static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5);
+  const int lane = threadIdx.x & 31;
+  if (p < R) {
+    const int t = __ldg(stok + p);
+    const float cs = __ldg(xcs + t);
+    const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<int64_t>(t) * H);
+    uint4* dst = reinterpret_cast<uint4*>(xs + static_cast<int64_t>(p) * H);
+#pragma unroll 4
+    for (int i = lane; i < (H >> 3); i += 32) dst[i] = bf16x8_to_f16(__ldg(src + i), cs);
+    if (lane == 0) xscale[p] = 1.f / cs;  // exact: cs is a normal power of two
   }
-  for (int i = threadIdx.x + 256 * kMaxV; i < nv; i += 256) {
-    const uint4 u = __ldg(xr + i);
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+  pdl_launch_dependents();
+}
+
+// ------------------------------------------------------------------ h rows -> fp16
+
+// One warp per sorted route p: hs[p] = fp16(h[p] * 2^c) with max |h[p]| * 2^c
+// in [2^14, 2^15), hscale[p] = 2^-c.  The row stays in registers between the
+// max and the conversion when I <= 32 * 8 * kKeep, longer rows are re-read.
+__global__ void __launch_bounds__(256) moe_hprep_kernel(const uint16_t* __restrict__ h, int R, int I,
+                                                        __half* __restrict__ hs, float* __restrict__ hscale) {
+  constexpr int kKeep = 8;
+  pdl_wait();
+  const int p = static_cast<int>((static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5);
+  const int lane = threadIdx.x & 31;
+  if (p < R) {
+    const uint4* src = reinterpret_cast<const uint4*>(h + static_cast<int64_t>(p) * I);
+    uint4* dst = reinterpret_cast<uint4*>(hs + static_cast<int64_t>(p) * I);
+    const int nv = I >> 3;
+    uint4 keep[kKeep];
+    float m = 0.f;
 #pragma unroll
-    for (int q = 0; q < 4; ++q)
-      mx = fmaxf(mx, fmaxf(fabsf(__uint_as_float(w[q] << 16)), fabsf(__uint_as_float(w[q] & 0xFFFF0000u))));
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
-  __syncthreads();
-  mx = 0.f;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) mx = fmaxf(mx, red[i]);
-  int c = 0;
-  if (mx > 0.f) {
-    int E;
-    frexpf(mx, &E);  // mx < 2^E
-    c = 15 - E;
-  }
-  const float cs = ldexpf(1.f, c);
-  uint4* dst = reinterpret_cast<uint4*>(xs + static_cast<int64_t>(pr) * H);
-  auto convert = [&](const uint4& u) {
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-    uint32_t o[4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const __half2 h2 = __floats2half2_rn(__uint_as_float(w[q] << 16) * cs, __uint_as_float(w[q] & 0xFFFF0000u) * cs);
-      o[q] = *reinterpret_cast<const uint32_t*>(&h2);
+    for (int j = 0; j < kKeep; ++j) {
+      const int i = lane + 32 * j;
+      keep[j] = i < nv ? __ldg(src + i) : make_uint4(0, 0, 0, 0);
+      m = bf16x8_absmax(keep[j], m);
     }
-    return make_uint4(o[0], o[1], o[2], o[3]);
-  };
+    for (int i = lane + 32 * kKeep; i < nv; i += 32) m = bf16x8_absmax(__ldg(src + i), m);
+    const int c = moe_pow2_exp(warp_max(m));
+    const float cs = ldexpf(1.f, c);
 #pragma unroll
-  for (int j = 0; j < kMaxV; ++j) {
-    const int i = threadIdx.x + 256 * j;
-    if (i < nv) dst[i] = convert(v[j]);
+    for (int j = 0; j < kKeep; ++j) {
+      const int i = lane + 32 * j;
+      if (i < nv) dst[i] = bf16x8_to_f16(keep[j], cs);
+    }
+    for (int i = lane + 32 * kKeep; i < nv; i += 32) dst[i] = bf16x8_to_f16(__ldg(src + i), cs);
+    if (lane == 0) hscale[p] = ldexpf(1.f, -c);
   }
-  for (int i = threadIdx.x + 256 * kMaxV; i < nv; i += 256) dst[i] = convert(__ldg(xr + i));
-  if (threadIdx.x == 0) xscale[pr] = ldexpf(1.f, -c);
   pdl_launch_dependents();
 }
 
@@ -712,21 +822,28 @@ cudaError_t launch_moe(const uint16_t* x, const float* logits, int64_t T, int64_
 
   cudaError_t err;
   // 1. router
+  float* xcs = reinterpret_cast<float*>(ws + L.xcs);
   err = launch_pdl(moe_route_kernel, dim3(static_cast<unsigned>((T + 7) / 8)), dim3(256), 0, stream, logits,
-                   static_cast<int>(T), E, top_k, ids, wts);
+                   static_cast<int>(T), E, top_k, ids, wts, x, static_cast<int>(H), xcs);
   if (err != cudaSuccess) return err;
   // 2. sort + tile lists
-  SortArgs sa{ids, R, E, top_k, static_cast<int>(I / 128), static_cast<int>(H / 128), offsets, sroute, stok, pos,
-              tiles_gu, tiles_d, hdr};
-  err = launch_pdl(moe_sort_kernel, dim3(1), dim3(1024), 0, stream, sa);
+  constexpr int kStageMax = 16384;  // routes staged in shared memory (64 KB)
+  SortArgs sa{ids,  R,   E,       top_k,    static_cast<int>(I / 128), static_cast<int>(H / 128), offsets, sroute,
+              stok, pos, tiles_gu, tiles_d, hdr, R <= kStageMax ? 1 : 0};
+  const int sort_smem = sa.stage ? 4 * R : 0;
+  if (sort_smem > 0) {
+    err = ensure_dyn_smem(reinterpret_cast<const void*>(moe_sort_kernel), sort_smem);
+    if (err != cudaSuccess) return err;
+  }
+  err = launch_pdl(moe_sort_kernel, dim3(1), dim3(1024), static_cast<size_t>(sort_smem), stream, sa);
   if (err != cudaSuccess) return err;
   __half* xs = reinterpret_cast<__half*>(ws + L.xs);
   float* xscale = reinterpret_cast<float*>(ws + L.xscale);
   __half* hs = reinterpret_cast<__half*>(ws + L.hs);
   float* hscale = reinterpret_cast<float*>(ws + L.hscale);
   // 3. x rows in sorted route order, fp16 with a power of two per route
-  err = launch_pdl(moe_gather_kernel, dim3(static_cast<unsigned>(R)), dim3(256), 0, stream, x, stok,
-                   static_cast<int>(H), xs, xscale);
+  err = launch_pdl(moe_gather_kernel, dim3(static_cast<unsigned>((R + 7) / 8)), dim3(256), 0, stream, x, stok,
+                   static_cast<const float*>(xcs), R, static_cast<int>(H), xs, xscale);
   if (err != cudaSuccess) return err;
   // 4. gate/up with fused SwiGLU
   {
@@ -755,8 +872,8 @@ cudaError_t launch_moe(const uint16_t* x, const float* logits, int64_t T, int64_
     if (err != cudaSuccess) return err;
   }
   // 5. h -> fp16 with a power of two per route
-  err = launch_sg_prep(reinterpret_cast<const uint16_t*>(h), nullptr, nullptr, I, 0, R, hs, hscale, nullptr, nullptr,
-                       stream);
+  err = launch_pdl(moe_hprep_kernel, dim3(static_cast<unsigned>((R + 7) / 8)), dim3(256), 0, stream,
+                   reinterpret_cast<const uint16_t*>(h), R, static_cast<int>(I), hs, hscale);
   if (err != cudaSuccess) return err;
   // 6. down with route weights
   {

@@ -140,16 +140,17 @@ __global__ void __launch_bounds__(256) sg_prep_kernel(const uint16_t* __restrict
     mm = fmaxf(mm, red[2][i]);
   }
   // c: max |b x| 2^c in [2^14, 2^15);  d: mm * l1 * 2^d <= 2^15 (l1 rounded up)
+  // (both at most 126: 2^c, 2^d and their inverses stay normal floats)
   int c = 0, d = 0;
   if (mx > 0.f) {
     int E;
     frexpf(mx, &E);  // mx < 2^E
-    c = 15 - E;
+    c = min(15 - E, 126);
   }
   if (mm > 0.f && l1 > 0.f) {
     int E;
     frexpf(mm * l1 * 1.0001f, &E);  // < 2^E
-    d = 15 - E;
+    d = min(15 - E, 126);
   }
   const float cs = ldexpf(1.f, c);
   uint4* dst = reinterpret_cast<uint4*>(xs + static_cast<int64_t>(t) * n);
