@@ -49,7 +49,8 @@ constexpr int TN_GU = 128;   // routes per gate/up tile
 constexpr int TN_D = 128;    // routes per down tile
 constexpr int kMaxE = 256;
 constexpr int kMaxTopK = 32;
-constexpr int kThreads = 320;
+constexpr int kExpWarps = 8;                 // expander warps: 2 threads per weight row
+constexpr int kThreads = (6 + kExpWarps) * 32;  // producer, MMA, expanders, 4 epilogue warps
 
 struct Tile {
   int e, rt, start, count;  // expert, 128-row tile, first sorted route, routes
@@ -427,10 +428,14 @@ template <bool GATEUP>
 struct MoeCfg {
   static constexpr int TN = GATEUP ? moe::TN_GU : moe::TN_D;  // routes per tile (max MMA N)
   static constexpr int NMAT = GATEUP ? 2 : 1;                 // weight matrices per tile
-  static constexpr int BKS = 64;                              // K per pipeline stage
-  static constexpr int NS = 4;                                // stages
-  static constexpr int XSTAGE = TN * BKS * 2;                 // bytes of one B stage (fp16)
-  static constexpr int ASTAGE = 128 * BKS * 2;                // bytes of one weight matrix stage
+  // K per pipeline stage: one scale group, two 64-wide (128-byte) swizzle
+  // atoms; long stages amortise the MMA issuer's barrier wait over 8 x NMAT MMAs
+  static constexpr int BKS = 128;
+  static constexpr int NS = GATEUP ? 2 : 3;                   // stages (192 KB either way)
+  static constexpr int XATOM = TN * 128;                      // bytes of one 64-wide atom of B
+  static constexpr int XSTAGE = 2 * XATOM;                    // bytes of one B stage (fp16)
+  static constexpr int AATOM = 128 * 128;                     // bytes of one 64-wide atom of A
+  static constexpr int ASTAGE = 2 * AATOM;                    // bytes of one weight matrix stage
   static constexpr uint32_t kTmemCols = GATEUP ? 512 : 256;   // two accumulator sets
 };
 
@@ -438,7 +443,7 @@ template <bool GATEUP>
 struct MoeSmem {
   alignas(1024) unsigned char x[MoeCfg<GATEUP>::NS][MoeCfg<GATEUP>::XSTAGE];
   alignas(1024) unsigned char a[MoeCfg<GATEUP>::NS][MoeCfg<GATEUP>::NMAT][MoeCfg<GATEUP>::ASTAGE];
-  uint64_t full_x[MoeCfg<GATEUP>::NS], full_a[MoeCfg<GATEUP>::NS], empty[MoeCfg<GATEUP>::NS];
+  uint64_t full[MoeCfg<GATEUP>::NS], empty[MoeCfg<GATEUP>::NS];
   uint64_t full_c[2], empty_c[2];
   uint32_t tmem_base;
 };
@@ -447,12 +452,13 @@ __device__ __forceinline__ void moe_st_shared_v4(uint32_t addr, uint32_t a, uint
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
 
-// Warp roles: 0 TMA producer (route rows of B), 1 MMA issuer, 2-5 expanders
-// (thread = weight row: 2 sign words + the group scale per matrix -> 32 fp16
-// pairs +-s in the 128B-swizzled K-major layout), 6-9 epilogue (thread =
-// TMEM lane).  One 64-wide K stage: NMAT x 4 MMAs (M = 128, N = the tile's
-// route count rounded up to 16, K = 16), all of K into one accumulator per
-// matrix per tile; two accumulator sets alternate between tiles.
+// Warp roles: 0 TMA producer (route rows of B), 1 MMA issuer, 2-9 expanders
+// (two threads per weight row: sign words + the group scale -> fp16 pairs +-s
+// in the 128B-swizzled K-major layout; gate/up: one matrix each, down: one
+// word pair of the stage each), 10-13 epilogue (thread = TMEM lane).  One
+// 128-wide K stage: NMAT x 8 MMAs (M = 128, N = the tile's route count rounded
+// up to 16, K = 16), all of K into one accumulator per matrix per tile; two
+// accumulator sets alternate between tiles.
 template <bool GATEUP>
 __global__ void __launch_bounds__(moe::kThreads, 1)
     moe_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const MoeGemmParams p) {
@@ -463,8 +469,9 @@ __global__ void __launch_bounds__(moe::kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::NS; ++i) {
-      mbar_init(&sm.full_x[i], 1);
-      mbar_init(&sm.full_a[i], 128);
+      // one barrier per stage: the expanders' arrivals plus the producer's
+      // arrival with the activation tile's transaction bytes
+      mbar_init(&sm.full[i], 32 * moe::kExpWarps + 1);
       mbar_init(&sm.empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -495,8 +502,9 @@ __global__ void __launch_bounds__(moe::kThreads, 1)
         for (int ks = 0; ks < NKS; ++ks, ++c) {
           const int s = c % C::NS;
           if (!mbar_wait(&sm.empty[s], ((c / C::NS) & 1) ^ 1)) goto done_prod;
-          mbar_arrive_expect_tx(&sm.full_x[s], C::XSTAGE);
-          tma_load_2d(sm.x[s], &tmap_b, ks * C::BKS, tl.start, &sm.full_x[s]);
+          mbar_arrive_expect_tx(&sm.full[s], C::XSTAGE);
+          tma_load_2d(sm.x[s], &tmap_b, ks * C::BKS, tl.start, &sm.full[s]);
+          tma_load_2d(sm.x[s] + C::XATOM, &tmap_b, ks * C::BKS + 64, tl.start, &sm.full[s]);
         }
       }
     done_prod:;
@@ -513,8 +521,7 @@ __global__ void __launch_bounds__(moe::kThreads, 1)
         tc_fence_after();
         for (int ks = 0; ks < NKS; ++ks, ++c) {
           const int s = c % C::NS;
-          if (!mbar_wait(&sm.full_x[s], (c / C::NS) & 1)) goto done_mma;
-          if (!mbar_wait(&sm.full_a[s], (c / C::NS) & 1)) goto done_mma;
+          if (!mbar_wait(&sm.full[s], (c / C::NS) & 1)) goto done_mma;
           tc_fence_after();
           const uint32_t xbase = smem_u32(sm.x[s]);
 #pragma unroll
@@ -522,9 +529,11 @@ __global__ void __launch_bounds__(moe::kThreads, 1)
             const uint32_t d = tmem + (cb * C::NMAT + mat) * C::TN;
             const uint32_t abase = smem_u32(sm.a[s][mat]);
 #pragma unroll
-            for (int kk = 0; kk < C::BKS / 16; ++kk)
-              tc_mma_ss(d, smem_desc_sw128(abase + kk * 32), smem_desc_sw128(xbase + kk * 32), idesc,
+            for (int kk = 0; kk < C::BKS / 16; ++kk) {
+              const uint32_t ao = (kk >> 2) * C::AATOM + (kk & 3) * 32, xo = (kk >> 2) * C::XATOM + (kk & 3) * 32;
+              tc_mma_ss(d, smem_desc_sw128(abase + ao), smem_desc_sw128(xbase + xo), idesc,
                         (ks > 0 || kk > 0) ? 1u : 0u);
+            }
           }
           tc_commit(&sm.empty[s]);
         }
@@ -532,16 +541,22 @@ __global__ void __launch_bounds__(moe::kThreads, 1)
       }
     done_mma:;
     }
-  } else if (warp < 6) {
-    // expanders: thread = weight row of the tile's 128-row block
+  } else if (warp < 2 + moe::kExpWarps) {
+    // expanders: two threads per weight row of the tile's 128-row block.
+    // gate/up: half h expands matrix h (gate, up), all four sign words of a
+    // 128-wide stage; down: half h expands words 2h, 2h+1 (swizzle atom h).
     constexpr int kPf = 4;
-    const int rl = (warp - 2) * 32 + lane;
+    constexpr int NW = GATEUP ? 4 : 2;  // sign words per thread per stage
+    const int et = (warp - 2) * 32 + lane;
+    const int rl = et & 127, half = et >> 7;
+    const int mat = GATEUP ? half : 0;
+    const int w0 = GATEUP ? 0 : 2 * half;  // first word of the stage this thread expands
     const int64_t wrow = p.K >> 5;
     // the stream's current tile: row pointers cached in registers, the tile
     // descriptor read once per tile (not once per stage)
     int ld_ti = blockIdx.x, ld_ks = 0;
-    const uint2* wp[C::NMAT];
-    const uint16_t* sp[C::NMAT];
+    const uint32_t* wp = nullptr;
+    const uint16_t* sp = nullptr;
     bool ld_valid = false;
     auto load_tile = [&]() {
       ld_valid = false;
@@ -550,27 +565,29 @@ __global__ void __launch_bounds__(moe::kThreads, 1)
         const int row = tl.rt * 128 + rl;
         ld_valid = row < p.rows;
         const int64_t ridx = static_cast<int64_t>(tl.e) * p.rows + (ld_valid ? row : 0);
-#pragma unroll
-        for (int mat = 0; mat < C::NMAT; ++mat) {
-          wp[mat] = reinterpret_cast<const uint2*>((mat ? p.u_signs : p.a_signs) + ridx * wrow);
-          sp[mat] = (mat ? p.u_scales : p.a_scales) + ridx * NG;
-        }
+        wp = (mat ? p.u_signs : p.a_signs) + ridx * wrow + w0;
+        sp = (mat ? p.u_scales : p.a_scales) + ridx * NG;
       }
     };
     load_tile();
-    auto fetch = [&](uint2 (&w)[C::NMAT], uint32_t (&sc)[C::NMAT]) {
+    auto fetch = [&](uint32_t (&w)[NW], uint32_t& sc) {
 #pragma unroll
-      for (int mat = 0; mat < C::NMAT; ++mat) {
-        w[mat] = make_uint2(0, 0);
-        sc[mat] = 0x3C00u;
-      }
+      for (int i = 0; i < NW; ++i) w[i] = 0;
+      sc = 0x3C00u;
       if (ld_ti < ntiles) {
         if (ld_valid) {
-#pragma unroll
-          for (int mat = 0; mat < C::NMAT; ++mat) {
-            w[mat] = __ldg(wp[mat] + ld_ks);
-            sc[mat] = __ldg(sp[mat] + (ld_ks >> 1));
+          if constexpr (NW == 4) {  // a row's words are 16-byte aligned (K % 128 == 0)
+            const uint4 u = __ldg(reinterpret_cast<const uint4*>(wp) + ld_ks);
+            w[0] = u.x;
+            w[1 % NW] = u.y;
+            w[2 % NW] = u.z;
+            w[3 % NW] = u.w;
+          } else {
+            const uint2 u = __ldg(reinterpret_cast<const uint2*>(wp + 4 * ld_ks));
+            w[0] = u.x;
+            w[1 % NW] = u.y;
           }
+          sc = __ldg(sp + ld_ks);  // one scale group per stage
         }
         if (++ld_ks == NKS) {
           ld_ks = 0;
@@ -579,8 +596,8 @@ __global__ void __launch_bounds__(moe::kThreads, 1)
         }
       }
     };
-    uint2 wr[kPf][C::NMAT];
-    uint32_t sr[kPf][C::NMAT];
+    uint32_t wr[kPf][NW];
+    uint32_t sr[kPf];
 #pragma unroll
     for (int j = 0; j < kPf; ++j) fetch(wr[j], sr[j]);
     const int my_tiles = (ntiles - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) /
@@ -593,41 +610,36 @@ __global__ void __launch_bounds__(moe::kThreads, 1)
 #pragma unroll
       for (int j = 0; j < kPf; ++j) {
         if (c0 + j >= my_stages) break;
-        uint2 cur[C::NMAT];
-        uint32_t ss[C::NMAT];
+        uint32_t cur[NW];
 #pragma unroll
-        for (int mat = 0; mat < C::NMAT; ++mat) {
-          cur[mat] = wr[j][mat];
-          ss[mat] = sr[j][mat] * 0x00010001u;  // the scale in both fp16 halves
-        }
+        for (int i = 0; i < NW; ++i) cur[i] = wr[j][i];
+        const uint32_t ss = sr[j] * 0x00010001u;  // the scale in both fp16 halves
         fetch(wr[j], sr[j]);
         const int s = c % C::NS;
         if (!mbar_wait_warp(&sm.empty[s], ((c / C::NS) & 1) ^ 1)) goto done_exp;
+        const uint32_t abase = smem_u32(sm.a[s][mat]) + row_off;  // + atom offset per word pair
 #pragma unroll
-        for (int mat = 0; mat < C::NMAT; ++mat) {
-          const uint32_t abase = smem_u32(sm.a[s][mat]) + row_off;
-          const uint32_t words[2] = {cur[mat].x, cur[mat].y};
+        for (int wi = 0; wi < NW; ++wi) {
+          const uint32_t w = cur[wi];
+          uint32_t rr[16];
 #pragma unroll
-          for (int wi = 0; wi < 2; ++wi) {
-            const uint32_t w = words[wi];
-            uint32_t rr[16];
+          for (int pp = 0; pp < 16; ++pp) {
+            const uint32_t src = (pp < 8) ? w : (w >> 16);
+            const int b = 2 * (pp & 7);
+            const uint32_t m = src & (3u << b);
+            const uint32_t tt = m * (0x40008000u >> b);
+            rr[pp] = (tt & 0x80008000u) | ss;
+          }
+          const int gw = w0 + wi;  // word of the stage: atom gw / 2, chunks 4 (gw % 2) + q
+          const uint32_t ab = abase + static_cast<uint32_t>((gw >> 1) * C::AATOM);
 #pragma unroll
-            for (int pp = 0; pp < 16; ++pp) {
-              const uint32_t src = (pp < 8) ? w : (w >> 16);
-              const int b = 2 * (pp & 7);
-              const uint32_t m = src & (3u << b);
-              const uint32_t tt = m * (0x40008000u >> b);
-              rr[pp] = (tt & 0x80008000u) | ss[mat];
-            }
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const uint32_t chunk = static_cast<uint32_t>(wi * 4 + q);
-              moe_st_shared_v4(abase + ((chunk ^ swz) << 4), rr[4 * q], rr[4 * q + 1], rr[4 * q + 2], rr[4 * q + 3]);
-            }
+          for (int q = 0; q < 4; ++q) {
+            const uint32_t chunk = static_cast<uint32_t>((gw & 1) * 4 + q);
+            moe_st_shared_v4(ab + ((chunk ^ swz) << 4), rr[4 * q], rr[4 * q + 1], rr[4 * q + 2], rr[4 * q + 3]);
           }
         }
         fence_async_shared();
-        mbar_arrive(&sm.full_a[s]);
+        mbar_arrive(&sm.full[s]);
         ++c;
       }
     }
