@@ -46,7 +46,7 @@ struct Smem {
   static constexpr int kXStage = BMT * BKS * 2;
   alignas(1024) unsigned char x[NS][kXStage];
   alignas(1024) unsigned char a[NS][kAStage];
-  uint64_t full_x[NS], full_a[NS], empty[NS];
+  uint64_t full[NS], empty[NS];
   uint64_t full_c[2], empty_c[2];
   uint32_t tmem_base;
 };
@@ -209,8 +209,9 @@ __global__ void __launch_bounds__(sg::kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int i = 0; i < NS; ++i) {
-      mbar_init(&sm.full_x[i], 1);
-      mbar_init(&sm.full_a[i], 128);
+      // one barrier per stage: the expanders' 128 arrivals plus the producer's
+      // arrival with the activation tile's transaction bytes (one wait for the MMA issuer)
+      mbar_init(&sm.full[i], 129);
       mbar_init(&sm.empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -242,8 +243,8 @@ __global__ void __launch_bounds__(sg::kThreads, 1)
         for (int ks = 0; ks < NKS; ++ks, ++c) {
           const int s = c % NS;
           if (!mbar_wait(&sm.empty[s], ((c / NS) & 1) ^ 1)) goto done_prod;
-          mbar_arrive_expect_tx(&sm.full_x[s], kXStage);
-          tma_load_2d(sm.x[s], &tmap_b, ks * BKS, mt * BM, &sm.full_x[s]);
+          mbar_arrive_expect_tx(&sm.full[s], kXStage);
+          tma_load_2d(sm.x[s], &tmap_b, ks * BKS, mt * BM, &sm.full[s]);
         }
       }
     done_prod:;
@@ -258,8 +259,7 @@ __global__ void __launch_bounds__(sg::kThreads, 1)
         const uint32_t d = tmem + cb * BM;
         for (int ks = 0; ks < NKS; ++ks, ++c) {
           const int s = c % NS;
-          if (!mbar_wait(&sm.full_x[s], (c / NS) & 1)) goto done_mma;
-          if (!mbar_wait(&sm.full_a[s], (c / NS) & 1)) goto done_mma;
+          if (!mbar_wait(&sm.full[s], (c / NS) & 1)) goto done_mma;
           tc_fence_after();
           const uint32_t xbase = smem_u32(sm.x[s]);
           const uint32_t abase = smem_u32(sm.a[s]);
@@ -337,7 +337,7 @@ __global__ void __launch_bounds__(sg::kThreads, 1)
           }
         }
         fence_async_shared();
-        mbar_arrive(&sm.full_a[s]);
+        mbar_arrive(&sm.full[s]);
         ++c;
       }
     }
