@@ -39,36 +39,36 @@ struct DbfdSmem {
   int wb1, wb2, w1, w2, xs, red, part, total;
 };
 
-template <int NB>
+template <int NB, int NW>
 __host__ __device__ inline DbfdSmem dbfd_layout(const GdParams& p1, const GdParams& p2) {
   using C = gd::Cfg<NB>;
-  const GdSmem L1 = gd_layout<NB>(p1.Tw, p1.NSw, p1.P, p1.S, p1.chunk, p1.NSc);
-  const GdSmem L2 = gd_layout<NB>(p2.Tw, p2.NSw, p2.P, p2.S, p2.chunk, p2.NSc);
+  const GdSmem L1 = gd_layout<NB, NW>(p1.Tw, p1.NSw, p1.P, p1.S, p1.chunk, p1.NSc);
+  const GdSmem L2 = gd_layout<NB, NW>(p2.Tw, p2.NSw, p2.P, p2.S, p2.chunk, p2.NSc);
   DbfdSmem M;
   M.wb1 = L1.warp_bytes;
   M.wb2 = L2.warp_bytes;
   M.w1 = 0;
-  M.w2 = gd::kWarps * M.wb1;
-  M.xs = M.w2 + gd::kWarps * M.wb2;
+  M.w2 = NW * M.wb1;
+  M.xs = M.w2 + NW * M.wb2;
   const int nsc = p1.NSc > p2.NSc ? p1.NSc : p2.NSc;
   M.red = M.xs + (nsc * C::SCR * 4 + 15) / 16 * 16;
   const int tw = p1.Tw > p2.Tw ? p1.Tw : p2.Tw;
-  M.part = M.red + gd::gd_red_bytes<NB>(tw);
+  M.part = M.red + gd::gd_red_bytes<NB, NW>(tw);
   const int chunk = p1.chunk > p2.chunk ? p1.chunk : p2.chunk;
   M.total = M.part + (p1.S > 1 ? p1.S * NB * chunk * 4 : 0);
   return M;
 }
 
-template <int NB>
-__global__ void __launch_bounds__(gd::kThreads, 1) dbf_direct_kernel(const GdParams p1, const GdParams p2,
+template <int NB, int NW>
+__global__ void __launch_bounds__(NW * 32, 1) dbf_direct_kernel(const GdParams p1, const GdParams p2,
                                                                      unsigned int* bar) {
   extern __shared__ __align__(16) unsigned char smem[];
-  const DbfdSmem M = dbfd_layout<NB>(p1, p2);
+  const DbfdSmem M = dbfd_layout<NB, NW>(p1, p2);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   unsigned char* wr1 = smem + M.w1 + warp * M.wb1;
   unsigned char* wr2 = smem + M.w2 + warp * M.wb2;
-  const GdSmem L1 = gd_layout<NB>(p1.Tw, p1.NSw, p1.P, p1.S, p1.chunk, p1.NSc);
-  const GdSmem L2 = gd_layout<NB>(p2.Tw, p2.NSw, p2.P, p2.S, p2.chunk, p2.NSc);
+  const GdSmem L1 = gd_layout<NB, NW>(p1.Tw, p1.NSw, p1.P, p1.S, p1.chunk, p1.NSc);
+  const GdSmem L2 = gd_layout<NB, NW>(p2.Tw, p2.NSw, p2.P, p2.S, p2.chunk, p2.NSc);
   unsigned char* wts1 = wr1 + L1.wts;
   float* scl1 = reinterpret_cast<float*>(wr1 + L1.scl);
   unsigned char* wts2 = wr2 + L2.wts;
@@ -96,10 +96,10 @@ __global__ void __launch_bounds__(gd::kThreads, 1) dbf_direct_kernel(const GdPar
     gd_finish_scales<NB>(p2, g2, lane, sreg, scl2);
   }
   // ---- phase 1: h_scaled = mid (.) (V . (b (.) x))
-  gd_prep_x<NB, false>(p1, g1, xs, warp, lane, xa);
+  gd_prep_x<NB, false, NW>(p1, g1, xs, warp, lane, xa);
   asm volatile("cp.async.wait_group 1;" ::: "memory");  // V landed (U may still be in flight)
   __syncthreads();
-  gd_finish<NB>(p1, g1, wts1, scl1, xs, red, part, warp, lane, true);
+  gd_finish<NB, NW>(p1, g1, wts1, scl1, xs, red, part, warp, lane, true);
   // ---- every CTA's h_scaled is in memory, and every reader of this CTA's
   // scratch and inbox is done with phase 1
   if (!grid_barrier(bar, gridDim.x)) {
@@ -109,10 +109,10 @@ __global__ void __launch_bounds__(gd::kThreads, 1) dbf_direct_kernel(const GdPar
   }
   // ---- phase 2: y = a (.) (U . h_scaled)
   gd_x_first<NB, true>(p2, g2, warp, lane, xa);
-  gd_prep_x<NB, true>(p2, g2, xs, warp, lane, xa);
+  gd_prep_x<NB, true, NW>(p2, g2, xs, warp, lane, xa);
   cp_async_wait_all();
   __syncthreads();
-  gd_finish<NB>(p2, g2, wts2, scl2, xs, red, part, warp, lane, false);
+  gd_finish<NB, NW>(p2, g2, wts2, scl2, xs, red, part, warp, lane, false);
 }
 
 // ------------------------------------------------------------------ host side
@@ -120,7 +120,7 @@ __global__ void __launch_bounds__(gd::kThreads, 1) dbf_direct_kernel(const GdPar
 // Plan of one product for a fixed cluster size S and cluster count Q (the chain
 // kernel needs both products on the same grid).  False if a cluster's rows do
 // not fit the warps.
-template <int NB>
+template <int NB, int NW>
 static bool dbfd_plan(int N, int NG, int S, int Q, GdParams* p) {
   using C = gd::Cfg<NB>;
   const int NT = (N + 7) / 8;
@@ -130,7 +130,7 @@ static bool dbfd_plan(int N, int NG, int S, int Q, GdParams* p) {
   if (nsc > gd::kMaxSets) return false;
   const int Tmax = (NT + Q - 1) / Q;
   int Wn = 0;
-  for (int w = 1; w <= gd::kWarps; w *= 2)
+  for (int w = 1; w <= NW; w *= 2)
     if ((Tmax + w - 1) / w <= gd::kMaxTw) {
       Wn = w;
       break;
@@ -148,7 +148,7 @@ static bool dbfd_plan(int N, int NG, int S, int Q, GdParams* p) {
   p->Q = Q;
   p->NT = NT;
   p->Wn = Wn;
-  p->Wg = gd::kWarps / Wn;
+  p->Wg = NW / Wn;
   p->Tw = (Tmax + Wn - 1) / Wn;
   p->NSw = (nsc + p->Wg - 1) / p->Wg;
   const int span = p->NSw * 16 * C::G;
@@ -163,11 +163,11 @@ static bool dbfd_plan(int N, int NG, int S, int Q, GdParams* p) {
   return true;
 }
 
-template <int NB>
+template <int NB, int NW>
 static int dbfd_max_clusters(int S, int smem_bytes) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(S * 64));
-  cfg.blockDim = dim3(gd::kThreads);
+  cfg.blockDim = dim3(NW * 32);
   cfg.dynamicSmemBytes = static_cast<size_t>(smem_bytes);
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -177,9 +177,9 @@ static int dbfd_max_clusters(int S, int smem_bytes) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  if (ensure_dyn_smem(reinterpret_cast<const void*>(dbf_direct_kernel<NB>), smem_bytes) !=
+  if (ensure_dyn_smem(reinterpret_cast<const void*>(dbf_direct_kernel<NB, NW>), smem_bytes) !=
           cudaSuccess ||
-      cudaOccupancyMaxActiveClusters(&n, dbf_direct_kernel<NB>, &cfg) != cudaSuccess) {
+      cudaOccupancyMaxActiveClusters(&n, dbf_direct_kernel<NB, NW>, &cfg) != cudaSuccess) {
     cudaGetLastError();
     return 0;
   }
@@ -201,7 +201,7 @@ static double dbfd_cost(const GdParams& p) {
   return (xprep + wts) / 128.0 + (p.S > 1 ? 800.0 : 0.0);
 }
 
-template <int NB>
+template <int NB, int NW>
 static cudaError_t launch_dbf_small_nb(const uint16_t* a, const uint32_t* B1, const uint16_t* mid,
                                        const uint32_t* B2, const uint16_t* bd, int m, int r, int n,
                                        const uint16_t* x, float* y, float* h, unsigned int* bar,
@@ -213,10 +213,10 @@ static cudaError_t launch_dbf_small_nb(const uint16_t* a, const uint32_t* B1, co
     int Q = num_sms / S;
     for (int iter = 0; iter < 4; ++iter) {
       GdParams p1 = {}, p2 = {};
-      if (!dbfd_plan<NB>(r, n / 128, S, Q, &p1) || !dbfd_plan<NB>(m, r / 128, S, Q, &p2)) break;
-      const int smem = dbfd_layout<NB>(p1, p2).total;
+      if (!dbfd_plan<NB, NW>(r, n / 128, S, Q, &p1) || !dbfd_plan<NB, NW>(m, r / 128, S, Q, &p2)) break;
+      const int smem = dbfd_layout<NB, NW>(p1, p2).total;
       if (smem > smem_cap) break;
-      const int occ = dbfd_max_clusters<NB>(S, smem);
+      const int occ = dbfd_max_clusters<NB, NW>(S, smem);
       if (occ <= 0) break;
       if (occ < Q) {  // every CTA must be resident for the grid barrier
         Q = occ;
@@ -245,14 +245,14 @@ static cudaError_t launch_dbf_small_nb(const uint16_t* a, const uint32_t* B1, co
   p2.x_f32 = 1;
   p2.rdiag = a;
   p2.y = y;
-  cudaError_t err = ensure_dyn_smem(reinterpret_cast<const void*>(dbf_direct_kernel<NB>), smem);
+  cudaError_t err = ensure_dyn_smem(reinterpret_cast<const void*>(dbf_direct_kernel<NB, NW>), smem);
   if (err != cudaSuccess) return err;
   if (getenv("W1_VERBOSE"))
-    fprintf(stderr, "dbf plan: B=%d -> clusters=%d split=%d warps=%dx%d / %dx%d smem=%d\n", NB, Q, S, p1.Wn,
-            p1.Wg, p2.Wn, p2.Wg, smem);
+    fprintf(stderr, "dbf plan: B=%d warps=%d -> clusters=%d split=%d warps=%dx%d / %dx%d smem=%d\n", NB, NW, Q, S,
+            p1.Wn, p1.Wg, p2.Wn, p2.Wg, smem);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(Q * S));
-  cfg.blockDim = dim3(gd::kThreads);
+  cfg.blockDim = dim3(NW * 32);
   cfg.dynamicSmemBytes = static_cast<size_t>(smem);
   cfg.stream = stream;
   cudaLaunchAttribute attr[2];
@@ -269,7 +269,7 @@ static cudaError_t launch_dbf_small_nb(const uint16_t* a, const uint32_t* B1, co
   }
   cfg.attrs = attr;
   cfg.numAttrs = na;
-  return cudaLaunchKernelEx(&cfg, dbf_direct_kernel<NB>, p1, p2, bar);
+  return cudaLaunchKernelEx(&cfg, dbf_direct_kernel<NB, NW>, p1, p2, bar);
 }
 
 size_t dbf_tc_workspace_bytes(int64_t r, int64_t n, int64_t B);
@@ -299,10 +299,12 @@ cudaError_t launch_dbf(const uint16_t* a, const uint32_t* B1, const uint16_t* mi
     return launch_dbf_tc(a, B1, mid, B2, b, m, r, n, x, B, y, workspace, stream, num_sms);
   unsigned int* bar = reinterpret_cast<unsigned int*>(workspace);
   float* h = reinterpret_cast<float*>(static_cast<unsigned char*>(workspace) + 256);
-  // batches of up to 8 rows through a fused chain kernel: the direct core for
-  // groups of up to 4 rows, the ring core (dbf_ring.cu) above, as measured;
-  // W1_DBF_PATH=direct|ring forces one (testing knob)
+  // batches of up to 8 rows through a fused chain kernel: the direct core (8
+  // warps per CTA for groups of up to 3 rows, 16 above, as measured; the ring
+  // core in dbf_ring.cu measured slower at every group size).  Testing knobs:
+  // W1_DBF_PATH=direct|ring forces a core, W1_DBF_WARPS=8|16 the warp count.
   const char* path = getenv("W1_DBF_PATH");
+  const char* wenv = getenv("W1_DBF_WARPS");
   DbfParams rp = {};
   rp.a = a;
   rp.mid = mid;
@@ -317,13 +319,17 @@ cudaError_t launch_dbf(const uint16_t* a, const uint32_t* B1, const uint16_t* mi
     const uint16_t* xg = x + b0 * n;
     float* yg = y + b0 * m;
     const int im = static_cast<int>(m), ir = static_cast<int>(r), in = static_cast<int>(n);
-    const bool direct = path ? path[0] == 'd' : nb <= 4;
+    const bool direct = path ? path[0] == 'd' : true;
+    const bool w16 = wenv ? atoi(wenv) == 16 : nb >= 4;
     cudaError_t err;
     if (direct) {
       switch (nb) {
-#define W1_DBF_CASE(NBV)                                                                                        \
-  case NBV:                                                                                                     \
-    err = launch_dbf_small_nb<NBV>(a, B1, mid, B2, b, im, ir, in, xg, yg, h, bar, stream, num_sms, smem_cap); \
+#define W1_DBF_CASE(NBV)                                                                                     \
+  case NBV:                                                                                                  \
+    err = w16 ? launch_dbf_small_nb<NBV, 16>(a, B1, mid, B2, b, im, ir, in, xg, yg, h, bar, stream, num_sms, \
+                                             smem_cap)                                                      \
+              : launch_dbf_small_nb<NBV, 8>(a, B1, mid, B2, b, im, ir, in, xg, yg, h, bar, stream, num_sms,  \
+                                            smem_cap);                                                      \
     break;
         W1_DBF_CASE(1)
         W1_DBF_CASE(2)
@@ -333,7 +339,10 @@ cudaError_t launch_dbf(const uint16_t* a, const uint32_t* B1, const uint16_t* mi
         W1_DBF_CASE(6)
         W1_DBF_CASE(7)
         default:
-          err = launch_dbf_small_nb<8>(a, B1, mid, B2, b, im, ir, in, xg, yg, h, bar, stream, num_sms, smem_cap);
+          err = w16 ? launch_dbf_small_nb<8, 16>(a, B1, mid, B2, b, im, ir, in, xg, yg, h, bar, stream, num_sms,
+                                                 smem_cap)
+                    : launch_dbf_small_nb<8, 8>(a, B1, mid, B2, b, im, ir, in, xg, yg, h, bar, stream, num_sms,
+                                                smem_cap);
           break;
 #undef W1_DBF_CASE
       }

@@ -1,9 +1,9 @@
 """dbf_apply on the GPU vs the fp64 oracle chain.
 
-Every test runs with each of the two fused small-batch chain kernels forced
-(W1_DBF_PATH=direct: the direct GEMV core, the default for groups of up to 4
-rows; =ring: the ring core, the default above); batches of 64 and more take
-the tensor-core path either way."""
+Every test runs with each fused small-batch chain kernel forced: the direct
+GEMV core (W1_DBF_PATH=direct, the default) with 8 and with 16 warps per CTA
+(W1_DBF_WARPS), and the ring core (=ring).  Batches of 64 and more take the
+tensor-core path either way."""
 import functools
 
 import numpy as np
@@ -17,9 +17,11 @@ from gpu_helpers import assert_within, bf16_dev, fp16_dev, words_dev
 pytestmark = pytest.mark.gpu
 
 
-@pytest.fixture(autouse=True, params=["direct", "ring"])
+@pytest.fixture(autouse=True, params=["direct8", "direct16", "ring"])
 def dbf_path(request, monkeypatch):
-    monkeypatch.setenv("W1_DBF_PATH", request.param)
+    monkeypatch.setenv("W1_DBF_PATH", "ring" if request.param == "ring" else "direct")
+    if request.param != "ring":
+        monkeypatch.setenv("W1_DBF_WARPS", request.param[6:])
     return request.param
 
 
