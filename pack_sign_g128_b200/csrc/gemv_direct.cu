@@ -94,6 +94,7 @@ struct GdParams {
   int lgGw;   // log2 of the power-of-two stride >= NSw * G (staging loops)
   int tq, tr;  // NT = Q * tq + tr
   int early;  // read weights before the grid dependency wait
+  int alias_red;  // the reduction buffer overlays the activation scratch (plans that need the room)
 };
 
 struct GdSmem {
@@ -103,16 +104,22 @@ struct GdSmem {
 // Per warp: staged sign words (8*Tw rows of P bytes), scales (float,
 // [group][row]).  Per CTA: activation scratch (nsc sets of SCR words), the
 // reduction buffer and (cluster) the owner partials.
+// With alias_red the reduction buffer starts at the activation scratch (it is
+// written only after every warp has finished its products).  The cluster
+// inbox never overlays anything: other CTAs may write it at any time.
 template <int NB, int NW = gd::kWarps>
-__host__ __device__ inline GdSmem gd_layout(int Tw, int NSw, int P, int S, int chunk, int nsc) {
+__host__ __device__ inline GdSmem gd_layout(int Tw, int NSw, int P, int S, int chunk, int nsc,
+                                            bool alias_red = false) {
   using C = gd::Cfg<NB>;
   GdSmem L;
   L.wts = 0;
   L.scl = L.wts + 8 * Tw * P;
   L.warp_bytes = (L.scl + NSw * C::G * 8 * Tw * 4 + 15) / 16 * 16;
   L.xs = NW * L.warp_bytes;
-  L.red = L.xs + (nsc * C::SCR * 4 + 15) / 16 * 16;
-  L.part = L.red + gd::gd_red_bytes<NB, NW>(Tw);
+  const int xs_bytes = (nsc * C::SCR * 4 + 15) / 16 * 16;
+  const int red_bytes = gd::gd_red_bytes<NB, NW>(Tw);
+  L.red = alias_red ? L.xs : L.xs + xs_bytes;
+  L.part = alias_red ? L.xs + (xs_bytes > red_bytes ? xs_bytes : red_bytes) : L.red + red_bytes;
   L.total = L.part + (S > 1 ? S * NB * chunk * 4 : 0);
   return L;
 }
@@ -522,6 +529,7 @@ __device__ __forceinline__ void gd_finish(const GdParams& p, const GdGeom& g, co
   // over the banks.
   const int r1 = lane >> 2, cq = lane & 3;
   const int GS = p.Wn * p.Tw * C::RED + 1;
+  if (p.alias_red) __syncthreads();  // every warp is done reading the activation scratch
   {
     float* wr = red + g.wg * GS + (g.wn * p.Tw * 8 + r1) * NCOL;
 #pragma unroll
@@ -591,7 +599,7 @@ __device__ __forceinline__ void gd_finish(const GdParams& p, const GdGeom& g, co
 template <int NB, int NW>
 __global__ void __launch_bounds__(NW * 32, 1) gemv_direct_kernel(const GdParams p) {
   extern __shared__ __align__(16) unsigned char smem[];
-  const GdSmem L = gd_layout<NB, NW>(p.Tw, p.NSw, p.P, p.S, p.chunk, p.NSc);
+  const GdSmem L = gd_layout<NB, NW>(p.Tw, p.NSw, p.P, p.S, p.chunk, p.NSc, p.alias_red != 0);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   unsigned char* wreg = smem + warp * L.warp_bytes;
   unsigned char* wts = wreg + L.wts;
@@ -659,7 +667,7 @@ static int gd_max_clusters(int S, int smem_bytes) {
 }
 
 struct GdPlan {
-  int S, Q, Wn, Wg, Tw, NSw, NSc, P, chunk, smem;
+  int S, Q, Wn, Wg, Tw, NSw, NSc, P, chunk, smem, alias_red;
   double cost;
 };
 
@@ -695,7 +703,12 @@ static bool gd_plan_for(int N, int NG, int S, int num_sms, int smem_cap, GdPlan*
     const int span = NSw * 16 * C::G;
     const int P = ((span / (16 * C::G)) & 1) ? span : span + 16 * C::G;  // odd multiple: bank spread
     const int chunk = (8 * Tmax + S - 1) / S;
-    const GdSmem L = gd_layout<NB, NW>(Tw, NSw, P, S, chunk, nsc);
+    GdSmem L = gd_layout<NB, NW>(Tw, NSw, P, S, chunk, nsc);
+    int alias_red = 0;
+    if (L.total > smem_cap) {  // first the reduction buffer over the activation scratch
+      L = gd_layout<NB, NW>(Tw, NSw, P, S, chunk, nsc, true);
+      alias_red = 1;
+    }
     if (L.total > smem_cap) {
       if (Q >= NT) return false;
       Q = std::min(NT, Q * 2);  // fewer rows per CTA
@@ -708,7 +721,7 @@ static bool gd_plan_for(int N, int NG, int S, int num_sms, int smem_cap, GdPlan*
     const double wts = 8.0 * Tmax * 128.0 * C::G * nsc * cw;      // per CTA
     const double ctas_per_sm = std::ceil(static_cast<double>(Q) * S / num_sms);
     const double cost = (xprep + wts) / 128.0 * ctas_per_sm + (S > 1 ? 800.0 : 0.0);
-    *out = GdPlan{S, Q, Wn, Wg, Tw, NSw, nsc, P, chunk, L.total, cost};
+    *out = GdPlan{S, Q, Wn, Wg, Tw, NSw, nsc, P, chunk, L.total, alias_red, cost};
     return true;
   }
   return false;
@@ -781,6 +794,7 @@ static cudaError_t launch_gemv_direct_nb(const GdParams& base, cudaStream_t stre
   p.P = plan.P;
   p.chunk = plan.chunk;
   p.NSc = plan.NSc;
+  p.alias_red = plan.alias_red;
   auto lg2 = [](int v) {
     int l = 0;
     while ((1 << l) < v) ++l;

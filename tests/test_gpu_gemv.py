@@ -110,9 +110,12 @@ def test_gemv_is_deterministic():
 
 
 @pytest.mark.parametrize("split", ["1", "2", "4", "8"])
-@pytest.mark.parametrize("N,K,B", [(4096, 4096, 1), (1000, 1152, 5), (4097, 2176, 8), (300, 1024, 2)])
+@pytest.mark.parametrize("N,K,B", [(4096, 4096, 1), (1000, 1152, 5), (4097, 2176, 8), (300, 1024, 2),
+                                   (4096, 11008, 8)])
 def test_gemv_direct_every_split(N, K, B, split, gemv_path, monkeypatch):
-    """The direct kernel's cluster K split (1..8 CTAs) on the same inputs."""
+    """The direct kernel's cluster K split (1..8 CTAs) on the same inputs.
+    4096 x 11008 at B = 8 needs the reduction buffer over the activation
+    scratch at 16 warps and small splits."""
     if not gemv_path.startswith("direct"):
         pytest.skip("split sweep is for the direct kernel")
     monkeypatch.setenv("W1_GEMV_SPLIT", split)
