@@ -68,8 +68,20 @@ def load() -> ctypes.CDLL:
     return lib
 
 
+_fns: dict = {}
+
+
+def fn(name: str):
+    """The ctypes function for `name` (looked up once)."""
+    f = _fns.get(name)
+    if f is None:
+        f = getattr(load(), name)
+        _fns[name] = f
+    return f
+
+
 def call(name: str, *args) -> int:
-    return getattr(load(), name)(*args)
+    return fn(name)(*args)
 
 
 def check(status: int, where: str) -> None:

@@ -17,14 +17,25 @@ from . import _lib
 def _ptr(t: torch.Tensor | None) -> int | None:
     if t is None:
         return None
+    if not t.is_cuda:
+        raise ValueError("tensor must be on a CUDA device")
     if not t.is_contiguous():
         raise ValueError("tensor must be contiguous")
     return t.data_ptr()
 
 
-def _stream(stream=None) -> int:
-    s = stream if stream is not None else torch.cuda.current_stream()
-    return s.cuda_stream
+# The raw handle of a device's current stream without building a Stream
+# object (a few microseconds per call otherwise); the public call is the
+# fallback where this torch build lacks it.
+_raw_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+
+
+def _stream(stream=None, t: torch.Tensor | None = None) -> int:
+    if stream is not None:
+        return stream.cuda_stream
+    if _raw_stream is not None and t is not None and t.is_cuda:
+        return _raw_stream(t.get_device())
+    return torch.cuda.current_stream().cuda_stream
 
 
 def sync_status(stream=None) -> int:
@@ -46,7 +57,7 @@ def w1_pack(W: torch.Tensor, signs: torch.Tensor | None = None, scales: torch.Te
         signs = torch.empty((N, K // 32), dtype=torch.int32, device=W.device)
     if scales is None:
         scales = torch.empty((N, K // 128), dtype=torch.float16, device=W.device)
-    st = _lib.call("w1_pack", _ptr(W), N, K, _ptr(signs), _ptr(scales), _stream(stream))
+    st = _lib.call("w1_pack", _ptr(W), N, K, _ptr(signs), _ptr(scales), _stream(stream, W))
     _lib.check(st, "w1_pack")
     return signs, scales
 
@@ -61,19 +72,16 @@ def w1_gemv(signs: torch.Tensor, scales: torch.Tensor, x: torch.Tensor, y: torch
     static_weights=True calls w1_gemv_ex with W1_GEMV_STATIC_WEIGHTS: the
     weights must not have been written by the kernel just before on the stream.
     """
-    N = signs.shape[0]
-    K = signs.shape[1] * 32
+    N, KW = signs.shape
     B = x.shape[0]
     if x.dtype != torch.bfloat16:
         raise TypeError("x must be bfloat16")
     if y is None:
         y = torch.empty((B, N), dtype=torch.float32, device=x.device)
-    if static_weights:
-        st = _lib.call("w1_gemv_ex", _ptr(signs), _ptr(scales), N, K, _ptr(x), B, _ptr(y),
-                       W1_GEMV_STATIC_WEIGHTS, _stream(stream))
-    else:
-        st = _lib.call("w1_gemv", _ptr(signs), _ptr(scales), N, K, _ptr(x), B, _ptr(y), _stream(stream))
-    _lib.check(st, "w1_gemv")
+    st = _lib.fn("w1_gemv_ex")(_ptr(signs), _ptr(scales), N, KW * 32, _ptr(x), B, _ptr(y),
+                               W1_GEMV_STATIC_WEIGHTS if static_weights else 0, _stream(stream, x))
+    if st != _lib.W1_OK:
+        raise _lib.W1Error(st, "w1_gemv")
     return y
 
 
@@ -123,7 +131,7 @@ def w1_gemm(signs: torch.Tensor, scales: torch.Tensor, x: torch.Tensor, y: torch
     base = _aligned256(workspace)
     avail = workspace.numel() - (base - workspace.data_ptr())
     st = _lib.call("w1_gemm", _ptr(signs), _ptr(scales), N, K, _ptr(x), M, _ptr(y),
-                   ctypes.c_void_p(base), avail, _stream(stream))
+                   ctypes.c_void_p(base), avail, _stream(stream, x))
     _lib.check(st, "w1_gemm")
     return y
 
@@ -150,7 +158,7 @@ def w1_moe_grouped(x: torch.Tensor, logits: torch.Tensor, gate, up, down, top_k:
         out = torch.empty((T, H), dtype=torch.float32, device=x.device)
     st = _lib.call("w1_moe_grouped", _ptr(x), _ptr(logits), T, H, I, E, top_k, _ptr(gate[0]), _ptr(gate[1]),
                    _ptr(up[0]), _ptr(up[1]), _ptr(down[0]), _ptr(down[1]), _ptr(out), _ptr(workspace),
-                   workspace.numel() * workspace.element_size(), _stream(stream))
+                   workspace.numel() * workspace.element_size(), _stream(stream, x))
     _lib.check(st, "w1_moe_grouped")
     return out
 
@@ -199,7 +207,7 @@ def dbf_apply(a: torch.Tensor, B1: torch.Tensor, mid: torch.Tensor, B2: torch.Te
     if y is None:
         y = torch.empty((B, m), dtype=torch.float32, device=x.device)
     st = _lib.call("dbf_apply", _ptr(a), _ptr(B1), _ptr(mid), _ptr(B2), _ptr(b), m, r, n, _ptr(x), B,
-                   _ptr(y), _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
+                   _ptr(y), _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream, x))
     _lib.check(st, "dbf_apply")
     return y
 
@@ -209,6 +217,6 @@ def dbf_apply_noalloc(a: torch.Tensor, B1: torch.Tensor, mid: torch.Tensor, B2: 
     """dbf_apply without a workspace (the library's static scratch); y must be given."""
     m, r, n, B = a.shape[0], mid.shape[0], b.shape[0], x.shape[0]
     st = _lib.call("dbf_apply_noalloc", _ptr(a), _ptr(B1), _ptr(mid), _ptr(B2), _ptr(b), m, r, n, _ptr(x), B,
-                   _ptr(y), _stream(stream))
+                   _ptr(y), _stream(stream, x))
     _lib.check(st, "dbf_apply_noalloc")
     return y
