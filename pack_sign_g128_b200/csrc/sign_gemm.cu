@@ -34,16 +34,20 @@ bool make_tmap_bf16_sw128(CUtensorMap* map, const void* base, int64_t rows, int6
 namespace sg {
 constexpr int BN = 128;   // weight rows per tile (MMA M, TMEM lanes)
 constexpr int BK = 128;   // K per scale group
-constexpr int BKS = 64;   // K per pipeline stage
-constexpr int NS = 4;     // stages
+// K per pipeline stage: one scale group in two 64-wide (128-byte) swizzle
+// atoms, so the MMA issuer's one barrier wait per stage covers 8 MMAs
+constexpr int BKS = 128;
 constexpr int kThreads = 320;  // 10 warps
-constexpr int kAStage = BN * BKS * 2;  // 16 KB
+constexpr int kAAtom = BN * 128;        // bytes of one 64-wide atom of the weight stage (16 KB)
+constexpr int kAStage = 2 * kAAtom;     // 32 KB
 
 // BMT tokens per tile (MMA N): 256 when there are enough tiles to fill the
 // GPU, 128 for few token rows (more tiles, each MMA half as long).
 template <int BMT>
 struct Smem {
-  static constexpr int kXStage = BMT * BKS * 2;
+  static constexpr int NS = BMT == 256 ? 2 : 3;  // stages (192 KB either way)
+  static constexpr int kXAtom = BMT * 128;       // bytes of one 64-wide atom of the token stage
+  static constexpr int kXStage = 2 * kXAtom;
   alignas(1024) unsigned char x[NS][kXStage];
   alignas(1024) unsigned char a[NS][kAStage];
   uint64_t full[NS], empty[NS];
@@ -201,7 +205,7 @@ template <bool PHASE1, int BM>
 __global__ void __launch_bounds__(sg::kThreads, 1)
     sg_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const SgParams p) {
   using namespace sg;
-  constexpr int kXStage = Smem<BM>::kXStage;
+  constexpr int kXStage = Smem<BM>::kXStage, kXAtom = Smem<BM>::kXAtom, NS = Smem<BM>::NS;
   constexpr uint32_t kIdesc = idesc_f16(BN, BM, 0, 0);  // fp16 x fp16 -> fp32
   constexpr uint32_t kTmemCols = 2 * BM;                // two accumulators of BM columns
   extern __shared__ unsigned char smem_raw[];
@@ -231,7 +235,7 @@ __global__ void __launch_bounds__(sg::kThreads, 1)
   const uint32_t tmem = sm.tmem_base;
   pdl_wait();
   const int ntiles = p.MT * p.NT;
-  const int NKS = p.NK * (BK / BKS);  // stages per tile
+  const int NKS = p.NK * (BK / BKS);  // stages per tile (one per scale group)
   const int my_tiles = (ntiles - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) /
                        static_cast<int>(gridDim.x);
 
@@ -245,6 +249,7 @@ __global__ void __launch_bounds__(sg::kThreads, 1)
           if (!mbar_wait(&sm.empty[s], ((c / NS) & 1) ^ 1)) goto done_prod;
           mbar_arrive_expect_tx(&sm.full[s], kXStage);
           tma_load_2d(sm.x[s], &tmap_b, ks * BKS, mt * BM, &sm.full[s]);
+          tma_load_2d(sm.x[s] + kXAtom, &tmap_b, ks * BKS + 64, mt * BM, &sm.full[s]);
         }
       }
     done_prod:;
@@ -264,9 +269,11 @@ __global__ void __launch_bounds__(sg::kThreads, 1)
           const uint32_t xbase = smem_u32(sm.x[s]);
           const uint32_t abase = smem_u32(sm.a[s]);
 #pragma unroll
-          for (int kk = 0; kk < BKS / 16; ++kk)
-            tc_mma_ss(d, smem_desc_sw128(abase + kk * 32), smem_desc_sw128(xbase + kk * 32), kIdesc,
+          for (int kk = 0; kk < BKS / 16; ++kk) {
+            const uint32_t ao = (kk >> 2) * kAAtom + (kk & 3) * 32, xo = (kk >> 2) * kXAtom + (kk & 3) * 32;
+            tc_mma_ss(d, smem_desc_sw128(abase + ao), smem_desc_sw128(xbase + xo), kIdesc,
                       (ks > 0 || kk > 0) ? 1u : 0u);
+          }
           tc_commit(&sm.empty[s]);
         }
         tc_commit(&sm.full_c[cb]);
@@ -274,24 +281,24 @@ __global__ void __launch_bounds__(sg::kThreads, 1)
     done_mma:;
     }
   } else if (warp < 6) {
-    // expanders: thread = weight row.  Per stage: 2 sign words (64 k) + the
-    // group scale -> 32 fp16 pairs +-s (s = the group scale, or 0x3C00 = 1.0;
-    // the sign bit comes straight from the word), stored as eight 16-byte
-    // chunks of the row in the 128B-swizzled K-major layout.  Words and scales
-    // stream through a kPf-deep register ring over this CTA's (tile, stage)
-    // sequence so L2 latency hides behind kPf stages.
-    constexpr int kPf = 8;
+    // expanders: thread = weight row.  Per stage: 4 sign words (one scale
+    // group, 128 k) + the group scale -> 64 fp16 pairs +-s (s = the group
+    // scale, or 0x3C00 = 1.0; the sign bit comes straight from the word),
+    // stored as 16-byte chunks of the row in the two 128B-swizzled K-major
+    // atoms.  Words and scales stream through a kPf-deep register ring over
+    // this CTA's (tile, stage) sequence so L2 latency hides behind kPf stages.
+    constexpr int kPf = 4;
     const int rl = (warp - 2) * 32 + lane;
     const int64_t wrow = p.K >> 5;
     int ld_tile = blockIdx.x, ld_ks = 0;
-    auto fetch = [&](uint2& w, uint32_t& sc) {
-      w = make_uint2(0, 0);
+    auto fetch = [&](uint4& w, uint32_t& sc) {
+      w = make_uint4(0, 0, 0, 0);
       sc = 0x3C00u;
       if (ld_tile < ntiles) {
         const int n = (ld_tile / p.MT) * BN + rl;
-        if (n < p.rows) {
-          w = __ldg(reinterpret_cast<const uint2*>(p.signs + static_cast<int64_t>(n) * wrow) + ld_ks);
-          if (p.gscales) sc = __ldg(p.gscales + static_cast<int64_t>(n) * p.NK + (ld_ks >> 1));
+        if (n < p.rows) {  // a row's words are 16-byte aligned (K % 128 == 0)
+          w = __ldg(reinterpret_cast<const uint4*>(p.signs + static_cast<int64_t>(n) * wrow) + ld_ks);
+          if (p.gscales) sc = __ldg(p.gscales + static_cast<int64_t>(n) * p.NK + ld_ks);
         }
         if (++ld_ks == NKS) {
           ld_ks = 0;
@@ -299,7 +306,7 @@ __global__ void __launch_bounds__(sg::kThreads, 1)
         }
       }
     };
-    uint2 wr[kPf];
+    uint4 wr[kPf];
     uint32_t sr[kPf];
 #pragma unroll
     for (int j = 0; j < kPf; ++j) fetch(wr[j], sr[j]);
@@ -311,15 +318,15 @@ __global__ void __launch_bounds__(sg::kThreads, 1)
 #pragma unroll
       for (int j = 0; j < kPf; ++j) {
         if (c0 + j >= my_stages) break;
-        const uint2 cur = wr[j];
+        const uint4 cur = wr[j];
         const uint32_t ss = sr[j] * 0x00010001u;  // the scale in both fp16 halves
         fetch(wr[j], sr[j]);
         const int s = c % NS;
         if (!mbar_wait_warp(&sm.empty[s], ((c / NS) & 1) ^ 1)) goto done_exp;
         const uint32_t abase = smem_u32(sm.a[s]) + row_off;
-        const uint32_t words[2] = {cur.x, cur.y};
+        const uint32_t words[4] = {cur.x, cur.y, cur.z, cur.w};
 #pragma unroll
-        for (int wi = 0; wi < 2; ++wi) {
+        for (int wi = 0; wi < 4; ++wi) {
           const uint32_t w = words[wi];
           uint32_t rr[16];
 #pragma unroll
@@ -330,10 +337,11 @@ __global__ void __launch_bounds__(sg::kThreads, 1)
             const uint32_t tt = m * (0x40008000u >> b);
             rr[pp] = (tt & 0x80008000u) | ss;
           }
+          const uint32_t ab = abase + static_cast<uint32_t>((wi >> 1) * kAAtom);  // atom wi / 2
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            const uint32_t chunk = static_cast<uint32_t>(wi * 4 + q);
-            st_shared_v4(abase + ((chunk ^ sw) << 4), rr[4 * q], rr[4 * q + 1], rr[4 * q + 2], rr[4 * q + 3]);
+            const uint32_t chunk = static_cast<uint32_t>((wi & 1) * 4 + q);
+            st_shared_v4(ab + ((chunk ^ sw) << 4), rr[4 * q], rr[4 * q + 1], rr[4 * q + 2], rr[4 * q + 3]);
           }
         }
         fence_async_shared();
