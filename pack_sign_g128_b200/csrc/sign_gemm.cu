@@ -119,9 +119,24 @@ __global__ void __launch_bounds__(256) sg_prep_kernel(const uint16_t* __restrict
       l1 += fabsf(v[q]);
     }
   }
+  // max |mid| (the same for every row): 16-byte loads, independent partial
+  // maxima, so the loads are in flight together (r % 8 == 0, 16-byte aligned)
   float mm = 0.f;
-  if (mid)
-    for (int j = threadIdx.x; j < r; j += blockDim.x) mm = fmaxf(mm, fabsf(__half2float(__ushort_as_half(mid[j]))));
+  if (mid) {
+    const uint4* mv = reinterpret_cast<const uint4*>(mid);
+    float m4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+    for (int j = threadIdx.x; j < (r >> 3); j += blockDim.x) {
+      const uint4 u = __ldg(mv + j);
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[q]));
+        m4[q] = fmaxf(m4[q], fmaxf(fabsf(f.x), fabsf(f.y)));
+      }
+    }
+    mm = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+  }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
