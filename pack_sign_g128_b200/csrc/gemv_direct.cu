@@ -14,9 +14,13 @@
 //    previous kernel in the stream (programmatic dependent launch);
 //  * quantises the activations of its K range once per CTA while those copies
 //    are in flight, then lets every warp run alone until the final reduction;
-//  * reduces a K split over a thread-block cluster with one barrier: partial
-//    sums are stored straight into the owning CTA's shared memory (DSMEM), and
-//    only the owner reads them.
+//  * reduces the warps' partial sums with several threads per output (a
+//    fixed-order butterfly), and a K split over a thread-block cluster with
+//    one barrier: partial sums are stored straight into the owning CTA's
+//    shared memory (DSMEM), and only the owner reads them.
+// The kernel runs with 8 warps per CTA (two CTAs fit an SM, so the next
+// launch's CTA can stage its weights early) or 16 (more latency hidden for
+// large K ranges and B >= 4); the dispatcher times both.
 //
 // Arithmetic (exact up to the fp32 fold):
 //  * Activations -> fixed point.  Per (batch row, group) x is scaled by
