@@ -368,6 +368,7 @@ def gemm_rows(torch, ops, synth, peaks, iters: int = 8):
 
 
 MOE = dict(T=512, H=2048, I=1024, E=64, top_k=8)
+MOE_DECODE_T = (1, 4, 8)   # decode-regime batches (per-route products)
 DBF_BATCHES = [1, 8, 512]
 
 
@@ -403,8 +404,39 @@ def moe_rows(torch, ops, synth, peaks, iters: int = 8):
     ms = statistics.median(times)
     flops = 2.0 * T * K * 3 * H * I
     tf = flops / (ms * 1e-3) / 1e12
-    return {"T": T, "H": H, "I": I, "E": E, "top_k": K, "ms": ms, "tokens/s": T / (ms * 1e-3),
-            "TFLOP/s": tf, "frac_bf16_burst": tf / peaks["bf16_tflops"], "launches_per_call": 7}
+    row = {"T": T, "H": H, "I": I, "E": E, "top_k": K, "ms": ms, "tokens/s": T / (ms * 1e-3),
+           "TFLOP/s": tf, "frac_bf16_burst": tf / peaks["bf16_tflops"], "launches_per_call": 7}
+    # decode regime: the first Td tokens of the same batch, a different token
+    # window per call, L2 flushed before each call; HBM-bound on the experts'
+    # packed weights that the call touches
+    per_expert = 3 * packed_bytes(I, H)  # gate, up (I x H) and down (H x I) have the same packed size
+    ids_all = np.argsort(-logits, axis=1, kind="stable")[:, :K]
+    decode = []
+    for Td in MOE_DECODE_T:
+        wsd = ops.moe_workspace(Td, H, I, E, K)
+        outd = torch.empty((Td, H), dtype=torch.float32, device=dev)
+        windows = [(i * Td) % (T - Td + 1) for i in range(iters + 2)]
+        for w0 in windows[:2]:
+            ops.w1_moe_grouped(xd[w0:w0 + Td], ld[w0:w0 + Td], G, U, D, K, out=outd, workspace=wsd)
+        torch.cuda.synchronize()
+        tms, touched = [], []
+        for w0 in windows[2:]:
+            flush.zero_()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record()
+            ops.w1_moe_grouped(xd[w0:w0 + Td], ld[w0:w0 + Td], G, U, D, K, out=outd, workspace=wsd)
+            b.record()
+            torch.cuda.synchronize()
+            tms.append(a.elapsed_time(b))
+            touched.append(len(np.unique(ids_all[w0:w0 + Td])) * per_expert)
+        dms = statistics.median(tms)
+        gbs = float(np.mean(touched)) / (dms * 1e-3) / 1e9
+        decode.append({"T": Td, "us": round(dms * 1e3, 2), "tokens/s": round(Td / (dms * 1e-3), 1),
+                       "weight_GB/s": round(gbs, 1), "frac_hbm": round(gbs / peaks["hbm_gbs"], 4),
+                       "launches_per_call": 4})
+    row["decode"] = decode
+    return row
 
 
 def dbf_rows(torch, ops, synth, peaks, l2_bytes: int, iters: int = 5):

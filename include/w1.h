@@ -188,12 +188,15 @@ size_t w1_gemm_workspace_size(int64_t M, int64_t K);
  *   copies of x rows and h rows in sorted route order with one power-of-two
  *   scale per route.  No state is carried between calls.  Calls sharing a
  *   workspace must not overlap.
- * Seven kernels on `stream`: router, counting sort, gather of x rows into
- * sorted order (fp16, exact per-route power of two), grouped gate/up GEMM
+ * T > 16: seven kernels on `stream`: router, counting sort, gather of x rows
+ * into sorted order (fp16, exact per-token power of two), grouped gate/up GEMM
  * (tcgen05, +-s fp16 weight operand, fused SwiGLU), h to fp16 per route,
  * grouped down GEMM (route weight applied), slot-ordered combine.
+ * T <= 16 (decode regime): four kernels: router, per-route gate/up products
+ * with fused SwiGLU, per-route down products (route weight applied), the
+ * same combine; the products are the batch-1 steps of w1_gemv.
  * Deterministic.  Accuracy per stage as w1_gemm: 1e-3 * sum|s x| for g, u and
- * D_e h.
+ * D_e h.  The workspace must be 1024-byte aligned (W1_ERR_ALIGN otherwise).
  */
 int w1_moe_grouped(const uint16_t* x, const float* router_logits, int64_t T, int64_t H, int64_t I, int64_t E,
                    int64_t top_k, const uint32_t* gate_signs, const uint16_t* gate_scales,

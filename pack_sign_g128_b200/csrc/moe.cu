@@ -10,6 +10,11 @@
 // expert-major compaction of route-specific inputs, shared gate/up inputs
 // kept un-duplicated, fused SwiGLU, skipped empty tiles.
 //
+// Up to 16 tokens (the decode regime) the layer runs as per-route products:
+// router, a fused gate/up + SwiGLU kernel, a down kernel, the combine (four
+// launches; see "decode regime" below).  Larger batches take the
+// expert-sorted tile pipeline.
+//
 // Seven launches on one stream (programmatic dependent launch between them):
 //  1. route_kernel     warp per token: fp32 softmax, top-k by logit, weights,
 //                      and the token's fp16 multiplier (a power of two).
@@ -768,6 +773,130 @@ __global__ void __launch_bounds__(256) moe_hprep_kernel(const uint16_t* __restri
   pdl_launch_dependents();
 }
 
+// ------------------------------------------------------------------ decode regime (T <= 8)
+
+// With a handful of tokens every expert sees about one route, so the tile
+// pipeline's 128-route MMA tiles would be almost empty.  Instead each route is
+// a batch-1 product on the direct GEMV steps (gemv_direct.cu): exact
+// fixed-point activation digits, int8 mma.sync on the sign bytes, one fold
+// per group.  A CTA takes one route and a block of output rows; each of its 8
+// warps owns 16 rows (two 8-row n-tiles) over all of K, so no cross-warp
+// reduction is needed.  Gate/up: warps 0-3 take 16 rows each of G_e, warps
+// 4-7 the same rows of U_e, and h = bf16(silu(g) u) is formed through shared
+// memory.  Down: 8 x 16 rows of D_e per CTA, times the route weight.
+namespace moed {
+constexpr int kWarps = 8;
+constexpr int kTw = 2;                   // 8-row n-tiles per warp
+constexpr int kRowsGu = 4 * 8 * kTw;     // gate/up rows per CTA (of each matrix)
+constexpr int kRowsD = kWarps * 8 * kTw; // down rows per CTA
+}  // namespace moed
+
+struct MoeDecParams {
+  const int* ids;            // [R] expert per route
+  const float* wts;          // [R] route weight
+  const uint16_t* x;         // gate/up: tokens [T][H] bf16; down: h [R][I] bf16
+  const uint32_t* signs0;    // gate/up: G, down: D   [E][rows][K/32]
+  const uint16_t* scales0;
+  const uint32_t* signs1;    // gate/up: U
+  const uint16_t* scales1;
+  __nv_bfloat16* h;          // gate/up output [R][I]
+  float* rout;               // down output [R][H]
+  int* pos;                  // gate/up: route -> its row of h / rout (identity here)
+  int R, top_k, rows, K, NG, P, lgGw;
+};
+
+__host__ __device__ inline GdSmem moed_layout(const MoeDecParams& q) {
+  return gd_layout<1, moed::kWarps>(moed::kTw, q.NG, q.P, 1, 0, q.NG);
+}
+
+template <bool GATEUP>
+__global__ void __launch_bounds__(moed::kWarps * 32, 1) moe_decode_kernel(const MoeDecParams q) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  __shared__ float gu[2][moed::kRowsGu];
+  const GdSmem L = moed_layout(q);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r = blockIdx.y;
+  pdl_wait();
+  pdl_launch_dependents();
+  const int e = q.ids[r];
+  // this warp's matrix and rows
+  const int mat = GATEUP ? (warp >> 2) : 0;
+  const int row0 = GATEUP ? blockIdx.x * moed::kRowsGu + (warp & 3) * 8 * moed::kTw
+                          : blockIdx.x * moed::kRowsD + warp * 8 * moed::kTw;
+  GdParams p = {};
+  const int64_t mrow = static_cast<int64_t>(e) * q.rows;  // the expert's first row
+  p.signs = (mat ? q.signs1 : q.signs0) + mrow * (q.K >> 5);
+  p.scales = (mat ? q.scales1 : q.scales0) + mrow * q.NG;
+  p.x = GATEUP ? static_cast<const void*>(q.x + static_cast<int64_t>(r / q.top_k) * q.K)
+               : static_cast<const void*>(q.x + static_cast<int64_t>(r) * q.K);
+  p.N = q.rows;
+  p.K = q.K;
+  p.NG = q.NG;
+  p.Tw = moed::kTw;
+  p.NSw = q.NG;
+  p.P = q.P;
+  p.lgGw = q.lgGw;
+  GdGeom g = {};
+  g.nsc = q.NG;
+  g.tw = moed::kTw;
+  g.nsw = q.NG;
+  g.row0 = row0;
+  g.nrows = max(0, min(8 * moed::kTw, q.rows - row0));
+  g.busy = g.nrows > 0;
+  g.ngw = q.NG;
+  unsigned char* wreg = smem + warp * L.warp_bytes;
+  unsigned char* wts = wreg + L.wts;
+  float* scl = reinterpret_cast<float*>(wreg + L.scl);
+  uint32_t* xs = reinterpret_cast<uint32_t*>(smem + L.xs);
+  uint16_t sreg[kGdSpl];
+  if (g.busy) gd_stage<1>(p, g, wts, lane);
+  else cp_async_commit();
+  gd_load_scales<1>(p, g, 0, lane, sreg);
+  uint4 xa[4];
+  gd_x_first<1, false>(p, g, warp, lane, xa);
+  gd_prep_x<1, false, moed::kWarps>(p, g, xs, warp, lane, xa);
+  gd_finish_scales<1>(p, g, lane, sreg, scl);
+  cp_async_wait_all();
+  __syncthreads();
+  float acc[gd::kMaxTp][gd::Cfg<1>::NN][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) acc[0][0][i] = acc[1][0][i] = 0.f;
+  if (g.busy) gd_compute<1, moed::kTw>(wts, p.P, scl, 8 * moed::kTw, xs, q.NG, lane, acc);
+  // digit columns -> row sums: a lane holds columns 2(lane&3), +1 of rows
+  // lane/4 (n-tile 0) and lane/4 + 8 (n-tile 1); columns past the three
+  // digits are zero, so the quad sum is the row's value
+  float v0 = acc[0][0][0] + acc[0][0][1], v1 = acc[0][0][2] + acc[0][0][3];
+#pragma unroll
+  for (int o = 1; o < 4; o <<= 1) {
+    v0 += __shfl_xor_sync(0xFFFFFFFFu, v0, o);
+    v1 += __shfl_xor_sync(0xFFFFFFFFu, v1, o);
+  }
+  const int rl = lane >> 2;
+  if (GATEUP) {
+    if ((lane & 3) == 0) {
+      const int base = (warp & 3) * 8 * moed::kTw;
+      gu[mat][base + rl] = v0;
+      gu[mat][base + 8 + rl] = v1;
+    }
+    __syncthreads();
+    if (blockIdx.x == 0 && threadIdx.x == 0) q.pos[r] = r;
+    for (int i = threadIdx.x; i < moed::kRowsGu; i += blockDim.x) {
+      const int row = blockIdx.x * moed::kRowsGu + i;
+      if (row < q.rows) {
+        const float gv = gu[0][i], uv = gu[1][i];
+        q.h[static_cast<int64_t>(r) * q.rows + row] = __float2bfloat16_rn(gv / (1.0f + expf(-gv)) * uv);
+      }
+    }
+  } else {
+    if ((lane & 3) == 0) {
+      const float wt = q.wts[r];
+      float* op = q.rout + static_cast<int64_t>(r) * q.rows;
+      if (row0 + rl < q.rows) op[row0 + rl] = wt * v0;
+      if (row0 + 8 + rl < q.rows) op[row0 + 8 + rl] = wt * v1;
+    }
+  }
+}
+
 // ------------------------------------------------------------------ 5. combine
 
 __global__ void __launch_bounds__(256) moe_combine_kernel(const float* __restrict__ rout, const int* __restrict__ pos,
@@ -813,6 +942,23 @@ static cudaError_t launch_pdl(Kern kernel, dim3 grid, dim3 block, size_t smem, c
   return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
+template <bool GATEUP>
+static cudaError_t launch_moe_decode(MoeDecParams q, cudaStream_t stream) {
+  auto lg2 = [](int v) {
+    int l = 0;
+    while ((1 << l) < v) ++l;
+    return l;
+  };
+  q.P = ((q.NG & 1) ? q.NG : q.NG + 1) * 16;  // odd multiple of 16 bytes per staged row: bank spread
+  q.lgGw = lg2(q.NG);
+  const int smem = moed_layout(q).total;
+  cudaError_t err = ensure_dyn_smem(reinterpret_cast<const void*>(moe_decode_kernel<GATEUP>), smem);
+  if (err != cudaSuccess) return err;
+  const int per = GATEUP ? moed::kRowsGu : moed::kRowsD;
+  const dim3 grid(static_cast<unsigned>((q.rows + per - 1) / per), static_cast<unsigned>(q.R));
+  return launch_pdl(moe_decode_kernel<GATEUP>, grid, dim3(moed::kWarps * 32), static_cast<size_t>(smem), stream, q);
+}
+
 cudaError_t launch_moe(const uint16_t* x, const float* logits, int64_t T, int64_t H, int64_t I, int E, int top_k,
                        const uint32_t* gs, const uint16_t* gc, const uint32_t* us, const uint16_t* uc,
                        const uint32_t* ds, const uint16_t* dc, float* out, void* workspace, cudaStream_t stream,
@@ -838,6 +984,51 @@ cudaError_t launch_moe(const uint16_t* x, const float* logits, int64_t T, int64_
   err = launch_pdl(moe_route_kernel, dim3(static_cast<unsigned>((T + 7) / 8)), dim3(256), 0, stream, logits,
                    static_cast<int>(T), E, top_k, ids, wts, x, static_cast<int>(H), xcs);
   if (err != cudaSuccess) return err;
+  // Decode regime: a few tokens, about one route per expert -> per-route
+  // products on the direct GEMV steps.  Measured on the OLMoE-like layer: 2x
+  // faster than the tile pipeline up to 8 tokens, still ahead at 16.
+  // W1_MOE_PATH=tiles|decode forces a path (testing knob).
+  constexpr int64_t kDecodeMaxT = 16;
+  const char* mpath = getenv("W1_MOE_PATH");
+  const bool decode =
+      (mpath ? mpath[0] == 'd' : T <= kDecodeMaxT) && H / 128 <= gd::kMaxSets && I / 128 <= gd::kMaxSets;
+  if (decode) {
+    MoeDecParams q = {};
+    q.ids = ids;
+    q.wts = wts;
+    q.x = x;
+    q.signs0 = gs;
+    q.scales0 = gc;
+    q.signs1 = us;
+    q.scales1 = uc;
+    q.h = h;
+    q.pos = pos;
+    q.R = R;
+    q.top_k = top_k;
+    q.rows = static_cast<int>(I);
+    q.K = static_cast<int>(H);
+    q.NG = static_cast<int>(H / 128);
+    err = launch_moe_decode<true>(q, stream);
+    if (err != cudaSuccess) return err;
+    MoeDecParams qd = q;
+    qd.x = reinterpret_cast<const uint16_t*>(h);
+    qd.signs0 = ds;
+    qd.scales0 = dc;
+    qd.signs1 = nullptr;
+    qd.scales1 = nullptr;
+    qd.rout = rout;
+    qd.rows = static_cast<int>(H);
+    qd.K = static_cast<int>(I);
+    qd.NG = static_cast<int>(I / 128);
+    err = launch_moe_decode<false>(qd, stream);
+    if (err != cudaSuccess) return err;
+    const int64_t total4 = T * (H / 4);
+    int64_t blocks = (total4 + 255) / 256;
+    if (blocks > 8 * num_sms) blocks = 8 * num_sms;
+    return launch_pdl(moe_combine_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, stream,
+                      static_cast<const float*>(rout), static_cast<const int*>(pos), static_cast<int>(T),
+                      static_cast<int>(H), top_k, out);
+  }
   // 2. sort + tile lists
   constexpr int kStageMax = 16384;  // routes staged in shared memory (64 KB)
   SortArgs sa{ids,  R,   E,       top_k,    static_cast<int>(I / 128), static_cast<int>(H / 128), offsets, sroute,

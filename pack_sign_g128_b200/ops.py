@@ -136,11 +136,20 @@ def w1_gemm(signs: torch.Tensor, scales: torch.Tensor, x: torch.Tensor, y: torch
     return y
 
 
+_MOE_WS_ALIGN = 1024  # w1_moe_grouped's workspace alignment
+
+
 def moe_workspace(T: int, H: int, I: int, E: int, top_k: int, device=None) -> torch.Tensor:
+    """Workspace for w1_moe_grouped (with slack: the call uses its 1024-byte aligned part)."""
     nbytes = _lib.call("w1_moe_workspace_size", T, H, I, E, top_k)
     if nbytes == 0:
         raise ValueError("invalid MoE sizes")
-    return torch.empty(nbytes, dtype=torch.uint8, device=device or "cuda")
+    return torch.empty(nbytes + _MOE_WS_ALIGN, dtype=torch.uint8, device=device or "cuda")
+
+
+def _moe_ws_offset(workspace: torch.Tensor) -> int:
+    p = workspace.data_ptr()
+    return (p + _MOE_WS_ALIGN - 1) // _MOE_WS_ALIGN * _MOE_WS_ALIGN - p
 
 
 def w1_moe_grouped(x: torch.Tensor, logits: torch.Tensor, gate, up, down, top_k: int,
@@ -156,9 +165,11 @@ def w1_moe_grouped(x: torch.Tensor, logits: torch.Tensor, gate, up, down, top_k:
         workspace = moe_workspace(T, H, I, E, top_k, x.device)
     if out is None:
         out = torch.empty((T, H), dtype=torch.float32, device=x.device)
+    off = _moe_ws_offset(workspace)
     st = _lib.call("w1_moe_grouped", _ptr(x), _ptr(logits), T, H, I, E, top_k, _ptr(gate[0]), _ptr(gate[1]),
-                   _ptr(up[0]), _ptr(up[1]), _ptr(down[0]), _ptr(down[1]), _ptr(out), _ptr(workspace),
-                   workspace.numel() * workspace.element_size(), _stream(stream, x))
+                   _ptr(up[0]), _ptr(up[1]), _ptr(down[0]), _ptr(down[1]), _ptr(out),
+                   ctypes.c_void_p(_ptr(workspace) + off),
+                   workspace.numel() * workspace.element_size() - off, _stream(stream, x))
     _lib.check(st, "w1_moe_grouped")
     return out
 
@@ -166,6 +177,7 @@ def w1_moe_grouped(x: torch.Tensor, logits: torch.Tensor, gate, up, down, top_k:
 def moe_workspace_views(workspace: torch.Tensor, T: int, H: int, I: int, E: int, top_k: int) -> dict:
     """Typed views of the MoE workspace (routing, sorted order, h) for inspection."""
     R = T * top_k
+    workspace = workspace[_moe_ws_offset(workspace):]  # the part the call used
 
     def up(v, a):
         return (v + a - 1) // a * a

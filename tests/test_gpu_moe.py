@@ -1,5 +1,7 @@
 """w1_moe_grouped on the GPU vs the fp64 oracle: routing exact, every stage
-within its bound, end to end with the bf16 intermediate propagated."""
+within its bound, end to end with the bf16 intermediate propagated.  Batches
+of up to 8 tokens take the decode path (per-route products), larger ones the
+expert-sorted tile pipeline; W1_MOE_PATH forces either."""
 import functools
 
 import numpy as np
@@ -84,7 +86,9 @@ def test_moe_config_olmoe_like():
 
 @pytest.mark.parametrize("T,H,I,E,K,seed,skew", [
     (16, 256, 128, 8, 2, 1, 0.0),      # tiny, ragged tiles
-    (1, 2048, 1024, 64, 8, 2, 0.0),    # one token (decode-like)
+    (1, 2048, 1024, 64, 8, 2, 0.0),    # one token: decode regime (per-route products)
+    (4, 2048, 1024, 64, 8, 5, 0.0),    # decode regime
+    (8, 512, 384, 16, 4, 6, 0.0),      # decode regime, experts shared by tokens
     (300, 384, 256, 16, 4, 3, 6.0),    # skewed routing: empty experts, multi-tile experts
     (130, 512, 384, 32, 8, 4, 0.0),
 ])
@@ -92,8 +96,17 @@ def test_moe_small_and_skewed(T, H, I, E, K, seed, skew):
     run_and_check(T, H, I, E, K, seed, skew)
 
 
-def test_moe_is_deterministic():
-    T, H, I, E, K = 64, 512, 256, 16, 4
+@pytest.mark.parametrize("path,T", [("tiles", 3), ("decode", 20)])
+def test_moe_forced_path(path, T, monkeypatch):
+    """Each path outside its default regime: the tile pipeline for a few
+    tokens, the per-route decode products for a larger batch."""
+    monkeypatch.setenv("W1_MOE_PATH", path)
+    run_and_check(T, 512, 256, 16, 4, 7)
+
+
+@pytest.mark.parametrize("T", [64, 4])
+def test_moe_is_deterministic(T):
+    H, I, E, K = 512, 256, 16, 4
     x, logits, G, U, D = moe_case(T, H, I, E, 7)
     dev = lambda p: (words_dev(p[0].reshape(-1, p[0].shape[-1])).view(p[0].shape[0], p[0].shape[1], -1),
                      fp16_dev(p[1].reshape(-1, p[1].shape[-1])).view(p[1].shape[0], p[1].shape[1], -1))
