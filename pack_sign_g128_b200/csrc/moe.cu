@@ -11,9 +11,9 @@
 // kept un-duplicated, fused SwiGLU, skipped empty tiles.
 //
 // Up to 16 tokens (the decode regime) the layer runs as per-route products:
-// router, a fused gate/up + SwiGLU kernel, a down kernel, the combine (four
-// launches; see "decode regime" below).  Larger batches take the
-// expert-sorted tile pipeline.
+// router, a fused gate/up + SwiGLU kernel, and a down kernel that also does
+// the slot-ordered combine (three launches; see "decode regime" below).
+// Larger batches take the expert-sorted tile pipeline.
 //
 // Seven launches on one stream (programmatic dependent launch between them):
 //  1. route_kernel     warp per token: fp32 softmax, top-k by logit, weights,
@@ -779,16 +779,15 @@ __global__ void __launch_bounds__(256) moe_hprep_kernel(const uint16_t* __restri
 // pipeline's 128-route MMA tiles would be almost empty.  Instead each route is
 // a batch-1 product on the direct GEMV steps (gemv_direct.cu): exact
 // fixed-point activation digits, int8 mma.sync on the sign bytes, one fold
-// per group.  A CTA takes one route and a block of output rows; each of its 8
-// warps owns 16 rows (two 8-row n-tiles) over all of K, so no cross-warp
-// reduction is needed.  Gate/up: warps 0-3 take 16 rows each of G_e, warps
-// 4-7 the same rows of U_e, and h = bf16(silu(g) u) is formed through shared
-// memory.  Down: 8 x 16 rows of D_e per CTA, times the route weight.
+// per group.  Gate/up: a CTA takes one route and 64 output rows; warps 0-3
+// own 16 rows each of G_e and warps 4-7 the same rows of U_e, each over all of
+// K (no cross-warp reduction), and h = bf16(silu(g) u) is formed through
+// shared memory.  Down + combine: moe_decode_down_kernel below.
 namespace moed {
 constexpr int kWarps = 8;
 constexpr int kTw = 2;                   // 8-row n-tiles per warp
 constexpr int kRowsGu = 4 * 8 * kTw;     // gate/up rows per CTA (of each matrix)
-constexpr int kRowsD = kWarps * 8 * kTw; // down rows per CTA
+constexpr int kSmemCap = 220 * 1024;     // dynamic shared memory the decode kernels may use
 }  // namespace moed
 
 struct MoeDecParams {
@@ -800,8 +799,7 @@ struct MoeDecParams {
   const uint32_t* signs1;    // gate/up: U
   const uint16_t* scales1;
   __nv_bfloat16* h;          // gate/up output [R][I]
-  float* rout;               // down output [R][H]
-  int* pos;                  // gate/up: route -> its row of h / rout (identity here)
+  int* pos;                  // gate/up: route -> its row of h (identity here)
   int R, top_k, rows, K, NG, P, lgGw;
 };
 
@@ -809,8 +807,7 @@ __host__ __device__ inline GdSmem moed_layout(const MoeDecParams& q) {
   return gd_layout<1, moed::kWarps>(moed::kTw, q.NG, q.P, 1, 0, q.NG);
 }
 
-template <bool GATEUP>
-__global__ void __launch_bounds__(moed::kWarps * 32, 1) moe_decode_kernel(const MoeDecParams q) {
+__global__ void __launch_bounds__(moed::kWarps * 32, 1) moe_decode_gateup_kernel(const MoeDecParams q) {
   extern __shared__ __align__(16) unsigned char smem[];
   __shared__ float gu[2][moed::kRowsGu];
   const GdSmem L = moed_layout(q);
@@ -819,16 +816,14 @@ __global__ void __launch_bounds__(moed::kWarps * 32, 1) moe_decode_kernel(const 
   pdl_wait();
   pdl_launch_dependents();
   const int e = q.ids[r];
-  // this warp's matrix and rows
-  const int mat = GATEUP ? (warp >> 2) : 0;
-  const int row0 = GATEUP ? blockIdx.x * moed::kRowsGu + (warp & 3) * 8 * moed::kTw
-                          : blockIdx.x * moed::kRowsD + warp * 8 * moed::kTw;
+  // this warp's matrix (0: G, 1: U) and rows
+  const int mat = warp >> 2;
+  const int row0 = blockIdx.x * moed::kRowsGu + (warp & 3) * 8 * moed::kTw;
   GdParams p = {};
   const int64_t mrow = static_cast<int64_t>(e) * q.rows;  // the expert's first row
   p.signs = (mat ? q.signs1 : q.signs0) + mrow * (q.K >> 5);
   p.scales = (mat ? q.scales1 : q.scales0) + mrow * q.NG;
-  p.x = GATEUP ? static_cast<const void*>(q.x + static_cast<int64_t>(r / q.top_k) * q.K)
-               : static_cast<const void*>(q.x + static_cast<int64_t>(r) * q.K);
+  p.x = q.x + static_cast<int64_t>(r / q.top_k) * q.K;
   p.N = q.rows;
   p.K = q.K;
   p.NG = q.NG;
@@ -872,27 +867,18 @@ __global__ void __launch_bounds__(moed::kWarps * 32, 1) moe_decode_kernel(const 
     v1 += __shfl_xor_sync(0xFFFFFFFFu, v1, o);
   }
   const int rl = lane >> 2;
-  if (GATEUP) {
-    if ((lane & 3) == 0) {
-      const int base = (warp & 3) * 8 * moed::kTw;
-      gu[mat][base + rl] = v0;
-      gu[mat][base + 8 + rl] = v1;
-    }
-    __syncthreads();
-    if (blockIdx.x == 0 && threadIdx.x == 0) q.pos[r] = r;
-    for (int i = threadIdx.x; i < moed::kRowsGu; i += blockDim.x) {
-      const int row = blockIdx.x * moed::kRowsGu + i;
-      if (row < q.rows) {
-        const float gv = gu[0][i], uv = gu[1][i];
-        q.h[static_cast<int64_t>(r) * q.rows + row] = __float2bfloat16_rn(gv / (1.0f + expf(-gv)) * uv);
-      }
-    }
-  } else {
-    if ((lane & 3) == 0) {
-      const float wt = q.wts[r];
-      float* op = q.rout + static_cast<int64_t>(r) * q.rows;
-      if (row0 + rl < q.rows) op[row0 + rl] = wt * v0;
-      if (row0 + 8 + rl < q.rows) op[row0 + 8 + rl] = wt * v1;
+  if ((lane & 3) == 0) {
+    const int base = (warp & 3) * 8 * moed::kTw;
+    gu[mat][base + rl] = v0;
+    gu[mat][base + 8 + rl] = v1;
+  }
+  __syncthreads();
+  if (blockIdx.x == 0 && threadIdx.x == 0) q.pos[r] = r;
+  for (int i = threadIdx.x; i < moed::kRowsGu; i += blockDim.x) {
+    const int row = blockIdx.x * moed::kRowsGu + i;
+    if (row < q.rows) {
+      const float gv = gu[0][i], uv = gu[1][i];
+      q.h[static_cast<int64_t>(r) * q.rows + row] = __float2bfloat16_rn(gv / (1.0f + expf(-gv)) * uv);
     }
   }
 }
@@ -942,8 +928,150 @@ static cudaError_t launch_pdl(Kern kernel, dim3 grid, dim3 block, size_t smem, c
   return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
-template <bool GATEUP>
-static cudaError_t launch_moe_decode(MoeDecParams q, cudaStream_t stream) {
+// Down products and the slot-ordered combine of the decode regime, fused:
+// one CTA per (token, RB output rows), RB = 16 x tokens (at most 128), so a
+// route's h is quantised by as many CTAs as there are row blocks, whatever
+// the batch.  Warp w takes slots w, w + 8, ...: it quantises that route's h
+// into its own digit scratch, stages RB rows of D_e at once and forms their
+// products 32 rows at a time (the direct GEMV steps at batch 1).  The slots'
+// partial sums (times the route weight) meet in shared memory, and RB
+// threads add them in slot order (deterministic) straight into out.
+struct MoeDownLayout {
+  int RB, P, wts, scl, xs, warp_bytes, part, total;
+};
+__host__ __device__ inline MoeDownLayout moe_down_layout(int NG, int RB) {
+  MoeDownLayout L;
+  L.RB = RB;
+  L.P = ((NG & 1) ? NG : NG + 1) * 16;  // odd multiple of 16 bytes per staged row: bank spread
+  L.wts = 0;
+  L.scl = (L.wts + RB * L.P + 15) / 16 * 16;
+  L.xs = (L.scl + NG * RB * 4 + 15) / 16 * 16;
+  L.warp_bytes = (L.xs + NG * gd::Cfg<1>::SCR * 4 + 15) / 16 * 16;
+  L.part = moed::kWarps * L.warp_bytes;
+  L.total = L.part + moe::kMaxTopK * RB * 4;
+  return L;
+}
+
+__global__ void __launch_bounds__(moed::kWarps * 32, 1) moe_decode_down_kernel(const MoeDecParams q, int RB,
+                                                                             float* __restrict__ out) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  const MoeDownLayout L = moe_down_layout(q.NG, RB);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.y, row0 = blockIdx.x * RB;
+  unsigned char* wreg = smem + warp * L.warp_bytes;
+  unsigned char* wts = wreg + L.wts;
+  float* scl = reinterpret_cast<float*>(wreg + L.scl);  // [group][RB rows]
+  uint32_t* xs = reinterpret_cast<uint32_t*>(wreg + L.xs);
+  float* part = reinterpret_cast<float*>(smem + L.part);  // [slot][RB rows]
+  pdl_wait();
+  pdl_launch_dependents();
+  for (int s = warp; s < q.top_k; s += moed::kWarps) {  // warp-uniform
+    const int r = t * q.top_k + s;
+    const int e = q.ids[r];
+    GdParams p = {};
+    const int64_t mrow = static_cast<int64_t>(e) * q.rows;
+    p.signs = q.signs0 + mrow * (q.K >> 5);
+    p.scales = q.scales0 + mrow * q.NG;
+    p.N = q.rows;
+    p.K = q.K;
+    p.NG = q.NG;
+    p.Tw = RB / 8;  // scale rows stride RB
+    p.NSw = q.NG;
+    p.P = L.P;
+    p.lgGw = q.lgGw;
+    GdGeom g = {};
+    g.nsc = q.NG;
+    g.tw = RB / 8;
+    g.nsw = q.NG;
+    g.row0 = row0;
+    g.nrows = max(0, min(RB, q.rows - row0));
+    g.busy = g.nrows > 0;
+    g.ngw = q.NG;
+    uint16_t sreg[kGdSpl];
+    if (g.busy) gd_stage<1>(p, g, wts, lane);
+    gd_load_scales<1>(p, g, 0, lane, sreg);
+    // this route's h -> digit scratch: a unit is one group (8 lanes x 16
+    // values), four units per pass of the warp
+    const uint16_t* hr = q.x + static_cast<int64_t>(r) * q.K;
+    for (int g0 = 0; g0 < q.NG; g0 += 4) {
+      const int gi = g0 + (lane >> 3), sub = lane & 7;
+      float v[16];
+      uint4 u0 = make_uint4(0, 0, 0, 0), u1 = u0;
+      if (gi < q.NG) {
+        const uint4* src = reinterpret_cast<const uint4*>(hr + gi * 128 + sub * 16);
+        u0 = src[0];
+        u1 = src[1];
+      }
+      const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        v[2 * i] = __uint_as_float(w[i] << 16);
+        v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+      }
+      quantise_item<1>(v, gi < q.NG, sub, xs + (gi < q.NG ? gi : 0) * gd::Cfg<1>::SCR);
+    }
+    gd_finish_scales<1>(p, g, lane, sreg, scl);
+    cp_async_wait_all();
+    __syncwarp();
+    const float wt = q.wts[r];
+    for (int c0 = 0; c0 < RB; c0 += 32) {  // 32 rows (4 n-tiles) or the last 16
+      float acc[gd::kMaxTp][gd::Cfg<1>::NN][4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[0][0][i] = acc[1][0][i] = 0.f;
+      const unsigned char* wc = wts + c0 * L.P;
+      const float* sc = scl + c0;
+      if (g.busy) {
+        if (RB - c0 >= 32) gd_compute<1, 4>(wc, L.P, sc, RB, xs, q.NG, lane, acc);
+        else gd_compute<1, 2>(wc, L.P, sc, RB, xs, q.NG, lane, acc);
+      }
+      // quad sums: rows lane/4 + {0, 8} (pair 0) and + {16, 24} (pair 1)
+      float v[4] = {acc[0][0][0] + acc[0][0][1], acc[0][0][2] + acc[0][0][3], acc[1][0][0] + acc[1][0][1],
+                    acc[1][0][2] + acc[1][0][3]};
+#pragma unroll
+      for (int o = 1; o < 4; o <<= 1)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) v[i] += __shfl_xor_sync(0xFFFFFFFFu, v[i], o);
+      if ((lane & 3) == 0) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int rr = c0 + 8 * i + (lane >> 2);
+          if (rr < RB) part[s * RB + rr] = wt * v[i];
+        }
+      }
+    }
+    __syncwarp();  // this warp's buffers are reused by its next slot
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < RB; i += blockDim.x) {
+    if (row0 + i < q.rows) {
+      float sum = 0.f;
+      for (int s = 0; s < q.top_k; ++s) sum += part[s * RB + i];
+      out[static_cast<int64_t>(t) * q.rows + row0 + i] = sum;
+    }
+  }
+}
+
+static cudaError_t launch_moe_decode_down(MoeDecParams q, int T, float* out, cudaStream_t stream) {
+  auto lg2 = [](int v) {
+    int l = 0;
+    while ((1 << l) < v) ++l;
+    return l;
+  };
+  q.lgGw = lg2(q.NG);
+  // rows per CTA: 16 x (tokens rounded down to a power of two, at most 8),
+  // halved while the shared memory would not fit
+  int RB = 16;
+  while (RB < 128 && 2 * RB <= 16 * T) RB *= 2;
+  while (RB > 16 && moe_down_layout(q.NG, RB).total > moed::kSmemCap) RB /= 2;
+  const int smem = moe_down_layout(q.NG, RB).total;
+  cudaError_t err = ensure_dyn_smem(reinterpret_cast<const void*>(moe_decode_down_kernel), smem);
+  if (err != cudaSuccess) return err;
+  const dim3 grid(static_cast<unsigned>((q.rows + RB - 1) / RB), static_cast<unsigned>(T));
+  return launch_pdl(moe_decode_down_kernel, grid, dim3(moed::kWarps * 32), static_cast<size_t>(smem), stream, q,
+                    RB, out);
+}
+
+static cudaError_t launch_moe_decode_gateup(MoeDecParams q, cudaStream_t stream) {
   auto lg2 = [](int v) {
     int l = 0;
     while ((1 << l) < v) ++l;
@@ -952,11 +1080,10 @@ static cudaError_t launch_moe_decode(MoeDecParams q, cudaStream_t stream) {
   q.P = ((q.NG & 1) ? q.NG : q.NG + 1) * 16;  // odd multiple of 16 bytes per staged row: bank spread
   q.lgGw = lg2(q.NG);
   const int smem = moed_layout(q).total;
-  cudaError_t err = ensure_dyn_smem(reinterpret_cast<const void*>(moe_decode_kernel<GATEUP>), smem);
+  cudaError_t err = ensure_dyn_smem(reinterpret_cast<const void*>(moe_decode_gateup_kernel), smem);
   if (err != cudaSuccess) return err;
-  const int per = GATEUP ? moed::kRowsGu : moed::kRowsD;
-  const dim3 grid(static_cast<unsigned>((q.rows + per - 1) / per), static_cast<unsigned>(q.R));
-  return launch_pdl(moe_decode_kernel<GATEUP>, grid, dim3(moed::kWarps * 32), static_cast<size_t>(smem), stream, q);
+  const dim3 grid(static_cast<unsigned>((q.rows + moed::kRowsGu - 1) / moed::kRowsGu), static_cast<unsigned>(q.R));
+  return launch_pdl(moe_decode_gateup_kernel, grid, dim3(moed::kWarps * 32), static_cast<size_t>(smem), stream, q);
 }
 
 cudaError_t launch_moe(const uint16_t* x, const float* logits, int64_t T, int64_t H, int64_t I, int E, int top_k,
@@ -990,8 +1117,14 @@ cudaError_t launch_moe(const uint16_t* x, const float* logits, int64_t T, int64_
   // W1_MOE_PATH=tiles|decode forces a path (testing knob).
   constexpr int64_t kDecodeMaxT = 16;
   const char* mpath = getenv("W1_MOE_PATH");
-  const bool decode =
-      (mpath ? mpath[0] == 'd' : T <= kDecodeMaxT) && H / 128 <= gd::kMaxSets && I / 128 <= gd::kMaxSets;
+  bool decode = (mpath ? mpath[0] == 'd' : T <= kDecodeMaxT) && H / 128 <= gd::kMaxSets && I / 128 <= gd::kMaxSets;
+  if (decode) {  // both decode kernels' shared memory must fit
+    MoeDecParams qg = {};
+    qg.NG = static_cast<int>(H / 128);
+    qg.P = ((qg.NG & 1) ? qg.NG : qg.NG + 1) * 16;
+    decode = moed_layout(qg).total <= moed::kSmemCap &&
+             moe_down_layout(static_cast<int>(I / 128), 16).total <= moed::kSmemCap;
+  }
   if (decode) {
     MoeDecParams q = {};
     q.ids = ids;
@@ -1008,7 +1141,7 @@ cudaError_t launch_moe(const uint16_t* x, const float* logits, int64_t T, int64_
     q.rows = static_cast<int>(I);
     q.K = static_cast<int>(H);
     q.NG = static_cast<int>(H / 128);
-    err = launch_moe_decode<true>(q, stream);
+    err = launch_moe_decode_gateup(q, stream);
     if (err != cudaSuccess) return err;
     MoeDecParams qd = q;
     qd.x = reinterpret_cast<const uint16_t*>(h);
@@ -1016,18 +1149,10 @@ cudaError_t launch_moe(const uint16_t* x, const float* logits, int64_t T, int64_
     qd.scales0 = dc;
     qd.signs1 = nullptr;
     qd.scales1 = nullptr;
-    qd.rout = rout;
     qd.rows = static_cast<int>(H);
     qd.K = static_cast<int>(I);
     qd.NG = static_cast<int>(I / 128);
-    err = launch_moe_decode<false>(qd, stream);
-    if (err != cudaSuccess) return err;
-    const int64_t total4 = T * (H / 4);
-    int64_t blocks = (total4 + 255) / 256;
-    if (blocks > 8 * num_sms) blocks = 8 * num_sms;
-    return launch_pdl(moe_combine_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, stream,
-                      static_cast<const float*>(rout), static_cast<const int*>(pos), static_cast<int>(T),
-                      static_cast<int>(H), top_k, out);
+    return launch_moe_decode_down(qd, static_cast<int>(T), out, stream);
   }
   // 2. sort + tile lists
   constexpr int kStageMax = 16384;  // routes staged in shared memory (64 KB)
