@@ -434,7 +434,7 @@ def moe_rows(torch, ops, synth, peaks, iters: int = 8):
         gbs = float(np.mean(touched)) / (dms * 1e-3) / 1e9
         decode.append({"T": Td, "us": round(dms * 1e3, 2), "tokens/s": round(Td / (dms * 1e-3), 1),
                        "weight_GB/s": round(gbs, 1), "frac_hbm": round(gbs / peaks["hbm_gbs"], 4),
-                       "launches_per_call": 3})
+                       "launches_per_call": 2 if Td <= 4 else 3})
     row["decode"] = decode
     return row
 

@@ -192,9 +192,10 @@ size_t w1_gemm_workspace_size(int64_t M, int64_t K);
  * into sorted order (fp16, exact per-token power of two), grouped gate/up GEMM
  * (tcgen05, +-s fp16 weight operand, fused SwiGLU), h to fp16 per route,
  * grouped down GEMM (route weight applied), slot-ordered combine.
- * T <= 16 (decode regime): three kernels: router, per-route gate/up products
- * with fused SwiGLU, per-token down products over the token's slots with the
- * slot-ordered combine fused; the products are the batch-1 steps of w1_gemv.
+ * T <= 16 (decode regime): per-route gate/up products with fused SwiGLU (up
+ * to 4 tokens each CTA routes its token; above, a router kernel runs first),
+ * then per-token down products over the token's slots with the slot-ordered
+ * combine fused; the products are the batch-1 steps of w1_gemv.
  * Deterministic.  Accuracy per stage as w1_gemm: 1e-3 * sum|s x| for g, u and
  * D_e h.  The workspace must be 1024-byte aligned (W1_ERR_ALIGN otherwise).
  */

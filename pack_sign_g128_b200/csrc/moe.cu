@@ -11,9 +11,10 @@
 // kept un-duplicated, fused SwiGLU, skipped empty tiles.
 //
 // Up to 16 tokens (the decode regime) the layer runs as per-route products:
-// router, a fused gate/up + SwiGLU kernel, and a down kernel that also does
-// the slot-ordered combine (three launches; see "decode regime" below).
-// Larger batches take the expert-sorted tile pipeline.
+// gate/up + SwiGLU (up to 4 tokens with the routing computed in each CTA,
+// else after the router kernel) and down with the slot-ordered combine (see
+// "decode regime" below).  Larger batches take the expert-sorted tile
+// pipeline.
 //
 // Seven launches on one stream (programmatic dependent launch between them):
 //  1. route_kernel     warp per token: fp32 softmax, top-k by logit, weights,
@@ -153,10 +154,60 @@ __device__ __forceinline__ float warp_max(float v) {
 
 // ------------------------------------------------------------------ 1. router
 
-// One warp per token.  Selection is by logit (the softmax is monotone, so this
-// is selection by probability without rounding ties); weights are fp32.  The
-// warp also finds the token's fp16 multiplier 2^c for the gate/up operand
-// (xcs[t]), once per token instead of once per route.
+// One warp routes one token from its E logits: fp32 softmax, the top_k
+// experts by logit (the softmax is monotone, so this is selection by
+// probability without rounding ties; ties to the lower index); lane 0 writes
+// ids[s], wts[s] for s < top_k.
+__device__ __forceinline__ void moe_route_token(const float* __restrict__ lp, int E, int top_k, int lane,
+                                                int* ids, float* wts) {
+  constexpr int PER = moe::kMaxE / 32;
+  float z[PER];
+#pragma unroll
+  for (int j = 0; j < PER; ++j) {
+    const int e = lane + 32 * j;
+    z[j] = (e < E) ? lp[e] : -INFINITY;
+  }
+  float mx = -INFINITY;
+#pragma unroll
+  for (int j = 0; j < PER; ++j) mx = fmaxf(mx, z[j]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+  float sum = 0.f;
+#pragma unroll
+  for (int j = 0; j < PER; ++j) sum += (lane + 32 * j < E) ? expf(z[j] - mx) : 0.f;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
+  for (int s = 0; s < top_k; ++s) {
+    // lane-local best: largest logit, lowest index on ties
+    float bz = -INFINITY;
+    int be = 0x7FFFFFFF;
+#pragma unroll
+    for (int j = 0; j < PER; ++j) {
+      const int e = lane + 32 * j;
+      if (e < E && (z[j] > bz || (z[j] == bz && e < be))) {
+        bz = z[j];
+        be = e;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float oz = __shfl_xor_sync(0xFFFFFFFFu, bz, o);
+      const int oe = __shfl_xor_sync(0xFFFFFFFFu, be, o);
+      if (oz > bz || (oz == bz && oe < be)) {
+        bz = oz;
+        be = oe;
+      }
+    }
+    if (lane == 0) {
+      ids[s] = be;
+      wts[s] = expf(bz - mx) / sum;
+    }
+    if ((be & 31) == lane) z[be >> 5] = -INFINITY;  // taken
+  }
+}
+
+// One warp per token: routing, and the token's fp16 multiplier 2^c for the
+// gate/up operand (xcs[t]), once per token instead of once per route.
 __global__ void __launch_bounds__(256) moe_route_kernel(const float* __restrict__ logits, int T, int E, int top_k,
                                                         int* __restrict__ ids, float* __restrict__ wts,
                                                         const uint16_t* __restrict__ x, int H,
@@ -165,51 +216,8 @@ __global__ void __launch_bounds__(256) moe_route_kernel(const float* __restrict_
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (warp < T) {
-    constexpr int PER = moe::kMaxE / 32;
-    float z[PER];
-    const float* lp = logits + static_cast<int64_t>(warp) * E;
-#pragma unroll
-    for (int j = 0; j < PER; ++j) {
-      const int e = lane + 32 * j;
-      z[j] = (e < E) ? lp[e] : -INFINITY;
-    }
-    float mx = -INFINITY;
-#pragma unroll
-    for (int j = 0; j < PER; ++j) mx = fmaxf(mx, z[j]);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
-    float sum = 0.f;
-#pragma unroll
-    for (int j = 0; j < PER; ++j) sum += (lane + 32 * j < E) ? expf(z[j] - mx) : 0.f;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
-    for (int s = 0; s < top_k; ++s) {
-      // lane-local best: largest logit, lowest index on ties
-      float bz = -INFINITY;
-      int be = 0x7FFFFFFF;
-#pragma unroll
-      for (int j = 0; j < PER; ++j) {
-        const int e = lane + 32 * j;
-        if (e < E && (z[j] > bz || (z[j] == bz && e < be))) {
-          bz = z[j];
-          be = e;
-        }
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const float oz = __shfl_xor_sync(0xFFFFFFFFu, bz, o);
-        const int oe = __shfl_xor_sync(0xFFFFFFFFu, be, o);
-        if (oz > bz || (oz == bz && oe < be)) {
-          bz = oz;
-          be = oe;
-        }
-      }
-      if (lane == 0) {
-        ids[warp * top_k + s] = be;
-        wts[warp * top_k + s] = expf(bz - mx) / sum;
-      }
-      if ((be & 31) == lane) z[be >> 5] = -INFINITY;  // taken
-    }
+    moe_route_token(logits + static_cast<int64_t>(warp) * E, E, top_k, lane, ids + warp * top_k,
+                    wts + warp * top_k);
     const uint4* xr = reinterpret_cast<const uint4*>(x + static_cast<int64_t>(warp) * H);
     float m = 0.f;
 #pragma unroll 4
@@ -791,8 +799,11 @@ constexpr int kSmemCap = 220 * 1024;     // dynamic shared memory the decode ker
 }  // namespace moed
 
 struct MoeDecParams {
-  const int* ids;            // [R] expert per route
-  const float* wts;          // [R] route weight
+  const float* logits;       // gate/up with self_route: router logits [T][E]
+  int E;
+  int self_route;            // gate/up: each CTA routes its token (else ids come from the router kernel)
+  int* ids;                  // [R] expert per route (written by gate/up, read by down)
+  float* wts;                // [R] route weight
   const uint16_t* x;         // gate/up: tokens [T][H] bf16; down: h [R][I] bf16
   const uint32_t* signs0;    // gate/up: G, down: D   [E][rows][K/32]
   const uint16_t* scales0;
@@ -812,10 +823,26 @@ __global__ void __launch_bounds__(moed::kWarps * 32, 1) moe_decode_gateup_kernel
   __shared__ float gu[2][moed::kRowsGu];
   const GdSmem L = moed_layout(q);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int r = blockIdx.y;
+  __shared__ int sid[moe::kMaxTopK];
+  __shared__ float swt[moe::kMaxTopK];
+  const int r = blockIdx.y, t = r / q.top_k, slot = r - t * q.top_k;
   pdl_wait();
   pdl_launch_dependents();
-  const int e = q.ids[r];
+  // self_route: the token's routing, computed by every CTA of the token from
+  // the router kernel's routine; the route's first row block records it
+  int e;
+  if (q.self_route) {
+    if (warp == 0) moe_route_token(q.logits + static_cast<int64_t>(t) * q.E, q.E, q.top_k, lane, sid, swt);
+    __syncthreads();
+    e = sid[slot];
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+      q.ids[r] = e;
+      q.wts[r] = swt[slot];
+    }
+  } else {
+    e = q.ids[r];
+  }
+  if (blockIdx.x == 0 && threadIdx.x == 0) q.pos[r] = r;
   // this warp's matrix (0: G, 1: U) and rows
   const int mat = warp >> 2;
   const int row0 = blockIdx.x * moed::kRowsGu + (warp & 3) * 8 * moed::kTw;
@@ -823,7 +850,7 @@ __global__ void __launch_bounds__(moed::kWarps * 32, 1) moe_decode_gateup_kernel
   const int64_t mrow = static_cast<int64_t>(e) * q.rows;  // the expert's first row
   p.signs = (mat ? q.signs1 : q.signs0) + mrow * (q.K >> 5);
   p.scales = (mat ? q.scales1 : q.scales0) + mrow * q.NG;
-  p.x = q.x + static_cast<int64_t>(r / q.top_k) * q.K;
+  p.x = q.x + static_cast<int64_t>(t) * q.K;
   p.N = q.rows;
   p.K = q.K;
   p.NG = q.NG;
@@ -873,7 +900,6 @@ __global__ void __launch_bounds__(moed::kWarps * 32, 1) moe_decode_gateup_kernel
     gu[mat][base + 8 + rl] = v1;
   }
   __syncthreads();
-  if (blockIdx.x == 0 && threadIdx.x == 0) q.pos[r] = r;
   for (int i = threadIdx.x; i < moed::kRowsGu; i += blockDim.x) {
     const int row = blockIdx.x * moed::kRowsGu + i;
     if (row < q.rows) {
@@ -1106,14 +1132,10 @@ cudaError_t launch_moe(const uint16_t* x, const float* logits, int64_t T, int64_
   const int R = static_cast<int>(T * top_k);
 
   cudaError_t err;
-  // 1. router
-  float* xcs = reinterpret_cast<float*>(ws + L.xcs);
-  err = launch_pdl(moe_route_kernel, dim3(static_cast<unsigned>((T + 7) / 8)), dim3(256), 0, stream, logits,
-                   static_cast<int>(T), E, top_k, ids, wts, x, static_cast<int>(H), xcs);
-  if (err != cudaSuccess) return err;
   // Decode regime: a few tokens, about one route per expert -> per-route
-  // products on the direct GEMV steps.  Measured on the OLMoE-like layer: 2x
-  // faster than the tile pipeline up to 8 tokens, still ahead at 16.
+  // products on the direct GEMV steps: gate/up (with the routing up to 4
+  // tokens), down with the combine.  Measured on the OLMoE-like layer: about 2x faster
+  // than the tile pipeline up to 8 tokens, still ahead at 16.
   // W1_MOE_PATH=tiles|decode forces a path (testing knob).
   constexpr int64_t kDecodeMaxT = 16;
   const char* mpath = getenv("W1_MOE_PATH");
@@ -1126,7 +1148,19 @@ cudaError_t launch_moe(const uint16_t* x, const float* logits, int64_t T, int64_
              moe_down_layout(static_cast<int>(I / 128), 16).total <= moed::kSmemCap;
   }
   if (decode) {
+    // up to 4 tokens each CTA routes its token (one launch less); above,
+    // the router kernel does it once per token
+    constexpr int64_t kSelfRouteMaxT = 4;
     MoeDecParams q = {};
+    q.logits = logits;
+    q.E = E;
+    q.self_route = T <= kSelfRouteMaxT ? 1 : 0;
+    if (!q.self_route) {
+      float* xcs = reinterpret_cast<float*>(ws + L.xcs);
+      err = launch_pdl(moe_route_kernel, dim3(static_cast<unsigned>((T + 7) / 8)), dim3(256), 0, stream, logits,
+                       static_cast<int>(T), E, top_k, ids, wts, x, static_cast<int>(H), xcs);
+      if (err != cudaSuccess) return err;
+    }
     q.ids = ids;
     q.wts = wts;
     q.x = x;
@@ -1154,6 +1188,11 @@ cudaError_t launch_moe(const uint16_t* x, const float* logits, int64_t T, int64_
     qd.NG = static_cast<int>(I / 128);
     return launch_moe_decode_down(qd, static_cast<int>(T), out, stream);
   }
+  // 1. router
+  float* xcs = reinterpret_cast<float*>(ws + L.xcs);
+  err = launch_pdl(moe_route_kernel, dim3(static_cast<unsigned>((T + 7) / 8)), dim3(256), 0, stream, logits,
+                   static_cast<int>(T), E, top_k, ids, wts, x, static_cast<int>(H), xcs);
+  if (err != cudaSuccess) return err;
   // 2. sort + tile lists
   constexpr int kStageMax = 16384;  // routes staged in shared memory (64 KB)
   SortArgs sa{ids,  R,   E,       top_k,    static_cast<int>(I / 128), static_cast<int>(H / 128), offsets, sroute,
