@@ -29,6 +29,11 @@ rational arithmetic:
 * Routed MoE -- every (token, slot) route carries an expert id and a route
   weight; gate/up consume the token's shared hidden state, down consumes the
   route's own intermediate (DBF post, section 4, MoE input topologies).
+* Rotated activations -- one orthogonal rotation of the input space, factored
+  as the Kronecker product of two small orthogonal matrices H and R; the
+  weights are binarised in the rotated coordinates and the activations take
+  the same rotation, so the product is unchanged (zhichai.net post on BWLA,
+  section 3 "OKT" and section 5).
 
 Readings where the pages are silent are listed in the repository's design
 notes: scale rule mean|w|; fp16 scale; LSB-first bit order inside uint32
@@ -271,6 +276,48 @@ def dbf_dense_ref(a_bits, B1_words, mid_bits, B2_words, b_bits, m: int, r: int, 
     U = 1.0 - 2.0 * unpack_bits_lsb_first(B1_words, r).astype(np.float64)
     V = 1.0 - 2.0 * unpack_bits_lsb_first(B2_words, n).astype(np.float64)
     return (a[:, None] * U) @ (mid[:, None] * (V * b[None, :]))
+
+
+# ---------------------------------------------------------------------------
+# Orthogonal-Kronecker rotation of the activations (zhichai.net post on BWLA,
+# sections 3 and 5).
+# ---------------------------------------------------------------------------
+
+
+def okt_rotate_ref(H, R, x) -> np.ndarray:
+    """Rotated activations x_rot = (H kron R)^T x for every batch row, float64.
+
+    H: [n1, n1], R: [n2, n2] (any float dtype, taken exactly), x: [B, K] with
+    K = n1 n2.  The post writes the rotation as H kron R with n1 n2 = K
+    (section 3) and applies its transpose to the activations (section 5).  For
+    y = W x with W [N, K] (outputs x inputs), the weights are stored as
+    W (H kron R), and W (H kron R) (H kron R)^T x = W x.  Read x[b, i n2 + j]
+    as X[i, j] (n1 x n2, row-major).  Then (A kron B) x is A X B^T, so
+    (H kron R)^T x is H^T X R.
+    """
+    H = np.asarray(H, dtype=np.float64)
+    R = np.asarray(R, dtype=np.float64)
+    x = np.asarray(x, dtype=np.float64)
+    n1, n2 = H.shape[0], R.shape[0]
+    Bn, K = x.shape
+    assert H.shape == (n1, n1) and R.shape == (n2, n2) and n1 * n2 == K
+    out = np.empty((Bn, K), dtype=np.float64)
+    for b in range(Bn):
+        X = x[b].reshape(n1, n2)
+        out[b] = (H.T @ X @ R).reshape(K)
+    return out
+
+
+def okt_gemv_ref(signs, scale_bits, H, R, x, K: int):
+    """y = w_hat (H kron R)^T x: the packed weights (stored in the rotated
+    coordinates) applied to the rotated activations, in float64.
+
+    Returns (y [B, N], bound [B, N], x_rot [B, K]); bound is
+    sum_k |s x_rot_k|, the scale of the product's error tolerance.
+    """
+    x_rot = okt_rotate_ref(H, R, x)
+    y, bound = matmul_ref(x_rot, signs, scale_bits, K)
+    return y, bound, x_rot
 
 
 # ---------------------------------------------------------------------------

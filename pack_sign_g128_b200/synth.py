@@ -13,12 +13,18 @@ Recipes (the pages' workloads stand in by shape; no model or dataset):
           expert gate/up I x H and down H x I fp32 ~ N(0, 0.02)
   dbf     seed 4: U (m x r) and V (r x n) uniform random sign bits;
           diagonals fp16 |N(0, 0.05)| + 0.01; x B x n bf16 ~ N(0, 1)
+  okt     seed 5: Kronecker factors H (n1 x n1) and R (n2 x n2), each the
+          Q factor of a seeded N(0, 1) matrix (columns signed so that the
+          triangular factor has a positive diagonal), rounded to fp32;
+          weights as stored after the rotation, N x K ~ N(0, 0.02) (an
+          orthogonal rotation of i.i.d. Gaussian rows is again i.i.d.
+          Gaussian, so these stand for W (H kron R)); x B x K bf16 ~ N(0, 1)
 """
 from __future__ import annotations
 
 import numpy as np
 
-SEEDS = {"tiny": 0, "gemv": 1, "gemm": 2, "moe": 3, "dbf": 4}
+SEEDS = {"tiny": 0, "gemv": 1, "gemm": 2, "moe": 3, "dbf": 4, "okt": 5}
 
 
 def rng(seed: int) -> np.random.Generator:
@@ -99,3 +105,19 @@ def dbf_case(m: int = 4096, r: int = 4096, n: int = 4096, B: int = 1, seed: int 
     b = diag_fp16(g, n)
     x = activations_bf16(g, B, n)
     return a, B1, mid, B2, b, x
+
+
+def orthogonal_f32(g: np.random.Generator, n: int) -> np.ndarray:
+    """A random n x n orthogonal matrix rounded to fp32 (Q of a Gaussian)."""
+    q, r = np.linalg.qr(g.standard_normal(size=(n, n)))
+    q = q * np.where(np.diag(r) < 0, -1.0, 1.0)[None, :]
+    return q.astype(np.float32)
+
+
+def okt_case(N: int, K: int, n1: int, n2: int, B: int, seed: int = SEEDS["okt"]):
+    """Returns H f32 [n1, n1], R f32 [n2, n2], rotated weights f32 [N, K], x bf16 [B, K]."""
+    assert n1 * n2 == K
+    g = rng(seed)
+    H = orthogonal_f32(g, n1)
+    R = orthogonal_f32(g, n2)
+    return H, R, weights(g, N, K), activations_bf16(g, B, K)

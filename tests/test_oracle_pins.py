@@ -414,3 +414,91 @@ def test_fast_pack_equals_plain_pack():
     s2, c2 = O.pack_ref_fast(W)
     assert np.array_equal(s1, s2)
     assert np.array_equal(c1, c2)
+
+
+# ---------------------------------------------------------------- rotated activations
+
+def _fwht(v):
+    """Unnormalised fast Walsh-Hadamard transform along axis 0 (butterflies)."""
+    v = np.array(v, dtype=np.float64)
+    h = 1
+    while h < v.shape[0]:
+        for i in range(0, v.shape[0], 2 * h):
+            a = v[i:i + h].copy()
+            b = v[i + h:i + 2 * h].copy()
+            v[i:i + h] = a + b
+            v[i + h:i + 2 * h] = a - b
+        h *= 2
+    return v
+
+
+@pytest.mark.parametrize("n1,n2", [(8, 16), (16, 16), (32, 4)])
+def test_okt_rotate_equals_explicit_kronecker_matrix(n1, n2):
+    """Brute force: build the K x K matrix (H kron R) and apply its transpose."""
+    g = synth.rng(50 + n1)
+    H = synth.orthogonal_f32(g, n1)
+    R = synth.orthogonal_f32(g, n2)
+    x = O.bf16_bits_to_f64(synth.activations_bf16(g, 3, n1 * n2))
+    M = np.kron(H.astype(np.float64), R.astype(np.float64))
+    ref = x @ M  # row b of this is (M^T x_b)^T
+    out = O.okt_rotate_ref(H, R, x)
+    assert np.max(np.abs(out - ref)) <= 1e-13 * np.max(np.abs(ref))
+
+
+def test_okt_rotate_hadamard_factor_is_a_walsh_hadamard_transform():
+    """H = Sylvester Hadamard / sqrt(n1), R = identity: each column j of the
+    n1 x n2 view is Walsh-Hadamard transformed (H is symmetric)."""
+    n1, n2 = 64, 8
+    H = _sylvester(n1) / 8.0
+    x = O.bf16_bits_to_f64(synth.activations_bf16(synth.rng(52), 2, n1 * n2))
+    out = O.okt_rotate_ref(H, np.eye(n2), x)
+    for b in range(2):
+        ref = _fwht(x[b].reshape(n1, n2)) / 8.0
+        assert np.max(np.abs(out[b].reshape(n1, n2) - ref)) <= 1e-14 * np.max(np.abs(ref))
+
+
+def test_okt_rotate_permutation_factor_permutes_columns():
+    """H = I, R a permutation matrix with R[pi(j), j] = 1: X R moves column
+    pi(j) of the n1 x n2 view to column j, exactly."""
+    n1, n2 = 4, 32
+    pi = synth.rng(53).permutation(n2)
+    R = np.zeros((n2, n2))
+    R[pi, np.arange(n2)] = 1.0
+    x = O.bf16_bits_to_f64(synth.activations_bf16(synth.rng(54), 2, n1 * n2))
+    out = O.okt_rotate_ref(np.eye(n1), R, x)
+    ref = x.reshape(2, n1, n2)[:, :, pi].reshape(2, n1 * n2)
+    assert np.array_equal(out, ref)
+
+
+def test_okt_rotate_preserves_norm_and_inverts():
+    """Orthogonal factors: ||x_rot|| = ||x||, and rotating by (H^T, R^T)
+    returns x (the rotation's inverse is its transpose)."""
+    n1, n2 = 64, 64
+    g = synth.rng(55)
+    H = np.linalg.qr(g.standard_normal((n1, n1)))[0]
+    R = np.linalg.qr(g.standard_normal((n2, n2)))[0]
+    x = O.bf16_bits_to_f64(synth.activations_bf16(g, 4, n1 * n2))
+    xr = O.okt_rotate_ref(H, R, x)
+    assert np.allclose(np.linalg.norm(xr, axis=1), np.linalg.norm(x, axis=1), rtol=1e-12, atol=0)
+    back = O.okt_rotate_ref(H.T, R.T, xr)
+    assert np.max(np.abs(back - x)) <= 1e-12 * np.max(np.abs(x))
+
+
+def test_okt_forward_equivalence():
+    """W x = (W (H kron R)) ((H kron R)^T x) for dense W, and the packed product
+    of the rotated weights is the dequantised rotated weights times x_rot."""
+    n1, n2, N = 16, 16, 40
+    K = n1 * n2
+    g = synth.rng(56)
+    H = np.linalg.qr(g.standard_normal((n1, n1)))[0]
+    R = np.linalg.qr(g.standard_normal((n2, n2)))[0]
+    W = g.standard_normal((N, K)) * 0.02
+    x = O.bf16_bits_to_f64(synth.activations_bf16(g, 2, K))
+    W_rot = W @ np.kron(H, R)
+    xr = O.okt_rotate_ref(H, R, x)
+    assert np.max(np.abs(xr @ W_rot.T - x @ W.T)) <= 1e-12 * np.max(np.abs(x @ W.T))
+    signs, scales = O.pack_ref(W_rot.astype(np.float32))
+    y, bound, x_rot = O.okt_gemv_ref(signs, scales, H, R, x, K)
+    w_hat = O.dequant_ref(signs, scales, K)
+    assert np.array_equal(x_rot, xr)
+    assert np.max(np.abs(y - xr @ w_hat.T)) <= 1e-13 * np.max(bound)
