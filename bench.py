@@ -509,6 +509,60 @@ def dbf_rows(torch, ops, synth, peaks, l2_bytes: int, iters: int = 5):
     return rows
 
 
+OKT_FACTORS = {4096: (64, 64), 11008: (86, 128)}
+
+
+def okt_rows(torch, ops, synth, combos, stream, reps: int = 3):
+    """Rotated-activation decode products on the sweep's pairs and weight copies
+    (timing only: any packed matrix times the same): per call, w1_okt_gemv
+    (rotation + product, weights static), w1_okt_rotate alone, and the plain
+    static-weights product on bf16 x for comparison.  CUDA graphs of R
+    back-to-back calls over the pair's rotating copies, CUDA events."""
+    dev = torch.device("cuda")
+    rows = []
+
+    def graph_us(fn, R):
+        with torch.cuda.stream(stream):
+            for r in range(3):
+                fn(r)
+        stream.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for r in range(R):
+                fn(r)
+        with torch.cuda.stream(stream):
+            g.replay()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(reps):
+                g.replay()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) * 1e3 / (reps * R)
+
+    for cb in combos:
+        N, K, B, R = cb["N"], cb["K"], cb["B"], cb["R"]
+        n1, n2 = OKT_FACTORS[K]
+        g = synth.rng(500 + K)
+        H = torch.from_numpy(synth.orthogonal_f32(g, n1)).to(dev)
+        Rm = torch.from_numpy(synth.orthogonal_f32(g, n2)).to(dev)
+        xr = torch.empty((B, K), dtype=torch.float32, device=dev)
+        x, y = cb["x"], cb["y"]
+        full = graph_us(lambda r: ops.w1_okt_gemv(cb["signs"][r], cb["scales"][r], H, Rm, x, y=y, x_rot=xr,
+                                                  static_weights=True), R)
+        rot = graph_us(lambda r: ops.w1_okt_rotate(H, Rm, x, x_rot=xr), R)
+        plain = graph_us(lambda r: ops.w1_gemv(cb["signs"][r], cb["scales"][r], x, y, static_weights=True), R)
+        rows.append({"N": N, "K": K, "B": B, "n1": n1, "n2": n2, "okt_gemv_us": round(full, 3),
+                     "rotate_us": round(rot, 3), "gemv_static_us": round(plain, 3),
+                     "added_us": round(full - plain, 3),
+                     "okt_weight_GB/s": round(cb["bytes"] / (full * 1e-6) / 1e9, 1)})
+    torch.cuda.synchronize()
+    return rows
+
+
 def cpu_oracle_gemv_sample(combos_spec, packed_host, max_seconds: float = 20.0):
     """Time the fp64 oracle on the sweep (one launch per pair) on the host."""
     from oracle import w1_oracle as O
@@ -583,6 +637,9 @@ def run_gpu(args):
             rows["dbf"] = dbf_rows(torch, ops, synth, peaks, l2)
         elif args.section == "gemv1":
             rows["gemv1"] = gemv_one(torch, ops, synth, args.shape)
+        elif args.section == "okt":
+            combos, stream = build_gemv_sweep(torch, ops, synth, l2)
+            rows["okt"] = okt_rows(torch, ops, synth, combos, stream)
         if rank == 0:
             print(json.dumps({"section": args.section, "rows": rows}), flush=True)
         return
@@ -632,6 +689,7 @@ def run_gpu(args):
         rows["gemm"] = gemm_rows(torch, ops, synth, peaks)
         rows["moe"] = moe_rows(torch, ops, synth, peaks)
         rows["dbf"] = dbf_rows(torch, ops, synth, peaks, l2)
+        rows["okt"] = okt_rows(torch, ops, synth, combos, stream)
     cpu = None
     if rank == 0 and world == 1 and not args.skip_cpu:
         packed_host = {}
@@ -757,7 +815,7 @@ def main():
                     help="N,K,B of the single GEMV that --section gemv1 launches (for ncu captures)")
     ap.add_argument("--choices", default=None,
                     help="JSON line of an earlier run: pin each GEMV pair to the kernel it chose (profiling)")
-    ap.add_argument("--section", default="all", choices=["all", "gemm", "moe", "dbf", "gemv1"],
+    ap.add_argument("--section", default="all", choices=["all", "gemm", "moe", "dbf", "gemv1", "okt"],
                     help="run one row only (for profiling); prints a rows-only JSON line")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -144,6 +144,48 @@ int w1_gemv_choice(int64_t N, int64_t K, int64_t B, uint32_t flags, char* out, s
 int w1_gemv_set_choice(int64_t N, int64_t K, int64_t B, uint32_t flags, const char* name);
 
 /*
+ * w1_okt_rotate -- rotated activations for weights binarised in rotated
+ * coordinates (zhichai.net post on BWLA, section 3 "OKT": one orthogonal
+ * rotation factored as a Kronecker product H kron R of two small orthogonal
+ * matrices, n1 n2 = K; section 5: the activations take the same rotation, so
+ * the product is unchanged).
+ *   x_rot[b] = (H kron R)^T x[b].  With x[b][i*n2 + j] read as X[i][j]
+ *   (n1 x n2, row-major), x_rot[b] viewed the same way is H^T X R.
+ *   H fp32 [n1][n1], R fp32 [n2][n2] (row-major; orthogonality is the
+ *   caller's, nothing checks it), x bf16 [B][K], x_rot fp32 [B][K] (device).
+ * Limits: n1 * n2 = K, K a multiple of 128 and <= 65536, 1 <= n1 <= 1024,
+ * 1 <= n2 <= 128, 1 <= B <= 65535; otherwise W1_ERR_SHAPE.  A shape whose
+ * staging exceeds the device's shared memory returns W1_ERR_UNSUPPORTED.
+ * Accuracy: each element is two fp32 dot products in a fixed order (over
+ * n1, then n2), so |x_rot - exact| <= (n1 + n2 + 2) * 2^-24 *
+ * (|H|^T |X| |R|)[i][j]; results are bitwise reproducible.
+ */
+int w1_okt_rotate(const float* H, int64_t n1, const float* R, int64_t n2, const uint16_t* x, int64_t B,
+                  float* x_rot, w1_stream_t stream);
+
+/*
+ * w1_okt_gemv -- decode product against weights stored in rotated
+ * coordinates: w1_okt_rotate, then the 1-bit product on the fp32 x_rot.
+ *   y[b][n] = sum_g s[n][g] * sum_{k in g} (1 - 2*bit[n][k]) * x_rot[b][k],
+ *   where signs/scales are w1_pack of W (H kron R), so y = W x up to the
+ *   binarisation.  1 <= B <= 8; the limits of w1_okt_rotate apply, with K
+ *   the weights' K.
+ *   x_rot: caller-owned fp32 [B][K] scratch; it receives the rotated
+ *   activations.  It must not alias x or y.
+ * flags: W1_GEMV_STATIC_WEIGHTS as for w1_gemv_ex.  The promise then also
+ * covers H and R, which the rotation may read before the preceding kernel
+ * completes.  Two kernels: the product launches while the rotation runs and
+ * stages its weights; it reads x_rot only after the rotation has finished.
+ * The product picks its kernel (the direct kernel, whose fp32 activation
+ * path this uses) by first-call timing, like w1_gemv.
+ * Accuracy: |y - y_exact| <= 1e-3 * sum_k |s x_rot_k| per element, plus the
+ * rotation's error carried through the product.
+ */
+int w1_okt_gemv(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t K, const float* H, int64_t n1,
+                const float* R, int64_t n2, const uint16_t* x, int64_t B, float* x_rot, float* y, uint32_t flags,
+                w1_stream_t stream);
+
+/*
  * w1_gemm -- prefill-regime product for many token rows (DBF post, section 4:
  * prompt processing amortises weight loads across columns).
  *   y[m][n] = sum_g s[n][g] * sum_{k in g} (1 - 2*bit[n][k]) * x[m][k].

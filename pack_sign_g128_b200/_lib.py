@@ -41,6 +41,8 @@ SIGNATURES = {
     "dbf_apply": (_int, [_p, _p, _p, _p, _p, _i64, _i64, _i64, _p, _i64, _p, _p, _sz, _p]),
     "dbf_workspace_size": (_sz, [_i64, _i64, _i64, _i64]),
     "dbf_apply_noalloc": (_int, [_p, _p, _p, _p, _p, _i64, _i64, _i64, _p, _i64, _p, _p]),
+    "w1_okt_rotate": (_int, [_p, _i64, _p, _i64, _p, _i64, _p, _p]),
+    "w1_okt_gemv": (_int, [_p, _p, _i64, _i64, _p, _i64, _p, _i64, _p, _i64, _p, _p, ctypes.c_uint32, _p]),
 }
 
 _lib = None

@@ -312,8 +312,8 @@ static cudaError_t launch_gemv_nb(const uint32_t* signs, const GemvParams& base,
 cudaError_t launch_gemv_tc(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t K, const uint16_t* x,
                            int B, float* y, bool static_weights, cudaStream_t stream, int num_sms, int force_s);
 cudaError_t launch_gemv_direct(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t K,
-                               const uint16_t* x, int B, float* y, bool static_weights, cudaStream_t stream,
-                               int num_sms, int smem_cap, int force_s, int warps);
+                               const void* x, bool x_f32, int B, float* y, bool static_weights,
+                               cudaStream_t stream, int num_sms, int smem_cap, int force_s, int warps);
 
 // The mma.sync ring kernel over row chunks (the fallback for shapes outside
 // the other two kernels' plans).
@@ -352,7 +352,9 @@ static cudaError_t launch_gemv_ring(const uint32_t* signs, const uint16_t* scale
 
 // ------------------------------------------------------------------ dispatch
 
-// Kernel and K split per (device, N, K, B, static weights), chosen by timing.
+// Kernel and K split per (device, N, K, B, static weights, activation type),
+// chosen by timing.  fp32 activations (the rotated-activation product) are
+// read only by the direct kernel, so only its candidates are timed for them.
 // The first call for a shape (outside stream capture) runs each candidate --
 // the direct kernel with K split 1, 2, 4, 8 at 8 and at 16 warps per CTA, the
 // tcgen05 kernel, the ring kernel -- three times plainly and twelve times back
@@ -374,6 +376,7 @@ struct GemvChoiceEntry {
   int64_t N, K;
   int B;
   bool st;
+  bool xf;  // fp32 activations (direct kernel only)
   GemvChoice c;
 };
 GemvChoiceEntry g_choice[256];
@@ -381,30 +384,37 @@ int g_nchoice = 0;
 std::mutex g_choice_mu;
 }  // namespace
 
+// x is bf16 [B][K], or fp32 [B][K] with xf (which only the direct kernel reads).
 static cudaError_t run_gemv_choice(const GemvChoice& c, const uint32_t* signs, const uint16_t* scales, int64_t N,
-                                   int64_t K, const uint16_t* x, int B, float* y, cudaStream_t stream, int num_sms,
-                                   int smem_cap, bool static_weights) {
+                                   int64_t K, const void* x, bool xf, int B, float* y, cudaStream_t stream,
+                                   int num_sms, int smem_cap, bool static_weights) {
+  const uint16_t* xb = static_cast<const uint16_t*>(x);
   switch (c.kind) {
     case 'd':
-      return launch_gemv_direct(signs, scales, N, K, x, B, y, static_weights, stream, num_sms, smem_cap, c.s, c.w);
+      return launch_gemv_direct(signs, scales, N, K, x, xf, B, y, static_weights, stream, num_sms, smem_cap, c.s,
+                                c.w);
     case 't':
-      return launch_gemv_tc(signs, scales, N, K, x, B, y, static_weights, stream, num_sms, c.s);
+      if (xf) return cudaErrorNotSupported;
+      return launch_gemv_tc(signs, scales, N, K, xb, B, y, static_weights, stream, num_sms, c.s);
     default:
-      return launch_gemv_ring(signs, scales, N, K, x, B, y, stream, num_sms, smem_cap);
+      if (xf) return cudaErrorNotSupported;
+      return launch_gemv_ring(signs, scales, N, K, xb, B, y, stream, num_sms, smem_cap);
   }
 }
 
 // The static rule with fallbacks (direct or tcgen05 first by batch, then ring).
+// With fp32 activations only the direct kernel applies: 8 warps, then 16.
 static cudaError_t run_gemv_rule(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t K,
-                                 const uint16_t* x, int B, float* y, cudaStream_t stream, int num_sms, int smem_cap,
-                                 bool static_weights) {
-  const GemvChoice first = B <= 4 ? GemvChoice{'d', 0, 8} : GemvChoice{'t', 0, 0};
-  const GemvChoice second = B <= 4 ? GemvChoice{'t', 0, 0} : GemvChoice{'d', 0, 8};
-  cudaError_t e = run_gemv_choice(first, signs, scales, N, K, x, B, y, stream, num_sms, smem_cap, static_weights);
+                                 const void* x, bool xf, int B, float* y, cudaStream_t stream, int num_sms,
+                                 int smem_cap, bool static_weights) {
+  const GemvChoice first = (B <= 4 || xf) ? GemvChoice{'d', 0, 8} : GemvChoice{'t', 0, 0};
+  const GemvChoice second = xf ? GemvChoice{'d', 0, 16} : (B <= 4 ? GemvChoice{'t', 0, 0} : GemvChoice{'d', 0, 8});
+  cudaError_t e =
+      run_gemv_choice(first, signs, scales, N, K, x, xf, B, y, stream, num_sms, smem_cap, static_weights);
   if (e != cudaErrorNotSupported) return e;
-  e = run_gemv_choice(second, signs, scales, N, K, x, B, y, stream, num_sms, smem_cap, static_weights);
-  if (e != cudaErrorNotSupported) return e;
-  return launch_gemv_ring(signs, scales, N, K, x, B, y, stream, num_sms, smem_cap);
+  e = run_gemv_choice(second, signs, scales, N, K, x, xf, B, y, stream, num_sms, smem_cap, static_weights);
+  if (e != cudaErrorNotSupported || xf) return e;
+  return launch_gemv_ring(signs, scales, N, K, static_cast<const uint16_t*>(x), B, y, stream, num_sms, smem_cap);
 }
 
 // One autotune measurement: `reps` back-to-back launches of candidate c
@@ -413,11 +423,11 @@ static cudaError_t run_gemv_rule(const uint32_t* signs, const uint16_t* scales, 
 // Returns 1 with *ms set, 0 when c does not fit or cannot be captured, -1 on
 // a device error (in *err).
 static int time_gemv_choice(const GemvChoice& c, const uint32_t* signs, const uint16_t* scales, int64_t N,
-                            int64_t K, const uint16_t* x, int B, float* y, cudaStream_t ts, int num_sms,
+                            int64_t K, const void* x, bool xf, int B, float* y, cudaStream_t ts, int num_sms,
                             int smem_cap, bool static_weights, int reps, cudaEvent_t e0, cudaEvent_t e1, float* ms,
                             cudaError_t* err) {
   for (int i = 0; i < 3; ++i) {
-    if (run_gemv_choice(c, signs, scales, N, K, x, B, y, ts, num_sms, smem_cap, static_weights) != cudaSuccess) {
+    if (run_gemv_choice(c, signs, scales, N, K, x, xf, B, y, ts, num_sms, smem_cap, static_weights) != cudaSuccess) {
       cudaGetLastError();
       return 0;
     }
@@ -429,7 +439,7 @@ static int time_gemv_choice(const GemvChoice& c, const uint32_t* signs, const ui
   }
   cudaError_t le = cudaSuccess;
   for (int i = 0; i < reps && le == cudaSuccess; ++i)
-    le = run_gemv_choice(c, signs, scales, N, K, x, B, y, ts, num_sms, smem_cap, static_weights);
+    le = run_gemv_choice(c, signs, scales, N, K, x, xf, B, y, ts, num_sms, smem_cap, static_weights);
   const cudaError_t ce = cudaStreamEndCapture(ts, &g);
   cudaGraphExec_t ge = nullptr;
   const bool built = le == cudaSuccess && ce == cudaSuccess && g && cudaGraphInstantiate(&ge, g, 0) == cudaSuccess;
@@ -450,12 +460,13 @@ static int time_gemv_choice(const GemvChoice& c, const uint32_t* signs, const ui
 }
 
 cudaError_t launch_gemv(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t K,
-                        const uint16_t* x, int B, float* y, cudaStream_t stream, int num_sms,
+                        const void* x, bool xf, int B, float* y, cudaStream_t stream, int num_sms,
                         int smem_cap, bool static_weights) {
   if (const char* path = getenv("W1_GEMV_PATH")) {
-    const GemvChoice c{path[0] == 'd' ? 'd' : (path[0] == 't' ? 't' : 'm'), 0,
+    // fp32 activations run the direct kernel whatever the knob names.
+    const GemvChoice c{(path[0] == 'd' || xf) ? 'd' : (path[0] == 't' ? 't' : 'm'), 0,
                        strcmp(path, "direct16") == 0 ? 16 : 8};
-    return run_gemv_choice(c, signs, scales, N, K, x, B, y, stream, num_sms, smem_cap, static_weights);
+    return run_gemv_choice(c, signs, scales, N, K, x, xf, B, y, stream, num_sms, smem_cap, static_weights);
   }
   int dev = 0;
   cudaGetDevice(&dev);
@@ -463,8 +474,8 @@ cudaError_t launch_gemv(const uint32_t* signs, const uint16_t* scales, int64_t N
     std::lock_guard<std::mutex> lock(g_choice_mu);
     for (int i = 0; i < g_nchoice; ++i) {
       const GemvChoiceEntry& e = g_choice[i];
-      if (e.dev == dev && e.N == N && e.K == K && e.B == B && e.st == static_weights)
-        return run_gemv_choice(e.c, signs, scales, N, K, x, B, y, stream, num_sms, smem_cap, static_weights);
+      if (e.dev == dev && e.N == N && e.K == K && e.B == B && e.st == static_weights && e.xf == xf)
+        return run_gemv_choice(e.c, signs, scales, N, K, x, xf, B, y, stream, num_sms, smem_cap, static_weights);
     }
   }
   cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
@@ -474,7 +485,7 @@ cudaError_t launch_gemv(const uint32_t* signs, const uint16_t* scales, int64_t N
   }
   const char* at = getenv("W1_GEMV_AUTOTUNE");
   if (cap != cudaStreamCaptureStatusNone || (at && at[0] == '0'))
-    return run_gemv_rule(signs, scales, N, K, x, B, y, stream, num_sms, smem_cap, static_weights);
+    return run_gemv_rule(signs, scales, N, K, x, xf, B, y, stream, num_sms, smem_cap, static_weights);
 
   const GemvChoice cands[] = {{'d', 1, 8},  {'d', 2, 8},  {'d', 4, 8},  {'d', 8, 8}, {'d', 1, 16},
                               {'d', 2, 16}, {'d', 4, 16}, {'d', 8, 16}, {'t', 0, 0}, {'m', 0, 0}};
@@ -501,19 +512,20 @@ cudaError_t launch_gemv(const uint32_t* signs, const uint16_t* scales, int64_t N
   if (setup != cudaSuccess) {
     release();
     cudaGetLastError();
-    return run_gemv_rule(signs, scales, N, K, x, B, y, stream, num_sms, smem_cap, static_weights);
+    return run_gemv_rule(signs, scales, N, K, x, xf, B, y, stream, num_sms, smem_cap, static_weights);
   }
   // The candidates run on one weight matrix that stays in L2, which flatters
   // the kernels least sensitive to memory latency; the static rule's kernel
   // is kept unless another is more than 5% faster.
-  const char rule_kind = B <= 4 ? 'd' : 't';
+  const char rule_kind = (B <= 4 || xf) ? 'd' : 't';
   GemvChoice best{0, 0, 0}, best_rule{0, 0, 0};
   float best_ms = 0.f, best_rule_ms = 0.f;
   cudaError_t fatal = cudaSuccess;
   for (const GemvChoice& c : cands) {
     float ms = 0.f;
-    const int r = time_gemv_choice(c, signs, scales, N, K, x, B, y, ts, num_sms, smem_cap, static_weights, kTimed,
-                                   e0, e1, &ms, &fatal);
+    if (xf && c.kind != 'd') continue;
+    const int r = time_gemv_choice(c, signs, scales, N, K, x, xf, B, y, ts, num_sms, smem_cap, static_weights,
+                                   kTimed, e0, e1, &ms, &fatal);
     if (r < 0) break;  // a device error: report it, choose nothing
     if (r == 0) continue;
     if (getenv("W1_VERBOSE"))
@@ -534,7 +546,8 @@ cudaError_t launch_gemv(const uint32_t* signs, const uint16_t* scales, int64_t N
   }
   release();
   if (fatal != cudaSuccess) return fatal;
-  if (best.kind == 0) return run_gemv_rule(signs, scales, N, K, x, B, y, stream, num_sms, smem_cap, static_weights);
+  if (best.kind == 0)
+    return run_gemv_rule(signs, scales, N, K, x, xf, B, y, stream, num_sms, smem_cap, static_weights);
   if (getenv("W1_VERBOSE"))
     fprintf(stderr, "w1_gemv tuned: N=%lld K=%lld B=%d static=%d -> %c split=%d warps=%d (%.2f us)\n",
             static_cast<long long>(N), static_cast<long long>(K), B, static_weights ? 1 : 0, best.kind, best.s,
@@ -542,9 +555,9 @@ cudaError_t launch_gemv(const uint32_t* signs, const uint16_t* scales, int64_t N
   {
     std::lock_guard<std::mutex> lock(g_choice_mu);
     const int i = g_nchoice < 256 ? g_nchoice++ : static_cast<int>((N + K + B) & 255);
-    g_choice[i] = GemvChoiceEntry{dev, N, K, B, static_weights, best};
+    g_choice[i] = GemvChoiceEntry{dev, N, K, B, static_weights, xf, best};
   }
-  return run_gemv_choice(best, signs, scales, N, K, x, B, y, stream, num_sms, smem_cap, static_weights);
+  return run_gemv_choice(best, signs, scales, N, K, x, xf, B, y, stream, num_sms, smem_cap, static_weights);
 }
 
 // Name of the cached choice for a shape ("direct/2", "direct16/1", "tc/0",
@@ -558,7 +571,7 @@ static int gemv_choice_name(int64_t N, int64_t K, int B, bool st, char* out, siz
     std::lock_guard<std::mutex> lock(g_choice_mu);
     for (int i = 0; i < g_nchoice; ++i) {
       const GemvChoiceEntry& e = g_choice[i];
-      if (e.dev == dev && e.N == N && e.K == K && e.B == B && e.st == st) c = e.c;
+      if (e.dev == dev && e.N == N && e.K == K && e.B == B && e.st == st && !e.xf) c = e.c;
     }
   }
   const char* kind = c.kind == 'd' ? (c.w == 16 ? "direct16" : "direct")
@@ -599,13 +612,13 @@ static int gemv_set_choice(int64_t N, int64_t K, int B, bool st, const GemvChoic
   std::lock_guard<std::mutex> lock(g_choice_mu);
   for (int i = 0; i < g_nchoice; ++i) {
     GemvChoiceEntry& e = g_choice[i];
-    if (e.dev == dev && e.N == N && e.K == K && e.B == B && e.st == st) {
+    if (e.dev == dev && e.N == N && e.K == K && e.B == B && e.st == st && !e.xf) {
       e.c = c;
       return W1_OK;
     }
   }
   const int i = g_nchoice < 256 ? g_nchoice++ : static_cast<int>((N + K + B) & 255);
-  g_choice[i] = GemvChoiceEntry{dev, N, K, B, st, c};
+  g_choice[i] = GemvChoiceEntry{dev, N, K, B, st, false, c};
   return W1_OK;
 }
 

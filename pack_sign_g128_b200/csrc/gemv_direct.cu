@@ -851,16 +851,17 @@ static cudaError_t launch_gemv_direct_nw(const GdParams& p, int B, cudaStream_t 
   }
 }
 
+// x is bf16 [B][K], or fp32 [B][K] when x_f32.
 cudaError_t launch_gemv_direct(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t K,
-                               const uint16_t* x, int B, float* y, bool static_weights, cudaStream_t stream,
-                               int num_sms, int smem_cap, int force_s, int warps) {
+                               const void* x, bool x_f32, int B, float* y, bool static_weights,
+                               cudaStream_t stream, int num_sms, int smem_cap, int force_s, int warps) {
   if (N > (int64_t)1 << 30 || K > (int64_t)1 << 30) return cudaErrorNotSupported;
   GdParams p = {};
   p.signs = signs;
   p.scales = scales;
   p.x = x;
   p.y = y;
-  p.x_f32 = 0;
+  p.x_f32 = x_f32 ? 1 : 0;
   p.N = static_cast<int>(N);
   p.K = static_cast<int>(K);
   p.NG = static_cast<int>(K / 128);

@@ -11,3 +11,4 @@
 #include "dbf_ring.cu"
 #include "dbf.cu"
 #include "moe.cu"
+#include "okt.cu"

@@ -13,8 +13,11 @@ namespace w1 {
 cudaError_t launch_pack(const float* W, int64_t N, int64_t K, uint32_t* signs, uint16_t* scales,
                         cudaStream_t stream, int num_sms);
 cudaError_t launch_gemv(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t K,
-                        const uint16_t* x, int B, float* y, cudaStream_t stream, int num_sms,
+                        const void* x, bool xf, int B, float* y, cudaStream_t stream, int num_sms,
                         int smem_cap, bool static_weights);
+bool okt_shape_ok(int64_t n1, int64_t n2, int64_t K);
+cudaError_t launch_okt_rotate(const float* H, int n1, const float* R, int n2, const uint16_t* x, int B, float* out,
+                              bool early, cudaStream_t stream, int num_sms, int smem_optin);
 cudaError_t launch_gemm(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t K,
                         const uint16_t* x, int64_t M, float* y, void* workspace, cudaStream_t stream,
                         int num_sms);
@@ -123,7 +126,7 @@ int w1_gemv_ex(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t
   int st = device_info(&d);
   if (st != W1_OK) return st;
   const int cap = d.smem_optin < 110 * 1024 ? d.smem_optin : 110 * 1024;
-  return launch_result(launch_gemv(signs, scales, N, K, x, static_cast<int>(B), y,
+  return launch_result(launch_gemv(signs, scales, N, K, x, false, static_cast<int>(B), y,
                                    reinterpret_cast<cudaStream_t>(stream), d.sms, cap,
                                    (flags & W1_GEMV_STATIC_WEIGHTS) != 0));
 }
@@ -131,6 +134,44 @@ int w1_gemv_ex(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t
 int w1_gemv(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t K,
             const uint16_t* x, int64_t B, float* y, w1_stream_t stream) {
   return w1_gemv_ex(signs, scales, N, K, x, B, y, 0u, stream);
+}
+
+int w1_okt_rotate(const float* H, int64_t n1, const float* R, int64_t n2, const uint16_t* x, int64_t B,
+                  float* x_rot, w1_stream_t stream) {
+  if (!H || !R || !x || !x_rot) return W1_ERR_NULL;
+  if (B < 1 || B > 65535 || n1 < 1 || n2 < 1 || n1 > 1024 || n2 > 128) return W1_ERR_SHAPE;
+  if (!okt_shape_ok(n1, n2, n1 * n2) || ((n1 * n2) % 128) != 0) return W1_ERR_SHAPE;
+  if (!aligned16(H) || !aligned16(R) || !aligned16(x) || !aligned16(x_rot)) return W1_ERR_ALIGN;
+  DeviceInfo d;
+  int st = device_info(&d);
+  if (st != W1_OK) return st;
+  return launch_result(launch_okt_rotate(H, static_cast<int>(n1), R, static_cast<int>(n2), x, static_cast<int>(B),
+                                         x_rot, false, reinterpret_cast<cudaStream_t>(stream), d.sms,
+                                         d.smem_optin));
+}
+
+int w1_okt_gemv(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t K, const float* H, int64_t n1,
+                const float* R, int64_t n2, const uint16_t* x, int64_t B, float* x_rot, float* y, uint32_t flags,
+                w1_stream_t stream) {
+  if (!signs || !scales || !H || !R || !x || !x_rot || !y) return W1_ERR_NULL;
+  if (N <= 0 || K <= 0 || (K % 128) != 0 || B < 1 || B > 8) return W1_ERR_SHAPE;
+  if (N > ((int64_t)1 << 30) || n1 < 1 || n2 < 1 || n1 > 1024 || n2 > 128 || !okt_shape_ok(n1, n2, K))
+    return W1_ERR_SHAPE;
+  if ((flags & ~static_cast<uint32_t>(W1_GEMV_STATIC_WEIGHTS)) != 0) return W1_ERR_SHAPE;
+  if (!aligned16(signs) || !aligned16(scales) || !aligned16(H) || !aligned16(R) || !aligned16(x) ||
+      !aligned16(x_rot) || !aligned16(y))
+    return W1_ERR_ALIGN;
+  DeviceInfo d;
+  int st = device_info(&d);
+  if (st != W1_OK) return st;
+  const bool static_weights = (flags & W1_GEMV_STATIC_WEIGHTS) != 0;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  st = launch_result(launch_okt_rotate(H, static_cast<int>(n1), R, static_cast<int>(n2), x, static_cast<int>(B),
+                                       x_rot, static_weights, s, d.sms, d.smem_optin));
+  if (st != W1_OK) return st;
+  const int cap = d.smem_optin < 110 * 1024 ? d.smem_optin : 110 * 1024;
+  return launch_result(launch_gemv(signs, scales, N, K, x_rot, true, static_cast<int>(B), y, s, d.sms, cap,
+                                   static_weights));
 }
 
 int w1_gemm(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t K,

@@ -85,6 +85,45 @@ def w1_gemv(signs: torch.Tensor, scales: torch.Tensor, x: torch.Tensor, y: torch
     return y
 
 
+def w1_okt_rotate(H: torch.Tensor, R: torch.Tensor, x: torch.Tensor, x_rot: torch.Tensor | None = None,
+                  stream=None) -> torch.Tensor:
+    """x_rot [B, K] fp32 = (H kron R)^T x for every row of x [B, K] bf16.
+
+    H fp32 [n1, n1] and R fp32 [n2, n2] are orthogonal, n1 * n2 = K."""
+    n1, n2 = H.shape[0], R.shape[0]
+    B, K = x.shape
+    if x.dtype != torch.bfloat16 or H.dtype != torch.float32 or R.dtype != torch.float32:
+        raise TypeError("x must be bfloat16, H and R float32")
+    if x_rot is None:
+        x_rot = torch.empty((B, K), dtype=torch.float32, device=x.device)
+    st = _lib.fn("w1_okt_rotate")(_ptr(H), n1, _ptr(R), n2, _ptr(x), B, _ptr(x_rot), _stream(stream, x))
+    if st != _lib.W1_OK:
+        raise _lib.W1Error(st, "w1_okt_rotate")
+    return x_rot
+
+
+def w1_okt_gemv(signs: torch.Tensor, scales: torch.Tensor, H: torch.Tensor, R: torch.Tensor, x: torch.Tensor,
+                y: torch.Tensor | None = None, x_rot: torch.Tensor | None = None, stream=None,
+                static_weights: bool = False) -> torch.Tensor:
+    """y [B, N] fp32 = the 1-bit matrix (packed in rotated coordinates) times
+    (H kron R)^T x, x [B, K] bf16, B <= 8.  x_rot (fp32 [B, K]) receives the
+    rotated activations; allocated here when omitted."""
+    N, KW = signs.shape
+    B, K = x.shape
+    if x.dtype != torch.bfloat16 or H.dtype != torch.float32 or R.dtype != torch.float32:
+        raise TypeError("x must be bfloat16, H and R float32")
+    if y is None:
+        y = torch.empty((B, N), dtype=torch.float32, device=x.device)
+    if x_rot is None:
+        x_rot = torch.empty((B, K), dtype=torch.float32, device=x.device)
+    st = _lib.fn("w1_okt_gemv")(_ptr(signs), _ptr(scales), N, KW * 32, _ptr(H), H.shape[0], _ptr(R), R.shape[0],
+                                _ptr(x), B, _ptr(x_rot), _ptr(y),
+                                W1_GEMV_STATIC_WEIGHTS if static_weights else 0, _stream(stream, x))
+    if st != _lib.W1_OK:
+        raise _lib.W1Error(st, "w1_okt_gemv")
+    return y
+
+
 def gemm_workspace(M: int, K: int, device=None) -> torch.Tensor:
     """Workspace bytes for w1_gemm (fp16 copy of x, token scales)."""
     n = _lib.call("w1_gemm_workspace_size", M, K)

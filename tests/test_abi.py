@@ -105,3 +105,28 @@ def test_moe_host_side_argument_errors(lib):
     bad[0] = None
     assert lib.w1_moe_grouped(*bad, ws, n, None) == _lib.W1_ERR_NULL
     assert lib.w1_moe_grouped(*base, ctypes.c_void_p((1 << 30) + 256), n, None) == _lib.W1_ERR_ALIGN
+
+
+def test_okt_host_side_argument_errors(lib):
+    good = ctypes.c_void_p(1 << 20)
+    odd = ctypes.c_void_p((1 << 20) + 4)
+    rot = lib.w1_okt_rotate
+    assert rot(None, 64, good, 64, good, 1, good, None) == _lib.W1_ERR_NULL
+    assert rot(good, 64, good, 64, good, 1, None, None) == _lib.W1_ERR_NULL
+    assert rot(good, 64, good, 32, good, 1, good, None) != _lib.W1_ERR_NULL   # n1 n2 = 2048: a valid K
+    assert rot(good, 3, good, 10, good, 1, good, None) == _lib.W1_ERR_SHAPE    # K = 30, not a multiple of 128
+    assert rot(good, 16, good, 256, good, 1, good, None) == _lib.W1_ERR_SHAPE  # n2 > 128
+    assert rot(good, 2048, good, 1, good, 1, good, None) == _lib.W1_ERR_SHAPE  # n1 > 1024
+    assert rot(good, 1024, good, 128, good, 1, good, None) == _lib.W1_ERR_SHAPE  # K > 65536
+    assert rot(good, 0, good, 128, good, 1, good, None) == _lib.W1_ERR_SHAPE
+    assert rot(good, 64, good, 64, good, 0, good, None) == _lib.W1_ERR_SHAPE
+    assert rot(good, 64, good, 64, good, 65536, good, None) == _lib.W1_ERR_SHAPE
+    assert rot(odd, 64, good, 64, good, 1, good, None) == _lib.W1_ERR_ALIGN
+    assert rot(good, 64, good, 64, good, 1, odd, None) == _lib.W1_ERR_ALIGN
+    g = lib.w1_okt_gemv
+    assert g(good, good, 16, 4096, good, 64, good, 64, good, 1, None, good, 0, None) == _lib.W1_ERR_NULL
+    assert g(good, good, 16, 4096, good, 64, good, 32, good, 1, good, good, 0, None) == _lib.W1_ERR_SHAPE  # 64*32 != K
+    assert g(good, good, 16, 4096, good, 64, good, 64, good, 9, good, good, 0, None) == _lib.W1_ERR_SHAPE  # B > 8
+    assert g(good, good, 16, 4096, good, 64, good, 64, good, 1, good, good, 2, None) == _lib.W1_ERR_SHAPE  # flag
+    assert g(good, good, 0, 4096, good, 64, good, 64, good, 1, good, good, 0, None) == _lib.W1_ERR_SHAPE
+    assert g(good, good, 16, 4096, good, 64, good, 64, good, 1, good, odd, 0, None) == _lib.W1_ERR_ALIGN
