@@ -29,6 +29,10 @@ rational arithmetic:
 * Routed MoE -- every (token, slot) route carries an expert id and a route
   weight; gate/up consume the token's shared hidden state, down consumes the
   route's own intermediate (DBF post, section 4, MoE input topologies).
+* Approximation residuals -- E = W - W_approx; the relative Frobenius
+  residual ||E||_F / ||W||_F and the relative spectral residual
+  ||E||_2 / ||W||_2, spectral norms by power iteration (DBF post, section 8
+  "Current measurements").
 * Rotated activations -- one orthogonal rotation of the input space, factored
   as the Kronecker product of two small orthogonal matrices H and R; the
   weights are binarised in the rotated coordinates and the activations take
@@ -276,6 +280,56 @@ def dbf_dense_ref(a_bits, B1_words, mid_bits, B2_words, b_bits, m: int, r: int, 
     U = 1.0 - 2.0 * unpack_bits_lsb_first(B1_words, r).astype(np.float64)
     V = 1.0 - 2.0 * unpack_bits_lsb_first(B2_words, n).astype(np.float64)
     return (a[:, None] * U) @ (mid[:, None] * (V * b[None, :]))
+
+
+# ---------------------------------------------------------------------------
+# Matrix-approximation measurement (DBF post, section 8 "Current
+# measurements": relative Frobenius and spectral residuals, each matrix
+# normalised by its own norm, spectral norms by fixed-seed 32-iteration power
+# iteration).
+# ---------------------------------------------------------------------------
+
+
+def residual_g128_ref(W, signs, scale_bits) -> np.ndarray:
+    """E = W - w_hat in float64 for a matrix and its 1-bit group-128 packing."""
+    W = np.asarray(W, dtype=np.float64)
+    return W - dequant_ref(signs, scale_bits, W.shape[1])
+
+
+def dbf_residual_ref(W, a_bits, B1_words, mid_bits, B2_words, b_bits, m: int, r: int, n: int) -> np.ndarray:
+    """E = W - diag(a) U diag(mid) V diag(b) in float64."""
+    return np.asarray(W, dtype=np.float64) - dbf_dense_ref(a_bits, B1_words, mid_bits, B2_words, b_bits, m, r, n)
+
+
+def sum_squares_ref(A) -> float:
+    """sum of A^2, exactly rounded once (math.fsum over float64 squares; the
+    squares of float32 values are exact in float64)."""
+    A = np.asarray(A, dtype=np.float64).ravel()
+    return math.fsum((A * A).tolist())
+
+
+def power_iteration_ref(A, v0, iters: int) -> float:
+    """Spectral norm estimate of A [m, n] by power iteration on A^T A.
+
+    v = v0 / ||v0||; then `iters` times: u = A v, w = A^T u, v = w / ||w||;
+    the estimate is ||A v||.  If some w is zero (A v = 0), the estimate is 0.
+    The section names the method, the iteration count and a fixed seed; the
+    start vector is the caller's (drawn from the fixed seed), and this update
+    order is the plainest reading.
+    """
+    A = np.asarray(A, dtype=np.float64)
+    v = np.asarray(v0, dtype=np.float64).copy()
+    nv = np.linalg.norm(v)
+    if nv == 0.0:
+        return 0.0
+    v /= nv
+    for _ in range(iters):
+        w = A.T @ (A @ v)
+        nw = np.linalg.norm(w)
+        if nw == 0.0:
+            return 0.0
+        v = w / nw
+    return float(np.linalg.norm(A @ v))
 
 
 # ---------------------------------------------------------------------------

@@ -502,3 +502,79 @@ def test_okt_forward_equivalence():
     w_hat = O.dequant_ref(signs, scales, K)
     assert np.array_equal(x_rot, xr)
     assert np.max(np.abs(y - xr @ w_hat.T)) <= 1e-13 * np.max(bound)
+
+
+# ---------------------------------------------------------------- approximation residuals
+
+def test_g128_residual_energy_closed_form():
+    """Per group, with w_hat = s sign(w): sum (w - w_hat)^2 = sum w^2 - 2 s sum|w| + 128 s^2
+    (sign(w) w = |w| under the signbit convention)."""
+    W = synth.weights(synth.rng(61), 24, 512)
+    W[0, :128] = 0.0
+    W[1, 5] = -0.0
+    s, c = O.pack_ref(W)
+    E = O.residual_g128_ref(W, s, c)
+    sc = O.fp16_bits_to_f64(c)
+    Wd = W.astype(np.float64)
+    expect = 0.0
+    for n in range(W.shape[0]):
+        for g in range(W.shape[1] // 128):
+            grp = Wd[n, 128 * g:128 * (g + 1)]
+            expect += np.sum(grp * grp) - 2.0 * sc[n, g] * np.sum(np.abs(grp)) + 128.0 * sc[n, g] ** 2
+    assert O.sum_squares_ref(E) == pytest.approx(expect, rel=1e-12)
+
+
+def test_g128_relative_frobenius_of_gaussian_weights():
+    """Gaussian weights: the mean-|w| sign code keeps 2/pi of the energy, so the
+    relative Frobenius residual is close to sqrt(1 - 2/pi) = 0.6028 (slightly
+    below it: each group fits its own scale)."""
+    W = synth.weights(synth.rng(62), 256, 2048)
+    s, c = O.pack_ref_fast(W)
+    rel = math.sqrt(O.sum_squares_ref(O.residual_g128_ref(W, s, c)) / O.sum_squares_ref(W))
+    assert 0.59 < rel < math.sqrt(1.0 - 2.0 / math.pi) + 1e-3
+
+
+def test_dbf_residual_of_its_own_reconstruction_is_zero():
+    """W built element by element as sum_k a_i U_ik mid_k V_kj b_j (no matmul):
+    the residual against the chain's dense form is zero up to rounding."""
+    m, r, n = 16, 32, 64
+    a, B1, mid, B2, b, _ = synth.dbf_case(m=m, r=r, n=n, B=1, seed=63)
+    av, mv, bv = (np.array(v, np.uint16).view(np.float16).astype(float) for v in (a, mid, b))
+
+    def sgn(words, row, col):
+        return 1 - 2 * ((int(words[row, col // 32]) >> (col % 32)) & 1)
+
+    W = np.array([[av[i] * bv[j] * math.fsum(sgn(B1, i, k) * mv[k] * sgn(B2, k, j) for k in range(r))
+                   for j in range(n)] for i in range(m)])
+    E = O.dbf_residual_ref(W, a, B1, mid, B2, b, m, r, n)
+    assert np.max(np.abs(E)) <= 1e-14 * np.max(np.abs(W))
+
+
+def test_sum_squares_is_exact_on_integers():
+    A = np.arange(-300, 301, dtype=np.float32).reshape(1, -1)
+    assert O.sum_squares_ref(A) == 2 * sum(k * k for k in range(1, 301))
+
+
+def test_power_iteration_diagonal_and_rank_one():
+    d = np.array([0.5, -7.0, 3.0, 1.0])
+    assert O.power_iteration_ref(np.diag(d), np.ones(4), 32) == pytest.approx(7.0, rel=1e-12)
+    g = synth.rng(64)
+    x, y = g.standard_normal(30), g.standard_normal(20)
+    sigma = np.linalg.norm(x) * np.linalg.norm(y)
+    assert O.power_iteration_ref(np.outer(x, y), g.standard_normal(20), 1) == pytest.approx(sigma, rel=1e-12)
+    assert O.power_iteration_ref(np.zeros((5, 3)), np.ones(3), 32) == 0.0
+
+
+def test_power_iteration_against_svd():
+    """A planted gap (10 vs 5) converges to the largest singular value from the
+    library SVD within rounding; without a gap the estimate never exceeds it."""
+    g = synth.rng(65)
+    Q1 = np.linalg.qr(g.standard_normal((60, 60)))[0]
+    Q2 = np.linalg.qr(g.standard_normal((40, 40)))[0]
+    sv = np.concatenate([[10.0, 5.0], g.uniform(0.0, 4.0, 38)])
+    A = Q1[:, :40] @ np.diag(sv) @ Q2.T
+    assert O.power_iteration_ref(A, g.standard_normal(40), 32) == pytest.approx(np.linalg.norm(A, 2), rel=1e-12)
+    B = g.standard_normal((50, 70))
+    est = O.power_iteration_ref(B, g.standard_normal(70), 32)
+    assert est <= np.linalg.norm(B, 2) * (1 + 1e-12)
+    assert est >= 0.9 * np.linalg.norm(B, 2)
