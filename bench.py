@@ -563,6 +563,72 @@ def okt_rows(torch, ops, synth, combos, stream, reps: int = 3):
     return rows
 
 
+FP32_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12  # CUDA-core FMA: SMs x lanes x 2 flops x max clock
+
+
+def measure_rows(torch, ops, synth, peaks, iters: int = 5):
+    """Approximation residuals on the 4096 x 4096 matrices (each call timed as
+    one CUDA graph replay after an L2 flush): the sign-code
+    residual sums (GB/s of W and packed bytes read), the DBF
+    residual (fp32 TFLOP/s of the reconstruction, 2 m n r), 32-iteration
+    power iteration, and the relative Frobenius / spectral residuals of the
+    1-bit code on the synthetic Gaussian matrix."""
+    dev = torch.device("cuda")
+    m = n = r = 4096
+    W, _ = synth.gemv_case(m, n, 1)
+    Wd = torch.from_numpy(W).to(dev)
+    signs, scales = ops.w1_pack(Wd)
+    a, B1, mid, B2, b, _ = synth.dbf_case(m=m, r=r, n=n, B=1)
+    to16 = lambda v: torch.from_numpy(v.view(np.int16)).to(dev).view(torch.float16)
+    tow = lambda v: torch.from_numpy(v.view(np.int32)).to(dev)
+    dargs = (to16(a), tow(B1), to16(mid), tow(B2), to16(b))
+    ws = ops.measure_workspace(m, n)
+    E = torch.empty((m, n), dtype=torch.float32, device=dev)
+    v0 = torch.from_numpy(synth.start_vector(n)).to(dev)
+    flush = torch.empty(int(512 * 2 ** 20), dtype=torch.uint8, device=dev)
+
+    st = torch.cuda.Stream()
+
+    def timed(fn):
+        # one call captured as a CUDA graph, so host time does not enter the
+        # events; L2 flushed before each replay
+        with torch.cuda.stream(st):
+            fn()
+        st.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=st):
+            fn()
+        ts = []
+        for _ in range(iters):
+            with torch.cuda.stream(st):
+                flush.zero_()
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record(st)
+                g.replay()
+                e1.record(st)
+            st.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        return statistics.median(ts)
+
+    res_ms = timed(lambda: ops.w1_residual(Wd, signs, scales, want_E=False, workspace=ws))
+    res_bytes = m * n * 4 + packed_bytes(m, n)
+    dbf_ms = timed(lambda: ops.dbf_residual(Wd, *dargs, want_E=False, workspace=ws))
+    dbf_tf = 2.0 * m * n * r / (dbf_ms * 1e-3) / 1e12
+    pi_ms = timed(lambda: ops.w1_power_iteration(Wd, v0, 32, workspace=ws))
+    ops.w1_residual(Wd, signs, scales, E=E, workspace=ws)
+    _, sums = ops.w1_residual(Wd, signs, scales, want_E=False, workspace=ws)
+    se, sw = (float(v) for v in sums.cpu())
+    rel_spec = float(ops.w1_power_iteration(E, v0, 32, workspace=ws)) / float(ops.w1_power_iteration(Wd, v0, 32, workspace=ws))
+    torch.cuda.synchronize()
+    return {"residual_g128": {"ms": round(res_ms, 4), "GB/s": round(res_bytes / (res_ms * 1e-3) / 1e9, 1),
+                              "frac_hbm": round(res_bytes / (res_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)},
+            "dbf_residual": {"ms": round(dbf_ms, 4), "fp32_TFLOP/s": round(dbf_tf, 1),
+                             "frac_fp32_cuda_core": round(dbf_tf / FP32_PEAK_TFLOPS, 4)},
+            "power_iteration_32": {"ms": round(pi_ms, 4), "launches": 3 * 32 + 3},
+            "g128_gaussian_4096": {"rel_frobenius": round((se / sw) ** 0.5, 5), "rel_spectral": round(rel_spec, 5)}}
+
+
 def cpu_oracle_gemv_sample(combos_spec, packed_host, max_seconds: float = 20.0):
     """Time the fp64 oracle on the sweep (one launch per pair) on the host."""
     from oracle import w1_oracle as O
@@ -637,6 +703,8 @@ def run_gpu(args):
             rows["dbf"] = dbf_rows(torch, ops, synth, peaks, l2)
         elif args.section == "gemv1":
             rows["gemv1"] = gemv_one(torch, ops, synth, args.shape)
+        elif args.section == "measure":
+            rows["measure"] = measure_rows(torch, ops, synth, peaks)
         elif args.section == "okt":
             combos, stream = build_gemv_sweep(torch, ops, synth, l2)
             rows["okt"] = okt_rows(torch, ops, synth, combos, stream)
@@ -690,6 +758,7 @@ def run_gpu(args):
         rows["moe"] = moe_rows(torch, ops, synth, peaks)
         rows["dbf"] = dbf_rows(torch, ops, synth, peaks, l2)
         rows["okt"] = okt_rows(torch, ops, synth, combos, stream)
+        rows["measure"] = measure_rows(torch, ops, synth, peaks)
     cpu = None
     if rank == 0 and world == 1 and not args.skip_cpu:
         packed_host = {}
@@ -815,7 +884,7 @@ def main():
                     help="N,K,B of the single GEMV that --section gemv1 launches (for ncu captures)")
     ap.add_argument("--choices", default=None,
                     help="JSON line of an earlier run: pin each GEMV pair to the kernel it chose (profiling)")
-    ap.add_argument("--section", default="all", choices=["all", "gemm", "moe", "dbf", "gemv1", "okt"],
+    ap.add_argument("--section", default="all", choices=["all", "gemm", "moe", "dbf", "gemv1", "okt", "measure"],
                     help="run one row only (for profiling); prints a rows-only JSON line")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -186,6 +186,62 @@ int w1_okt_gemv(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_
                 w1_stream_t stream);
 
 /*
+ * Approximation residuals ("LLM binarization episode 01: DBF", section 8
+ * "Current measurements": the relative Frobenius residual ||E||_F / ||W||_F
+ * and the relative spectral residual ||E||_2 / ||W||_2 of E = W - W_approx,
+ * each matrix normalised by its own norm, spectral norms by fixed-seed
+ * 32-iteration power iteration).  Measurement calls, not part of a product.
+ * Every sum below has a fixed order (a per-CTA tree, then the CTAs in index
+ * order), so results are bitwise reproducible for a shape on a device.
+ *
+ * w1_measure_workspace_size -- bytes of device workspace that w1_residual,
+ * dbf_residual and w1_power_iteration need for an m x n matrix (0 for
+ * invalid sizes).  One workspace serves all three calls, one at a time per
+ * stream.
+ */
+size_t w1_measure_workspace_size(int64_t m, int64_t n);
+
+/*
+ * w1_residual -- E = W - w_hat for a matrix and its group-128 sign code
+ * (w_hat as in w1_gemv), and sums[0] = sum E^2, sums[1] = sum W^2.
+ *   W fp32 [N][K]; signs [N][K/32], scales [N][K/128] (device, read only).
+ *   E fp32 [N][K] out (each element w - w_hat rounded once to fp32), or NULL.
+ *   sums: device double[2] out; each square is taken of the fp32 values in
+ *   fp64.
+ *   workspace: device, >= w1_measure_workspace_size(N, K) bytes, else
+ *   W1_ERR_WORKSPACE.
+ */
+int w1_residual(const float* W, int64_t N, int64_t K, const uint32_t* signs, const uint16_t* scales, float* E,
+                double* sums, void* workspace, size_t ws_bytes, w1_stream_t stream);
+
+/*
+ * dbf_residual -- the same for a DBF matrix W_approx = diag(a) U diag(mid)
+ * V diag(b) (dbf_apply's operands; m, r, n multiples of 128 and
+ * (m/128)(n/128) <= 8192, else W1_ERR_SHAPE).
+ *   W_approx[i][j] = (acc_ij * a_i) * b_j in fp32, where acc_ij is the sum
+ *   over k ascending of U_ik * (mid_k V_kj) in fp32; so
+ *   |W_approx - exact| <= (r + 2) * 2^-24 * |a_i| |b_j| sum_k |mid_k|.
+ *   E fp32 [m][n] out (or NULL), sums as for w1_residual.  W_approx is never
+ *   stored.
+ */
+int dbf_residual(const float* W, const uint16_t* a, const uint32_t* B1, const uint16_t* mid, const uint32_t* B2,
+                 const uint16_t* b, int64_t m, int64_t r, int64_t n, float* E, double* sums, void* workspace,
+                 size_t ws_bytes, w1_stream_t stream);
+
+/*
+ * w1_power_iteration -- spectral norm estimate of A (fp32 [m][n], n a
+ * multiple of 4) by power iteration on A^T A from the start vector v0 (fp32
+ * [n]; the fixed-seed draw is the caller's):
+ *   v = v0 / ||v0||; `iters` times: u = A v, w = A^T u, v = w / ||w||;
+ *   *sigma = ||A v|| (device double).  A zero vector along the way gives 0.
+ * All vectors and sums are fp64; A is read as given.  The relative spectral
+ * residual is this on E (from w1_residual / dbf_residual) divided by this
+ * on W.
+ */
+int w1_power_iteration(const float* A, int64_t m, int64_t n, const float* v0, int64_t iters, double* sigma,
+                       void* workspace, size_t ws_bytes, w1_stream_t stream);
+
+/*
  * w1_gemm -- prefill-regime product for many token rows (DBF post, section 4:
  * prompt processing amortises weight loads across columns).
  *   y[m][n] = sum_g s[n][g] * sum_{k in g} (1 - 2*bit[n][k]) * x[m][k].

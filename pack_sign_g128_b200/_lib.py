@@ -42,6 +42,10 @@ SIGNATURES = {
     "dbf_workspace_size": (_sz, [_i64, _i64, _i64, _i64]),
     "dbf_apply_noalloc": (_int, [_p, _p, _p, _p, _p, _i64, _i64, _i64, _p, _i64, _p, _p]),
     "w1_okt_rotate": (_int, [_p, _i64, _p, _i64, _p, _i64, _p, _p]),
+    "w1_measure_workspace_size": (_sz, [_i64, _i64]),
+    "w1_residual": (_int, [_p, _i64, _i64, _p, _p, _p, _p, _p, _sz, _p]),
+    "dbf_residual": (_int, [_p, _p, _p, _p, _p, _p, _i64, _i64, _i64, _p, _p, _p, _sz, _p]),
+    "w1_power_iteration": (_int, [_p, _i64, _i64, _p, _i64, _p, _p, _sz, _p]),
     "w1_okt_gemv": (_int, [_p, _p, _i64, _i64, _p, _i64, _p, _i64, _p, _i64, _p, _p, ctypes.c_uint32, _p]),
 }
 

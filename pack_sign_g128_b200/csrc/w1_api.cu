@@ -16,6 +16,14 @@ cudaError_t launch_gemv(const uint32_t* signs, const uint16_t* scales, int64_t N
                         const void* x, bool xf, int B, float* y, cudaStream_t stream, int num_sms,
                         int smem_cap, bool static_weights);
 bool okt_shape_ok(int64_t n1, int64_t n2, int64_t K);
+size_t measure_workspace_bytes(int64_t m, int64_t n);
+cudaError_t launch_residual_g128(const float* W, int64_t N, int64_t K, const uint32_t* signs, const uint16_t* scales,
+                                 float* E, double* sums, void* workspace, cudaStream_t stream, int num_sms);
+cudaError_t launch_dbf_residual(const float* W, const uint16_t* a, const uint32_t* B1, const uint16_t* mid,
+                                const uint32_t* B2, const uint16_t* b, int64_t m, int64_t r, int64_t n, float* E,
+                                double* sums, void* workspace, cudaStream_t stream);
+cudaError_t launch_power_iteration(const float* A, int64_t m, int64_t n, const float* v0, int64_t iters,
+                                   double* sigma, void* workspace, cudaStream_t stream, int num_sms);
 cudaError_t launch_okt_rotate(const float* H, int n1, const float* R, int n2, const uint16_t* x, int B, float* out,
                               bool early, cudaStream_t stream, int num_sms, int smem_optin);
 cudaError_t launch_gemm(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t K,
@@ -134,6 +142,61 @@ int w1_gemv_ex(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t
 int w1_gemv(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t K,
             const uint16_t* x, int64_t B, float* y, w1_stream_t stream) {
   return w1_gemv_ex(signs, scales, N, K, x, B, y, 0u, stream);
+}
+
+size_t w1_measure_workspace_size(int64_t m, int64_t n) {
+  if (m <= 0 || n <= 0 || m > ((int64_t)1 << 31) - 1 || n > ((int64_t)1 << 31) - 1) return 0;
+  return measure_workspace_bytes(m, n);
+}
+
+static inline bool aligned8(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 7u) == 0; }
+
+int w1_residual(const float* W, int64_t N, int64_t K, const uint32_t* signs, const uint16_t* scales, float* E,
+                double* sums, void* workspace, size_t ws_bytes, w1_stream_t stream) {
+  if (!W || !signs || !scales || !sums) return W1_ERR_NULL;
+  if (N <= 0 || K <= 0 || (K % 128) != 0 || N > ((int64_t)1 << 31) - 1 || K > ((int64_t)1 << 30))
+    return W1_ERR_SHAPE;
+  if (!workspace || ws_bytes < measure_workspace_bytes(N, K)) return W1_ERR_WORKSPACE;
+  if (!aligned16(W) || !aligned16(signs) || !aligned16(scales) || (E && !aligned16(E)) || !aligned16(workspace) ||
+      !aligned8(sums))
+    return W1_ERR_ALIGN;
+  DeviceInfo d;
+  int st = device_info(&d);
+  if (st != W1_OK) return st;
+  return launch_result(launch_residual_g128(W, N, K, signs, scales, E, sums, workspace,
+                                            reinterpret_cast<cudaStream_t>(stream), d.sms));
+}
+
+int dbf_residual(const float* W, const uint16_t* a, const uint32_t* B1, const uint16_t* mid, const uint32_t* B2,
+                 const uint16_t* b, int64_t m, int64_t r, int64_t n, float* E, double* sums, void* workspace,
+                 size_t ws_bytes, w1_stream_t stream) {
+  if (!W || !a || !B1 || !mid || !B2 || !b || !sums) return W1_ERR_NULL;
+  if (m <= 0 || r <= 0 || n <= 0 || (m % 128) != 0 || (r % 128) != 0 || (n % 128) != 0) return W1_ERR_SHAPE;
+  if ((m / 128) * (n / 128) > 8192 || r > ((int64_t)1 << 24)) return W1_ERR_SHAPE;
+  if (!workspace || ws_bytes < measure_workspace_bytes(m, n)) return W1_ERR_WORKSPACE;
+  if (!aligned16(W) || !aligned16(a) || !aligned16(B1) || !aligned16(mid) || !aligned16(B2) || !aligned16(b) ||
+      (E && !aligned16(E)) || !aligned16(workspace) || !aligned8(sums))
+    return W1_ERR_ALIGN;
+  DeviceInfo d;
+  int st = device_info(&d);
+  if (st != W1_OK) return st;
+  return launch_result(launch_dbf_residual(W, a, B1, mid, B2, b, m, r, n, E, sums, workspace,
+                                           reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int w1_power_iteration(const float* A, int64_t m, int64_t n, const float* v0, int64_t iters, double* sigma,
+                       void* workspace, size_t ws_bytes, w1_stream_t stream) {
+  if (!A || !v0 || !sigma) return W1_ERR_NULL;
+  if (m <= 0 || n <= 0 || (n % 4) != 0 || m > ((int64_t)1 << 31) - 1 || n > ((int64_t)1 << 28) || iters < 0 ||
+      iters > 100000)
+    return W1_ERR_SHAPE;
+  if (!workspace || ws_bytes < measure_workspace_bytes(m, n)) return W1_ERR_WORKSPACE;
+  if (!aligned16(A) || !aligned16(v0) || !aligned16(workspace) || !aligned8(sigma)) return W1_ERR_ALIGN;
+  DeviceInfo d;
+  int st = device_info(&d);
+  if (st != W1_OK) return st;
+  return launch_result(launch_power_iteration(A, m, n, v0, iters, sigma, workspace,
+                                              reinterpret_cast<cudaStream_t>(stream), d.sms));
 }
 
 int w1_okt_rotate(const float* H, int64_t n1, const float* R, int64_t n2, const uint16_t* x, int64_t B,

@@ -124,6 +124,69 @@ def w1_okt_gemv(signs: torch.Tensor, scales: torch.Tensor, H: torch.Tensor, R: t
     return y
 
 
+def measure_workspace(m: int, n: int, device=None) -> torch.Tensor:
+    """Workspace for w1_residual / dbf_residual / w1_power_iteration on m x n."""
+    nbytes = _lib.call("w1_measure_workspace_size", m, n)
+    if nbytes == 0:
+        raise ValueError("invalid measurement sizes")
+    return torch.empty(nbytes, dtype=torch.uint8, device=device or "cuda")
+
+
+def w1_residual(W: torch.Tensor, signs: torch.Tensor, scales: torch.Tensor, E: torch.Tensor | None = None,
+                want_E: bool = True, workspace: torch.Tensor | None = None, stream=None):
+    """(E fp32 [N, K] or None, sums fp64 [2] = (sum E^2, sum W^2)) for W and its packing."""
+    N, K = W.shape
+    if W.dtype != torch.float32:
+        raise TypeError("W must be float32")
+    if want_E and E is None:
+        E = torch.empty((N, K), dtype=torch.float32, device=W.device)
+    sums = torch.empty(2, dtype=torch.float64, device=W.device)
+    if workspace is None:
+        workspace = measure_workspace(N, K, W.device)
+    st = _lib.fn("w1_residual")(_ptr(W), N, K, _ptr(signs), _ptr(scales), _ptr(E) if want_E else None, _ptr(sums),
+                                _ptr(workspace), workspace.numel(), _stream(stream, W))
+    if st != _lib.W1_OK:
+        raise _lib.W1Error(st, "w1_residual")
+    return (E if want_E else None), sums
+
+
+def dbf_residual(W: torch.Tensor, a: torch.Tensor, B1: torch.Tensor, mid: torch.Tensor, B2: torch.Tensor,
+                 b: torch.Tensor, E: torch.Tensor | None = None, want_E: bool = True,
+                 workspace: torch.Tensor | None = None, stream=None):
+    """(E fp32 [m, n] or None, sums fp64 [2]) for W against diag(a) U diag(mid) V diag(b)."""
+    m, n = W.shape
+    r = mid.shape[0]
+    if W.dtype != torch.float32:
+        raise TypeError("W must be float32")
+    if want_E and E is None:
+        E = torch.empty((m, n), dtype=torch.float32, device=W.device)
+    sums = torch.empty(2, dtype=torch.float64, device=W.device)
+    if workspace is None:
+        workspace = measure_workspace(m, n, W.device)
+    st = _lib.fn("dbf_residual")(_ptr(W), _ptr(a), _ptr(B1), _ptr(mid), _ptr(B2), _ptr(b), m, r, n,
+                                 _ptr(E) if want_E else None, _ptr(sums), _ptr(workspace), workspace.numel(),
+                                 _stream(stream, W))
+    if st != _lib.W1_OK:
+        raise _lib.W1Error(st, "dbf_residual")
+    return (E if want_E else None), sums
+
+
+def w1_power_iteration(A: torch.Tensor, v0: torch.Tensor, iters: int = 32, workspace: torch.Tensor | None = None,
+                       stream=None) -> torch.Tensor:
+    """Spectral norm estimate of A fp32 [m, n] (fp64 scalar tensor on the device)."""
+    m, n = A.shape
+    if A.dtype != torch.float32 or v0.dtype != torch.float32:
+        raise TypeError("A and v0 must be float32")
+    sigma = torch.empty((), dtype=torch.float64, device=A.device)
+    if workspace is None:
+        workspace = measure_workspace(m, n, A.device)
+    st = _lib.fn("w1_power_iteration")(_ptr(A), m, n, _ptr(v0), iters, _ptr(sigma), _ptr(workspace),
+                                       workspace.numel(), _stream(stream, A))
+    if st != _lib.W1_OK:
+        raise _lib.W1Error(st, "w1_power_iteration")
+    return sigma
+
+
 def gemm_workspace(M: int, K: int, device=None) -> torch.Tensor:
     """Workspace bytes for w1_gemm (fp16 copy of x, token scales)."""
     n = _lib.call("w1_gemm_workspace_size", M, K)

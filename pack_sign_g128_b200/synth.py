@@ -19,12 +19,13 @@ Recipes (the pages' workloads stand in by shape; no model or dataset):
           weights as stored after the rotation, N x K ~ N(0, 0.02) (an
           orthogonal rotation of i.i.d. Gaussian rows is again i.i.d.
           Gaussian, so these stand for W (H kron R)); x B x K bf16 ~ N(0, 1)
+  power   seed 6: power-iteration start vectors, fp32 ~ N(0, 1)
 """
 from __future__ import annotations
 
 import numpy as np
 
-SEEDS = {"tiny": 0, "gemv": 1, "gemm": 2, "moe": 3, "dbf": 4, "okt": 5}
+SEEDS = {"tiny": 0, "gemv": 1, "gemm": 2, "moe": 3, "dbf": 4, "okt": 5, "power": 6}
 
 
 def rng(seed: int) -> np.random.Generator:
@@ -121,3 +122,8 @@ def okt_case(N: int, K: int, n1: int, n2: int, B: int, seed: int = SEEDS["okt"])
     H = orthogonal_f32(g, n1)
     R = orthogonal_f32(g, n2)
     return H, R, weights(g, N, K), activations_bf16(g, B, K)
+
+
+def start_vector(n: int, seed: int = SEEDS["power"]) -> np.ndarray:
+    """The fixed-seed start vector of a power iteration, fp32 [n] ~ N(0, 1)."""
+    return normal_f32(rng(seed), (n,))

@@ -130,3 +130,32 @@ def test_okt_host_side_argument_errors(lib):
     assert g(good, good, 16, 4096, good, 64, good, 64, good, 1, good, good, 2, None) == _lib.W1_ERR_SHAPE  # flag
     assert g(good, good, 0, 4096, good, 64, good, 64, good, 1, good, good, 0, None) == _lib.W1_ERR_SHAPE
     assert g(good, good, 16, 4096, good, 64, good, 64, good, 1, good, odd, 0, None) == _lib.W1_ERR_ALIGN
+
+
+def test_measure_host_side_argument_errors(lib):
+    good = ctypes.c_void_p(1 << 20)
+    odd = ctypes.c_void_p((1 << 20) + 4)
+    ws = lib.w1_measure_workspace_size(256, 512)
+    assert ws > 0 and lib.w1_measure_workspace_size(0, 512) == 0
+    assert lib.w1_measure_workspace_size(4096, 4096) >= 8 * (4096 + 65 * 4096)
+    res = lib.w1_residual
+    assert res(None, 256, 512, good, good, None, good, good, ws, None) == _lib.W1_ERR_NULL
+    assert res(good, 256, 500, good, good, None, good, good, ws, None) == _lib.W1_ERR_SHAPE
+    assert res(good, 0, 512, good, good, None, good, good, ws, None) == _lib.W1_ERR_SHAPE
+    assert res(good, 256, 512, good, good, None, good, None, ws, None) == _lib.W1_ERR_WORKSPACE
+    assert res(good, 256, 512, good, good, None, good, good, ws - 1, None) == _lib.W1_ERR_WORKSPACE
+    assert res(good, 256, 512, good, good, odd, good, good, ws, None) == _lib.W1_ERR_ALIGN
+    d = lib.dbf_residual
+    wsd = lib.w1_measure_workspace_size(256, 384)
+    args = [good] * 6
+    assert d(None, *args[1:], 256, 128, 384, None, good, good, wsd, None) == _lib.W1_ERR_NULL
+    assert d(*args, 256, 100, 384, None, good, good, wsd, None) == _lib.W1_ERR_SHAPE
+    assert d(*args, 256 * 128, 128, 256 * 128, None, good, good, 1 << 40, None) == _lib.W1_ERR_SHAPE  # too many tiles
+    assert d(*args, 256, 128, 384, None, good, good, wsd - 8, None) == _lib.W1_ERR_WORKSPACE
+    assert d(*args, 256, 128, 384, None, odd, good, wsd, None) == _lib.W1_ERR_ALIGN  # sums not 8-aligned
+    pi = lib.w1_power_iteration
+    assert pi(None, 64, 64, good, 32, good, good, ws, None) == _lib.W1_ERR_NULL
+    assert pi(good, 64, 66, good, 32, good, good, ws, None) == _lib.W1_ERR_SHAPE
+    assert pi(good, 64, 64, good, -1, good, good, ws, None) == _lib.W1_ERR_SHAPE
+    assert pi(good, 64, 64, good, 32, good, None, ws, None) == _lib.W1_ERR_WORKSPACE
+    assert pi(odd, 64, 64, good, 32, good, good, ws, None) == _lib.W1_ERR_ALIGN
