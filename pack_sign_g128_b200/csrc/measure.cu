@@ -17,7 +17,8 @@
 //
 // Every sum has a fixed order: a CTA reduces its threads through a fixed
 // shuffle tree and then its warps in order; the last CTA to finish (a ticket
-// counter) adds the per-CTA partials in CTA order.  Results are bitwise
+// counter) adds the per-CTA partials the same way, thread t taking partials
+// t, t + 256, ... in order.  Results are bitwise
 // reproducible for a given shape and device.
 #include <algorithm>
 #include <cstdint>
@@ -52,7 +53,8 @@ __device__ __forceinline__ double meas_block_sum(double v, double* red) {
 }
 
 // Per-CTA partial pair -> partials[cta] (cta = linear CTA index of ncta); the
-// last CTA to finish adds all partials in CTA order into out[0..1].
+// last CTA to finish adds all partials into out[0..1]: thread t takes
+// partials t, t + kThreads, ... in order, then the fixed tree.
 __device__ __forceinline__ void meas_finish_pair(double e2, double w2, double* partials, unsigned int* ticket,
                                                  double* out) {
   const unsigned int cta = blockIdx.y * gridDim.x + blockIdx.x;
@@ -68,15 +70,19 @@ __device__ __forceinline__ void meas_finish_pair(double e2, double w2, double* p
     last = atomicAdd(ticket, 1u) == ncta - 1;
   }
   __syncthreads();
-  if (last && threadIdx.x == 0) {
+  if (last) {  // uniform across the CTA
     __threadfence();
     double se = 0.0, sw = 0.0;
-    for (unsigned int c = 0; c < ncta; ++c) {
+    for (unsigned int c = threadIdx.x; c < ncta; c += meas::kThreads) {
       se += __ldcg(partials + 2 * c);
       sw += __ldcg(partials + 2 * c + 1);
     }
-    out[0] = se;
-    out[1] = sw;
+    se = meas_block_sum(se, red);
+    sw = meas_block_sum(sw, red);
+    if (threadIdx.x == 0) {
+      out[0] = se;
+      out[1] = sw;
+    }
   }
 }
 
