@@ -85,6 +85,13 @@ def w1_gemv(signs: torch.Tensor, scales: torch.Tensor, x: torch.Tensor, y: torch
     return y
 
 
+def _check_kron(H: torch.Tensor, R: torch.Tensor, K: int) -> None:
+    if H.dim() != 2 or H.shape[0] != H.shape[1] or R.dim() != 2 or R.shape[0] != R.shape[1]:
+        raise ValueError("H and R must be square matrices")
+    if H.shape[0] * R.shape[0] != K:
+        raise ValueError(f"n1 * n2 = {H.shape[0]} * {R.shape[0]} is not K = {K}")
+
+
 def w1_okt_rotate(H: torch.Tensor, R: torch.Tensor, x: torch.Tensor, x_rot: torch.Tensor | None = None,
                   stream=None) -> torch.Tensor:
     """x_rot [B, K] fp32 = (H kron R)^T x for every row of x [B, K] bf16.
@@ -94,6 +101,7 @@ def w1_okt_rotate(H: torch.Tensor, R: torch.Tensor, x: torch.Tensor, x_rot: torc
     B, K = x.shape
     if x.dtype != torch.bfloat16 or H.dtype != torch.float32 or R.dtype != torch.float32:
         raise TypeError("x must be bfloat16, H and R float32")
+    _check_kron(H, R, K)
     if x_rot is None:
         x_rot = torch.empty((B, K), dtype=torch.float32, device=x.device)
     st = _lib.fn("w1_okt_rotate")(_ptr(H), n1, _ptr(R), n2, _ptr(x), B, _ptr(x_rot), _stream(stream, x))
@@ -112,6 +120,9 @@ def w1_okt_gemv(signs: torch.Tensor, scales: torch.Tensor, H: torch.Tensor, R: t
     B, K = x.shape
     if x.dtype != torch.bfloat16 or H.dtype != torch.float32 or R.dtype != torch.float32:
         raise TypeError("x must be bfloat16, H and R float32")
+    if KW * 32 != K:
+        raise ValueError(f"x has K = {K} columns, the packed weights {KW * 32}")
+    _check_kron(H, R, K)
     if y is None:
         y = torch.empty((B, N), dtype=torch.float32, device=x.device)
     if x_rot is None:
@@ -138,6 +149,8 @@ def w1_residual(W: torch.Tensor, signs: torch.Tensor, scales: torch.Tensor, E: t
     N, K = W.shape
     if W.dtype != torch.float32:
         raise TypeError("W must be float32")
+    if tuple(signs.shape) != (N, K // 32) or tuple(scales.shape) != (N, K // 128):
+        raise ValueError("signs / scales do not match W's shape")
     if want_E and E is None:
         E = torch.empty((N, K), dtype=torch.float32, device=W.device)
     sums = torch.empty(2, dtype=torch.float64, device=W.device)
@@ -158,6 +171,9 @@ def dbf_residual(W: torch.Tensor, a: torch.Tensor, B1: torch.Tensor, mid: torch.
     r = mid.shape[0]
     if W.dtype != torch.float32:
         raise TypeError("W must be float32")
+    if (a.shape[0] != m or b.shape[0] != n or tuple(B1.shape) != (m, r // 32)
+            or tuple(B2.shape) != (r, n // 32)):
+        raise ValueError("DBF operands do not match W's shape")
     if want_E and E is None:
         E = torch.empty((m, n), dtype=torch.float32, device=W.device)
     sums = torch.empty(2, dtype=torch.float64, device=W.device)
@@ -177,6 +193,8 @@ def w1_power_iteration(A: torch.Tensor, v0: torch.Tensor, iters: int = 32, works
     m, n = A.shape
     if A.dtype != torch.float32 or v0.dtype != torch.float32:
         raise TypeError("A and v0 must be float32")
+    if v0.numel() != n:
+        raise ValueError(f"v0 has {v0.numel()} entries, A has {n} columns")
     sigma = torch.empty((), dtype=torch.float64, device=A.device)
     if workspace is None:
         workspace = measure_workspace(m, n, A.device)

@@ -159,3 +159,29 @@ def test_measure_host_side_argument_errors(lib):
     assert pi(good, 64, 64, good, -1, good, good, ws, None) == _lib.W1_ERR_SHAPE
     assert pi(good, 64, 64, good, 32, good, None, ws, None) == _lib.W1_ERR_WORKSPACE
     assert pi(odd, 64, 64, good, 32, good, good, ws, None) == _lib.W1_ERR_ALIGN
+
+
+def test_binding_shape_checks_run_before_any_device_work():
+    """The torch binding rejects mismatched shapes before marshalling pointers
+    (CPU tensors: the shape error must come first, not the CUDA-tensor check)."""
+    import torch
+    from pack_sign_g128_b200 import ops
+    x = torch.zeros((1, 4096), dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="is not K"):
+        ops.w1_okt_rotate(torch.zeros((64, 64)), torch.zeros((32, 32)), x)
+    with pytest.raises(ValueError, match="square"):
+        ops.w1_okt_rotate(torch.zeros((64, 32)), torch.zeros((64, 64)), x)
+    signs = torch.zeros((16, 64), dtype=torch.int32)
+    scales = torch.zeros((16, 16), dtype=torch.float16)
+    with pytest.raises(ValueError, match="columns, the packed weights"):
+        ops.w1_okt_gemv(signs, scales, torch.zeros((64, 64)), torch.zeros((64, 64)), x)
+    with pytest.raises(ValueError, match="do not match"):
+        ops.w1_residual(torch.zeros((16, 4096)), signs, scales)
+    with pytest.raises(ValueError, match="entries"):
+        ops.w1_power_iteration(torch.zeros((8, 16)), torch.zeros(12))
+    h16 = lambda k: torch.zeros(k, dtype=torch.float16)
+    w = lambda r, c: torch.zeros((r, c), dtype=torch.int32)
+    with pytest.raises(ValueError, match="DBF operands"):
+        ops.dbf_residual(torch.zeros((128, 256)), h16(128), w(128, 4), h16(128), w(128, 4), h16(256))
+    with pytest.raises(ValueError, match="CUDA"):  # well-formed CPU tensors reach the device check
+        ops.w1_power_iteration(torch.zeros((8, 16)), torch.zeros(16))
