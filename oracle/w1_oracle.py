@@ -301,6 +301,37 @@ def dbf_residual_ref(W, a_bits, B1_words, mid_bits, B2_words, b_bits, m: int, r:
     return np.asarray(W, dtype=np.float64) - dbf_dense_ref(a_bits, B1_words, mid_bits, B2_words, b_bits, m, r, n)
 
 
+def dbf_reproject_mid_ref(W, a_bits, B1_words, B2_words, b_bits, m: int, r: int, n: int):
+    """Least-squares middle diagonal for fixed signs and outer scalers.
+
+    DBF post, section 1.2: one final linear least-squares reprojection of the
+    middle diagonal, with U, V, a and b held fixed.  W_approx(mid) =
+    sum_k mid_k P_k with P_k = (a * U[:, k]) (V[k, :] * b)^T is linear in mid, so
+    the minimiser of ||W - W_approx(mid)||_F solves the normal equations
+    G mid = c with G_kl = <P_k, P_l> = (U^T diag(a^2) U)_kl (V diag(b^2) V^T)_kl
+    and c_k = <W, P_k> = (a * U[:, k])^T W (V[k, :] * b).  A singular G (more
+    middle entries than independent P_k) takes the minimum-norm solution.
+
+    Returns (mid float64 [r], fp16 bits [r] of RNE(mid)): the storage keeps
+    the diagonals in fp16, so the stored diagonal is the rounded solution.
+    """
+    W = np.asarray(W, dtype=np.float64)
+    a = fp16_bits_to_f64(a_bits)
+    b = fp16_bits_to_f64(b_bits)
+    U = 1.0 - 2.0 * unpack_bits_lsb_first(B1_words, r).astype(np.float64)   # [m, r]
+    V = 1.0 - 2.0 * unpack_bits_lsb_first(B2_words, n).astype(np.float64)   # [r, n]
+    Pu = a[:, None] * U           # columns p_k
+    Qv = V * b[None, :]           # rows q_k
+    G = (Pu.T @ Pu) * (Qv @ Qv.T)
+    c = np.einsum("ik,ij,kj->k", Pu, W, Qv)
+    try:
+        mid = np.linalg.solve(G, c)
+    except np.linalg.LinAlgError:
+        mid = np.linalg.lstsq(G, c, rcond=None)[0]
+    bits = np.array([round_to_fp16_bits(Fraction(abs(v))) | (0x8000 if v < 0 else 0) for v in mid], dtype=np.uint16)
+    return mid, bits
+
+
 def sum_squares_ref(A) -> float:
     """sum of A^2, exactly rounded once (math.fsum over float64 squares; the
     squares of float32 values are exact in float64)."""

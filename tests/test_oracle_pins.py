@@ -578,3 +578,64 @@ def test_power_iteration_against_svd():
     est = O.power_iteration_ref(B, g.standard_normal(70), 32)
     assert est <= np.linalg.norm(B, 2) * (1 + 1e-12)
     assert est >= 0.9 * np.linalg.norm(B, 2)
+
+
+# ---------------------------------------------------------------- D_mid reprojection
+
+def _dbf_factors(m, r, n, seed):
+    a, B1, mid, B2, b, _ = synth.dbf_case(m=m, r=r, n=n, B=1, seed=seed)
+    return a, B1, mid, B2, b
+
+
+def test_reproject_recovers_the_middle_diagonal_of_an_exact_dbf():
+    m, r, n = 64, 32, 96
+    a, B1, mid, B2, b = _dbf_factors(m, r, n, 80)
+    W = O.dbf_dense_ref(a, B1, mid, B2, b, m, r, n)
+    got, bits = O.dbf_reproject_mid_ref(W, a, B1, B2, b, m, r, n)
+    assert np.max(np.abs(got - O.fp16_bits_to_f64(mid))) <= 1e-10 * np.max(np.abs(got))
+    assert np.array_equal(bits, mid)  # the exact fp16 values come back
+
+
+def test_reproject_matches_lstsq_on_the_explicit_design_matrix():
+    """Independent formulation: least squares over the m n x r matrix whose
+    columns are vec((a * U[:, k]) (V[k, :] * b)^T)."""
+    m, r, n = 32, 32, 64
+    a, B1, _, B2, b = _dbf_factors(m, r, n, 81)
+    W = synth.weights(synth.rng(82), m, n, std=0.05).astype(np.float64)
+    av, bv = O.fp16_bits_to_f64(a), O.fp16_bits_to_f64(b)
+
+    def sgn(words, row, col):
+        return 1 - 2 * ((int(words[row, col // 32]) >> (col % 32)) & 1)
+
+    X = np.empty((m * n, r))
+    for k in range(r):
+        p = np.array([av[i] * sgn(B1, i, k) for i in range(m)])
+        q = np.array([sgn(B2, k, j) * bv[j] for j in range(n)])
+        X[:, k] = np.outer(p, q).ravel()
+    ref = np.linalg.lstsq(X, W.ravel(), rcond=None)[0]
+    got, _ = O.dbf_reproject_mid_ref(W, a, B1, B2, b, m, r, n)
+    assert np.max(np.abs(got - ref)) <= 1e-9 * np.max(np.abs(ref))
+    # the residual is orthogonal to every column (the normal equations)
+    res = W.ravel() - X @ got
+    assert np.max(np.abs(X.T @ res)) <= 1e-9 * np.max(np.abs(X.T @ W.ravel()))
+
+
+def test_reproject_is_optimal_and_bits_round_to_nearest():
+    """Random perturbations of the solution raise the error; the stored bits
+    are numpy's round-to-nearest fp16 of the solution."""
+    m, r, n = 48, 32, 64
+    a, B1, _, B2, b = _dbf_factors(m, r, n, 83)
+    W = synth.weights(synth.rng(84), m, n, std=0.05).astype(np.float64)
+    got, bits = O.dbf_reproject_mid_ref(W, a, B1, B2, b, m, r, n)
+    av, bv = O.fp16_bits_to_f64(a), O.fp16_bits_to_f64(b)
+    U = 1.0 - 2.0 * O.unpack_bits_lsb_first(B1, r)
+    V = 1.0 - 2.0 * O.unpack_bits_lsb_first(B2, n)
+
+    def err(mid):
+        return float(np.sum((W - (av[:, None] * U) @ (mid[:, None] * V * bv[None, :])) ** 2))
+
+    e0 = err(got)
+    g = synth.rng(85)
+    for _ in range(8):
+        assert err(got + 1e-3 * g.standard_normal(r)) > e0
+    assert np.array_equal(bits, got.astype(np.float16).view(np.uint16))
