@@ -21,16 +21,41 @@ def _pack_experts(Wt):
     return s.reshape(E, rows, K // 32), c.reshape(E, rows, K // 128)
 
 
+def tied_logits(T, E, seed):
+    """Router logits full of exact ties: all-zero rows, constant rows, rows of
+    values that each appear twice, and rows whose top value is unique but
+    whose next values tie.  Ties in the logits are ties in the probabilities,
+    which the routing breaks toward the lower expert index."""
+    g = np.random.default_rng(seed)
+    L = np.empty((T, E), dtype=np.float32)
+    for t in range(T):
+        kind = t % 4
+        if kind == 0:
+            L[t] = 0.0
+        elif kind == 1:
+            L[t] = np.float32(g.normal())
+        elif kind == 2:
+            vals = g.normal(size=(E + 1) // 2).astype(np.float32)
+            L[t] = np.repeat(vals, 2)[:E][g.permutation(E)]
+        else:
+            L[t] = g.normal(size=E).astype(np.float32) - 4.0
+            L[t, g.integers(0, E)] = 3.0
+            L[t, g.choice(E, size=min(E - 1, 6), replace=False)[:5]] = 1.25
+    return L
+
+
 @functools.lru_cache(maxsize=None)
-def moe_case(T, H, I, E, seed, skew=0.0):
+def moe_case(T, H, I, E, seed, skew=0.0, ties=False):
     x, logits, gate, up, down = synth.moe_case(T=T, H=H, I=I, E=E, seed=seed)
     if skew:
         logits = logits + np.float32(skew) * np.linspace(1.0, 0.0, E, dtype=np.float32)[None, :]
+    if ties:
+        logits = tied_logits(T, E, seed)
     return x, logits, _pack_experts(gate), _pack_experts(up), _pack_experts(down)
 
 
-def run_and_check(T, H, I, E, K, seed, skew=0.0):
-    x, logits, G, U, D = moe_case(T, H, I, E, seed, skew)
+def run_and_check(T, H, I, E, K, seed, skew=0.0, ties=False):
+    x, logits, G, U, D = moe_case(T, H, I, E, seed, skew, ties)
     dev = lambda p: (words_dev(p[0].reshape(-1, p[0].shape[-1])).view(p[0].shape[0], p[0].shape[1], -1),
                      fp16_dev(p[1].reshape(-1, p[1].shape[-1])).view(p[1].shape[0], p[1].shape[1], -1))
     ws = ops.moe_workspace(T, H, I, E, K)
@@ -115,3 +140,15 @@ def test_moe_is_deterministic(T):
     b = ops.w1_moe_grouped(*args).cpu().numpy()
     assert ops.sync_status() == _lib.W1_OK
     assert np.array_equal(a, b)
+
+
+@pytest.mark.parametrize("path", ["default", "tiles", "decode"])
+@pytest.mark.parametrize("T", [5, 24])
+def test_moe_routing_ties_go_to_the_lower_expert(path, T, monkeypatch):
+    """Exactly tied router logits on both paths (the decode path routes up to
+    4 tokens inside its gate/up kernel, more in the router kernel): the expert
+    ids must equal the oracle's, whose ties go to the lower expert index."""
+    if path != "default":
+        monkeypatch.setenv("W1_MOE_PATH", path)
+    run_and_check(T, 512, 256, 16, 4, 9, ties=True)
+    run_and_check(min(T, 3), 512, 256, 16, 4, 10, ties=True)

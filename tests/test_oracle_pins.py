@@ -639,3 +639,99 @@ def test_reproject_is_optimal_and_bits_round_to_nearest():
     for _ in range(8):
         assert err(got + 1e-3 * g.standard_normal(r)) > e0
     assert np.array_equal(bits, got.astype(np.float16).view(np.uint16))
+
+
+# ---------------------------------------------------------------- 16-bit input formats
+
+def _ieee_decode(bits: int, ebits: int, mbits: int) -> float:
+    """Value of a binary floating-point pattern from the IEEE 754 field layout
+    (sign, biased exponent, fraction; exponent 0 = subnormal), exact in
+    Python rationals; inf for an all-ones exponent with a zero fraction."""
+    sign = -1 if (bits >> (ebits + mbits)) & 1 else 1
+    e = (bits >> mbits) & ((1 << ebits) - 1)
+    f = bits & ((1 << mbits) - 1)
+    bias = (1 << (ebits - 1)) - 1
+    if e == (1 << ebits) - 1:
+        assert f == 0
+        return sign * math.inf
+    if e == 0:
+        v = Fraction(f, 1 << mbits) * Fraction(2) ** (1 - bias)
+    else:
+        v = (1 + Fraction(f, 1 << mbits)) * Fraction(2) ** (e - bias)
+    return math.copysign(float(v), sign)
+
+
+def test_bf16_widening_hand_written_patterns():
+    pats = {0x3F80: 1.0, 0xC000: -2.0, 0x3FC0: 1.5, 0x0080: 2.0 ** -126, 0x0001: 2.0 ** -133,
+            0x007F: 127 * 2.0 ** -133, 0x7F7F: (2.0 - 2.0 ** -7) * 2.0 ** 127, 0x7F80: math.inf,
+            0xFF80: -math.inf, 0x4049: 3.140625, 0x0000: 0.0}
+    got = O.bf16_bits_to_f64(np.array(list(pats), dtype=np.uint16))
+    assert got.tolist() == list(pats.values())
+    neg0 = O.bf16_bits_to_f64(np.array([0x8000], dtype=np.uint16))[0]
+    assert neg0 == 0.0 and math.copysign(1.0, neg0) == -1.0
+
+
+def test_bf16_and_fp16_widening_match_the_field_layout_for_every_pattern():
+    # brute force over all 65536 patterns except NaNs (all-ones exponent with a
+    # nonzero fraction): bf16 = 1/8/7 with bias 127, binary16 = 1/5/10 with bias 15
+    allp = np.arange(1 << 16, dtype=np.uint32)
+    for fn, eb, mb in ((O.bf16_bits_to_f64, 8, 7), (O.fp16_bits_to_f64, 5, 10)):
+        emask = ((1 << eb) - 1) << mb
+        keep = ~(((allp & emask) == emask) & ((allp & ((1 << mb) - 1)) != 0))
+        pats = allp[keep]
+        got = fn(pats.astype(np.uint16))
+        want = np.array([_ieee_decode(int(p), eb, mb) for p in pats], dtype=np.float64)
+        assert np.array_equal(got, want)
+        assert np.array_equal(np.signbit(got), (pats >> 15).astype(bool))
+
+
+def test_bf16_widening_inverts_the_library_rounding_of_bf16_exact_values():
+    torch = pytest.importorskip("torch")
+    g = np.random.default_rng(17)
+    # values with at most 8 significant bits over the whole exponent range
+    # (normal and subnormal), so the library's float32 -> bf16 conversion is exact
+    man = g.integers(128, 256, 5000).astype(np.float64)
+    ex = g.integers(-133, 120, 5000)
+    sub = g.integers(1, 128, 500).astype(np.float64) * 2.0 ** -133   # bf16 subnormals
+    v = np.concatenate([man * np.exp2(ex.astype(np.float64)), sub])
+    v *= np.where(g.random(v.size) < 0.5, -1.0, 1.0)
+    bits = torch.tensor(v.astype(np.float32)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(O.bf16_bits_to_f64(bits), v.astype(np.float32).astype(np.float64))
+
+
+def test_fast_pack_equals_plain_pack_on_wide_exponent_spreads():
+    # a few thousand groups whose magnitudes span up to 31 binades (the int64
+    # alignment window) and beyond (the exact fallback), with random signs,
+    # subnormals and zeros mixed in
+    g = np.random.default_rng(41)
+    rows, K = 96, 4096
+    W = np.empty((rows, K), dtype=np.float32)
+    for n in range(rows):
+        for c in range(K // 128):
+            spread = int(g.integers(0, 40))
+            top = int(g.integers(-126, 100))
+            ex = top - g.integers(0, spread + 1, 128)
+            man = g.random(128) + 1.0
+            v = np.ldexp(man, ex).astype(np.float32)
+            if g.random() < 0.2:
+                v[g.integers(0, 128, 8)] = np.float32(2.0 ** -149) * g.integers(1, 1 << 20, 8)
+            if g.random() < 0.1:
+                v[g.integers(0, 128, 16)] = 0.0
+            if c % 4 == 0:
+                # mean exactly on an fp16 rounding midpoint (fp16 value + half
+                # an ulp), with or without a tie-breaker far below the
+                # alignment window of the largest value
+                h = np.float16(np.exp2(g.uniform(-13, 15)) * (1 + g.random()))
+                if not np.isfinite(h) or h == 0 or h >= np.float16(65504):
+                    h = np.float16(1.5)
+                M = np.float32((float(h) + float(np.nextafter(h, np.float16(np.inf)))) / 2)
+                v = np.full(128, M, dtype=np.float32)
+                v[126] = np.float32(2.0) * M
+                v[127] = np.float32(2.0) ** int(g.integers(-149, -60)) if g.random() < 0.5 else 0.0
+                v = v[g.permutation(128)]
+            v *= np.where(g.random(128) < 0.5, -1.0, 1.0).astype(np.float32)
+            W[n, c * 128:(c + 1) * 128] = v
+    s1, c1 = O.pack_ref(W)
+    s2, c2 = O.pack_ref_fast(W)
+    assert np.array_equal(s1, s2)
+    assert np.array_equal(c1, c2)
