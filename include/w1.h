@@ -70,6 +70,22 @@ const char* w1_status_string(int status);
  * synchronisation itself failed. */
 int w1_sync_status(w1_stream_t stream);
 
+/* Process-wide testing and tuning knobs (no counterpart on the pages).  Each
+ * starts from its W1_* environment variable, read once on first use; no call
+ * reads the environment after that.  `value` NULL or "" restores the value
+ * the environment gave.  Host-side only and not synchronised with calls in
+ * flight on other host threads.
+ *   "gemv_path"     "direct" | "direct16" | "tc" | "ring" | "flat" forces one GEMV kernel (W1_GEMV_PATH)
+ *   "gemv_split"    1 | 2 | 4 | 8: forced K split of the split-capable GEMV kernels (W1_GEMV_SPLIT)
+ *   "gemv_autotune" "0": the static kernel rule instead of first-call timing (W1_GEMV_AUTOTUNE)
+ *   "moe_path"      "tiles" | "decode" forces a routed-MoE path (W1_MOE_PATH)
+ *   "dbf_path"      "fused" | "twostep" forces a small-batch DBF chain form (W1_DBF_PATH)
+ *   "dbf_warps"     8 | 16 warps per CTA of the small-batch DBF chain (W1_DBF_WARPS)
+ *   "verbose"       nonzero prints plans and choices on stderr (W1_VERBOSE)
+ * Returns W1_ERR_NULL for a NULL name, W1_ERR_SHAPE for an unknown name or
+ * value. */
+int w1_set_knob(const char* name, const char* value);
+
 /*
  * w1_pack -- binarise W along K ("Behaviour-Relearned Quantization", step 02;
  * sign convention: DBF post, section 1).
@@ -346,6 +362,10 @@ size_t dbf_workspace_size(int64_t m, int64_t r, int64_t n, int64_t B);
  * (256 bytes + 4*8*16384 bytes, held on every GPU that loads the library until
  * the process exits).  It allocates nothing and calls no allocating routine.
  *   Limit: r <= 16384, else W1_ERR_TOO_LARGE (other limits as dbf_apply).
+ *   Every batch size runs the small-batch chain, in groups of up to 8 rows
+ *   one after another: unlike dbf_apply it never takes the tensor-core path
+ *   (that path needs a workspace that grows with B), so from B = 64 up it
+ *   costs about ceil(B/8) times a group of 8 (64 launches at B = 512).
  *   The first call on a device looks up the array's device address (with that
  *   device current); make that first call before any stream capture.
  *   Every call shares the one array and clears its barrier count first; calls

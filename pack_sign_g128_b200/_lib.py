@@ -29,6 +29,7 @@ _sz = ctypes.c_size_t
 SIGNATURES = {
     "w1_status_string": (ctypes.c_char_p, [_int]),
     "w1_sync_status": (_int, [_p]),
+    "w1_set_knob": (_int, [ctypes.c_char_p, ctypes.c_char_p]),
     "w1_pack": (_int, [_p, _i64, _i64, _p, _p, _p]),
     "w1_gemv": (_int, [_p, _p, _i64, _i64, _p, _i64, _p, _p]),
     "w1_gemv_ex": (_int, [_p, _p, _i64, _i64, _p, _i64, _p, ctypes.c_uint32, _p]),

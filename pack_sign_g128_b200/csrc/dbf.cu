@@ -247,7 +247,7 @@ static cudaError_t launch_dbf_small_nb(const uint16_t* a, const uint32_t* B1, co
   p2.y = y;
   cudaError_t err = ensure_dyn_smem(reinterpret_cast<const void*>(dbf_direct_kernel<NB, NW>), smem);
   if (err != cudaSuccess) return err;
-  if (getenv("W1_VERBOSE"))
+  if (knob(kKnobVerbose))
     fprintf(stderr, "dbf plan: B=%d warps=%d -> clusters=%d split=%d warps=%dx%d / %dx%d smem=%d\n", NB, NW, Q, S,
             p1.Wn, p1.Wg, p2.Wn, p2.Wg, smem);
   cudaLaunchConfig_t cfg = {};
@@ -299,66 +299,39 @@ cudaError_t launch_dbf(const uint16_t* a, const uint32_t* B1, const uint16_t* mi
     return launch_dbf_tc(a, B1, mid, B2, b, m, r, n, x, B, y, workspace, stream, num_sms);
   unsigned int* bar = reinterpret_cast<unsigned int*>(workspace);
   float* h = reinterpret_cast<float*>(static_cast<unsigned char*>(workspace) + 256);
-  // batches of up to 8 rows through a fused chain kernel: the direct core (8
-  // warps per CTA for groups of up to 3 rows, 16 above, as measured; the ring
-  // core in dbf_ring.cu measured slower at every group size).  Testing knobs:
-  // W1_DBF_PATH=direct|ring forces a core, W1_DBF_WARPS=8|16 the warp count.
-  const char* path = getenv("W1_DBF_PATH");
-  const char* wenv = getenv("W1_DBF_WARPS");
-  DbfParams rp = {};
-  rp.a = a;
-  rp.mid = mid;
-  rp.b = b;
-  rp.bar = bar;
-  rp.h = h;
-  rp.m = static_cast<int>(m);
-  rp.r = static_cast<int>(r);
-  rp.n = static_cast<int>(n);
+  // Batches of up to 8 rows through the fused chain kernel: 8 warps per CTA
+  // for groups of up to 3 rows, 16 above (as measured).  The dbf_warps knob
+  // forces 8 or 16.
+  const int wknob = knob(kKnobDbfWarps);
+  const int im = static_cast<int>(m), ir = static_cast<int>(r), in = static_cast<int>(n);
   for (int64_t b0 = 0; b0 < B; b0 += 8) {
     const int nb = static_cast<int>((B - b0) < 8 ? (B - b0) : 8);
     const uint16_t* xg = x + b0 * n;
     float* yg = y + b0 * m;
-    const int im = static_cast<int>(m), ir = static_cast<int>(r), in = static_cast<int>(n);
-    const bool direct = path ? path[0] == 'd' : true;
-    const bool w16 = wenv ? atoi(wenv) == 16 : nb >= 4;
+    const bool w16 = wknob ? wknob == 16 : nb >= 4;
     cudaError_t err;
-    if (direct) {
-      switch (nb) {
-#define W1_DBF_CASE(NBV)                                                                                     \
-  case NBV:                                                                                                  \
+    switch (nb) {
+#define W1_DBF_CASE(NBV)                                                                                   \
+  case NBV:                                                                                                \
     err = w16 ? launch_dbf_small_nb<NBV, 16>(a, B1, mid, B2, b, im, ir, in, xg, yg, h, bar, stream, num_sms, \
-                                             smem_cap)                                                      \
+                                             smem_cap)                                                    \
               : launch_dbf_small_nb<NBV, 8>(a, B1, mid, B2, b, im, ir, in, xg, yg, h, bar, stream, num_sms,  \
-                                            smem_cap);                                                      \
+                                            smem_cap);                                                    \
     break;
-        W1_DBF_CASE(1)
-        W1_DBF_CASE(2)
-        W1_DBF_CASE(3)
-        W1_DBF_CASE(4)
-        W1_DBF_CASE(5)
-        W1_DBF_CASE(6)
-        W1_DBF_CASE(7)
-        default:
-          err = w16 ? launch_dbf_small_nb<8, 16>(a, B1, mid, B2, b, im, ir, in, xg, yg, h, bar, stream, num_sms,
-                                                 smem_cap)
-                    : launch_dbf_small_nb<8, 8>(a, B1, mid, B2, b, im, ir, in, xg, yg, h, bar, stream, num_sms,
-                                                smem_cap);
-          break;
+      W1_DBF_CASE(1)
+      W1_DBF_CASE(2)
+      W1_DBF_CASE(3)
+      W1_DBF_CASE(4)
+      W1_DBF_CASE(5)
+      W1_DBF_CASE(6)
+      W1_DBF_CASE(7)
+      default:
+        err = w16 ? launch_dbf_small_nb<8, 16>(a, B1, mid, B2, b, im, ir, in, xg, yg, h, bar, stream, num_sms,
+                                               smem_cap)
+                  : launch_dbf_small_nb<8, 8>(a, B1, mid, B2, b, im, ir, in, xg, yg, h, bar, stream, num_sms,
+                                              smem_cap);
+        break;
 #undef W1_DBF_CASE
-      }
-    } else {
-      rp.x = xg;
-      rp.y = yg;
-      switch (nb) {
-        case 1: err = launch_dbf_ring_nb<1>(rp, B1, B2, stream, num_sms, smem_cap); break;
-        case 2: err = launch_dbf_ring_nb<2>(rp, B1, B2, stream, num_sms, smem_cap); break;
-        case 3: err = launch_dbf_ring_nb<3>(rp, B1, B2, stream, num_sms, smem_cap); break;
-        case 4: err = launch_dbf_ring_nb<4>(rp, B1, B2, stream, num_sms, smem_cap); break;
-        case 5: err = launch_dbf_ring_nb<5>(rp, B1, B2, stream, num_sms, smem_cap); break;
-        case 6: err = launch_dbf_ring_nb<6>(rp, B1, B2, stream, num_sms, smem_cap); break;
-        case 7: err = launch_dbf_ring_nb<7>(rp, B1, B2, stream, num_sms, smem_cap); break;
-        default: err = launch_dbf_ring_nb<8>(rp, B1, B2, stream, num_sms, smem_cap); break;
-      }
     }
     if (err != cudaSuccess) return err;
   }

@@ -255,7 +255,7 @@ template <int NB>
 static cudaError_t launch_gemv_nb(const uint32_t* signs, const GemvParams& base, cudaStream_t stream, int num_sms,
                                   int smem_cap) {
   int force = 0;
-  if (const char* f = getenv("W1_GEMV_SPLIT")) force = atoi(f);  // tuning knob: force the K split
+  force = knob(kKnobGemvSplit);  // tuning knob: force the K split
   if (force != 1 && force != 2 && force != 4 && force != 8) force = 0;
   int dev = 0;
   cudaGetDevice(&dev);
@@ -279,7 +279,7 @@ static cudaError_t launch_gemv_nb(const uint32_t* signs, const GemvParams& base,
     const int i = g_plan_count < 64 ? g_plan_count++ : (base.rows + base.NG + NB) & 63;
     g_plan_cache[i] = GemvPlanEntry{base.rows, base.NG, NB, num_sms, smem_cap, dev, force, plan};
   }
-  if (getenv("W1_VERBOSE"))
+  if (knob(kKnobVerbose))
     fprintf(stderr, "w1_gemv plan: rows=%d NG=%d B=%d -> clusters=%d split=%d box=%d stages=%d tiles=%d smem=%d\n",
             base.rows, base.NG, NB, plan.Q, plan.S, plan.bw, plan.ns, plan.max_tiles, plan.smem);
   GemvParams p = base;
@@ -462,10 +462,10 @@ static int time_gemv_choice(const GemvChoice& c, const uint32_t* signs, const ui
 cudaError_t launch_gemv(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t K,
                         const void* x, bool xf, int B, float* y, cudaStream_t stream, int num_sms,
                         int smem_cap, bool static_weights) {
-  if (const char* path = getenv("W1_GEMV_PATH")) {
+  if (const int path = knob(kKnobGemvPath)) {
     // fp32 activations run the direct kernel whatever the knob names.
-    const GemvChoice c{(path[0] == 'd' || xf) ? 'd' : (path[0] == 't' ? 't' : 'm'), 0,
-                       strcmp(path, "direct16") == 0 ? 16 : 8};
+    const bool direct = path == kGemvDirect8 || path == kGemvDirect16 || xf;
+    const GemvChoice c{direct ? 'd' : (path == kGemvTc ? 't' : 'm'), 0, path == kGemvDirect16 ? 16 : 8};
     return run_gemv_choice(c, signs, scales, N, K, x, xf, B, y, stream, num_sms, smem_cap, static_weights);
   }
   int dev = 0;
@@ -483,8 +483,7 @@ cudaError_t launch_gemv(const uint32_t* signs, const uint16_t* scales, int64_t N
     cudaGetLastError();
     cap = cudaStreamCaptureStatusActive;
   }
-  const char* at = getenv("W1_GEMV_AUTOTUNE");
-  if (cap != cudaStreamCaptureStatusNone || (at && at[0] == '0'))
+  if (cap != cudaStreamCaptureStatusNone || knob(kKnobGemvAutotune) == 0)
     return run_gemv_rule(signs, scales, N, K, x, xf, B, y, stream, num_sms, smem_cap, static_weights);
 
   const GemvChoice cands[] = {{'d', 1, 8},  {'d', 2, 8},  {'d', 4, 8},  {'d', 8, 8}, {'d', 1, 16},
@@ -528,7 +527,7 @@ cudaError_t launch_gemv(const uint32_t* signs, const uint16_t* scales, int64_t N
                                    kTimed, e0, e1, &ms, &fatal);
     if (r < 0) break;  // a device error: report it, choose nothing
     if (r == 0) continue;
-    if (getenv("W1_VERBOSE"))
+    if (knob(kKnobVerbose))
       fprintf(stderr, "w1_gemv candidate: N=%lld K=%lld B=%d %c split=%d warps=%d %.2f us\n",
               static_cast<long long>(N), static_cast<long long>(K), B, c.kind, c.s, c.w, ms * 1e3f / kTimed);
     if (best.kind == 0 || ms < best_ms) {
@@ -548,7 +547,7 @@ cudaError_t launch_gemv(const uint32_t* signs, const uint16_t* scales, int64_t N
   if (fatal != cudaSuccess) return fatal;
   if (best.kind == 0)
     return run_gemv_rule(signs, scales, N, K, x, xf, B, y, stream, num_sms, smem_cap, static_weights);
-  if (getenv("W1_VERBOSE"))
+  if (knob(kKnobVerbose))
     fprintf(stderr, "w1_gemv tuned: N=%lld K=%lld B=%d static=%d -> %c split=%d warps=%d (%.2f us)\n",
             static_cast<long long>(N), static_cast<long long>(K), B, static_weights ? 1 : 0, best.kind, best.s,
             best.w, best_ms * 1e3f / kTimed);

@@ -744,7 +744,7 @@ template <int NB, int NW>
 static bool gd_cached_plan(int N, int NG, int num_sms, int smem_cap, int force_s, GdPlan* out) {
   int force = force_s;
   if (!force)
-    if (const char* f = getenv("W1_GEMV_SPLIT")) force = atoi(f);  // tuning knob: force the K split
+    force = knob(kKnobGemvSplit);  // tuning knob: force the K split
   if (force != 1 && force != 2 && force != 4 && force != 8) force = 0;
   int dev = 0;
   cudaGetDevice(&dev);
@@ -781,7 +781,7 @@ static cudaError_t launch_gemv_direct_nb(const GdParams& base, cudaStream_t stre
                                          int force_s) {
   GdPlan plan;
   if (!gd_cached_plan<NB, NW>(base.N, base.NG, num_sms, smem_cap, force_s, &plan)) return cudaErrorNotSupported;
-  if (getenv("W1_VERBOSE"))
+  if (knob(kKnobVerbose))
     fprintf(stderr,
             "w1_gemv(direct) plan: N=%d NG=%d B=%d warps=%d -> clusters=%d split=%d warps=%dx%d tiles/warp=%d "
             "sets/warp=%d smem=%d\n",

@@ -483,7 +483,7 @@ template <int NB>
 static bool gemv_tc_cached_plan(int N, int NG, int num_sms, int force_s, GemvTcPlan* out) {
   int force = force_s;
   if (!force)
-    if (const char* f = getenv("W1_GEMV_SPLIT")) force = atoi(f);  // tuning knob: force the K split
+    force = knob(kKnobGemvSplit);  // tuning knob: force the K split
   if (force != 1 && force != 2 && force != 4 && force != 8) force = 0;
   int dev = 0;
   cudaGetDevice(&dev);
@@ -510,7 +510,7 @@ template <int NB>
 static cudaError_t launch_gemv_tc_nb(const GemvTcParams& base, cudaStream_t stream, int num_sms, int force_s) {
   GemvTcPlan plan;
   if (!gemv_tc_cached_plan<NB>(base.N, base.NG, num_sms, force_s, &plan)) return cudaErrorNotSupported;
-  if (getenv("W1_VERBOSE"))
+  if (knob(kKnobVerbose))
     fprintf(stderr, "w1_gemv(tc) plan: N=%d NG=%d B=%d -> clusters=%d split=%d groups=%d smem=%d\n", base.N,
             base.NG, NB, plan.Q, plan.S, plan.max_ng, plan.smem);
   GemvTcParams p = base;

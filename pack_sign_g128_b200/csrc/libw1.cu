@@ -8,7 +8,6 @@
 #include "sign_gemm.cu"
 #include "gemm.cu"
 #include "dbf_tc.cu"
-#include "dbf_ring.cu"
 #include "dbf.cu"
 #include "moe.cu"
 #include "okt.cu"

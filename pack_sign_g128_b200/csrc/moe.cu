@@ -781,7 +781,7 @@ __global__ void __launch_bounds__(256) moe_hprep_kernel(const uint16_t* __restri
   pdl_launch_dependents();
 }
 
-// ------------------------------------------------------------------ decode regime (T <= 8)
+// ------------------------------------------------------------------ decode regime (T <= kDecodeMaxT = 16)
 
 // With a handful of tokens every expert sees about one route, so the tile
 // pipeline's 128-route MMA tiles would be almost empty.  Instead each route is
@@ -1136,10 +1136,10 @@ cudaError_t launch_moe(const uint16_t* x, const float* logits, int64_t T, int64_
   // products on the direct GEMV steps: gate/up (with the routing up to 4
   // tokens), down with the combine.  Measured on the OLMoE-like layer: about 2x faster
   // than the tile pipeline up to 8 tokens, still ahead at 16.
-  // W1_MOE_PATH=tiles|decode forces a path (testing knob).
+  // The moe_path knob (tiles | decode) forces a path for testing.
   constexpr int64_t kDecodeMaxT = 16;
-  const char* mpath = getenv("W1_MOE_PATH");
-  bool decode = (mpath ? mpath[0] == 'd' : T <= kDecodeMaxT) && H / 128 <= gd::kMaxSets && I / 128 <= gd::kMaxSets;
+  const int mpath = knob(kKnobMoePath);
+  bool decode = (mpath ? mpath == 2 : T <= kDecodeMaxT) && H / 128 <= gd::kMaxSets && I / 128 <= gd::kMaxSets;
   if (decode) {  // both decode kernels' shared memory must fit
     MoeDecParams qg = {};
     qg.NG = static_cast<int>(H / 128);

@@ -203,17 +203,8 @@ cudaError_t launch_okt_rotate(const float* H, int n1, const float* R, int n2, co
   p.early = early ? 1 : 0;
   const size_t smem = okt_smem_bytes(n1, n2, p.RS);
   if (smem > static_cast<size_t>(smem_optin)) return cudaErrorNotSupported;
-  // The dynamic shared memory limit is raised once per device, to the most
-  // any launch so far has needed.
-  static int s_smem_set[64] = {};
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  const cudaError_t e = ensure_dyn_smem(reinterpret_cast<const void*>(okt_rotate_kernel), static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= 64 || static_cast<int>(smem) > s_smem_set[dev]) {
-    e = cudaFuncSetAttribute(okt_rotate_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    if (dev >= 0 && dev < 64) s_smem_set[dev] = static_cast<int>(smem);
-  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>((n1 + p.RS - 1) / p.RS), static_cast<unsigned>(B), 1);
   cfg.blockDim = dim3(okt::kThreads, 1, 1);

@@ -8,16 +8,19 @@
 // group scale is folded into the weight operand, which is exact because s is
 // an fp16 value and a sign flip only sets its top bit.)
 //  * sg_prep_kernel: xs = fp16(x * 2^c_t) per token row (exact scaling).
-//  * sg_gemm_kernel: one CTA per SM, persistent over 128 x 256 output tiles
-//    (128 weight rows x 256 tokens; 128 tokens when that fills more SMs), swap-AB: D^T (TMEM, fp32, 256 columns,
-//    two accumulators) = A (shared memory, +-s fp16) x xs^T (shared memory,
-//    fp16, by TMA), 128 x 256 x 16 MMAs (N = 256 keeps the tensor pipe busy
-//    per instruction).  Pipeline stages are 64 wide in K (one 128-byte swizzle
-//    row of fp16), four deep:
-//    warp 0 TMA producer (xs: one 256 x 64 box per stage); warp 1 MMA issuer
-//    (4 MMAs per stage, all of K into one accumulator per tile); warps 2-5
-//    expanders (thread = weight row: 2 sign words + the group scale -> 32
-//    fp16 pairs, written in the 128B-swizzled K-major layout the MMA reads);
+//  * sg_gemm_kernel: one CTA per SM, persistent over output tiles of 128
+//    weight rows x BM tokens (BM = 256, or 128 when 256-token tiles would not
+//    fill the GPU), swap-AB: D^T (TMEM, fp32, two accumulators of BM columns)
+//    = A (shared memory, +-s fp16) x xs^T (shared memory, fp16, by TMA),
+//    128 x BM x 16 MMAs.  Pipeline stages are 128 wide in K (one scale group,
+//    two 64-wide 128-byte swizzle atoms), 2 deep at BM = 256 and 3 deep at
+//    BM = 128 (192 KB either way):
+//    warp 0 TMA producer (xs: two BM x 64 boxes per stage, whose transaction
+//    bytes complete on the stage's full barrier); warp 1 MMA issuer (one wait
+//    per stage, then 8 MMAs, all of K into one accumulator per tile); warps
+//    2-5 expanders (thread = weight row: 4 sign words + the group scale -> 64
+//    fp16 pairs +-s, written as 16-byte chunks in the 128B-swizzled K-major
+//    layout the MMA reads, words prefetched 4 stages ahead in registers);
 //    warps 6-9 epilogue (thread = TMEM lane: row diagonal and token scale,
 //    store), draining one accumulator while the MMA fills the other.
 // Products of +-s and fp16 are exact in the tensor core; accumulation is fp32.

@@ -112,6 +112,19 @@ int w1_sync_status(w1_stream_t stream) {
   return static_cast<int>(v);
 }
 
+int w1_set_knob(const char* name, const char* value) {
+  if (!name) return W1_ERR_NULL;
+  for (int i = 0; i < kKnobCount; ++i) {
+    if (strcmp(name, knob_spec(i).name) != 0) continue;
+    KnobTable& t = knob_table();
+    int v = t.env[i];
+    if (value && *value && !parse_knob(i, value, &v)) return W1_ERR_SHAPE;
+    t.v[i].store(v, std::memory_order_relaxed);
+    return W1_OK;
+  }
+  return W1_ERR_SHAPE;
+}
+
 int w1_pack(const float* W, int64_t N, int64_t K, uint32_t* signs, uint16_t* scales,
             w1_stream_t stream) {
   if (!W || !signs || !scales) return W1_ERR_NULL;

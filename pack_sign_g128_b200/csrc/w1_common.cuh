@@ -393,3 +393,79 @@ inline cudaError_t ensure_dyn_smem(const void* kernel, int bytes) {
   return cudaSuccess;
 }
 }  // namespace w1
+
+// Host: process-wide testing and tuning knobs.  They are read from the W1_*
+// environment variables once, on first use, and can be changed afterwards
+// with w1_set_knob (include/w1.h); no launch path reads the environment.
+//   gemv_path     W1_GEMV_PATH      0 = dispatch, else a forced GEMV kernel
+//   gemv_split    W1_GEMV_SPLIT     forced K split of the split-capable GEMV kernels (0 = planner)
+//   gemv_autotune W1_GEMV_AUTOTUNE  0 = static rule instead of first-call timing
+//   moe_path      W1_MOE_PATH       0 = by token count, 1 = tiles, 2 = decode
+//   dbf_path      W1_DBF_PATH       0 = by batch, else a forced small-batch chain form
+//   dbf_warps     W1_DBF_WARPS      0 = by group size, 8 or 16 warps per CTA
+//   verbose       W1_VERBOSE        nonzero: plans and choices on stderr
+#include <atomic>
+#include <cstdlib>
+#include <cstring>
+namespace w1 {
+enum KnobId { kKnobGemvPath, kKnobGemvSplit, kKnobGemvAutotune, kKnobMoePath, kKnobDbfPath, kKnobDbfWarps,
+              kKnobVerbose, kKnobCount };
+// GEMV kernels a knob can force (also the kinds of the dispatcher's choices).
+enum GemvPathKnob { kGemvAuto = 0, kGemvDirect8 = 1, kGemvDirect16 = 2, kGemvTc = 3, kGemvRing = 4, kGemvFlat = 5 };
+enum DbfPathKnob { kDbfAuto = 0, kDbfFused = 1, kDbfTwoStep = 2 };
+
+struct KnobSpec {
+  const char* name;  // w1_set_knob name
+  const char* env;   // environment variable read at first use
+  int dflt;
+  const char* words[6];  // accepted words for values 1..6 (else an integer)
+};
+inline const KnobSpec& knob_spec(int id) {
+  static const KnobSpec specs[kKnobCount] = {
+      {"gemv_path", "W1_GEMV_PATH", 0, {"direct", "direct16", "tc", "ring", "flat", nullptr}},
+      {"gemv_split", "W1_GEMV_SPLIT", 0, {nullptr}},
+      {"gemv_autotune", "W1_GEMV_AUTOTUNE", 1, {nullptr}},
+      {"moe_path", "W1_MOE_PATH", 0, {"tiles", "decode", nullptr}},
+      {"dbf_path", "W1_DBF_PATH", 0, {"fused", "twostep", nullptr}},
+      {"dbf_warps", "W1_DBF_WARPS", 0, {nullptr}},
+      {"verbose", "W1_VERBOSE", 0, {nullptr}},
+  };
+  return specs[id];
+}
+// Parses a knob value: one of the spec's words (-> 1-based index) or an
+// integer.  Returns false for anything else.
+inline bool parse_knob(int id, const char* v, int* out) {
+  const KnobSpec& s = knob_spec(id);
+  for (int i = 0; i < 6 && s.words[i]; ++i)
+    if (strcmp(v, s.words[i]) == 0) {
+      *out = i + 1;
+      return true;
+    }
+  char* end = nullptr;
+  const long n = strtol(v, &end, 10);
+  if (end == v || *end != '\0' || n < 0 || n > 1 << 20) return false;
+  *out = static_cast<int>(n);
+  return true;
+}
+struct KnobTable {
+  std::atomic<int> v[kKnobCount];
+  int env[kKnobCount];  // the value the environment gave (restored by w1_set_knob(name, NULL))
+  KnobTable() {
+    for (int i = 0; i < kKnobCount; ++i) {
+      int val = knob_spec(i).dflt;
+      const char* e = getenv(knob_spec(i).env);
+      if (e && *e) {
+        int p = 0;
+        if (parse_knob(i, e, &p)) val = p;
+      }
+      env[i] = val;
+      v[i].store(val, std::memory_order_relaxed);
+    }
+  }
+};
+inline KnobTable& knob_table() {
+  static KnobTable t;  // thread-safe initialisation (C++11 statics)
+  return t;
+}
+inline int knob(int id) { return knob_table().v[id].load(std::memory_order_relaxed); }
+}  // namespace w1

@@ -43,6 +43,13 @@ def sync_status(stream=None) -> int:
     return _lib.call("w1_sync_status", _stream(stream))
 
 
+def set_knob(name: str, value: str | int | None) -> None:
+    """Set a process-wide testing / tuning knob of the library (w1_set_knob);
+    None restores the value the W1_* environment variable gave."""
+    v = None if value is None else str(value).encode()
+    _lib.check(_lib.call("w1_set_knob", name.encode(), v), f"w1_set_knob({name})")
+
+
 def status_string(status: int) -> str:
     return _lib.call("w1_status_string", int(status)).decode()
 

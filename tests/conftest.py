@@ -16,3 +16,18 @@ def pytest_configure(config):
 @pytest.fixture(scope="session")
 def golden_dir():
     return os.path.join(ROOT, "tests", "golden")
+
+
+@pytest.fixture
+def knob():
+    """Set library knobs (w1_set_knob) for one test; restored afterwards."""
+    from pack_sign_g128_b200 import ops
+    names = []
+
+    def setter(name, value):
+        ops.set_knob(name, value)
+        names.append(name)
+
+    yield setter
+    for n in reversed(names):
+        ops.set_knob(n, None)

@@ -43,6 +43,23 @@ def test_status_strings(lib):
         assert lib.w1_status_string(code).decode().startswith(name)
 
 
+def test_knobs_accept_their_words_and_reject_the_rest(lib):
+    ok = [("gemv_path", "direct"), ("gemv_path", "direct16"), ("gemv_path", "tc"), ("gemv_path", "ring"),
+          ("gemv_path", "flat"), ("gemv_split", "4"), ("gemv_autotune", "0"), ("moe_path", "tiles"),
+          ("moe_path", "decode"), ("dbf_path", "fused"), ("dbf_path", "twostep"), ("dbf_warps", "16"),
+          ("verbose", "1")]
+    try:
+        for name, value in ok:
+            assert lib.w1_set_knob(name.encode(), value.encode()) == _lib.W1_OK, (name, value)
+        assert lib.w1_set_knob(b"gemv_path", b"fast") == _lib.W1_ERR_SHAPE
+        assert lib.w1_set_knob(b"gemv_split", b"-1") == _lib.W1_ERR_SHAPE
+        assert lib.w1_set_knob(b"no_such_knob", b"1") == _lib.W1_ERR_SHAPE
+        assert lib.w1_set_knob(None, b"1") == _lib.W1_ERR_NULL
+    finally:
+        for name in {n for n, _ in ok}:
+            assert lib.w1_set_knob(name.encode(), None) == _lib.W1_OK
+
+
 def test_host_side_argument_errors(lib):
     good = ctypes.c_void_p(1 << 20)     # never dereferenced: calls fail validation first
     odd = ctypes.c_void_p((1 << 20) + 4)

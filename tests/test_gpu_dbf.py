@@ -1,8 +1,7 @@
 """dbf_apply on the GPU vs the fp64 oracle chain.
 
-Every test runs with each fused small-batch chain kernel forced: the direct
-GEMV core (W1_DBF_PATH=direct, the default) with 8 and with 16 warps per CTA
-(W1_DBF_WARPS), and the ring core (=ring).  Batches of 64 and more take the
+Every test runs with the fused small-batch chain kernel forced to 8 and to 16
+warps per CTA (the dbf_warps knob).  Batches of 64 and more take the
 tensor-core path either way."""
 import functools
 
@@ -17,11 +16,9 @@ from gpu_helpers import assert_within, bf16_dev, fp16_dev, words_dev
 pytestmark = pytest.mark.gpu
 
 
-@pytest.fixture(autouse=True, params=["direct8", "direct16", "ring"])
-def dbf_path(request, monkeypatch):
-    monkeypatch.setenv("W1_DBF_PATH", "ring" if request.param == "ring" else "direct")
-    if request.param != "ring":
-        monkeypatch.setenv("W1_DBF_WARPS", request.param[6:])
+@pytest.fixture(autouse=True, params=["fused8", "fused16"])
+def dbf_path(request, knob):
+    knob("dbf_warps", request.param[5:])
     return request.param
 
 

@@ -1,9 +1,9 @@
 """w1_gemv on the GPU vs the fp64 oracle (element-wise, 1e-3 * sum|s x| bound).
 
-Every test runs on each kernel: the direct kernel with 8 and with 16 warps
-per CTA (W1_GEMV_PATH=direct / direct16, the default wherever its plan fits),
-the tcgen05 kernel (=tc) and the mma.sync ring kernel (=mma, the fallback for
-other shapes)."""
+Every test runs on each kernel, forced with the gemv_path knob: the direct
+kernel with 8 and with 16 warps per CTA (direct / direct16), the tcgen05
+kernel (tc) and the mma.sync ring kernel (ring, the fallback for other
+shapes)."""
 import functools
 
 import numpy as np
@@ -17,9 +17,9 @@ from gpu_helpers import assert_within, bf16_dev, fp16_dev, words_dev
 pytestmark = pytest.mark.gpu
 
 
-@pytest.fixture(autouse=True, params=["direct", "direct16", "tc", "mma"])
-def gemv_path(request, monkeypatch):
-    monkeypatch.setenv("W1_GEMV_PATH", request.param)
+@pytest.fixture(autouse=True, params=["direct", "direct16", "tc", "ring"])
+def gemv_path(request, knob):
+    knob("gemv_path", request.param)
     return request.param
 
 
@@ -112,13 +112,13 @@ def test_gemv_is_deterministic():
 @pytest.mark.parametrize("split", ["1", "2", "4", "8"])
 @pytest.mark.parametrize("N,K,B", [(4096, 4096, 1), (1000, 1152, 5), (4097, 2176, 8), (300, 1024, 2),
                                    (4096, 11008, 8)])
-def test_gemv_direct_every_split(N, K, B, split, gemv_path, monkeypatch):
+def test_gemv_direct_every_split(N, K, B, split, gemv_path, knob):
     """The direct kernel's cluster K split (1..8 CTAs) on the same inputs.
     4096 x 11008 at B = 8 needs the reduction buffer over the activation
     scratch at 16 warps and small splits."""
     if not gemv_path.startswith("direct"):
         pytest.skip("split sweep is for the direct kernel")
-    monkeypatch.setenv("W1_GEMV_SPLIT", split)
+    knob("gemv_split", split)
     W, x = synth.gemv_case(N, K, B, seed=N + B)
     s, c = O.pack_ref_fast(W)
     try:

@@ -11,10 +11,10 @@ pytestmark = pytest.mark.gpu
 
 
 @pytest.fixture(autouse=True)
-def default_dispatch(monkeypatch):
-    monkeypatch.delenv("W1_GEMV_PATH", raising=False)
-    monkeypatch.delenv("W1_GEMV_SPLIT", raising=False)
-    monkeypatch.delenv("W1_GEMV_AUTOTUNE", raising=False)
+def default_dispatch(knob):
+    knob("gemv_path", "0")
+    knob("gemv_split", "0")
+    knob("gemv_autotune", "1")
 
 
 @pytest.mark.parametrize("N,K,B", [(4096, 4096, 1), (4096, 4096, 4), (4096, 4096, 8), (1000, 1152, 3),
@@ -33,8 +33,8 @@ def test_tuned_dispatch_parity_and_reproducibility(N, K, B):
     assert np.array_equal(first.cpu().numpy(), second.cpu().numpy())
 
 
-def test_autotune_off_uses_the_rule(monkeypatch):
-    monkeypatch.setenv("W1_GEMV_AUTOTUNE", "0")
+def test_autotune_off_uses_the_rule(knob):
+    knob("gemv_autotune", "0")
     N, K, B = 300, 1024, 5
     W, x = synth.gemv_case(N, K, B, seed=11)
     s, c = O.pack_ref_fast(W)

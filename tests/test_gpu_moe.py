@@ -1,7 +1,7 @@
 """w1_moe_grouped on the GPU vs the fp64 oracle: routing exact, every stage
 within its bound, end to end with the bf16 intermediate propagated.  Batches
 of up to 8 tokens take the decode path (per-route products), larger ones the
-expert-sorted tile pipeline; W1_MOE_PATH forces either."""
+expert-sorted tile pipeline; the moe_path knob forces either."""
 import functools
 
 import numpy as np
@@ -122,10 +122,10 @@ def test_moe_small_and_skewed(T, H, I, E, K, seed, skew):
 
 
 @pytest.mark.parametrize("path,T", [("tiles", 3), ("decode", 20)])
-def test_moe_forced_path(path, T, monkeypatch):
+def test_moe_forced_path(path, T, knob):
     """Each path outside its default regime: the tile pipeline for a few
     tokens, the per-route decode products for a larger batch."""
-    monkeypatch.setenv("W1_MOE_PATH", path)
+    knob("moe_path", path)
     run_and_check(T, 512, 256, 16, 4, 7)
 
 
@@ -144,11 +144,11 @@ def test_moe_is_deterministic(T):
 
 @pytest.mark.parametrize("path", ["default", "tiles", "decode"])
 @pytest.mark.parametrize("T", [5, 24])
-def test_moe_routing_ties_go_to_the_lower_expert(path, T, monkeypatch):
+def test_moe_routing_ties_go_to_the_lower_expert(path, T, knob):
     """Exactly tied router logits on both paths (the decode path routes up to
     4 tokens inside its gate/up kernel, more in the router kernel): the expert
     ids must equal the oracle's, whose ties go to the lower expert index."""
     if path != "default":
-        monkeypatch.setenv("W1_MOE_PATH", path)
+        knob("moe_path", path)
     run_and_check(T, 512, 256, 16, 4, 9, ties=True)
     run_and_check(min(T, 3), 512, 256, 16, 4, 10, ties=True)

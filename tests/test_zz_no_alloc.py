@@ -23,7 +23,9 @@ pytestmark = pytest.mark.gpu
 
 def test_noalloc_matches_workspace_entry_point_twice():
     lib = _lib.load()
-    for seed, (m, r, n, B) in [(0, (4096, 4096, 4096, 8)), (1, (1000, 640, 1152, 5))]:
+    # B = 20: three groups of up to 8 rows through the one static array in
+    # sequence (the barrier count and the intermediate are reused)
+    for seed, (m, r, n, B) in [(0, (4096, 4096, 4096, 8)), (1, (1000, 640, 1152, 5)), (2, (1000, 640, 1152, 20))]:
         case = synth.dbf_case(m=m, r=r, n=n, B=B, seed=40 + seed)
         a, B1, mid, B2, b, x = case
         dv = [fp16_dev(a), words_dev(B1), fp16_dev(mid), words_dev(B2), fp16_dev(b), bf16_dev(x)]
