@@ -42,8 +42,8 @@ GEMM_SHAPES = [(14336, 4096), (4096, 14336), (14336, 14336)]
 GEMM_M = 2048
 WORKLOAD = ("decode GEMV sweep: (out x in) 4096x4096, 11008x4096, 4096x11008 at B = 1, 4, 8; "
             "1-bit signs + fp16 scale per 128 weights; x bf16 N(0,1); W N(0,0.02)")
-KERNEL_OF_CHOICE = {"direct": "gemv_direct_kernel", "direct16": "gemv_direct_kernel", "tc": "gemv_tc_kernel",
-                    "ring": "gemv_kernel"}
+KERNEL_OF_CHOICE = {"flat": "gemv_flat_kernel", "flat16": "gemv_flat_kernel", "direct": "gemv_direct_kernel",
+                    "direct16": "gemv_direct_kernel", "tc": "gemv_tc_kernel", "ring": "gemv_kernel"}
 # DRAM bytes per launch from ncu captures (dram__bytes_read.sum + write), with the
 # shape captured; see profiles/.  Used to report the dominant kernel's traffic.
 CAPTURED_TRAFFIC = {
@@ -629,24 +629,90 @@ def measure_rows(torch, ops, synth, peaks, iters: int = 5):
             "g128_gaussian_4096": {"rel_frobenius": round((se / sw) ** 0.5, 5), "rel_spectral": round(rel_spec, 5)}}
 
 
-def cpu_oracle_gemv_sample(combos_spec, packed_host, max_seconds: float = 20.0):
-    """Time the fp64 oracle on the sweep (one launch per pair) on the host."""
+def cpu_oracle_sweep(max_pack_rows: int | None = None):
+    """The fp64 oracle on the whole decode GEMV sweep on the host cores: each
+    shape's weights packed by the oracle (pack_ref_fast), then one product per
+    (shape, batch) pair, every pair at full size.  Phases timed separately:
+    pack, dequantise (dequant_ref) and the whole product call (matmul_ref, which
+    dequantises again, multiplies and forms the tolerance scale).  Returns the
+    packed bytes processed, the per-phase seconds and the per-pair rows."""
     from oracle import w1_oracle as O
     from pack_sign_g128_b200 import synth
-    t_total = 0.0
-    b_total = 0
-    done = []
-    for (N, K, B) in combos_spec:
-        s, c = packed_host[(N, K)]
-        x = O.bf16_bits_to_f64(synth.activations_bf16(synth.rng(100 + B), B, K))
+    rows = []
+    t_pack = t_deq = t_prod = 0.0
+    nbytes = 0
+    for (N, K) in GEMV_SHAPES:
+        W, _ = synth.gemv_case(N, K, 1)
+        if max_pack_rows is not None:
+            W = W[:max_pack_rows]
+        n_rows = W.shape[0]
         t0 = time.perf_counter()
-        O.matmul_ref(x, s, c, K)
-        t_total += time.perf_counter() - t0
-        b_total += packed_bytes(N, K)
-        done.append(f"{N}x{K}xB{B}")
-        if t_total > max_seconds:
-            break
-    return b_total, t_total, done
+        s, c = O.pack_ref_fast(W)
+        tp = time.perf_counter() - t0
+        t_pack += tp
+        for B in GEMV_BATCHES:
+            x = O.bf16_bits_to_f64(synth.activations_bf16(synth.rng(100 + B), B, K))
+            t0 = time.perf_counter()
+            O.dequant_ref(s, c, K)
+            td = time.perf_counter() - t0
+            t0 = time.perf_counter()
+            O.matmul_ref(x, s, c, K)
+            tm = time.perf_counter() - t0
+            t_deq += td
+            t_prod += tm
+            nbytes += packed_bytes(n_rows, K)
+            rows.append({"N": n_rows, "K": K, "B": B, "dequant_s": round(td, 4), "matmul_ref_s": round(tm, 4),
+                         "GB/s": round(packed_bytes(n_rows, K) / tm / 1e9, 5)})
+    return nbytes, {"pack_s": round(t_pack, 3), "dequant_s": round(t_deq, 3), "matmul_ref_s": round(t_prod, 3)}, rows
+
+
+def cpu_oracle_rows(budget_s: float = 40.0):
+    """The oracle on the other configurations, full size, in order, until the
+    time budget is spent (rows not reached are listed as skipped): prefill
+    GEMM per shape (dequantise + fp64 BLAS product + tolerance scale), the
+    routed MoE layer, the DBF chain 4096^3 at B = 512."""
+    from oracle import w1_oracle as O
+    from pack_sign_g128_b200 import synth
+    out = {"gemm": [], "moe": None, "dbf": None, "skipped": []}
+    spent = 0.0
+    for (N, K) in GEMM_SHAPES:
+        if spent > budget_s:
+            out["skipped"].append(f"gemm {N}x{K}")
+            continue
+        W, x = synth.gemm_case(GEMM_M, N, K)
+        s, c = O.pack_ref_fast(W)
+        del W
+        xf = O.bf16_bits_to_f64(x)
+        t0 = time.perf_counter()
+        O.matmul_ref(xf, s, c, K)
+        t = time.perf_counter() - t0
+        spent += t
+        out["gemm"].append({"M": GEMM_M, "N": N, "K": K, "matmul_ref_s": round(t, 3),
+                            "TFLOP/s": round(2.0 * GEMM_M * N * K / t / 1e12, 5)})
+    if spent <= budget_s:
+        T, H, I, E, k = MOE["T"], MOE["H"], MOE["I"], MOE["E"], MOE["top_k"]
+        x, logits, gate, up, down = synth.moe_case(T=T, H=H, I=I, E=E)
+        pk = []
+        for Wt in (gate, up, down):
+            s_, c_ = O.pack_ref_fast(Wt.reshape(-1, Wt.shape[-1]))
+            pk.append((s_.reshape(E, Wt.shape[1], -1), c_.reshape(E, Wt.shape[1], -1)))
+        t0 = time.perf_counter()
+        O.moe_ref(O.bf16_bits_to_f64(x), logits, pk[0], pk[1], pk[2], H, I, E, k)
+        t = time.perf_counter() - t0
+        spent += t
+        out["moe"] = {"T": T, "s": round(t, 3), "tokens/s": round(T / t, 2)}
+    else:
+        out["skipped"].append("moe")
+    if spent <= budget_s:
+        a, B1, mid, B2, b, x = synth.dbf_case(m=4096, r=4096, n=4096, B=512)
+        t0 = time.perf_counter()
+        O.dbf_ref(a, B1, mid, B2, b, O.bf16_bits_to_f64(x), 4096, 4096, 4096)
+        t = time.perf_counter() - t0
+        spent += t
+        out["dbf"] = {"B": 512, "s": round(t, 3), "TFLOP/s": round(2.0 * 512 * 2 * 4096 ** 2 / t / 1e12, 5)}
+    else:
+        out["skipped"].append("dbf B=512")
+    return out
 
 
 def blas_threads() -> int:
@@ -761,16 +827,15 @@ def run_gpu(args):
         rows["measure"] = measure_rows(torch, ops, synth, peaks)
     cpu = None
     if rank == 0 and world == 1 and not args.skip_cpu:
-        packed_host = {}
-        for cb in combos:
-            key = (cb["N"], cb["K"])
-            if key not in packed_host:
-                packed_host[key] = (cb["signs"][0].cpu().numpy().view(np.uint32),
-                                    cb["scales"][0].cpu().view(torch.int16).numpy().view(np.uint16))
-        spec = [(cb["N"], cb["K"], cb["B"]) for cb in combos]
-        nb, secs, done = cpu_oracle_gemv_sample(spec, packed_host)
+        nb, phases, cpu_pairs = cpu_oracle_sweep()
+        secs = phases["matmul_ref_s"]
         cpu = {"value": nb / secs / 1e9, "unit": "GB/s", "cores": blas_threads(), "kind": "oracle",
-               "sample": f"fp64 numpy oracle (dequantise + BLAS matmul), one product per pair: {', '.join(done)}"}
+               "sample": "fp64 numpy oracle on the whole sweep: every (shape, batch) pair once at full size "
+                         "(weights packed by the oracle, pack time reported apart); value = packed bytes / "
+                         "seconds of matmul_ref (dequantise + fp64 BLAS product + tolerance scale)",
+               "phases": phases, "pairs": cpu_pairs}
+        if not args.skip_extra:
+            rows["cpu"] = cpu_oracle_rows()
 
     out = {
         "metric": METRIC,
@@ -818,24 +883,25 @@ def run_reference(args):
         return
     from oracle import w1_oracle as O
     from pack_sign_g128_b200 import synth
-    # bounded sample: 512 output rows of each shape, every batch
-    rows_per = 512
+    # each step: the whole sweep, every (shape, batch) pair once at full size;
+    # the oracle packs each shape's weights once, before the timed steps
     packed = {}
     for (N, K) in GEMV_SHAPES:
         W, _ = synth.gemv_case(N, K, 1)
-        packed[(N, K)] = O.pack_ref_fast(W[:rows_per])
+        packed[(N, K)] = O.pack_ref_fast(W)
+        del W
     spec = [(N, K, B) for (N, K) in GEMV_SHAPES for B in GEMV_BATCHES]
+    xs = {(K, B): O.bf16_bits_to_f64(synth.activations_bf16(synth.rng(100 + B), B, K)) for (_, K, B) in spec}
 
     def one_step():
         t = 0.0
         nbytes = 0
         for (N, K, B) in spec:
             s, c = packed[(N, K)]
-            x = O.bf16_bits_to_f64(synth.activations_bf16(synth.rng(100 + B), B, K))
             t0 = time.perf_counter()
-            O.matmul_ref(x, s, c, K)
+            O.matmul_ref(xs[(K, B)], s, c, K)
             t += time.perf_counter() - t0
-            nbytes += packed_bytes(rows_per, K)
+            nbytes += packed_bytes(N, K)
         return nbytes, t
 
     for _ in range(args.warmup):
@@ -847,7 +913,8 @@ def run_reference(args):
         nb += b
         secs += t
     value = nb / secs / 1e9
-    sample = f"fp64 numpy oracle, first {rows_per} rows of each sweep shape at B = 1, 4, 8"
+    sample = ("fp64 numpy oracle (matmul_ref: dequantise + BLAS product + tolerance scale), every sweep pair "
+              "once per step at full size; weights packed by the oracle before the timed steps")
     out = {
         "impl": "reference",
         "metric": METRIC,

@@ -81,6 +81,22 @@ bool make_tmap_u32_rows(CUtensorMap* map, const void* base, int64_t rows, int64_
   return r == CUDA_SUCCESS;
 }
 
+// 2-D uint32 tensor map over row-major sign words [rows][words]: box {32 words
+// (8 groups of 128 weights), box_rows}, 128-byte swizzle, zero fill out of
+// bounds (rows past N, words past K / 32).
+bool make_tmap_u32_sw128(CUtensorMap* map, const void* base, int64_t rows, int64_t words, int box_rows) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn || box_rows < 1 || box_rows > 256) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(words), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(words) * 4};
+  cuuint32_t box[2] = {32, static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 size_t gemm_workspace_bytes(int64_t M, int64_t K) {
   const size_t xs_bytes = (static_cast<size_t>(M) * K * 2 + 1023) / 1024 * 1024;
   return xs_bytes + (static_cast<size_t>(M) * 4 + 255) / 256 * 256;

@@ -311,6 +311,9 @@ static cudaError_t launch_gemv_nb(const uint32_t* signs, const GemvParams& base,
 
 cudaError_t launch_gemv_tc(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t K, const uint16_t* x,
                            int B, float* y, bool static_weights, cudaStream_t stream, int num_sms, int force_s);
+cudaError_t launch_gemv_flat(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t K, const uint16_t* x,
+                             int B, float* y, bool static_weights, cudaStream_t stream, int num_sms, int smem_cap,
+                             int split, int warps);
 cudaError_t launch_gemv_direct(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t K,
                                const void* x, bool x_f32, int B, float* y, bool static_weights,
                                cudaStream_t stream, int num_sms, int smem_cap, int force_s, int warps);
@@ -367,9 +370,9 @@ static cudaError_t launch_gemv_ring(const uint32_t* signs, const uint16_t* scale
 // knob; a forced kernel whose plan does not fit fails with W1_ERR_UNSUPPORTED).
 namespace {
 struct GemvChoice {
-  char kind;  // 'd' direct, 't' tcgen05, 'm' ring
-  int s;      // forced K split, 0 = the kernel's planner
-  int w;      // direct kernel: warps per CTA (8 or 16)
+  char kind;  // 'f' fp8 (gemv_flat.cu), 'd' direct, 't' tcgen05, 'm' ring
+  int s;      // forced K split, 0 = the kernel's planner (flat: 1)
+  int w;      // flat and direct kernels: warps per CTA (8 or 16)
 };
 struct GemvChoiceEntry {
   int dev;
@@ -390,6 +393,9 @@ static cudaError_t run_gemv_choice(const GemvChoice& c, const uint32_t* signs, c
                                    int num_sms, int smem_cap, bool static_weights) {
   const uint16_t* xb = static_cast<const uint16_t*>(x);
   switch (c.kind) {
+    case 'f':
+      if (xf) return cudaErrorNotSupported;
+      return launch_gemv_flat(signs, scales, N, K, xb, B, y, static_weights, stream, num_sms, smem_cap, c.s, c.w);
     case 'd':
       return launch_gemv_direct(signs, scales, N, K, x, xf, B, y, static_weights, stream, num_sms, smem_cap, c.s,
                                 c.w);
@@ -402,11 +408,17 @@ static cudaError_t run_gemv_choice(const GemvChoice& c, const uint32_t* signs, c
   }
 }
 
-// The static rule with fallbacks (direct or tcgen05 first by batch, then ring).
-// With fp32 activations only the direct kernel applies: 8 warps, then 16.
+// The static rule with fallbacks: bf16 activations the fp8 kernel (8 warps,
+// no split), then direct or tcgen05 by batch, then ring; fp32 activations
+// only the direct kernel: 8 warps, then 16.
 static cudaError_t run_gemv_rule(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t K,
                                  const void* x, bool xf, int B, float* y, cudaStream_t stream, int num_sms,
                                  int smem_cap, bool static_weights) {
+  if (!xf) {
+    const cudaError_t ef = run_gemv_choice(GemvChoice{'f', 0, 8}, signs, scales, N, K, x, xf, B, y, stream, num_sms,
+                                           smem_cap, static_weights);
+    if (ef != cudaErrorNotSupported) return ef;
+  }
   const GemvChoice first = (B <= 4 || xf) ? GemvChoice{'d', 0, 8} : GemvChoice{'t', 0, 0};
   const GemvChoice second = xf ? GemvChoice{'d', 0, 16} : (B <= 4 ? GemvChoice{'t', 0, 0} : GemvChoice{'d', 0, 8});
   cudaError_t e =
@@ -465,7 +477,10 @@ cudaError_t launch_gemv(const uint32_t* signs, const uint16_t* scales, int64_t N
   if (const int path = knob(kKnobGemvPath)) {
     // fp32 activations run the direct kernel whatever the knob names.
     const bool direct = path == kGemvDirect8 || path == kGemvDirect16 || xf;
-    const GemvChoice c{direct ? 'd' : (path == kGemvTc ? 't' : 'm'), 0, path == kGemvDirect16 ? 16 : 8};
+    const bool flat = path == kGemvFlat || path == kGemvFlat16;
+    const int split = knob(kKnobGemvSplit);
+    const GemvChoice c{direct ? 'd' : (flat ? 'f' : (path == kGemvTc ? 't' : 'm')), flat ? split : 0,
+                       (path == kGemvDirect16 || path == kGemvFlat16) ? 16 : 8};
     return run_gemv_choice(c, signs, scales, N, K, x, xf, B, y, stream, num_sms, smem_cap, static_weights);
   }
   int dev = 0;
@@ -486,8 +501,9 @@ cudaError_t launch_gemv(const uint32_t* signs, const uint16_t* scales, int64_t N
   if (cap != cudaStreamCaptureStatusNone || knob(kKnobGemvAutotune) == 0)
     return run_gemv_rule(signs, scales, N, K, x, xf, B, y, stream, num_sms, smem_cap, static_weights);
 
-  const GemvChoice cands[] = {{'d', 1, 8},  {'d', 2, 8},  {'d', 4, 8},  {'d', 8, 8}, {'d', 1, 16},
-                              {'d', 2, 16}, {'d', 4, 16}, {'d', 8, 16}, {'t', 0, 0}, {'m', 0, 0}};
+  const GemvChoice cands[] = {{'f', 1, 8},  {'f', 2, 8},  {'f', 4, 8},  {'f', 1, 16}, {'f', 2, 16}, {'f', 4, 16},
+                              {'d', 1, 8},  {'d', 2, 8},  {'d', 4, 8},  {'d', 8, 8},  {'d', 1, 16}, {'d', 2, 16},
+                              {'d', 4, 16}, {'d', 8, 16}, {'t', 0, 0},  {'m', 0, 0}};
   constexpr int kTimed = 12;
   // A private stream, ordered after the caller's work so far, takes the
   // captures (the caller's stream is not captured or reordered).
@@ -516,7 +532,7 @@ cudaError_t launch_gemv(const uint32_t* signs, const uint16_t* scales, int64_t N
   // The candidates run on one weight matrix that stays in L2, which flatters
   // the kernels least sensitive to memory latency; the static rule's kernel
   // is kept unless another is more than 5% faster.
-  const char rule_kind = (B <= 4 || xf) ? 'd' : 't';
+  const char rule_kind = xf ? 'd' : 'f';
   GemvChoice best{0, 0, 0}, best_rule{0, 0, 0};
   float best_ms = 0.f, best_rule_ms = 0.f;
   cudaError_t fatal = cudaSuccess;
@@ -573,14 +589,15 @@ static int gemv_choice_name(int64_t N, int64_t K, int B, bool st, char* out, siz
       if (e.dev == dev && e.N == N && e.K == K && e.B == B && e.st == st && !e.xf) c = e.c;
     }
   }
-  const char* kind = c.kind == 'd' ? (c.w == 16 ? "direct16" : "direct")
-                                    : (c.kind == 't' ? "tc" : (c.kind == 'm' ? "ring" : ""));
+  const char* kind = c.kind == 'f'   ? (c.w == 16 ? "flat16" : "flat")
+                     : c.kind == 'd' ? (c.w == 16 ? "direct16" : "direct")
+                                     : (c.kind == 't' ? "tc" : (c.kind == 'm' ? "ring" : ""));
   if (c.kind == 0) return snprintf(out, out_len, "%s", "");
   return snprintf(out, out_len, "%s/%d", kind, c.s);
 }
 
-// Parses "direct/<s>", "direct16/<s>", "tc/<s>", "ring/<s>" (w1_gemv_choice's
-// notation); false for anything else.
+// Parses "flat/<s>", "flat16/<s>", "direct/<s>", "direct16/<s>", "tc/<s>",
+// "ring/<s>" (w1_gemv_choice's notation); false for anything else.
 static bool parse_gemv_choice(const char* name, GemvChoice* c) {
   const char* slash = strchr(name, '/');
   if (!slash) return false;
@@ -589,7 +606,10 @@ static bool parse_gemv_choice(const char* name, GemvChoice* c) {
   const long sp = strtol(slash + 1, &end, 10);
   if (end == slash + 1 || *end != '\0' || sp < 0 || sp > 8) return false;
   auto is = [&](const char* k) { return strlen(k) == len && strncmp(name, k, len) == 0; };
-  if (is("direct") || is("direct16")) {
+  if (is("flat") || is("flat16")) {
+    if (sp != 1 && sp != 2 && sp != 4 && sp != 8) return false;
+    *c = GemvChoice{'f', static_cast<int>(sp), is("flat16") ? 16 : 8};
+  } else if (is("direct") || is("direct16")) {
     if (sp != 1 && sp != 2 && sp != 4 && sp != 8) return false;
     *c = GemvChoice{'d', static_cast<int>(sp), is("direct16") ? 16 : 8};
   } else if (is("tc")) {

@@ -411,18 +411,19 @@ namespace w1 {
 enum KnobId { kKnobGemvPath, kKnobGemvSplit, kKnobGemvAutotune, kKnobMoePath, kKnobDbfPath, kKnobDbfWarps,
               kKnobVerbose, kKnobCount };
 // GEMV kernels a knob can force (also the kinds of the dispatcher's choices).
-enum GemvPathKnob { kGemvAuto = 0, kGemvDirect8 = 1, kGemvDirect16 = 2, kGemvTc = 3, kGemvRing = 4, kGemvFlat = 5 };
+enum GemvPathKnob { kGemvAuto = 0, kGemvDirect8 = 1, kGemvDirect16 = 2, kGemvTc = 3, kGemvRing = 4, kGemvFlat = 5,
+                    kGemvFlat16 = 6 };
 enum DbfPathKnob { kDbfAuto = 0, kDbfFused = 1, kDbfTwoStep = 2 };
 
 struct KnobSpec {
   const char* name;  // w1_set_knob name
   const char* env;   // environment variable read at first use
   int dflt;
-  const char* words[6];  // accepted words for values 1..6 (else an integer)
+  const char* words[7];  // accepted words for values 1..7 (else an integer)
 };
 inline const KnobSpec& knob_spec(int id) {
   static const KnobSpec specs[kKnobCount] = {
-      {"gemv_path", "W1_GEMV_PATH", 0, {"direct", "direct16", "tc", "ring", "flat", nullptr}},
+      {"gemv_path", "W1_GEMV_PATH", 0, {"direct", "direct16", "tc", "ring", "flat", "flat16", nullptr}},
       {"gemv_split", "W1_GEMV_SPLIT", 0, {nullptr}},
       {"gemv_autotune", "W1_GEMV_AUTOTUNE", 1, {nullptr}},
       {"moe_path", "W1_MOE_PATH", 0, {"tiles", "decode", nullptr}},
@@ -436,7 +437,7 @@ inline const KnobSpec& knob_spec(int id) {
 // integer.  Returns false for anything else.
 inline bool parse_knob(int id, const char* v, int* out) {
   const KnobSpec& s = knob_spec(id);
-  for (int i = 0; i < 6 && s.words[i]; ++i)
+  for (int i = 0; i < 7 && s.words[i]; ++i)
     if (strcmp(v, s.words[i]) == 0) {
       *out = i + 1;
       return true;

@@ -1,7 +1,8 @@
 """w1_gemv on the GPU vs the fp64 oracle (element-wise, 1e-3 * sum|s x| bound).
 
-Every test runs on each kernel, forced with the gemv_path knob: the direct
-kernel with 8 and with 16 warps per CTA (direct / direct16), the tcgen05
+Every test runs on each kernel, forced with the gemv_path knob: the fp8 kernel
+with 8 and with 16 warps per CTA (flat / flat16, bf16 activations), the
+int8 direct kernel with 8 and 16 warps (direct / direct16), the tcgen05
 kernel (tc) and the mma.sync ring kernel (ring, the fallback for other
 shapes)."""
 import functools
@@ -17,7 +18,7 @@ from gpu_helpers import assert_within, bf16_dev, fp16_dev, words_dev
 pytestmark = pytest.mark.gpu
 
 
-@pytest.fixture(autouse=True, params=["direct", "direct16", "tc", "ring"])
+@pytest.fixture(autouse=True, params=["flat", "flat16", "direct", "direct16", "tc", "ring"])
 def gemv_path(request, knob):
     knob("gemv_path", request.param)
     return request.param
@@ -113,11 +114,11 @@ def test_gemv_is_deterministic():
 @pytest.mark.parametrize("N,K,B", [(4096, 4096, 1), (1000, 1152, 5), (4097, 2176, 8), (300, 1024, 2),
                                    (4096, 11008, 8)])
 def test_gemv_direct_every_split(N, K, B, split, gemv_path, knob):
-    """The direct kernel's cluster K split (1..8 CTAs) on the same inputs.
-    4096 x 11008 at B = 8 needs the reduction buffer over the activation
-    scratch at 16 warps and small splits."""
-    if not gemv_path.startswith("direct"):
-        pytest.skip("split sweep is for the direct kernel")
+    """The cluster K split (1..8 CTAs) of the fp8 and direct kernels on the
+    same inputs.  4096 x 11008 at B = 8 needs the direct kernel's reduction
+    buffer over the activation scratch at 16 warps and small splits."""
+    if not (gemv_path.startswith("direct") or gemv_path.startswith("flat")):
+        pytest.skip("split sweep is for the split-capable kernels")
     knob("gemv_split", split)
     W, x = synth.gemv_case(N, K, B, seed=N + B)
     s, c = O.pack_ref_fast(W)
