@@ -59,7 +59,8 @@ typedef enum {
   W1_ERR_TIMEOUT = 7,     /* device: a bounded wait gave up                      */
   W1_ERR_WORKSPACE = 8,   /* workspace missing or too small                      */
   W1_ERR_UNSUPPORTED = 9, /* current device is not sm_100 (B200 class)           */
-  W1_ERR_TOO_LARGE = 10   /* sizes exceed dbf_apply_noalloc's static scratch     */
+  W1_ERR_TOO_LARGE = 10,  /* sizes exceed dbf_apply_noalloc's static scratch     */
+  W1_ERR_NOT_CONVERGED = 11 /* device: an iterative solve hit its iteration limit */
 } w1_status;
 
 /* Static, human-readable name of a status code. */
@@ -243,6 +244,39 @@ int w1_residual(const float* W, int64_t N, int64_t K, const uint32_t* signs, con
 int dbf_residual(const float* W, const uint16_t* a, const uint32_t* B1, const uint16_t* mid, const uint32_t* B2,
                  const uint16_t* b, int64_t m, int64_t r, int64_t n, float* E, double* sums, void* workspace,
                  size_t ws_bytes, w1_stream_t stream);
+
+/*
+ * dbf_reproject_mid -- least-squares refit of the DBF middle diagonal ("LLM
+ * binarization episode 01: DBF", section 1.2 "What we inherit from DBF": one
+ * final linear least-squares reprojection of the middle diagonal, the signs
+ * and the outer scalers held fixed).  With P_k = (a * U[:, k]) (V[k, :] * b)^T
+ * (U, V the +-1 matrices of B1, B2; a, b as in dbf_apply), the minimiser of
+ * ||W - sum_k mid_k P_k||_F solves G mid = c with
+ *   G_kl = (U^T diag(a^2) U)_kl (V diag(b^2) V^T)_kl,  c_k = <W, P_k>.
+ * G and c are formed in fp64 (G exactly while the partial sums of the a^2 and
+ * b^2 terms span under 2^53: for fp16 diagonals in [0.01, 0.3] and m, n <=
+ * 65536, always); the system is solved by conjugate gradients in fp64 from
+ * mid = 0, which for a singular G converges to the minimum-norm solution
+ * (what least squares gives).  Model-conversion work, not per-token work.
+ *   W fp32 [m][n]; a fp16 [m]; B1 [m][r/32]; B2 [r][n/32]; b fp16 [n]
+ *     (device, read only).  1 <= m <= 2^24; r, n multiples of 128;
+ *     r <= 16384; n <= 2^24; else W1_ERR_SHAPE.
+ *   max_iter: iteration limit (0 <= max_iter <= 2^30); tol: stop when
+ *     ||c - G mid||_2 <= tol ||c||_2 (tol >= 0; 1e-13 is enough for fp16
+ *     output).  Reaching max_iter first records W1_ERR_NOT_CONVERGED in the
+ *     device status word and keeps the last iterate.
+ *   mid: fp16 [r] out, the solution rounded once to nearest-even (an
+ *     overflow to inf records W1_ERR_RANGE).  mid64: fp64 [r] out, or NULL.
+ *   info: device int[2] out, or NULL: iterations taken, converged (1) or not.
+ *   workspace: device, >= dbf_reproject_mid_workspace_size(m, r, n) bytes
+ *     (8 r^2 for G plus O(m r / 16 + n r / 8)), 16-byte aligned.
+ * Every sum has a fixed order: results are bitwise reproducible for a shape
+ * on a device.  Uses a cooperative launch (one CTA per SM at most).
+ */
+size_t dbf_reproject_mid_workspace_size(int64_t m, int64_t r, int64_t n);
+int dbf_reproject_mid(const float* W, const uint16_t* a, const uint32_t* B1, const uint32_t* B2, const uint16_t* b,
+                      int64_t m, int64_t r, int64_t n, int64_t max_iter, double tol, uint16_t* mid, double* mid64,
+                      int* info, void* workspace, size_t ws_bytes, w1_stream_t stream);
 
 /*
  * w1_power_iteration -- spectral norm estimate of A (fp32 [m][n], n a

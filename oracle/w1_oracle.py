@@ -324,10 +324,11 @@ def dbf_reproject_mid_ref(W, a_bits, B1_words, B2_words, b_bits, m: int, r: int,
     Qv = V * b[None, :]           # rows q_k
     G = (Pu.T @ Pu) * (Qv @ Qv.T)
     c = np.einsum("ik,ij,kj->k", Pu, W, Qv)
-    try:
-        mid = np.linalg.solve(G, c)
-    except np.linalg.LinAlgError:
-        mid = np.linalg.lstsq(G, c, rcond=None)[0]
+    # least squares on the normal equations (SVD, numpy's default cutoff):
+    # G^-1 c for a nonsingular G, the minimum-norm solution for a singular
+    # one -- an LU solve would return an arbitrary split between dependent
+    # P_k whenever rounding hides an exact singularity from the pivoting
+    mid = np.linalg.lstsq(G, c, rcond=None)[0]
     bits = np.array([round_to_fp16_bits(Fraction(abs(v))) | (0x8000 if v < 0 else 0) for v in mid], dtype=np.uint16)
     return mid, bits
 

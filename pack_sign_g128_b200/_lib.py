@@ -14,11 +14,12 @@ LIB_PATH = os.path.join(_HERE, "libw1.so")
 W1_STATUS = {
     0: "W1_OK", 1: "W1_ERR_NULL", 2: "W1_ERR_SHAPE", 3: "W1_ERR_ALIGN", 4: "W1_ERR_NONFINITE",
     5: "W1_ERR_RANGE", 6: "W1_ERR_CUDA", 7: "W1_ERR_TIMEOUT", 8: "W1_ERR_WORKSPACE",
-    9: "W1_ERR_UNSUPPORTED", 10: "W1_ERR_TOO_LARGE",
+    9: "W1_ERR_UNSUPPORTED", 10: "W1_ERR_TOO_LARGE", 11: "W1_ERR_NOT_CONVERGED",
 }
 W1_OK, W1_ERR_NULL, W1_ERR_SHAPE, W1_ERR_ALIGN, W1_ERR_NONFINITE = 0, 1, 2, 3, 4
 W1_ERR_RANGE, W1_ERR_CUDA, W1_ERR_TIMEOUT, W1_ERR_WORKSPACE, W1_ERR_UNSUPPORTED = 5, 6, 7, 8, 9
 W1_ERR_TOO_LARGE = 10
+W1_ERR_NOT_CONVERGED = 11
 
 _p = ctypes.c_void_p
 _i64 = ctypes.c_int64
@@ -47,6 +48,9 @@ SIGNATURES = {
     "w1_residual": (_int, [_p, _i64, _i64, _p, _p, _p, _p, _p, _sz, _p]),
     "dbf_residual": (_int, [_p, _p, _p, _p, _p, _p, _i64, _i64, _i64, _p, _p, _p, _sz, _p]),
     "w1_power_iteration": (_int, [_p, _i64, _i64, _p, _i64, _p, _p, _sz, _p]),
+    "dbf_reproject_mid_workspace_size": (_sz, [_i64, _i64, _i64]),
+    "dbf_reproject_mid": (_int, [_p, _p, _p, _p, _p, _i64, _i64, _i64, _i64, ctypes.c_double, _p, _p, _p, _p, _sz,
+                                 _p]),
     "w1_okt_gemv": (_int, [_p, _p, _i64, _i64, _p, _i64, _p, _i64, _p, _i64, _p, _p, ctypes.c_uint32, _p]),
 }
 

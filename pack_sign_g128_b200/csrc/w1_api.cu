@@ -36,6 +36,12 @@ cudaError_t launch_dbf(const uint16_t* a, const uint32_t* B1, const uint16_t* mi
                        float* y, void* workspace, cudaStream_t stream, int num_sms, int smem_cap,
                        bool allow_tensor_path);
 size_t dbf_workspace_bytes(int64_t m, int64_t r, int64_t n, int64_t B);
+bool reproject_shape_ok(int64_t m, int64_t r, int64_t n);
+size_t reproject_workspace_bytes(int64_t m, int64_t r, int64_t n);
+cudaError_t launch_reproject_mid(const float* W, const uint16_t* a, const uint32_t* B1, const uint32_t* B2,
+                                 const uint16_t* b, int64_t m, int64_t r, int64_t n, int max_iter, double tol,
+                                 uint16_t* mid, double* mid64, int* info, void* workspace, cudaStream_t stream,
+                                 int num_sms);
 
 struct DeviceInfo {
   bool ok = false;
@@ -99,6 +105,7 @@ const char* w1_status_string(int status) {
     case W1_ERR_WORKSPACE: return "W1_ERR_WORKSPACE: workspace missing or too small";
     case W1_ERR_UNSUPPORTED: return "W1_ERR_UNSUPPORTED: device is not sm_100";
     case W1_ERR_TOO_LARGE: return "W1_ERR_TOO_LARGE: sizes exceed the static scratch of dbf_apply_noalloc";
+    case W1_ERR_NOT_CONVERGED: return "W1_ERR_NOT_CONVERGED: the iterative solve stopped at its iteration limit";
     default: return "unknown w1 status";
   }
 }
@@ -178,6 +185,24 @@ int w1_residual(const float* W, int64_t N, int64_t K, const uint32_t* signs, con
   if (st != W1_OK) return st;
   return launch_result(launch_residual_g128(W, N, K, signs, scales, E, sums, workspace,
                                             reinterpret_cast<cudaStream_t>(stream), d.sms));
+}
+
+size_t dbf_reproject_mid_workspace_size(int64_t m, int64_t r, int64_t n) { return reproject_workspace_bytes(m, r, n); }
+
+int dbf_reproject_mid(const float* W, const uint16_t* a, const uint32_t* B1, const uint32_t* B2, const uint16_t* b,
+                      int64_t m, int64_t r, int64_t n, int64_t max_iter, double tol, uint16_t* mid, double* mid64,
+                      int* info, void* workspace, size_t ws_bytes, w1_stream_t stream) {
+  if (!W || !a || !B1 || !B2 || !b || !mid) return W1_ERR_NULL;
+  if (!reproject_shape_ok(m, r, n) || max_iter < 0 || max_iter > (int64_t(1) << 30) || !(tol >= 0.0)) return W1_ERR_SHAPE;
+  if (!workspace || ws_bytes < reproject_workspace_bytes(m, r, n)) return W1_ERR_WORKSPACE;
+  if (!aligned16(W) || !aligned16(a) || !aligned16(B1) || !aligned16(B2) || !aligned16(b) || !aligned16(mid) ||
+      (mid64 && !aligned16(mid64)) || (info && !aligned8(info)) || !aligned16(workspace))
+    return W1_ERR_ALIGN;
+  DeviceInfo d;
+  int st = device_info(&d);
+  if (st != W1_OK) return st;
+  return launch_result(launch_reproject_mid(W, a, B1, B2, b, m, r, n, static_cast<int>(max_iter), tol, mid, mid64,
+                                            info, workspace, reinterpret_cast<cudaStream_t>(stream), d.sms));
 }
 
 int dbf_residual(const float* W, const uint16_t* a, const uint32_t* B1, const uint16_t* mid, const uint32_t* B2,

@@ -194,6 +194,34 @@ def dbf_residual(W: torch.Tensor, a: torch.Tensor, B1: torch.Tensor, mid: torch.
     return (E if want_E else None), sums
 
 
+def dbf_reproject_workspace_size(m: int, r: int, n: int) -> int:
+    return int(_lib.fn("dbf_reproject_mid_workspace_size")(m, r, n))
+
+
+def dbf_reproject_mid(W: torch.Tensor, a: torch.Tensor, B1: torch.Tensor, B2: torch.Tensor, b: torch.Tensor,
+                      max_iter: int = 200, tol: float = 1e-13, workspace: torch.Tensor | None = None, stream=None):
+    """Least-squares middle diagonal for fixed signs and outer scalers:
+    (mid fp16 [r], mid fp64 [r], info int32 [2] = iterations, converged)."""
+    m, n = W.shape
+    r = B1.shape[1] * 32
+    if W.dtype != torch.float32:
+        raise TypeError("W must be float32")
+    if a.shape[0] != m or b.shape[0] != n or B1.shape[0] != m or tuple(B2.shape) != (r, n // 32):
+        raise ValueError("DBF operands do not match W's shape")
+    mid = torch.empty(r, dtype=torch.float16, device=W.device)
+    mid64 = torch.empty(r, dtype=torch.float64, device=W.device)
+    info = torch.zeros(2, dtype=torch.int32, device=W.device)
+    need = dbf_reproject_workspace_size(m, r, n)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=W.device)
+    st = _lib.fn("dbf_reproject_mid")(_ptr(W), _ptr(a), _ptr(B1), _ptr(B2), _ptr(b), m, r, n, max_iter, tol,
+                                      _ptr(mid), _ptr(mid64), _ptr(info), _ptr(workspace), workspace.numel(),
+                                      _stream(stream, W))
+    if st != _lib.W1_OK:
+        raise _lib.W1Error(st, "dbf_reproject_mid")
+    return mid, mid64, info
+
+
 def w1_power_iteration(A: torch.Tensor, v0: torch.Tensor, iters: int = 32, workspace: torch.Tensor | None = None,
                        stream=None) -> torch.Tensor:
     """Spectral norm estimate of A fp32 [m, n] (fp64 scalar tensor on the device)."""

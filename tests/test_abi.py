@@ -46,7 +46,8 @@ def test_status_strings(lib):
 def test_knobs_accept_their_words_and_reject_the_rest(lib):
     ok = [("gemv_path", "direct"), ("gemv_path", "direct16"), ("gemv_path", "tc"), ("gemv_path", "ring"),
           ("gemv_path", "flat"), ("gemv_split", "4"), ("gemv_autotune", "0"), ("moe_path", "tiles"),
-          ("moe_path", "decode"), ("dbf_path", "fused"), ("dbf_path", "twostep"), ("dbf_warps", "16"),
+          ("moe_path", "decode"), ("moe_path", "grouped"), ("dbf_path", "fused"), ("dbf_path", "twostep"), ("dbf_warps", "16"),
+          ("dbf_rank_split", "4"),
           ("verbose", "1")]
     try:
         for name, value in ok:
@@ -176,6 +177,36 @@ def test_measure_host_side_argument_errors(lib):
     assert pi(good, 64, 64, good, -1, good, good, ws, None) == _lib.W1_ERR_SHAPE
     assert pi(good, 64, 64, good, 32, good, None, ws, None) == _lib.W1_ERR_WORKSPACE
     assert pi(odd, 64, 64, good, 32, good, good, ws, None) == _lib.W1_ERR_ALIGN
+
+
+def test_reproject_host_side_argument_errors(lib):
+    good = ctypes.c_void_p(1 << 20)
+    odd = ctypes.c_void_p((1 << 20) + 4)
+    ws = lib.dbf_reproject_mid_workspace_size(256, 128, 384)
+    assert ws >= 8 * 128 * 128
+    assert lib.dbf_reproject_mid_workspace_size(256, 100, 384) == 0
+    assert lib.dbf_reproject_mid_workspace_size(256, 16384 + 128, 384) == 0
+    assert lib.dbf_reproject_mid_workspace_size(0, 128, 384) == 0
+    f = lib.dbf_reproject_mid
+    ops5 = [good] * 5
+
+    def call(*, W=good, m=256, r=128, n=384, it=50, tol=1e-13, mid=good, mid64=None, info=None, wsp=good, wsb=ws):
+        return f(W, *ops5[1:], m, r, n, it, tol, mid, mid64, info, wsp, wsb, None)
+
+    assert call(W=None) == _lib.W1_ERR_NULL
+    assert call(mid=None) == _lib.W1_ERR_NULL
+    assert call(r=100) == _lib.W1_ERR_SHAPE
+    assert call(n=200) == _lib.W1_ERR_SHAPE
+    assert call(m=0) == _lib.W1_ERR_SHAPE
+    assert call(r=16384 + 128) == _lib.W1_ERR_SHAPE
+    assert call(it=-1) == _lib.W1_ERR_SHAPE
+    assert call(tol=-1.0) == _lib.W1_ERR_SHAPE
+    assert call(tol=float("nan")) == _lib.W1_ERR_SHAPE
+    assert call(wsp=None) == _lib.W1_ERR_WORKSPACE
+    assert call(wsb=ws - 1) == _lib.W1_ERR_WORKSPACE
+    assert call(W=odd) == _lib.W1_ERR_ALIGN
+    assert call(mid64=odd) == _lib.W1_ERR_ALIGN
+    assert call(info=ctypes.c_void_p((1 << 20) + 2)) == _lib.W1_ERR_ALIGN
 
 
 def test_binding_shape_checks_run_before_any_device_work():

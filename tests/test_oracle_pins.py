@@ -620,6 +620,30 @@ def test_reproject_matches_lstsq_on_the_explicit_design_matrix():
     assert np.max(np.abs(X.T @ res)) <= 1e-9 * np.max(np.abs(X.T @ W.ravel()))
 
 
+def test_reproject_singular_design_takes_the_minimum_norm_solution():
+    """Two equal columns of U and the matching two equal rows of V make
+    P_k1 = P_k2: the least-squares minimiser is not unique, and the one of
+    minimum norm (what lstsq on the explicit m n x r design matrix returns)
+    splits the weight evenly between k1 and k2."""
+    m, r, n = 32, 32, 64
+    a, B1, _, B2, b = _dbf_factors(m, r, n, 86)
+    k1, k2 = 3, 20
+    U = O.unpack_bits_lsb_first(B1, r).astype(np.uint8)
+    U[:, k2] = U[:, k1]
+    B1 = np.packbits(U, axis=1, bitorder="little").view(np.uint32).reshape(m, r // 32)
+    B2 = B2.copy()
+    B2[k2] = B2[k1]
+    W = synth.weights(synth.rng(87), m, n, std=0.05).astype(np.float64)
+    av, bv = O.fp16_bits_to_f64(a), O.fp16_bits_to_f64(b)
+    Us = 1.0 - 2.0 * U
+    Vs = 1.0 - 2.0 * O.unpack_bits_lsb_first(B2, n)
+    X = np.stack([np.outer(av * Us[:, k], Vs[k] * bv).ravel() for k in range(r)], axis=1)
+    ref = np.linalg.lstsq(X, W.ravel(), rcond=None)[0]
+    got, _ = O.dbf_reproject_mid_ref(W, a, B1, B2, b, m, r, n)
+    assert abs(ref[k1] - ref[k2]) <= 1e-12 * np.max(np.abs(ref))
+    assert np.max(np.abs(got - ref)) <= 1e-9 * np.max(np.abs(ref))
+
+
 def test_reproject_is_optimal_and_bits_round_to_nearest():
     """Random perturbations of the solution raise the error; the stored bits
     are numpy's round-to-nearest fp16 of the solution."""
