@@ -8,10 +8,14 @@
 // section 1 "The representation" and section 4: x_scaled = D_in x,
 // h = V x_scaled, h_scaled = D_mid h, y_core = U h_scaled, y = D_out y_core).
 //
-// Small batch (B < 64, groups of up to 8 rows): ONE kernel runs both binary
-// products -- the joint V-D_mid-U kernel with a grid-wide synchronisation that
-// the DBF post (section 7, "CUDA/HIP: a starting point") proposes for CUDA --
-// built from the steps of the direct GEMV kernel (gemv_direct.cu).  Each CTA
+// Small batch (B < 64, groups of up to 8 rows), two forms chosen by the group
+// size (both from the steps of the direct GEMV kernel, gemv_direct.cu):
+//  * up to 2 rows: two launches, h_scaled = mid (.) (V . (b (.) x)) into the
+//    workspace, then y = a (.) (U . h_scaled) (its K split over r is the
+//    pages' "split rank", section 5 item 5);
+//  * from 3 rows: ONE kernel runs both binary products -- the joint
+//    V-D_mid-U kernel with a grid-wide synchronisation that the DBF post
+//    (section 7, "CUDA/HIP: a starting point") proposes for CUDA.  Each CTA
 //  1. issues the asynchronous copies of its slices of BOTH sign matrices at
 //     once (two commit groups), so U streams in while V . (b x) is computed;
 //  2. phase 1: int8-MMA product of V with b (.) x (the column diagonal applied
@@ -277,6 +281,10 @@ cudaError_t launch_dbf_tc(const uint16_t* a, const uint32_t* B1, const uint16_t*
                           const uint16_t* b, int64_t m, int64_t r, int64_t n, const uint16_t* x, int64_t B, float* y,
                           void* workspace, cudaStream_t stream, int num_sms);
 
+cudaError_t launch_gemv_direct_diag(const uint32_t* signs, int64_t N, int64_t K, const void* x, bool x_f32,
+                                    const uint16_t* cdiag, const uint16_t* rdiag, int B, float* y, bool early,
+                                    cudaStream_t stream, int num_sms, int smem_cap, int warps, int force_s);
+
 // Batches of at least this many rows run on the tensor-core path.
 constexpr int64_t kDbfTensorMinBatch = 64;
 
@@ -303,6 +311,7 @@ cudaError_t launch_dbf(const uint16_t* a, const uint32_t* B1, const uint16_t* mi
   // for groups of up to 3 rows, 16 above (as measured).  The dbf_warps knob
   // forces 8 or 16.
   const int wknob = knob(kKnobDbfWarps);
+  const int pknob = knob(kKnobDbfPath);  // 0: default, 1: fused, 2: two launches
   const int im = static_cast<int>(m), ir = static_cast<int>(r), in = static_cast<int>(n);
   for (int64_t b0 = 0; b0 < B; b0 += 8) {
     const int nb = static_cast<int>((B - b0) < 8 ? (B - b0) : 8);
@@ -310,6 +319,29 @@ cudaError_t launch_dbf(const uint16_t* a, const uint32_t* B1, const uint16_t* mi
     float* yg = y + b0 * m;
     const bool w16 = wknob ? wknob == 16 : nb >= 4;
     cudaError_t err;
+    // Default form by the measured A/B on the 4096^3 chain (graphs of
+    // back-to-back calls): two launches are faster up to 2 rows per group
+    // (8.1 vs 11.1 us at 1 row, 11.6 vs 14.6 at 2), the fused kernel from 3
+    // rows on (14.9 vs 17.3 at 4, 17.9 vs 20.9 at 8, with the best rank
+    // split for the two launches).
+    const bool two = pknob ? pknob == kDbfTwoStep : nb <= 2;
+    if (two) {
+      // Two launches of the direct GEMV core ("LLM binarization episode 01:
+      // DBF", section 4: x_scaled = D_in x, h = V x_scaled, h_scaled = D_mid
+      // h, then y = D_out (U h_scaled)): h_scaled in fp32 through the
+      // workspace; U may be read before the first launch completes (that
+      // launch writes only h).  The second product contracts over r: its
+      // K split is the split-rank form of section 5 item 5 (r partitioned
+      // over the CTAs of a cluster, partial outputs added in a fixed order
+      // through distributed shared memory); dbf_rank_split forces it.
+      const int warps = wknob ? wknob : (nb >= 4 ? 16 : 8);
+      err = launch_gemv_direct_diag(B2, r, n, xg, false, b, mid, nb, h, false, stream, num_sms, smem_cap, warps, 0);
+      if (err == cudaSuccess)
+        err = launch_gemv_direct_diag(B1, m, r, h, true, nullptr, a, nb, yg, true, stream, num_sms, smem_cap, warps,
+                                      knob(kKnobDbfRankSplit));
+      if (err != cudaSuccess) return err;
+      continue;
+    }
     switch (nb) {
 #define W1_DBF_CASE(NBV)                                                                                   \
   case NBV:                                                                                                \

@@ -82,6 +82,7 @@ struct GdParams {
   const void* x;           // [B][K] bf16, or fp32 with x_f32
   const uint16_t* cdiag;   // fp16 [K] multiplied into x (bf16 x only), or nullptr
   const uint16_t* rdiag;   // fp16 [N] multiplied into y, or nullptr
+  const int* xrows;        // batch row b reads row xrows[b] of x (nullptr: row b)
   float* y;                // [B][N]
   int x_f32;
   int N, K, NG;
@@ -422,14 +423,15 @@ __device__ __forceinline__ void gd_load_unit(const GdParams& p, const GdGeom& g,
     const int gi = (g.cs0 + sl) * G + gj;
     if (gi < p.NG) {
       const int64_t k0 = static_cast<int64_t>(gi) * 128 + sub * 16;
+      const int64_t xr = p.xrows ? p.xrows[b] : b;
       if (XF32) {
         const uint4* src =
-            reinterpret_cast<const uint4*>(static_cast<const float*>(p.x) + static_cast<int64_t>(b) * p.K + k0);
+            reinterpret_cast<const uint4*>(static_cast<const float*>(p.x) + xr * p.K + k0);
 #pragma unroll
         for (int i = 0; i < 4; ++i) r[i] = __ldcg(src + i);
       } else {
         const uint4* src =
-            reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.x) + static_cast<int64_t>(b) * p.K + k0);
+            reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.x) + xr * p.K + k0);
         r[0] = __ldg(src);
         r[1] = __ldg(src + 1);
         if (p.cdiag) {
@@ -868,6 +870,33 @@ cudaError_t launch_gemv_direct(const uint32_t* signs, const uint16_t* scales, in
   p.early = static_weights ? 1 : 0;
   // A 16-warp CTA never shares an SM with the next launch's CTA (registers),
   // so its plans may use up to twice the shared memory cap of 8-warp plans.
+  if (warps == 16)
+    return launch_gemv_direct_nw<16>(p, B, stream, num_sms, std::min(2 * smem_cap, 200 * 1024), force_s);
+  return launch_gemv_direct_nw<8>(p, B, stream, num_sms, smem_cap, force_s);
+}
+
+// One product with diagonals and no group scales (a step of the DBF chain):
+// y[b][row] = rdiag[row] * sum_k s(row, k) * cdiag[k] * x[b][k], cdiag only
+// for bf16 x (nullptr: none).  early: the sign words were not written by the
+// kernel this launch follows (they may be read before its grid dependency
+// wait).  force_s: CTAs per cluster splitting K (0 = planner).  Same
+// planning and kernels as launch_gemv_direct.
+cudaError_t launch_gemv_direct_diag(const uint32_t* signs, int64_t N, int64_t K, const void* x, bool x_f32,
+                                    const uint16_t* cdiag, const uint16_t* rdiag, int B, float* y, bool early,
+                                    cudaStream_t stream, int num_sms, int smem_cap, int warps, int force_s) {
+  if (N > (int64_t)1 << 30 || K > (int64_t)1 << 30 || (x_f32 && cdiag)) return cudaErrorNotSupported;
+  GdParams p = {};
+  p.signs = signs;
+  p.scales = nullptr;
+  p.x = x;
+  p.y = y;
+  p.x_f32 = x_f32 ? 1 : 0;
+  p.cdiag = cdiag;
+  p.rdiag = rdiag;
+  p.N = static_cast<int>(N);
+  p.K = static_cast<int>(K);
+  p.NG = static_cast<int>(K / 128);
+  p.early = early ? 1 : 0;
   if (warps == 16)
     return launch_gemv_direct_nw<16>(p, B, stream, num_sms, std::min(2 * smem_cap, 200 * 1024), force_s);
   return launch_gemv_direct_nw<8>(p, B, stream, num_sms, smem_cap, force_s);

@@ -63,7 +63,7 @@ struct Cfg {
   static constexpr int NCOL = BF ? NB : 3 * NB;  // result columns per row
   static constexpr int MAXT = 8;                 // 16-row tiles per CTA (R <= 128)
   static constexpr int UPL = 2;                  // int8 form: activation units per lane and pass
-  static constexpr int GW = (BF ? 8 : 4) * 64;   // fragment-buffer words per group (MMA steps x 32 lanes x 2)
+  static constexpr int GW = BF ? 0 : 4 * 64;     // int8 form: digit words per group (4 MMAs x 32 lanes x 2)
 };
 }  // namespace fl
 
@@ -209,27 +209,15 @@ __device__ __forceinline__ void fl_quantise_unit(const uint4 (&r)[2], bool store
   }
 }
 
-// bf16 form: this lane's B pairs of batch row b = lane/4 for one group --
-// elements (m, m+16) and (m+8, m+24) of word cq for MMA step m -- into the
-// group's fragment buffer [m][lane] (uint2), from the 32 activation values of
-// word cq (16 bf16x2 words X).
-__device__ __forceinline__ void fl_stage_bf16(const uint4 (&xv)[4], uint2* frag, int lane) {
-  const uint32_t X[16] = {xv[0].x, xv[0].y, xv[0].z, xv[0].w, xv[1].x, xv[1].y, xv[1].z, xv[1].w,
-                          xv[2].x, xv[2].y, xv[2].z, xv[2].w, xv[3].x, xv[3].y, xv[3].z, xv[3].w};
-#pragma unroll
-  for (int m = 0; m < 8; ++m) {
-    const uint32_t sel = (m & 1) ? 0x7632u : 0x5410u;
-    frag[m * 32 + lane] = make_uint2(prmt(X[m / 2], X[8 + m / 2], sel), prmt(X[4 + m / 2], X[12 + m / 2], sel));
-  }
-}
-
 // The warp's products over its groups for all T tiles of the CTA's rows,
 // then (after a CTA barrier: the reduction buffer overlays the fragment
 // buffers) its partial sums into red[warp][row][col].
-//  1. The activations of all the warp's groups go to its fragment buffer in
-//     MMA order (int8: quantised digits; bf16: the values, permuted).
+//  1. int8 form: the activations of all the warp's groups are quantised into
+//     its digit buffer in MMA fragment order.
 //  2. Groups run GI at a time (GI T <= 8 accumulator chains), MMA steps
-//     outermost, so consecutive MMAs never depend on each other.
+//     outermost, so consecutive MMAs never depend on each other; the bf16
+//     form builds its B pairs from activations held in registers, the next
+//     block's loads in flight.
 // acc[t][e][c]: partial sum of row 16 t + lane/4 + 8 e, result column
 // 2 (lane%4) + c (int8: digit column 3b + d, bf16: batch row).
 // `prologue` is the grid dependency wait and what must follow it.
@@ -240,36 +228,19 @@ __device__ __forceinline__ void fl_products(const FlParams& p, int row0, int g0,
                                             Prologue&& prologue) {
   using C = fl::Cfg<NB>;
   constexpr int STEPS = C::BF ? 8 : 4;            // MMAs per group and tile
-  constexpr int GI = 8 / T >= 4 ? 4 : (8 / T >= 2 ? 2 : 1);  // groups per block
+  // groups per block: GI T <= 8 accumulator chains; the bf16 form also holds
+  // two blocks' activations in registers (16 words per group), so it takes at
+  // most 2 groups, 1 with 16 warps
+  constexpr int GI0 = 8 / T >= 4 ? 4 : (8 / T >= 2 ? 2 : 1);
+  constexpr int GI = C::BF ? (NW == 16 ? 1 : (GI0 > 2 ? 2 : GI0)) : GI0;
   float acc[T][2][2];
 #pragma unroll
   for (int t = 0; t < T; ++t) acc[t][0][0] = acc[t][0][1] = acc[t][1][0] = acc[t][1][1] = 0.f;
   bool ok = true;
   const int r1 = lane >> 2, cq = lane & 3;
   prologue();
-  // ---- 1. activations -> fragment buffer
-  if constexpr (C::BF) {
-    // lane (r1, cq): batch row r1's elements of word cq, every group of the
-    // warp, up to 4 groups' loads in flight at once
-    constexpr int XG = 4;
-    for (int gl = 0; gl < nwg; gl += XG) {
-      uint4 xv[XG][4];
-#pragma unroll
-      for (int g = 0; g < XG; ++g) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) xv[g][i] = make_uint4(0, 0, 0, 0);
-        if (r1 < NB && gl + g < nwg) {
-          const uint4* src = reinterpret_cast<const uint4*>(
-              p.x + static_cast<int64_t>(r1) * p.K + static_cast<int64_t>(g0 + wg0 + gl + g) * 128 + 32 * cq);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) xv[g][i] = __ldg(src + i);
-        }
-      }
-#pragma unroll
-      for (int g = 0; g < XG; ++g)
-        if (gl + g < nwg) fl_stage_bf16(xv[g], reinterpret_cast<uint2*>(dig + (gl + g) * C::GW), lane);
-    }
-  } else {
+  // ---- 1. int8 form: activations -> digit fragments in shared memory
+  if constexpr (!C::BF) {
     const int U = nwg * NB * 8;
     constexpr int UPL = C::UPL;
     uint4 xr[UPL][2];
@@ -309,6 +280,23 @@ __device__ __forceinline__ void fl_products(const FlParams& p, int row0, int g0,
     cw[c] = cd[c] == 0 ? 131072.f : (cd[c] == 1 ? 512.f : (cd[c] == 2 ? 2.f : 0.f));  // 2 W_d
   }
   // ---- 2. products, GI groups at a time
+  // bf16 form: lane (r1, cq) holds batch row r1's 32 elements of word cq of
+  // each group of a block (16 bf16x2 words), the next block's loads in flight
+  auto load_x = [&](int gb, uint4 (&xv)[GI][4]) {
+#pragma unroll
+    for (int g = 0; g < GI; ++g) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) xv[g][i] = make_uint4(0, 0, 0, 0);
+      if (C::BF && r1 < NB && gb + g < nwg) {
+        const uint4* src = reinterpret_cast<const uint4*>(
+            p.x + static_cast<int64_t>(r1) * p.K + static_cast<int64_t>(g0 + wg0 + gb + g) * 128 + 32 * cq);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) xv[g][i] = __ldg(src + i);
+      }
+    }
+  };
+  uint4 xcur[GI][4], xnext[GI][4];
+  if constexpr (C::BF) load_x(0, xcur);
   int waited = -1;  // highest box this warp has waited for
   for (int gb = 0; gb < nwg; gb += GI) {
     // sign words of the block's groups: rows 16 t + r1 (+8), word cq, from the
@@ -331,6 +319,7 @@ __device__ __forceinline__ void fl_products(const FlParams& p, int row0, int g0,
       }
     }
     const int ng = min(GI, nwg - gb);
+    if constexpr (C::BF) load_x(gb + GI, xnext);
     using Acc = typename std::conditional<C::BF, float, int>::type;
     Acc cc[GI][T][4];
 #pragma unroll
@@ -341,8 +330,19 @@ __device__ __forceinline__ void fl_products(const FlParams& p, int row0, int g0,
       constexpr int m = decltype(mc)::value;
       uint2 bb[GI];
 #pragma unroll
-      for (int g = 0; g < GI; ++g)
-        bb[g] = g < ng ? reinterpret_cast<const uint2*>(dig + (gb + g) * C::GW)[m * 32 + lane] : make_uint2(0, 0);
+      for (int g = 0; g < GI; ++g) {
+        if constexpr (C::BF) {
+          // elements (m, m+16) and (m+8, m+24) of the lane's word as the B pairs
+          const uint32_t X[16] = {xcur[g][0].x, xcur[g][0].y, xcur[g][0].z, xcur[g][0].w,
+                                  xcur[g][1].x, xcur[g][1].y, xcur[g][1].z, xcur[g][1].w,
+                                  xcur[g][2].x, xcur[g][2].y, xcur[g][2].z, xcur[g][2].w,
+                                  xcur[g][3].x, xcur[g][3].y, xcur[g][3].z, xcur[g][3].w};
+          constexpr uint32_t sel = (m & 1) ? 0x7632u : 0x5410u;
+          bb[g] = make_uint2(prmt(X[m / 2], X[8 + m / 2], sel), prmt(X[4 + m / 2], X[12 + m / 2], sel));
+        } else {
+          bb[g] = g < ng ? reinterpret_cast<const uint2*>(dig + (gb + g) * C::GW)[m * 32 + lane] : make_uint2(0, 0);
+        }
+      }
 #pragma unroll
       for (int g = 0; g < GI; ++g)
 #pragma unroll
@@ -406,6 +406,12 @@ __device__ __forceinline__ void fl_products(const FlParams& p, int row0, int g0,
         }
       }
     }
+    if constexpr (C::BF) {
+#pragma unroll
+      for (int g = 0; g < GI; ++g)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) xcur[g][k] = xnext[g][k];
+    }
   }
   if (threadIdx.x < 32 && nwg == 0) fl_wait(sbar);  // the copy completes inside the CTA's lifetime
   __syncthreads();  // every warp is done with the fragment buffers the reduction overlays
@@ -452,25 +458,18 @@ __global__ void __launch_bounds__(NW * 32, 1) gemv_flat_kernel(const __grid_cons
     asm volatile("prefetch.tensormap [%0];" ::"l"(&tmap) : "memory");
   }
   __syncthreads();
-  // box b holds CTA-local groups [bs, bs + 8), bs = min(8 b, G - 8) (the last
-  // box overlaps its neighbour rather than reaching past the CTA's range)
+  // The weight copies.  Box b holds CTA-local groups [bs, bs + 8), bs =
+  // min(8 b, G - 8) (the last box overlaps its neighbour rather than reaching
+  // past the CTA's range).  The scale block [rows][NG] is contiguous: one bulk
+  // copy (a tail under 16 bytes, when rows * NG is not a multiple of 8, with
+  // plain loads before the barrier arrival).
   auto issue = [&]() {
-    if (threadIdx.x == 0)
+    if (threadIdx.x == 0) {
       for (int b = 0; b < nbox; ++b) {
         const int bs = G >= fl::kBoxG ? min(b * fl::kBoxG, G - fl::kBoxG) : 0;
         mbar_arrive_expect_tx(&bars[b], static_cast<uint32_t>(p.R * 128));
         tma_load_2d(smem + L.wts + b * p.R * 128, &tmap, (g0 + bs) * 4, row0, &bars[b]);
       }
-  };
-  if (p.early) issue();
-  // The grid dependency wait, then the scales: the scale block [rows][NG] is
-  // contiguous, one bulk copy (a tail under 16 bytes, when rows * NG is not a
-  // multiple of 8, with plain loads before the barrier arrival).
-  auto prologue = [&]() {
-    pdl_wait();
-    pdl_launch_dependents();
-    if (!p.early) issue();
-    if (threadIdx.x == 0) {
       const uint32_t sbytes = static_cast<uint32_t>(rows) * p.NG * 2;
       const uint32_t sbulk = sbytes & ~15u;
       const uint16_t* ssrc = p.scales + static_cast<int64_t>(row0) * p.NG;
@@ -480,6 +479,14 @@ __global__ void __launch_bounds__(NW * 32, 1) gemv_flat_kernel(const __grid_cons
         bulk_g2s(reinterpret_cast<unsigned char*>(scl) + off, reinterpret_cast<const unsigned char*>(ssrc) + off,
                  min(32768u, sbulk - off), &sbar);
     }
+  };
+  // The next launch in the stream may start now: its own grid dependency wait
+  // orders everything it reads or writes after this grid.
+  pdl_launch_dependents();
+  if (p.early) issue();
+  auto prologue = [&]() {
+    pdl_wait();
+    if (!p.early) issue();
   };
   // ---- this warp's groups [wg0, wg1) of the CTA's range
   const int wg0 = (warp * G) / NW, wg1 = ((warp + 1) * G) / NW, nwg = wg1 - wg0;

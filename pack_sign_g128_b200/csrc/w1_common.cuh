@@ -400,16 +400,17 @@ inline cudaError_t ensure_dyn_smem(const void* kernel, int bytes) {
 //   gemv_path     W1_GEMV_PATH      0 = dispatch, else a forced GEMV kernel
 //   gemv_split    W1_GEMV_SPLIT     forced K split of the split-capable GEMV kernels (0 = planner)
 //   gemv_autotune W1_GEMV_AUTOTUNE  0 = static rule instead of first-call timing
-//   moe_path      W1_MOE_PATH       0 = by token count, 1 = tiles, 2 = decode
+//   moe_path      W1_MOE_PATH       0 = by token count, 1 = tiles, 2 = decode, 3 = decode grouped by expert
 //   dbf_path      W1_DBF_PATH       0 = by batch, else a forced small-batch chain form
 //   dbf_warps     W1_DBF_WARPS      0 = by group size, 8 or 16 warps per CTA
+//   dbf_rank_split W1_DBF_RANK_SPLIT two-launch chain: CTAs per cluster that split r in U . h (0 = planner)
 //   verbose       W1_VERBOSE        nonzero: plans and choices on stderr
 #include <atomic>
 #include <cstdlib>
 #include <cstring>
 namespace w1 {
 enum KnobId { kKnobGemvPath, kKnobGemvSplit, kKnobGemvAutotune, kKnobMoePath, kKnobDbfPath, kKnobDbfWarps,
-              kKnobVerbose, kKnobCount };
+              kKnobDbfRankSplit, kKnobVerbose, kKnobCount };
 // GEMV kernels a knob can force (also the kinds of the dispatcher's choices).
 enum GemvPathKnob { kGemvAuto = 0, kGemvDirect8 = 1, kGemvDirect16 = 2, kGemvTc = 3, kGemvRing = 4, kGemvFlat = 5,
                     kGemvFlat16 = 6 };
@@ -426,9 +427,10 @@ inline const KnobSpec& knob_spec(int id) {
       {"gemv_path", "W1_GEMV_PATH", 0, {"direct", "direct16", "tc", "ring", "flat", "flat16", nullptr}},
       {"gemv_split", "W1_GEMV_SPLIT", 0, {nullptr}},
       {"gemv_autotune", "W1_GEMV_AUTOTUNE", 1, {nullptr}},
-      {"moe_path", "W1_MOE_PATH", 0, {"tiles", "decode", nullptr}},
+      {"moe_path", "W1_MOE_PATH", 0, {"tiles", "decode", "grouped", nullptr}},
       {"dbf_path", "W1_DBF_PATH", 0, {"fused", "twostep", nullptr}},
       {"dbf_warps", "W1_DBF_WARPS", 0, {nullptr}},
+      {"dbf_rank_split", "W1_DBF_RANK_SPLIT", 0, {nullptr}},
       {"verbose", "W1_VERBOSE", 0, {nullptr}},
   };
   return specs[id];

@@ -1,7 +1,8 @@
 """dbf_apply on the GPU vs the fp64 oracle chain.
 
-Every test runs with the fused small-batch chain kernel forced to 8 and to 16
-warps per CTA (the dbf_warps knob).  Batches of 64 and more take the
+Every test runs with each small-batch chain form -- the fused chain kernel and
+two launches of the direct GEMV core (the dbf_path knob) -- forced to 8 and to
+16 warps per CTA (the dbf_warps knob).  Batches of 64 and more take the
 tensor-core path either way."""
 import functools
 
@@ -16,9 +17,11 @@ from gpu_helpers import assert_within, bf16_dev, fp16_dev, words_dev
 pytestmark = pytest.mark.gpu
 
 
-@pytest.fixture(autouse=True, params=["fused8", "fused16"])
+@pytest.fixture(autouse=True, params=["fused8", "fused16", "twostep8", "twostep16"])
 def dbf_path(request, knob):
-    knob("dbf_warps", request.param[5:])
+    form, warps = (request.param[:-2], request.param[-2:]) if request.param.endswith("16") else (request.param[:-1], "8")
+    knob("dbf_path", form)
+    knob("dbf_warps", warps)
     return request.param
 
 
@@ -55,17 +58,25 @@ def test_dbf_config(B):
     check(synth.dbf_case(B=B), f"4096^3 B={B}")
 
 
-def test_dbf_config_batch512():
+def _tensor_path_once(dbf_path):
+    if dbf_path != "fused8":
+        pytest.skip("batches of 64 and more take the tensor-core path under every small-batch form")
+
+
+def test_dbf_config_batch512(dbf_path):
+    _tensor_path_once(dbf_path)
     check(synth.dbf_case(B=512), "4096^3 B=512")
 
 
 @pytest.mark.parametrize("m,r,n,B", [(300, 384, 256, 64), (4096, 1024, 2048, 200), (129, 128, 128, 65)])
-def test_dbf_tensor_path_ragged(m, r, n, B):
+def test_dbf_tensor_path_ragged(m, r, n, B, dbf_path):
+    _tensor_path_once(dbf_path)
     check(synth.dbf_case(m=m, r=r, n=n, B=B, seed=m + r + n + B), f"tensor path {m}x{r}x{n} B={B}")
 
 
-def test_dbf_tensor_path_extreme_scales():
+def test_dbf_tensor_path_extreme_scales(dbf_path):
     """Inputs spanning many binades: the per-row fp16 scalings must not overflow."""
+    _tensor_path_once(dbf_path)
     a, B1, mid, B2, b, x = synth.dbf_case(m=512, r=512, n=512, B=96, seed=77)
     xf = synth.normal_f32(synth.rng(78), (96, 512))
     xf[0] *= 1e30
@@ -108,9 +119,11 @@ def test_dbf_workspace_reuse_and_determinism():
     assert np.array_equal(y1, y2)
 
 
-def test_dbf_barrier_timeout_reports_status():
+def test_dbf_barrier_timeout_reports_status(dbf_path):
     """A barrier count that no arrival can complete: every CTA's bounded wait
     runs out, the call reports W1_ERR_TIMEOUT and the context stays usable."""
+    if dbf_path.startswith("twostep"):
+        pytest.skip("the two-launch form has no grid barrier")
     case = synth.dbf_case(m=256, r=256, n=256, B=1, seed=10)
     a, B1, mid, B2, b, x = case
     ws = ops.dbf_workspace(256, 256, 256, 1)
@@ -122,3 +135,19 @@ def test_dbf_barrier_timeout_reports_status():
     assert st == _lib.W1_OK
     ref = O.dbf_ref(a, B1, mid, B2, b, O.bf16_bits_to_f64(x), 256, 256, 256)
     assert_within(y, ref["y"], ref["bound"], what="after timeout")
+
+
+@pytest.mark.parametrize("split", [1, 2, 4, 8])
+@pytest.mark.parametrize("m,r,n,B", [(4096, 4096, 4096, 1), (1000, 640, 1152, 5), (512, 2048, 256, 8)])
+def test_dbf_twostep_rank_split(m, r, n, B, split, dbf_path, knob):
+    """The two-launch form with r split over 1-8 CTAs of a cluster in U . h
+    (DBF post, section 5 item 5, "Split rank"); splits whose plan does not
+    fit the shape report W1_ERR_UNSUPPORTED before any launch."""
+    if dbf_path != "twostep8":
+        pytest.skip("one form is enough: the split applies to the two-launch chain")
+    knob("dbf_rank_split", str(split))
+    case = synth.dbf_case(m=m, r=r, n=n, B=B, seed=m + r + n + B + split)
+    try:
+        check(case, f"{m}x{r}x{n} B={B} rank split {split}")
+    except _lib.W1Error as e:
+        assert e.status == _lib.W1_ERR_UNSUPPORTED and split > 1
