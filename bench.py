@@ -368,8 +368,8 @@ def gemm_rows(torch, ops, synth, peaks, iters: int = 8):
 
 
 MOE = dict(T=512, H=2048, I=1024, E=64, top_k=8)
-MOE_DECODE_T = (1, 4, 8)   # decode-regime batches (per-route products)
-DBF_BATCHES = [1, 8, 512]
+MOE_DECODE_T = (1, 4, 8, 16)   # decode-regime batches
+DBF_BATCHES = [1, 2, 4, 8, 512]
 
 
 def moe_rows(torch, ops, synth, peaks, iters: int = 8):
@@ -406,35 +406,56 @@ def moe_rows(torch, ops, synth, peaks, iters: int = 8):
     tf = flops / (ms * 1e-3) / 1e12
     row = {"T": T, "H": H, "I": I, "E": E, "top_k": K, "ms": ms, "tokens/s": T / (ms * 1e-3),
            "TFLOP/s": tf, "frac_bf16_burst": tf / peaks["bf16_tflops"], "launches_per_call": 7}
-    # decode regime: the first Td tokens of the same batch, a different token
-    # window per call, L2 flushed before each call; HBM-bound on the experts'
-    # packed weights that the call touches
+    # decode regime: Td tokens of the same batch, a different token window
+    # per call, each call one CUDA graph replay (no host time inside the
+    # events) after an L2 flush; HBM-bound on the experts' packed weights that
+    # the call touches.  Both decode forms: per-route products and the
+    # products grouped by expert (moe_path knob).
     per_expert = 3 * packed_bytes(I, H)  # gate, up (I x H) and down (H x I) have the same packed size
     ids_all = np.argsort(-logits, axis=1, kind="stable")[:, :K]
+    st = torch.cuda.Stream()
     decode = []
     for Td in MOE_DECODE_T:
         wsd = ops.moe_workspace(Td, H, I, E, K)
         outd = torch.empty((Td, H), dtype=torch.float32, device=dev)
-        windows = [(i * Td) % (T - Td + 1) for i in range(iters + 2)]
-        for w0 in windows[:2]:
-            ops.w1_moe_grouped(xd[w0:w0 + Td], ld[w0:w0 + Td], G, U, D, K, out=outd, workspace=wsd)
-        torch.cuda.synchronize()
-        tms, touched = [], []
-        for w0 in windows[2:]:
-            flush.zero_()
-            a = torch.cuda.Event(enable_timing=True)
-            b = torch.cuda.Event(enable_timing=True)
-            a.record()
-            ops.w1_moe_grouped(xd[w0:w0 + Td], ld[w0:w0 + Td], G, U, D, K, out=outd, workspace=wsd)
-            b.record()
-            torch.cuda.synchronize()
-            tms.append(a.elapsed_time(b))
-            touched.append(len(np.unique(ids_all[w0:w0 + Td])) * per_expert)
-        dms = statistics.median(tms)
-        gbs = float(np.mean(touched)) / (dms * 1e-3) / 1e9
-        decode.append({"T": Td, "us": round(dms * 1e3, 2), "tokens/s": round(Td / (dms * 1e-3), 1),
-                       "weight_GB/s": round(gbs, 1), "frac_hbm": round(gbs / peaks["hbm_gbs"], 4),
-                       "launches_per_call": 2 if Td <= 4 else 3})
+        windows = [(i * Td) % (T - Td + 1) for i in range(iters)]
+        touched = [len(np.unique(ids_all[w0:w0 + Td])) * per_expert for w0 in windows]
+        entry = {"T": Td}
+        for form in ("decode", "grouped"):
+            ops.set_knob("moe_path", form)
+            try:
+                call = lambda w0: ops.w1_moe_grouped(xd[w0:w0 + Td], ld[w0:w0 + Td], G, U, D, K, out=outd,
+                                                     workspace=wsd, stream=st)
+                with torch.cuda.stream(st):
+                    for w0 in windows[:2]:
+                        call(w0)
+                st.synchronize()
+                graphs = []
+                for w0 in windows:
+                    g = torch.cuda.CUDAGraph()
+                    with torch.cuda.graph(g, stream=st):
+                        call(w0)
+                    graphs.append(g)
+                tms = []
+                for g in graphs:
+                    with torch.cuda.stream(st):
+                        flush.zero_()
+                        a = torch.cuda.Event(enable_timing=True)
+                        b = torch.cuda.Event(enable_timing=True)
+                        a.record(st)
+                        g.replay()
+                        b.record(st)
+                    st.synchronize()
+                    tms.append(a.elapsed_time(b))
+                del graphs
+            finally:
+                ops.set_knob("moe_path", None)
+            dms = statistics.median(tms)
+            gbs = float(np.mean(touched)) / (dms * 1e-3) / 1e9
+            entry[form] = {"us": round(dms * 1e3, 2), "tokens/s": round(Td / (dms * 1e-3), 1),
+                           "weight_GB/s": round(gbs, 1), "frac_hbm": round(gbs / peaks["hbm_gbs"], 4),
+                           "launches_per_call": (2 if Td <= 4 else 3) if form == "decode" else 4}
+        decode.append(entry)
     row["decode"] = decode
     return row
 
@@ -464,28 +485,55 @@ def dbf_rows(torch, ops, synth, peaks, l2_bytes: int, iters: int = 5):
                 B1s[i] = B1s[0].clone()
                 B2s[i] = B2s[0].clone()
             st = torch.cuda.Stream()
-            with torch.cuda.stream(st):
-                for i in range(3):
-                    ops.dbf_apply(ad, B1s[i], md, B2s[i], bd, xd, y=y, workspace=ws)
-            st.synchronize()
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=st):
-                for i in range(R):
-                    ops.dbf_apply(ad, B1s[i], md, B2s[i], bd, xd, y=y, workspace=ws)
-            g.replay()
-            torch.cuda.synchronize()
-            e0 = torch.cuda.Event(enable_timing=True)
-            e1 = torch.cuda.Event(enable_timing=True)
-            e0.record()
-            for _ in range(iters):
+
+            def graph_us():
+                with torch.cuda.stream(st):
+                    for i in range(3):
+                        ops.dbf_apply(ad, B1s[i], md, B2s[i], bd, xd, y=y, workspace=ws)
+                st.synchronize()
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=st):
+                    for i in range(R):
+                        ops.dbf_apply(ad, B1s[i], md, B2s[i], bd, xd, y=y, workspace=ws)
                 g.replay()
-            e1.record()
-            torch.cuda.synchronize()
-            us = e0.elapsed_time(e1) * 1e3 / (iters * R)
+                torch.cuda.synchronize()
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record()
+                for _ in range(iters):
+                    g.replay()
+                e1.record()
+                torch.cuda.synchronize()
+                return e0.elapsed_time(e1) * 1e3 / (iters * R)
+
+            us = graph_us()
             gbs = alg_bytes / (us * 1e-6) / 1e9
-            rows.append({"B": B, "us_per_call": round(us, 3), "GB/s": round(gbs, 1),
-                         "frac_hbm": round(gbs / peaks["hbm_gbs"], 4), "calls": R})
-            del B1s, B2s, g
+            row = {"B": B, "us_per_call": round(us, 3), "GB/s": round(gbs, 1),
+                   "frac_hbm": round(gbs / peaks["hbm_gbs"], 4), "calls": R}
+            # the small-batch chain forms side by side (fused kernel vs two launches)
+            forms = {}
+            for form in ("fused", "twostep"):
+                ops.set_knob("dbf_path", form)
+                try:
+                    forms[form] = round(graph_us(), 3)
+                finally:
+                    ops.set_knob("dbf_path", None)
+            row["us_by_form"] = forms
+            # split rank: r partitioned over the CTAs of a cluster in U . h (two-launch form)
+            splits = {}
+            for sp in (1, 2, 4, 8):
+                ops.set_knob("dbf_path", "twostep")
+                ops.set_knob("dbf_rank_split", sp)
+                try:
+                    splits[str(sp)] = round(graph_us(), 3)
+                except RuntimeError:
+                    splits[str(sp)] = None  # no plan with this split for the shape
+                finally:
+                    ops.set_knob("dbf_path", None)
+                    ops.set_knob("dbf_rank_split", None)
+            row["us_twostep_by_rank_split"] = splits
+            rows.append(row)
+            del B1s, B2s
         else:
             B1d, B2d = tow(B1), tow(B2)
             flush = torch.empty(int(512 * 2 ** 20), dtype=torch.uint8, device=dev)
@@ -616,6 +664,31 @@ def measure_rows(torch, ops, synth, peaks, iters: int = 5):
     dbf_ms = timed(lambda: ops.dbf_residual(Wd, *dargs, want_E=False, workspace=ws))
     dbf_tf = 2.0 * m * n * r / (dbf_ms * 1e-3) / 1e12
     pi_ms = timed(lambda: ops.w1_power_iteration(Wd, v0, 32, workspace=ws))
+    # least-squares refit of the DBF middle diagonal against W (fp64 Grams,
+    # right-hand side and conjugate-gradient solve): 2 x m r^2 / 2 (symmetric
+    # Grams) + m n r multiply-adds
+    rws = torch.empty(ops.dbf_reproject_workspace_size(m, r, n), dtype=torch.uint8, device=dev)
+    rp_out = {}
+
+    def reproject():
+        rp_out["r"] = ops.dbf_reproject_mid(Wd, dargs[0], dargs[1], dargs[3], dargs[4], workspace=rws)
+
+    reproject()  # eager: one cooperative launch among a few plain ones, ~10 ms
+    st.synchronize()
+    rts = []
+    for _ in range(3):
+        with torch.cuda.stream(st):
+            flush.zero_()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(st)
+            reproject()
+            e1.record(st)
+        st.synchronize()
+        rts.append(e0.elapsed_time(e1))
+    rp_ms = statistics.median(rts)
+    rp_info = rp_out["r"][2].cpu().tolist()
+    rp_fma = m * r * r + m * n * r
     ops.w1_residual(Wd, signs, scales, E=E, workspace=ws)
     _, sums = ops.w1_residual(Wd, signs, scales, want_E=False, workspace=ws)
     se, sw = (float(v) for v in sums.cpu())
@@ -626,6 +699,8 @@ def measure_rows(torch, ops, synth, peaks, iters: int = 5):
             "dbf_residual": {"ms": round(dbf_ms, 4), "fp32_TFLOP/s": round(dbf_tf, 1),
                              "frac_fp32_cuda_core": round(dbf_tf / FP32_PEAK_TFLOPS, 4)},
             "power_iteration_32": {"ms": round(pi_ms, 4), "launches": 3 * 32 + 3},
+            "reproject_mid": {"ms": round(rp_ms, 4), "cg_iterations": rp_info[0], "converged": rp_info[1],
+                              "fp64_fma": rp_fma, "fp64_TFLOP/s": round(2.0 * rp_fma / (rp_ms * 1e-3) / 1e12, 2)},
             "g128_gaussian_4096": {"rel_frobenius": round((se / sw) ** 0.5, 5), "rel_spectral": round(rel_spec, 5)}}
 
 

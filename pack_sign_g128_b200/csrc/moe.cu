@@ -1077,6 +1077,284 @@ __global__ void __launch_bounds__(moed::kWarps * 32, 1) moe_decode_down_kernel(c
   }
 }
 
+// ------------------------------------------------------------------ decode regime, grouped by expert
+// "LLM binarization episode 01: DBF", section 7 item 1: with a few tokens,
+// products specialised to the observed expert counts, so that the tokens
+// routed to one expert read its packed weights once.  The list kernel routes
+// the tokens and groups the routes by expert (route order within an expert);
+// then one CTA per (expert, row block) stages the expert's rows once and runs
+// the direct GEMV steps with the expert's routes as its batch rows -- a
+// 1..8-row product chosen by the route count, 8 routes at a time above --
+// for gate/up (+ SwiGLU) and for down (x the route weight); the combine adds
+// each token's slots in slot order.
+namespace moeg {
+constexpr int kMaxT = 16;                     // tokens of the grouped decode path
+constexpr int kMaxR = kMaxT * moe::kMaxTopK;  // routes
+constexpr int kRowsD = 16 * moed::kWarps;     // down rows per CTA (16 per warp)
+constexpr int kRedCols = 24;                  // digit columns of an 8-row batch
+}  // namespace moeg
+
+struct MoeGroupList {
+  int* nexp;       // [1] experts with at least one route
+  int* exp_id;     // [E] expert of list slot i (ascending)
+  int* exp_cnt;    // [E] its route count
+  int* exp_start;  // [E] its first position in sroute
+  int* sroute;     // [R] routes grouped by expert, route order within an expert
+};
+
+// One CTA: warp t routes token t (the router's routine), then the routes are
+// counted per expert and listed.  pos[r] = r (the combine reads route rows).
+__global__ void __launch_bounds__(512) moe_decode_list_kernel(const float* __restrict__ logits, int T, int E,
+                                                              int top_k, int* __restrict__ ids,
+                                                              float* __restrict__ wts, int* __restrict__ pos,
+                                                              MoeGroupList gl) {
+  __shared__ int sid[moeg::kMaxR];
+  __shared__ float swt[moeg::kMaxR];
+  __shared__ int cnt[moe::kMaxE], start[moe::kMaxE];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int R = T * top_k;
+  pdl_wait();
+  if (warp < T)
+    moe_route_token(logits + static_cast<int64_t>(warp) * E, E, top_k, lane, sid + warp * top_k, swt + warp * top_k);
+  __syncthreads();
+  for (int r = threadIdx.x; r < R; r += blockDim.x) {
+    ids[r] = sid[r];
+    wts[r] = swt[r];
+    pos[r] = r;
+  }
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int c = 0;
+    for (int r = 0; r < R; ++r) c += sid[r] == e;
+    cnt[e] = c;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int st = 0, nl = 0;
+    for (int e = 0; e < E; ++e) {
+      start[e] = st;
+      if (cnt[e]) {
+        gl.exp_id[nl] = e;
+        gl.exp_cnt[nl] = cnt[e];
+        gl.exp_start[nl] = st;
+        ++nl;
+      }
+      st += cnt[e];
+    }
+    gl.nexp[0] = nl;
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    if (!cnt[e]) continue;
+    int j = start[e];
+    for (int r = 0; r < R; ++r)
+      if (sid[r] == e) gl.sroute[j++] = r;
+  }
+  pdl_launch_dependents();
+}
+
+// Shared memory of the grouped kernels: per-warp staged rows and scales (as
+// the batch-1 decode kernels), the activation digits for 8 batch rows, the
+// per-warp digit-column partials.
+struct MoeGroupLayout {
+  int warp_bytes, xs, red, total;
+};
+__host__ __device__ inline MoeGroupLayout moeg_layout(int NG, int P) {
+  const GdSmem L = gd_layout<1, moed::kWarps>(moed::kTw, NG, P, 1, 0, NG);
+  MoeGroupLayout M;
+  M.warp_bytes = L.warp_bytes;
+  M.xs = moed::kWarps * L.warp_bytes;
+  M.red = M.xs + (NG * gd::Cfg<8>::SCR * 4 + 15) / 16 * 16;
+  M.total = M.red + moed::kWarps * 16 * moeg::kRedCols * 4;
+  return M;
+}
+
+// One batch of NB routes of the CTA's expert: digits of the NB input rows
+// (p.xrows), every warp's products over its 16 rows and all of K, the digit
+// columns of each (row, route) summed -> emit(row in CTA, b, value).
+template <int NB, class Emit>
+__device__ __forceinline__ void moeg_batch(const GdParams& p, const GdGeom& g, const unsigned char* wts,
+                                           const float* scl, uint32_t* xs, float* red, int warp, int lane,
+                                           int rows_cta, Emit&& emit) {
+  using C = gd::Cfg<NB>;
+  uint4 xa[4];
+  gd_x_first<NB, false>(p, g, warp, lane, xa);
+  gd_prep_x<NB, false, moed::kWarps>(p, g, xs, warp, lane, xa);
+  __syncthreads();  // every unit's digits stored
+  float acc[gd::kMaxTp][C::NN][4];
+#pragma unroll
+  for (int tp = 0; tp < gd::kMaxTp; ++tp)
+#pragma unroll
+    for (int nn = 0; nn < C::NN; ++nn)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[tp][nn][e] = 0.f;
+  if (g.busy) gd_compute<NB, moed::kTw>(wts, p.P, scl, 8 * moed::kTw, xs, p.NG, lane, acc);
+  const int r1 = lane >> 2, cq = lane & 3;
+  float* rw = red + warp * 16 * moeg::kRedCols;
+#pragma unroll
+  for (int nn = 0; nn < C::NN; ++nn)
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      const int col = 8 * nn + 2 * cq + c;
+      if (col < C::NCOL) {
+        rw[r1 * moeg::kRedCols + col] = acc[0][nn][c];
+        rw[(r1 + 8) * moeg::kRedCols + col] = acc[0][nn][2 + c];
+      }
+    }
+  __syncthreads();
+  for (int o = threadIdx.x; o < rows_cta * NB; o += blockDim.x) {
+    const int i = o / NB, b = o - i * NB;
+    emit(i, b, red);
+  }
+  __syncthreads();  // digits and partials are rewritten by the next batch
+}
+
+// Rows of this warp inside the CTA's block, and its GEMV geometry.
+__device__ __forceinline__ GdGeom moeg_geom(int NG, int rows, int row0) {
+  GdGeom g = {};
+  g.nsc = NG;
+  g.tw = moed::kTw;
+  g.nsw = NG;
+  g.row0 = row0;
+  g.nrows = max(0, min(8 * moed::kTw, rows - row0));
+  g.busy = g.nrows > 0;
+  g.ngw = NG;
+  return g;
+}
+
+template <bool GATEUP>
+__global__ void __launch_bounds__(moed::kWarps * 32, 1) moe_decode_grouped_kernel(const MoeDecParams q,
+                                                                                  MoeGroupList gl,
+                                                                                  float* __restrict__ rout) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  __shared__ int xrow[8], route[8];
+  const MoeGroupLayout L = moeg_layout(q.NG, q.P);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  pdl_wait();
+  pdl_launch_dependents();
+  const int slot = blockIdx.y;
+  if (slot >= *gl.nexp) return;  // uniform over the CTA
+  const int e = gl.exp_id[slot], cnt = gl.exp_cnt[slot], st0 = gl.exp_start[slot];
+  // gate/up: warps 0-3 own 16 rows each of G_e, warps 4-7 the same rows of
+  // U_e (64 rows per CTA); down: warp w owns rows 16 w .. of the CTA's 128
+  const int mat = GATEUP ? warp >> 2 : 0;
+  const int rows_cta = GATEUP ? moed::kRowsGu : moeg::kRowsD;
+  const int row0 = blockIdx.x * rows_cta + (GATEUP ? (warp & 3) : warp) * 16;
+  GdParams p = {};
+  const int64_t mrow = static_cast<int64_t>(e) * q.rows;
+  p.signs = (mat ? q.signs1 : q.signs0) + mrow * (q.K >> 5);
+  p.scales = (mat ? q.scales1 : q.scales0) + mrow * q.NG;
+  p.x = q.x;
+  p.xrows = xrow;
+  p.N = q.rows;
+  p.K = q.K;
+  p.NG = q.NG;
+  p.Tw = moed::kTw;
+  p.NSw = q.NG;
+  p.P = q.P;
+  p.lgGw = q.lgGw;
+  const GdGeom g = moeg_geom(q.NG, q.rows, row0);
+  unsigned char* wreg = smem + warp * L.warp_bytes;
+  unsigned char* wts = wreg;
+  float* scl = reinterpret_cast<float*>(wreg + gd_layout<1, moed::kWarps>(moed::kTw, q.NG, q.P, 1, 0, q.NG).scl);
+  uint32_t* xs = reinterpret_cast<uint32_t*>(smem + L.xs);
+  float* red = reinterpret_cast<float*>(smem + L.red);
+  // the expert's rows, staged once for all its routes
+  uint16_t sreg[kGdSpl];
+  if (g.busy) gd_stage<1>(p, g, wts, lane);
+  else cp_async_commit();
+  gd_load_scales<1>(p, g, 0, lane, sreg);
+  gd_finish_scales<1>(p, g, lane, sreg, scl);
+  cp_async_wait_all();
+  for (int c0 = 0; c0 < cnt; c0 += 8) {
+    const int nb = min(8, cnt - c0);
+    if (threadIdx.x < nb) {
+      const int r = gl.sroute[st0 + c0 + threadIdx.x];
+      route[threadIdx.x] = r;
+      xrow[threadIdx.x] = GATEUP ? r / q.top_k : r;  // gate/up reads the token, down the route's h
+    }
+    __syncthreads();  // staged rows and scales, and the batch's rows, visible to all warps
+    auto emit = [&](int i, int b, const float* rd) {
+      const int row = blockIdx.x * rows_cta + i;
+      if (row >= q.rows) return;
+      if (GATEUP) {
+        const int wg = i >> 4, rr = i & 15;
+        const float* rg = rd + (wg * 16 + rr) * moeg::kRedCols + 3 * b;
+        const float* ru = rd + ((wg + 4) * 16 + rr) * moeg::kRedCols + 3 * b;
+        const float gv = (rg[0] + rg[1]) + rg[2], uv = (ru[0] + ru[1]) + ru[2];
+        q.h[static_cast<int64_t>(route[b]) * q.rows + row] = __float2bfloat16_rn(gv / (1.0f + expf(-gv)) * uv);
+      } else {
+        const float* rv = rd + i * moeg::kRedCols + 3 * b;
+        const int r = route[b];
+        rout[static_cast<int64_t>(r) * q.rows + row] = q.wts[r] * ((rv[0] + rv[1]) + rv[2]);
+      }
+    };
+    switch (nb) {  // uniform over the CTA
+      case 1: moeg_batch<1>(p, g, wts, scl, xs, red, warp, lane, rows_cta, emit); break;
+      case 2: moeg_batch<2>(p, g, wts, scl, xs, red, warp, lane, rows_cta, emit); break;
+      case 3: moeg_batch<3>(p, g, wts, scl, xs, red, warp, lane, rows_cta, emit); break;
+      case 4: moeg_batch<4>(p, g, wts, scl, xs, red, warp, lane, rows_cta, emit); break;
+      case 5: moeg_batch<5>(p, g, wts, scl, xs, red, warp, lane, rows_cta, emit); break;
+      case 6: moeg_batch<6>(p, g, wts, scl, xs, red, warp, lane, rows_cta, emit); break;
+      case 7: moeg_batch<7>(p, g, wts, scl, xs, red, warp, lane, rows_cta, emit); break;
+      default: moeg_batch<8>(p, g, wts, scl, xs, red, warp, lane, rows_cta, emit); break;
+    }
+  }
+}
+
+// The grouped decode layer: list, gate/up, down, combine (four launches).
+static cudaError_t launch_moe_decode_grouped(MoeDecParams q, int T, int H, int I, MoeGroupList gl,
+                                             const uint32_t* ds, const uint16_t* dc, float* rout, int* pos,
+                                             float* out, cudaStream_t stream, int num_sms) {
+  auto lg2 = [](int v) {
+    int l = 0;
+    while ((1 << l) < v) ++l;
+    return l;
+  };
+  cudaError_t err = launch_pdl(moe_decode_list_kernel, dim3(1), dim3(512), 0, stream, q.logits, T, q.E, q.top_k,
+                               q.ids, q.wts, pos, gl);
+  if (err != cudaSuccess) return err;
+  const unsigned slots = static_cast<unsigned>(q.E < q.R ? q.E : q.R);  // most experts a call can touch
+  // gate/up (+ SwiGLU): K = H, rows = I
+  MoeDecParams qg = q;
+  qg.rows = I;
+  qg.K = H;
+  qg.NG = H / 128;
+  qg.P = ((qg.NG & 1) ? qg.NG : qg.NG + 1) * 16;  // odd multiple of 16 bytes per staged row: bank spread
+  qg.lgGw = lg2(qg.NG);
+  int smem = moeg_layout(qg.NG, qg.P).total;
+  err = ensure_dyn_smem(reinterpret_cast<const void*>(moe_decode_grouped_kernel<true>), smem);
+  if (err != cudaSuccess) return err;
+  err = launch_pdl(moe_decode_grouped_kernel<true>,
+                   dim3(static_cast<unsigned>((I + moed::kRowsGu - 1) / moed::kRowsGu), slots),
+                   dim3(moed::kWarps * 32), static_cast<size_t>(smem), stream, qg, gl, rout);
+  if (err != cudaSuccess) return err;
+  // down (x the route weight): K = I, rows = H, x = h [R][I]
+  MoeDecParams qd = q;
+  qd.x = reinterpret_cast<const uint16_t*>(q.h);
+  qd.signs0 = ds;
+  qd.scales0 = dc;
+  qd.signs1 = nullptr;
+  qd.scales1 = nullptr;
+  qd.rows = H;
+  qd.K = I;
+  qd.NG = I / 128;
+  qd.P = ((qd.NG & 1) ? qd.NG : qd.NG + 1) * 16;
+  qd.lgGw = lg2(qd.NG);
+  smem = moeg_layout(qd.NG, qd.P).total;
+  err = ensure_dyn_smem(reinterpret_cast<const void*>(moe_decode_grouped_kernel<false>), smem);
+  if (err != cudaSuccess) return err;
+  err = launch_pdl(moe_decode_grouped_kernel<false>,
+                   dim3(static_cast<unsigned>((H + moeg::kRowsD - 1) / moeg::kRowsD), slots),
+                   dim3(moed::kWarps * 32), static_cast<size_t>(smem), stream, qd, gl, rout);
+  if (err != cudaSuccess) return err;
+  // out[t] = its slots in slot order
+  const int64_t total4 = static_cast<int64_t>(T) * (H / 4);
+  int64_t blocks = (total4 + 255) / 256;
+  if (blocks > 8 * num_sms) blocks = 8 * num_sms;
+  return launch_pdl(moe_combine_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, stream,
+                    static_cast<const float*>(rout), static_cast<const int*>(pos), T, H, q.top_k, out);
+}
+
 static cudaError_t launch_moe_decode_down(MoeDecParams q, int T, float* out, cudaStream_t stream) {
   auto lg2 = [](int v) {
     int l = 0;
@@ -1139,7 +1417,8 @@ cudaError_t launch_moe(const uint16_t* x, const float* logits, int64_t T, int64_
   // The moe_path knob (tiles | decode) forces a path for testing.
   constexpr int64_t kDecodeMaxT = 16;
   const int mpath = knob(kKnobMoePath);
-  bool decode = (mpath ? mpath == 2 : T <= kDecodeMaxT) && H / 128 <= gd::kMaxSets && I / 128 <= gd::kMaxSets;
+  bool decode = (mpath ? (mpath == 2 || mpath == 3) : T <= kDecodeMaxT) && H / 128 <= gd::kMaxSets &&
+                I / 128 <= gd::kMaxSets;
   if (decode) {  // both decode kernels' shared memory must fit
     MoeDecParams qg = {};
     qg.NG = static_cast<int>(H / 128);
@@ -1149,13 +1428,19 @@ cudaError_t launch_moe(const uint16_t* x, const float* logits, int64_t T, int64_
   }
   if (decode) {
     // up to 4 tokens each CTA routes its token (one launch less); above,
-    // the router kernel does it once per token
+    // the router kernel does it once per token.  The grouped form (one
+    // product per touched expert, its routes as the batch rows) is taken by
+    // the moe_path knob "grouped" (up to 16 tokens).
     constexpr int64_t kSelfRouteMaxT = 4;
+    auto pad16 = [](int ng) { return ((ng & 1) ? ng : ng + 1) * 16; };
+    const int ngh = static_cast<int>(H / 128), ngi = static_cast<int>(I / 128);
+    const bool grouped = mpath == 3 && T <= moeg::kMaxT && moeg_layout(ngh, pad16(ngh)).total <= moed::kSmemCap &&
+                         moeg_layout(ngi, pad16(ngi)).total <= moed::kSmemCap;
     MoeDecParams q = {};
     q.logits = logits;
     q.E = E;
-    q.self_route = T <= kSelfRouteMaxT ? 1 : 0;
-    if (!q.self_route) {
+    q.self_route = T <= kSelfRouteMaxT && !grouped ? 1 : 0;
+    if (!q.self_route && !grouped) {
       float* xcs = reinterpret_cast<float*>(ws + L.xcs);
       err = launch_pdl(moe_route_kernel, dim3(static_cast<unsigned>((T + 7) / 8)), dim3(256), 0, stream, logits,
                        static_cast<int>(T), E, top_k, ids, wts, x, static_cast<int>(H), xcs);
@@ -1175,6 +1460,12 @@ cudaError_t launch_moe(const uint16_t* x, const float* logits, int64_t T, int64_
     q.rows = static_cast<int>(I);
     q.K = static_cast<int>(H);
     q.NG = static_cast<int>(H / 128);
+    if (grouped) {
+      int* tl = reinterpret_cast<int*>(ws + L.tiles_gu);
+      const MoeGroupList gl{hdr, offsets, tl, tl + E, sroute};
+      return launch_moe_decode_grouped(q, static_cast<int>(T), static_cast<int>(H), static_cast<int>(I), gl, ds, dc,
+                                       rout, pos, out, stream, num_sms);
+    }
     err = launch_moe_decode_gateup(q, stream);
     if (err != cudaSuccess) return err;
     MoeDecParams qd = q;

@@ -1,7 +1,9 @@
 """w1_moe_grouped on the GPU vs the fp64 oracle: routing exact, every stage
 within its bound, end to end with the bf16 intermediate propagated.  Batches
-of up to 8 tokens take the decode path (per-route products), larger ones the
-expert-sorted tile pipeline; the moe_path knob forces either."""
+of up to 16 tokens take the decode path (per-route products), larger ones the
+expert-sorted tile pipeline; the moe_path knob forces either, or the decode
+path grouped by expert (one product per touched expert, its routes as the
+batch rows)."""
 import functools
 
 import numpy as np
@@ -19,6 +21,16 @@ def _pack_experts(Wt):
     E, rows, K = Wt.shape
     s, c = O.pack_ref_fast(Wt.reshape(E * rows, K))
     return s.reshape(E, rows, K // 32), c.reshape(E, rows, K // 128)
+
+
+def shared_logits(T, E, K, seed):
+    """Every token prefers the same K experts (decreasing with the expert
+    index), so each of them is routed by all T tokens."""
+    g = np.random.default_rng(seed)
+    L = g.normal(size=(T, E)).astype(np.float32) - 8.0
+    L[:, :K] = np.float32(4.0) + np.linspace(1.0, 0.0, K, dtype=np.float32)[None, :] + \
+        np.float32(0.01) * g.normal(size=(T, K)).astype(np.float32)
+    return L
 
 
 def tied_logits(T, E, seed):
@@ -45,17 +57,19 @@ def tied_logits(T, E, seed):
 
 
 @functools.lru_cache(maxsize=None)
-def moe_case(T, H, I, E, seed, skew=0.0, ties=False):
+def moe_case(T, H, I, E, seed, skew=0.0, ties=False, shared_k=0):
     x, logits, gate, up, down = synth.moe_case(T=T, H=H, I=I, E=E, seed=seed)
     if skew:
         logits = logits + np.float32(skew) * np.linspace(1.0, 0.0, E, dtype=np.float32)[None, :]
     if ties:
         logits = tied_logits(T, E, seed)
+    if shared_k:
+        logits = shared_logits(T, E, shared_k, seed)
     return x, logits, _pack_experts(gate), _pack_experts(up), _pack_experts(down)
 
 
-def run_and_check(T, H, I, E, K, seed, skew=0.0, ties=False):
-    x, logits, G, U, D = moe_case(T, H, I, E, seed, skew, ties)
+def run_and_check(T, H, I, E, K, seed, skew=0.0, ties=False, shared=False):
+    x, logits, G, U, D = moe_case(T, H, I, E, seed, skew, ties, K if shared else 0)
     dev = lambda p: (words_dev(p[0].reshape(-1, p[0].shape[-1])).view(p[0].shape[0], p[0].shape[1], -1),
                      fp16_dev(p[1].reshape(-1, p[1].shape[-1])).view(p[1].shape[0], p[1].shape[1], -1))
     ws = ops.moe_workspace(T, H, I, E, K)
@@ -142,7 +156,25 @@ def test_moe_is_deterministic(T):
     assert np.array_equal(a, b)
 
 
-@pytest.mark.parametrize("path", ["default", "tiles", "decode"])
+@pytest.mark.parametrize("T,H,I,E,K,seed,skew,shared", [
+    (1, 2048, 1024, 64, 8, 2, 0.0, False),    # one token: every count is 1
+    (4, 2048, 1024, 64, 8, 5, 0.0, False),
+    (8, 2048, 1024, 64, 8, 11, 0.0, False),   # the OLMoE-like layer at 8 tokens
+    (8, 512, 384, 16, 4, 6, 0.0, False),      # experts shared by several tokens
+    (16, 512, 256, 16, 4, 12, 0.0, False),    # the largest grouped batch
+    (16, 512, 384, 8, 4, 13, 6.0, False),     # skewed: counts above 8 (two batches per expert)
+    (16, 384, 256, 16, 4, 14, 0.0, True),     # every token on the same 4 experts: 16 routes each
+    (11, 256, 128, 8, 2, 15, 0.0, True),      # 11 routes per expert: batches of 8 and 3
+])
+def test_moe_grouped_decode(T, H, I, E, K, seed, skew, shared, knob):
+    """The decode path grouped by expert (DBF post, section 7 item 1: products
+    specialised to the observed expert counts), including forced shared
+    experts whose routes exceed one 8-row batch."""
+    knob("moe_path", "grouped")
+    run_and_check(T, H, I, E, K, seed, skew, shared=shared)
+
+
+@pytest.mark.parametrize("path", ["default", "tiles", "decode", "grouped"])
 @pytest.mark.parametrize("T", [5, 24])
 def test_moe_routing_ties_go_to_the_lower_expert(path, T, knob):
     """Exactly tied router logits on both paths (the decode path routes up to
