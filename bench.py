@@ -280,6 +280,45 @@ def time_gemv_static(torch, combos, stream, reps: int = 3):
     return out
 
 
+def time_gemv_floor(torch, ops, combos, stream, reps: int = 3):
+    """Per pair, the per-launch floor: w1_stream_probe over the same rotating
+    weight copies (sign words + scales), in the same CUDA-graph form as the
+    products (back-to-back launches, programmatic dependent launch), with the
+    loads after the dependency wait (as the headline chain) and before it (as
+    W1_GEMV_STATIC_WEIGHTS).  Outside the timed steps."""
+    dev = torch.device("cuda")
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    ctas = 2 * sms
+    out = torch.zeros(ctas, dtype=torch.int32, device=dev)
+    res = []
+    for cb in combos:
+        us = {}
+        for early in (False, True):
+            def chain(cb=cb, early=early):
+                for r in range(cb["R"]):
+                    ops.w1_stream_probe(cb["signs"][r], cb["scales"][r], out, ctas, early, stream=stream)
+            chain()
+            stream.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                chain()
+            with torch.cuda.stream(stream):
+                g.replay()
+            torch.cuda.synchronize()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(stream):
+                e0.record(stream)
+                for _ in range(reps):
+                    g.replay()
+                e1.record(stream)
+            torch.cuda.synchronize()
+            us["static" if early else "plain"] = e0.elapsed_time(e1) * 1e3 / (reps * cb["R"])
+            del g
+        res.append(us)
+    return res
+
+
 def gemv_e2e(torch, ops, combos, steps: int):
     """The same sweep through the public API (eager w1_gemv calls, no graphs).
     Every step copies its inputs host->device from pinned memory (each pair's
@@ -372,8 +411,9 @@ MOE_DECODE_T = (1, 4, 8, 16)   # decode-regime batches
 DBF_BATCHES = [1, 2, 4, 8, 512]
 
 
-def moe_rows(torch, ops, synth, peaks, iters: int = 8):
-    """Routed MoE layer (OLMoE-like): tokens/s and TFLOP/s, L2 flushed per call."""
+def moe_rows(torch, ops, synth, peaks, iters: int = 8, only_t: int | None = None):
+    """Routed MoE layer (OLMoE-like): tokens/s and TFLOP/s, L2 flushed per call.
+    only_t: just that decode batch (a small case for ncu), no 512-token layer."""
     dev = torch.device("cuda")
     T, H, I, E, K = MOE["T"], MOE["H"], MOE["I"], MOE["E"], MOE["top_k"]
     x, logits, gate, up, down = synth.moe_case(T=T, H=H, I=I, E=E)
@@ -388,11 +428,11 @@ def moe_rows(torch, ops, synth, peaks, iters: int = 8):
     ws = ops.moe_workspace(T, H, I, E, K)
     out = torch.empty((T, H), dtype=torch.float32, device=dev)
     flush = torch.empty(int(512 * 2 ** 20), dtype=torch.uint8, device=dev)
-    for _ in range(3):
+    for _ in range(0 if only_t else 3):
         ops.w1_moe_grouped(xd, ld, G, U, D, K, out=out, workspace=ws)
     torch.cuda.synchronize()
-    times = []
-    for _ in range(iters):
+    times = [] if not only_t else [float("nan")]
+    for _ in range(0 if only_t else iters):
         flush.zero_()
         a = torch.cuda.Event(enable_timing=True)
         b = torch.cuda.Event(enable_timing=True)
@@ -415,7 +455,7 @@ def moe_rows(torch, ops, synth, peaks, iters: int = 8):
     ids_all = np.argsort(-logits, axis=1, kind="stable")[:, :K]
     st = torch.cuda.Stream()
     decode = []
-    for Td in MOE_DECODE_T:
+    for Td in (MOE_DECODE_T if not only_t else (only_t,)):
         wsd = ops.moe_workspace(Td, H, I, E, K)
         outd = torch.empty((Td, H), dtype=torch.float32, device=dev)
         windows = [(i * Td) % (T - Td + 1) for i in range(iters)]
@@ -460,13 +500,13 @@ def moe_rows(torch, ops, synth, peaks, iters: int = 8):
     return row
 
 
-def dbf_rows(torch, ops, synth, peaks, l2_bytes: int, iters: int = 5):
+def dbf_rows(torch, ops, synth, peaks, l2_bytes: int, iters: int = 5, only_b: int | None = None):
     """DBF chain 4096^3: B = 1, 8 as GB/s of sign bytes (rotating copies > 4x L2,
     CUDA graph of back-to-back calls); B = 512 as TFLOP/s (L2 flushed)."""
     dev = torch.device("cuda")
     m = r = n = 4096
     rows = []
-    for B in DBF_BATCHES:
+    for B in (DBF_BATCHES if not only_b else (only_b,)):
         a, B1, mid, B2, b, x = synth.dbf_case(m=m, r=r, n=n, B=B)
         to16 = lambda v: torch.from_numpy(v.view(np.int16)).to(dev).view(torch.float16)
         tow = lambda v: torch.from_numpy(v.view(np.int32)).to(dev)
@@ -839,9 +879,9 @@ def run_gpu(args):
         if args.section == "gemm":
             rows["gemm"] = gemm_rows(torch, ops, synth, peaks)
         elif args.section == "moe":
-            rows["moe"] = moe_rows(torch, ops, synth, peaks)
+            rows["moe"] = moe_rows(torch, ops, synth, peaks, only_t=args.moe_t)
         elif args.section == "dbf":
-            rows["dbf"] = dbf_rows(torch, ops, synth, peaks, l2)
+            rows["dbf"] = dbf_rows(torch, ops, synth, peaks, l2, only_b=args.dbf_b)
         elif args.section == "gemv1":
             rows["gemv1"] = gemv_one(torch, ops, synth, args.shape)
         elif args.section == "measure":
@@ -863,8 +903,9 @@ def run_gpu(args):
     value = all_bytes / (t_max * 1e-3) / 1e9
 
     static_us = time_gemv_static(torch, combos, stream)
+    floor_us = time_gemv_floor(torch, ops, combos, stream)
     gemv_rows = []
-    for cb, ms, st_us in zip(combos, per_pair_ms, static_us):
+    for cb, ms, st_us, fl in zip(combos, per_pair_ms, static_us, floor_us):
         per_launch_us = ms * 1e3 / (cb["R"] * args.steps)
         gbs = cb["bytes"] / (per_launch_us * 1e-6) / 1e9
         gemv_rows.append({"N": cb["N"], "K": cb["K"], "B": cb["B"], "launches": cb["R"],
@@ -873,7 +914,11 @@ def run_gpu(args):
                           "us_per_launch": round(per_launch_us, 3), "GB/s": round(gbs, 1),
                           "frac_hbm": round(gbs / peaks["hbm_gbs"], 4),
                           "static_weights_us_per_launch": round(st_us, 3),
-                          "static_weights_GB/s": round(cb["bytes"] / (st_us * 1e-6) / 1e9, 1)})
+                          "static_weights_GB/s": round(cb["bytes"] / (st_us * 1e-6) / 1e9, 1),
+                          # the launch floor (w1_stream_probe over the same bytes, same launch form)
+                          "floor_us": round(fl["plain"], 3), "x_floor": round(per_launch_us / fl["plain"], 2),
+                          "floor_static_us": round(fl["static"], 3),
+                          "x_floor_static": round(st_us / fl["static"], 2)})
     # roofline of the dominant kernel (largest share of the step's device time)
     per_kernel = {}
     for cb, ms, row in zip(combos, per_pair_ms, gemv_rows):
@@ -1024,6 +1069,8 @@ def main():
                     help="issue the sweep's launches one by one instead of CUDA graphs (for ncu launch lists)")
     ap.add_argument("--shape", default="4096,4096,1",
                     help="N,K,B of the single GEMV that --section gemv1 launches (for ncu captures)")
+    ap.add_argument("--dbf-b", type=int, default=None, help="--section dbf: that batch only (profiling)")
+    ap.add_argument("--moe-t", type=int, default=None, help="--section moe: that decode batch only (profiling)")
     ap.add_argument("--choices", default=None,
                     help="JSON line of an earlier run: pin each GEMV pair to the kernel it chose (profiling)")
     ap.add_argument("--section", default="all", choices=["all", "gemm", "moe", "dbf", "gemv1", "okt", "measure"],

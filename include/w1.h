@@ -246,6 +246,23 @@ int dbf_residual(const float* W, const uint16_t* a, const uint32_t* B1, const ui
                  size_t ws_bytes, w1_stream_t stream);
 
 /*
+ * w1_stream_probe -- the per-launch floor of a decode product (a measurement
+ * aid; the pages have no counterpart).  Reads the byte ranges [a, a + abytes)
+ * and [b, b + bbytes) once with 16-byte loads spread over `ctas` CTAs, every
+ * load of a thread issued before any is used, and adds one word per CTA into
+ * out[cta] (so the loads cannot be dropped; the values mean nothing).  Timed
+ * as back-to-back launches over a product's sign words and scales, it is the
+ * memory work of that product and nothing else.
+ *   flags: 1 = issue the loads before the programmatic-dependent-launch wait
+ *   (the analogue of W1_GEMV_STATIC_WEIGHTS), 0 = after it.
+ *   abytes > 0, bbytes >= 0, both multiples of 16; 1 <= ctas <= 65535; else
+ *   W1_ERR_SHAPE.  a, b (if bbytes > 0) and out (uint32 [ctas]) 16-byte
+ *   aligned, else W1_ERR_ALIGN.
+ */
+int w1_stream_probe(const void* a, int64_t abytes, const void* b, int64_t bbytes, int64_t ctas, uint32_t flags,
+                    uint32_t* out, w1_stream_t stream);
+
+/*
  * dbf_reproject_mid -- least-squares refit of the DBF middle diagonal ("LLM
  * binarization episode 01: DBF", section 1.2 "What we inherit from DBF": one
  * final linear least-squares reprojection of the middle diagonal, the signs
@@ -374,8 +391,11 @@ size_t w1_moe_workspace_size(int64_t T, int64_t H, int64_t I, int64_t E, int64_t
  *   zero again (after a W1_ERR_TIMEOUT the caller must re-zero it).  After a call
  *   it holds h_scaled (fp32 [min(B,8)][r], byte offset 256) of the last group
  *   of up to 8 batch rows.  Calls sharing a workspace must not overlap.
- * Both binary products run in one kernel for each group of up to 8 batch rows
- * (int8 tensor-core products, a grid-wide barrier between them).  Accuracy:
+ * Below 64 rows the batch runs in groups of up to 8 rows: a group of 1-2 rows
+ * as two products (V then U, h_scaled through the workspace; U's K split
+ * over r is the pages' "split rank", section 5 item 5), a group of 3-8 rows
+ * as one kernel with a grid-wide barrier between the two products (section
+ * 7).  From 64 rows on, two tensor-core sign GEMMs.  Accuracy:
  * |y - y_exact| <= 1e-3 * |a_i| * sum_j |mid_j h_j| per element.
  */
 int dbf_apply(const uint16_t* a, const uint32_t* B1, const uint16_t* mid, const uint32_t* B2,

@@ -412,4 +412,53 @@ cudaError_t launch_power_iteration(const float* A, int64_t m, int64_t n, const f
   return e;
 }
 
+// ---------------------------------------------------------------- launch floor
+// Reads two byte ranges (a product's sign words and scales) with 16-byte
+// loads, every load of a thread issued before any is used, and folds them
+// into one word per CTA (so that the loads cannot be dropped).  It does the
+// memory work of a decode product and nothing else: back-to-back launches of
+// it give the per-launch floor a product kernel is measured against.
+// early: the loads are issued before the grid dependency wait (as a product
+// with W1_GEMV_STATIC_WEIGHTS does), else after it.
+constexpr int kProbeThreads = 256;
+constexpr int kProbeLoads = 8;  // 16-byte loads per thread and pass
+__global__ void __launch_bounds__(kProbeThreads) stream_probe_kernel(const uint4* __restrict__ a, int64_t na,
+                                                                     const uint4* __restrict__ b, int64_t nb,
+                                                                     int early, uint32_t* __restrict__ out) {
+  pdl_launch_dependents();
+  if (!early) pdl_wait();
+  const int64_t n = na + nb;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * kProbeThreads;
+  uint32_t acc = 0;
+  for (int64_t i0 = static_cast<int64_t>(blockIdx.x) * kProbeThreads + threadIdx.x; i0 < n;
+       i0 += kProbeLoads * stride) {
+    uint4 v[kProbeLoads];
+#pragma unroll
+    for (int j = 0; j < kProbeLoads; ++j) {
+      const int64_t i = i0 + j * stride;
+      v[j] = i < na ? __ldcs(a + i) : (i < n ? __ldcs(b + (i - na)) : make_uint4(0, 0, 0, 0));
+    }
+#pragma unroll
+    for (int j = 0; j < kProbeLoads; ++j) acc += v[j].x ^ v[j].y ^ v[j].z ^ v[j].w;
+  }
+  if (early) pdl_wait();
+  acc = __reduce_add_sync(0xFFFFFFFFu, acc);
+  if ((threadIdx.x & 31) == 0) atomicAdd(out + blockIdx.x, acc);
+}
+
+cudaError_t launch_stream_probe(const void* a, int64_t abytes, const void* b, int64_t bbytes, int ctas, bool early,
+                                uint32_t* out, cudaStream_t stream) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(ctas));
+  cfg.blockDim = dim3(kProbeThreads);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, stream_probe_kernel, static_cast<const uint4*>(a), abytes / 16,
+                            static_cast<const uint4*>(b), bbytes / 16, early ? 1 : 0, out);
+}
+
 }  // namespace w1

@@ -10,11 +10,12 @@
 // expert-major compaction of route-specific inputs, shared gate/up inputs
 // kept un-duplicated, fused SwiGLU, skipped empty tiles.
 //
-// Up to 16 tokens (the decode regime) the layer runs as per-route products:
+// Up to 8 tokens (the decode regime) the layer runs as per-route products:
 // gate/up + SwiGLU (up to 4 tokens with the routing computed in each CTA,
 // else after the router kernel) and down with the slot-ordered combine (see
-// "decode regime" below).  Larger batches take the expert-sorted tile
-// pipeline.
+// "decode regime" below); from 9 to 16 tokens as products grouped by expert
+// (see "decode regime, grouped by expert").  Larger batches take the
+// expert-sorted tile pipeline.
 //
 // Seven launches on one stream (programmatic dependent launch between them):
 //  1. route_kernel     warp per token: fp32 softmax, top-k by logit, weights,
@@ -1084,14 +1085,17 @@ __global__ void __launch_bounds__(moed::kWarps * 32, 1) moe_decode_down_kernel(c
 // the tokens and groups the routes by expert (route order within an expert);
 // then one CTA per (expert, row block) stages the expert's rows once and runs
 // the direct GEMV steps with the expert's routes as its batch rows -- a
-// 1..8-row product chosen by the route count, 8 routes at a time above --
-// for gate/up (+ SwiGLU) and for down (x the route weight); the combine adds
-// each token's slots in slot order.
+// 1..4-row product chosen by the route count, 4 routes at a time above (the
+// rows stay staged) -- for gate/up (+ SwiGLU) and for down (x the route
+// weight); the combine adds each token's slots in slot order.  Batches of at
+// most 4 rows keep a CTA within half an SM (registers and shared memory), so
+// two CTAs share each SM.
 namespace moeg {
 constexpr int kMaxT = 16;                     // tokens of the grouped decode path
 constexpr int kMaxR = kMaxT * moe::kMaxTopK;  // routes
 constexpr int kRowsD = 16 * moed::kWarps;     // down rows per CTA (16 per warp)
-constexpr int kRedCols = 24;                  // digit columns of an 8-row batch
+constexpr int kBatch = 4;                     // routes per product batch
+constexpr int kRedCols = 3 * kBatch;          // digit columns of a batch
 }  // namespace moeg
 
 struct MoeGroupList {
@@ -1163,7 +1167,7 @@ __host__ __device__ inline MoeGroupLayout moeg_layout(int NG, int P) {
   MoeGroupLayout M;
   M.warp_bytes = L.warp_bytes;
   M.xs = moed::kWarps * L.warp_bytes;
-  M.red = M.xs + (NG * gd::Cfg<8>::SCR * 4 + 15) / 16 * 16;
+  M.red = M.xs + (NG * gd::Cfg<moeg::kBatch>::SCR * 4 + 15) / 16 * 16;
   M.total = M.red + moed::kWarps * 16 * moeg::kRedCols * 4;
   return M;
 }
@@ -1222,11 +1226,11 @@ __device__ __forceinline__ GdGeom moeg_geom(int NG, int rows, int row0) {
 }
 
 template <bool GATEUP>
-__global__ void __launch_bounds__(moed::kWarps * 32, 1) moe_decode_grouped_kernel(const MoeDecParams q,
+__global__ void __launch_bounds__(moed::kWarps * 32, 2) moe_decode_grouped_kernel(const MoeDecParams q,
                                                                                   MoeGroupList gl,
                                                                                   float* __restrict__ rout) {
   extern __shared__ __align__(16) unsigned char smem[];
-  __shared__ int xrow[8], route[8];
+  __shared__ int xrow[moeg::kBatch], route[moeg::kBatch];
   const MoeGroupLayout L = moeg_layout(q.NG, q.P);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   pdl_wait();
@@ -1265,8 +1269,8 @@ __global__ void __launch_bounds__(moed::kWarps * 32, 1) moe_decode_grouped_kerne
   gd_load_scales<1>(p, g, 0, lane, sreg);
   gd_finish_scales<1>(p, g, lane, sreg, scl);
   cp_async_wait_all();
-  for (int c0 = 0; c0 < cnt; c0 += 8) {
-    const int nb = min(8, cnt - c0);
+  for (int c0 = 0; c0 < cnt; c0 += moeg::kBatch) {
+    const int nb = min(moeg::kBatch, cnt - c0);
     if (threadIdx.x < nb) {
       const int r = gl.sroute[st0 + c0 + threadIdx.x];
       route[threadIdx.x] = r;
@@ -1292,11 +1296,7 @@ __global__ void __launch_bounds__(moed::kWarps * 32, 1) moe_decode_grouped_kerne
       case 1: moeg_batch<1>(p, g, wts, scl, xs, red, warp, lane, rows_cta, emit); break;
       case 2: moeg_batch<2>(p, g, wts, scl, xs, red, warp, lane, rows_cta, emit); break;
       case 3: moeg_batch<3>(p, g, wts, scl, xs, red, warp, lane, rows_cta, emit); break;
-      case 4: moeg_batch<4>(p, g, wts, scl, xs, red, warp, lane, rows_cta, emit); break;
-      case 5: moeg_batch<5>(p, g, wts, scl, xs, red, warp, lane, rows_cta, emit); break;
-      case 6: moeg_batch<6>(p, g, wts, scl, xs, red, warp, lane, rows_cta, emit); break;
-      case 7: moeg_batch<7>(p, g, wts, scl, xs, red, warp, lane, rows_cta, emit); break;
-      default: moeg_batch<8>(p, g, wts, scl, xs, red, warp, lane, rows_cta, emit); break;
+      default: moeg_batch<4>(p, g, wts, scl, xs, red, warp, lane, rows_cta, emit); break;
     }
   }
 }
@@ -1428,13 +1428,18 @@ cudaError_t launch_moe(const uint16_t* x, const float* logits, int64_t T, int64_
   }
   if (decode) {
     // up to 4 tokens each CTA routes its token (one launch less); above,
-    // the router kernel does it once per token.  The grouped form (one
-    // product per touched expert, its routes as the batch rows) is taken by
-    // the moe_path knob "grouped" (up to 16 tokens).
+    // the router kernel does it once per token.  From 9 tokens the grouped
+    // form (one product per touched expert, its routes as the batch rows)
+    // replaces the per-route products; the moe_path knob forces either.
     constexpr int64_t kSelfRouteMaxT = 4;
     auto pad16 = [](int ng) { return ((ng & 1) ? ng : ng + 1) * 16; };
     const int ngh = static_cast<int>(H / 128), ngi = static_cast<int>(I / 128);
-    const bool grouped = mpath == 3 && T <= moeg::kMaxT && moeg_layout(ngh, pad16(ngh)).total <= moed::kSmemCap &&
+    // Grouped by default from 9 tokens on: measured on the OLMoE-like layer
+    // (graph replays, L2 flushed), 74.8 vs 93.0 us at 16 tokens, 57.3 vs
+    // 54.3 at 8, slower below (20.5 / 29.7 us at 1 token: two launches more).
+    constexpr int64_t kGroupedMinT = 9;
+    const bool want_grouped = mpath ? mpath == 3 : T >= kGroupedMinT;
+    const bool grouped = want_grouped && T <= moeg::kMaxT && moeg_layout(ngh, pad16(ngh)).total <= moed::kSmemCap &&
                          moeg_layout(ngi, pad16(ngi)).total <= moed::kSmemCap;
     MoeDecParams q = {};
     q.logits = logits;

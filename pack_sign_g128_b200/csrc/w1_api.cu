@@ -36,6 +36,8 @@ cudaError_t launch_dbf(const uint16_t* a, const uint32_t* B1, const uint16_t* mi
                        float* y, void* workspace, cudaStream_t stream, int num_sms, int smem_cap,
                        bool allow_tensor_path);
 size_t dbf_workspace_bytes(int64_t m, int64_t r, int64_t n, int64_t B);
+cudaError_t launch_stream_probe(const void* a, int64_t abytes, const void* b, int64_t bbytes, int ctas, bool early,
+                                uint32_t* out, cudaStream_t stream);
 bool reproject_shape_ok(int64_t m, int64_t r, int64_t n);
 size_t reproject_workspace_bytes(int64_t m, int64_t r, int64_t n);
 cudaError_t launch_reproject_mid(const float* W, const uint16_t* a, const uint32_t* B1, const uint32_t* B2,
@@ -185,6 +187,20 @@ int w1_residual(const float* W, int64_t N, int64_t K, const uint32_t* signs, con
   if (st != W1_OK) return st;
   return launch_result(launch_residual_g128(W, N, K, signs, scales, E, sums, workspace,
                                             reinterpret_cast<cudaStream_t>(stream), d.sms));
+}
+
+int w1_stream_probe(const void* a, int64_t abytes, const void* b, int64_t bbytes, int64_t ctas, uint32_t flags,
+                    uint32_t* out, w1_stream_t stream) {
+  if (!a || !out || (bbytes > 0 && !b)) return W1_ERR_NULL;
+  if (abytes <= 0 || bbytes < 0 || (abytes % 16) != 0 || (bbytes % 16) != 0 || ctas < 1 || ctas > 65535 ||
+      (flags & ~1u) != 0)
+    return W1_ERR_SHAPE;
+  if (!aligned16(a) || (bbytes > 0 && !aligned16(b)) || !aligned16(out)) return W1_ERR_ALIGN;
+  DeviceInfo d;
+  int st = device_info(&d);
+  if (st != W1_OK) return st;
+  return launch_result(launch_stream_probe(a, abytes, b, bbytes, static_cast<int>(ctas), (flags & 1u) != 0, out,
+                                           reinterpret_cast<cudaStream_t>(stream)));
 }
 
 size_t dbf_reproject_mid_workspace_size(int64_t m, int64_t r, int64_t n) { return reproject_workspace_bytes(m, r, n); }

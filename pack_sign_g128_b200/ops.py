@@ -194,6 +194,19 @@ def dbf_residual(W: torch.Tensor, a: torch.Tensor, B1: torch.Tensor, mid: torch.
     return (E if want_E else None), sums
 
 
+def w1_stream_probe(a: torch.Tensor, b: torch.Tensor | None, out: torch.Tensor, ctas: int, early: bool,
+                    stream=None) -> None:
+    """Launch the per-launch floor probe over a's and b's bytes (see include/w1.h)."""
+    if out.dtype != torch.int32 or out.numel() < ctas:
+        raise ValueError("out must be int32 with at least `ctas` elements")
+    ab = a.numel() * a.element_size()
+    bb = 0 if b is None else b.numel() * b.element_size()
+    st = _lib.fn("w1_stream_probe")(_ptr(a), ab, _ptr(b) if b is not None else None, bb, ctas, 1 if early else 0,
+                                    _ptr(out), _stream(stream, a))
+    if st != _lib.W1_OK:
+        raise _lib.W1Error(st, "w1_stream_probe")
+
+
 def dbf_reproject_workspace_size(m: int, r: int, n: int) -> int:
     return int(_lib.fn("dbf_reproject_mid_workspace_size")(m, r, n))
 

@@ -179,6 +179,22 @@ def test_measure_host_side_argument_errors(lib):
     assert pi(odd, 64, 64, good, 32, good, good, ws, None) == _lib.W1_ERR_ALIGN
 
 
+def test_stream_probe_host_side_argument_errors(lib):
+    good = ctypes.c_void_p(1 << 20)
+    odd = ctypes.c_void_p((1 << 20) + 4)
+    f = lib.w1_stream_probe
+    assert f(None, 1024, None, 0, 148, 0, good, None) == _lib.W1_ERR_NULL
+    assert f(good, 1024, None, 16, 148, 0, good, None) == _lib.W1_ERR_NULL   # b missing for bbytes > 0
+    assert f(good, 1024, good, 16, 148, 0, None, None) == _lib.W1_ERR_NULL
+    assert f(good, 0, None, 0, 148, 0, good, None) == _lib.W1_ERR_SHAPE
+    assert f(good, 1000, None, 0, 148, 0, good, None) == _lib.W1_ERR_SHAPE
+    assert f(good, 1024, good, 8, 148, 0, good, None) == _lib.W1_ERR_SHAPE
+    assert f(good, 1024, None, 0, 0, 0, good, None) == _lib.W1_ERR_SHAPE
+    assert f(good, 1024, None, 0, 148, 2, good, None) == _lib.W1_ERR_SHAPE
+    assert f(odd, 1024, None, 0, 148, 0, good, None) == _lib.W1_ERR_ALIGN
+    assert f(good, 1024, good, 16, 148, 1, odd, None) == _lib.W1_ERR_ALIGN
+
+
 def test_reproject_host_side_argument_errors(lib):
     good = ctypes.c_void_p(1 << 20)
     odd = ctypes.c_void_p((1 << 20) + 4)

@@ -1,10 +1,10 @@
 """w1_gemv on the GPU vs the fp64 oracle (element-wise, 1e-3 * sum|s x| bound).
 
-Every test runs on each kernel, forced with the gemv_path knob: the fp8 kernel
-with 8 and with 16 warps per CTA (flat / flat16, bf16 activations), the
-int8 direct kernel with 8 and 16 warps (direct / direct16), the tcgen05
-kernel (tc) and the mma.sync ring kernel (ring, the fallback for other
-shapes)."""
+Every test runs on each kernel, forced with the gemv_path knob: the
+register-fed kernel with 8 and with 16 warps per CTA (flat / flat16: int8
+activation digits up to 2 rows, bf16 activations above), the int8 direct
+kernel with 8 and 16 warps (direct / direct16), the tcgen05 kernel (tc) and
+the mma.sync ring kernel (ring, the fallback for other shapes)."""
 import functools
 
 import numpy as np

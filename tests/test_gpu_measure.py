@@ -121,3 +121,26 @@ def test_relative_spectral_residual_g128():
     rel_ref = O.power_iteration_ref(E_ref, v, 32) / O.power_iteration_ref(W, v, 32)
     assert rel == pytest.approx(rel_ref, rel=1e-9)
     assert 0.3 < rel < 1.0
+
+
+@pytest.mark.parametrize("abytes,bbytes,ctas,early", [(2359296, 0, 296, False), (4096 * 1024 // 8, 4096 * 8 * 2, 148, True),
+                                                      (16, 48, 3, True), (6340608, 16, 1000, False)])
+def test_stream_probe_reads_every_byte_once(abytes, bbytes, ctas, early):
+    """w1_stream_probe folds each 16-byte chunk of both ranges into its CTA's
+    word; the words' sum is the sum over all chunks of x ^ y ^ z ^ w (mod 2^32)
+    whatever the CTA count -- so every chunk was read exactly once."""
+    g = np.random.default_rng(abytes + bbytes + ctas)
+    a = g.integers(0, 2 ** 32, size=abytes // 4, dtype=np.uint32)
+    b = g.integers(0, 2 ** 32, size=max(bbytes // 4, 4), dtype=np.uint32)[: bbytes // 4]
+    out = torch.zeros(ctas, dtype=torch.int32, device=dev())
+    bd = words_dev(b) if bbytes else None
+    ops.w1_stream_probe(words_dev(a), bd, out, ctas, early)
+    assert ops.sync_status() == _lib.W1_OK
+
+    def fold(v):
+        q = v.reshape(-1, 4)
+        return int(np.sum((q[:, 0] ^ q[:, 1] ^ q[:, 2] ^ q[:, 3]).astype(np.uint64)) % (1 << 32))
+
+    want = (fold(a) + (fold(b) if bbytes else 0)) % (1 << 32)
+    got = int(np.sum(out.cpu().numpy().view(np.uint32).astype(np.uint64)) % (1 << 32))
+    assert got == want

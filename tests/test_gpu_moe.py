@@ -1,9 +1,9 @@
 """w1_moe_grouped on the GPU vs the fp64 oracle: routing exact, every stage
 within its bound, end to end with the bf16 intermediate propagated.  Batches
-of up to 16 tokens take the decode path (per-route products), larger ones the
-expert-sorted tile pipeline; the moe_path knob forces either, or the decode
-path grouped by expert (one product per touched expert, its routes as the
-batch rows)."""
+of up to 8 tokens take the decode path (per-route products), 9 to 16 the
+decode path grouped by expert (one product per touched expert, its routes as
+the batch rows), larger ones the expert-sorted tile pipeline; the moe_path
+knob forces any of them."""
 import functools
 
 import numpy as np
@@ -162,14 +162,14 @@ def test_moe_is_deterministic(T):
     (8, 2048, 1024, 64, 8, 11, 0.0, False),   # the OLMoE-like layer at 8 tokens
     (8, 512, 384, 16, 4, 6, 0.0, False),      # experts shared by several tokens
     (16, 512, 256, 16, 4, 12, 0.0, False),    # the largest grouped batch
-    (16, 512, 384, 8, 4, 13, 6.0, False),     # skewed: counts above 8 (two batches per expert)
+    (16, 512, 384, 8, 4, 13, 6.0, False),     # skewed: counts above 4 (several batches per expert)
     (16, 384, 256, 16, 4, 14, 0.0, True),     # every token on the same 4 experts: 16 routes each
-    (11, 256, 128, 8, 2, 15, 0.0, True),      # 11 routes per expert: batches of 8 and 3
+    (11, 256, 128, 8, 2, 15, 0.0, True),      # 11 routes per expert: batches of 4, 4 and 3
 ])
 def test_moe_grouped_decode(T, H, I, E, K, seed, skew, shared, knob):
     """The decode path grouped by expert (DBF post, section 7 item 1: products
     specialised to the observed expert counts), including forced shared
-    experts whose routes exceed one 8-row batch."""
+    experts whose routes exceed one 4-row batch."""
     knob("moe_path", "grouped")
     run_and_check(T, H, I, E, K, seed, skew, shared=shared)
 
