@@ -44,11 +44,16 @@ WORKLOAD = ("decode GEMV sweep: (out x in) 4096x4096, 11008x4096, 4096x11008 at 
             "1-bit signs + fp16 scale per 128 weights; x bf16 N(0,1); W N(0,0.02)")
 KERNEL_OF_CHOICE = {"flat": "gemv_flat_kernel", "flat16": "gemv_flat_kernel", "direct": "gemv_direct_kernel",
                     "direct16": "gemv_direct_kernel", "tc": "gemv_tc_kernel", "ring": "gemv_kernel"}
-# DRAM bytes per launch from ncu captures (dram__bytes_read.sum + write), with the
-# shape captured; see profiles/.  Used to report the dominant kernel's traffic.
+# DRAM bytes of one launch (dram__bytes_read.sum + dram__bytes_write.sum) from
+# ncu captures of the decode products, per (N, K, B) pair and kernel choice
+# (profiles/ names each capture and its command).  A pair's own figure is
+# used as is; the line's traffic is the launch-weighted mean over the
+# dominant kernel's pairs, reported only when every one of them has a
+# capture for the kernel it chose.
 CAPTURED_TRAFFIC = {
-    "gemv_tc_kernel": {"shape": (4096, 11008, 8), "bytes": 6585344},
-    "gemv_direct_kernel": {"shape": (4096, 4096, 1), "bytes": 2426880},
+    # (N, K, B, choice): bytes per launch
+    (4096, 4096, 1, "flat/1"): 2437376,
+    (4096, 4096, 8, "flat16/1"): 2494720,
 }
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -929,12 +934,19 @@ def run_gpu(args):
     dom = max(per_kernel, key=lambda k: per_kernel[k]["ms"])
     dk = per_kernel[dom]
     achieved = dk["bytes"] / (dk["ms"] * 1e-3) / 1e9
-    traffic = None
-    cap = CAPTURED_TRAFFIC.get(dom)
-    if cap is not None:
-        n_, k_, _b = cap["shape"]
-        # scale the captured DRAM bytes to this kernel's mean launch by algorithmic bytes
-        traffic = round(cap["bytes"] / packed_bytes(n_, k_) * dk["bytes"] / dk["launches"])
+    # DRAM traffic per launch: each pair's own capture (none scaled from another pair)
+    cap_bytes = 0.0
+    cap_all = True
+    for cb, row in zip(combos, gemv_rows):
+        if row["kernel"] != dom:
+            continue
+        t = CAPTURED_TRAFFIC.get((cb["N"], cb["K"], cb["B"], row["choice"]))
+        row["traffic_bytes_per_launch"] = t
+        if t is None:
+            cap_all = False
+        else:
+            cap_bytes += t * cb["R"] * args.steps
+    traffic = round(cap_bytes / dk["launches"]) if cap_all else None
     dom_share = dk["ms"] / sum(per_pair_ms)
 
     e2e = gemv_e2e(torch, ops, combos, max(1, min(args.steps, 3)))
@@ -968,7 +980,7 @@ def run_gpu(args):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "s8 x s8 -> s32 MMA (mma.sync or tcgen05 kind::i8, chosen per shape by timing) + f32 scale fold; x bf16, 1-bit weights, fp16 scales",
+        "dtype": "s8 x s8 -> s32 (B <= 2) or bf16 x +-1 bf16 -> f32 (B >= 3) mma.sync, kernel chosen per shape by timing, + f32 scale fold; x bf16, 1-bit weights, fp16 scales",
         "data": "synthetic",
         "config": {"workload": WORKLOAD, "launches_per_step": launches_per_step,
                    "packed_bytes_per_step": bytes_per_step,
@@ -980,7 +992,9 @@ def run_gpu(args):
                      "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
                      "traffic": traffic, "kernel": dom, "time_share": round(dom_share, 4),
                      "algorithmic_bytes_per_launch": round(dk["bytes"] / dk["launches"]),
-                     "traffic_note": "ncu DRAM bytes of one captured launch, scaled by algorithmic bytes",
+                     "traffic_note": ("launch-weighted mean of each pair's own ncu capture (DRAM read + write "
+                                      "bytes of one launch); null unless every pair of the kernel has one; "
+                                      "per-pair figures in rows.gemv[*].traffic_bytes_per_launch"),
                      "peak_kind": peaks_kind},
         "cpu_baseline": cpu,
         "e2e": {k: e2e[k] for k in ("value", "unit", "h2d_bytes_per_step", "d2h_bytes_per_step")},
