@@ -51,9 +51,17 @@ KERNEL_OF_CHOICE = {"flat": "gemv_flat_kernel", "flat16": "gemv_flat_kernel", "d
 # dominant kernel's pairs, reported only when every one of them has a
 # capture for the kernel it chose.
 CAPTURED_TRAFFIC = {
-    # (N, K, B, choice): bytes per launch
-    (4096, 4096, 1, "flat/1"): 2437376,
-    (4096, 4096, 8, "flat16/1"): 2494720,
+    # (N, K, B, choice): bytes per launch (mean over the pair's launches of one
+    # eager sweep, profiles/gemv_sweep_traffic.md)
+    (4096, 4096, 1, "flat/1"): 2437361,
+    (4096, 4096, 4, "flat16/1"): 2462227,
+    (4096, 4096, 8, "flat16/1"): 2494788,
+    (11008, 4096, 1, "flat/1"): 6443886,
+    (11008, 4096, 4, "flat/1"): 6465972,
+    (11008, 4096, 8, "flat/1"): 6498901,
+    (4096, 11008, 1, "flat16/2"): 6462866,
+    (4096, 11008, 4, "flat16/1"): 6498892,
+    (4096, 11008, 8, "flat16/1"): 6586883,
 }
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -706,7 +714,8 @@ def measure_rows(torch, ops, synth, peaks, iters: int = 5):
 
     res_ms = timed(lambda: ops.w1_residual(Wd, signs, scales, want_E=False, workspace=ws))
     res_bytes = m * n * 4 + packed_bytes(m, n)
-    dbf_ms = timed(lambda: ops.dbf_residual(Wd, *dargs, want_E=False, workspace=ws))
+    dws = torch.empty(ops.dbf_residual_workspace_size(m, r, n), dtype=torch.uint8, device=dev)
+    dbf_ms = timed(lambda: ops.dbf_residual(Wd, *dargs, want_E=False, workspace=dws))
     dbf_tf = 2.0 * m * n * r / (dbf_ms * 1e-3) / 1e12
     pi_ms = timed(lambda: ops.w1_power_iteration(Wd, v0, 32, workspace=ws))
     # least-squares refit of the DBF middle diagonal against W (fp64 Grams,
@@ -741,8 +750,9 @@ def measure_rows(torch, ops, synth, peaks, iters: int = 5):
     torch.cuda.synchronize()
     return {"residual_g128": {"ms": round(res_ms, 4), "GB/s": round(res_bytes / (res_ms * 1e-3) / 1e9, 1),
                               "frac_hbm": round(res_bytes / (res_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)},
-            "dbf_residual": {"ms": round(dbf_ms, 4), "fp32_TFLOP/s": round(dbf_tf, 1),
-                             "frac_fp32_cuda_core": round(dbf_tf / FP32_PEAK_TFLOPS, 4)},
+            "dbf_residual": {"ms": round(dbf_ms, 4), "TFLOP/s": round(dbf_tf, 1),
+                             "note": "2 m n r on the tensor cores (fp16 x +-1 products, fp32 accumulation)",
+                             "frac_bf16_burst": round(dbf_tf / peaks["bf16_tflops"], 4)},
             "power_iteration_32": {"ms": round(pi_ms, 4), "launches": 3 * 32 + 3},
             "reproject_mid": {"ms": round(rp_ms, 4), "cg_iterations": rp_info[0], "converged": rp_info[1],
                               "fp64_fma": rp_fma, "fp64_TFLOP/s": round(2.0 * rp_fma / (rp_ms * 1e-3) / 1e12, 2)},
