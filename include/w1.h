@@ -211,10 +211,10 @@ int w1_okt_gemv(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_
  * Every sum below has a fixed order (a per-CTA tree, then the CTAs in index
  * order), so results are bitwise reproducible for a shape on a device.
  *
- * w1_measure_workspace_size -- bytes of device workspace that w1_residual,
- * dbf_residual and w1_power_iteration need for an m x n matrix (0 for
- * invalid sizes).  One workspace serves all three calls, one at a time per
- * stream.
+ * w1_measure_workspace_size -- bytes of device workspace that w1_residual
+ * and w1_power_iteration need for an m x n matrix (0 for invalid sizes); one
+ * workspace serves both, one call at a time per stream.  dbf_residual needs
+ * dbf_residual_workspace_size (larger).
  */
 size_t w1_measure_workspace_size(int64_t m, int64_t n);
 
@@ -236,11 +236,15 @@ int w1_residual(const float* W, int64_t N, int64_t K, const uint32_t* signs, con
  * V diag(b) (dbf_apply's operands; m, r, n multiples of 128 and
  * (m/128)(n/128) <= 8192, else W1_ERR_SHAPE).
  *   W_approx[i][j] = (acc_ij * a_i) * b_j in fp32, where acc_ij is the sum
- *   over k ascending of U_ik * (mid_k V_kj) in fp32; so
+ *   over k of U_ik * (mid_k V_kj) with fp32 accumulation (tensor cores: the
+ *   products are exact in fp16); so
  *   |W_approx - exact| <= (r + 2) * 2^-24 * |a_i| |b_j| sum_k |mid_k|.
- *   E fp32 [m][n] out (or NULL), sums as for w1_residual.  W_approx is never
- *   stored.
+ *   E fp32 [m][n] out (or NULL), sums as for w1_residual.
+ *   workspace: device, >= dbf_residual_workspace_size(m, r, n) bytes (it
+ *   holds mid (.) V^T in fp16 and W_approx^T in fp32: about 2 n r + 4 n m),
+ *   else W1_ERR_WORKSPACE.
  */
+size_t dbf_residual_workspace_size(int64_t m, int64_t r, int64_t n);
 int dbf_residual(const float* W, const uint16_t* a, const uint32_t* B1, const uint16_t* mid, const uint32_t* B2,
                  const uint16_t* b, int64_t m, int64_t r, int64_t n, float* E, double* sums, void* workspace,
                  size_t ws_bytes, w1_stream_t stream);

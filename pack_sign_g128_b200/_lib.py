@@ -47,6 +47,7 @@ SIGNATURES = {
     "w1_measure_workspace_size": (_sz, [_i64, _i64]),
     "w1_residual": (_int, [_p, _i64, _i64, _p, _p, _p, _p, _p, _sz, _p]),
     "dbf_residual": (_int, [_p, _p, _p, _p, _p, _p, _i64, _i64, _i64, _p, _p, _p, _sz, _p]),
+    "dbf_residual_workspace_size": (_sz, [_i64, _i64, _i64]),
     "w1_power_iteration": (_int, [_p, _i64, _i64, _p, _i64, _p, _p, _sz, _p]),
     "w1_stream_probe": (_int, [_p, _i64, _p, _i64, _i64, ctypes.c_uint32, _p, _p]),
     "dbf_reproject_mid_workspace_size": (_sz, [_i64, _i64, _i64]),

@@ -6,11 +6,12 @@
 // residual_g128_kernel  E = W - w_hat for the group-128 sign code, with
 //                       sum E^2 and sum W^2.  HBM-bound: reads W and the
 //                       packed bytes once, writes E if asked.
-// dbf_residual_kernel   the same for diag(a) U diag(mid) V diag(b): 128 x 128
-//                       tiles of W_approx formed on CUDA cores (8 x 8 outputs
-//                       per thread, +-1 times +-mid products summed over r in
-//                       fp32), E and the sums in the epilogue; W_approx is
-//                       never stored.  ALU-bound: 2 m n r flops.
+// dres_* + sign GEMM    the same for diag(a) U diag(mid) V diag(b): W_approx^T
+//                       formed on the tensor cores by the sign GEMM
+//                       (sign_gemm.cu: +-1 rows of U times H = mid (.) V^T in
+//                       fp16, exact products, fp32 accumulation, row diagonal
+//                       a, token scale b), then E and the sums through a
+//                       transposing shared tile.  2 m n r flops on tcgen05.
 // pi_* kernels          power iteration on A^T A in fp64 (A read as fp32):
 //                       A v by a warp per row, A^T u by column partial sums
 //                       over row chunks, the norm by one CTA.
@@ -122,97 +123,68 @@ __global__ void __launch_bounds__(meas::kThreads) residual_g128_kernel(const flo
 }
 
 // ----------------------------------------------------------------- DBF chain
+// W_approx = diag(a) U diag(mid) V diag(b) on the tensor cores: with
+// H[j][k] = mid_k V_kj (fp16, exact: a sign on an fp16 value), the sign GEMM
+// (sign_gemm.cu, +-1 rows of U, fp32 accumulation over k in TMEM) forms
+// W_approx^T[j][i] = (a_i sum_k U_ik H[j][k]) b_j with n as its token rows;
+// then E = W - W_approx and the sums, through a transposing shared tile.
 
-namespace dres {
-constexpr int kTile = 128;  // rows and columns of W per CTA
-constexpr int kMicro = 8;   // rows and columns per thread
-constexpr int kChunk = 32;  // r per staging step (one U word per row)
-}  // namespace dres
-
-struct DbfResParams {
-  const float* W;
-  const uint16_t* a;
-  const uint32_t* U;  // [m][r/32]
-  const uint16_t* mid;
-  const uint32_t* V;  // [r][n/32]
-  const uint16_t* b;
-  float* E;
-  int m, r, n;
-  double* partials;
-  unsigned int* ticket;
-  double* out;
-};
-
-__global__ void __launch_bounds__(meas::kThreads) dbf_residual_kernel(DbfResParams p) {
-  using namespace dres;
-  __shared__ uint32_t Vs[kChunk][kTile / 32];
-  __shared__ float Ms[kChunk];
-  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-  const int i0 = blockIdx.y * kTile + ty * kMicro;  // this thread's first row
-  const int j0 = blockIdx.x * kTile + tx * kMicro;  // and first column
-  const int rw = p.r >> 5, nw = p.n >> 5;
+// H [n][r] (fp16 bits: mid_k with V's sign) and bs [n] = b as float.  One
+// warp per 32 x 32 block of V: lane l holds row k = 32 kb + l's word.
+__global__ void __launch_bounds__(meas::kThreads) dres_h_kernel(const uint32_t* __restrict__ V,
+                                                                 const uint16_t* __restrict__ mid,
+                                                                 const uint16_t* __restrict__ b, int r, int n,
+                                                                 uint16_t* __restrict__ H, float* __restrict__ bs) {
   pdl_wait();
-  float acc[kMicro][kMicro];
-#pragma unroll
-  for (int u = 0; u < kMicro; ++u)
-#pragma unroll
-    for (int v = 0; v < kMicro; ++v) acc[u][v] = 0.f;
-
-  for (int kc = 0; kc < rw; ++kc) {
-    __syncthreads();
-    if (threadIdx.x < kChunk * (kTile / 32)) {
-      const int kk = threadIdx.x >> 2, c = threadIdx.x & 3;
-      Vs[kk][c] = __ldg(p.V + static_cast<size_t>(kc * kChunk + kk) * nw + (blockIdx.x * kTile >> 5) + c);
-    } else if (threadIdx.x < kChunk * (kTile / 32) + kChunk) {
-      const int kk = threadIdx.x - kChunk * (kTile / 32);
-      Ms[kk] = meas_half_to_float(__ldg(p.mid + kc * kChunk + kk));
-    }
-    uint32_t uw[kMicro];
-#pragma unroll
-    for (int u = 0; u < kMicro; ++u) uw[u] = __ldg(p.U + static_cast<size_t>(i0 + u) * rw + kc);
-    __syncthreads();
-    const int vshift = (tx * kMicro) & 31, vword = (tx * kMicro) >> 5;
+  const int lane = threadIdx.x & 31;
+  const int64_t blk = static_cast<int64_t>(blockIdx.x) * (meas::kThreads / 32) + (threadIdx.x >> 5);
+  const int nw = n >> 5, rw = r >> 5;
+  if (blk < static_cast<int64_t>(nw) * rw) {  // warp-uniform
+    const int kb = static_cast<int>(blk / nw), jb = static_cast<int>(blk - static_cast<int64_t>(kb) * nw);
+    const int k = kb * 32 + lane;
+    const uint32_t w = __ldg(V + static_cast<int64_t>(k) * nw + jb);
+    const uint32_t mk = __ldg(mid + k);
 #pragma unroll 4
-    for (int kk = 0; kk < kChunk; ++kk) {
-      const float mk = Ms[kk];
-      const uint32_t vb = Vs[kk][vword] >> vshift;
-      float vm[kMicro], su[kMicro];
-#pragma unroll
-      for (int v = 0; v < kMicro; ++v) vm[v] = ((vb >> v) & 1u) ? -mk : mk;
-#pragma unroll
-      for (int u = 0; u < kMicro; ++u) su[u] = ((uw[u] >> kk) & 1u) ? -1.f : 1.f;
-#pragma unroll
-      for (int u = 0; u < kMicro; ++u)
-#pragma unroll
-        for (int v = 0; v < kMicro; ++v) acc[u][v] = fmaf(su[u], vm[v], acc[u][v]);
-    }
+    for (int jj = 0; jj < 32; ++jj)
+      H[static_cast<int64_t>(jb * 32 + jj) * r + k] = static_cast<uint16_t>(mk ^ (((w >> jj) & 1u) << 15));
+    if (kb == 0) bs[jb * 32 + lane] = meas_half_to_float(__ldg(b + jb * 32 + lane));
   }
+  pdl_launch_dependents();
+}
 
-  // W_approx = (acc a_i) b_j in fp32; E = W - W_approx.
+// E = W - W_approx (W_approx read transposed through a 64 x 64 shared tile),
+// sum E^2 and sum W^2.  CTAs stride over the tiles.
+namespace dres {
+constexpr int kT = 64;
+}
+__global__ void __launch_bounds__(meas::kThreads) dres_e_kernel(const float* __restrict__ W,
+                                                                 const float* __restrict__ WaT, int m, int n,
+                                                                 float* __restrict__ E, double* partials,
+                                                                 unsigned int* ticket, double* out) {
+  using dres::kT;
+  __shared__ float T[kT][kT + 1];
+  pdl_wait();
+  const int tn = n / kT, tiles = (m / kT) * tn;
   double e2 = 0.0, w2 = 0.0;
-  float bj[kMicro];
-#pragma unroll
-  for (int v = 0; v < kMicro; ++v) bj[v] = meas_half_to_float(__ldg(p.b + j0 + v));
-#pragma unroll
-  for (int u = 0; u < kMicro; ++u) {
-    const float ai = meas_half_to_float(__ldg(p.a + i0 + u));
-    const float4* wr = reinterpret_cast<const float4*>(p.W + static_cast<size_t>(i0 + u) * p.n + j0);
-    const float4 w0 = __ldcs(wr), w1 = __ldcs(wr + 1);
-    const float wv[kMicro] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-    float ev[kMicro];
-#pragma unroll
-    for (int v = 0; v < kMicro; ++v) {
-      ev[v] = wv[v] - (acc[u][v] * ai) * bj[v];
-      e2 += static_cast<double>(ev[v]) * ev[v];
-      w2 += static_cast<double>(wv[v]) * wv[v];
+  for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
+    const int i0 = (t / tn) * kT, j0 = (t % tn) * kT;
+    __syncthreads();  // the previous tile's reads are done
+    for (int e = threadIdx.x; e < kT * kT; e += meas::kThreads) {
+      const int jj = e / kT, ii = e % kT;
+      T[jj][ii] = __ldcs(WaT + static_cast<int64_t>(j0 + jj) * m + i0 + ii);
     }
-    if (p.E) {
-      float4* er = reinterpret_cast<float4*>(p.E + static_cast<size_t>(i0 + u) * p.n + j0);
-      __stcs(er, make_float4(ev[0], ev[1], ev[2], ev[3]));
-      __stcs(er + 1, make_float4(ev[4], ev[5], ev[6], ev[7]));
+    __syncthreads();
+    for (int e = threadIdx.x; e < kT * kT; e += meas::kThreads) {
+      const int ii = e / kT, jj = e % kT;
+      const int64_t o = static_cast<int64_t>(i0 + ii) * n + j0 + jj;
+      const float w = __ldcs(W + o);
+      const float ev = w - T[jj][ii];
+      e2 += static_cast<double>(ev) * ev;
+      w2 += static_cast<double>(w) * w;
+      if (E) __stcs(E + o, ev);
     }
   }
-  meas_finish_pair(e2, w2, p.partials, p.ticket, p.out);
+  meas_finish_pair(e2, w2, partials, ticket, out);
 }
 
 // ----------------------------------------------------------------- power iteration
@@ -357,32 +329,59 @@ cudaError_t launch_residual_g128(const float* W, int64_t N, int64_t K, const uin
                      scales, E, ws.partials, ws.ticket, sums);
 }
 
+// The sign GEMM's parameter block and launcher (sign_gemm.cu, the same
+// translation unit of libw1).
+template <bool HALF_OUT>
+cudaError_t launch_sg_gemm(const SgParams& p, const void* bmat, int64_t bcols, cudaStream_t stream, int num_sms);
+
+// Workspace of dbf_residual: the measurement header, H [n][r] fp16,
+// W_approx^T [n][m] fp32, b [n] fp32.
+struct DresWs {
+  size_t h, wat, bs, total;
+};
+static DresWs dres_ws(int64_t m, int64_t r, int64_t n) {
+  DresWs d;
+  d.h = meas_align(measure_workspace_bytes(m, n));
+  d.wat = d.h + meas_align(static_cast<size_t>(2) * n * r);
+  d.bs = d.wat + meas_align(static_cast<size_t>(4) * n * m);
+  d.total = d.bs + meas_align(static_cast<size_t>(4) * n);
+  return d;
+}
+size_t dbf_residual_workspace_bytes(int64_t m, int64_t r, int64_t n) {
+  if (m <= 0 || r <= 0 || n <= 0) return 0;
+  return dres_ws(m, r, n).total;
+}
+
 cudaError_t launch_dbf_residual(const float* W, const uint16_t* a, const uint32_t* B1, const uint16_t* mid,
                                 const uint32_t* B2, const uint16_t* b, int64_t m, int64_t r, int64_t n, float* E,
-                                double* sums, void* workspace, cudaStream_t stream) {
+                                double* sums, void* workspace, cudaStream_t stream, int num_sms) {
   MeasWs ws = meas_ws(workspace, m, n);
-  const int64_t tiles = (m / dres::kTile) * (n / dres::kTile);
-  if (tiles > meas::kMaxResidualCtas || n / dres::kTile > 65535 || m / dres::kTile > 65535)
-    return cudaErrorNotSupported;
+  const DresWs L = dres_ws(m, r, n);
+  unsigned char* base = static_cast<unsigned char*>(workspace);
+  uint16_t* H = reinterpret_cast<uint16_t*>(base + L.h);
+  float* WaT = reinterpret_cast<float*>(base + L.wat);
+  float* bs = reinterpret_cast<float*>(base + L.bs);
   cudaError_t e = cudaMemsetAsync(ws.ticket, 0, sizeof(unsigned int), stream);
   if (e != cudaSuccess) return e;
-  DbfResParams p;
-  p.W = W;
-  p.a = a;
-  p.U = B1;
-  p.mid = mid;
-  p.V = B2;
-  p.b = b;
-  p.E = E;
-  p.m = static_cast<int>(m);
-  p.r = static_cast<int>(r);
-  p.n = static_cast<int>(n);
-  p.partials = ws.partials;
-  p.ticket = ws.ticket;
-  p.out = sums;
-  return meas_launch(dbf_residual_kernel, dim3(static_cast<unsigned>(n / dres::kTile),
-                                               static_cast<unsigned>(m / dres::kTile)),
-                     stream, p);
+  const int64_t hwarps = (n / 32) * (r / 32);
+  e = meas_launch(dres_h_kernel, dim3(static_cast<unsigned>((hwarps + 7) / 8)), stream, B2, mid, b,
+                  static_cast<int>(r), static_cast<int>(n), H, bs);
+  if (e != cudaSuccess) return e;
+  SgParams p = {};
+  p.signs = B1;
+  p.gscales = nullptr;
+  p.rdiag = a;
+  p.s1 = bs;
+  p.out_f = WaT;
+  p.M = static_cast<int>(n);
+  p.rows = static_cast<int>(m);
+  p.K = static_cast<int>(r);
+  e = launch_sg_gemm<false>(p, H, r, stream, num_sms);
+  if (e != cudaSuccess) return e;
+  const int64_t tiles = (m / dres::kT) * (n / dres::kT);
+  const int grid = static_cast<int>(std::min<int64_t>(tiles, std::min(8 * num_sms, meas::kMaxResidualCtas)));
+  return meas_launch(dres_e_kernel, dim3(static_cast<unsigned>(grid)), stream, W, static_cast<const float*>(WaT),
+                     static_cast<int>(m), static_cast<int>(n), E, ws.partials, ws.ticket, sums);
 }
 
 cudaError_t launch_power_iteration(const float* A, int64_t m, int64_t n, const float* v0, int64_t iters,

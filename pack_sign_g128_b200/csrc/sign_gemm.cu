@@ -304,7 +304,9 @@ __global__ void __launch_bounds__(sg::kThreads, 1)
     // scale, or 0x3C00 = 1.0; the sign bit comes straight from the word),
     // stored as 16-byte chunks of the row in the two 128B-swizzled K-major
     // atoms.  Words and scales stream through a kPf-deep register ring over
-    // this CTA's (tile, stage) sequence so L2 latency hides behind kPf stages.
+    // this CTA's (tile, stage) sequence so L2 latency hides behind kPf stages
+    // (8 deep for 128-token tiles measured slower: 0.114 vs 0.075 ms for the
+    // 4096^3 DBF chain at 512 rows).
     constexpr int kPf = 4;
     const int rl = (warp - 2) * 32 + lane;
     const int64_t wrow = p.K >> 5;

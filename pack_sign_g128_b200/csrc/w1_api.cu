@@ -21,7 +21,8 @@ cudaError_t launch_residual_g128(const float* W, int64_t N, int64_t K, const uin
                                  float* E, double* sums, void* workspace, cudaStream_t stream, int num_sms);
 cudaError_t launch_dbf_residual(const float* W, const uint16_t* a, const uint32_t* B1, const uint16_t* mid,
                                 const uint32_t* B2, const uint16_t* b, int64_t m, int64_t r, int64_t n, float* E,
-                                double* sums, void* workspace, cudaStream_t stream);
+                                double* sums, void* workspace, cudaStream_t stream, int num_sms);
+size_t dbf_residual_workspace_bytes(int64_t m, int64_t r, int64_t n);
 cudaError_t launch_power_iteration(const float* A, int64_t m, int64_t n, const float* v0, int64_t iters,
                                    double* sigma, void* workspace, cudaStream_t stream, int num_sms);
 cudaError_t launch_okt_rotate(const float* H, int n1, const float* R, int n2, const uint16_t* x, int B, float* out,
@@ -227,7 +228,7 @@ int dbf_residual(const float* W, const uint16_t* a, const uint32_t* B1, const ui
   if (!W || !a || !B1 || !mid || !B2 || !b || !sums) return W1_ERR_NULL;
   if (m <= 0 || r <= 0 || n <= 0 || (m % 128) != 0 || (r % 128) != 0 || (n % 128) != 0) return W1_ERR_SHAPE;
   if ((m / 128) * (n / 128) > 8192 || r > ((int64_t)1 << 24)) return W1_ERR_SHAPE;
-  if (!workspace || ws_bytes < measure_workspace_bytes(m, n)) return W1_ERR_WORKSPACE;
+  if (!workspace || ws_bytes < dbf_residual_workspace_bytes(m, r, n)) return W1_ERR_WORKSPACE;
   if (!aligned16(W) || !aligned16(a) || !aligned16(B1) || !aligned16(mid) || !aligned16(B2) || !aligned16(b) ||
       (E && !aligned16(E)) || !aligned16(workspace) || !aligned8(sums))
     return W1_ERR_ALIGN;
@@ -235,7 +236,12 @@ int dbf_residual(const float* W, const uint16_t* a, const uint32_t* B1, const ui
   int st = device_info(&d);
   if (st != W1_OK) return st;
   return launch_result(launch_dbf_residual(W, a, B1, mid, B2, b, m, r, n, E, sums, workspace,
-                                           reinterpret_cast<cudaStream_t>(stream)));
+                                           reinterpret_cast<cudaStream_t>(stream), d.sms));
+}
+
+size_t dbf_residual_workspace_size(int64_t m, int64_t r, int64_t n) {
+  if (m <= 0 || r <= 0 || n <= 0 || (m % 128) != 0 || (r % 128) != 0 || (n % 128) != 0) return 0;
+  return dbf_residual_workspace_bytes(m, r, n);
 }
 
 int w1_power_iteration(const float* A, int64_t m, int64_t n, const float* v0, int64_t iters, double* sigma,

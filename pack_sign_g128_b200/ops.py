@@ -170,6 +170,10 @@ def w1_residual(W: torch.Tensor, signs: torch.Tensor, scales: torch.Tensor, E: t
     return (E if want_E else None), sums
 
 
+def dbf_residual_workspace_size(m: int, r: int, n: int) -> int:
+    return int(_lib.fn("dbf_residual_workspace_size")(m, r, n))
+
+
 def dbf_residual(W: torch.Tensor, a: torch.Tensor, B1: torch.Tensor, mid: torch.Tensor, B2: torch.Tensor,
                  b: torch.Tensor, E: torch.Tensor | None = None, want_E: bool = True,
                  workspace: torch.Tensor | None = None, stream=None):
@@ -185,7 +189,7 @@ def dbf_residual(W: torch.Tensor, a: torch.Tensor, B1: torch.Tensor, mid: torch.
         E = torch.empty((m, n), dtype=torch.float32, device=W.device)
     sums = torch.empty(2, dtype=torch.float64, device=W.device)
     if workspace is None:
-        workspace = measure_workspace(m, n, W.device)
+        workspace = torch.empty(max(dbf_residual_workspace_size(m, r, n), 1), dtype=torch.uint8, device=W.device)
     st = _lib.fn("dbf_residual")(_ptr(W), _ptr(a), _ptr(B1), _ptr(mid), _ptr(B2), _ptr(b), m, r, n,
                                  _ptr(E) if want_E else None, _ptr(sums), _ptr(workspace), workspace.numel(),
                                  _stream(stream, W))

@@ -164,7 +164,8 @@ def test_measure_host_side_argument_errors(lib):
     assert res(good, 256, 512, good, good, None, good, good, ws - 1, None) == _lib.W1_ERR_WORKSPACE
     assert res(good, 256, 512, good, good, odd, good, good, ws, None) == _lib.W1_ERR_ALIGN
     d = lib.dbf_residual
-    wsd = lib.w1_measure_workspace_size(256, 384)
+    wsd = lib.dbf_residual_workspace_size(256, 128, 384)
+    assert wsd >= 2 * 384 * 128 + 4 * 384 * 256 and lib.dbf_residual_workspace_size(256, 100, 384) == 0
     args = [good] * 6
     assert d(None, *args[1:], 256, 128, 384, None, good, good, wsd, None) == _lib.W1_ERR_NULL
     assert d(*args, 256, 100, 384, None, good, good, wsd, None) == _lib.W1_ERR_SHAPE
