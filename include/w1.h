@@ -107,8 +107,9 @@ int w1_pack(const float* W, int64_t N, int64_t K, uint32_t* signs, uint16_t* sca
  * a time; section 5: sign selection and addition).
  *   y[b][n] = sum_g s[n][g] * sum_{k in g} (1 - 2*bit[n][k]) * x[b][k],  1 <= B <= 8.
  *   signs [N][K/32], scales [N][K/128], x bf16 [B][K], y fp32 [B][N] (all device).
- * Accuracy: |y - y_exact| <= 1e-3 * sum_k |s x_k| per element (x is taken as
- * 24-bit fixed point per 128-group, fp32 accumulation).
+ * Accuracy: |y - y_exact| <= 1e-3 * sum_k |s x_k| per element (fp32
+ * accumulation; the int8 kernels take x as 24-bit fixed point per 128-group,
+ * the bf16 ones multiply x unchanged by +-1).
  * Kernel choice: the first call for a new (N, K, B) on a device, when `stream`
  * is not being captured, times the candidate kernels and K splits on `stream`
  * with the caller's buffers and keeps the fastest; that call blocks the host

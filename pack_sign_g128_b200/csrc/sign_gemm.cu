@@ -452,7 +452,9 @@ template <bool PHASE1>
 cudaError_t launch_sg_gemm(const SgParams& p, const void* bmat, int64_t bcols, cudaStream_t stream, int num_sms) {
   const int nt = (p.rows + sg::BN - 1) / sg::BN;
   const int tiles256 = ((p.M + 255) / 256) * nt;
-  if (tiles256 >= num_sms) return launch_sg_gemm_bm<PHASE1, 256>(p, bmat, bcols, stream, num_sms);
+  const int force = knob(kKnobSgBm);  // tuning knob: force the token tile
+  if (force == 256 || (force != 128 && tiles256 >= num_sms))
+    return launch_sg_gemm_bm<PHASE1, 256>(p, bmat, bcols, stream, num_sms);
   return launch_sg_gemm_bm<PHASE1, 128>(p, bmat, bcols, stream, num_sms);
 }
 

@@ -82,7 +82,8 @@ def test_dbf_residual_of_a_dbf_matrix_is_small():
 
 
 @pytest.mark.parametrize("m,n,iters", [(512, 1024, 32), (4096, 4096, 32), (300, 1160, 32), (1, 128, 32),
-                                       (64, 4, 32), (1000, 2048, 0), (777, 512, 5)])
+                                       (64, 4, 32), (1000, 2048, 0), (777, 512, 5), (200, 8192, 7),
+                                       (96, 8320, 4)])
 def test_power_iteration_parity(m, n, iters):
     A = synth.weights(synth.rng(74), m, n, std=1.0)
     v0 = synth.start_vector(n)
