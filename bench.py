@@ -944,19 +944,23 @@ def run_gpu(args):
     dom = max(per_kernel, key=lambda k: per_kernel[k]["ms"])
     dk = per_kernel[dom]
     achieved = dk["bytes"] / (dk["ms"] * 1e-3) / 1e9
-    # DRAM traffic per launch: each pair's own capture (none scaled from another pair)
+    # DRAM traffic per launch: each pair's own capture (none scaled from another
+    # pair); the line's figure is the launch-weighted mean over the pairs whose
+    # first-call choice has a capture, with the share of launches it covers
     cap_bytes = 0.0
-    cap_all = True
+    cap_launches = 0
     for cb, row in zip(combos, gemv_rows):
         if row["kernel"] != dom:
             continue
         t = CAPTURED_TRAFFIC.get((cb["N"], cb["K"], cb["B"], row["choice"]))
         row["traffic_bytes_per_launch"] = t
-        if t is None:
-            cap_all = False
-        else:
+        if t is not None:
             cap_bytes += t * cb["R"] * args.steps
-    traffic = round(cap_bytes / dk["launches"]) if cap_all else None
+            cap_launches += cb["R"] * args.steps
+    traffic = round(cap_bytes / cap_launches) if cap_launches else None
+    cap_alg = sum(cb["bytes"] * cb["R"] * args.steps for cb, row in zip(combos, gemv_rows)
+                  if row["kernel"] == dom and row.get("traffic_bytes_per_launch") is not None)
+    traffic_vs_alg = round(cap_bytes / cap_alg, 4) if cap_alg else None
     dom_share = dk["ms"] / sum(per_pair_ms)
 
     e2e = gemv_e2e(torch, ops, combos, max(1, min(args.steps, 3)))
@@ -1003,8 +1007,10 @@ def run_gpu(args):
                      "traffic": traffic, "kernel": dom, "time_share": round(dom_share, 4),
                      "algorithmic_bytes_per_launch": round(dk["bytes"] / dk["launches"]),
                      "traffic_note": ("launch-weighted mean of each pair's own ncu capture (DRAM read + write "
-                                      "bytes of one launch); null unless every pair of the kernel has one; "
+                                      "bytes of one launch) over the pairs whose kernel choice was captured; "
                                       "per-pair figures in rows.gemv[*].traffic_bytes_per_launch"),
+                     "traffic_launch_coverage": round(cap_launches / dk["launches"], 4),
+                     "traffic_vs_algorithmic": traffic_vs_alg,
                      "peak_kind": peaks_kind},
         "cpu_baseline": cpu,
         "e2e": {k: e2e[k] for k in ("value", "unit", "h2d_bytes_per_step", "d2h_bytes_per_step")},
