@@ -565,12 +565,15 @@ def dbf_rows(torch, ops, synth, peaks, l2_bytes: int, iters: int = 5, only_b: in
                    "frac_hbm": round(gbs / peaks["hbm_gbs"], 4), "calls": R}
             # the small-batch chain forms side by side (fused kernel vs two launches)
             forms = {}
-            for form in ("fused", "twostep"):
+            for form, core in (("fused", None), ("twostep", None), ("twostep", "direct")):
                 ops.set_knob("dbf_path", form)
+                if core:
+                    ops.set_knob("dbf_core", core)
                 try:
-                    forms[form] = round(graph_us(), 3)
+                    forms[form + ("_" + core if core else "")] = round(graph_us(), 3)
                 finally:
                     ops.set_knob("dbf_path", None)
+                    ops.set_knob("dbf_core", None)
             row["us_by_form"] = forms
             # split rank: r partitioned over the CTAs of a cluster in U . h (two-launch form)
             splits = {}

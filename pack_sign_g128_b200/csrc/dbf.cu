@@ -284,6 +284,9 @@ cudaError_t launch_dbf_tc(const uint16_t* a, const uint32_t* B1, const uint16_t*
 cudaError_t launch_gemv_direct_diag(const uint32_t* signs, int64_t N, int64_t K, const void* x, bool x_f32,
                                     const uint16_t* cdiag, const uint16_t* rdiag, int B, float* y, bool early,
                                     cudaStream_t stream, int num_sms, int smem_cap, int warps, int force_s);
+cudaError_t launch_gemv_flat_diag(const uint32_t* signs, int64_t N, int64_t K, const void* x, bool x_f32,
+                                  const uint16_t* cdiag, const uint16_t* rdiag, int B, float* y, bool early,
+                                  cudaStream_t stream, int num_sms, int smem_cap, int split, int warps);
 
 // Batches of at least this many rows run on the tensor-core path.
 constexpr int64_t kDbfTensorMinBatch = 64;
@@ -334,11 +337,25 @@ cudaError_t launch_dbf(const uint16_t* a, const uint32_t* B1, const uint16_t* mi
       // K split is the split-rank form of section 5 item 5 (r partitioned
       // over the CTAs of a cluster, partial outputs added in a fixed order
       // through distributed shared memory); dbf_rank_split forces it.
+      // Each product on the register-fed GEMV core (1-2 rows, int8 digits)
+      // where its plan fits and no rank split is forced, else on the direct
+      // core.
       const int warps = wknob ? wknob : (nb >= 4 ? 16 : 8);
-      err = launch_gemv_direct_diag(B2, r, n, xg, false, b, mid, nb, h, false, stream, num_sms, smem_cap, warps, 0);
-      if (err == cudaSuccess)
-        err = launch_gemv_direct_diag(B1, m, r, h, true, nullptr, a, nb, yg, true, stream, num_sms, smem_cap, warps,
-                                      knob(kKnobDbfRankSplit));
+      const int rsplit = knob(kKnobDbfRankSplit);
+      const int cknob = knob(kKnobDbfCore);  // 0: flat where it fits, 1: flat, 2: direct
+      const bool try_flat = cknob != 2 && nb <= 2;
+      err = cudaErrorNotSupported;
+      if (try_flat) err = launch_gemv_flat_diag(B2, r, n, xg, false, b, mid, nb, h, false, stream, num_sms, smem_cap, 0, 8);
+      if (err == cudaErrorNotSupported)
+        err = launch_gemv_direct_diag(B2, r, n, xg, false, b, mid, nb, h, false, stream, num_sms, smem_cap, warps, 0);
+      if (err == cudaSuccess) {
+        err = cudaErrorNotSupported;
+        if (try_flat && rsplit == 0)
+          err = launch_gemv_flat_diag(B1, m, r, h, true, nullptr, a, nb, yg, true, stream, num_sms, smem_cap, 0, 8);
+        if (err == cudaErrorNotSupported)
+          err = launch_gemv_direct_diag(B1, m, r, h, true, nullptr, a, nb, yg, true, stream, num_sms, smem_cap, warps,
+                                        rsplit);
+      }
       if (err != cudaSuccess) return err;
       continue;
     }

@@ -79,6 +79,11 @@ struct FlParams {
   int gw;     // max groups per warp
   int chunk;  // rows owned per CTA in the cluster reduction
   int early;  // read weights before the grid dependency wait
+  // diagonal form (a step of the DBF chain; no group scales):
+  // y[b][n] = rdiag[n] * sum_k s(n, k) * (cdiag[k] *) x[b][k]
+  const uint16_t* cdiag;  // fp16 [K], bf16 x only, or nullptr
+  const uint16_t* rdiag;  // fp16 [N], or nullptr
+  int x_f32;              // x is fp32 [B][K]
 };
 
 struct FlSmem {
@@ -150,17 +155,11 @@ __device__ __forceinline__ bool fl_wait(uint64_t* bar) { return mbar_wait_warp(b
 // Lanes of the 8-lane set of one (group, batch row) share the group maximum;
 // lane (cq, h) == (0, 0) writes the fold factors f1, f2 (2^(E-22) = f1 f2)
 // and X f (X = the sum of the group's 23-bit integers).
-__device__ __forceinline__ void fl_quantise_unit(const uint4 (&r)[2], bool store, uint32_t* dig, float* fold, int b,
-                                                 int cq, int h) {
-  const uint32_t w[8] = {r[0].x, r[0].y, r[0].z, r[0].w, r[1].x, r[1].y, r[1].z, r[1].w};
-  float v[16];
+__device__ __forceinline__ void fl_quantise_values(const float (&v)[16], bool store, uint32_t* dig, float* fold,
+                                                   int b, int cq, int h) {
   float m8[8];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    v[2 * j] = __uint_as_float(w[j] << 16);
-    v[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
-    m8[j] = fmaxf(fabsf(v[2 * j]), fabsf(v[2 * j + 1]));
-  }
+  for (int j = 0; j < 8; ++j) m8[j] = fmaxf(fabsf(v[2 * j]), fabsf(v[2 * j + 1]));
 #pragma unroll
   for (int s = 4; s >= 1; s >>= 1)
 #pragma unroll
@@ -208,6 +207,17 @@ __device__ __forceinline__ void fl_quantise_unit(const uint4 (&r)[2], bool store
     fold[b * 4 + 2] = (static_cast<float>(xs) * f1) * f2;
   }
 }
+__device__ __forceinline__ void fl_quantise_unit(const uint4 (&r)[2], bool store, uint32_t* dig, float* fold, int b,
+                                                 int cq, int h) {
+  const uint32_t w[8] = {r[0].x, r[0].y, r[0].z, r[0].w, r[1].x, r[1].y, r[1].z, r[1].w};
+  float v[16];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    v[2 * j] = __uint_as_float(w[j] << 16);
+    v[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+  }
+  fl_quantise_values(v, store, dig, fold, b, cq, h);
+}
 
 // The warp's products over its groups for all T tiles of the CTA's rows,
 // then (after a CTA barrier: the reduction buffer overlays the fragment
@@ -221,7 +231,7 @@ __device__ __forceinline__ void fl_quantise_unit(const uint4 (&r)[2], bool store
 // acc[t][e][c]: partial sum of row 16 t + lane/4 + 8 e, result column
 // 2 (lane%4) + c (int8: digit column 3b + d, bf16: batch row).
 // `prologue` is the grid dependency wait and what must follow it.
-template <int NB, int NW, int T, class Prologue>
+template <int NB, int NW, int T, bool DIAG, class Prologue>
 __device__ __forceinline__ void fl_products(const FlParams& p, int row0, int g0, int G, int wg0, int nwg,
                                             const unsigned char* wts, uint64_t* bars, int nbox, uint32_t* dig,
                                             float* fold, const uint16_t* scl, uint64_t* sbar, int lane, float* red,
@@ -240,7 +250,54 @@ __device__ __forceinline__ void fl_products(const FlParams& p, int row0, int g0,
   const int r1 = lane >> 2, cq = lane & 3;
   prologue();
   // ---- 1. int8 form: activations -> digit fragments in shared memory
-  if constexpr (!C::BF) {
+  if constexpr (DIAG) {
+    // fp32 x (read through L2: the preceding launch wrote it), or bf16 x
+    // times the column diagonal (exact in fp32)
+    static_assert(!C::BF, "the diagonal form has the int8 products only");
+    const int U = nwg * NB * 8;
+    for (int u = lane; u - lane < U; u += 32) {  // trip count uniform over the warp
+      const int gl = u / (8 * NB), b = (u >> 3) % NB, ucq = (u >> 1) & 3, h = u & 1;
+      float v[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) v[i] = 0.f;
+      if (u < U) {
+        const int64_t k0 = static_cast<int64_t>(g0 + wg0 + gl) * 128 + 32 * ucq + 16 * h;
+        if (p.x_f32) {
+          const float4* src = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(p.x) +
+                                                              static_cast<int64_t>(b) * p.K + k0);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float4 f = __ldcg(src + i);
+            v[4 * i] = f.x;
+            v[4 * i + 1] = f.y;
+            v[4 * i + 2] = f.z;
+            v[4 * i + 3] = f.w;
+          }
+        } else {
+          const uint4* src = reinterpret_cast<const uint4*>(p.x + static_cast<int64_t>(b) * p.K + k0);
+          const uint4 r0 = __ldg(src), r1x = __ldg(src + 1);
+          const uint32_t w[8] = {r0.x, r0.y, r0.z, r0.w, r1x.x, r1x.y, r1x.z, r1x.w};
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            v[2 * j] = __uint_as_float(w[j] << 16);
+            v[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+          }
+          if (p.cdiag) {
+            const uint4* dg = reinterpret_cast<const uint4*>(p.cdiag + k0);
+            const uint4 d0 = __ldg(dg), d1 = __ldg(dg + 1);
+            const uint32_t dd[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&dd[j]));
+              v[2 * j] *= f.x;  // bf16 x fp16: exact in fp32
+              v[2 * j + 1] *= f.y;
+            }
+          }
+        }
+      }
+      fl_quantise_values(v, u < U, dig + gl * C::GW, fold + gl * NB * 4, b, ucq, h);
+    }
+  } else if constexpr (!C::BF) {
     const int U = nwg * NB * 8;
     constexpr int UPL = C::UPL;
     uint4 xr[UPL][2];
@@ -384,7 +441,7 @@ __device__ __forceinline__ void fl_products(const FlParams& p, int row0, int g0,
           acc[t][1][1] = fmaf(s1, cc[g][t][3], acc[t][1][1]);
         }
       } else {
-        // acc += s * (f1 f2 2 W_d C + [d = hi] f X)
+        // acc += s * (f1 f2 2 W_d C + [d = hi] f X)   (s = 1 in the diagonal form)
         float f1[2], f2[2], fx[2];
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
@@ -395,8 +452,8 @@ __device__ __forceinline__ void fl_products(const FlParams& p, int row0, int g0,
         }
 #pragma unroll
         for (int t = 0; t < T; ++t) {
-          const float s0 = __half2float(__ushort_as_half(sg[16 * t * p.NG]));
-          const float s1 = __half2float(__ushort_as_half(sg[(16 * t + 8) * p.NG]));
+          const float s0 = DIAG ? 1.f : __half2float(__ushort_as_half(sg[16 * t * p.NG]));
+          const float s1 = DIAG ? 1.f : __half2float(__ushort_as_half(sg[(16 * t + 8) * p.NG]));
 #pragma unroll
           for (int c = 0; c < 2; ++c) {
             acc[t][0][c] = fmaf(s0, (cw[c] * static_cast<float>(cc[g][t][c]) * f1[c]) * f2[c] + fx[c], acc[t][0][c]);
@@ -428,7 +485,7 @@ __device__ __forceinline__ void fl_products(const FlParams& p, int row0, int g0,
     }
 }
 
-template <int NB, int NW>
+template <int NB, int NW, bool DIAG = false>
 __global__ void __launch_bounds__(NW * 32, 1) gemv_flat_kernel(const __grid_constant__ CUtensorMap tmap,
                                                                const FlParams p) {
   using C = fl::Cfg<NB>;
@@ -470,14 +527,18 @@ __global__ void __launch_bounds__(NW * 32, 1) gemv_flat_kernel(const __grid_cons
         mbar_arrive_expect_tx(&bars[b], static_cast<uint32_t>(p.R * 128));
         tma_load_2d(smem + L.wts + b * p.R * 128, &tmap, (g0 + bs) * 4, row0, &bars[b]);
       }
-      const uint32_t sbytes = static_cast<uint32_t>(rows) * p.NG * 2;
-      const uint32_t sbulk = sbytes & ~15u;
-      const uint16_t* ssrc = p.scales + static_cast<int64_t>(row0) * p.NG;
-      for (uint32_t i = sbulk / 2; i < sbytes / 2; ++i) scl[i] = __ldg(ssrc + i);
-      mbar_arrive_expect_tx(&sbar, sbulk);
-      for (uint32_t off = 0; off < sbulk; off += 32768)
-        bulk_g2s(reinterpret_cast<unsigned char*>(scl) + off, reinterpret_cast<const unsigned char*>(ssrc) + off,
-                 min(32768u, sbulk - off), &sbar);
+      if (DIAG) {
+        mbar_arrive(&sbar);  // no group scales
+      } else {
+        const uint32_t sbytes = static_cast<uint32_t>(rows) * p.NG * 2;
+        const uint32_t sbulk = sbytes & ~15u;
+        const uint16_t* ssrc = p.scales + static_cast<int64_t>(row0) * p.NG;
+        for (uint32_t i = sbulk / 2; i < sbytes / 2; ++i) scl[i] = __ldg(ssrc + i);
+        mbar_arrive_expect_tx(&sbar, sbulk);
+        for (uint32_t off = 0; off < sbulk; off += 32768)
+          bulk_g2s(reinterpret_cast<unsigned char*>(scl) + off, reinterpret_cast<const unsigned char*>(ssrc) + off,
+                   min(32768u, sbulk - off), &sbar);
+      }
     }
   };
   // The next launch in the stream may start now: its own grid dependency wait
@@ -496,7 +557,8 @@ __global__ void __launch_bounds__(NW * 32, 1) gemv_flat_kernel(const __grid_cons
   switch (p.T) {  // uniform over the grid
 #define W1_FL_CASE(TV) \
   case TV:                                                                                                \
-    fl_products<NB, NW, TV>(p, row0, g0, G, wg0, nwg, wts, bars, nbox, dig, fold, scl, &sbar, lane, red, prologue); \
+    fl_products<NB, NW, TV, DIAG>(p, row0, g0, G, wg0, nwg, wts, bars, nbox, dig, fold, scl, &sbar, lane, red, \
+                                  prologue);                                                                   \
     break;
     W1_FL_CASE(1)
     W1_FL_CASE(2)
@@ -533,6 +595,7 @@ __global__ void __launch_bounds__(NW * 32, 1) gemv_flat_kernel(const __grid_cons
         sum += (rp[0] + rp[1]) + rp[2];
       }
     }
+    if (DIAG && p.rdiag && row0 + r < p.N) sum *= __half2float(__ushort_as_half(p.rdiag[row0 + r]));
     if (p.S == 1) {
       if (row0 + r < p.N) p.y[static_cast<int64_t>(b) * p.N + row0 + r] = sum;
     } else {
@@ -549,6 +612,7 @@ __global__ void __launch_bounds__(NW * 32, 1) gemv_flat_kernel(const __grid_cons
       float sum = 0.f;
       for (int c = 0; c < p.S; ++c) sum += inbox[(c * NB + b) * p.chunk + ro];
       const int row = row0 + lo + ro;
+      if (DIAG && p.rdiag && row < p.N) sum *= __half2float(__ushort_as_half(p.rdiag[row]));
       if (row < p.N) p.y[static_cast<int64_t>(b) * p.N + row] = sum;
     }
   }
@@ -588,7 +652,7 @@ static bool fl_plan_for(int N, int NG, int S, int num_sms, int smem_cap, FlPlan*
   return true;
 }
 
-template <int NB, int NW>
+template <int NB, int NW, bool DIAG = false>
 static cudaError_t launch_gemv_flat_nb(const FlParams& base, cudaStream_t stream, int num_sms, int smem_cap, int S) {
   FlPlan plan;
   if (!fl_plan_for<NB, NW>(base.N, base.NG, S, num_sms, smem_cap, &plan)) return cudaErrorNotSupported;
@@ -604,7 +668,7 @@ static cudaError_t launch_gemv_flat_nb(const FlParams& base, cudaStream_t stream
   p.chunk = plan.chunk;
   CUtensorMap tmap;
   if (!make_tmap_u32_sw128(&tmap, base.signs, base.N, base.K / 32, plan.R)) return cudaErrorInvalidValue;
-  cudaError_t err = ensure_dyn_smem(reinterpret_cast<const void*>(gemv_flat_kernel<NB, NW>), plan.smem);
+  cudaError_t err = ensure_dyn_smem(reinterpret_cast<const void*>(gemv_flat_kernel<NB, NW, DIAG>), plan.smem);
   if (err != cudaSuccess) return err;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(plan.Q * plan.S));
@@ -625,7 +689,7 @@ static cudaError_t launch_gemv_flat_nb(const FlParams& base, cudaStream_t stream
   }
   cfg.attrs = attr;
   cfg.numAttrs = na;
-  return cudaLaunchKernelEx(&cfg, gemv_flat_kernel<NB, NW>, tmap, p);
+  return cudaLaunchKernelEx(&cfg, gemv_flat_kernel<NB, NW, DIAG>, tmap, p);
 }
 
 template <int NW>
@@ -665,6 +729,43 @@ cudaError_t launch_gemv_flat(const uint32_t* signs, const uint16_t* scales, int6
   for (int S = split > 0 ? split : 1; S <= 8; S *= 2) {
     const cudaError_t e = warps == 16 ? launch_gemv_flat_nw<16>(p, B, stream, num_sms, smem_cap, S)
                                       : launch_gemv_flat_nw<8>(p, B, stream, num_sms, smem_cap, S);
+    if (e != cudaErrorNotSupported || split > 0) return e;
+  }
+  return cudaErrorNotSupported;
+}
+
+// The diagonal form (a step of the DBF chain, no group scales), 1 or 2 batch
+// rows: y[b][n] = rdiag[n] * sum_k s(n, k) * (cdiag[k] *) x[b][k], x bf16
+// [B][K] (with the fp16 column diagonal cdiag, or nullptr) or fp32 [B][K]
+// (x_f32; no cdiag); rdiag fp16 [N] or nullptr.  early: the sign words were
+// not written by the kernel this launch follows.  split as for
+// launch_gemv_flat; cudaErrorNotSupported when no plan fits.
+cudaError_t launch_gemv_flat_diag(const uint32_t* signs, int64_t N, int64_t K, const void* x, bool x_f32,
+                                  const uint16_t* cdiag, const uint16_t* rdiag, int B, float* y, bool early,
+                                  cudaStream_t stream, int num_sms, int smem_cap, int split, int warps) {
+  if (N > (int64_t)1 << 30 || K > (int64_t)1 << 30 || B < 1 || B > 2 || (x_f32 && cdiag))
+    return cudaErrorNotSupported;
+  FlParams p = {};
+  p.signs = signs;
+  p.scales = nullptr;
+  p.x = static_cast<const uint16_t*>(x);
+  p.y = y;
+  p.N = static_cast<int>(N);
+  p.K = static_cast<int>(K);
+  p.NG = static_cast<int>(K / 128);
+  p.early = early ? 1 : 0;
+  p.cdiag = cdiag;
+  p.rdiag = rdiag;
+  p.x_f32 = x_f32 ? 1 : 0;
+  smem_cap = std::min(2 * smem_cap, 227 * 1024);
+  for (int S = split > 0 ? split : 1; S <= 8; S *= 2) {
+    cudaError_t e;
+    if (warps == 16)
+      e = B == 1 ? launch_gemv_flat_nb<1, 16, true>(p, stream, num_sms, smem_cap, S)
+                 : launch_gemv_flat_nb<2, 16, true>(p, stream, num_sms, smem_cap, S);
+    else
+      e = B == 1 ? launch_gemv_flat_nb<1, 8, true>(p, stream, num_sms, smem_cap, S)
+                 : launch_gemv_flat_nb<2, 8, true>(p, stream, num_sms, smem_cap, S);
     if (e != cudaErrorNotSupported || split > 0) return e;
   }
   return cudaErrorNotSupported;

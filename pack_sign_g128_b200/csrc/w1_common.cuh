@@ -405,13 +405,14 @@ inline cudaError_t ensure_dyn_smem(const void* kernel, int bytes) {
 //   dbf_warps     W1_DBF_WARPS      0 = by group size, 8 or 16 warps per CTA
 //   dbf_rank_split W1_DBF_RANK_SPLIT two-launch chain: CTAs per cluster that split r in U . h (0 = planner)
 //   sg_bm         W1_SG_BM          sign GEMM token tile: 0 = by tile count, else 128 or 256
+//   dbf_core      W1_DBF_CORE       two-launch chain's GEMV core: 0 = register-fed where it fits, 1 = same, 2 = direct
 //   verbose       W1_VERBOSE        nonzero: plans and choices on stderr
 #include <atomic>
 #include <cstdlib>
 #include <cstring>
 namespace w1 {
 enum KnobId { kKnobGemvPath, kKnobGemvSplit, kKnobGemvAutotune, kKnobMoePath, kKnobDbfPath, kKnobDbfWarps,
-              kKnobDbfRankSplit, kKnobSgBm, kKnobVerbose, kKnobCount };
+              kKnobDbfRankSplit, kKnobSgBm, kKnobDbfCore, kKnobVerbose, kKnobCount };
 // GEMV kernels a knob can force (also the kinds of the dispatcher's choices).
 enum GemvPathKnob { kGemvAuto = 0, kGemvDirect8 = 1, kGemvDirect16 = 2, kGemvTc = 3, kGemvRing = 4, kGemvFlat = 5,
                     kGemvFlat16 = 6 };
@@ -433,6 +434,7 @@ inline const KnobSpec& knob_spec(int id) {
       {"dbf_warps", "W1_DBF_WARPS", 0, {nullptr}},
       {"dbf_rank_split", "W1_DBF_RANK_SPLIT", 0, {nullptr}},
       {"sg_bm", "W1_SG_BM", 0, {nullptr}},
+      {"dbf_core", "W1_DBF_CORE", 0, {"flat", "direct", nullptr}},
       {"verbose", "W1_VERBOSE", 0, {nullptr}},
   };
   return specs[id];

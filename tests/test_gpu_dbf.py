@@ -1,8 +1,9 @@
 """dbf_apply on the GPU vs the fp64 oracle chain.
 
 Every test runs with each small-batch chain form -- the fused chain kernel and
-two launches of the direct GEMV core (the dbf_path knob) -- forced to 8 and to
-16 warps per CTA (the dbf_warps knob).  Batches of 64 and more take the
+two launches of a GEMV core (the dbf_path knob; groups of 1-2 rows take the
+register-fed core, or the direct core with dbf_core=direct) -- forced to 8
+and to 16 warps per CTA (the dbf_warps knob).  Batches of 64 and more take the
 tensor-core path either way."""
 import functools
 
@@ -17,9 +18,12 @@ from gpu_helpers import assert_within, bf16_dev, fp16_dev, words_dev
 pytestmark = pytest.mark.gpu
 
 
-@pytest.fixture(autouse=True, params=["fused8", "fused16", "twostep8", "twostep16"])
+@pytest.fixture(autouse=True, params=["fused8", "fused16", "twostep8", "twostep16", "twostepdirect8"])
 def dbf_path(request, knob):
     form, warps = (request.param[:-2], request.param[-2:]) if request.param.endswith("16") else (request.param[:-1], "8")
+    if form == "twostepdirect":
+        form = "twostep"
+        knob("dbf_core", "direct")  # the direct GEMV core for 1-2 rows too
     knob("dbf_path", form)
     knob("dbf_warps", warps)
     return request.param
