@@ -79,9 +79,14 @@ int w1_sync_status(w1_stream_t stream);
  *   "gemv_path"     "direct" | "direct16" | "tc" | "ring" | "flat" forces one GEMV kernel (W1_GEMV_PATH)
  *   "gemv_split"    1 | 2 | 4 | 8: forced K split of the split-capable GEMV kernels (W1_GEMV_SPLIT)
  *   "gemv_autotune" "0": the static kernel rule instead of first-call timing (W1_GEMV_AUTOTUNE)
- *   "moe_path"      "tiles" | "decode" forces a routed-MoE path (W1_MOE_PATH)
+ *   "moe_path"      "tiles" | "decode" | "grouped" forces a routed-MoE path (W1_MOE_PATH)
  *   "dbf_path"      "fused" | "twostep" forces a small-batch DBF chain form (W1_DBF_PATH)
  *   "dbf_warps"     8 | 16 warps per CTA of the small-batch DBF chain (W1_DBF_WARPS)
+ *   "dbf_rank_split" 1..8 CTAs per cluster splitting r in the two-launch chain's U . h (W1_DBF_RANK_SPLIT)
+ *   "dbf_core"      "flat" | "direct": the two-launch chain's GEMV core (W1_DBF_CORE)
+ *   "sg_bm"         128 | 256 forces the sign GEMM's token tile (W1_SG_BM)
+ *   "sg_exp"        4 | 8 forces the sign GEMM's expander warps per CTA (W1_SG_EXP)
+ *   "sg_a"          "smem" | "tmem": where the sign GEMM's 128-token tiles keep the weight operand (W1_SG_A)
  *   "verbose"       nonzero prints plans and choices on stderr (W1_VERBOSE)
  * Returns W1_ERR_NULL for a NULL name, W1_ERR_SHAPE for an unknown name or
  * value. */

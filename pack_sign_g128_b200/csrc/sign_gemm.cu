@@ -11,18 +11,21 @@
 //  * sg_gemm_kernel: one CTA per SM, persistent over output tiles of 128
 //    weight rows x BM tokens (BM = 256, or 128 when 256-token tiles would not
 //    fill the GPU), swap-AB: D^T (TMEM, fp32, two accumulators of BM columns)
-//    = A (shared memory, +-s fp16) x xs^T (shared memory, fp16, by TMA),
-//    128 x BM x 16 MMAs.  Pipeline stages are 128 wide in K (one scale group,
-//    two 64-wide 128-byte swizzle atoms), 2 deep at BM = 256 and 3 deep at
-//    BM = 128 (192 KB either way):
+//    = A (+-s fp16) x xs^T (shared memory, fp16, by TMA), 128 x BM x 16 MMAs.
+//    A sits in shared memory (BM = 256) or in TMEM (BM = 128: row = lane, k
+//    pairs along the columns, beside the accumulators), which takes its
+//    writes and the MMA's reads of it off shared memory.  Pipeline stages are
+//    128 wide in K (one scale group, two 64-wide 128-byte swizzle atoms of
+//    xs), 2 deep at BM = 256 (192 KB), 4 deep with A in TMEM (128 KB):
 //    warp 0 TMA producer (xs: two BM x 64 boxes per stage, whose transaction
 //    bytes complete on the stage's full barrier); warp 1 MMA issuer (one wait
-//    per stage, then 8 MMAs, all of K into one accumulator per tile); warps
-//    2-5 expanders (thread = weight row: 4 sign words + the group scale -> 64
-//    fp16 pairs +-s, written as 16-byte chunks in the 128B-swizzled K-major
-//    layout the MMA reads, words prefetched 4 stages ahead in registers);
-//    warps 6-9 epilogue (thread = TMEM lane: row diagonal and token scale,
-//    store), draining one accumulator while the MMA fills the other.
+//    per stage, then 8 MMAs, all of K into one accumulator per tile); 4 or 8
+//    expander warps (thread = weight row, all of a stage or one 64-wide half:
+//    sign words + the group scale -> fp16 pairs +-s, written as 16-byte
+//    chunks in the 128B-swizzled K-major layout the MMA reads, or as TMEM
+//    columns; words prefetched 4 stages ahead in registers); 4 epilogue warps
+//    (thread = TMEM lane: row diagonal and token scale, store), draining one
+//    accumulator while the MMA fills the other.
 // Products of +-s and fp16 are exact in the tensor core; accumulation is fp32.
 #include <cstdint>
 #include <cuda.h>
@@ -35,24 +38,41 @@ namespace w1 {
 bool make_tmap_bf16_sw128(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int box_rows);
 
 namespace sg {
+// Expander warps per CTA for 256- and 128-token tiles, and where 128-token
+// tiles keep the weight operand.  Measured (one B200, the 4096^3 DBF chain at
+// 512 rows / the 2048 x 14336 x 4096 GEMM forced to 128-token tiles):
+// shared memory, 4 expanders 0.089 ms / 0.300 ms; TMEM, 4: 0.083 / 0.300;
+// TMEM, 8: 0.077 / 0.284.  256-token tiles: 8 expanders no faster (0.208 vs
+// 0.203 ms), and TMEM has no room for their weight stages beside two
+// 256-column accumulators.
+constexpr int kExp256 = 4;
+constexpr int kExp128 = 8;
+constexpr bool kTmemA128 = true;
 constexpr int BN = 128;   // weight rows per tile (MMA M, TMEM lanes)
 constexpr int BK = 128;   // K per scale group
 // K per pipeline stage: one scale group in two 64-wide (128-byte) swizzle
 // atoms, so the MMA issuer's one barrier wait per stage covers 8 MMAs
 constexpr int BKS = 128;
-constexpr int kThreads = 320;  // 10 warps
+// Warps: 0 TMA producer, 1 MMA issuer, 2 .. 2+EXP-1 expanders, then 4 epilogue
+// warps.  EXP = 4 (thread = weight row, whole stage) or 8 (thread = weight
+// row, one 64-wide atom of the stage).
+template <int EXP>
+constexpr int threads_for() { return (2 + EXP + 4) * 32; }
 constexpr int kAAtom = BN * 128;        // bytes of one 64-wide atom of the weight stage (16 KB)
 constexpr int kAStage = 2 * kAAtom;     // 32 KB
 
 // BMT tokens per tile (MMA N): 256 when there are enough tiles to fill the
-// GPU, 128 for few token rows (more tiles, each MMA half as long).
-template <int BMT>
+// GPU, 128 for few token rows (more tiles, each MMA half as long).  TA: the
+// weight operand lives in TMEM (128-token tiles only), so shared memory holds
+// only the token stages, 4 deep.
+template <int BMT, bool TA>
 struct Smem {
-  static constexpr int NS = BMT == 256 ? 2 : 3;  // stages (192 KB either way)
-  static constexpr int kXAtom = BMT * 128;       // bytes of one 64-wide atom of the token stage
+  static_assert(!TA || BMT == 128, "TMEM weight operand: 128-token tiles");
+  static constexpr int NS = TA ? 4 : BMT == 256 ? 2 : 3;  // stages (128 / 192 KB)
+  static constexpr int kXAtom = BMT * 128;                // bytes of one 64-wide atom of the token stage
   static constexpr int kXStage = 2 * kXAtom;
   alignas(1024) unsigned char x[NS][kXStage];
-  alignas(1024) unsigned char a[NS][kAStage];
+  alignas(1024) unsigned char a[TA ? 1 : NS][TA ? 16 : kAStage];
   uint64_t full[NS], empty[NS];
   uint64_t full_c[2], empty_c[2];
   uint32_t tmem_base;
@@ -219,21 +239,28 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
 
-template <bool PHASE1, int BM>
-__global__ void __launch_bounds__(sg::kThreads, 1)
+template <bool PHASE1, int BM, int EXP, bool TA>
+__global__ void __launch_bounds__(sg::threads_for<EXP>(), 1)
     sg_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const SgParams p) {
   using namespace sg;
-  constexpr int kXStage = Smem<BM>::kXStage, kXAtom = Smem<BM>::kXAtom, NS = Smem<BM>::NS;
+  using S = Smem<BM, TA>;
+  static_assert(EXP == 4 || EXP == 8, "expander warps");
+  constexpr int kWpr = 16 / EXP;  // sign words per expander thread and stage
+  constexpr int kXStage = S::kXStage, kXAtom = S::kXAtom, NS = S::NS;
   constexpr uint32_t kIdesc = idesc_f16(BN, BM, 0, 0);  // fp16 x fp16 -> fp32
-  constexpr uint32_t kTmemCols = 2 * BM;                // two accumulators of BM columns
+  // TMEM: two accumulators of BM columns; with TA also NS weight stages of
+  // BKS / 2 columns (row = lane, k pairs along the columns) from column 2 BM
+  constexpr uint32_t kACol = 2 * BM;
+  constexpr uint32_t kTmemCols = TA ? 512 : 2 * BM;
+  static_assert(!TA || kACol + NS * (BKS / 2) <= kTmemCols, "TMEM columns");
   extern __shared__ unsigned char smem_raw[];
-  Smem<BM>& sm = *reinterpret_cast<Smem<BM>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  S& sm = *reinterpret_cast<S*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int i = 0; i < NS; ++i) {
-      // one barrier per stage: the expanders' 128 arrivals plus the producer's
+      // one barrier per stage: the expanders' 32 EXP arrivals plus the producer's
       // arrival with the activation tile's transaction bytes (one wait for the MMA issuer)
-      mbar_init(&sm.full[i], 129);
+      mbar_init(&sm.full[i], 32 * EXP + 1);
       mbar_init(&sm.empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -285,12 +312,17 @@ __global__ void __launch_bounds__(sg::kThreads, 1)
           if (!mbar_wait(&sm.full[s], (c / NS) & 1)) goto done_mma;
           tc_fence_after();
           const uint32_t xbase = smem_u32(sm.x[s]);
-          const uint32_t abase = smem_u32(sm.a[s]);
 #pragma unroll
           for (int kk = 0; kk < BKS / 16; ++kk) {
-            const uint32_t ao = (kk >> 2) * kAAtom + (kk & 3) * 32, xo = (kk >> 2) * kXAtom + (kk & 3) * 32;
-            tc_mma_ss(d, smem_desc_sw128(abase + ao), smem_desc_sw128(xbase + xo), kIdesc,
-                      (ks > 0 || kk > 0) ? 1u : 0u);
+            const uint32_t xo = (kk >> 2) * kXAtom + (kk & 3) * 32;
+            if constexpr (TA) {
+              tc_mma_ts(d, tmem + kACol + s * (BKS / 2) + kk * 8, smem_desc_sw128(xbase + xo), kIdesc,
+                        (ks > 0 || kk > 0) ? 1u : 0u);
+            } else {
+              const uint32_t ao = (kk >> 2) * kAAtom + (kk & 3) * 32;
+              tc_mma_ss(d, smem_desc_sw128(smem_u32(sm.a[s]) + ao), smem_desc_sw128(xbase + xo), kIdesc,
+                        (ks > 0 || kk > 0) ? 1u : 0u);
+            }
           }
           tc_commit(&sm.empty[s]);
         }
@@ -298,17 +330,20 @@ __global__ void __launch_bounds__(sg::kThreads, 1)
       }
     done_mma:;
     }
-  } else if (warp < 6) {
-    // expanders: thread = weight row.  Per stage: 4 sign words (one scale
-    // group, 128 k) + the group scale -> 64 fp16 pairs +-s (s = the group
-    // scale, or 0x3C00 = 1.0; the sign bit comes straight from the word),
-    // stored as 16-byte chunks of the row in the two 128B-swizzled K-major
-    // atoms.  Words and scales stream through a kPf-deep register ring over
-    // this CTA's (tile, stage) sequence so L2 latency hides behind kPf stages
-    // (8 deep for 128-token tiles measured slower: 0.114 vs 0.075 ms for the
+  } else if (warp < 2 + EXP) {
+    // expanders: thread = weight row = TMEM lane (and, with 8 expander warps,
+    // one of the stage's two 64-wide halves).  Per stage: 4 sign words (one
+    // scale group, 128 k) + the group scale -> 64 fp16 pairs +-s (s = the
+    // group scale, or 0x3C00 = 1.0; the sign bit comes straight from the
+    // word), stored as 16-byte chunks of the row in the two 128B-swizzled
+    // K-major atoms, or (TA) as 16 TMEM columns per word in the row's lane.
+    // Words and scales stream through a kPf-deep register ring over this
+    // CTA's (tile, stage) sequence so L2 latency hides behind kPf stages (8
+    // deep for 128-token tiles measured slower: 0.114 vs 0.075 ms for the
     // 4096^3 DBF chain at 512 rows).
     constexpr int kPf = 4;
-    const int rl = (warp - 2) * 32 + lane;
+    const int rl = (warp & 3) * 32 + lane;  // a warp reaches TMEM lanes 32 (warp % 4) ..
+    const int half = EXP == 8 ? (warp - 2) >> 2 : 0;  // the atom this thread writes (8 expander warps)
     const int64_t wrow = p.K >> 5;
     int ld_tile = blockIdx.x, ld_ks = 0;
     auto fetch = [&](uint4& w, uint32_t& sc) {
@@ -317,7 +352,14 @@ __global__ void __launch_bounds__(sg::kThreads, 1)
       if (ld_tile < ntiles) {
         const int n = (ld_tile / p.MT) * BN + rl;
         if (n < p.rows) {  // a row's words are 16-byte aligned (K % 128 == 0)
-          w = __ldg(reinterpret_cast<const uint4*>(p.signs + static_cast<int64_t>(n) * wrow) + ld_ks);
+          if (EXP == 4) {
+            w = __ldg(reinterpret_cast<const uint4*>(p.signs + static_cast<int64_t>(n) * wrow) + ld_ks);
+          } else {
+            const uint2 h2 =
+                __ldg(reinterpret_cast<const uint2*>(p.signs + static_cast<int64_t>(n) * wrow) + 2 * ld_ks + half);
+            w.x = h2.x;
+            w.y = h2.y;
+          }
           if (p.gscales) sc = __ldg(p.gscales + static_cast<int64_t>(n) * p.NK + ld_ks);
         }
         if (++ld_ks == NKS) {
@@ -343,10 +385,13 @@ __global__ void __launch_bounds__(sg::kThreads, 1)
         fetch(wr[j], sr[j]);
         const int s = c % NS;
         if (!mbar_wait_warp(&sm.empty[s], ((c / NS) & 1) ^ 1)) goto done_exp;
-        const uint32_t abase = smem_u32(sm.a[s]) + row_off;
+        if constexpr (TA) tc_fence_after();  // the stage's MMAs (commit) before its TMEM is rewritten
+        const uint32_t abase = TA ? tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16) + kACol + s * (BKS / 2) +
+                                        static_cast<uint32_t>(half * (BKS / 4))
+                                  : smem_u32(sm.a[s]) + row_off + static_cast<uint32_t>(half * kAAtom);
         const uint32_t words[4] = {cur.x, cur.y, cur.z, cur.w};
 #pragma unroll
-        for (int wi = 0; wi < 4; ++wi) {
+        for (int wi = 0; wi < kWpr; ++wi) {
           const uint32_t w = words[wi];
           uint32_t rr[16];
 #pragma unroll
@@ -357,14 +402,23 @@ __global__ void __launch_bounds__(sg::kThreads, 1)
             const uint32_t tt = m * (0x40008000u >> b);
             rr[pp] = (tt & 0x80008000u) | ss;
           }
-          const uint32_t ab = abase + static_cast<uint32_t>((wi >> 1) * kAAtom);  // atom wi / 2
+          if constexpr (TA) {
+            tmem_st16(abase + wi * 16, rr);  // columns: k pairs 16 wi .. 16 wi + 15 of this part
+          } else {
+            const uint32_t ab = abase + static_cast<uint32_t>((wi >> 1) * kAAtom);  // atom wi / 2
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const uint32_t chunk = static_cast<uint32_t>((wi & 1) * 4 + q);
-            st_shared_v4(ab + ((chunk ^ sw) << 4), rr[4 * q], rr[4 * q + 1], rr[4 * q + 2], rr[4 * q + 3]);
+            for (int q = 0; q < 4; ++q) {
+              const uint32_t chunk = static_cast<uint32_t>((wi & 1) * 4 + q);
+              st_shared_v4(ab + ((chunk ^ sw) << 4), rr[4 * q], rr[4 * q + 1], rr[4 * q + 2], rr[4 * q + 3]);
+            }
           }
         }
-        fence_async_shared();
+        if constexpr (TA) {
+          tc_wait_st();
+          tc_fence_before();
+        } else {
+          fence_async_shared();
+        }
         mbar_arrive(&sm.full[s]);
         ++c;
       }
@@ -421,7 +475,7 @@ __global__ void __launch_bounds__(sg::kThreads, 1)
 
 // ------------------------------------------------------------------ host side
 
-template <bool PHASE1, int BM>
+template <bool PHASE1, int BM, int EXP, bool TA>
 static cudaError_t launch_sg_gemm_bm(SgParams p, const void* bmat, int64_t bcols, cudaStream_t stream, int num_sms) {
   using namespace sg;
   p.MT = (p.M + BM - 1) / BM;
@@ -430,13 +484,14 @@ static cudaError_t launch_sg_gemm_bm(SgParams p, const void* bmat, int64_t bcols
   CUtensorMap tm;
   // fp16 and bf16 share the 2-byte element layout the tensor map describes; box {64, BM}
   if (!make_tmap_bf16_sw128(&tm, bmat, p.M, bcols, BM)) return cudaErrorInvalidValue;
-  const size_t smem = sizeof(Smem<BM>) + 1024;
-  cudaError_t err = ensure_dyn_smem(reinterpret_cast<const void*>(sg_gemm_kernel<PHASE1, BM>), static_cast<int>(smem));
+  const size_t smem = sizeof(Smem<BM, TA>) + 1024;
+  auto kern = sg_gemm_kernel<PHASE1, BM, EXP, TA>;
+  cudaError_t err = ensure_dyn_smem(reinterpret_cast<const void*>(kern), static_cast<int>(smem));
   if (err != cudaSuccess) return err;
   const int ntiles = p.MT * p.NT;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(ntiles < num_sms ? ntiles : num_sms));
-  cfg.blockDim = dim3(kThreads);
+  cfg.blockDim = dim3(threads_for<EXP>());
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
@@ -444,18 +499,34 @@ static cudaError_t launch_sg_gemm_bm(SgParams p, const void* bmat, int64_t bcols
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, sg_gemm_kernel<PHASE1, BM>, tm, p);
+  return cudaLaunchKernelEx(&cfg, kern, tm, p);
 }
 
 // p: signs, gscales, rdiag, s1, s2, outputs, M, rows, K (tiles are derived here).
+// Token tile: 256 when that gives at least one tile per SM, else 128.
+// Expander warps: kExp256 / kExp128 by token tile (the expansion of a stage
+// costs the same whatever the tile; a 128-token tile's MMAs take half as
+// long).  Weight operand of 128-token tiles: kTmemA128 (TMEM or shared memory).
 template <bool PHASE1>
 cudaError_t launch_sg_gemm(const SgParams& p, const void* bmat, int64_t bcols, cudaStream_t stream, int num_sms) {
   const int nt = (p.rows + sg::BN - 1) / sg::BN;
   const int tiles256 = ((p.M + 255) / 256) * nt;
-  const int force = knob(kKnobSgBm);  // tuning knob: force the token tile
-  if (force == 256 || (force != 128 && tiles256 >= num_sms))
-    return launch_sg_gemm_bm<PHASE1, 256>(p, bmat, bcols, stream, num_sms);
-  return launch_sg_gemm_bm<PHASE1, 128>(p, bmat, bcols, stream, num_sms);
+  const int force = knob(kKnobSgBm);  // tuning knobs: token tile, expander warps, weight operand
+  const int fexp = knob(kKnobSgExp);
+  const int fa = knob(kKnobSgA);
+  if (force == 256 || (force != 128 && tiles256 >= num_sms)) {
+    if (fexp == 8 || (fexp != 4 && sg::kExp256 == 8))
+      return launch_sg_gemm_bm<PHASE1, 256, 8, false>(p, bmat, bcols, stream, num_sms);
+    return launch_sg_gemm_bm<PHASE1, 256, 4, false>(p, bmat, bcols, stream, num_sms);
+  }
+  const bool ta = fa == 2 || (fa != 1 && sg::kTmemA128);
+  const bool e8 = fexp == 8 || (fexp != 4 && sg::kExp128 == 8);
+  if (ta) {
+    return e8 ? launch_sg_gemm_bm<PHASE1, 128, 8, true>(p, bmat, bcols, stream, num_sms)
+              : launch_sg_gemm_bm<PHASE1, 128, 4, true>(p, bmat, bcols, stream, num_sms);
+  }
+  return e8 ? launch_sg_gemm_bm<PHASE1, 128, 8, false>(p, bmat, bcols, stream, num_sms)
+            : launch_sg_gemm_bm<PHASE1, 128, 4, false>(p, bmat, bcols, stream, num_sms);
 }
 
 cudaError_t launch_sg_prep(const uint16_t* x, const uint16_t* bdiag, const uint16_t* mid, int64_t n, int64_t r,

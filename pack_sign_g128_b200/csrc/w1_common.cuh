@@ -289,6 +289,14 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
       : "r"(taddr)
       : "memory");
 }
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+          taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
@@ -406,13 +414,15 @@ inline cudaError_t ensure_dyn_smem(const void* kernel, int bytes) {
 //   dbf_rank_split W1_DBF_RANK_SPLIT two-launch chain: CTAs per cluster that split r in U . h (0 = planner)
 //   sg_bm         W1_SG_BM          sign GEMM token tile: 0 = by tile count, else 128 or 256
 //   dbf_core      W1_DBF_CORE       two-launch chain's GEMV core: 0 = register-fed where it fits, 1 = same, 2 = direct
+//   sg_exp        W1_SG_EXP         sign GEMM expander warps: 0 = by token tile, else 4 or 8
+//   sg_a          W1_SG_A           sign GEMM weight operand of 128-token tiles: 0 = default, 1 = smem, 2 = TMEM
 //   verbose       W1_VERBOSE        nonzero: plans and choices on stderr
 #include <atomic>
 #include <cstdlib>
 #include <cstring>
 namespace w1 {
 enum KnobId { kKnobGemvPath, kKnobGemvSplit, kKnobGemvAutotune, kKnobMoePath, kKnobDbfPath, kKnobDbfWarps,
-              kKnobDbfRankSplit, kKnobSgBm, kKnobDbfCore, kKnobVerbose, kKnobCount };
+              kKnobDbfRankSplit, kKnobSgBm, kKnobDbfCore, kKnobSgExp, kKnobSgA, kKnobVerbose, kKnobCount };
 // GEMV kernels a knob can force (also the kinds of the dispatcher's choices).
 enum GemvPathKnob { kGemvAuto = 0, kGemvDirect8 = 1, kGemvDirect16 = 2, kGemvTc = 3, kGemvRing = 4, kGemvFlat = 5,
                     kGemvFlat16 = 6 };
@@ -435,6 +445,8 @@ inline const KnobSpec& knob_spec(int id) {
       {"dbf_rank_split", "W1_DBF_RANK_SPLIT", 0, {nullptr}},
       {"sg_bm", "W1_SG_BM", 0, {nullptr}},
       {"dbf_core", "W1_DBF_CORE", 0, {"flat", "direct", nullptr}},
+      {"sg_exp", "W1_SG_EXP", 0, {nullptr}},
+      {"sg_a", "W1_SG_A", 0, {"smem", "tmem", nullptr}},
       {"verbose", "W1_VERBOSE", 0, {nullptr}},
   };
   return specs[id];

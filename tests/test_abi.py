@@ -47,7 +47,8 @@ def test_knobs_accept_their_words_and_reject_the_rest(lib):
     ok = [("gemv_path", "direct"), ("gemv_path", "direct16"), ("gemv_path", "tc"), ("gemv_path", "ring"),
           ("gemv_path", "flat"), ("gemv_split", "4"), ("gemv_autotune", "0"), ("moe_path", "tiles"),
           ("moe_path", "decode"), ("moe_path", "grouped"), ("dbf_path", "fused"), ("dbf_path", "twostep"), ("dbf_warps", "16"),
-          ("dbf_rank_split", "4"), ("sg_bm", "256"), ("dbf_core", "direct"),
+          ("dbf_rank_split", "4"), ("sg_bm", "256"), ("dbf_core", "direct"), ("sg_exp", "8"), ("sg_a", "tmem"),
+          ("sg_a", "smem"),
           ("verbose", "1")]
     try:
         for name, value in ok:

@@ -63,3 +63,24 @@ def test_gemm_integer_inputs_bit_exact():
     y = run_gemm(s, sc, synth.f32_to_bf16_bits(xi))
     y_ref, _ = O.matmul_ref(xi.astype(np.float64), s, sc, K)
     assert np.array_equal(y, y_ref)
+
+
+@pytest.mark.parametrize("bm,exp,a", [(128, 4, "smem"), (128, 8, "smem"), (128, 4, "tmem"), (128, 8, "tmem"),
+                                      (256, 4, "smem"), (256, 8, "smem")])
+def test_gemm_every_kernel_form(knob, bm, exp, a):
+    """Each token tile x expander count x weight-operand place on a ragged case
+    with several tiles per CTA (persistent loop, both accumulators, stage ring
+    wrapping across tiles): within the bound, and bit for bit equal to the
+    shared-memory, 4-expander form of the same tile (same MMAs, same order)."""
+    M, N, K = 1100, 2200, 1152
+    s, c = packed(N, K, 91)
+    x = synth.activations_bf16(synth.rng(92), M, K)
+    knob("sg_bm", bm)
+    knob("sg_exp", exp)
+    knob("sg_a", a)
+    y = run_gemm(s, c, x)
+    y_ref, bound = O.matmul_ref(O.bf16_bits_to_f64(x), s, c, K)
+    assert_within(y, y_ref, bound, what=f"bm={bm} exp={exp} a={a}")
+    knob("sg_exp", 4)
+    knob("sg_a", "smem")
+    assert np.array_equal(y, run_gemm(s, c, x))
