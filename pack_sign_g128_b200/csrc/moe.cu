@@ -438,36 +438,26 @@ struct MoeGemmParams {
   int out_ld;                // leading dimension of the output
 };
 
-// TA: the weight operand (+-s fp16) in TMEM (row = lane, k pairs along the
-// columns) instead of shared memory.  TMEM then holds NACC accumulator sets
-// of NMAT x TN columns from column 0 and NS weight stages of NMAT x 64
-// columns after them: down keeps two accumulator sets (256 + 4 x 64 columns),
-// gate/up one (256 + 2 x 128), so its epilogue no longer overlaps the next
-// tile's MMAs.
-template <bool GATEUP, bool TA>
+template <bool GATEUP>
 struct MoeCfg {
   static constexpr int TN = GATEUP ? moe::TN_GU : moe::TN_D;  // routes per tile (max MMA N)
   static constexpr int NMAT = GATEUP ? 2 : 1;                 // weight matrices per tile
   // K per pipeline stage: one scale group, two 64-wide (128-byte) swizzle
   // atoms; long stages amortise the MMA issuer's barrier wait over 8 x NMAT MMAs
   static constexpr int BKS = 128;
-  static constexpr int NS = TA ? (GATEUP ? 2 : 4) : (GATEUP ? 2 : 3);  // stages
+  static constexpr int NS = GATEUP ? 2 : 3;                   // stages (192 KB either way)
   static constexpr int XATOM = TN * 128;                      // bytes of one 64-wide atom of B
   static constexpr int XSTAGE = 2 * XATOM;                    // bytes of one B stage (fp16)
   static constexpr int AATOM = 128 * 128;                     // bytes of one 64-wide atom of A
   static constexpr int ASTAGE = 2 * AATOM;                    // bytes of one weight matrix stage
-  static constexpr int NACC = TA && GATEUP ? 1 : 2;           // accumulator sets
-  static constexpr uint32_t ACOL = NACC * NMAT * TN;          // TA: first weight-stage column
-  static constexpr uint32_t kTmemCols = TA ? 512 : GATEUP ? 512 : 256;
-  static_assert(!TA || ACOL + NS * NMAT * (BKS / 2) <= kTmemCols, "TMEM columns");
+  static constexpr uint32_t kTmemCols = GATEUP ? 512 : 256;   // two accumulator sets
 };
 
-template <bool GATEUP, bool TA>
+template <bool GATEUP>
 struct MoeSmem {
-  using C = MoeCfg<GATEUP, TA>;
-  alignas(1024) unsigned char x[C::NS][C::XSTAGE];
-  alignas(1024) unsigned char a[TA ? 1 : C::NS][C::NMAT][TA ? 16 : C::ASTAGE];
-  uint64_t full[C::NS], empty[C::NS];
+  alignas(1024) unsigned char x[MoeCfg<GATEUP>::NS][MoeCfg<GATEUP>::XSTAGE];
+  alignas(1024) unsigned char a[MoeCfg<GATEUP>::NS][MoeCfg<GATEUP>::NMAT][MoeCfg<GATEUP>::ASTAGE];
+  uint64_t full[MoeCfg<GATEUP>::NS], empty[MoeCfg<GATEUP>::NS];
   uint64_t full_c[2], empty_c[2];
   uint32_t tmem_base;
 };
@@ -477,20 +467,19 @@ __device__ __forceinline__ void moe_st_shared_v4(uint32_t addr, uint32_t a, uint
 }
 
 // Warp roles: 0 TMA producer (route rows of B), 1 MMA issuer, 2-9 expanders
-// (two threads per weight row = TMEM lane: sign words + the group scale ->
-// fp16 pairs +-s in the 128B-swizzled K-major layout, or TMEM columns;
-// gate/up: one matrix each, down: one word pair of the stage each), 10-13
-// epilogue (thread = TMEM lane).  One 128-wide K stage: NMAT x 8 MMAs (M =
-// 128, N = the tile's route count rounded up to 16, K = 16), all of K into
-// one accumulator per matrix per tile; NACC accumulator sets alternate
-// between tiles.
-template <bool GATEUP, bool TA>
+// (two threads per weight row: sign words + the group scale -> fp16 pairs +-s
+// in the 128B-swizzled K-major layout; gate/up: one matrix each, down: one
+// word pair of the stage each), 10-13 epilogue (thread = TMEM lane).  One
+// 128-wide K stage: NMAT x 8 MMAs (M = 128, N = the tile's route count rounded
+// up to 16, K = 16), all of K into one accumulator per matrix per tile; two
+// accumulator sets alternate between tiles.
+template <bool GATEUP>
 __global__ void __launch_bounds__(moe::kThreads, 1)
     moe_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const MoeGemmParams p) {
-  using C = MoeCfg<GATEUP, TA>;
+  using C = MoeCfg<GATEUP>;
   extern __shared__ unsigned char smem_raw[];
-  MoeSmem<GATEUP, TA>& sm =
-      *reinterpret_cast<MoeSmem<GATEUP, TA>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  MoeSmem<GATEUP>& sm =
+      *reinterpret_cast<MoeSmem<GATEUP>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::NS; ++i) {
@@ -541,8 +530,8 @@ __global__ void __launch_bounds__(moe::kThreads, 1)
         const moe::Tile tl = p.tiles[ti];
         const int n_mma = ((tl.count + 15) >> 4) << 4;
         const uint32_t idesc = idesc_f16(128, n_mma, 0, 0);  // fp16 x fp16 -> fp32
-        const int cb = tli % C::NACC;
-        if (!mbar_wait(&sm.empty_c[cb], ((tli / C::NACC) & 1) ^ 1)) goto done_mma;
+        const int cb = tli & 1;
+        if (!mbar_wait(&sm.empty_c[cb], ((tli >> 1) & 1) ^ 1)) goto done_mma;
         tc_fence_after();
         for (int ks = 0; ks < NKS; ++ks, ++c) {
           const int s = c % C::NS;
@@ -552,17 +541,12 @@ __global__ void __launch_bounds__(moe::kThreads, 1)
 #pragma unroll
           for (int mat = 0; mat < C::NMAT; ++mat) {
             const uint32_t d = tmem + (cb * C::NMAT + mat) * C::TN;
+            const uint32_t abase = smem_u32(sm.a[s][mat]);
 #pragma unroll
             for (int kk = 0; kk < C::BKS / 16; ++kk) {
-              const uint32_t xo = (kk >> 2) * C::XATOM + (kk & 3) * 32;
-              if constexpr (TA) {
-                tc_mma_ts(d, tmem + C::ACOL + (s * C::NMAT + mat) * (C::BKS / 2) + kk * 8,
-                          smem_desc_sw128(xbase + xo), idesc, (ks > 0 || kk > 0) ? 1u : 0u);
-              } else {
-                const uint32_t ao = (kk >> 2) * C::AATOM + (kk & 3) * 32;
-                tc_mma_ss(d, smem_desc_sw128(smem_u32(sm.a[s][mat]) + ao), smem_desc_sw128(xbase + xo), idesc,
-                          (ks > 0 || kk > 0) ? 1u : 0u);
-              }
+              const uint32_t ao = (kk >> 2) * C::AATOM + (kk & 3) * 32, xo = (kk >> 2) * C::XATOM + (kk & 3) * 32;
+              tc_mma_ss(d, smem_desc_sw128(abase + ao), smem_desc_sw128(xbase + xo), idesc,
+                        (ks > 0 || kk > 0) ? 1u : 0u);
             }
           }
           tc_commit(&sm.empty[s]);
@@ -577,8 +561,8 @@ __global__ void __launch_bounds__(moe::kThreads, 1)
     // 128-wide stage; down: half h expands words 2h, 2h+1 (swizzle atom h).
     constexpr int kPf = 4;
     constexpr int NW = GATEUP ? 4 : 2;  // sign words per thread per stage
-    const int rl = (warp & 3) * 32 + lane;  // a warp reaches TMEM lanes 32 (warp % 4) ..
-    const int half = (warp - 2) >> 2;
+    const int et = (warp - 2) * 32 + lane;
+    const int rl = et & 127, half = et >> 7;
     const int mat = GATEUP ? half : 0;
     const int w0 = GATEUP ? 0 : 2 * half;  // first word of the stage this thread expands
     const int64_t wrow = p.K >> 5;
@@ -647,10 +631,7 @@ __global__ void __launch_bounds__(moe::kThreads, 1)
         fetch(wr[j], sr[j]);
         const int s = c % C::NS;
         if (!mbar_wait_warp(&sm.empty[s], ((c / C::NS) & 1) ^ 1)) goto done_exp;
-        if constexpr (TA) tc_fence_after();  // the stage's MMAs (commit) before its TMEM is rewritten
-        const uint32_t abase = TA ? tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16) + C::ACOL +
-                                        (s * C::NMAT + mat) * (C::BKS / 2)
-                                  : smem_u32(sm.a[s][mat]) + row_off;  // + atom offset per word pair
+        const uint32_t abase = smem_u32(sm.a[s][mat]) + row_off;  // + atom offset per word pair
 #pragma unroll
         for (int wi = 0; wi < NW; ++wi) {
           const uint32_t w = cur[wi];
@@ -664,23 +645,14 @@ __global__ void __launch_bounds__(moe::kThreads, 1)
             rr[pp] = (tt & 0x80008000u) | ss;
           }
           const int gw = w0 + wi;  // word of the stage: atom gw / 2, chunks 4 (gw % 2) + q
-          if constexpr (TA) {
-            tmem_st16(abase + gw * 16, rr);  // columns: k pairs 16 gw .. 16 gw + 15
-          } else {
-            const uint32_t ab = abase + static_cast<uint32_t>((gw >> 1) * C::AATOM);
+          const uint32_t ab = abase + static_cast<uint32_t>((gw >> 1) * C::AATOM);
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const uint32_t chunk = static_cast<uint32_t>((gw & 1) * 4 + q);
-              moe_st_shared_v4(ab + ((chunk ^ swz) << 4), rr[4 * q], rr[4 * q + 1], rr[4 * q + 2], rr[4 * q + 3]);
-            }
+          for (int q = 0; q < 4; ++q) {
+            const uint32_t chunk = static_cast<uint32_t>((gw & 1) * 4 + q);
+            moe_st_shared_v4(ab + ((chunk ^ swz) << 4), rr[4 * q], rr[4 * q + 1], rr[4 * q + 2], rr[4 * q + 3]);
           }
         }
-        if constexpr (TA) {
-          tc_wait_st();
-          tc_fence_before();
-        } else {
-          fence_async_shared();
-        }
+        fence_async_shared();
         mbar_arrive(&sm.full[s]);
         ++c;
       }
@@ -696,8 +668,8 @@ __global__ void __launch_bounds__(moe::kThreads, 1)
       const moe::Tile tl = p.tiles[ti];
       const int row = tl.rt * 128 + rl;
       const bool valid = row < p.rows;
-      const int cb = tli % C::NACC;
-      if (!mbar_wait_warp(&sm.full_c[cb], (tli / C::NACC) & 1)) goto done_epi;
+      const int cb = tli & 1;
+      if (!mbar_wait_warp(&sm.full_c[cb], (tli >> 1) & 1)) goto done_epi;
       tc_fence_after();
 #pragma unroll 1
       for (int q4 = 0; q4 < C::TN / 32; ++q4) {
@@ -982,29 +954,6 @@ static cudaError_t launch_pdl(Kern kernel, dim3 grid, dim3 block, size_t smem, c
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
-
-// Where each grouped GEMM keeps its weight operand (moe_a knob: 0 = the
-// defaults below, 1 = shared memory, 2 = TMEM for both, 3 = TMEM for down only).
-constexpr bool kMoeGateupTmemA = false;
-constexpr bool kMoeDownTmemA = false;
-static bool moe_a_gateup_tmem() {
-  const int k = knob(kKnobMoeA);
-  return k == 2 || (k == 0 && kMoeGateupTmemA);
-}
-static bool moe_a_down_tmem() {
-  const int k = knob(kKnobMoeA);
-  return k == 2 || k == 3 || (k == 0 && kMoeDownTmemA);
-}
-
-template <bool GATEUP, bool TA>
-static cudaError_t launch_moe_gemm(const CUtensorMap& tm, const MoeGemmParams& p, int grid, cudaStream_t stream) {
-  const size_t smem = sizeof(MoeSmem<GATEUP, TA>) + 1024;
-  cudaError_t err =
-      ensure_dyn_smem(reinterpret_cast<const void*>(moe_gemm_kernel<GATEUP, TA>), static_cast<int>(smem));
-  if (err != cudaSuccess) return err;
-  return launch_pdl(moe_gemm_kernel<GATEUP, TA>, dim3(grid), dim3(moe::kThreads), smem, stream, tm, p);
-}
-
 
 // Down products and the slot-ordered combine of the decode regime, fused:
 // one CTA per (token, RB output rows), RB = 16 x tokens (at most 128), so a
@@ -1578,9 +1527,11 @@ cudaError_t launch_moe(const uint16_t* x, const float* logits, int64_t T, int64_
     p.rows = static_cast<int>(I);
     p.K = static_cast<int>(H);
     p.out_ld = static_cast<int>(I);
+    const size_t smem = sizeof(MoeSmem<true>) + 1024;
+    err = ensure_dyn_smem(reinterpret_cast<const void*>(moe_gemm_kernel<true>), static_cast<int>(smem));
+    if (err != cudaSuccess) return err;
     const int grid = L.max_tiles_gu < num_sms ? L.max_tiles_gu : num_sms;
-    err = moe_a_gateup_tmem() ? launch_moe_gemm<true, true>(tm, p, grid, stream)
-                              : launch_moe_gemm<true, false>(tm, p, grid, stream);
+    err = launch_pdl(moe_gemm_kernel<true>, dim3(grid), dim3(moe::kThreads), smem, stream, tm, p);
     if (err != cudaSuccess) return err;
   }
   // 5. h -> fp16 with a power of two per route
@@ -1604,9 +1555,11 @@ cudaError_t launch_moe(const uint16_t* x, const float* logits, int64_t T, int64_
     p.rows = static_cast<int>(H);
     p.K = static_cast<int>(I);
     p.out_ld = static_cast<int>(H);
+    const size_t smem = sizeof(MoeSmem<false>) + 1024;
+    err = ensure_dyn_smem(reinterpret_cast<const void*>(moe_gemm_kernel<false>), static_cast<int>(smem));
+    if (err != cudaSuccess) return err;
     const int grid = L.max_tiles_d < num_sms ? L.max_tiles_d : num_sms;
-    err = moe_a_down_tmem() ? launch_moe_gemm<false, true>(tm, p, grid, stream)
-                            : launch_moe_gemm<false, false>(tm, p, grid, stream);
+    err = launch_pdl(moe_gemm_kernel<false>, dim3(grid), dim3(moe::kThreads), smem, stream, tm, p);
     if (err != cudaSuccess) return err;
   }
   // 5. combine

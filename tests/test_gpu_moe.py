@@ -143,15 +143,6 @@ def test_moe_forced_path(path, T, knob):
     run_and_check(T, 512, 256, 16, 4, 7)
 
 
-@pytest.mark.parametrize("where", ["smem", "tmem", "tmemdown"])
-def test_moe_tiles_every_weight_operand_place(where, knob):
-    """The tile pipeline's grouped GEMMs with the weight operand in shared
-    memory or TMEM (gate/up with one accumulator set, down with two), on
-    skewed routing (empty experts, multi-tile experts, several tiles per CTA)."""
-    knob("moe_a", where)
-    run_and_check(300, 384, 256, 16, 4, 3, 6.0)
-
-
 @pytest.mark.parametrize("T", [64, 4])
 def test_moe_is_deterministic(T):
     H, I, E, K = 512, 256, 16, 4
