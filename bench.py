@@ -565,15 +565,22 @@ def dbf_rows(torch, ops, synth, peaks, l2_bytes: int, iters: int = 5, only_b: in
                    "frac_hbm": round(gbs / peaks["hbm_gbs"], 4), "calls": R}
             # the small-batch chain forms side by side (fused kernel vs two launches)
             forms = {}
-            for form, core in (("fused", None), ("twostep", None), ("twostep", "direct")):
+            for form, core, warps in (("fused", None, None), ("twostep", None, None), ("twostep", "direct", None),
+                                      ("twostep", None, 8)):
+                if warps and B <= 2:
+                    continue  # 8 warps is already the default there
                 ops.set_knob("dbf_path", form)
                 if core:
                     ops.set_knob("dbf_core", core)
+                if warps:
+                    ops.set_knob("dbf_warps", warps)
                 try:
-                    forms[form + ("_" + core if core else "")] = round(graph_us(), 3)
+                    key = form + ("_" + core if core else "") + (f"_w{warps}" if warps else "")
+                    forms[key] = round(graph_us(), 3)
                 finally:
                     ops.set_knob("dbf_path", None)
                     ops.set_knob("dbf_core", None)
+                    ops.set_knob("dbf_warps", None)
             row["us_by_form"] = forms
             # split rank: r partitioned over the CTAs of a cluster in U . h (two-launch form)
             splits = {}

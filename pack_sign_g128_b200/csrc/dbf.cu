@@ -343,15 +343,16 @@ cudaError_t launch_dbf(const uint16_t* a, const uint32_t* B1, const uint16_t* mi
       const int warps = wknob ? wknob : (nb >= 4 ? 16 : 8);
       const int rsplit = knob(kKnobDbfRankSplit);
       const int cknob = knob(kKnobDbfCore);  // 0: flat where it fits, 1: flat, 2: direct
-      const bool try_flat = cknob != 2 && nb <= 2;
+      const bool try_flat = cknob != 2 && nb <= 4;
+      const int fw = wknob ? wknob : (nb <= 2 ? 8 : 16);  // the register-fed core's warps
       err = cudaErrorNotSupported;
-      if (try_flat) err = launch_gemv_flat_diag(B2, r, n, xg, false, b, mid, nb, h, false, stream, num_sms, smem_cap, 0, 8);
+      if (try_flat) err = launch_gemv_flat_diag(B2, r, n, xg, false, b, mid, nb, h, false, stream, num_sms, smem_cap, 0, fw);
       if (err == cudaErrorNotSupported)
         err = launch_gemv_direct_diag(B2, r, n, xg, false, b, mid, nb, h, false, stream, num_sms, smem_cap, warps, 0);
       if (err == cudaSuccess) {
         err = cudaErrorNotSupported;
         if (try_flat && rsplit == 0)
-          err = launch_gemv_flat_diag(B1, m, r, h, true, nullptr, a, nb, yg, true, stream, num_sms, smem_cap, 0, 8);
+          err = launch_gemv_flat_diag(B1, m, r, h, true, nullptr, a, nb, yg, true, stream, num_sms, smem_cap, 0, fw);
         if (err == cudaErrorNotSupported)
           err = launch_gemv_direct_diag(B1, m, r, h, true, nullptr, a, nb, yg, true, stream, num_sms, smem_cap, warps,
                                         rsplit);

@@ -39,6 +39,10 @@
 //    the activations enter unchanged, the weights become bf16 +-1 pairs
 //    (one shift and one LOP3 per two weights); mma.sync m16n8k16 bf16 -> f32;
 //    the group scale multiplies each group's f32 partial sums.
+// The diagonal form (a step of the DBF chain: fp32 or diagonal-scaled input,
+// no group scales, a row diagonal on the outputs) feeds the int8 digits from
+// the fp32 values for B <= 2, and for B = 3, 4 splits each fp32 value into
+// bf16 high and low parts, two MMA columns per batch row (error 2^-17 |v|).
 // K order inside one MMA is free as long as A and B agree; the activation
 // values are placed in the order the sign-bit extraction produces, and the
 // canonical weight bytes are read unchanged.
@@ -46,6 +50,7 @@
 #include <cstdint>
 #include <cstdio>
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <mutex>
 #include <type_traits>
@@ -57,10 +62,13 @@ namespace w1 {
 namespace fl {
 constexpr int kMaxBox = 48;  // TMA boxes (8 groups each) per CTA
 constexpr int kBoxG = 8;     // groups per box (128 bytes of sign words per row)
-template <int NB>
+template <int NB, bool DIAG = false>
 struct Cfg {
-  static constexpr bool BF = NB >= 3;            // bf16 products, batch rows as the MMA columns
-  static constexpr int NCOL = BF ? NB : 3 * NB;  // result columns per row
+  static constexpr bool BF = NB >= 3;  // bf16 products, batch rows as the MMA columns
+  // result columns per row: int8 digits 3 per batch row; bf16 one per batch
+  // row, or two (the bf16 high and low parts of an fp32 input) in the diagonal form
+  static constexpr int NCOL = BF ? (DIAG ? 2 * NB : NB) : 3 * NB;
+  static_assert(NCOL <= 8, "one 8-column n-tile");
   static constexpr int MAXT = 8;                 // 16-row tiles per CTA (R <= 128)
   static constexpr int UPL = 2;                  // int8 form: activation units per lane and pass
   static constexpr int GW = BF ? 0 : 4 * 64;     // int8 form: digit words per group (4 MMAs x 32 lanes x 2)
@@ -93,9 +101,9 @@ struct FlSmem {
 // Shared memory from a 1024-byte aligned base: the swizzled sign boxes, the
 // digit buffers (int8 form; the reduction buffer overlays them), the scales,
 // the fold factors, the cluster inbox.
-template <int NB, int NW>
+template <int NB, int NW, bool DIAG>
 __host__ __device__ inline FlSmem fl_layout(int R, int G, int gw, int NG, int S, int chunk) {
-  using C = fl::Cfg<NB>;
+  using C = fl::Cfg<NB, DIAG>;
   FlSmem L;
   const int nbox = (G + fl::kBoxG - 1) / fl::kBoxG;
   const int dig_bytes = NW * gw * C::GW * 4;
@@ -236,7 +244,7 @@ __device__ __forceinline__ void fl_products(const FlParams& p, int row0, int g0,
                                             const unsigned char* wts, uint64_t* bars, int nbox, uint32_t* dig,
                                             float* fold, const uint16_t* scl, uint64_t* sbar, int lane, float* red,
                                             Prologue&& prologue) {
-  using C = fl::Cfg<NB>;
+  using C = fl::Cfg<NB, DIAG>;
   constexpr int STEPS = C::BF ? 8 : 4;            // MMAs per group and tile
   // groups per block: GI T <= 8 accumulator chains; the bf16 form also holds
   // two blocks' activations in registers (16 words per group), so it takes at
@@ -250,10 +258,9 @@ __device__ __forceinline__ void fl_products(const FlParams& p, int row0, int g0,
   const int r1 = lane >> 2, cq = lane & 3;
   prologue();
   // ---- 1. int8 form: activations -> digit fragments in shared memory
-  if constexpr (DIAG) {
+  if constexpr (DIAG && !C::BF) {
     // fp32 x (read through L2: the preceding launch wrote it), or bf16 x
     // times the column diagonal (exact in fp32)
-    static_assert(!C::BF, "the diagonal form has the int8 products only");
     const int U = nwg * NB * 8;
     for (int u = lane; u - lane < U; u += 32) {  // trip count uniform over the warp
       const int gl = u / (8 * NB), b = (u >> 3) % NB, ucq = (u >> 1) & 3, h = u & 1;
@@ -338,13 +345,78 @@ __device__ __forceinline__ void fl_products(const FlParams& p, int row0, int g0,
   }
   // ---- 2. products, GI groups at a time
   // bf16 form: lane (r1, cq) holds batch row r1's 32 elements of word cq of
-  // each group of a block (16 bf16x2 words), the next block's loads in flight
+  // each group of a block (16 bf16x2 words), the next block's loads in flight.
+  // Diagonal form: column r1 = 2 b + part holds the high (part 0) or low
+  // (part 1) bf16 part of batch row b's fp32 input v = fp32 x or bf16 x times
+  // the column diagonal: hi = bf16(v), lo = bf16(v - hi) (v - hi exact), so
+  // hi + lo = v to 2^-17 |v|.
   auto load_x = [&](int gb, uint4 (&xv)[GI][4]) {
 #pragma unroll
     for (int g = 0; g < GI; ++g) {
 #pragma unroll
       for (int i = 0; i < 4; ++i) xv[g][i] = make_uint4(0, 0, 0, 0);
-      if (C::BF && r1 < NB && gb + g < nwg) {
+      if constexpr (C::BF && DIAG) {
+        const int b = r1 >> 1;
+        if (b < NB && gb + g < nwg) {
+          const int64_t k0 = static_cast<int64_t>(g0 + wg0 + gb + g) * 128 + 32 * cq;
+          float v[32];
+          if (p.x_f32) {
+            const float4* src = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(p.x) +
+                                                                static_cast<int64_t>(b) * p.K + k0);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const float4 f = __ldcg(src + i);
+              v[4 * i] = f.x;
+              v[4 * i + 1] = f.y;
+              v[4 * i + 2] = f.z;
+              v[4 * i + 3] = f.w;
+            }
+          } else {
+            const uint4* src = reinterpret_cast<const uint4*>(p.x + static_cast<int64_t>(b) * p.K + k0);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const uint4 u = __ldg(src + i);
+              const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                v[8 * i + 2 * j] = __uint_as_float(w[j] << 16);
+                v[8 * i + 2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+              }
+            }
+            if (p.cdiag) {
+              const uint4* dg = reinterpret_cast<const uint4*>(p.cdiag + k0);
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const uint4 u = __ldg(dg + i);
+                const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                  const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[j]));
+                  v[8 * i + 2 * j] *= f.x;  // bf16 x fp16: exact in fp32
+                  v[8 * i + 2 * j + 1] *= f.y;
+                }
+              }
+            }
+          }
+          const bool low = r1 & 1;
+          uint32_t o[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            float e[2];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const float hi = __bfloat162float(__float2bfloat16_rn(v[2 * j + h]));
+              e[h] = low ? v[2 * j + h] - hi : hi;
+            }
+            const __nv_bfloat162 pr = __floats2bfloat162_rn(e[0], e[1]);
+            o[j] = *reinterpret_cast<const uint32_t*>(&pr);
+          }
+          xv[g][0] = make_uint4(o[0], o[1], o[2], o[3]);
+          xv[g][1] = make_uint4(o[4], o[5], o[6], o[7]);
+          xv[g][2] = make_uint4(o[8], o[9], o[10], o[11]);
+          xv[g][3] = make_uint4(o[12], o[13], o[14], o[15]);
+        }
+      } else if (C::BF && r1 < NB && gb + g < nwg) {
         const uint4* src = reinterpret_cast<const uint4*>(
             p.x + static_cast<int64_t>(r1) * p.K + static_cast<int64_t>(g0 + wg0 + gb + g) * 128 + 32 * cq);
 #pragma unroll
@@ -433,8 +505,8 @@ __device__ __forceinline__ void fl_products(const FlParams& p, int row0, int g0,
         // acc += s * C
 #pragma unroll
         for (int t = 0; t < T; ++t) {
-          const float s0 = __half2float(__ushort_as_half(sg[16 * t * p.NG]));
-          const float s1 = __half2float(__ushort_as_half(sg[(16 * t + 8) * p.NG]));
+          const float s0 = DIAG ? 1.f : __half2float(__ushort_as_half(sg[16 * t * p.NG]));
+          const float s1 = DIAG ? 1.f : __half2float(__ushort_as_half(sg[(16 * t + 8) * p.NG]));
           acc[t][0][0] = fmaf(s0, cc[g][t][0], acc[t][0][0]);
           acc[t][0][1] = fmaf(s0, cc[g][t][1], acc[t][0][1]);
           acc[t][1][0] = fmaf(s1, cc[g][t][2], acc[t][1][0]);
@@ -488,7 +560,7 @@ __device__ __forceinline__ void fl_products(const FlParams& p, int row0, int g0,
 template <int NB, int NW, bool DIAG = false>
 __global__ void __launch_bounds__(NW * 32, 1) gemv_flat_kernel(const __grid_constant__ CUtensorMap tmap,
                                                                const FlParams p) {
-  using C = fl::Cfg<NB>;
+  using C = fl::Cfg<NB, DIAG>;
   constexpr int NCOL = C::NCOL;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem =
@@ -504,7 +576,7 @@ __global__ void __launch_bounds__(NW * 32, 1) gemv_flat_kernel(const __grid_cons
   const int G = max(0, min(p.NG, g0 + p.G) - g0);  // this CTA's groups
   const int rows = max(0, min(p.R, p.N - row0));   // this CTA's rows inside N
   const int nbox = (G + fl::kBoxG - 1) / fl::kBoxG;
-  const FlSmem L = fl_layout<NB, NW>(p.R, p.G, p.gw, p.NG, p.S, p.chunk);
+  const FlSmem L = fl_layout<NB, NW, DIAG>(p.R, p.G, p.gw, p.NG, p.S, p.chunk);
   const unsigned char* wts = smem + L.wts;
   uint16_t* scl = reinterpret_cast<uint16_t*>(smem + L.scl);
   if (p.S > 1) cluster_arrive_relaxed();  // matched by the wait before the first remote store
@@ -585,7 +657,13 @@ __global__ void __launch_bounds__(NW * 32, 1) gemv_flat_kernel(const __grid_cons
   for (int o = threadIdx.x; o < O; o += NW * 32) {
     const int r = o / NB, b = o - r * NB;
     float sum = 0.f;
-    if constexpr (C::BF) {
+    if constexpr (C::BF && DIAG) {
+#pragma unroll 4
+      for (int w = 0; w < NW; ++w) {
+        const float* rp = red + (w * p.R + r) * NCOL + 2 * b;
+        sum += rp[0] + rp[1];
+      }
+    } else if constexpr (C::BF) {
 #pragma unroll 4
       for (int w = 0; w < NW; ++w) sum += red[(w * p.R + r) * NCOL + b];
     } else {
@@ -595,8 +673,9 @@ __global__ void __launch_bounds__(NW * 32, 1) gemv_flat_kernel(const __grid_cons
         sum += (rp[0] + rp[1]) + rp[2];
       }
     }
-    if (DIAG && p.rdiag && row0 + r < p.N) sum *= __half2float(__ushort_as_half(p.rdiag[row0 + r]));
     if (p.S == 1) {
+      // (with a K split the owner applies the row diagonal to the cluster's sum)
+      if (DIAG && p.rdiag && row0 + r < p.N) sum *= __half2float(__ushort_as_half(p.rdiag[row0 + r]));
       if (row0 + r < p.N) p.y[static_cast<int64_t>(b) * p.N + row0 + r] = sum;
     } else {
       const int owner = r / p.chunk;
@@ -630,9 +709,9 @@ struct FlPlan {
 
 // Rows per CTA: the fewest 16-row tiles that cover N with at most one
 // cluster of S CTAs per S SMs; groups per CTA: ceil(NG / S).
-template <int NB, int NW>
+template <int NB, int NW, bool DIAG>
 static bool fl_plan_for(int N, int NG, int S, int num_sms, int smem_cap, FlPlan* out) {
-  using C = fl::Cfg<NB>;
+  using C = fl::Cfg<NB, DIAG>;
   if (S < 1 || S > 8 || S > NG) return false;
   const int tiles = (N + 15) / 16;
   const int qmax = num_sms / S;
@@ -645,7 +724,7 @@ static bool fl_plan_for(int N, int NG, int S, int num_sms, int smem_cap, FlPlan*
   if ((G + fl::kBoxG - 1) / fl::kBoxG > fl::kMaxBox) return false;
   const int gw = (G + NW - 1) / NW;
   const int chunk = (R + S - 1) / S;
-  const FlSmem L = fl_layout<NB, NW>(R, G, gw, NG, S, chunk);
+  const FlSmem L = fl_layout<NB, NW, DIAG>(R, G, gw, NG, S, chunk);
   const int smem = L.total + 1024;  // alignment slack for the swizzled boxes
   if (smem > smem_cap) return false;
   *out = FlPlan{S, Q, R, T, G, gw, chunk, smem};
@@ -655,7 +734,7 @@ static bool fl_plan_for(int N, int NG, int S, int num_sms, int smem_cap, FlPlan*
 template <int NB, int NW, bool DIAG = false>
 static cudaError_t launch_gemv_flat_nb(const FlParams& base, cudaStream_t stream, int num_sms, int smem_cap, int S) {
   FlPlan plan;
-  if (!fl_plan_for<NB, NW>(base.N, base.NG, S, num_sms, smem_cap, &plan)) return cudaErrorNotSupported;
+  if (!fl_plan_for<NB, NW, DIAG>(base.N, base.NG, S, num_sms, smem_cap, &plan)) return cudaErrorNotSupported;
   if (knob(kKnobVerbose))
     fprintf(stderr, "w1_gemv(flat) plan: N=%d NG=%d B=%d warps=%d -> clusters=%d split=%d rows/CTA=%d smem=%d\n",
             base.N, base.NG, NB, NW, plan.Q, plan.S, plan.R, plan.smem);
@@ -734,8 +813,9 @@ cudaError_t launch_gemv_flat(const uint32_t* signs, const uint16_t* scales, int6
   return cudaErrorNotSupported;
 }
 
-// The diagonal form (a step of the DBF chain, no group scales), 1 or 2 batch
-// rows: y[b][n] = rdiag[n] * sum_k s(n, k) * (cdiag[k] *) x[b][k], x bf16
+// The diagonal form (a step of the DBF chain, no group scales), 1 to 4 batch
+// rows (1-2: int8 digits; 3-4: bf16 high and low parts of the fp32 input as
+// two MMA columns per row): y[b][n] = rdiag[n] * sum_k s(n, k) * (cdiag[k] *) x[b][k], x bf16
 // [B][K] (with the fp16 column diagonal cdiag, or nullptr) or fp32 [B][K]
 // (x_f32; no cdiag); rdiag fp16 [N] or nullptr.  early: the sign words were
 // not written by the kernel this launch follows.  split as for
@@ -743,7 +823,7 @@ cudaError_t launch_gemv_flat(const uint32_t* signs, const uint16_t* scales, int6
 cudaError_t launch_gemv_flat_diag(const uint32_t* signs, int64_t N, int64_t K, const void* x, bool x_f32,
                                   const uint16_t* cdiag, const uint16_t* rdiag, int B, float* y, bool early,
                                   cudaStream_t stream, int num_sms, int smem_cap, int split, int warps) {
-  if (N > (int64_t)1 << 30 || K > (int64_t)1 << 30 || B < 1 || B > 2 || (x_f32 && cdiag))
+  if (N > (int64_t)1 << 30 || K > (int64_t)1 << 30 || B < 1 || B > 4 || (x_f32 && cdiag))
     return cudaErrorNotSupported;
   FlParams p = {};
   p.signs = signs;
@@ -760,12 +840,21 @@ cudaError_t launch_gemv_flat_diag(const uint32_t* signs, int64_t N, int64_t K, c
   smem_cap = std::min(2 * smem_cap, 227 * 1024);
   for (int S = split > 0 ? split : 1; S <= 8; S *= 2) {
     cudaError_t e;
-    if (warps == 16)
-      e = B == 1 ? launch_gemv_flat_nb<1, 16, true>(p, stream, num_sms, smem_cap, S)
-                 : launch_gemv_flat_nb<2, 16, true>(p, stream, num_sms, smem_cap, S);
-    else
-      e = B == 1 ? launch_gemv_flat_nb<1, 8, true>(p, stream, num_sms, smem_cap, S)
-                 : launch_gemv_flat_nb<2, 8, true>(p, stream, num_sms, smem_cap, S);
+    if (warps == 16) {
+      switch (B) {
+        case 1: e = launch_gemv_flat_nb<1, 16, true>(p, stream, num_sms, smem_cap, S); break;
+        case 2: e = launch_gemv_flat_nb<2, 16, true>(p, stream, num_sms, smem_cap, S); break;
+        case 3: e = launch_gemv_flat_nb<3, 16, true>(p, stream, num_sms, smem_cap, S); break;
+        default: e = launch_gemv_flat_nb<4, 16, true>(p, stream, num_sms, smem_cap, S); break;
+      }
+    } else {
+      switch (B) {
+        case 1: e = launch_gemv_flat_nb<1, 8, true>(p, stream, num_sms, smem_cap, S); break;
+        case 2: e = launch_gemv_flat_nb<2, 8, true>(p, stream, num_sms, smem_cap, S); break;
+        case 3: e = launch_gemv_flat_nb<3, 8, true>(p, stream, num_sms, smem_cap, S); break;
+        default: e = launch_gemv_flat_nb<4, 8, true>(p, stream, num_sms, smem_cap, S); break;
+      }
+    }
     if (e != cudaErrorNotSupported || split > 0) return e;
   }
   return cudaErrorNotSupported;
