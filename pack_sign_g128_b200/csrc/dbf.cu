@@ -236,7 +236,7 @@ static cudaError_t launch_dbf_small_nb(const uint16_t* a, const uint32_t* B1, co
       break;
     }
   }
-  if (best_smem == 0) return cudaErrorInvalidConfiguration;
+  if (best_smem == 0) return cudaErrorNotSupported;  // no co-resident plan: the caller takes two launches
   GdParams p1 = best1, p2 = best2;
   const int smem = best_smem, S = p1.S, Q = p1.Q;
   p1.signs = B2;
@@ -328,39 +328,8 @@ cudaError_t launch_dbf(const uint16_t* a, const uint32_t* B1, const uint16_t* mi
     // rows on (14.9 vs 17.3 at 4, 17.9 vs 20.9 at 8, with the best rank
     // split for the two launches).
     const bool two = pknob ? pknob == kDbfTwoStep : nb <= 2;
-    if (two) {
-      // Two launches of the direct GEMV core ("LLM binarization episode 01:
-      // DBF", section 4: x_scaled = D_in x, h = V x_scaled, h_scaled = D_mid
-      // h, then y = D_out (U h_scaled)): h_scaled in fp32 through the
-      // workspace; U may be read before the first launch completes (that
-      // launch writes only h).  The second product contracts over r: its
-      // K split is the split-rank form of section 5 item 5 (r partitioned
-      // over the CTAs of a cluster, partial outputs added in a fixed order
-      // through distributed shared memory); dbf_rank_split forces it.
-      // Each product on the register-fed GEMV core (1-2 rows, int8 digits)
-      // where its plan fits and no rank split is forced, else on the direct
-      // core.
-      const int warps = wknob ? wknob : (nb >= 4 ? 16 : 8);
-      const int rsplit = knob(kKnobDbfRankSplit);
-      const int cknob = knob(kKnobDbfCore);  // 0: flat where it fits, 1: flat, 2: direct
-      const bool try_flat = cknob != 2 && nb <= 4;
-      const int fw = wknob ? wknob : (nb <= 2 ? 8 : 16);  // the register-fed core's warps
-      err = cudaErrorNotSupported;
-      if (try_flat) err = launch_gemv_flat_diag(B2, r, n, xg, false, b, mid, nb, h, false, stream, num_sms, smem_cap, 0, fw);
-      if (err == cudaErrorNotSupported)
-        err = launch_gemv_direct_diag(B2, r, n, xg, false, b, mid, nb, h, false, stream, num_sms, smem_cap, warps, 0);
-      if (err == cudaSuccess) {
-        err = cudaErrorNotSupported;
-        if (try_flat && rsplit == 0)
-          err = launch_gemv_flat_diag(B1, m, r, h, true, nullptr, a, nb, yg, true, stream, num_sms, smem_cap, 0, fw);
-        if (err == cudaErrorNotSupported)
-          err = launch_gemv_direct_diag(B1, m, r, h, true, nullptr, a, nb, yg, true, stream, num_sms, smem_cap, warps,
-                                        rsplit);
-      }
-      if (err != cudaSuccess) return err;
-      continue;
-    }
-    switch (nb) {
+    if (!two) {
+      switch (nb) {
 #define W1_DBF_CASE(NBV)                                                                                   \
   case NBV:                                                                                                \
     err = w16 ? launch_dbf_small_nb<NBV, 16>(a, B1, mid, B2, b, im, ir, in, xg, yg, h, bar, stream, num_sms, \
@@ -368,20 +337,54 @@ cudaError_t launch_dbf(const uint16_t* a, const uint32_t* B1, const uint16_t* mi
               : launch_dbf_small_nb<NBV, 8>(a, B1, mid, B2, b, im, ir, in, xg, yg, h, bar, stream, num_sms,  \
                                             smem_cap);                                                    \
     break;
-      W1_DBF_CASE(1)
-      W1_DBF_CASE(2)
-      W1_DBF_CASE(3)
-      W1_DBF_CASE(4)
-      W1_DBF_CASE(5)
-      W1_DBF_CASE(6)
-      W1_DBF_CASE(7)
-      default:
-        err = w16 ? launch_dbf_small_nb<8, 16>(a, B1, mid, B2, b, im, ir, in, xg, yg, h, bar, stream, num_sms,
-                                               smem_cap)
-                  : launch_dbf_small_nb<8, 8>(a, B1, mid, B2, b, im, ir, in, xg, yg, h, bar, stream, num_sms,
-                                              smem_cap);
-        break;
+        W1_DBF_CASE(1)
+        W1_DBF_CASE(2)
+        W1_DBF_CASE(3)
+        W1_DBF_CASE(4)
+        W1_DBF_CASE(5)
+        W1_DBF_CASE(6)
+        W1_DBF_CASE(7)
+        default:
+          err = w16 ? launch_dbf_small_nb<8, 16>(a, B1, mid, B2, b, im, ir, in, xg, yg, h, bar, stream, num_sms,
+                                                 smem_cap)
+                    : launch_dbf_small_nb<8, 8>(a, B1, mid, B2, b, im, ir, in, xg, yg, h, bar, stream, num_sms,
+                                                smem_cap);
+          break;
 #undef W1_DBF_CASE
+      }
+      // a chain whose two products admit no co-resident plan (very long K)
+      // runs as two launches instead
+      if (err != cudaErrorNotSupported) {
+        if (err != cudaSuccess) return err;
+        continue;
+      }
+    }
+    // Two launches of a GEMV core ("LLM binarization episode 01: DBF",
+    // section 4: x_scaled = D_in x, h = V x_scaled, h_scaled = D_mid h, then
+    // y = D_out (U h_scaled)): h_scaled in fp32 through the workspace; U may
+    // be read before the first launch completes (that launch writes only h).
+    // The second product contracts over r: its K split is the split-rank
+    // form of section 5 item 5 (r partitioned over the CTAs of a cluster,
+    // partial outputs added in a fixed order through distributed shared
+    // memory); dbf_rank_split forces it.  Each product on the register-fed
+    // GEMV core (1-4 rows) where its plan fits and no rank split is forced,
+    // else on the direct core.
+    const int warps = wknob ? wknob : (nb >= 4 ? 16 : 8);
+    const int rsplit = knob(kKnobDbfRankSplit);
+    const int cknob = knob(kKnobDbfCore);  // 0: flat where it fits, 1: flat, 2: direct
+    const bool try_flat = cknob != 2 && nb <= 4;
+    const int fw = wknob ? wknob : (nb <= 2 ? 8 : 16);  // the register-fed core's warps
+    err = cudaErrorNotSupported;
+    if (try_flat) err = launch_gemv_flat_diag(B2, r, n, xg, false, b, mid, nb, h, false, stream, num_sms, smem_cap, 0, fw);
+    if (err == cudaErrorNotSupported)
+      err = launch_gemv_direct_diag(B2, r, n, xg, false, b, mid, nb, h, false, stream, num_sms, smem_cap, warps, 0);
+    if (err == cudaSuccess) {
+      err = cudaErrorNotSupported;
+      if (try_flat && rsplit == 0)
+        err = launch_gemv_flat_diag(B1, m, r, h, true, nullptr, a, nb, yg, true, stream, num_sms, smem_cap, 0, fw);
+      if (err == cudaErrorNotSupported)
+        err = launch_gemv_direct_diag(B1, m, r, h, true, nullptr, a, nb, yg, true, stream, num_sms, smem_cap, warps,
+                                      rsplit);
     }
     if (err != cudaSuccess) return err;
   }
