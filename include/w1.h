@@ -58,7 +58,7 @@ typedef enum {
   W1_ERR_CUDA = 6,        /* CUDA launch / runtime error                         */
   W1_ERR_TIMEOUT = 7,     /* device: a bounded wait gave up                      */
   W1_ERR_WORKSPACE = 8,   /* workspace missing or too small                      */
-  W1_ERR_UNSUPPORTED = 9, /* current device is not sm_100 (B200 class)           */
+  W1_ERR_UNSUPPORTED = 9, /* device is not sm_100 (B200 class), or no kernel plan fits the sizes */
   W1_ERR_TOO_LARGE = 10,  /* sizes exceed dbf_apply_noalloc's static scratch     */
   W1_ERR_NOT_CONVERGED = 11 /* device: an iterative solve hit its iteration limit */
 } w1_status;
@@ -401,11 +401,11 @@ size_t w1_moe_workspace_size(int64_t T, int64_t H, int64_t I, int64_t E, int64_t
  *   zero again (after a W1_ERR_TIMEOUT the caller must re-zero it).  After a call
  *   it holds h_scaled (fp32 [min(B,8)][r], byte offset 256) of the last group
  *   of up to 8 batch rows.  Calls sharing a workspace must not overlap.
- * Below 64 rows the batch runs in groups of up to 8 rows: a group of 1-2 rows
+ * Below 64 rows the batch runs in groups of up to 8 rows: a group of 1-4 rows
  * as two products (V then U, h_scaled through the workspace; U's K split
- * over r is the pages' "split rank", section 5 item 5), a group of 3-8 rows
+ * over r is the pages' "split rank", section 5 item 5), a group of 5-8 rows
  * as one kernel with a grid-wide barrier between the two products (section
- * 7).  From 64 rows on, two tensor-core sign GEMMs.  Accuracy:
+ * 7; two products when that kernel has no co-resident plan).  From 64 rows on, two tensor-core sign GEMMs.  Accuracy:
  * |y - y_exact| <= 1e-3 * |a_i| * sum_j |mid_j h_j| per element.
  */
 int dbf_apply(const uint16_t* a, const uint32_t* B1, const uint16_t* mid, const uint32_t* B2,

@@ -9,11 +9,13 @@
 // h = V x_scaled, h_scaled = D_mid h, y_core = U h_scaled, y = D_out y_core).
 //
 // Small batch (B < 64, groups of up to 8 rows), two forms chosen by the group
-// size (both from the steps of the direct GEMV kernel, gemv_direct.cu):
-//  * up to 2 rows: two launches, h_scaled = mid (.) (V . (b (.) x)) into the
-//    workspace, then y = a (.) (U . h_scaled) (its K split over r is the
-//    pages' "split rank", section 5 item 5);
-//  * from 3 rows: ONE kernel runs both binary products -- the joint
+// size:
+//  * up to 4 rows: two launches of a GEMV core (the register-fed core of
+//    gemv_flat.cu, or the direct core of gemv_direct.cu), h_scaled = mid (.)
+//    (V . (b (.) x)) into the workspace, then y = a (.) (U . h_scaled) (its K
+//    split over r is the pages' "split rank", section 5 item 5);
+//  * from 5 rows: ONE kernel (the steps of the direct GEMV kernel) runs both
+//    binary products -- the joint
 //    V-D_mid-U kernel with a grid-wide synchronisation that the DBF post
 //    (section 7, "CUDA/HIP: a starting point") proposes for CUDA.  Each CTA
 //  1. issues the asynchronous copies of its slices of BOTH sign matrices at
@@ -290,6 +292,9 @@ cudaError_t launch_gemv_flat_diag(const uint32_t* signs, int64_t N, int64_t K, c
 
 // Batches of at least this many rows run on the tensor-core path.
 constexpr int64_t kDbfTensorMinBatch = 64;
+// Groups of up to this many rows run as two GEMV launches, larger ones (up to
+// 8) as the fused chain kernel.
+constexpr int kDbfTwoStepMaxRows = 4;
 
 size_t dbf_workspace_bytes(int64_t m, int64_t r, int64_t n, int64_t B) {
   (void)m;
@@ -323,11 +328,12 @@ cudaError_t launch_dbf(const uint16_t* a, const uint32_t* B1, const uint16_t* mi
     const bool w16 = wknob ? wknob == 16 : nb >= 4;
     cudaError_t err;
     // Default form by the measured A/B on the 4096^3 chain (graphs of
-    // back-to-back calls): two launches are faster up to 2 rows per group
-    // (8.1 vs 11.1 us at 1 row, 11.6 vs 14.6 at 2), the fused kernel from 3
-    // rows on (14.9 vs 17.3 at 4, 17.9 vs 20.9 at 8, with the best rank
-    // split for the two launches).
-    const bool two = pknob ? pknob == kDbfTwoStep : nb <= 2;
+    // back-to-back calls, us per call, fused / two launches): 1 row 11.1 /
+    // 8.1, 2 rows 14.5 / 10.1, 3 rows 16.2 / 13.5, 4 rows 14.9 / 12.6 (U . h
+    // with r split over 2 CTAs of a cluster; 14.5 on the register-fed core),
+    // 8 rows 17.8 / 19.1 (best split).  So two launches up to 4 rows, the
+    // fused kernel from 5.
+    const bool two = pknob ? pknob == kDbfTwoStep : nb <= kDbfTwoStepMaxRows;
     if (!two) {
       switch (nb) {
 #define W1_DBF_CASE(NBV)                                                                                   \
@@ -370,7 +376,9 @@ cudaError_t launch_dbf(const uint16_t* a, const uint32_t* B1, const uint16_t* mi
     // GEMV core (1-4 rows) where its plan fits and no rank split is forced,
     // else on the direct core.
     const int warps = wknob ? wknob : (nb >= 4 ? 16 : 8);
-    const int rsplit = knob(kKnobDbfRankSplit);
+    const int rknob = knob(kKnobDbfRankSplit);
+    // 4 rows: U . h on the direct core with r split over 2 CTAs by default
+    const int rsplit = rknob ? rknob : (nb == 4 ? 2 : 0);
     const int cknob = knob(kKnobDbfCore);  // 0: flat where it fits, 1: flat, 2: direct
     const bool try_flat = cknob != 2 && nb <= 4;
     const int fw = wknob ? wknob : (nb <= 2 ? 8 : 16);  // the register-fed core's warps
@@ -385,6 +393,8 @@ cudaError_t launch_dbf(const uint16_t* a, const uint32_t* B1, const uint16_t* mi
       if (err == cudaErrorNotSupported)
         err = launch_gemv_direct_diag(B1, m, r, h, true, nullptr, a, nb, yg, true, stream, num_sms, smem_cap, warps,
                                       rsplit);
+      if (err == cudaErrorNotSupported && rknob == 0 && rsplit != 0)  // the default split does not fit: planner
+        err = launch_gemv_direct_diag(B1, m, r, h, true, nullptr, a, nb, yg, true, stream, num_sms, smem_cap, warps, 0);
     }
     if (err != cudaSuccess) return err;
   }

@@ -106,7 +106,7 @@ const char* w1_status_string(int status) {
     case W1_ERR_CUDA: return "W1_ERR_CUDA: CUDA error";
     case W1_ERR_TIMEOUT: return "W1_ERR_TIMEOUT: bounded device wait gave up";
     case W1_ERR_WORKSPACE: return "W1_ERR_WORKSPACE: workspace missing or too small";
-    case W1_ERR_UNSUPPORTED: return "W1_ERR_UNSUPPORTED: device is not sm_100";
+    case W1_ERR_UNSUPPORTED: return "W1_ERR_UNSUPPORTED: device is not sm_100, or no kernel plan fits these sizes";
     case W1_ERR_TOO_LARGE: return "W1_ERR_TOO_LARGE: sizes exceed the static scratch of dbf_apply_noalloc";
     case W1_ERR_NOT_CONVERGED: return "W1_ERR_NOT_CONVERGED: the iterative solve stopped at its iteration limit";
     default: return "unknown w1 status";

@@ -1,7 +1,7 @@
 """dbf_apply on the GPU vs the fp64 oracle chain.
 
 Every test runs with each small-batch chain form -- the fused chain kernel and
-two launches of a GEMV core (the dbf_path knob; groups of 1-2 rows take the
+two launches of a GEMV core (the dbf_path knob; groups of 1-4 rows take the
 register-fed core, or the direct core with dbf_core=direct) -- forced to 8
 and to 16 warps per CTA (the dbf_warps knob).  Batches of 64 and more take the
 tensor-core path either way."""
@@ -23,7 +23,7 @@ def dbf_path(request, knob):
     form, warps = (request.param[:-2], request.param[-2:]) if request.param.endswith("16") else (request.param[:-1], "8")
     if form == "twostepdirect":
         form = "twostep"
-        knob("dbf_core", "direct")  # the direct GEMV core for 1-2 rows too
+        knob("dbf_core", "direct")  # the direct GEMV core for 1-4 rows too
     knob("dbf_path", form)
     knob("dbf_warps", warps)
     return request.param
