@@ -87,7 +87,6 @@ int w1_sync_status(w1_stream_t stream);
  *   "sg_bm"         128 | 256 forces the sign GEMM's token tile (W1_SG_BM)
  *   "sg_exp"        4 | 8 forces the sign GEMM's expander warps per CTA (W1_SG_EXP)
  *   "sg_a"          "smem" | "tmem": where the sign GEMM's 128-token tiles keep the weight operand (W1_SG_A)
- *   "sg_sk"         "off" | "on": the sign GEMM's stream-K schedule (W1_SG_SK)
  *   "verbose"       nonzero prints plans and choices on stderr (W1_VERBOSE)
  * Returns W1_ERR_NULL for a NULL name, W1_ERR_SHAPE for an unknown name or
  * value. */
@@ -330,14 +329,10 @@ int w1_power_iteration(const float* A, int64_t m, int64_t n, const float* v0, in
  * blockwise scale is applied inside the MMA and all of K accumulates in one
  * fp32 TMEM tile.  Same accuracy bound as w1_gemv.
  * workspace: >= w1_gemm_workspace_size(M, K) bytes of device memory, 256-byte
- *   aligned (the fp16 copy of x, the token scales and, from M = 256 on, the
- *   stream-K partial tiles and flags, about 19 MB); contents on entry are
+ *   aligned (the fp16 copy of x and the token scales); contents on entry are
  *   ignored, nothing is carried between calls; calls sharing a workspace must
  *   not overlap.  Too small / null: W1_ERR_WORKSPACE; misaligned: W1_ERR_ALIGN.
- * Two kernels on `stream` (prep, GEMM).  With stream-K the output tiles' K
- * stages are split evenly over the CTAs; a tile split between CTAs adds its
- * fp32 partial sums in a fixed CTA order, so results are deterministic for a
- * given GPU (SM count) but may differ in the last bits from an unsplit tile.
+ * Two kernels on `stream` (prep, GEMM).
  */
 int w1_gemm(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t K,
             const uint16_t* x, int64_t M, float* y, void* workspace, size_t ws_bytes,

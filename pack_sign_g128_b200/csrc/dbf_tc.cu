@@ -27,12 +27,10 @@ struct SgParams;
 namespace dbftc {
 // Workspace of the tensor path (after the 256-byte barrier header):
 // per-row scales (float [B] 2^-c_t, float [B] 2^d_t), x_s fp16 [B][n],
-// h_s fp16 [B][r], and from 256 rows on the sign GEMMs' stream-K partial
-// slots and flags (shared by the two GEMMs, one after the other).
+// h_s fp16 [B][r].
 struct Ws {
-  size_t cscale, dscale, dinv, xs, hs, sk, total;
+  size_t cscale, dscale, dinv, xs, hs, total;
 };
-constexpr int64_t kSkMinB = 256;  // from this many rows: the sign GEMMs' stream-K slots
 __host__ __device__ inline Ws ws_layout(int64_t B, int64_t r, int64_t n) {
   Ws w;
   size_t off = 256;
@@ -46,8 +44,6 @@ __host__ __device__ inline Ws ws_layout(int64_t B, int64_t r, int64_t n) {
   off += (2 * B * n + 1023) / 1024 * 1024;
   w.hs = off;
   off += (2 * B * r + 1023) / 1024 * 1024;
-  w.sk = off;
-  if (B >= kSkMinB) off += sg_sk_workspace_bytes();
   w.total = off;
   return w;
 }
@@ -60,8 +56,7 @@ size_t dbf_tc_workspace_bytes(int64_t r, int64_t n, int64_t B) { return dbftc::w
 template <bool HALF_OUT>
 cudaError_t launch_sg_gemm(const SgParams& p, const void* bmat, int64_t bcols, cudaStream_t stream, int num_sms);
 cudaError_t launch_sg_prep(const uint16_t* x, const uint16_t* bdiag, const uint16_t* mid, int64_t n, int64_t r,
-                          int64_t B, __half* xs, float* cscale, float* dscale, float* dinv, void* sk_ws,
-                          cudaStream_t stream);
+                          int64_t B, __half* xs, float* cscale, float* dscale, float* dinv, cudaStream_t stream);
 
 cudaError_t launch_dbf_tc(const uint16_t* a, const uint32_t* B1, const uint16_t* mid, const uint32_t* B2,
                           const uint16_t* b, int64_t m, int64_t r, int64_t n, const uint16_t* x, int64_t B, float* y,
@@ -74,14 +69,9 @@ cudaError_t launch_dbf_tc(const uint16_t* a, const uint32_t* B1, const uint16_t*
   float* di = reinterpret_cast<float*>(ws + L.dinv);
   __half* xs = reinterpret_cast<__half*>(ws + L.xs);
   __half* hs = reinterpret_cast<__half*>(ws + L.hs);
-  void* sk_ws = B >= kSkMinB ? ws + L.sk : nullptr;
-  cudaError_t err = launch_sg_prep(x, b, mid, n, r, B, xs, cs, ds, di, sk_ws, stream);
+  cudaError_t err = launch_sg_prep(x, b, mid, n, r, B, xs, cs, ds, di, stream);
   if (err != cudaSuccess) return err;
-  float* skp = sk_ws ? static_cast<float*>(sk_ws) : nullptr;
-  unsigned int* skf = sk_ws ? sg_sk_flags(sk_ws) : nullptr;
   SgParams p1 = {};
-  p1.sk_part = skp;
-  p1.sk_flag = skf;
   p1.signs = B2;
   p1.rdiag = mid;
   p1.s1 = cs;
@@ -94,8 +84,6 @@ cudaError_t launch_dbf_tc(const uint16_t* a, const uint32_t* B1, const uint16_t*
   if (err != cudaSuccess) return err;
   // phase 2 undoes the intermediate's scale: s1 = 2^-d
   SgParams p2 = {};
-  p2.sk_part = skp;
-  p2.sk_flag = skf;
   p2.signs = B1;
   p2.rdiag = a;
   p2.s1 = di;

@@ -24,8 +24,7 @@ namespace w1 {
 template <bool HALF_OUT>
 cudaError_t launch_sg_gemm(const SgParams& p, const void* bmat, int64_t bcols, cudaStream_t stream, int num_sms);
 cudaError_t launch_sg_prep(const uint16_t* x, const uint16_t* bdiag, const uint16_t* mid, int64_t n, int64_t r,
-                          int64_t B, __half* xs, float* cscale, float* dscale, float* dinv, void* sk_ws,
-                          cudaStream_t stream);
+                          int64_t B, __half* xs, float* cscale, float* dscale, float* dinv, cudaStream_t stream);
 
 // ------------------------------------------------------------------ host side
 
@@ -98,12 +97,9 @@ bool make_tmap_u32_sw128(CUtensorMap* map, const void* base, int64_t rows, int64
   return r == CUDA_SUCCESS;
 }
 
-// Workspace: xs fp16 [M][K], the token scales, and (from 256 tokens on) the
-// sign GEMM's stream-K partial slots and flags.
-constexpr int64_t kGemmSkMinM = 256;
 size_t gemm_workspace_bytes(int64_t M, int64_t K) {
   const size_t xs_bytes = (static_cast<size_t>(M) * K * 2 + 1023) / 1024 * 1024;
-  return xs_bytes + (static_cast<size_t>(M) * 4 + 255) / 256 * 256 + (M >= kGemmSkMinM ? sg_sk_workspace_bytes() : 0);
+  return xs_bytes + (static_cast<size_t>(M) * 4 + 255) / 256 * 256;
 }
 
 cudaError_t launch_gemm(const uint32_t* signs, const uint16_t* scales, int64_t N, int64_t K,
@@ -112,16 +108,9 @@ cudaError_t launch_gemm(const uint32_t* signs, const uint16_t* scales, int64_t N
   const size_t xs_bytes = (static_cast<size_t>(M) * K * 2 + 1023) / 1024 * 1024;
   __half* xs = static_cast<__half*>(workspace);
   float* cscale = reinterpret_cast<float*>(static_cast<unsigned char*>(workspace) + xs_bytes);
-  void* sk_ws = M >= kGemmSkMinM ? static_cast<unsigned char*>(workspace) + xs_bytes +
-                                       (static_cast<size_t>(M) * 4 + 255) / 256 * 256
-                                 : nullptr;
-  cudaError_t err = launch_sg_prep(x, nullptr, nullptr, K, 0, M, xs, cscale, nullptr, nullptr, sk_ws, stream);
+  cudaError_t err = launch_sg_prep(x, nullptr, nullptr, K, 0, M, xs, cscale, nullptr, nullptr, stream);
   if (err != cudaSuccess) return err;
   SgParams p = {};
-  if (sk_ws) {
-    p.sk_part = static_cast<float*>(sk_ws);
-    p.sk_flag = sg_sk_flags(sk_ws);
-  }
   p.signs = signs;
   p.gscales = scales;
   p.s1 = cscale;

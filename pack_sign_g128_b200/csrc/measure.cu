@@ -337,15 +337,14 @@ cudaError_t launch_sg_gemm(const SgParams& p, const void* bmat, int64_t bcols, c
 // Workspace of dbf_residual: the measurement header, H [n][r] fp16,
 // W_approx^T [n][m] fp32, b [n] fp32.
 struct DresWs {
-  size_t h, wat, bs, sk, total;
+  size_t h, wat, bs, total;
 };
 static DresWs dres_ws(int64_t m, int64_t r, int64_t n) {
   DresWs d;
   d.h = meas_align(measure_workspace_bytes(m, n));
   d.wat = d.h + meas_align(static_cast<size_t>(2) * n * r);
   d.bs = d.wat + meas_align(static_cast<size_t>(4) * n * m);
-  d.sk = d.bs + meas_align(static_cast<size_t>(4) * n);
-  d.total = d.sk + (n >= 256 ? meas_align(sg_sk_workspace_bytes()) : 0);  // the sign GEMM's stream-K slots
+  d.total = d.bs + meas_align(static_cast<size_t>(4) * n);
   return d;
 }
 size_t dbf_residual_workspace_bytes(int64_t m, int64_t r, int64_t n) {
@@ -364,18 +363,11 @@ cudaError_t launch_dbf_residual(const float* W, const uint16_t* a, const uint32_
   float* bs = reinterpret_cast<float*>(base + L.bs);
   cudaError_t e = cudaMemsetAsync(ws.ticket, 0, sizeof(unsigned int), stream);
   if (e != cudaSuccess) return e;
-  void* sk_ws = n >= 256 ? base + L.sk : nullptr;
-  if (sk_ws) e = cudaMemsetAsync(sg_sk_flags(sk_ws), 0, kSgSkFlagBytes, stream);
-  if (e != cudaSuccess) return e;
   const int64_t hwarps = (n / 32) * (r / 32);
   e = meas_launch(dres_h_kernel, dim3(static_cast<unsigned>((hwarps + 7) / 8)), stream, B2, mid, b,
                   static_cast<int>(r), static_cast<int>(n), H, bs);
   if (e != cudaSuccess) return e;
   SgParams p = {};
-  if (sk_ws) {
-    p.sk_part = static_cast<float*>(sk_ws);
-    p.sk_flag = sg_sk_flags(sk_ws);
-  }
   p.signs = B1;
   p.gscales = nullptr;
   p.rdiag = a;

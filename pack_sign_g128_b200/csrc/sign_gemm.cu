@@ -27,7 +27,6 @@
 //    (thread = TMEM lane: row diagonal and token scale, store), draining one
 //    accumulator while the MMA fills the other.
 // Products of +-s and fp16 are exact in the tensor core; accumulation is fp32.
-#include <algorithm>
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_fp16.h>
@@ -90,8 +89,7 @@ struct Smem {
 __global__ void __launch_bounds__(256) sg_prep_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ bdiag,
                                                       const uint16_t* __restrict__ mid, int n, int r,
                                                       __half* __restrict__ xs, float* __restrict__ cscale,
-                                                      float* __restrict__ dscale, float* __restrict__ dinv,
-                                                      unsigned int* __restrict__ zflags, int nz) {
+                                                      float* __restrict__ dscale, float* __restrict__ dinv) {
   // 16-byte vectors (8 values); the row stays in registers between the
   // reductions and the conversion when n <= 8 * 256 * kMaxV, else it is re-read.
   constexpr int kMaxV = 4;
@@ -215,8 +213,6 @@ __global__ void __launch_bounds__(256) sg_prep_kernel(const uint16_t* __restrict
     if (i < nv) convert(i, keep[j]);
   }
   for (int i = threadIdx.x + 256 * kMaxV; i < nv; i += 256) convert(i, __ldg(xr + i));
-  if (zflags && t == 0)  // the stream-K flags of the GEMMs that follow start at zero
-    for (int i = threadIdx.x; i < nz; i += blockDim.x) zflags[i] = 0u;
   if (threadIdx.x == 0) {
     cscale[t] = ldexpf(1.f, -c);
     if (dscale) dscale[t] = ldexpf(1.f, d);
@@ -236,67 +232,8 @@ struct SgParams {
   const float* s2;         // per token: 2^d (phase 1) or unused
   __half* out_h;           // phase 1 output [M][rows]
   float* out_f;            // phase 2 output [M][rows]
-  // stream-K (optional): per-CTA fp32 partial tiles [kSkMaxCtas][128 x 256]
-  // and their ready flags [kSkMaxCtas] (zero before the launch; the kernel
-  // leaves them zero)
-  float* sk_part;
-  unsigned int* sk_flag;
   int M, rows, K, MT, NT, NK;
-  int sk;  // set by the launcher: 1 = the CTAs split the (tile, stage) sequence evenly
 };
-
-// Stream-K.  The output tiles' K stages, tile-major, form one sequence that
-// the G CTAs split into equal contiguous ranges, so no CTA runs a whole tile
-// more than another.  A CTA's range is a list of units (tile, first stage,
-// end stage): only its first unit can start inside a tile and only its last
-// can end inside one.  A unit that does not start at stage 0 writes its
-// fp32 accumulator to the CTA's partial slot and raises the CTA's flag; the
-// CTA whose unit holds the tile's stage 0 (its last unit) waits for the
-// flags of the following CTAs that hold the rest of the tile, adds their
-// partials in CTA order (a fixed order: deterministic), runs the epilogue
-// and clears the flags.  Every CTA is resident (one per SM, G <= SMs).
-namespace sg {
-constexpr int kSkMaxCtas = 148;               // CTAs (and partial slots) of a stream-K launch
-constexpr int kSkSlotFloats = 128 * 256;      // one 128 x 256 fp32 partial tile
-}  // namespace sg
-// Stream-K workspace: the partial slots, then the flags (4 per CTA).
-constexpr size_t kSgSkFlagBytes = (static_cast<size_t>(sg::kSkMaxCtas) * 4 * 4 + 255) / 256 * 256;
-__host__ __device__ inline size_t sg_sk_workspace_bytes() {
-  return static_cast<size_t>(sg::kSkMaxCtas) * sg::kSkSlotFloats * 4 + kSgSkFlagBytes;
-}
-__host__ __device__ inline unsigned int* sg_sk_flags(void* ws) {
-  return reinterpret_cast<unsigned int*>(static_cast<unsigned char*>(ws) +
-                                         static_cast<size_t>(sg::kSkMaxCtas) * sg::kSkSlotFloats * 4);
-}
-
-// The i-th unit of CTA b (false past the last): tile, stages [ks0, ks1).
-__device__ __forceinline__ bool sg_unit(const SgParams& p, int NKS, int ntiles, int i, int& tile, int& ks0, int& ks1) {
-  const int G = static_cast<int>(gridDim.x), b = static_cast<int>(blockIdx.x);
-  if (!p.sk) {
-    tile = b + i * G;
-    ks0 = 0;
-    ks1 = NKS;
-    return tile < ntiles;
-  }
-  const int64_t S = static_cast<int64_t>(ntiles) * NKS;
-  const int64_t lo = S * b / G, hi = S * (b + 1) / G;
-  const int64_t t0 = lo / NKS;
-  tile = static_cast<int>(t0 + i);
-  const int64_t base = static_cast<int64_t>(tile) * NKS;
-  if (base >= hi) return false;
-  ks0 = i == 0 ? static_cast<int>(lo - base) : 0;
-  ks1 = static_cast<int>(min(static_cast<int64_t>(NKS), hi - base));
-  return true;
-}
-// The CTA whose range holds stage s of the sequence.
-__device__ __forceinline__ int sg_sk_cta_of(int64_t s, int64_t S) {
-  return static_cast<int>(((s + 1) * static_cast<int64_t>(gridDim.x) - 1) / S);
-}
-__device__ __forceinline__ unsigned int sg_ld_acquire(const unsigned int* f) {
-  unsigned int v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(f) : "memory");
-  return v;
-}
 
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
@@ -344,21 +281,15 @@ __global__ void __launch_bounds__(sg::threads_for<EXP>(), 1)
   pdl_wait();
   const int ntiles = p.MT * p.NT;
   const int NKS = p.NK * (BK / BKS);  // stages per tile (one per scale group)
-  // this CTA's units: whole tiles b, b + G, ..., or (stream-K) one contiguous
-  // range of the (tile, stage) sequence
-  int my_stages = 0;
-  {
-    int tile, ks0, ks1;
-    for (int i = 0; sg_unit(p, NKS, ntiles, i, tile, ks0, ks1); ++i) my_stages += ks1 - ks0;
-  }
+  const int my_tiles = (ntiles - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) /
+                       static_cast<int>(gridDim.x);
 
   if (warp == 0) {
     if (lane == 0) {
       uint32_t c = 0;
-      int tile, ks0, ks1;
-      for (int i = 0; sg_unit(p, NKS, ntiles, i, tile, ks0, ks1); ++i) {
+      for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
         const int mt = tile % p.MT;
-        for (int ks = ks0; ks < ks1; ++ks, ++c) {
+        for (int ks = 0; ks < NKS; ++ks, ++c) {
           const int s = c % NS;
           if (!mbar_wait(&sm.empty[s], ((c / NS) & 1) ^ 1)) goto done_prod;
           mbar_arrive_expect_tx(&sm.full[s], kXStage);
@@ -371,13 +302,12 @@ __global__ void __launch_bounds__(sg::threads_for<EXP>(), 1)
   } else if (warp == 1) {
     if (lane == 0) {
       uint32_t c = 0, tl = 0;
-      int tile, ks0, ks1;
-      for (; sg_unit(p, NKS, ntiles, static_cast<int>(tl), tile, ks0, ks1); ++tl) {
+      for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++tl) {
         const int cb = tl & 1;
         if (!mbar_wait(&sm.empty_c[cb], ((tl >> 1) & 1) ^ 1)) goto done_mma;
         tc_fence_after();
         const uint32_t d = tmem + cb * BM;
-        for (int ks = ks0; ks < ks1; ++ks, ++c) {
+        for (int ks = 0; ks < NKS; ++ks, ++c) {
           const int s = c % NS;
           if (!mbar_wait(&sm.full[s], (c / NS) & 1)) goto done_mma;
           tc_fence_after();
@@ -387,11 +317,11 @@ __global__ void __launch_bounds__(sg::threads_for<EXP>(), 1)
             const uint32_t xo = (kk >> 2) * kXAtom + (kk & 3) * 32;
             if constexpr (TA) {
               tc_mma_ts(d, tmem + kACol + s * (BKS / 2) + kk * 8, smem_desc_sw128(xbase + xo), kIdesc,
-                        (ks > ks0 || kk > 0) ? 1u : 0u);
+                        (ks > 0 || kk > 0) ? 1u : 0u);
             } else {
               const uint32_t ao = (kk >> 2) * kAAtom + (kk & 3) * 32;
               tc_mma_ss(d, smem_desc_sw128(smem_u32(sm.a[s]) + ao), smem_desc_sw128(xbase + xo), kIdesc,
-                        (ks > ks0 || kk > 0) ? 1u : 0u);
+                        (ks > 0 || kk > 0) ? 1u : 0u);
             }
           }
           tc_commit(&sm.empty[s]);
@@ -415,12 +345,11 @@ __global__ void __launch_bounds__(sg::threads_for<EXP>(), 1)
     const int rl = (warp & 3) * 32 + lane;  // a warp reaches TMEM lanes 32 (warp % 4) ..
     const int half = EXP == 8 ? (warp - 2) >> 2 : 0;  // the atom this thread writes (8 expander warps)
     const int64_t wrow = p.K >> 5;
-    int ld_i = 0, ld_tile = 0, ld_ks = 0, ld_ks1 = 0;
-    bool ld_ok = sg_unit(p, NKS, ntiles, 0, ld_tile, ld_ks, ld_ks1);
+    int ld_tile = blockIdx.x, ld_ks = 0;
     auto fetch = [&](uint4& w, uint32_t& sc) {
       w = make_uint4(0, 0, 0, 0);
       sc = 0x3C00u;
-      if (ld_ok) {
+      if (ld_tile < ntiles) {
         const int n = (ld_tile / p.MT) * BN + rl;
         if (n < p.rows) {  // a row's words are 16-byte aligned (K % 128 == 0)
           if (EXP == 4) {
@@ -433,13 +362,17 @@ __global__ void __launch_bounds__(sg::threads_for<EXP>(), 1)
           }
           if (p.gscales) sc = __ldg(p.gscales + static_cast<int64_t>(n) * p.NK + ld_ks);
         }
-        if (++ld_ks == ld_ks1) ld_ok = sg_unit(p, NKS, ntiles, ++ld_i, ld_tile, ld_ks, ld_ks1);
+        if (++ld_ks == NKS) {
+          ld_ks = 0;
+          ld_tile += gridDim.x;
+        }
       }
     };
     uint4 wr[kPf];
     uint32_t sr[kPf];
 #pragma unroll
     for (int j = 0; j < kPf; ++j) fetch(wr[j], sr[j]);
+    const int my_stages = my_tiles * NKS;
     const uint32_t row_off = static_cast<uint32_t>(rl) * 128u;
     const uint32_t sw = static_cast<uint32_t>(rl & 7);
     uint32_t c = 0;
@@ -492,20 +425,12 @@ __global__ void __launch_bounds__(sg::threads_for<EXP>(), 1)
     }
   done_exp:;
   } else {
-    // epilogue: one accumulator per unit.  A whole tile, or the stage-0 unit
-    // of a split tile plus the partials of the CTAs that hold the rest of it
-    // (stream-K), is scaled by the row diagonal and the token scales and
-    // stored; any other unit of a split tile goes to this CTA's partial slot.
-    // Warp q of the epilogue handles TMEM lanes (rows) 32 q .. 32 q + 31 and
-    // waits only for the same rows of the other CTAs' partials (one flag per
-    // CTA and row quarter), so the four warps never wait for one another.
+    // epilogue: one accumulator per tile, scaled by the row diagonal and the token scales
     const int quarter = warp & 3;
     const int rl = quarter * 32 + lane;
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
-    const int64_t S_all = static_cast<int64_t>(ntiles) * NKS;
     uint32_t tl = 0;
-    int tile, ks0, ks1;
-    for (; sg_unit(p, NKS, ntiles, static_cast<int>(tl), tile, ks0, ks1); ++tl) {
+    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++tl) {
       const int mt = tile % p.MT, nt = tile / p.MT;
       const int n = nt * BN + rl;
       const bool valid = n < p.rows;
@@ -514,66 +439,12 @@ __global__ void __launch_bounds__(sg::threads_for<EXP>(), 1)
       if (!mbar_wait_warp(&sm.full_c[cb], (tl >> 1) & 1)) goto done_epi;
       tc_fence_after();
       const int mrem = min(BM, p.M - mt * BM);
-      if (ks0 > 0) {
-        // a later part of a split tile: raw fp32 sums to the partial slot
-        float* slot = p.sk_part + static_cast<int64_t>(blockIdx.x) * kSkSlotFloats;
-#pragma unroll 1
-        for (int q4 = 0; q4 < BM / 32; ++q4) {
-          if (q4 * 32 >= mrem) break;
-          uint32_t rr[32];
-          tmem_ld32(tmem + lane_addr + cb * BM + q4 * 32, rr);
-          tc_wait_ld();
-          float4* dst = reinterpret_cast<float4*>(slot + (q4 * 128 + rl) * 32);
-#pragma unroll
-          for (int j = 0; j < 8; ++j)
-            dst[j] = make_float4(__uint_as_float(rr[4 * j]), __uint_as_float(rr[4 * j + 1]),
-                                 __uint_as_float(rr[4 * j + 2]), __uint_as_float(rr[4 * j + 3]));
-        }
-        tc_fence_before();
-        mbar_arrive(&sm.empty_c[cb]);
-        __syncwarp();
-        if (lane == 0) {
-          __threadfence();
-          asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p.sk_flag + blockIdx.x * 4 + quarter), "r"(1u)
-                       : "memory");
-        }
-        continue;
-      }
-      // stage 0 of the tile: the CTAs after this one that hold its other stages
-      const int c_last = ks1 == NKS ? static_cast<int>(blockIdx.x)
-                                    : sg_sk_cta_of(static_cast<int64_t>(tile) * NKS + NKS - 1, S_all);
-      bool have = true;
-      for (int c = blockIdx.x + 1; c <= c_last; ++c) {
-        const unsigned int* f = p.sk_flag + c * 4 + quarter;
-        uint32_t i = 0;
-        while (sg_ld_acquire(f) == 0u && ++i < kSpinLimit) {
-          if (i > 64) __nanosleep(64);
-        }
-        if (i >= kSpinLimit) have = false;
-      }
-      __syncwarp();
-      if (!have) set_status(W1_ERR_TIMEOUT);
 #pragma unroll 1
       for (int q4 = 0; q4 < BM / 32; ++q4) {
         if (q4 * 32 >= mrem) break;
         uint32_t rr[32];
         tmem_ld32(tmem + lane_addr + cb * BM + q4 * 32, rr);
         tc_wait_ld();
-        float v[32];
-#pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(rr[j]);
-        for (int c = blockIdx.x + 1; c <= c_last && have; ++c) {  // CTA order: a fixed sum order
-          const float4* src =
-              reinterpret_cast<const float4*>(p.sk_part + static_cast<int64_t>(c) * kSkSlotFloats + (q4 * 128 + rl) * 32);
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const float4 u = __ldcg(src + j);
-            v[4 * j] += u.x;
-            v[4 * j + 1] += u.y;
-            v[4 * j + 2] += u.z;
-            v[4 * j + 3] += u.w;
-          }
-        }
         if (valid) {
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
@@ -581,10 +452,10 @@ __global__ void __launch_bounds__(sg::threads_for<EXP>(), 1)
             if (m < mrem) {
               const int64_t tok = static_cast<int64_t>(mt) * BM + m;
               if (PHASE1) {
-                const float o = rd * v[j] * (__ldg(p.s1 + tok) * __ldg(p.s2 + tok));
-                p.out_h[tok * p.rows + n] = __float2half_rn(o);
+                const float v = rd * __uint_as_float(rr[j]) * (__ldg(p.s1 + tok) * __ldg(p.s2 + tok));
+                p.out_h[tok * p.rows + n] = __float2half_rn(v);
               } else {
-                p.out_f[tok * p.rows + n] = rd * v[j] * __ldg(p.s1 + tok);
+                p.out_f[tok * p.rows + n] = rd * __uint_as_float(rr[j]) * __ldg(p.s1 + tok);
               }
             }
           }
@@ -592,9 +463,6 @@ __global__ void __launch_bounds__(sg::threads_for<EXP>(), 1)
       }
       tc_fence_before();
       mbar_arrive(&sm.empty_c[cb]);
-      __syncwarp();
-      if (lane == 0)  // the partials are consumed: clear their flags for the next launch
-        for (int c = blockIdx.x + 1; c <= c_last; ++c) p.sk_flag[c * 4 + quarter] = 0u;
     }
   done_epi:;
   }
@@ -621,19 +489,8 @@ static cudaError_t launch_sg_gemm_bm(SgParams p, const void* bmat, int64_t bcols
   cudaError_t err = ensure_dyn_smem(reinterpret_cast<const void*>(kern), static_cast<int>(smem));
   if (err != cudaSuccess) return err;
   const int ntiles = p.MT * p.NT;
-  // Stream-K where whole tiles would leave the last round of tiles part
-  // empty (at least 4% more time than an even split) and every CTA gets at
-  // least 4 stages; needs the workspace's partial slots.
-  const int G = std::min(num_sms, kSkMaxCtas);
-  const int64_t stages = static_cast<int64_t>(ntiles) * (p.K / BKS);
-  const int64_t rounds = (ntiles + G - 1) / G;
-  const int fsk = knob(kKnobSgSk);  // tuning knob: 1 off, 2 on (where the workspace allows)
-  p.sk = 0;
-  if (p.sk_part && p.sk_flag && BM <= 256 && stages >= 4 * static_cast<int64_t>(G) && fsk != 1 &&
-      (fsk == 2 || static_cast<double>(rounds) * G >= 1.04 * ntiles))
-    p.sk = 1;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(p.sk ? G : (ntiles < num_sms ? ntiles : num_sms)));
+  cfg.gridDim = dim3(static_cast<unsigned>(ntiles < num_sms ? ntiles : num_sms));
   cfg.blockDim = dim3(threads_for<EXP>());
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
@@ -673,8 +530,7 @@ cudaError_t launch_sg_gemm(const SgParams& p, const void* bmat, int64_t bcols, c
 }
 
 cudaError_t launch_sg_prep(const uint16_t* x, const uint16_t* bdiag, const uint16_t* mid, int64_t n, int64_t r,
-                          int64_t B, __half* xs, float* cscale, float* dscale, float* dinv, void* sk_ws,
-                          cudaStream_t stream) {
+                          int64_t B, __half* xs, float* cscale, float* dscale, float* dinv, cudaStream_t stream) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(B));
   cfg.blockDim = dim3(256);
@@ -684,9 +540,8 @@ cudaError_t launch_sg_prep(const uint16_t* x, const uint16_t* bdiag, const uint1
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  unsigned int* zf = sk_ws ? sg_sk_flags(sk_ws) : nullptr;
   return cudaLaunchKernelEx(&cfg, sg_prep_kernel, x, bdiag, mid, static_cast<int>(n), static_cast<int>(r), xs, cscale,
-                            dscale, dinv, zf, sg::kSkMaxCtas * 4);
+                            dscale, dinv);
 }
 
 }  // namespace w1

@@ -416,14 +416,13 @@ inline cudaError_t ensure_dyn_smem(const void* kernel, int bytes) {
 //   dbf_core      W1_DBF_CORE       two-launch chain's GEMV core: 0 = register-fed where it fits, 1 = same, 2 = direct
 //   sg_exp        W1_SG_EXP         sign GEMM expander warps: 0 = by token tile, else 4 or 8
 //   sg_a          W1_SG_A           sign GEMM weight operand of 128-token tiles: 0 = default, 1 = smem, 2 = TMEM
-//   sg_sk         W1_SG_SK          sign GEMM stream-K schedule: 0 = by tile count, 1 = off, 2 = on
 //   verbose       W1_VERBOSE        nonzero: plans and choices on stderr
 #include <atomic>
 #include <cstdlib>
 #include <cstring>
 namespace w1 {
 enum KnobId { kKnobGemvPath, kKnobGemvSplit, kKnobGemvAutotune, kKnobMoePath, kKnobDbfPath, kKnobDbfWarps,
-              kKnobDbfRankSplit, kKnobSgBm, kKnobDbfCore, kKnobSgExp, kKnobSgA, kKnobSgSk, kKnobVerbose, kKnobCount };
+              kKnobDbfRankSplit, kKnobSgBm, kKnobDbfCore, kKnobSgExp, kKnobSgA, kKnobVerbose, kKnobCount };
 // GEMV kernels a knob can force (also the kinds of the dispatcher's choices).
 enum GemvPathKnob { kGemvAuto = 0, kGemvDirect8 = 1, kGemvDirect16 = 2, kGemvTc = 3, kGemvRing = 4, kGemvFlat = 5,
                     kGemvFlat16 = 6 };
@@ -448,7 +447,6 @@ inline const KnobSpec& knob_spec(int id) {
       {"dbf_core", "W1_DBF_CORE", 0, {"flat", "direct", nullptr}},
       {"sg_exp", "W1_SG_EXP", 0, {nullptr}},
       {"sg_a", "W1_SG_A", 0, {"smem", "tmem", nullptr}},
-      {"sg_sk", "W1_SG_SK", 0, {"off", "on", nullptr}},
       {"verbose", "W1_VERBOSE", 0, {nullptr}},
   };
   return specs[id];

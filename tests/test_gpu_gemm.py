@@ -84,22 +84,3 @@ def test_gemm_every_kernel_form(knob, bm, exp, a):
     knob("sg_exp", 4)
     knob("sg_a", "smem")
     assert np.array_equal(y, run_gemm(s, c, x))
-
-
-@pytest.mark.parametrize("M,N,K,bm", [(1100, 2200, 1152, 128), (1100, 2200, 1152, 256), (512, 4096, 4096, 128),
-                                      (300, 1000, 384, 256)])
-def test_gemm_stream_k(knob, M, N, K, bm):
-    """The stream-K schedule (tiles' K stages split evenly over the CTAs, split
-    tiles summed in CTA order) against the whole-tile schedule: both within
-    the bound, each bitwise reproducible."""
-    s, c = packed(N, K, 93)
-    x = synth.activations_bf16(synth.rng(94), M, K)
-    y_ref, bound = O.matmul_ref(O.bf16_bits_to_f64(x), s, c, K)
-    knob("sg_bm", bm)
-    knob("sg_sk", "on")
-    y_sk = run_gemm(s, c, x)
-    assert_within(y_sk, y_ref, bound, what=f"stream-K {M}x{N}x{K} bm={bm}")
-    assert np.array_equal(y_sk, run_gemm(s, c, x))
-    knob("sg_sk", "off")
-    y_t = run_gemm(s, c, x)
-    assert_within(y_t, y_ref, bound, what=f"whole tiles {M}x{N}x{K} bm={bm}")
