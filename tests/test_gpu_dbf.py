@@ -92,7 +92,8 @@ def test_dbf_tensor_path_extreme_scales(dbf_path):
 @pytest.mark.parametrize("m,r,n,B", [(200, 384, 256, 3), (1, 128, 128, 1), (1000, 640, 1152, 5),
                                      (4096, 1024, 2048, 2), (33, 256, 128, 7),
                                      # long K in either product: the GEMV cores split K over a cluster
-                                     (128, 512, 32768, 1), (128, 32768, 256, 2), (300, 12288, 12288, 1)])
+                                     (128, 512, 32768, 1), (128, 32768, 256, 2), (300, 12288, 12288, 1),
+                                     (300, 512, 32768, 3), (128, 32768, 256, 4), (1000, 640, 1152, 4)])
 def test_dbf_ragged(m, r, n, B):
     check(synth.dbf_case(m=m, r=r, n=n, B=B, seed=m + r + n + B), f"{m}x{r}x{n} B={B}")
 
