@@ -87,6 +87,7 @@ int w1_sync_status(w1_stream_t stream);
  *   "sg_bm"         128 | 256 forces the sign GEMM's token tile (W1_SG_BM)
  *   "sg_exp"        4 | 8 forces the sign GEMM's expander warps per CTA (W1_SG_EXP)
  *   "sg_a"          "smem" | "tmem": where the sign GEMM's 128-token tiles keep the weight operand (W1_SG_A)
+ *   "moe_tw"        2 | 4: 8-row n-tiles per warp in the decode MoE's per-route gate/up (W1_MOE_TW)
  *   "verbose"       nonzero prints plans and choices on stderr (W1_VERBOSE)
  * Returns W1_ERR_NULL for a NULL name, W1_ERR_SHAPE for an unknown name or
  * value. */

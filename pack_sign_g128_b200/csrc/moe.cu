@@ -815,14 +815,20 @@ struct MoeDecParams {
   int R, top_k, rows, K, NG, P, lgGw;
 };
 
-__host__ __device__ inline GdSmem moed_layout(const MoeDecParams& q) {
-  return gd_layout<1, moed::kWarps>(moed::kTw, q.NG, q.P, 1, 0, q.NG);
+__host__ __device__ inline GdSmem moed_layout(const MoeDecParams& q, int tw = moed::kTw) {
+  return gd_layout<1, moed::kWarps>(tw, q.NG, q.P, 1, 0, q.NG);
 }
 
+// TWG 8-row n-tiles per warp: 2 (16 rows of G or U per warp, 64 per CTA) or
+// 4 (32 per warp, 128 per CTA: half the CTAs, each activation fragment and
+// fold shared by two MMA tiles, the token's x quantised half as often).
+template <int TWG>
 __global__ void __launch_bounds__(moed::kWarps * 32, 1) moe_decode_gateup_kernel(const MoeDecParams q) {
+  constexpr int kRows = 4 * 8 * TWG;  // rows of each matrix per CTA
+  constexpr int TP = (TWG + 1) / 2;   // 16-row MMA tiles per warp
   extern __shared__ __align__(16) unsigned char smem[];
-  __shared__ float gu[2][moed::kRowsGu];
-  const GdSmem L = moed_layout(q);
+  __shared__ float gu[2][kRows];
+  const GdSmem L = moed_layout(q, TWG);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   __shared__ int sid[moe::kMaxTopK];
   __shared__ float swt[moe::kMaxTopK];
@@ -846,7 +852,7 @@ __global__ void __launch_bounds__(moed::kWarps * 32, 1) moe_decode_gateup_kernel
   if (blockIdx.x == 0 && threadIdx.x == 0) q.pos[r] = r;
   // this warp's matrix (0: G, 1: U) and rows
   const int mat = warp >> 2;
-  const int row0 = blockIdx.x * moed::kRowsGu + (warp & 3) * 8 * moed::kTw;
+  const int row0 = blockIdx.x * kRows + (warp & 3) * 8 * TWG;
   GdParams p = {};
   const int64_t mrow = static_cast<int64_t>(e) * q.rows;  // the expert's first row
   p.signs = (mat ? q.signs1 : q.signs0) + mrow * (q.K >> 5);
@@ -855,16 +861,16 @@ __global__ void __launch_bounds__(moed::kWarps * 32, 1) moe_decode_gateup_kernel
   p.N = q.rows;
   p.K = q.K;
   p.NG = q.NG;
-  p.Tw = moed::kTw;
+  p.Tw = TWG;
   p.NSw = q.NG;
   p.P = q.P;
   p.lgGw = q.lgGw;
   GdGeom g = {};
   g.nsc = q.NG;
-  g.tw = moed::kTw;
+  g.tw = TWG;
   g.nsw = q.NG;
   g.row0 = row0;
-  g.nrows = max(0, min(8 * moed::kTw, q.rows - row0));
+  g.nrows = max(0, min(8 * TWG, q.rows - row0));
   g.busy = g.nrows > 0;
   g.ngw = q.NG;
   unsigned char* wreg = smem + warp * L.warp_bytes;
@@ -883,26 +889,31 @@ __global__ void __launch_bounds__(moed::kWarps * 32, 1) moe_decode_gateup_kernel
   __syncthreads();
   float acc[gd::kMaxTp][gd::Cfg<1>::NN][4];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) acc[0][0][i] = acc[1][0][i] = 0.f;
-  if (g.busy) gd_compute<1, moed::kTw>(wts, p.P, scl, 8 * moed::kTw, xs, q.NG, lane, acc);
-  // digit columns -> row sums: a lane holds columns 2(lane&3), +1 of rows
-  // lane/4 (n-tile 0) and lane/4 + 8 (n-tile 1); columns past the three
-  // digits are zero, so the quad sum is the row's value
-  float v0 = acc[0][0][0] + acc[0][0][1], v1 = acc[0][0][2] + acc[0][0][3];
+  for (int tp = 0; tp < gd::kMaxTp; ++tp)
 #pragma unroll
-  for (int o = 1; o < 4; o <<= 1) {
-    v0 += __shfl_xor_sync(0xFFFFFFFFu, v0, o);
-    v1 += __shfl_xor_sync(0xFFFFFFFFu, v1, o);
-  }
+    for (int i = 0; i < 4; ++i) acc[tp][0][i] = 0.f;
+  if (g.busy) gd_compute<1, TWG>(wts, p.P, scl, 8 * TWG, xs, q.NG, lane, acc);
+  // digit columns -> row sums: a lane holds columns 2(lane&3), +1 of rows
+  // 16 tp + lane/4 and 16 tp + lane/4 + 8 of each MMA tile tp; columns past
+  // the three digits are zero, so the quad sum is the row's value
   const int rl = lane >> 2;
-  if ((lane & 3) == 0) {
-    const int base = (warp & 3) * 8 * moed::kTw;
-    gu[mat][base + rl] = v0;
-    gu[mat][base + 8 + rl] = v1;
+  const int base = (warp & 3) * 8 * TWG;
+#pragma unroll
+  for (int tp = 0; tp < TP; ++tp) {
+    float v0 = acc[tp][0][0] + acc[tp][0][1], v1 = acc[tp][0][2] + acc[tp][0][3];
+#pragma unroll
+    for (int o = 1; o < 4; o <<= 1) {
+      v0 += __shfl_xor_sync(0xFFFFFFFFu, v0, o);
+      v1 += __shfl_xor_sync(0xFFFFFFFFu, v1, o);
+    }
+    if ((lane & 3) == 0) {
+      gu[mat][base + 16 * tp + rl] = v0;
+      if (16 * tp + 8 < 8 * TWG) gu[mat][base + 16 * tp + 8 + rl] = v1;
+    }
   }
   __syncthreads();
-  for (int i = threadIdx.x; i < moed::kRowsGu; i += blockDim.x) {
-    const int row = blockIdx.x * moed::kRowsGu + i;
+  for (int i = threadIdx.x; i < kRows; i += blockDim.x) {
+    const int row = blockIdx.x * kRows + i;
     if (row < q.rows) {
       const float gv = gu[0][i], uv = gu[1][i];
       q.h[static_cast<int64_t>(r) * q.rows + row] = __float2bfloat16_rn(gv / (1.0f + expf(-gv)) * uv);
@@ -1375,7 +1386,7 @@ static cudaError_t launch_moe_decode_down(MoeDecParams q, int T, float* out, cud
                     RB, out);
 }
 
-static cudaError_t launch_moe_decode_gateup(MoeDecParams q, cudaStream_t stream) {
+static cudaError_t launch_moe_decode_gateup(MoeDecParams q, cudaStream_t stream, int num_sms) {
   auto lg2 = [](int v) {
     int l = 0;
     while ((1 << l) < v) ++l;
@@ -1383,11 +1394,25 @@ static cudaError_t launch_moe_decode_gateup(MoeDecParams q, cudaStream_t stream)
   };
   q.P = ((q.NG & 1) ? q.NG : q.NG + 1) * 16;  // odd multiple of 16 bytes per staged row: bank spread
   q.lgGw = lg2(q.NG);
+  // 128 rows per CTA where that still gives every SM a CTA, else 64
+  // (moe_tw knob: 2 or 4 n-tiles per warp)
+  const int tk = knob(kKnobMoeTw);
+  const bool wide = tk ? tk == 4
+                       : static_cast<int64_t>((q.rows + 127) / 128) * q.R >= num_sms &&
+                             moed_layout(q, 4).total <= moed::kSmemCap;
+  if (wide) {
+    const int smem = moed_layout(q, 4).total;
+    cudaError_t err = ensure_dyn_smem(reinterpret_cast<const void*>(moe_decode_gateup_kernel<4>), smem);
+    if (err != cudaSuccess) return err;
+    const dim3 grid(static_cast<unsigned>((q.rows + 127) / 128), static_cast<unsigned>(q.R));
+    return launch_pdl(moe_decode_gateup_kernel<4>, grid, dim3(moed::kWarps * 32), static_cast<size_t>(smem), stream, q);
+  }
   const int smem = moed_layout(q).total;
-  cudaError_t err = ensure_dyn_smem(reinterpret_cast<const void*>(moe_decode_gateup_kernel), smem);
+  cudaError_t err = ensure_dyn_smem(reinterpret_cast<const void*>(moe_decode_gateup_kernel<moed::kTw>), smem);
   if (err != cudaSuccess) return err;
   const dim3 grid(static_cast<unsigned>((q.rows + moed::kRowsGu - 1) / moed::kRowsGu), static_cast<unsigned>(q.R));
-  return launch_pdl(moe_decode_gateup_kernel, grid, dim3(moed::kWarps * 32), static_cast<size_t>(smem), stream, q);
+  return launch_pdl(moe_decode_gateup_kernel<moed::kTw>, grid, dim3(moed::kWarps * 32), static_cast<size_t>(smem),
+                    stream, q);
 }
 
 cudaError_t launch_moe(const uint16_t* x, const float* logits, int64_t T, int64_t H, int64_t I, int E, int top_k,
@@ -1471,7 +1496,7 @@ cudaError_t launch_moe(const uint16_t* x, const float* logits, int64_t T, int64_
       return launch_moe_decode_grouped(q, static_cast<int>(T), static_cast<int>(H), static_cast<int>(I), gl, ds, dc,
                                        rout, pos, out, stream, num_sms);
     }
-    err = launch_moe_decode_gateup(q, stream);
+    err = launch_moe_decode_gateup(q, stream, num_sms);
     if (err != cudaSuccess) return err;
     MoeDecParams qd = q;
     qd.x = reinterpret_cast<const uint16_t*>(h);

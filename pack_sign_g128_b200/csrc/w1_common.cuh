@@ -414,6 +414,7 @@ inline cudaError_t ensure_dyn_smem(const void* kernel, int bytes) {
 //   dbf_rank_split W1_DBF_RANK_SPLIT two-launch chain: CTAs per cluster that split r in U . h (0 = planner)
 //   sg_bm         W1_SG_BM          sign GEMM token tile: 0 = by tile count, else 128 or 256
 //   dbf_core      W1_DBF_CORE       two-launch chain's GEMV core: 0 = register-fed where it fits, 1 = same, 2 = direct
+//   moe_tw        W1_MOE_TW         decode MoE gate/up: 8-row n-tiles per warp, 0 = by CTA count, else 2 or 4
 //   sg_exp        W1_SG_EXP         sign GEMM expander warps: 0 = by token tile, else 4 or 8
 //   sg_a          W1_SG_A           sign GEMM weight operand of 128-token tiles: 0 = default, 1 = smem, 2 = TMEM
 //   verbose       W1_VERBOSE        nonzero: plans and choices on stderr
@@ -422,7 +423,7 @@ inline cudaError_t ensure_dyn_smem(const void* kernel, int bytes) {
 #include <cstring>
 namespace w1 {
 enum KnobId { kKnobGemvPath, kKnobGemvSplit, kKnobGemvAutotune, kKnobMoePath, kKnobDbfPath, kKnobDbfWarps,
-              kKnobDbfRankSplit, kKnobSgBm, kKnobDbfCore, kKnobSgExp, kKnobSgA, kKnobVerbose, kKnobCount };
+              kKnobDbfRankSplit, kKnobSgBm, kKnobDbfCore, kKnobSgExp, kKnobSgA, kKnobMoeTw, kKnobVerbose, kKnobCount };
 // GEMV kernels a knob can force (also the kinds of the dispatcher's choices).
 enum GemvPathKnob { kGemvAuto = 0, kGemvDirect8 = 1, kGemvDirect16 = 2, kGemvTc = 3, kGemvRing = 4, kGemvFlat = 5,
                     kGemvFlat16 = 6 };
@@ -447,6 +448,7 @@ inline const KnobSpec& knob_spec(int id) {
       {"dbf_core", "W1_DBF_CORE", 0, {"flat", "direct", nullptr}},
       {"sg_exp", "W1_SG_EXP", 0, {nullptr}},
       {"sg_a", "W1_SG_A", 0, {"smem", "tmem", nullptr}},
+      {"moe_tw", "W1_MOE_TW", 0, {nullptr}},
       {"verbose", "W1_VERBOSE", 0, {nullptr}},
   };
   return specs[id];

@@ -48,7 +48,7 @@ def test_knobs_accept_their_words_and_reject_the_rest(lib):
           ("gemv_path", "flat"), ("gemv_split", "4"), ("gemv_autotune", "0"), ("moe_path", "tiles"),
           ("moe_path", "decode"), ("moe_path", "grouped"), ("dbf_path", "fused"), ("dbf_path", "twostep"), ("dbf_warps", "16"),
           ("dbf_rank_split", "4"), ("sg_bm", "256"), ("dbf_core", "direct"), ("sg_exp", "8"), ("sg_a", "tmem"),
-          ("sg_a", "smem"),
+          ("sg_a", "smem"), ("moe_tw", "4"),
           ("verbose", "1")]
     try:
         for name, value in ok:

@@ -143,6 +143,16 @@ def test_moe_forced_path(path, T, knob):
     run_and_check(T, 512, 256, 16, 4, 7)
 
 
+@pytest.mark.parametrize("tw", [2, 4])
+@pytest.mark.parametrize("T,H,I", [(3, 512, 384), (8, 2048, 1024)])
+def test_moe_decode_gateup_rows_per_warp(tw, T, H, I, knob):
+    """The per-route gate/up kernel with 16 or 32 rows of each matrix per warp
+    (64 or 128 per CTA; I = 384 leaves a ragged last block of 128)."""
+    knob("moe_path", "decode")
+    knob("moe_tw", tw)
+    run_and_check(T, H, I, 16, 4, 12 + tw)
+
+
 @pytest.mark.parametrize("T", [64, 4])
 def test_moe_is_deterministic(T):
     H, I, E, K = 512, 256, 16, 4
