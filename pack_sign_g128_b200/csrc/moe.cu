@@ -1394,11 +1394,14 @@ static cudaError_t launch_moe_decode_gateup(MoeDecParams q, cudaStream_t stream,
   };
   q.P = ((q.NG & 1) ? q.NG : q.NG + 1) * 16;  // odd multiple of 16 bytes per staged row: bank spread
   q.lgGw = lg2(q.NG);
-  // 128 rows per CTA where that still gives every SM a CTA, else 64
-  // (moe_tw knob: 2 or 4 n-tiles per warp)
+  // 128 rows per CTA where that gives between one and two CTAs per SM, else
+  // 64 (moe_tw knob: 2 or 4 n-tiles per warp).  Measured on the OLMoE-like
+  // layer (us per layer, 64 / 128 rows): 2 tokens 24.6 / 26.1 (64 CTAs of
+  // 128 rows), 4 tokens 36.9 / 34.8 (256), 8 tokens 54.3 / 56.3 (512).
   const int tk = knob(kKnobMoeTw);
+  const int64_t ctas128 = static_cast<int64_t>((q.rows + 127) / 128) * q.R;
   const bool wide = tk ? tk == 4
-                       : static_cast<int64_t>((q.rows + 127) / 128) * q.R >= num_sms &&
+                       : ctas128 >= num_sms && ctas128 < 2 * static_cast<int64_t>(num_sms) &&
                              moed_layout(q, 4).total <= moed::kSmemCap;
   if (wide) {
     const int smem = moed_layout(q, 4).total;
