@@ -339,8 +339,8 @@ __global__ void __launch_bounds__(sg::threads_for<EXP>(), 1)
     // K-major atoms, or (TA) as 16 TMEM columns per word in the row's lane.
     // Words and scales stream through a kPf-deep register ring over this
     // CTA's (tile, stage) sequence so L2 latency hides behind kPf stages (8
-    // deep for 128-token tiles measured slower: 0.114 vs 0.075 ms for the
-    // 4096^3 DBF chain at 512 rows).
+    // deep measured slower on the 4096^3 DBF chain at 512 rows: 0.114 vs
+    // 0.075 ms with 4 expander warps, 0.095 vs 0.083 ms with 8 against 4).
     constexpr int kPf = 4;
     const int rl = (warp & 3) * 32 + lane;  // a warp reaches TMEM lanes 32 (warp % 4) ..
     const int half = EXP == 8 ? (warp - 2) >> 2 : 0;  // the atom this thread writes (8 expander warps)
