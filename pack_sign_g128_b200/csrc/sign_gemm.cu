@@ -338,9 +338,10 @@ __global__ void __launch_bounds__(sg::threads_for<EXP>(), 1)
     // word), stored as 16-byte chunks of the row in the two 128B-swizzled
     // K-major atoms, or (TA) as 16 TMEM columns per word in the row's lane.
     // Words and scales stream through a kPf-deep register ring over this
-    // CTA's (tile, stage) sequence so L2 latency hides behind kPf stages (8
+    // CTA's (tile, stage) sequence so L2 latency hides behind kPf stages.  8
     // deep measured slower on the 4096^3 DBF chain at 512 rows: 0.114 vs
-    // 0.075 ms with 4 expander warps, 0.095 vs 0.083 ms with 8 against 4).
+    // 0.075 ms with 4 expander warps; with 8, 0.095 ms where 4 expander
+    // warps at depth 4 took 0.083 on the same GPU.
     constexpr int kPf = 4;
     const int rl = (warp & 3) * 32 + lane;  // a warp reaches TMEM lanes 32 (warp % 4) ..
     const int half = EXP == 8 ? (warp - 2) >> 2 : 0;  // the atom this thread writes (8 expander warps)
